@@ -1,0 +1,385 @@
+"""Pins for the fp64 KDA oracle: checks against what the recurrence fixes
+independently of the oracle's own code.
+
+Each ``pin_*`` takes an oracle library handle (so the planted-mutation test
+can run the same battery against deliberately broken builds of the oracle)
+and raises AssertionError on failure.  Inputs are small and seeded.
+
+What pins what (recurrence: delta rule with a channel-wise forget gate, CSDN
+post on the Kimi K3 technical report, section 一.1):
+  * pin_identity_beta0        beta=0, alpha=1 leaves the state unchanged, o = S0^T q
+  * pin_orthonormal_retrieval beta=1, alpha=1, orthonormal keys: S^T k_j = v_j exactly
+  * pin_self_query            beta=1, |k|=1, q=k gives o_t = v_t for any S and alpha
+  * pin_decay_closed_form     beta=0: S_t = Diag(exp(G_t)) S_0 (closed form)
+  * pin_golden_fixtures       hand-worked values under tests/golden/
+  * pin_brute_force           dense (I - beta k k^T) Diag(alpha) products, tiny T and d
+  * pin_chunked_form          chunk-parallel algebra ("Kimi K3 开源日来了", FlashKDA
+                              section: parallel inside a chunk, serial between chunks)
+                              equals the oracle for C in {1, 16, 64, T}
+  * pin_split_combine         zero-start state + transition, combined, equals the
+                              unsplit run ("Kimi K3 开源日来了", Infra section, first layer)
+  * pin_snapshot_tagging      snapshots hold exactly the first j*stride tokens
+  * pin_contraction_bound     ||S_t|| <= ||S_{t-1}|| + beta ||k|| ||v||
+  * pin_resume                prefill(0..L) == prefill(jS..L) started from snapshot j
+  * pin_decode_matches_prefill L decode steps == a prefill of L tokens
+  * pin_decode_slots          decode writes the slot it is told to and no other
+  * pin_varlen_isolation      a packed request equals the same request run alone
+"""
+from __future__ import annotations
+
+import os
+
+import numpy as np
+
+import oracle
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _rng(seed):
+    return np.random.default_rng(seed)
+
+
+def _unit(x):
+    return x / np.linalg.norm(x, axis=-1, keepdims=True)
+
+
+def rand_inputs(lengths, H, dk, dv, seed=0, gate_lo=-5.0, s0_std=None):
+    rng = _rng(seed)
+    T = int(sum(lengths))
+    q = _unit(rng.standard_normal((T, H, dk)))
+    k = _unit(rng.standard_normal((T, H, dk)))
+    v = rng.standard_normal((T, H, dv))
+    g = gate_lo * (1.0 / (1.0 + np.exp(-rng.standard_normal((T, H, dk)))))
+    beta = 1.0 / (1.0 + np.exp(-rng.standard_normal((T, H))))
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int64)
+    s0 = None if s0_std is None else s0_std * rng.standard_normal((len(lengths), H, dk, dv))
+    return dict(q=q, k=k, v=v, g=g, beta=beta, cu=cu, s0=s0)
+
+
+def _run(lib, x, stride=0, n_threads=2):
+    return oracle.prefill(x["q"], x["k"], x["v"], x["g"], x["beta"], x["cu"], x["s0"],
+                          snapshot_stride=stride, n_threads=n_threads, lib=lib)
+
+
+# ----------------------------------------------------------------------------
+# Independent restatements used as pins (written from the definition, not from
+# the oracle source).
+# ----------------------------------------------------------------------------
+
+def brute_force_chain(q, k, v, g, beta, s0):
+    """Dense transition matrices: S_t = A_t S_{t-1} + beta k v^T with
+    A_t = (I - beta_t k_t k_t^T) Diag(alpha_t).  Returns (o [L,dv], states [L,dk,dv])."""
+    L, dk = k.shape
+    S = s0.copy()
+    outs, states = [], []
+    for t in range(L):
+        A = (np.eye(dk) - beta[t] * np.outer(k[t], k[t])) @ np.diag(np.exp(g[t]))
+        S = A @ S + beta[t] * np.outer(k[t], v[t])
+        outs.append(S.T @ q[t])
+        states.append(S.copy())
+    return np.array(outs), np.array(states)
+
+
+def chunked_chain(q, k, v, g, beta, s0, C):
+    """Chunk-parallel form derived by unrolling the recurrence inside a chunk.
+
+    With G_t = sum_{s<=t} g_s (chunk-local) and gamma_t = exp(G_t):
+      A_ij = sum_c k_ic k_jc exp(G_ic - G_jc)  (j < i),  P_ij = same with q_i (j <= i)
+      (I + Diag(beta) A) U = Diag(beta) (V - (gamma*K) S0)
+      O = (gamma*Q) S0 + P U,   S_C = Diag(gamma_C) S0 + ((gamma_C/gamma)*K)^T U
+    The exponent differences are formed before exponentiation, so nothing
+    over- or underflows in fp64 at these sizes.
+    """
+    L, dk = k.shape
+    dv = v.shape[1]
+    S = s0.copy()
+    O = np.zeros((L, dv))
+    for c0 in range(0, L, C):
+        sl = slice(c0, min(c0 + C, L))
+        K, Q, V, b = k[sl], q[sl], v[sl], beta[sl]
+        n = K.shape[0]
+        G = np.cumsum(g[sl], axis=0)
+        ii, jj = np.meshgrid(np.arange(n), np.arange(n), indexing="ij")
+        D = G[:, None, :] - G[None, :, :]
+        D = np.where((ii >= jj)[:, :, None], D, -np.inf)
+        E = np.exp(D)
+        A = np.einsum("ic,jc,ijc->ij", K, K, E) * (ii > jj)
+        P = np.einsum("ic,jc,ijc->ij", Q, K, E) * (ii >= jj)
+        gam = np.exp(G)
+        Tinv = np.linalg.inv(np.eye(n) + b[:, None] * A)
+        W = Tinv @ (b[:, None] * gam * K)
+        Ut = Tinv @ (b[:, None] * V)
+        U = Ut - W @ S
+        O[sl] = (gam * Q) @ S + P @ U
+        tail = np.exp(G[-1][None, :] - G)
+        S = np.exp(G[-1])[:, None] * S + (tail * K).T @ U
+    return O, S
+
+
+def read_golden(name):
+    """Parse a fixture: header keys dk/dv/s0, then 'token <inputs> | <S_t> <o_t>'."""
+    dk = dv = None
+    s0 = None
+    toks = []
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.split("#", 1)[0].strip()
+            if not line:
+                continue
+            key, rest = line.split(None, 1)
+            if key == "dk":
+                dk = int(rest)
+            elif key == "dv":
+                dv = int(rest)
+            elif key == "s0":
+                s0 = np.array([float(x) for x in rest.split()]).reshape(dk, dv)
+            elif key == "token":
+                lhs, rhs = rest.split("|")
+                a = [float(x) for x in lhs.split()]
+                e = [float(x) for x in rhs.split()]
+                kk = a[0:dk]
+                vv = a[dk:dk + dv]
+                qq = a[dk + dv:2 * dk + dv]
+                bb = a[2 * dk + dv]
+                al = a[2 * dk + dv + 1:3 * dk + dv + 1]
+                toks.append(dict(k=kk, v=vv, q=qq, beta=bb, alpha=al,
+                                 S=np.array(e[:dk * dv]).reshape(dk, dv), o=np.array(e[dk * dv:])))
+    return dk, dv, s0, toks
+
+
+# ----------------------------------------------------------------------------
+# Pins
+# ----------------------------------------------------------------------------
+
+def pin_identity_beta0(lib):
+    x = rand_inputs([5, 0, 9], H=2, dk=6, dv=4, seed=1, s0_std=1.0)
+    x["beta"][:] = 0.0
+    x["g"][:] = 0.0
+    r = _run(lib, x)
+    assert np.array_equal(r["final_state"], x["s0"]), "beta=0, alpha=1 must leave S unchanged"
+    for req in range(3):
+        for t in range(x["cu"][req], x["cu"][req + 1]):
+            for h in range(2):
+                ref = x["s0"][req, h].T @ x["q"][t, h]
+                np.testing.assert_allclose(r["o"][t, h], ref, rtol=0, atol=1e-13)
+
+
+def pin_orthonormal_retrieval(lib):
+    rng = _rng(2)
+    dk, dv, n = 8, 5, 6
+    Qm, _ = np.linalg.qr(rng.standard_normal((dk, dk)))
+    k = Qm[:, :n].T[:, None, :]                     # n orthonormal keys, H=1
+    v = rng.standard_normal((n, 1, dv))
+    x = dict(q=k.copy(), k=k, v=v, g=np.zeros((n, 1, dk)), beta=np.ones((n, 1)),
+             cu=np.array([0, n], dtype=np.int64), s0=None)
+    S = _run(lib, x)["final_state"][0, 0]
+    for j in range(n):
+        np.testing.assert_allclose(S.T @ k[j, 0], v[j, 0], rtol=0, atol=1e-12)
+
+
+def pin_self_query(lib):
+    x = rand_inputs([17], H=2, dk=8, dv=3, seed=3, s0_std=1.0)
+    x["beta"][:] = 1.0
+    x["q"] = x["k"].copy()
+    r = _run(lib, x)
+    np.testing.assert_allclose(r["o"], x["v"], rtol=0, atol=1e-12)
+
+
+def pin_decay_closed_form(lib):
+    x = rand_inputs([7, 11], H=3, dk=5, dv=4, seed=4, s0_std=1.0)
+    x["beta"][:] = 0.0
+    r = _run(lib, x)
+    for req in range(2):
+        lo, hi = x["cu"][req], x["cu"][req + 1]
+        for h in range(3):
+            G = np.cumsum(x["g"][lo:hi, h], axis=0)
+            for i, t in enumerate(range(lo, hi)):
+                St = np.exp(G[i])[:, None] * x["s0"][req, h]
+                np.testing.assert_allclose(r["o"][t, h], St.T @ x["q"][t, h], rtol=1e-12,
+                                           atol=1e-14)
+            np.testing.assert_allclose(r["final_state"][req, h],
+                                       np.exp(G[-1])[:, None] * x["s0"][req, h],
+                                       rtol=1e-12, atol=1e-14)
+
+
+def pin_golden_fixtures(lib):
+    for name in ("scalar_d1.txt", "two_channel_dk2.txt"):
+        dk, dv, s0, toks = read_golden(name)
+        L = len(toks)
+        q = np.array([t["q"] for t in toks])[:, None, :]
+        k = np.array([t["k"] for t in toks])[:, None, :]
+        v = np.array([t["v"] for t in toks])[:, None, :]
+        g = np.log(np.array([t["alpha"] for t in toks]))[:, None, :]
+        beta = np.array([t["beta"] for t in toks])[:, None]
+        # states after each prefix come from snapshots at stride 1
+        r = oracle.prefill(q, k, v, g, beta, np.array([0, L]), s0[None, None],
+                           snapshot_stride=1, lib=lib)
+        for i, t in enumerate(toks):
+            np.testing.assert_allclose(r["snapshots"][i, 0], t["S"], rtol=0, atol=1e-12,
+                                       err_msg=f"{name} token {i + 1} state")
+            np.testing.assert_allclose(r["o"][i, 0], t["o"], rtol=0, atol=1e-12,
+                                       err_msg=f"{name} token {i + 1} output")
+
+
+def pin_brute_force(lib):
+    cases = [([16], 1, 8, 8, -5.0), ([3, 16, 1], 2, 4, 6, -0.1), ([12, 5], 2, 7, 3, -1.0)]
+    for seed, (lengths, H, dk, dv, gate_lo) in enumerate(cases):
+        x = rand_inputs(lengths, H, dk, dv, seed=10 + seed, s0_std=0.5, gate_lo=gate_lo)
+        stride = 4
+        r = _run(lib, x, stride=stride)
+        cs = r["cu_snapshots"]
+        for req in range(len(lengths)):
+            lo, hi = x["cu"][req], x["cu"][req + 1]
+            for h in range(H):
+                sl = slice(lo, hi)
+                o, states = brute_force_chain(x["q"][sl, h], x["k"][sl, h], x["v"][sl, h],
+                                              x["g"][sl, h], x["beta"][sl, h], x["s0"][req, h])
+                np.testing.assert_allclose(r["o"][sl, h], o, rtol=0, atol=1e-13)
+                fin = states[-1] if hi > lo else x["s0"][req, h]
+                np.testing.assert_allclose(r["final_state"][req, h], fin, rtol=0, atol=1e-13)
+                for j in range(1, (hi - lo) // stride + 1):
+                    np.testing.assert_allclose(r["snapshots"][cs[req] + j - 1, h],
+                                               states[j * stride - 1], rtol=0, atol=1e-13)
+
+
+def pin_chunked_form(lib):
+    for gate_lo in (-5.0, -0.05):   # strong decay (exponent range) and weak (long range)
+        _chunked_case(lib, gate_lo)
+
+
+def _chunked_case(lib, gate_lo):
+    L, H, dk, dv = 150, 2, 8, 6
+    x = rand_inputs([L], H, dk, dv, seed=21, s0_std=0.3, gate_lo=gate_lo)
+    r = _run(lib, x)
+    for C in (1, 16, 64, L):
+        for h in range(H):
+            O, S = chunked_chain(x["q"][:, h], x["k"][:, h], x["v"][:, h], x["g"][:, h],
+                                 x["beta"][:, h], x["s0"][0, h], C)
+            np.testing.assert_allclose(O, r["o"][:, h], rtol=0, atol=1e-10,
+                                       err_msg=f"chunked C={C}")
+            np.testing.assert_allclose(S, r["final_state"][0, h], rtol=0, atol=1e-10)
+
+
+def pin_split_combine(lib):
+    # weak decay, so the transition M stays far from zero and its errors show
+    L, H, dk, dv, seg = 96, 2, 6, 5, 24
+    x = rand_inputs([L], H, dk, dv, seed=31, s0_std=0.7, gate_lo=-0.05)
+    full = _run(lib, x, stride=seg)
+    seg_cu = np.arange(0, L + 1, seg)
+    s_loc, m = oracle.chunk_local_state(x["k"], x["v"], x["g"], x["beta"], seg_cu, lib=lib)
+    s_in, s_fin = oracle.state_combine(s_loc, m, x["s0"][0], lib=lib)
+    np.testing.assert_allclose(s_fin, full["final_state"][0], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(s_in[0], x["s0"][0], rtol=0, atol=0)
+    for s in range(1, len(seg_cu) - 1):
+        np.testing.assert_allclose(s_in[s], full["snapshots"][s - 1], rtol=0, atol=1e-12)
+    # M alone: brute-force product of the dense transitions of segment 1, head 1
+    lo, hi = seg_cu[1], seg_cu[2]
+    Mref = np.eye(dk)
+    for t in range(lo, hi):
+        A = (np.eye(dk) - x["beta"][t, 1] * np.outer(x["k"][t, 1], x["k"][t, 1])) \
+            @ np.diag(np.exp(x["g"][t, 1]))
+        Mref = A @ Mref
+    np.testing.assert_allclose(m[1, 1], Mref, rtol=0, atol=1e-13)
+
+
+def pin_snapshot_tagging(lib):
+    """beta=1, alpha=1, one-hot keys: the write at position p replaces row p mod dk
+    with v_p, so each row of a snapshot names the last position written into it."""
+    dk, dv, stride = 8, 1, 4
+    lengths = [19, 8, 3]
+    T = sum(lengths)
+    cu = np.concatenate([[0], np.cumsum(lengths)]).astype(np.int64)
+    k = np.zeros((T, 1, dk))
+    v = np.zeros((T, 1, dv))
+    for r_ in range(len(lengths)):
+        for p in range(lengths[r_]):
+            k[cu[r_] + p, 0, p % dk] = 1.0
+            v[cu[r_] + p, 0, 0] = 100 * (r_ + 1) + p + 1   # encodes request and position
+    x = dict(q=k.copy(), k=k, v=v, g=np.zeros((T, 1, dk)), beta=np.ones((T, 1)), cu=cu, s0=None)
+    r = _run(lib, x, stride=stride)
+    assert r["snapshots"].shape[0] == sum(L // stride for L in lengths)
+    idx = 0
+    for r_, L in enumerate(lengths):
+        for j in range(1, L // stride + 1):
+            n = j * stride                      # tokens consumed
+            exp_ = np.zeros(dk)
+            for p in range(n):
+                exp_[p % dk] = 100 * (r_ + 1) + p + 1
+            assert np.array_equal(r["snapshots"][idx, 0, :, 0], exp_), (r_, j)
+            idx += 1
+
+
+def pin_contraction_bound(lib):
+    x = rand_inputs([40], H=1, dk=6, dv=4, seed=41, s0_std=2.0)
+    state = np.ascontiguousarray(x["s0"].copy())
+    for t in range(40):
+        prev = np.linalg.norm(state[0, 0], 2)
+        oracle.decode_step(x["q"][t:t + 1], x["k"][t:t + 1], x["v"][t:t + 1],
+                           x["g"][t:t + 1], x["beta"][t:t + 1], state, lib=lib)
+        bound = prev + x["beta"][t, 0] * np.linalg.norm(x["k"][t, 0]) * np.linalg.norm(x["v"][t, 0])
+        assert np.linalg.norm(state[0, 0], 2) <= bound * (1 + 1e-12)
+
+
+def pin_resume(lib):
+    L, stride = 45, 8
+    x = rand_inputs([L], H=2, dk=5, dv=5, seed=51, s0_std=0.4, gate_lo=-0.1)
+    full = _run(lib, x, stride=stride)
+    for j in (1, 3, 5):
+        cut = j * stride
+        y = {kk: (vv[cut:] if kk in ("q", "k", "v", "g", "beta") else vv) for kk, vv in x.items()}
+        y["cu"] = np.array([0, L - cut], dtype=np.int64)
+        y["s0"] = full["snapshots"][j - 1][None]
+        part = _run(lib, y)
+        np.testing.assert_allclose(part["o"], full["o"][cut:], rtol=0, atol=1e-12)
+        np.testing.assert_allclose(part["final_state"], full["final_state"], rtol=0, atol=1e-12)
+
+
+def pin_decode_matches_prefill(lib):
+    L, N, H, dk, dv = 12, 3, 2, 6, 5
+    x = rand_inputs([L] * N, H, dk, dv, seed=61, s0_std=0.5, gate_lo=-0.2)
+    full = _run(lib, x)
+    state = np.ascontiguousarray(x["s0"].copy())
+    for t in range(L):
+        rows = [x["cu"][n] + t for n in range(N)]
+        o = oracle.decode_step(x["q"][rows], x["k"][rows], x["v"][rows], x["g"][rows],
+                               x["beta"][rows], state, lib=lib)
+        np.testing.assert_allclose(o, full["o"][rows], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(state, full["final_state"], rtol=0, atol=1e-12)
+
+
+def pin_decode_slots(lib):
+    x = rand_inputs([1, 1, 1], H=2, dk=4, dv=3, seed=71)
+    rng = _rng(72)
+    pool = rng.standard_normal((5, 2, 4, 3))
+    state = np.ascontiguousarray(pool.copy())
+    slot = np.array([4, 0, 2], dtype=np.int64)
+    oracle.decode_step(x["q"], x["k"], x["v"], x["g"], x["beta"], state, slot=slot, lib=lib)
+    for s in (1, 3):
+        assert np.array_equal(state[s], pool[s]), "untouched slots must not change"
+    for n, s in enumerate(slot):
+        _, states = brute_force_chain(x["q"][n:n + 1, 0], x["k"][n:n + 1, 0], x["v"][n:n + 1, 0],
+                                      x["g"][n:n + 1, 0], x["beta"][n:n + 1, 0], pool[s, 0])
+        np.testing.assert_allclose(state[s, 0], states[-1], rtol=0, atol=1e-13)
+
+
+def pin_varlen_isolation(lib):
+    lengths = [13, 0, 30, 7]
+    x = rand_inputs(lengths, H=2, dk=5, dv=4, seed=81, s0_std=0.5, gate_lo=-0.2)
+    packed = _run(lib, x, stride=4)
+    for r_ in range(len(lengths)):
+        lo, hi = x["cu"][r_], x["cu"][r_ + 1]
+        y = {kk: (vv[lo:hi] if kk in ("q", "k", "v", "g", "beta") else vv) for kk, vv in x.items()}
+        y["cu"] = np.array([0, hi - lo], dtype=np.int64)
+        y["s0"] = x["s0"][r_:r_ + 1]
+        alone = _run(lib, y, stride=4)
+        assert np.array_equal(alone["o"], packed["o"][lo:hi])
+        assert np.array_equal(alone["final_state"][0], packed["final_state"][r_])
+        cs = packed["cu_snapshots"]
+        assert np.array_equal(alone["snapshots"], packed["snapshots"][cs[r_]:cs[r_ + 1]])
+
+
+ALL_PINS = [pin_identity_beta0, pin_orthonormal_retrieval, pin_self_query,
+            pin_decay_closed_form, pin_golden_fixtures, pin_brute_force, pin_chunked_form,
+            pin_split_combine, pin_snapshot_tagging, pin_contraction_bound, pin_resume,
+            pin_decode_matches_prefill, pin_decode_slots, pin_varlen_isolation]
