@@ -1,0 +1,460 @@
+#!/usr/bin/env python
+"""Benchmark of the KDA hot path on B200.
+
+One step = one chunked prefill (kda_prefill_chunked through the C ABI) of the
+varlen workload: 64 requests with lengths log-uniform on [128, 4096] (seed 0,
+73,490 tokens), H=32, d_k=d_v=128, bf16 q/k/v, fp32 g/beta, fp32 outputs,
+zero initial states, final states returned.  Inputs are generated on the
+device before timing and are larger than L2 (about 2.7 GB per step), so no
+L2 flush is needed between steps.
+
+Also reported on the same JSON line: the decode step (256 requests x 32
+heads x 128x128 fp32 states, GB/s against HBM), the end-to-end number
+through host buffers, the oracle timed on the host cores, and SM clocks
+sampled during the timed region.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+
+For N > 1 it runs under torchrun, one process per GPU, each rank an
+independent replica of the workload (the work shards by request with no
+collective; only the timing uses a max over ranks).
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = ("KDA prefill tokens/s + TFLOP/s (H=32,d=128,T=64K); decode state GB/s vs HBM peak")
+CHUNK = 64
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+
+
+# ---------------------------------------------------------------------------
+# algorithmic work per unit
+# ---------------------------------------------------------------------------
+
+def prefill_flops_per_token_head(dk: int, dv: int, C: int = CHUNK) -> int:
+    """Triangular C x C tiles counted as half: A, P (C(C-1)/2 / C(C+1)/2 dots of
+    length dk), T K and T V, P U, plus the three dense C x d x d state products."""
+    return C * (3 * dk + 2 * dv) + 6 * dk * dv
+
+
+def prefill_bytes(T: int, H: int, dk: int, dv: int, n_req: int, in_bytes: int = 2,
+                  out_bytes: int = 4, initial: bool = False, final: bool = True) -> int:
+    per_th = in_bytes * (2 * dk + dv) + 4 * dk + 4 + out_bytes * dv
+    state = n_req * H * dk * dv * 4
+    return T * H * per_th + (state if initial else 0) + (state if final else 0)
+
+
+def decode_bytes(N: int, H: int, d: int, in_bytes: int = 2, out_bytes: int = 4) -> int:
+    per = 2 * d * d * 4 + in_bytes * 3 * d + 4 * d + 4 + out_bytes * d
+    return N * H * per
+
+
+# ---------------------------------------------------------------------------
+# clocks sampled during the timed region
+# ---------------------------------------------------------------------------
+
+class ClockSampler:
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        try:
+            fd, self.path = tempfile.mkstemp(suffix=".csv")
+            os.close(fd)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}",
+                 "--format=csv,noheader,nounits", "-lms", "100", "-f", self.path],
+                stdout=subprocess.DEVNULL, stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.proc = None
+
+    def stop(self) -> dict:
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 9:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        mx = [float(r[2]) for r in rows if r[2].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for r in rows for i in range(4) if r[5 + i] == "Active"})
+        pw = [float(r[3]) for r in rows if r[3].replace(".", "").isdigit()]
+        return {"sm_mhz": statistics.median(sm) if sm else None,
+                "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
+                "samples": len(rows), "power_w_max": max(pw) if pw else None}
+
+
+def load_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as f:
+            p = json.load(f)
+        return p, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ---------------------------------------------------------------------------
+# distributed plumbing (timing only; the workload has no collective)
+# ---------------------------------------------------------------------------
+
+def dist_setup():
+    import torch
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+
+        import torch.distributed as dist
+        torch.cuda.set_device(local)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ---------------------------------------------------------------------------
+# CPU oracle timing (reported baseline; also the reference arm)
+# ---------------------------------------------------------------------------
+
+def sample_chains(lengths, H):
+    """Four heads per request (h = r, r+8, r+16, r+24 mod H): 256 chains."""
+    return [(r, (r + 8 * j) % H) for r in range(len(lengths)) for j in range(4)]
+
+
+def time_oracle(inp, pairs) -> dict:
+    import numpy as np
+    import torch
+
+    import oracle
+    cu = [int(c) for c in inp.cu_seqlens.cpu().tolist()]
+    parts = {n: [] for n in ("q", "k", "v", "g", "beta")}
+    lens = []
+    for (r, h) in pairs:
+        lo, hi = cu[r], cu[r + 1]
+        lens.append(hi - lo)
+        for n in parts:
+            t = getattr(inp, n)
+            parts[n].append(t[lo:hi, h:h + 1].cpu())
+    cat = {n: torch.cat(v, 0).double().numpy() for n, v in parts.items()}
+    pcu = np.concatenate([[0], np.cumsum(lens)])
+    threads = os.cpu_count() or 1
+    t0 = time.perf_counter()
+    oracle.prefill(cat["q"], cat["k"], cat["v"], cat["g"], cat["beta"], pcu, None,
+                   want_o=True, n_threads=threads)
+    dt = time.perf_counter() - t0
+    token_heads = int(pcu[-1])
+    return {"seconds": dt, "token_heads": token_heads, "cores": threads}
+
+
+def cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+# ---------------------------------------------------------------------------
+# arms
+# ---------------------------------------------------------------------------
+
+def workload_inputs(device, seed):
+    from decode_kda_chunked_b200 import inputs as I
+    return I.varlen(device=device, seed=seed)
+
+
+def workload_config(inp, world):
+    return {"workload": "varlen packed prefill: 64 requests, lengths log-uniform on [128, 4096] "
+                        "(seed 0), H=32, d_k=d_v=128, bf16 q/k/v, fp32 g/beta/o/state, "
+                        "zero initial states, final states out",
+            "n_req": inp.n_req, "total_tokens": inp.total_tokens, "H": 32, "d": 128,
+            "global_batch": inp.n_req * world, "seq_len": inp.total_tokens,
+            "parallelism": f"replicas x{world} (requests shard, no collective)",
+            "l2": "inputs larger than L2 (no flush)"}
+
+
+def run_reference(args, world, rank):
+    if rank != 0:
+        return
+    import torch
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    inp = workload_inputs(dev, 0)
+    H = 32
+    pairs_all = sample_chains(inp.lengths, H)
+    # each step: a bounded sample of 64 chains (one quarter of the CPU-baseline set)
+    per_step = [pairs_all[i::4] for i in range(4)]
+    for i in range(args.warmup):
+        time_oracle(inp, per_step[i % 4])
+    total_s, total_th, cores = 0.0, 0, 1
+    for i in range(args.steps):
+        r = time_oracle(inp, per_step[i % 4])
+        total_s += r["seconds"]
+        total_th += r["token_heads"]
+        cores = r["cores"]
+    value = total_th / H / total_s
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "tokens/s",
+            "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+            "ms_per_step": 1e3 * total_s / args.steps, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": workload_config(inp, 1),
+            "cpu_baseline": {"value": value, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+                             "sample": "64 (request, head) chains per step (one head per "
+                                       "request), tokens/s scaled to H=32",
+                             "cpu": cpu_model()},
+            "e2e": {"value": value, "unit": "tokens/s", "h2d_bytes_per_step": 0,
+                    "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+def run_ours(args, world, rank, local):
+    import torch
+
+    import decode_kda_chunked_b200 as kda
+    from decode_kda_chunked_b200 import _lib
+    from decode_kda_chunked_b200 import inputs as I
+
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    lib = kda.load()
+    inp = workload_inputs(dev, seed=rank)
+    T, H, dk, dv = inp.total_tokens, 32, 128, 128
+    n_req = inp.n_req
+    cu_host = torch.tensor([0] + list(__import__("itertools").accumulate(inp.lengths)),
+                           dtype=torch.int32)
+    o = torch.empty(T, H, dv, device=dev)
+    fin = torch.empty(n_req, H, dk, dv, device=dev)
+    a = _lib.make_prefill_args(inp.q, inp.k, inp.v, inp.g, inp.beta, inp.cu_seqlens, o, None, fin,
+                               0, None, None, cu_host)
+    ws_bytes = max(lib.kda_prefill_workspace_size(__import__("ctypes").byref(a)), 256)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        kda.kda_prefill_chunked(inp.q, inp.k, inp.v, inp.g, inp.beta, inp.cu_seqlens, o, None,
+                                fin, 0, None, None, cu_seqlens_host=cu_host, workspace=ws,
+                                stream=stream)
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    assert kda.kda_get_device_status() == 0
+    barrier(world)
+    torch.cuda.synchronize()
+
+    sampler = ClockSampler(local)
+    sampler.start()
+    time.sleep(0.3)
+    starts = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    ends = [torch.cuda.Event(enable_timing=True) for _ in range(args.steps)]
+    for i in range(args.steps):
+        starts[i].record(stream)
+        step()
+        ends[i].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    per_step_ms = [s.elapsed_time(e) for s, e in zip(starts, ends)]
+    total_ms = starts[0].elapsed_time(ends[-1])
+    total_ms = max_over_ranks(total_ms, world)
+    launch_ms = statistics.mean(per_step_ms)
+
+    peaks, peak_kind = load_peaks()
+    flops = prefill_flops_per_token_head(dk, dv) * T * H
+    bytes_ = prefill_bytes(T, H, dk, dv, n_req, in_bytes=2, out_bytes=4, final=True)
+    achieved_gbs = bytes_ / (launch_ms * 1e-3) / 1e9
+    tflops = flops / (launch_ms * 1e-3) / 1e12
+    value = world * T * args.steps / (total_ms * 1e-3)
+    tc = kda.kda_prefill_uses_tensor_cores(dk, dv)
+
+    line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+            "dtype": "bf16" if tc else "f32", "data": "synthetic",
+            "config": workload_config(inp, world),
+            "tflops": tflops,
+            "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"],
+                         "unit": "GB/s", "frac": achieved_gbs / peaks["hbm_gbs"],
+                         "traffic": None, "peak_kind": peak_kind,
+                         "algorithmic_bytes_per_launch": bytes_,
+                         "launch_ms": launch_ms,
+                         "tensor_frac": tflops / peaks["bf16_tflops"],
+                         "kernel": "prefill (schedule + chunked prefill launches)"},
+            "gpu_launches": 2 * args.steps,
+            "clocks": clocks}
+
+    if not args.no_decode:
+        line["decode"] = bench_decode(args, dev, peaks, peak_kind, rank)
+    if not args.no_e2e:
+        line["e2e"] = bench_e2e(args, inp, dev, world)
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        r = time_oracle(inp, sample_chains(inp.lengths, H))
+        line["cpu_baseline"] = {"value": r["token_heads"] / H / r["seconds"], "unit": "tokens/s",
+                                "cores": r["cores"], "kind": "oracle",
+                                "sample": f"{len(sample_chains(inp.lengths, H))} (request, head) "
+                                          f"chains of the workload ({r['token_heads']} "
+                                          f"token-heads, 4 heads per request), tokens/s "
+                                          f"scaled to H=32",
+                                "seconds": r["seconds"], "cpu": cpu_model()}
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def bench_decode(args, dev, peaks, peak_kind, rank):
+    import torch
+
+    import decode_kda_chunked_b200 as kda
+    from decode_kda_chunked_b200 import inputs as I
+    N, H, d = 256, 32, 128
+    steps = max(args.steps, 10)
+    warm = max(args.warmup, 3)
+    x = I.decode(steps + warm, N=N, H=H, d=d, device=dev, seed=rank)
+    state = x.state
+    o = torch.empty(N, H, d, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step(t):
+        kda.kda_decode_step(x.q[t], x.k[t], x.v[t], x.g[t], x.beta[t], state, o, stream=stream)
+
+    for t in range(warm):
+        step(t)
+    torch.cuda.synchronize()
+    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * steps)]
+    for i in range(steps):
+        ev[2 * i].record(stream)
+        step(warm + i)
+        ev[2 * i + 1].record(stream)
+    torch.cuda.synchronize()
+    per = [ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(steps)]
+    ms = statistics.mean(per)
+    b = decode_bytes(N, H, d)
+    gbs = b / (ms * 1e-3) / 1e9
+    return {"workload": "256 requests x H=32 x 128x128 fp32 states, 1 bf16 token each; state "
+                        "pool 512 MiB > L2",
+            "value": gbs, "unit": "GB/s", "ms_per_step": ms, "steps": steps,
+            "bytes_per_step": b,
+            "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": gbs / peaks["hbm_gbs"], "peak_kind": peak_kind,
+                         "frac_of_nominal_8tbs": gbs / 8000.0}}
+
+
+def bench_e2e(args, inp, dev, world):
+    """Same metric through the public entry point with host buffers: every step
+    copies that step's inputs from pinned host memory and reads o and the final
+    states back to pinned host memory inside the timed region."""
+    import torch
+
+    import decode_kda_chunked_b200 as kda
+    T, H, dv, dk = inp.total_tokens, 32, 128, 128
+    names = ("q", "k", "v", "g", "beta", "cu_seqlens")
+    host = {n: getattr(inp, n).cpu().pin_memory() for n in names}
+    devb = {n: torch.empty_like(getattr(inp, n)) for n in names}
+    o = torch.empty(T, H, dv, device=dev)
+    fin = torch.empty(inp.n_req, H, dk, dv, device=dev)
+    o_h = torch.empty(o.shape, dtype=o.dtype).pin_memory()
+    fin_h = torch.empty(fin.shape, dtype=fin.dtype).pin_memory()
+    cu_host = host["cu_seqlens"]
+    stream = torch.cuda.current_stream(dev)
+    h2d = sum(t.numel() * t.element_size() for t in host.values())
+    d2h = o.numel() * 4 + fin.numel() * 4
+    steps = max(2, min(args.steps, 5))
+
+    def step():
+        for n in names:
+            devb[n].copy_(host[n], non_blocking=True)
+        kda.kda_prefill_chunked(devb["q"], devb["k"], devb["v"], devb["g"], devb["beta"],
+                                devb["cu_seqlens"], o, None, fin, 0, None, None,
+                                cu_seqlens_host=cu_host, stream=stream)
+        o_h.copy_(o, non_blocking=True)
+        fin_h.copy_(fin, non_blocking=True)
+
+    step()
+    torch.cuda.synchronize()
+    barrier(world)
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(steps):
+        step()
+    e.record(stream)
+    torch.cuda.synchronize()
+    ms = max_over_ranks(s.elapsed_time(e), world)
+    return {"value": world * T * steps / (ms * 1e-3), "unit": "tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": steps,
+            "ms_per_step": ms / steps}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=10)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-decode", action="store_true")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3  # the timing rules ask for at least 3 warm-up steps
+    world, rank, local = dist_setup() if args.impl == "ours" else (
+        int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0)
+    try:
+        if args.impl == "reference":
+            run_reference(args, world, rank)
+        else:
+            run_ours(args, world, rank, local)
+    finally:
+        if world > 1 and args.impl == "ours":
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

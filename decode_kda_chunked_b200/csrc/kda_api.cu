@@ -1,0 +1,307 @@
+// Host side of libkda.so: the C ABI declared in include/kda.h.
+//
+// Every entry point validates its arguments on the host and returns an error
+// code before launching anything; it allocates no device memory (scratch is
+// the caller's workspace) and never synchronises except in
+// kda_get_device_status().
+#include <cstdlib>
+#include <cstring>
+
+#include "kda_internal.cuh"
+
+namespace kda {
+
+// Per-device status word.  Kernels OR STATUS_* bits into it; the host reads
+// and clears it in kda_get_device_status().
+__device__ unsigned int g_device_status;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+unsigned int *g_status_addr[kMaxDevices];  // cached device address per ordinal
+
+constexpr int kMaxScheduledRequests = 16384;  // longer lists run in index order
+
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+bool env_flag(const char *name) {
+  const char *v = std::getenv(name);
+  return v && v[0] && std::strcmp(v, "0") != 0;
+}
+
+bool valid_dtype(kda_dtype d) { return d == KDA_BF16 || d == KDA_F32; }
+size_t dsize(kda_dtype d) { return d == KDA_BF16 ? 2 : 4; }
+
+struct Range {
+  const char *lo, *hi;
+};
+Range span(const void *p, size_t bytes) {
+  const char *c = static_cast<const char *>(p);
+  return {c, c + bytes};
+}
+bool overlap(Range a, Range b) {
+  return a.lo && b.lo && a.lo < b.hi && b.lo < a.hi;
+}
+
+bool head_dims_supported(int dk, int dv) { return dk == dv && (dk == 64 || dk == 128); }
+
+kda_status check_prefill(const kda_prefill_args *a) {
+  if (!a) return KDA_ERR_INVALID_ARG;
+  if (a->n_req < 0 || a->total_tokens < 0 || a->H <= 0 || a->dk <= 0 || a->dv <= 0)
+    return KDA_ERR_INVALID_ARG;
+  if (!valid_dtype(a->in_dtype) || !valid_dtype(a->out_dtype)) return KDA_ERR_INVALID_ARG;
+  if (!head_dims_supported(a->dk, a->dv)) return KDA_ERR_UNSUPPORTED;
+  if (a->snapshot_stride < 0 || a->snapshot_stride % KDA_CHUNK != 0) return KDA_ERR_INVALID_ARG;
+  if (a->n_req == 0) return KDA_OK;
+  if (!a->cu_seqlens) return KDA_ERR_INVALID_ARG;
+  if (a->total_tokens > 0 && (!a->q || !a->k || !a->v || !a->g || !a->beta || !a->o))
+    return KDA_ERR_INVALID_ARG;
+  if (a->snapshot_stride > 0 && (!a->cu_snapshots || !a->snapshots)) return KDA_ERR_INVALID_ARG;
+  const void *ptrs[] = {a->q, a->k, a->v, a->g, a->beta, a->cu_seqlens, a->initial_state,
+                        a->o, a->final_state, a->cu_snapshots, a->snapshots};
+  for (const void *p : ptrs)
+    if (p && !aligned16(p)) return KDA_ERR_INVALID_ARG;
+  if (a->cu_seqlens_host) {
+    const int32_t *cu = a->cu_seqlens_host;
+    if (cu[0] != 0) return KDA_ERR_INVALID_ARG;
+    for (int r = 0; r < a->n_req; ++r)
+      if (cu[r + 1] < cu[r]) return KDA_ERR_INVALID_ARG;
+    if (cu[a->n_req] != a->total_tokens) return KDA_ERR_INVALID_ARG;
+  }
+  // outputs must not overlap inputs (final_state may alias initial_state exactly)
+  const size_t T = (size_t)a->total_tokens, H = (size_t)a->H, dk = (size_t)a->dk,
+               dv = (size_t)a->dv, n = (size_t)a->n_req;
+  const size_t st = n * H * dk * dv * 4;
+  Range in[] = {span(a->q, T * H * dk * dsize(a->in_dtype)),
+                span(a->k, T * H * dk * dsize(a->in_dtype)),
+                span(a->v, T * H * dv * dsize(a->in_dtype)), span(a->g, T * H * dk * 4),
+                span(a->beta, T * H * 4), span(a->cu_seqlens, (n + 1) * 4)};
+  Range o = span(a->o, T * H * dv * dsize(a->out_dtype));
+  Range fs = span(a->final_state, st);
+  Range is = span(a->initial_state, st);
+  for (Range r : in) {
+    if (overlap(o, r) || overlap(fs, r)) return KDA_ERR_INVALID_ARG;
+  }
+  if (overlap(o, fs) || overlap(o, is)) return KDA_ERR_INVALID_ARG;
+  if (a->final_state && a->initial_state && a->final_state != a->initial_state &&
+      overlap(fs, is))
+    return KDA_ERR_INVALID_ARG;
+  return KDA_OK;
+}
+
+size_t prefill_ws(int n_req) {
+  if (n_req <= 1 || n_req > kMaxScheduledRequests) return 0;
+  return align256((size_t)n_req * sizeof(int32_t));
+}
+
+kda_status from_cuda(cudaError_t e) { return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA; }
+
+}  // namespace
+
+unsigned int *device_status_word() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  if (!g_status_addr[dev]) {
+    void *addr = nullptr;
+    if (cudaGetSymbolAddress(&addr, g_device_status) != cudaSuccess) return nullptr;
+    g_status_addr[dev] = static_cast<unsigned int *>(addr);
+  }
+  return g_status_addr[dev];
+}
+
+}  // namespace kda
+
+using namespace kda;
+
+extern "C" {
+
+size_t kda_prefill_workspace_size(const kda_prefill_args *args) {
+  if (check_prefill(args) != KDA_OK) return 0;
+  return prefill_ws(args->n_req);
+}
+
+kda_status kda_prefill_chunked(const kda_prefill_args *a, void *workspace,
+                               size_t workspace_bytes, void *stream) {
+  kda_status st = check_prefill(a);
+  if (st != KDA_OK) return st;
+  if (a->n_req == 0) return KDA_OK;
+  const size_t need = prefill_ws(a->n_req);
+  if (need > 0 && (!workspace || workspace_bytes < need ||
+                   (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0))
+    return KDA_ERR_WORKSPACE;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  PrefillParams p{};
+  p.q = a->q; p.k = a->k; p.v = a->v; p.g = a->g; p.beta = a->beta;
+  p.cu_seqlens = a->cu_seqlens;
+  p.initial_state = a->initial_state;
+  p.o = a->o;
+  p.final_state = a->final_state;
+  p.cu_snapshots = a->cu_snapshots;
+  p.snapshots = a->snapshots;
+  p.n_req = a->n_req; p.total_tokens = a->total_tokens;
+  p.H = a->H; p.dk = a->dk; p.dv = a->dv;
+  p.snapshot_stride = a->snapshot_stride;
+  p.validate = env_flag("KDA_VALIDATE");
+  p.status = device_status_word();
+  if (!p.status) return KDA_ERR_CUDA;
+  if (need > 0) {
+    int32_t *order = static_cast<int32_t *>(workspace);
+    cudaError_t e = launch_schedule(a->cu_seqlens, a->n_req, order, s);
+    if (e != cudaSuccess) return KDA_ERR_CUDA;
+    p.order = order;
+  }
+  const bool use_tc = prefill_tc_supported(a->dk, a->dv, a->in_dtype) && !env_flag("KDA_FORCE_SIMT");
+  if (use_tc) return from_cuda(launch_prefill_tc(p, a->in_dtype, a->out_dtype, s));
+  p.n_slices = prefill_simt_slices(a->dk, a->dv, false);
+  return from_cuda(launch_prefill_simt(p, a->in_dtype, a->out_dtype, s));
+}
+
+size_t kda_local_state_workspace_size(const kda_local_state_args *a) {
+  (void)a;
+  return 0;
+}
+
+kda_status kda_chunk_local_state(const kda_local_state_args *a, void *workspace,
+                                 size_t workspace_bytes, void *stream) {
+  (void)workspace;
+  (void)workspace_bytes;
+  if (!a) return KDA_ERR_INVALID_ARG;
+  if (a->n_seg <= 0 || a->total_tokens < 0 || a->H <= 0) return KDA_ERR_INVALID_ARG;
+  if (!valid_dtype(a->in_dtype)) return KDA_ERR_INVALID_ARG;
+  if (!head_dims_supported(a->dk, a->dv)) return KDA_ERR_UNSUPPORTED;
+  if (!a->seg_cu || !a->s_loc || !a->m) return KDA_ERR_INVALID_ARG;
+  if (a->total_tokens > 0 && (!a->k || !a->v || !a->g || !a->beta)) return KDA_ERR_INVALID_ARG;
+  const void *ptrs[] = {a->k, a->v, a->g, a->beta, a->seg_cu, a->s_loc, a->m};
+  for (const void *p : ptrs)
+    if (p && !aligned16(p)) return KDA_ERR_INVALID_ARG;
+  if (a->seg_cu_host) {
+    if (a->seg_cu_host[0] != 0 || a->seg_cu_host[a->n_seg] != a->total_tokens)
+      return KDA_ERR_INVALID_ARG;
+    for (int s = 0; s < a->n_seg; ++s)
+      if (a->seg_cu_host[s + 1] < a->seg_cu_host[s]) return KDA_ERR_INVALID_ARG;
+  }
+  const size_t T = (size_t)a->total_tokens, H = (size_t)a->H, dk = (size_t)a->dk,
+               dv = (size_t)a->dv, n = (size_t)a->n_seg;
+  Range outs[] = {span(a->s_loc, n * H * dk * dv * 4), span(a->m, n * H * dk * dk * 4)};
+  Range ins[] = {span(a->k, T * H * dk * dsize(a->in_dtype)),
+                 span(a->v, T * H * dv * dsize(a->in_dtype)), span(a->g, T * H * dk * 4),
+                 span(a->beta, T * H * 4), span(a->seg_cu, (n + 1) * 4)};
+  if (overlap(outs[0], outs[1])) return KDA_ERR_INVALID_ARG;
+  for (Range o : outs)
+    for (Range i : ins)
+      if (overlap(o, i)) return KDA_ERR_INVALID_ARG;
+
+  PrefillParams p{};
+  p.k = a->k; p.v = a->v; p.g = a->g; p.beta = a->beta;
+  p.cu_seqlens = a->seg_cu;
+  p.n_req = a->n_seg; p.total_tokens = a->total_tokens;
+  p.H = a->H; p.dk = a->dk; p.dv = a->dv;
+  p.local_mode = 1;
+  p.s_loc = a->s_loc;
+  p.m = a->m;
+  p.validate = env_flag("KDA_VALIDATE");
+  p.status = device_status_word();
+  if (!p.status) return KDA_ERR_CUDA;
+  p.n_slices = prefill_simt_slices(a->dk, a->dv, true);
+  return from_cuda(launch_prefill_simt(p, a->in_dtype, KDA_F32, static_cast<cudaStream_t>(stream)));
+}
+
+kda_status kda_state_combine(const float *s_loc, const float *m, const float *s_init,
+                             int32_t n_seg, int32_t H, int32_t dk, int32_t dv, float *s_in,
+                             float *s_final, void *stream) {
+  if (n_seg <= 0 || H <= 0 || dk <= 0 || dv <= 0) return KDA_ERR_INVALID_ARG;
+  if (!head_dims_supported(dk, dv)) return KDA_ERR_UNSUPPORTED;
+  if (!s_loc || !m) return KDA_ERR_INVALID_ARG;
+  const void *ptrs[] = {s_loc, m, s_init, s_in, s_final};
+  for (const void *p : ptrs)
+    if (p && !aligned16(p)) return KDA_ERR_INVALID_ARG;
+  const size_t n = n_seg, h = H, k = dk, v = dv;
+  Range ins[] = {span(s_loc, n * h * k * v * 4), span(m, n * h * k * k * 4),
+                 span(s_init, h * k * v * 4)};
+  Range outs[] = {span(s_in, n * h * k * v * 4), span(s_final, h * k * v * 4)};
+  if (overlap(outs[0], outs[1])) return KDA_ERR_INVALID_ARG;
+  for (Range o : outs)
+    for (Range i : ins)
+      if (overlap(o, i)) return KDA_ERR_INVALID_ARG;
+  return from_cuda(launch_combine(s_loc, m, s_init, n_seg, H, dk, dv, s_in, s_final,
+                                  static_cast<cudaStream_t>(stream)));
+}
+
+kda_status kda_decode_step(const kda_decode_args *a, void *stream) {
+  if (!a) return KDA_ERR_INVALID_ARG;
+  if (a->n < 0 || a->H <= 0 || a->dk <= 0 || a->dv <= 0 || a->n_slots < 0)
+    return KDA_ERR_INVALID_ARG;
+  if (!valid_dtype(a->in_dtype) || !valid_dtype(a->out_dtype)) return KDA_ERR_INVALID_ARG;
+  if (!head_dims_supported(a->dk, a->dv)) return KDA_ERR_UNSUPPORTED;
+  if (a->n == 0) return KDA_OK;
+  if (!a->q || !a->k || !a->v || !a->g || !a->beta || !a->state || !a->o)
+    return KDA_ERR_INVALID_ARG;
+  if (!a->slot && a->n_slots < a->n) return KDA_ERR_INVALID_ARG;
+  const void *ptrs[] = {a->q, a->k, a->v, a->g, a->beta, a->state, a->slot, a->o};
+  for (const void *p : ptrs)
+    if (p && !aligned16(p)) return KDA_ERR_INVALID_ARG;
+  const size_t n = a->n, H = a->H, dk = a->dk, dv = a->dv;
+  Range st = span(a->state, (size_t)a->n_slots * H * dk * dv * 4);
+  Range o = span(a->o, n * H * dv * dsize(a->out_dtype));
+  Range ins[] = {span(a->q, n * H * dk * dsize(a->in_dtype)),
+                 span(a->k, n * H * dk * dsize(a->in_dtype)),
+                 span(a->v, n * H * dv * dsize(a->in_dtype)), span(a->g, n * H * dk * 4),
+                 span(a->beta, n * H * 4), span(a->slot, a->slot ? n * 4 : 0)};
+  if (overlap(o, st)) return KDA_ERR_INVALID_ARG;
+  for (Range i : ins)
+    if (overlap(o, i) || overlap(st, i)) return KDA_ERR_INVALID_ARG;
+  DecodeParams p{};
+  p.q = a->q; p.k = a->k; p.v = a->v; p.g = a->g; p.beta = a->beta;
+  p.state = a->state; p.slot = a->slot; p.o = a->o;
+  p.n = a->n; p.H = a->H; p.dk = a->dk; p.dv = a->dv; p.n_slots = a->n_slots;
+  p.validate = env_flag("KDA_VALIDATE");
+  p.status = device_status_word();
+  if (!p.status) return KDA_ERR_CUDA;
+  return from_cuda(launch_decode(p, a->in_dtype, a->out_dtype, static_cast<cudaStream_t>(stream)));
+}
+
+int32_t kda_snapshot_count(int32_t len, int32_t stride) {
+  return (stride > 0 && len > 0) ? len / stride : 0;
+}
+
+kda_status kda_get_device_status(void *stream) {
+  if (cudaStreamSynchronize(static_cast<cudaStream_t>(stream)) != cudaSuccess) return KDA_ERR_CUDA;
+  unsigned int *addr = device_status_word();
+  if (!addr) return KDA_ERR_CUDA;
+  unsigned int word = 0;
+  if (cudaMemcpy(&word, addr, sizeof(word), cudaMemcpyDeviceToHost) != cudaSuccess)
+    return KDA_ERR_CUDA;
+  if (word != 0) {
+    const unsigned int zero = 0;
+    if (cudaMemcpy(addr, &zero, sizeof(zero), cudaMemcpyHostToDevice) != cudaSuccess)
+      return KDA_ERR_CUDA;
+  }
+  if (word & STATUS_TIMEOUT) return KDA_ERR_TIMEOUT;
+  if (word & STATUS_GATE_RANGE) return KDA_ERR_GATE_RANGE;
+  if (word & STATUS_BAD_SEQLENS) return KDA_ERR_INVALID_ARG;
+  return KDA_OK;
+}
+
+const char *kda_status_string(kda_status status) {
+  switch (status) {
+    case KDA_OK: return "KDA_OK";
+    case KDA_ERR_INVALID_ARG: return "KDA_ERR_INVALID_ARG";
+    case KDA_ERR_UNSUPPORTED: return "KDA_ERR_UNSUPPORTED";
+    case KDA_ERR_CUDA: return "KDA_ERR_CUDA";
+    case KDA_ERR_GATE_RANGE: return "KDA_ERR_GATE_RANGE";
+    case KDA_ERR_TIMEOUT: return "KDA_ERR_TIMEOUT";
+    case KDA_ERR_WORKSPACE: return "KDA_ERR_WORKSPACE";
+  }
+  return "KDA_ERR_UNKNOWN";
+}
+
+int32_t kda_version(void) { return KDA_VERSION; }
+
+int32_t kda_prefill_uses_tensor_cores(int32_t dk, int32_t dv, kda_dtype in_dtype) {
+  return (prefill_tc_supported(dk, dv, in_dtype) && !env_flag("KDA_FORCE_SIMT")) ? 1 : 0;
+}
+
+}  // extern "C"

@@ -1,0 +1,90 @@
+// Internal declarations shared by the libkda.so translation units.
+// Nothing here is part of the public C ABI (include/kda.h).
+#pragma once
+
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "kda.h"
+
+namespace kda {
+
+// Bits of the per-device status word (device-side error reporting).
+enum : unsigned int {
+  STATUS_GATE_RANGE = 1u << 0,   // g outside [-5, 0] or beta outside [0, 1]
+  STATUS_TIMEOUT = 1u << 1,      // a bounded wait gave up
+  STATUS_BAD_SEQLENS = 1u << 2,  // cu_seqlens inconsistent with total_tokens
+};
+
+constexpr int kChunk = KDA_CHUNK;
+constexpr float kGateLower = -5.0f;
+
+// Device code reports errors by OR-ing STATUS_* bits into the per-device
+// status word whose address the host passes in every parameter block
+// (`status`).  Kernels never trap.
+__device__ __forceinline__ void set_status(unsigned int *status, unsigned int bits) {
+  if (status) atomicOr(status, bits);
+}
+
+// Parameters of the chunked prefill kernels (plain pointers, resolved sizes).
+struct PrefillParams {
+  const void *q, *k, *v;
+  const float *g, *beta;
+  const int32_t *cu_seqlens;
+  const int32_t *order;          // work order over requests (longest first) or NULL
+  const float *initial_state;    // NULL = zeros
+  void *o;                       // NULL = not written (local-state mode)
+  float *final_state;            // NULL = not written
+  const int32_t *cu_snapshots;
+  float *snapshots;
+  int n_req, total_tokens, H, dk, dv;
+  int snapshot_stride;
+  int n_slices;                  // column slices per (request, head)
+  int validate;
+  unsigned int *status;
+  // local-state mode: columns [0, dv) of the augmented state are S_loc (V,
+  // zero start), columns [dv, dv + dk) are M (zero V, identity start).
+  int local_mode;
+  float *s_loc;                  // [n_seg, H, dk, dv]
+  float *m;                      // [n_seg, H, dk, dk]
+};
+
+struct DecodeParams {
+  const void *q, *k, *v;
+  const float *g, *beta;
+  float *state;
+  const int32_t *slot;
+  void *o;
+  int n, H, dk, dv, n_slots;
+  int validate;
+  unsigned int *status;
+};
+
+// Launchers (return cudaGetLastError() of the launch).
+cudaError_t launch_prefill_simt(const PrefillParams &p, kda_dtype in_dtype, kda_dtype out_dtype,
+                                cudaStream_t stream);
+cudaError_t launch_prefill_tc(const PrefillParams &p, kda_dtype in_dtype, kda_dtype out_dtype,
+                              cudaStream_t stream);
+bool prefill_tc_supported(int dk, int dv, kda_dtype in_dtype);
+int prefill_simt_slices(int dk, int dv, bool local_mode);
+cudaError_t launch_schedule(const int32_t *cu_seqlens, int n_req, int32_t *order,
+                            cudaStream_t stream);
+cudaError_t launch_decode(const DecodeParams &p, kda_dtype in_dtype, kda_dtype out_dtype,
+                          cudaStream_t stream);
+cudaError_t launch_combine(const float *s_loc, const float *m, const float *s_init, int n_seg,
+                           int H, int dk, int dv, float *s_in, float *s_final,
+                           cudaStream_t stream);
+unsigned int *device_status_word();  // address of the current device's status word
+
+// Element loads/stores shared by the kernels.
+__device__ __forceinline__ float load_elem(const float *p, size_t i) { return p[i]; }
+__device__ __forceinline__ float load_elem(const __nv_bfloat16 *p, size_t i) {
+  return __bfloat162float(p[i]);
+}
+__device__ __forceinline__ void store_elem(float *p, size_t i, float x) { p[i] = x; }
+__device__ __forceinline__ void store_elem(__nv_bfloat16 *p, size_t i, float x) {
+  p[i] = __float2bfloat16_rn(x);
+}
+
+}  // namespace kda
