@@ -205,15 +205,21 @@ def cpu_model() -> str:
 # arms
 # ---------------------------------------------------------------------------
 
-def workload_inputs(device, seed):
+def workload_inputs(device, seed, n_req=None):
+    """The varlen workload; ``n_req`` keeps only its first requests (small
+    cases for profiler captures)."""
     from decode_kda_chunked_b200 import inputs as I
-    return I.varlen(device=device, seed=seed)
+    if n_req is None:
+        return I.varlen(device=device, seed=seed)
+    lens = I.varlen_lengths(0)[:n_req]
+    return I.make_prefill_inputs(lens, H=32, dk=128, dv=128, seed=seed, device=device)
 
 
 def workload_config(inp, world):
+    subset = "" if inp.n_req == 64 else f" (first {inp.n_req} requests only)"
     return {"workload": "varlen packed prefill: 64 requests, lengths log-uniform on [128, 4096] "
                         "(seed 0), H=32, d_k=d_v=128, bf16 q/k/v, fp32 g/beta/o/state, "
-                        "zero initial states, final states out",
+                        "zero initial states, final states out" + subset,
             "n_req": inp.n_req, "total_tokens": inp.total_tokens, "H": 32, "d": 128,
             "global_batch": inp.n_req * world, "seq_len": inp.total_tokens,
             "parallelism": f"replicas x{world} (requests shard, no collective)",
@@ -263,7 +269,7 @@ def run_ours(args, world, rank, local):
     dev = torch.device("cuda", local)
     torch.cuda.set_device(dev)
     lib = kda.load()
-    inp = workload_inputs(dev, seed=rank)
+    inp = workload_inputs(dev, seed=rank, n_req=args.prefill_requests)
     T, H, dk, dv = inp.total_tokens, 32, 128, 128
     n_req = inp.n_req
     cu_host = torch.tensor([0] + list(__import__("itertools").accumulate(inp.lengths)),
@@ -352,7 +358,7 @@ def bench_decode(args, dev, peaks, peak_kind, rank):
 
     import decode_kda_chunked_b200 as kda
     from decode_kda_chunked_b200 import inputs as I
-    N, H, d = 256, 32, 128
+    N, H, d = args.decode_requests, 32, 128
     steps = max(args.steps, 10)
     warm = max(args.warmup, 3)
     x = I.decode(steps + warm, N=N, H=H, d=d, device=dev, seed=rank)
@@ -376,8 +382,8 @@ def bench_decode(args, dev, peaks, peak_kind, rank):
     ms = statistics.mean(per)
     b = decode_bytes(N, H, d)
     gbs = b / (ms * 1e-3) / 1e9
-    return {"workload": "256 requests x H=32 x 128x128 fp32 states, 1 bf16 token each; state "
-                        "pool 512 MiB > L2",
+    return {"workload": f"{N} requests x H=32 x 128x128 fp32 states, 1 bf16 token each; "
+                        f"state pool {N * H * d * d * 4 >> 20} MiB",
             "value": gbs, "unit": "GB/s", "ms_per_step": ms, "steps": steps,
             "bytes_per_step": b,
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -440,6 +446,10 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--prefill-requests", type=int, default=None,
+                    help="keep only the first N requests of the varlen workload (profiling)")
+    ap.add_argument("--decode-requests", type=int, default=256,
+                    help="requests in the decode step (256 in the standard workload)")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3  # the timing rules ask for at least 3 warm-up steps
