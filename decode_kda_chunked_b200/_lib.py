@@ -60,7 +60,7 @@ _lock = threading.Lock()
 EXPORTS = ("kda_prefill_workspace_size", "kda_prefill_chunked", "kda_local_state_workspace_size",
            "kda_chunk_local_state", "kda_state_combine", "kda_decode_step", "kda_snapshot_count",
            "kda_get_device_status", "kda_status_string", "kda_version",
-           "kda_prefill_uses_tensor_cores")
+           "kda_prefill_uses_tensor_cores", "kda_prefill_chunked_noalloc")
 
 
 def load(path: str = LIB_PATH):
@@ -95,6 +95,8 @@ def load(path: str = LIB_PATH):
         lib.kda_status_string.argtypes = [ctypes.c_int]
         lib.kda_version.restype = _i32
         lib.kda_version.argtypes = []
+        lib.kda_prefill_chunked_noalloc.restype = ctypes.c_int
+        lib.kda_prefill_chunked_noalloc.argtypes = [P(PrefillArgs), _vp]
         lib.kda_prefill_uses_tensor_cores.restype = _i32
         lib.kda_prefill_uses_tensor_cores.argtypes = [_i32, _i32, ctypes.c_int]
         _lib = lib

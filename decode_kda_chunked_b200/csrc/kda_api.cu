@@ -305,3 +305,41 @@ int32_t kda_prefill_uses_tensor_cores(int32_t dk, int32_t dv, kda_dtype in_dtype
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Allocation-free prefill: the workspace of kda_prefill_chunked (the
+// longest-first request order) comes from a fixed array in this library.
+// ---------------------------------------------------------------------------
+
+namespace kda {
+namespace {
+
+// Scratch of kda_prefill_chunked_noalloc.  Host code must not use this name
+// as a device address: it is a host-side stand-in.  The device address comes
+// from cudaGetSymbolAddress, looked up once per device.
+static __device__ __align__(256) int32_t g_noalloc_order[KDA_NOALLOC_MAX_REQUESTS];
+
+int32_t *g_noalloc_addr[kMaxDevices];  // device address of g_noalloc_order per ordinal
+
+// Per-device set-up on the first call with that device current.
+int32_t *noalloc_scratch() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
+  if (!g_noalloc_addr[dev]) {
+    int32_t *ptr = nullptr;
+    if (cudaGetSymbolAddress((void **)&ptr, g_noalloc_order) != cudaSuccess) return nullptr;
+    g_noalloc_addr[dev] = ptr;
+  }
+  return g_noalloc_addr[dev];
+}
+
+}  // namespace
+}  // namespace kda
+
+extern "C" kda_status kda_prefill_chunked_noalloc(const kda_prefill_args *args, void *stream) {
+  if (!args) return KDA_ERR_INVALID_ARG;
+  if (args->n_req > KDA_NOALLOC_MAX_REQUESTS) return KDA_ERR_WORKSPACE;
+  int32_t *scratch = kda::noalloc_scratch();
+  if (!scratch) return KDA_ERR_CUDA;
+  return kda_prefill_chunked(args, scratch, sizeof(kda::g_noalloc_order), stream);
+}

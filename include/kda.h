@@ -146,6 +146,39 @@ size_t kda_prefill_workspace_size(const kda_prefill_args *args);
 kda_status kda_prefill_chunked(const kda_prefill_args *args, void *workspace,
                                size_t workspace_bytes, void *stream);
 
+/* Largest n_req that kda_prefill_chunked_noalloc accepts. */
+#define KDA_NOALLOC_MAX_REQUESTS 16384
+
+/*
+ * Allocation-free variant of kda_prefill_chunked.  The pages have no
+ * counterpart to this entry point; it exists for callers that cannot hand
+ * the library a device workspace, for example:
+ *   - an inference engine that reserves all device memory for its own pools
+ *     at start-up and has no buffer to spare for a plug-in kernel;
+ *   - a custom-op or plug-in host whose interface gives the op no way to
+ *     request scratch memory;
+ *   - latency-critical code that cannot call cudaMalloc, which may
+ *     synchronise the device and take milliseconds.
+ *
+ * Same arguments, results and error codes as kda_prefill_chunked, except
+ * that the scratch (one int32 per request: the longest-first work order)
+ * lives in a fixed array inside libkda.so instead of a caller workspace:
+ *   - the array holds KDA_NOALLOC_MAX_REQUESTS int32 (64 KiB) and is resident
+ *     on every GPU that loads the library until the process exits;
+ *   - n_req > KDA_NOALLOC_MAX_REQUESTS returns KDA_ERR_WORKSPACE and launches
+ *     nothing;
+ *   - the first call on each device looks up the array's device address
+ *     (cudaGetSymbolAddress) with that device current; make that first call
+ *     before any stream capture;
+ *   - every call on a device shares the one array, which keeps the last
+ *     call's contents.  Nothing in it needs to start at zero: each call
+ *     rewrites entries 0 .. n_req-1 before reading them.  Calls that overlap
+ *     on the GPU (for example on two streams of the same device) race on the
+ *     array, so serialise them;
+ *   - it calls no cudaMalloc, cudaFree or other allocating routine.
+ */
+kda_status kda_prefill_chunked_noalloc(const kda_prefill_args *args, void *stream);
+
 /* ------------------------------------------------------------------------ */
 /* Context-parallel split of one long sequence into segments.               */
 /* ------------------------------------------------------------------------ */
