@@ -153,7 +153,9 @@ kda_status kda_prefill_chunked(const kda_prefill_args *a, void *workspace,
     if (e != cudaSuccess) return KDA_ERR_CUDA;
     p.order = order;
   }
-  const bool use_tc = prefill_tc_supported(a->dk, a->dv, a->in_dtype) && !env_flag("KDA_FORCE_SIMT");
+  // the tensor-core kernel needs at least one token to build its TMA maps
+  const bool use_tc = prefill_tc_supported(a->dk, a->dv, a->in_dtype) && a->total_tokens > 0 &&
+                      !env_flag("KDA_FORCE_SIMT");
   if (use_tc) return from_cuda(launch_prefill_tc(p, a->in_dtype, a->out_dtype, s));
   p.n_slices = prefill_simt_slices(a->dk, a->dv, false);
   return from_cuda(launch_prefill_simt(p, a->in_dtype, a->out_dtype, s));

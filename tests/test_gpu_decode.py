@@ -17,7 +17,7 @@ def _step_inputs(x, t):
 
 
 @pytest.mark.parametrize("d", [64, 128])
-@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "fp32"])
 def test_decode_small_every_element(d, dtype):
     steps, N, H = 20, 5, 3
     x = I.decode(steps, N=N, H=H, d=d, dtype=dtype, seed=3)

@@ -67,7 +67,7 @@ RAGGED = [1, 63, 64, 65, 127, 128, 200, 0, 513]
 
 
 @pytest.mark.parametrize("d", [64, 128])
-@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32], ids=["bf16", "fp32"])
 def test_ragged_varlen(d, dtype):
     inp = I.make_prefill_inputs(RAGGED, H=3, dk=d, dv=d, dtype=dtype, seed=7, s0_std=0.1)
     out = run_prefill(inp, stride=64)
@@ -81,6 +81,20 @@ def test_weak_decay_long_memory():
                                 s0_std=0.1, gate_scale=0.02)
     out = run_prefill(inp, stride=128)
     check_all_chains(inp, out, 128, TOL_BF16)
+
+
+def test_tensor_core_and_simt_kernels_agree(monkeypatch):
+    """bf16 inputs with d=128 run on the tcgen05 kernel; KDA_FORCE_SIMT=1 runs the
+    fp32 SIMT kernel on the same inputs.  Both must agree within tolerance."""
+    assert kda.kda_prefill_uses_tensor_cores(128, 128)
+    inp = I.make_prefill_inputs([333, 64, 700], H=3, dk=128, dv=128, seed=29, s0_std=0.1,
+                                gate_scale=0.5)
+    tc = run_prefill(inp, stride=64)
+    monkeypatch.setenv("KDA_FORCE_SIMT", "1")
+    assert not kda.kda_prefill_uses_tensor_cores(128, 128)
+    simt = run_prefill(inp, stride=64)
+    for n in ("o", "final_state", "snapshots"):
+        assert rel_err(tc[n], simt[n]) <= TOL_BF16, n
 
 
 def test_bf16_output():
