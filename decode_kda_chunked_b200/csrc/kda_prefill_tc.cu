@@ -29,9 +29,13 @@
 // swizzle in shared memory): bf16 operands for the gate-scaled products would
 // cost about 2e-3 of relative accuracy, tf32 stays near 5e-4.
 //
-// One CTA (4 warps) runs one (request, head) chain: 128 threads, TMEM lane =
-// thread.  Thread 0 issues TMA loads and MMAs; every wait is bounded and a
-// timeout is reported through the status word.
+// One CTA runs one (request, head) chain with 16 worker warps and one control
+// warp.  Worker warp w reaches the TMEM lane quarter w % 4, and the four warps
+// sharing a quarter split the columns.  The control warp issues the TMA loads
+// and every tcgen05.mma; workers and control hand off through mbarriers
+// (operands ready / MMA done / raw tiles consumed), so MMA issue never stalls
+// a worker warp.  Every wait is bounded; a timeout is reported through the
+// status word.
 #include "kda_internal.cuh"
 #include "kda_sm100.cuh"
 
@@ -42,36 +46,44 @@ using namespace sm100;
 
 constexpr int C = 64;     // chunk
 constexpr int DH = 128;   // head dim (dk = dv)
-constexpr int NT = 128;   // threads per CTA
+constexpr int NT = 512;   // worker threads per CTA: 16 warps (plus one control warp)
+constexpr float LOG2E = 1.4426950408889634f;
+
+// Thread (g, l): warp w = tid / 32 owns TMEM lane quarter w % 4, so
+// l = 32 (w % 4) + tid % 32 is the thread's TMEM lane, and g = w / 4 picks a
+// quarter of the columns (32 of 128, or 16 of 64).
 
 // ---- shared memory map (byte offsets from a 1024-aligned base) ----
 constexpr uint32_t OFF_KRAW = 0;        // bf16 [64 x 128]: 2 TMA boxes of 64 cols (SW128)
 constexpr uint32_t OFF_QRAW = 16384;
 constexpr uint32_t OFF_VRAW = 32768;
-constexpr uint32_t OFF_GRAW = 49152;    // fp32 [64 x 128]: 4 TMA boxes of 32 cols (SW128)
+constexpr uint32_t OFF_GRAW = 49152;    // fp32 [64 x 128]: 4 TMA boxes of 32 cols (SW128);
+                                        // rewritten in place with log2(e) * cumsum(g)
 constexpr uint32_t RAW_BYTES = 81920;
-constexpr uint32_t OFF_R = 81920;       // 4 x [16 x 128] tf32 B operands; later W [64 x 128]
+constexpr uint32_t OFF_R = 81920;       // 4 x [16 x 128] tf32 B operands (R_b); then T-solve
+                                        // scratch (two [64 x 64] fp32); then W [64 x 128]
+constexpr uint32_t OFF_MS = OFF_R;          // beta*A strict lower, rotated rows
+constexpr uint32_t OFF_TI = OFF_R + 16384;  // T = (I + beta A)^-1, rotated rows
 constexpr uint32_t OFF_GQ = 114688;     // (gamma*Q) [64 x 128] tf32 B operand
 constexpr uint32_t OFF_KHT = 147456;    // Khat^T [128 x 64] tf32 B operand
 constexpr uint32_t OFF_TB = 180224;     // T Diag(beta) [64 x 64] tf32 B operand
 constexpr uint32_t OFF_P = 196608;      // P [64 x 64] tf32 B operand
-constexpr uint32_t OFF_E = 212992;      // E[b*4+a][128] = exp(G_ra - G_rb), b <= a (8 KB)
-constexpr uint32_t OFF_EGR = 221184;    // exp(G_rb)[4][128] (2 KB)
-constexpr uint32_t OFF_BETA = 223232;   // beta[64]
-constexpr uint32_t OFF_BAR = 223488;    // mbarriers + TMEM base + flags
-constexpr uint32_t SMEM_BYTES = 223616;
+constexpr uint32_t OFF_E = 212992;      // E[b*4+a][128] = exp(G_ra - G_rb), b <= a; then
+                                        // the T-solve products ([2][16][17], then [32][33])
+constexpr uint32_t OFF_Y = OFF_E;
+constexpr uint32_t OFF_EGR = 221184;    // exp(G_rb)[4][128]
+constexpr uint32_t OFF_SEG = 223232;    // cumsum segment totals [4][128]
+constexpr uint32_t OFF_GR2 = 225280;    // log2(e) * G at block ends [4][128]
+constexpr uint32_t OFF_BETA = 227328;   // beta[64]
+constexpr uint32_t OFF_BAR = 227584;    // mbarriers + TMEM base + flags
+constexpr uint32_t SMEM_BYTES = 227680;
 constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;  // alignment slack
-// T-solve scratch lives in the raw-tile region once the raw tiles are consumed.
-constexpr uint32_t OFF_MS = 0;          // beta*A strict lower, fp32 [64][65]
-constexpr uint32_t OFF_TI = 16640;      // T = (I + beta A)^-1, fp32 [64][65]
-constexpr uint32_t OFF_Y = 33280;       // level products, fp32 [3][16][17]
-constexpr int LD = 65;
 
 // ---- TMEM column map (512 columns x 128 lanes of fp32) ----
 constexpr uint32_t TM_S = 0;     // S^T (lane = value channel, col = key channel)
-constexpr uint32_t TM_L = 128;   // A-operand scratch: L_b; later V^T [0,64) and (gK)^T [64,128)
+constexpr uint32_t TM_L = 128;   // A-operand buffer 0: L_b; later V^T [0,64), (gK)^T [64,128)
 constexpr uint32_t TM_AP = 256;  // A (lanes 0..63) and P (lanes 64..127), col = j
-constexpr uint32_t TM_X1 = 320;  // W^T, later O^T
+constexpr uint32_t TM_X1 = 320;  // W^T, later O^T   (X1..X2 is A-operand buffer 1 for L_b)
 constexpr uint32_t TM_X2 = 384;  // U~^T -> U^T
 constexpr uint32_t TM_COLS = 512;
 
@@ -79,11 +91,21 @@ struct TcMaps {
   CUtensorMap q, k, v, g;
 };
 
-__device__ __forceinline__ float bf16_at(const unsigned char *tile, int t, int c) {
+__device__ __forceinline__ uint32_t bf16_off(int t, int c) {
   // bf16 [64 x 128] as two 64-column SW128 boxes
-  const uint32_t off = (uint32_t)(c >> 6) * 8192u + (uint32_t)t * 128u +
-                       ((uint32_t)(((c & 63) >> 3) ^ (t & 7)) << 4) + (uint32_t)(c & 7) * 2u;
-  return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(tile + off));
+  return (uint32_t)(c >> 6) * 8192u + (uint32_t)t * 128u +
+         ((uint32_t)(((c & 63) >> 3) ^ (t & 7)) << 4) + (uint32_t)(c & 7) * 2u;
+}
+__device__ __forceinline__ float bf16_at(const unsigned char *tile, int t, int c) {
+  return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(tile + bf16_off(t, c)));
+}
+// four consecutive channels c..c+3 (c % 4 == 0) of row t
+__device__ __forceinline__ void bf16_x4(const unsigned char *tile, int t, int c, float *x) {
+  const uint2 u = *reinterpret_cast<const uint2 *>(tile + bf16_off(t, c));
+  x[0] = __uint_as_float(u.x << 16);
+  x[1] = __uint_as_float(u.x & 0xFFFF0000u);
+  x[2] = __uint_as_float(u.y << 16);
+  x[3] = __uint_as_float(u.y & 0xFFFF0000u);
 }
 __device__ __forceinline__ uint32_t g_off(int t, int c) {
   // fp32 [64 x 128] as four 32-column SW128 boxes
@@ -95,22 +117,36 @@ __device__ __forceinline__ float tf32_rna(float x) {
   asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
   return __uint_as_float(r);
 }
+// [64 x 64] fp32 scratch with each row rotated by its index: row and column
+// walks of a warp both hit 32 distinct banks.
+__device__ __forceinline__ int rot(int r, int c) { return r * 64 + ((c + r) & 63); }
 
 template <typename TOut>
-__global__ void __launch_bounds__(NT, 1)
+__global__ void __launch_bounds__(NT + 32, 1)
     prefill_tc_kernel(const PrefillParams p, const __grid_constant__ TcMaps maps) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char *sm = reinterpret_cast<unsigned char *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   float *sE = reinterpret_cast<float *>(sm + OFF_E);
   float *sEgr = reinterpret_cast<float *>(sm + OFF_EGR);
+  float *sSeg = reinterpret_cast<float *>(sm + OFF_SEG);
+  float *sGr2 = reinterpret_cast<float *>(sm + OFF_GR2);
   float *sB = reinterpret_cast<float *>(sm + OFF_BETA);
-  uint64_t *bar_tma = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
-  uint64_t *bar_mma = bar_tma + 1;
-  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bar_tma + 2);
-  int *s_abort = reinterpret_cast<int *>(s_tmem + 1);
+  uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
+  uint64_t *bar_tma = bars + 0;      // TMA -> workers: raw tiles landed
+  uint64_t *bar_raw = bars + 1;      // workers -> control: raw tiles consumed (16 warps)
+  uint64_t *bar_opsap = bars + 2;    // workers -> control: two L_b buffers built (16 warps)
+  uint64_t *bar_ops = bars + 4;      // workers -> control: next MMA group's operands ready
+  uint64_t *bar_ap = bars + 5;       // control -> workers: A/P MMAs of a round done
+  uint64_t *bar_mma = bars + 7;      // control -> workers: MMA group done
+  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bars + 8);
+  volatile int *s_abort = reinterpret_cast<volatile int *>(s_tmem + 1);
 
-  const int tid = threadIdx.x, warp = tid >> 5;
+  const int tid = threadIdx.x, warp = tid >> 5, lane_id = tid & 31;
+  const bool control = warp == NT / 32;            // warp 16: TMA and MMA issue
+  const int l = ((warp & 3) << 5) | lane_id;       // TMEM lane of a worker thread
+  const int g = (warp >> 2) & 3;                   // worker column quarter
+  const uint32_t lane = (uint32_t)((warp & 3) * 32) << 16;
   const int H = p.H;
   const int r = p.order ? p.order[blockIdx.x / H] : blockIdx.x / H;
   const int h = blockIdx.x % H;
@@ -130,383 +166,429 @@ __global__ void __launch_bounds__(NT, 1)
   if (warp == 0) tmem_alloc(s_tmem, TM_COLS);
   if (tid == 0) {
     mbar_init(bar_tma, 1);
+    mbar_init(bar_raw, NT / 32);
+    mbar_init(bar_opsap, NT / 32);
+    mbar_init(bar_ops, NT / 32);
+    mbar_init(bar_ap, 1);
     mbar_init(bar_mma, 1);
     *s_abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-    tma_prefetch_desc(&maps.q);
-    tma_prefetch_desc(&maps.k);
-    tma_prefetch_desc(&maps.v);
-    tma_prefetch_desc(&maps.g);
   }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tm = *s_tmem;
-  const uint32_t lane = (uint32_t)(warp * 32) << 16;  // this warp's TMEM lane quarter
+  const int n_chunks = (len + C - 1) / C;
 
-  uint32_t tma_phase = 0, mma_phase = 0;
-  auto issue_tma = [&](int c0) {
-    mbar_expect_tx(bar_tma, RAW_BYTES);
-    const int y = bos + c0;
-    for (int half = 0; half < 2; ++half) {
-      const int x = h * DH + 64 * half;
-      tma_load_2d(sm + OFF_KRAW + 8192 * half, &maps.k, x, y, bar_tma);
-      tma_load_2d(sm + OFF_QRAW + 8192 * half, &maps.q, x, y, bar_tma);
-      tma_load_2d(sm + OFF_VRAW + 8192 * half, &maps.v, x, y, bar_tma);
+  if (control) {
+    // ======================= control warp: TMA + MMA issue =======================
+    if (lane_id == 0) {
+      tma_prefetch_desc(&maps.q);
+      tma_prefetch_desc(&maps.k);
+      tma_prefetch_desc(&maps.v);
+      tma_prefetch_desc(&maps.g);
+      auto issue_tma = [&](int c0) {
+        mbar_expect_tx(bar_tma, RAW_BYTES);
+        const int y = bos + c0;
+        for (int half = 0; half < 2; ++half) {
+          const int x = h * DH + 64 * half;
+          tma_load_2d(sm + OFF_KRAW + 8192 * half, &maps.k, x, y, bar_tma);
+          tma_load_2d(sm + OFF_QRAW + 8192 * half, &maps.q, x, y, bar_tma);
+          tma_load_2d(sm + OFF_VRAW + 8192 * half, &maps.v, x, y, bar_tma);
+        }
+        for (int qd = 0; qd < 4; ++qd)
+          tma_load_2d(sm + OFF_GRAW + 8192 * qd, &maps.g, h * DH + 32 * qd, y, bar_tma);
+      };
+      uint32_t ph_raw = 0, ph_opsap[1] = {0}, ph_ops = 0;
+      auto cwait = [&](uint64_t *bar, uint32_t &ph) -> bool {
+        const bool good = *s_abort == 0 && mbar_wait(bar, ph);
+        ph ^= 1u;
+        if (!good) {
+          *s_abort = 1;
+          set_status(p.status, STATUS_TIMEOUT);
+        }
+        tc_fence_after();
+        return good;
+      };
+      if (n_chunks > 0) issue_tma(0);
+      for (int ci = 0; ci < n_chunks; ++ci) {
+        bool good = true;
+        for (int pair = 0; pair < 2 && good; ++pair) {  // A | P: blocks 2*pair, 2*pair+1
+          if (!(good = cwait(bar_opsap, ph_opsap[0]))) break;
+          const uint32_t id = idesc_tf32(16);
+          const int b0 = 2 * pair;
+          const uint32_t r0 = smem_u32(sm + OFF_R + b0 * 8192), r1 = r0 + 8192;
+          // two independent accumulation chains, interleaved so their latencies overlap
+#pragma unroll
+          for (int s = 0; s < DH / 8; ++s) {
+            mma_tf32_ts(tm + TM_AP + 16 * b0, tm + TM_L + 8 * s, sw128_desc(r0, 16, s), id, s > 0);
+            mma_tf32_ts(tm + TM_AP + 16 * b0 + 16, tm + TM_X1 + 8 * s, sw128_desc(r1, 16, s), id,
+                        s > 0);
+          }
+          mma_commit(bar_ap);
+        }
+        if (!good || !cwait(bar_raw, ph_raw)) break;
+        if (ci + 1 < n_chunks) issue_tma((ci + 1) * C);
+        if (!cwait(bar_ops, ph_ops)) break;  // T Diag(beta), V^T, (gK)^T ready
+        {
+          const uint32_t id = idesc_tf32(64);
+          const uint32_t tb = smem_u32(sm + OFF_TB);
+#pragma unroll
+          for (int s = 0; s < C / 8; ++s) {
+            mma_tf32_ts(tm + TM_X2, tm + TM_L + 8 * s, sw128_desc(tb, C, s), id, s > 0);
+            mma_tf32_ts(tm + TM_X1, tm + TM_L + 64 + 8 * s, sw128_desc(tb, C, s), id, s > 0);
+          }
+          mma_commit(bar_mma);
+        }
+        if (!cwait(bar_ops, ph_ops)) break;  // W operand ready
+        {
+          const uint32_t idn = idesc_tf32(64, true), id = idesc_tf32(64);
+          const uint32_t wb = smem_u32(sm + OFF_R), qb = smem_u32(sm + OFF_GQ);
+#pragma unroll
+          for (int s = 0; s < DH / 8; ++s) {
+            mma_tf32_ts(tm + TM_X2, tm + TM_S + 8 * s, sw128_desc(wb, C, s), idn, true);
+            mma_tf32_ts(tm + TM_X1, tm + TM_S + 8 * s, sw128_desc(qb, C, s), id, s > 0);
+          }
+          mma_commit(bar_mma);
+        }
+        if (!cwait(bar_ops, ph_ops)) break;  // S^T scaled by gamma_63
+        {
+          const uint32_t id64 = idesc_tf32(64), id128 = idesc_tf32(128);
+          const uint32_t pb = smem_u32(sm + OFF_P), kb = smem_u32(sm + OFF_KHT);
+#pragma unroll
+          for (int s = 0; s < C / 8; ++s) {
+            mma_tf32_ts(tm + TM_X1, tm + TM_X2 + 8 * s, sw128_desc(pb, C, s), id64, true);
+            mma_tf32_ts(tm + TM_S, tm + TM_X2 + 8 * s, sw128_desc(kb, DH, s), id128, true);
+          }
+          mma_commit(bar_mma);
+        }
+      }
     }
-    for (int qd = 0; qd < 4; ++qd)
-      tma_load_2d(sm + OFF_GRAW + 8192 * qd, &maps.g, h * DH + 32 * qd, y, bar_tma);
-  };
-  // thread 0 waits on an mbarrier, then the CTA synchronises; a timeout aborts the CTA
-  auto wait_bar = [&](uint64_t *bar, uint32_t &phase) -> bool {
-    if (tid == 0) {
-      if (!mbar_wait(bar, phase)) {
+  } else {
+    // ======================= 16 worker warps =======================
+    uint32_t ph_tma = 0, ph_ap[1] = {0}, ph_mma = 0;
+    auto wsync = [&]() { named_sync(1, NT); };
+    // every worker waits, then the workers synchronise so an abort is seen by all
+    auto wwait = [&](uint64_t *bar, uint32_t &ph) -> bool {
+      if (!(*s_abort == 0 && mbar_wait(bar, ph))) {
         *s_abort = 1;
         set_status(p.status, STATUS_TIMEOUT);
       }
-    }
-    phase ^= 1u;
-    __syncthreads();
-    tc_fence_after();
-    return *s_abort == 0;
-  };
-  auto commit_and_wait = [&]() -> bool {
-    if (tid == 0) mma_commit(bar_mma);
-    return wait_bar(bar_mma, mma_phase);
-  };
+      ph ^= 1u;
+      wsync();
+      tc_fence_after();
+      return *s_abort == 0;
+    };
+    // one arrival per warp once all its lanes' writes are visible to the async proxy
+    auto warp_arrive = [&](uint64_t *bar) {
+      fence_async_smem();
+      tc_fence_before();
+      __syncwarp();
+      if (lane_id == 0) mbar_arrive(bar);
+    };
 
-  if (tid == 0 && len > 0) issue_tma(0);
-
-  // ---- initial state -> S^T in TMEM (lane v holds S[:, v]) ----
-  {
-    const float *s0 = p.initial_state ? p.initial_state + ((size_t)(r * H + h)) * DH * DH : nullptr;
-    for (int q = 0; q < 4; ++q) {
+    // initial state -> S^T in TMEM (lane v holds S[:, v])
+    {
+      const float *s0 =
+          p.initial_state ? p.initial_state + ((size_t)(r * H + h)) * DH * DH : nullptr;
       float v[32];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = s0 ? s0[(size_t)(32 * q + j) * DH + tid] : 0.f;
-      tmem_st32(tm + lane + TM_S + 32 * q, v);
+      for (int j = 0; j < 32; ++j) v[j] = s0 ? s0[(size_t)(32 * g + j) * DH + l] : 0.f;
+      tmem_st32(tm + lane + TM_S + 32 * g, v);
+      tmem_wait_st();
     }
-    tmem_wait_st();
-  }
 
-  bool ok = true;
-  for (int c0 = 0; c0 < len && ok; c0 += C) {
-    const int n = min(C, len - c0);
-    if (tid < C) {
-      float b = 0.f;
-      if (tid < n) {
-        b = p.beta[(size_t)(bos + c0 + tid) * H + h];
-        if (p.validate && !(b >= 0.f && b <= 1.f)) set_status(p.status, STATUS_GATE_RANGE);
-      }
-      sB[tid] = b;
-    }
-    if (!(ok = wait_bar(bar_tma, tma_phase))) break;
-
-    // ---- a2: cumulative gate (thread = channel), block-end tables -------------
-    {
-      const int c = tid;
-      float acc = 0.f, gr[4];
-#pragma unroll 8
-      for (int t = 0; t < C; ++t) {
-        float *gp = reinterpret_cast<float *>(sm + OFF_GRAW + g_off(t, c));
-        float gv = 0.f;
-        if (t < n) {
-          gv = *gp;
-          if (p.validate && !(gv >= kGateLower && gv <= 0.f)) set_status(p.status, STATUS_GATE_RANGE);
+    bool ok = true;
+    for (int ci = 0; ci < n_chunks && ok; ++ci) {
+      const int c0 = ci * C;
+      const int n = min(C, len - c0);
+      if (tid < C) {
+        float b = 0.f;
+        if (tid < n) {
+          b = p.beta[(size_t)(bos + c0 + tid) * H + h];
+          if (p.validate && !(b >= 0.f && b <= 1.f)) set_status(p.status, STATUS_GATE_RANGE);
         }
-        acc += gv;
-        *gp = acc;
-        if ((t & 15) == 15) gr[t >> 4] = acc;
+        sB[tid] = b;
       }
-#pragma unroll
-      for (int b = 0; b < 4; ++b) {
-        sEgr[b * DH + c] = __expf(gr[b]);
-#pragma unroll
-        for (int a = 0; a < 4; ++a)
-          if (a >= b) sE[(b * 4 + a) * DH + c] = __expf(gr[a] - gr[b]);
-      }
-    }
-    __syncthreads();
+      if (!(ok = wwait(bar_tma, ph_tma))) break;
 
-    // ---- a3 operands (thread = row): own-block factors, R_b, Khat^T, gamma*Q ----
-    const bool kside = tid < C;
-    const int i = tid & (C - 1);
-    const int bi = i >> 4;
-    const bool valid = i < n;
-    float Lst[DH];
-    {
-      const unsigned char *xraw = sm + (kside ? OFF_KRAW : OFF_QRAW);
-      const int rb = 16 * bi + 15;
+      // ---- a2: cumulative gate (thread = channel l, tokens 16g..16g+15) --------
+      {
+        float gv[16];
 #pragma unroll
-      for (int c = 0; c < DH; c += 4) {
-        const float4 gi = *reinterpret_cast<const float4 *>(sm + OFF_GRAW + g_off(i, c));
-        const float4 grb = *reinterpret_cast<const float4 *>(sm + OFF_GRAW + g_off(rb, c));
-        float x[4], f[4];
-        const float giv[4] = {gi.x, gi.y, gi.z, gi.w}, grv[4] = {grb.x, grb.y, grb.z, grb.w};
-#pragma unroll
-        for (int e = 0; e < 4; ++e) {
-          x[e] = valid ? bf16_at(xraw, i, c + e) : 0.f;
-          f[e] = __expf(giv[e] - grv[e]);
-          Lst[c + e] = x[e] * f[e];
+        for (int j = 0; j < 16; ++j) {
+          const int t = 16 * g + j;
+          gv[j] = (t < n) ? *reinterpret_cast<const float *>(sm + OFF_GRAW + g_off(t, l)) : 0.f;
         }
-        if (kside) {
-          // R_b row (i % 16) of block bi: k_i exp(G_rb - G_i); Khat = R * exp(G_63 - G_rb)
-          float rv[4];
+        if (p.validate)
 #pragma unroll
-          for (int e = 0; e < 4; ++e) rv[e] = tf32_rna(x[e] * __expf(grv[e] - giv[e]));
-          *reinterpret_cast<float4 *>(sm + OFF_R + bi * 8192 + sw128_chunk(16, i & 15, c)) =
-              make_float4(rv[0], rv[1], rv[2], rv[3]);
+          for (int j = 0; j < 16; ++j)
+            if (!(gv[j] >= kGateLower && gv[j] <= 0.f)) set_status(p.status, STATUS_GATE_RANGE);
+#pragma unroll
+        for (int j = 1; j < 16; ++j) gv[j] += gv[j - 1];
+        sSeg[g * DH + l] = gv[15];
+        wsync();
+        float off = 0.f;
+        for (int gg = 0; gg < g; ++gg) off += sSeg[gg * DH + l];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          gv[j] = (gv[j] + off) * LOG2E;
+          *reinterpret_cast<float *>(sm + OFF_GRAW + g_off(16 * g + j, l)) = gv[j];
+        }
+        sGr2[g * DH + l] = gv[15];
+        wsync();
+        sEgr[g * DH + l] = ex2(gv[15]);
+        for (int b = 0; b <= g; ++b) sE[(b * 4 + g) * DH + l] = ex2(gv[15] - sGr2[b * DH + l]);
+        wsync();
+      }
+
+      // ---- a3 operands (thread = row i, channels 32g..32g+31) -----------------
+      const bool kside = l < C;
+      const int i = l & (C - 1);
+      const int bi = i >> 4;
+      const bool valid = i < n;
+      float Lst[32];
+      {
+        const unsigned char *xraw = sm + (kside ? OFF_KRAW : OFF_QRAW);
+        const int rb = 16 * bi + 15;
+#pragma unroll
+        for (int cc = 0; cc < 8; ++cc) {
+          const int c = 32 * g + 4 * cc;
+          const float4 gi = *reinterpret_cast<const float4 *>(sm + OFF_GRAW + g_off(i, c));
+          const float4 grb = *reinterpret_cast<const float4 *>(sm + OFF_GRAW + g_off(rb, c));
+          float x[4];
+          bf16_x4(xraw, i, c, x);
+          const float giv[4] = {gi.x, gi.y, gi.z, gi.w}, grv[4] = {grb.x, grb.y, grb.z, grb.w};
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
-            const float kh = x[e] * __expf(grv[e] - giv[e]) * sE[(bi * 4 + 3) * DH + c + e];
-            *reinterpret_cast<float *>(sm + OFF_KHT + sw128_offset(DH, c + e, i)) = tf32_rna(kh);
+            if (!valid) x[e] = 0.f;
+            Lst[4 * cc + e] = x[e] * ex2(giv[e] - grv[e]);
+          }
+          if (kside) {
+            // R_b row (i % 16) of block bi: k_i exp(G_rb - G_i); Khat = R * exp(G_63 - G_rb)
+            float rv[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) rv[e] = x[e] * ex2(grv[e] - giv[e]);
+            *reinterpret_cast<float4 *>(sm + OFF_R + bi * 8192 + sw128_chunk(16, i & 15, c)) =
+                make_float4(tf32_rna(rv[0]), tf32_rna(rv[1]), tf32_rna(rv[2]), tf32_rna(rv[3]));
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              *reinterpret_cast<float *>(sm + OFF_KHT + sw128_offset(DH, c + e, i)) =
+                  tf32_rna(rv[e] * sE[(bi * 4 + 3) * DH + c + e]);
+          } else {
+            float gq[4];
+#pragma unroll
+            for (int e = 0; e < 4; ++e) gq[e] = tf32_rna(Lst[4 * cc + e] * sEgr[bi * DH + c + e]);
+            *reinterpret_cast<float4 *>(sm + OFF_GQ + sw128_chunk(C, i, c)) =
+                make_float4(gq[0], gq[1], gq[2], gq[3]);
+          }
+        }
+      }
+
+      // ---- a3: A and P, two 16-column blocks per round (two L_b buffers) -------
+      for (int pair = 0; pair < 2 && ok; ++pair) {
+#pragma unroll
+        for (int bb = 0; bb < 2; ++bb) {
+          const int b = 2 * pair + bb;
+          float v[32];
+#pragma unroll
+          for (int j = 0; j < 32; ++j)
+            v[j] = (b <= bi) ? tf32_rna(Lst[j] * sE[(b * 4 + bi) * DH + 32 * g + j]) : 0.f;
+          tmem_st32(tm + lane + (bb ? TM_X1 : TM_L) + 32 * g, v);
+        }
+        tmem_wait_st();
+        warp_arrive(bar_opsap);
+        ok = wwait(bar_ap, ph_ap[0]);
+      }
+      if (!ok) break;
+
+      // ---- V^T and (gamma*K)^T into TMEM (thread = channel l, tokens 16g..) ----
+      {
+        float v[16], w[16];
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int t = 16 * g + j;
+          const float G2 = *reinterpret_cast<const float *>(sm + OFF_GRAW + g_off(t, l));
+          v[j] = (t < n) ? tf32_rna(bf16_at(sm + OFF_VRAW, t, l)) : 0.f;
+          w[j] = (t < n) ? tf32_rna(bf16_at(sm + OFF_KRAW, t, l) * ex2(G2)) : 0.f;
+        }
+        tmem_st16(tm + lane + TM_L + 16 * g, v);
+        tmem_st16(tm + lane + TM_L + 64 + 16 * g, w);
+        tmem_wait_st();
+      }
+      warp_arrive(bar_raw);  // raw tiles consumed: the next chunk's TMA may start
+
+      // ---- a4: T = (I + Diag(beta) A)^-1 (blocked, fp32), P operand ------------
+      float *Ms = reinterpret_cast<float *>(sm + OFF_MS);
+      float *Ti = reinterpret_cast<float *>(sm + OFF_TI);
+      float *Ys = reinterpret_cast<float *>(sm + OFF_Y);
+      {
+        float a[16];
+        tmem_ld16(tm + lane + TM_AP + 16 * g, a);
+        tmem_wait_ld();
+        if (kside) {
+          const float bi_ = sB[i];
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int c = 16 * g + j;
+            Ms[rot(i, c)] = (c < i) ? bi_ * a[j] : 0.f;
           }
         } else {
-          float gq[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) gq[e] = tf32_rna(Lst[c + e] * sEgr[bi * DH + c + e]);
-          *reinterpret_cast<float4 *>(sm + OFF_GQ + sw128_chunk(C, i, c)) =
-              make_float4(gq[0], gq[1], gq[2], gq[3]);
+          for (int j = 0; j < 16; j += 4) {
+            const int c = 16 * g + j;
+            *reinterpret_cast<float4 *>(sm + OFF_P + sw128_chunk(C, i, c)) =
+                make_float4(c + 0 <= i ? tf32_rna(a[j]) : 0.f, c + 1 <= i ? tf32_rna(a[j + 1]) : 0.f,
+                            c + 2 <= i ? tf32_rna(a[j + 2]) : 0.f,
+                            c + 3 <= i ? tf32_rna(a[j + 3]) : 0.f);
+          }
         }
       }
-    }
-    fence_async_smem();
-
-    // ---- a3: A and P, one 16-column block at a time -------------------------
-    for (int b = 0; b < 4 && ok; ++b) {
+      wsync();
+      // diagonal 16x16 blocks: forward substitution, one column per 16 lanes, shuffles
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        float v[32];
+      for (int rho = 0; rho < 2; ++rho) {
+        const int task = 4 * warp + 2 * rho + (lane_id >> 4);
+        const int o = 16 * (task >> 4), jj = task & 15, k = lane_id & 15;
+        float m[16];
 #pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int c = 32 * q + j;
-          v[j] = (b <= bi) ? tf32_rna(Lst[c] * sE[(b * 4 + bi) * DH + c]) : 0.f;
+        for (int q = 0; q < 16; ++q) m[q] = Ms[rot(o + k, o + q)];
+        float x = (k == jj) ? 1.f : 0.f;
+#pragma unroll
+        for (int q = 0; q < 15; ++q) {
+          const float xq = __shfl_sync(0xffffffffu, x, (lane_id & 16) | q);
+          if (q >= jj && k > q) x -= m[q] * xq;
         }
-        tmem_st32(tm + lane + TM_L + 32 * q, v);
+        Ti[rot(o + k, o + jj)] = (k >= jj) ? x : 0.f;
       }
-      tmem_wait_st();
-      tc_fence_before();
-      __syncthreads();
-      if (tid == 0) {
-        tc_fence_after();
-        const uint32_t id = idesc_tf32(16);
-        const uint32_t rb = smem_u32(sm + OFF_R + b * 8192);
-#pragma unroll 1
-        for (int s = 0; s < DH / 8; ++s)
-          mma_tf32_ts(tm + TM_AP + 16 * b, tm + TM_L + 8 * s, sw128_desc(rb, 16, s), id, s > 0);
-      }
-      ok = commit_and_wait();
-    }
-    if (!ok) break;
-
-    // ---- V^T and (gamma*K)^T into TMEM (thread = channel) -------------------
-    {
-      const int c = tid;
-      float v[32];
-      for (int q = 0; q < 2; ++q) {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int t = 32 * q + j;
-          v[j] = (t < n) ? tf32_rna(bf16_at(sm + OFF_VRAW, t, c)) : 0.f;
-        }
-        tmem_st32(tm + lane + TM_L + 32 * q, v);
-      }
-      for (int q = 0; q < 2; ++q) {
-#pragma unroll
-        for (int j = 0; j < 32; ++j) {
-          const int t = 32 * q + j;
-          const float G = *reinterpret_cast<const float *>(sm + OFF_GRAW + g_off(t, c));
-          v[j] = (t < n) ? tf32_rna(bf16_at(sm + OFF_KRAW, t, c) * __expf(G)) : 0.f;
-        }
-        tmem_st32(tm + lane + TM_L + 64 + 32 * q, v);
-      }
-      tmem_wait_st();
-    }
-    __syncthreads();  // raw tiles consumed: the region becomes T-solve scratch
-
-    // ---- a4: T = (I + Diag(beta) A)^-1 (blocked, fp32), P operand ------------
-    float *Ms = reinterpret_cast<float *>(sm + OFF_MS);
-    float *Ti = reinterpret_cast<float *>(sm + OFF_TI);
-    float *Ys = reinterpret_cast<float *>(sm + OFF_Y);
-    {
-      float a[64];
-      tmem_ld32(tm + lane + TM_AP, a);
-      tmem_ld32(tm + lane + TM_AP + 32, a + 32);
-      tmem_wait_ld();
-      if (kside) {
-        const float bi_ = sB[i];
-#pragma unroll
-        for (int j = 0; j < 64; ++j) Ms[i * LD + j] = (j < i) ? bi_ * a[j] : 0.f;
-      } else {
-#pragma unroll
-        for (int j = 0; j < 64; j += 4)
-          *reinterpret_cast<float4 *>(sm + OFF_P + sw128_chunk(C, i, j)) =
-              make_float4(j + 0 <= i ? tf32_rna(a[j]) : 0.f, j + 1 <= i ? tf32_rna(a[j + 1]) : 0.f,
-                          j + 2 <= i ? tf32_rna(a[j + 2]) : 0.f,
-                          j + 3 <= i ? tf32_rna(a[j + 3]) : 0.f);
-      }
-    }
-    __syncthreads();
-    if (tid < C) {  // diagonal 16x16 blocks by forward substitution, one column per thread
-      const int blk = tid >> 4, jj = tid & 15, o = 16 * blk;
-      float x[16];
-#pragma unroll
-      for (int k = 0; k < 16; ++k) {
-        float acc = (k == jj) ? 1.f : 0.f;
-#pragma unroll
-        for (int l = 0; l < 16; ++l)
-          if (l < k && l >= jj) acc -= Ms[(o + k) * LD + o + l] * x[l];
-        x[k] = (k < jj) ? 0.f : acc;
-        Ti[(o + k) * LD + o + jj] = x[k];
-      }
-    }
-    __syncthreads();
-    for (int d = 1; d < 4; ++d) {  // off-diagonal blocks, level by level
-      const int nblk = 4 - d;
-      for (int e = tid; e < nblk * 256; e += NT) {  // Y = sum_c Ms_{a,c} T_{c,b}
-        const int bb = e >> 8, k = (e >> 4) & 15, j = e & 15, a = bb + d;
-        float acc = 0.f;
-        for (int cb = bb; cb < a; ++cb)
-#pragma unroll
-          for (int l = 0; l < 16; ++l)
-            acc += Ms[(16 * a + k) * LD + 16 * cb + l] * Ti[(16 * cb + l) * LD + 16 * bb + j];
-        Ys[(bb * 16 + k) * 17 + j] = acc;
-      }
-      __syncthreads();
-      for (int e = tid; e < nblk * 256; e += NT) {  // T_ab = -T_aa Y
-        const int bb = e >> 8, k = (e >> 4) & 15, j = e & 15, a = bb + d;
+      wsync();
+      // 16 -> 32: T_ab = -T_aa (N_ab T_bb) for (a, b) = (1, 0) and (3, 2); T lower triangular
+      {
+        const int blk = tid >> 8, k = (tid >> 4) & 15, j = tid & 15;
+        const int a = 2 * blk + 1, b = 2 * blk;
         float acc = 0.f;
 #pragma unroll
-        for (int l = 0; l < 16; ++l)
-          acc += Ti[(16 * a + k) * LD + 16 * a + l] * Ys[(bb * 16 + l) * 17 + j];
-        Ti[(16 * a + k) * LD + 16 * bb + j] = -acc;
-      }
-      __syncthreads();
-    }
-    if (kside) {  // TB = T Diag(beta), row i
+        for (int q = 0; q < 16; ++q)
+          if (q >= j) acc += Ms[rot(16 * a + k, 16 * b + q)] * Ti[rot(16 * b + q, 16 * b + j)];
+        Ys[(blk * 16 + k) * 17 + j] = acc;
+        wsync();
+        float t = 0.f;
 #pragma unroll
-      for (int j = 0; j < 64; j += 4) {
-        float v4[4];
-#pragma unroll
-        for (int e = 0; e < 4; ++e)
-          v4[e] = (j + e <= i) ? tf32_rna(Ti[i * LD + j + e] * sB[j + e]) : 0.f;
-        *reinterpret_cast<float4 *>(sm + OFF_TB + sw128_chunk(C, i, j)) =
-            make_float4(v4[0], v4[1], v4[2], v4[3]);
+        for (int q = 0; q < 16; ++q)
+          if (q <= k) t += Ti[rot(16 * a + k, 16 * a + q)] * Ys[(blk * 16 + q) * 17 + j];
+        Ti[rot(16 * a + k, 16 * b + j)] = -t;
+        wsync();
       }
-    }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-    if (tid == 0 && c0 + C < len) issue_tma(c0 + C);  // prefetch the next chunk
-
-    // ---- a4: U~^T = V^T TB^T, W^T = (gK)^T TB^T ------------------------------
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t id = idesc_tf32(64);
-      const uint32_t tb = smem_u32(sm + OFF_TB);
-#pragma unroll 1
-      for (int s = 0; s < C / 8; ++s) {
-        mma_tf32_ts(tm + TM_X2, tm + TM_L + 8 * s, sw128_desc(tb, C, s), id, s > 0);
-        mma_tf32_ts(tm + TM_X1, tm + TM_L + 64 + 8 * s, sw128_desc(tb, C, s), id, s > 0);
+      // 32 -> 64: T[32:64, 0:32] = -T[32:64, 32:64] (N[32:64, 0:32] T[0:32, 0:32])
+      {
+        const int ii = tid >> 4, j0 = tid & 15;  // rows ii, columns j0 and j0 + 16
+        float y0 = 0.f, y1 = 0.f;
+#pragma unroll 8
+        for (int q = 0; q < 32; ++q) {
+          const float nv = Ms[rot(32 + ii, q)];
+          if (q >= j0) y0 += nv * Ti[rot(q, j0)];
+          if (q >= j0 + 16) y1 += nv * Ti[rot(q, j0 + 16)];
+        }
+        Ys[ii * 33 + j0] = y0;
+        Ys[ii * 33 + j0 + 16] = y1;
+        wsync();
+        float t0 = 0.f, t1 = 0.f;
+#pragma unroll 8
+        for (int q = 0; q < 32; ++q) {
+          if (q <= ii) {
+            const float tv = Ti[rot(32 + ii, 32 + q)];
+            t0 += tv * Ys[q * 33 + j0];
+            t1 += tv * Ys[q * 33 + j0 + 16];
+          }
+        }
+        Ti[rot(32 + ii, j0)] = -t0;
+        Ti[rot(32 + ii, j0 + 16)] = -t1;
+        wsync();
       }
-    }
-    if (!(ok = commit_and_wait())) break;
-
-    // ---- W operand (rows = tokens, K = key channels) from W^T ---------------
-    {
-      float w[64];
-      tmem_ld32(tm + lane + TM_X1, w);
-      tmem_ld32(tm + lane + TM_X1 + 32, w + 32);
-      tmem_wait_ld();
+      if (kside) {  // TB = T Diag(beta): row i, columns 16g..16g+15
 #pragma unroll
-      for (int t = 0; t < C; ++t)
-        *reinterpret_cast<float *>(sm + OFF_R + sw128_offset(C, t, tid)) = tf32_rna(w[t]);
-    }
-    fence_async_smem();
-    tc_fence_before();
-    __syncthreads();
-
-    // ---- a5: U^T = U~^T - S^T W^T ; O^T = S^T (gamma Q)^T ---------------------
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t idn = idesc_tf32(64, true), id = idesc_tf32(64);
-      const uint32_t wb = smem_u32(sm + OFF_R), qb = smem_u32(sm + OFF_GQ);
-#pragma unroll 1
-      for (int s = 0; s < DH / 8; ++s) {
-        mma_tf32_ts(tm + TM_X2, tm + TM_S + 8 * s, sw128_desc(wb, C, s), idn, true);
-        mma_tf32_ts(tm + TM_X1, tm + TM_S + 8 * s, sw128_desc(qb, C, s), id, s > 0);
+        for (int j = 0; j < 16; j += 4) {
+          const int c = 16 * g + j;
+          float v4[4];
+#pragma unroll
+          for (int e = 0; e < 4; ++e)
+            v4[e] = (c + e <= i) ? tf32_rna(Ti[rot(i, c + e)] * sB[c + e]) : 0.f;
+          *reinterpret_cast<float4 *>(sm + OFF_TB + sw128_chunk(C, i, c)) =
+              make_float4(v4[0], v4[1], v4[2], v4[3]);
+        }
       }
-    }
-    if (!(ok = commit_and_wait())) break;
+      warp_arrive(bar_ops);  // -> W^T, U~^T MMAs
+      if (!(ok = wwait(bar_mma, ph_mma))) break;
 
-    // ---- S^T <- S^T Diag(gamma_63): column c scaled by exp(G_63,c) -----------
-    for (int q = 0; q < 4; ++q) {
-      float v[32];
-      tmem_ld32(tm + lane + TM_S + 32 * q, v);
-      tmem_wait_ld();
-#pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] *= sEgr[3 * DH + 32 * q + j];
-      tmem_st32(tm + lane + TM_S + 32 * q, v);
-    }
-    tmem_wait_st();
-    tc_fence_before();
-    __syncthreads();
-
-    // ---- a5: O^T += U^T P^T ; S^T += U^T Khat --------------------------------
-    if (tid == 0) {
-      tc_fence_after();
-      const uint32_t id64 = idesc_tf32(64), id128 = idesc_tf32(128);
-      const uint32_t pb = smem_u32(sm + OFF_P), kb = smem_u32(sm + OFF_KHT);
-#pragma unroll 1
-      for (int s = 0; s < C / 8; ++s) {
-        mma_tf32_ts(tm + TM_X1, tm + TM_X2 + 8 * s, sw128_desc(pb, C, s), id64, true);
-        mma_tf32_ts(tm + TM_S, tm + TM_X2 + 8 * s, sw128_desc(kb, DH, s), id128, true);
-      }
-    }
-    if (!(ok = commit_and_wait())) break;
-
-    // ---- a6: outputs (lane = value channel) and snapshots --------------------
-    if (go) {
-      float o[64];
-      tmem_ld32(tm + lane + TM_X1, o);
-      tmem_ld32(tm + lane + TM_X1 + 32, o + 32);
-      tmem_wait_ld();
-#pragma unroll
-      for (int t = 0; t < C; ++t)
-        if (t < n) store_elem(go, ((size_t)(bos + c0 + t) * H + h) * DH + tid, o[t]);
-    }
-    if (snaps_ok && n == C && (c0 + C) % p.snapshot_stride == 0) {
-      const size_t row = (size_t)p.cu_snapshots[r] + (c0 + C) / p.snapshot_stride - 1;
-      float *dst = p.snapshots + (row * H + h) * (size_t)DH * DH;
-      for (int q = 0; q < 4; ++q) {
-        float v[32];
-        tmem_ld32(tm + lane + TM_S + 32 * q, v);
+      // ---- W operand (rows = tokens, K = key channels) from W^T ---------------
+      {
+        float w[16];
+        tmem_ld16(tm + lane + TM_X1 + 16 * g, w);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) dst[(size_t)(32 * q + j) * DH + tid] = v[j];
+        for (int j = 0; j < 16; ++j)
+          *reinterpret_cast<float *>(sm + OFF_R + sw128_offset(C, 16 * g + j, l)) = tf32_rna(w[j]);
       }
-    }
-    tc_fence_before();
-    __syncthreads();
-  }
+      warp_arrive(bar_ops);  // -> U^T -= S^T W^T, O^T = S^T (gQ)^T
+      if (!(ok = wwait(bar_mma, ph_mma))) break;
 
-  if (ok && p.final_state) {
-    float *dst = p.final_state + ((size_t)(r * H + h)) * DH * DH;
-    tc_fence_after();
-    for (int q = 0; q < 4; ++q) {
+      // ---- S^T <- S^T Diag(gamma_63): column c scaled by exp(G_63,c) -----------
+      {
+        float v[32];
+        tmem_ld32(tm + lane + TM_S + 32 * g, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) v[j] *= sEgr[3 * DH + 32 * g + j];
+        tmem_st32(tm + lane + TM_S + 32 * g, v);
+        tmem_wait_st();
+      }
+      warp_arrive(bar_ops);  // -> O^T += U^T P^T, S^T += U^T Khat
+      if (!(ok = wwait(bar_mma, ph_mma))) break;
+
+      // ---- a6: outputs (lane = value channel, tokens 16g..) and snapshots -------
+      if (go) {
+        float o[16];
+        tmem_ld16(tm + lane + TM_X1 + 16 * g, o);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int t = 16 * g + j;
+          if (t < n) store_elem(go, ((size_t)(bos + c0 + t) * H + h) * DH + l, o[j]);
+        }
+      }
+      if (snaps_ok && n == C && (c0 + C) % p.snapshot_stride == 0) {
+        const size_t row = (size_t)p.cu_snapshots[r] + (c0 + C) / p.snapshot_stride - 1;
+        float *dst = p.snapshots + (row * H + h) * (size_t)DH * DH;
+        float v[32];
+        tmem_ld32(tm + lane + TM_S + 32 * g, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) dst[(size_t)(32 * g + j) * DH + l] = v[j];
+      }
+      tc_fence_before();
+      wsync();
+    }
+
+    if (ok && p.final_state) {
+      float *dst = p.final_state + ((size_t)(r * H + h)) * DH * DH;
+      tc_fence_after();
       float v[32];
-      tmem_ld32(tm + lane + TM_S + 32 * q, v);
+      tmem_ld32(tm + lane + TM_S + 32 * g, v);
       tmem_wait_ld();
 #pragma unroll
-      for (int j = 0; j < 32; ++j) dst[(size_t)(32 * q + j) * DH + tid] = v[j];
+      for (int j = 0; j < 32; ++j) dst[(size_t)(32 * g + j) * DH + l] = v[j];
     }
   }
-  if (!ok && tid == 0) {
-    // give in-flight copies and MMAs a bounded chance to land before TMEM is freed
-    mbar_wait(bar_tma, tma_phase, 100000000ull);
-    mbar_wait(bar_mma, mma_phase, 100000000ull);
-  }
+
   tc_fence_before();
+  __syncthreads();
+  if (*s_abort && tid == 0) {
+    // the CTA gave up: give in-flight copies and MMAs a bounded chance to land
+    mbar_wait(bar_tma, 0, 100000000ull);
+    mbar_wait(bar_tma, 1, 100000000ull);
+    mbar_wait(bar_mma, 0, 100000000ull);
+    mbar_wait(bar_mma, 1, 100000000ull);
+  }
   __syncthreads();
   if (warp == 0) {
     tc_fence_after();
@@ -549,12 +631,12 @@ cudaError_t launch_prefill_tc(const PrefillParams &p, kda_dtype in_dtype, kda_dt
     e = cudaFuncSetAttribute(prefill_tc_kernel<__nv_bfloat16>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_ALLOC);
     if (e != cudaSuccess) return e;
-    prefill_tc_kernel<__nv_bfloat16><<<(unsigned)(p.n_req * p.H), NT, SMEM_ALLOC, stream>>>(p, maps);
+    prefill_tc_kernel<__nv_bfloat16><<<(unsigned)(p.n_req * p.H), NT + 32, SMEM_ALLOC, stream>>>(p, maps);
   } else {
     e = cudaFuncSetAttribute(prefill_tc_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)SMEM_ALLOC);
     if (e != cudaSuccess) return e;
-    prefill_tc_kernel<float><<<(unsigned)(p.n_req * p.H), NT, SMEM_ALLOC, stream>>>(p, maps);
+    prefill_tc_kernel<float><<<(unsigned)(p.n_req * p.H), NT + 32, SMEM_ALLOC, stream>>>(p, maps);
   }
   return cudaGetLastError();
 }
