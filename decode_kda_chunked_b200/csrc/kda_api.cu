@@ -4,6 +4,7 @@
 // code before launching anything; it allocates no device memory (scratch is
 // the caller's workspace) and never synchronises except in
 // kda_get_device_status().
+#include <cstdio>
 #include <cstdlib>
 #include <cstring>
 
@@ -96,7 +97,12 @@ size_t prefill_ws(int n_req) {
   return align256((size_t)n_req * sizeof(int32_t));
 }
 
-kda_status from_cuda(cudaError_t e) { return e == cudaSuccess ? KDA_OK : KDA_ERR_CUDA; }
+// A failed CUDA call becomes KDA_ERR_CUDA; with KDA_VERBOSE=1 its message goes to stderr.
+kda_status from_cuda(cudaError_t e) {
+  if (e == cudaSuccess) return KDA_OK;
+  if (env_flag("KDA_VERBOSE")) std::fprintf(stderr, "libkda: CUDA error: %s\n", cudaGetErrorString(e));
+  return KDA_ERR_CUDA;
+}
 
 }  // namespace
 

@@ -60,31 +60,37 @@ constexpr uint32_t OFF_VRAW = 32768;
 constexpr uint32_t OFF_GRAW = 49152;    // fp32 [64 x 128]: 4 TMA boxes of 32 cols (SW128);
                                         // rewritten in place with log2(e) * cumsum(g)
 constexpr uint32_t RAW_BYTES = 81920;
-constexpr uint32_t OFF_R = 81920;       // 4 x [16 x 128] tf32 B operands (R_b); then T-solve
-                                        // scratch (two [64 x 64] fp32); then W [64 x 128]
-constexpr uint32_t OFF_MS = OFF_R;          // beta*A strict lower, rotated rows
-constexpr uint32_t OFF_TI = OFF_R + 16384;  // T = (I + beta A)^-1, rotated rows
-constexpr uint32_t OFF_GQ = 114688;     // (gamma*Q) [64 x 128] tf32 B operand
-constexpr uint32_t OFF_KHT = 147456;    // Khat^T [128 x 64] tf32 B operand
-constexpr uint32_t OFF_TB = 180224;     // T Diag(beta) [64 x 64] tf32 B operand
-constexpr uint32_t OFF_P = 196608;      // P [64 x 64] tf32 B operand
-constexpr uint32_t OFF_E = 212992;      // E[b*4+a][128] = exp(G_ra - G_rb), b <= a; then
+// Once every raw tile is read, the raw region holds the B operands R'_a of
+// the A|P products: row block a has 16(a+1) rows at byte 8192 a(a+1)/2.
+__host__ __device__ constexpr uint32_t rp_off(int a) { return 4096u * a * (a + 1); }
+constexpr uint32_t OFF_R = 81920;       // T-solve scratch (two [64 x 65] fp32); then W [64 x 128]
+constexpr int LDT = 65;                 // padded row stride of the T-solve scratch
+constexpr uint32_t OFF_MS = OFF_R;                  // beta*A strict lower
+constexpr uint32_t OFF_TI = OFF_R + 64 * LDT * 4;   // T = (I + beta A)^-1
+constexpr uint32_t OFF_GQ = 115712;     // (gamma*Q) [64 x 128] tf32 B operand
+constexpr uint32_t OFF_KHT = 148480;    // Khat^T [128 x 64] tf32 B operand
+constexpr uint32_t OFF_TB = 181248;     // T Diag(beta) [64 x 64] tf32 B operand
+constexpr uint32_t OFF_P = 197632;      // P [64 x 64] tf32 B operand
+constexpr uint32_t OFF_E = 214016;      // E[b*4+a][128] = exp(G_ra - G_rb), b <= a; then
                                         // the T-solve products ([2][16][17], then [32][33])
 constexpr uint32_t OFF_Y = OFF_E;
-constexpr uint32_t OFF_EGR = 221184;    // exp(G_rb)[4][128]
-constexpr uint32_t OFF_SEG = 223232;    // cumsum segment totals [4][128]
-constexpr uint32_t OFF_GR2 = 225280;    // log2(e) * G at block ends [4][128]
-constexpr uint32_t OFF_BETA = 227328;   // beta[64]
-constexpr uint32_t OFF_BAR = 227584;    // mbarriers + TMEM base + flags
-constexpr uint32_t SMEM_BYTES = 227680;
+constexpr uint32_t OFF_EGR = 222208;    // exp(G_rb)[4][128]
+constexpr uint32_t OFF_SEG = 224256;    // cumsum segment totals [4][128]
+constexpr uint32_t OFF_GR2 = 226304;    // log2(e) * G at block ends [4][128]
+constexpr uint32_t OFF_BETA = 228352;   // beta[64]
+constexpr uint32_t OFF_BAR = 228608;    // mbarriers + TMEM base + flags
+constexpr uint32_t SMEM_BYTES = 228704;
+static_assert(OFF_TI + 64 * LDT * 4 <= OFF_GQ, "T-solve scratch must fit the R region");
 constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;  // alignment slack
 
 // ---- TMEM column map (512 columns x 128 lanes of fp32) ----
 constexpr uint32_t TM_S = 0;     // S^T (lane = value channel, col = key channel)
-constexpr uint32_t TM_L = 128;   // A-operand buffer 0: L_b; later V^T [0,64), (gK)^T [64,128)
-constexpr uint32_t TM_AP = 256;  // A (lanes 0..63) and P (lanes 64..127), col = j
-constexpr uint32_t TM_X1 = 320;  // W^T, later O^T   (X1..X2 is A-operand buffer 1 for L_b)
-constexpr uint32_t TM_X2 = 384;  // U~^T -> U^T
+constexpr uint32_t TM_L = 128;   // L* (A operand of A|P); later V^T [0,64), (gK)^T [64,128)
+// A (lanes 0..63) | P (lanes 64..127) of rows in block a: 16(a+1) columns at TM_AP + 8a(a+1)
+constexpr uint32_t TM_AP = 256;  // up to column 416
+__host__ __device__ constexpr uint32_t ap_col(int a) { return TM_AP + 8u * a * (a + 1); }
+constexpr uint32_t TM_X1 = 256;  // W^T, later O^T   (alias A|P once the solve has read it)
+constexpr uint32_t TM_X2 = 320;  // U~^T -> U^T      (alias A|P)
 constexpr uint32_t TM_COLS = 512;
 
 struct TcMaps {
@@ -117,9 +123,9 @@ __device__ __forceinline__ float tf32_rna(float x) {
   asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
   return __uint_as_float(r);
 }
-// [64 x 64] fp32 scratch with each row rotated by its index: row and column
-// walks of a warp both hit 32 distinct banks.
-__device__ __forceinline__ int rot(int r, int c) { return r * 64 + ((c + r) & 63); }
+// [64 x 65] fp32 scratch: the padded stride puts a warp's row walk and column
+// walk on 32 distinct banks and keeps addresses affine in the loop indices.
+__device__ __forceinline__ int rot(int r, int c) { return r * LDT + c; }
 
 template <typename TOut>
 __global__ void __launch_bounds__(NT + 32, 1)
@@ -213,17 +219,16 @@ __global__ void __launch_bounds__(NT + 32, 1)
       if (n_chunks > 0) issue_tma(0);
       for (int ci = 0; ci < n_chunks; ++ci) {
         bool good = true;
-        for (int pair = 0; pair < 2 && good; ++pair) {  // A | P: blocks 2*pair, 2*pair+1
-          if (!(good = cwait(bar_opsap, ph_opsap[0]))) break;
-          const uint32_t id = idesc_tf32(16);
-          const int b0 = 2 * pair;
-          const uint32_t r0 = smem_u32(sm + OFF_R + b0 * 8192), r1 = r0 + 8192;
-          // two independent accumulation chains, interleaved so their latencies overlap
+        // A | P: row block a against its R'_a (N = 16(a+1)); four interleaved chains
+        if (!(good = cwait(bar_opsap, ph_opsap[0]))) break;
+        {
+          const uint32_t rp = smem_u32(sm);
 #pragma unroll
           for (int s = 0; s < DH / 8; ++s) {
-            mma_tf32_ts(tm + TM_AP + 16 * b0, tm + TM_L + 8 * s, sw128_desc(r0, 16, s), id, s > 0);
-            mma_tf32_ts(tm + TM_AP + 16 * b0 + 16, tm + TM_X1 + 8 * s, sw128_desc(r1, 16, s), id,
-                        s > 0);
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+              mma_tf32_ts(tm + ap_col(a), tm + TM_L + 8 * s, sw128_desc(rp + rp_off(a), 16 * (a + 1), s),
+                          idesc_tf32(16 * (a + 1)), s > 0);
           }
           mma_commit(bar_ap);
         }
@@ -298,19 +303,23 @@ __global__ void __launch_bounds__(NT + 32, 1)
       tmem_wait_st();
     }
 
+    // beta of the chunk about to start, loaded one chunk ahead (threads 0..63)
+    auto load_beta = [&](int c0) -> float {
+      float b = 0.f;
+      if (tid < C && c0 + tid < len) {
+        b = p.beta[(size_t)(bos + c0 + tid) * H + h];
+        if (p.validate && !(b >= 0.f && b <= 1.f)) set_status(p.status, STATUS_GATE_RANGE);
+      }
+      return b;
+    };
+    float beta_next = load_beta(0);
     bool ok = true;
     for (int ci = 0; ci < n_chunks && ok; ++ci) {
       const int c0 = ci * C;
       const int n = min(C, len - c0);
-      if (tid < C) {
-        float b = 0.f;
-        if (tid < n) {
-          b = p.beta[(size_t)(bos + c0 + tid) * H + h];
-          if (p.validate && !(b >= 0.f && b <= 1.f)) set_status(p.status, STATUS_GATE_RANGE);
-        }
-        sB[tid] = b;
-      }
+      if (tid < C) sB[tid] = beta_next;
       if (!(ok = wwait(bar_tma, ph_tma))) break;
+      beta_next = load_beta(c0 + C);
 
       // ---- a2: cumulative gate (thread = channel l, tokens 16g..16g+15) --------
       {
@@ -343,16 +352,22 @@ __global__ void __launch_bounds__(NT + 32, 1)
       }
 
       // ---- a3 operands (thread = row i, channels 32g..32g+31) -----------------
+      // L*_i = x_i exp(G_i - G_rb) with r_b the last row of i's own block (x = k or q),
+      // into TMEM; R_i = k_i exp(G_rb - G_i) kept for the B operands R'_a below.
       const bool kside = l < C;
       const int i = l & (C - 1);
       const int bi = i >> 4;
       const bool valid = i < n;
-      float Lst[32];
+      float Rv[32];
       {
         const unsigned char *xraw = sm + (kside ? OFF_KRAW : OFF_QRAW);
         const int rb = 16 * bi + 15;
 #pragma unroll
-        for (int cc = 0; cc < 8; ++cc) {
+        for (int half = 0; half < 2; ++half) {
+        float Lv[16];
+#pragma unroll
+        for (int c4 = 0; c4 < 4; ++c4) {
+          const int cc = 4 * half + c4;
           const int c = 32 * g + 4 * cc;
           const float4 gi = *reinterpret_cast<const float4 *>(sm + OFF_GRAW + g_off(i, c));
           const float4 grb = *reinterpret_cast<const float4 *>(sm + OFF_GRAW + g_off(rb, c));
@@ -362,70 +377,88 @@ __global__ void __launch_bounds__(NT + 32, 1)
 #pragma unroll
           for (int e = 0; e < 4; ++e) {
             if (!valid) x[e] = 0.f;
-            Lst[4 * cc + e] = x[e] * ex2(giv[e] - grv[e]);
+            const float lst = x[e] * ex2(giv[e] - grv[e]);
+            Lv[4 * c4 + e] = tf32_rna(lst);
+            if (kside) {
+              Rv[4 * cc + e] = x[e] * ex2(grv[e] - giv[e]);
+            } else {
+              Rv[4 * cc + e] = lst;  // Q side: gamma*Q = L* exp(G_rb)
+            }
           }
           if (kside) {
-            // R_b row (i % 16) of block bi: k_i exp(G_rb - G_i); Khat = R * exp(G_63 - G_rb)
-            float rv[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) rv[e] = x[e] * ex2(grv[e] - giv[e]);
-            *reinterpret_cast<float4 *>(sm + OFF_R + bi * 8192 + sw128_chunk(16, i & 15, c)) =
-                make_float4(tf32_rna(rv[0]), tf32_rna(rv[1]), tf32_rna(rv[2]), tf32_rna(rv[3]));
+            // Khat = R * exp(G_63 - G_rb), stored transposed (rows = channels)
 #pragma unroll
             for (int e = 0; e < 4; ++e)
               *reinterpret_cast<float *>(sm + OFF_KHT + sw128_offset(DH, c + e, i)) =
-                  tf32_rna(rv[e] * sE[(bi * 4 + 3) * DH + c + e]);
+                  tf32_rna(Rv[4 * cc + e] * sE[(bi * 4 + 3) * DH + c + e]);
           } else {
             float gq[4];
 #pragma unroll
-            for (int e = 0; e < 4; ++e) gq[e] = tf32_rna(Lst[4 * cc + e] * sEgr[bi * DH + c + e]);
+            for (int e = 0; e < 4; ++e) gq[e] = tf32_rna(Rv[4 * cc + e] * sEgr[bi * DH + c + e]);
             *reinterpret_cast<float4 *>(sm + OFF_GQ + sw128_chunk(C, i, c)) =
                 make_float4(gq[0], gq[1], gq[2], gq[3]);
           }
         }
-      }
-
-      // ---- a3: A and P, two 16-column blocks per round (two L_b buffers) -------
-      for (int pair = 0; pair < 2 && ok; ++pair) {
-#pragma unroll
-        for (int bb = 0; bb < 2; ++bb) {
-          const int b = 2 * pair + bb;
-          float v[32];
-#pragma unroll
-          for (int j = 0; j < 32; ++j)
-            v[j] = (b <= bi) ? tf32_rna(Lst[j] * sE[(b * 4 + bi) * DH + 32 * g + j]) : 0.f;
-          tmem_st32(tm + lane + (bb ? TM_X1 : TM_L) + 32 * g, v);
+        tmem_st16(tm + lane + TM_L + 32 * g + 16 * half, Lv);
         }
-        tmem_wait_st();
-        warp_arrive(bar_opsap);
-        ok = wwait(bar_ap, ph_ap[0]);
       }
-      if (!ok) break;
-
-      // ---- V^T and (gamma*K)^T into TMEM (thread = channel l, tokens 16g..) ----
+      // V^T and (gamma*K)^T (thread = channel l, tokens 16g..16g+15), held in registers
+      // (v is bf16, so it is exact in tf32 and is kept packed, two values per register)
+      uint32_t vT2[8];
+      float gkT[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int t = 16 * g + j;
+        const float G2 = *reinterpret_cast<const float *>(sm + OFF_GRAW + g_off(t, l));
+        const uint32_t vb = (t < n) ? (uint32_t)*reinterpret_cast<const unsigned short *>(
+                                          sm + OFF_VRAW + bf16_off(t, l))
+                                    : 0u;
+        if (j & 1) vT2[j >> 1] |= vb << 16; else vT2[j >> 1] = vb;
+        gkT[j] = (t < n) ? tf32_rna(bf16_at(sm + OFF_KRAW, t, l) * ex2(G2)) : 0.f;
+      }
+      wsync();  // every raw tile read: the raw region now takes the R'_a operands
+      if (kside) {
+        // R'_a row i = R_i exp(G_ra - G_rb) for every row block a >= bi
+        for (int a = bi; a < 4; ++a) {
+          const int rows = 16 * (a + 1);
+#pragma unroll
+          for (int cc = 0; cc < 8; ++cc) {
+            const int c = 32 * g + 4 * cc;
+            const float *ea = sE + (bi * 4 + a) * DH + c;
+            *reinterpret_cast<float4 *>(sm + rp_off(a) + sw128_chunk(rows, i, c)) =
+                make_float4(tf32_rna(Rv[4 * cc] * ea[0]), tf32_rna(Rv[4 * cc + 1] * ea[1]),
+                            tf32_rna(Rv[4 * cc + 2] * ea[2]), tf32_rna(Rv[4 * cc + 3] * ea[3]));
+          }
+        }
+      }
+      tmem_wait_st();
+      warp_arrive(bar_opsap);  // -> A|P MMAs
+      if (!(ok = wwait(bar_ap, ph_ap[0]))) break;
       {
-        float v[16], w[16];
+        float vT[16];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int t = 16 * g + j;
-          const float G2 = *reinterpret_cast<const float *>(sm + OFF_GRAW + g_off(t, l));
-          v[j] = (t < n) ? tf32_rna(bf16_at(sm + OFF_VRAW, t, l)) : 0.f;
-          w[j] = (t < n) ? tf32_rna(bf16_at(sm + OFF_KRAW, t, l) * ex2(G2)) : 0.f;
-        }
-        tmem_st16(tm + lane + TM_L + 16 * g, v);
-        tmem_st16(tm + lane + TM_L + 64 + 16 * g, w);
-        tmem_wait_st();
+        for (int j = 0; j < 16; ++j)
+          vT[j] = __uint_as_float((j & 1) ? (vT2[j >> 1] & 0xFFFF0000u) : (vT2[j >> 1] << 16));
+        tmem_st16(tm + lane + TM_L + 16 * g, vT);  // L* is dead: the W / U~ A operands
       }
-      warp_arrive(bar_raw);  // raw tiles consumed: the next chunk's TMA may start
+      tmem_st16(tm + lane + TM_L + 64 + 16 * g, gkT);
+      tmem_wait_st();
+      warp_arrive(bar_raw);  // R'_a consumed: the next chunk's TMA may start
 
       // ---- a4: T = (I + Diag(beta) A)^-1 (blocked, fp32), P operand ------------
       float *Ms = reinterpret_cast<float *>(sm + OFF_MS);
       float *Ti = reinterpret_cast<float *>(sm + OFF_TI);
       float *Ys = reinterpret_cast<float *>(sm + OFF_Y);
       {
-        float a[16];
-        tmem_ld16(tm + lane + TM_AP + 16 * g, a);
+        // this warp's 32 rows span two row blocks; load both blocks' columns
+        const int a_lo = 2 * (warp & 1);
+        float a[16], a_hi[16];
+        tmem_ld16(tm + lane + ap_col(a_lo) + 16 * g, a);
+        tmem_ld16(tm + lane + ap_col(a_lo + 1) + 16 * g, a_hi);
         tmem_wait_ld();
+        if (lane_id >= 16)
+#pragma unroll
+          for (int j = 0; j < 16; ++j) a[j] = a_hi[j];
         if (kside) {
           const float bi_ = sB[i];
 #pragma unroll
