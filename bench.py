@@ -338,6 +338,9 @@ def run_ours(args, world, rank, local):
 
     if not args.no_decode:
         line["decode"] = bench_decode(args, dev, peaks, peak_kind, rank)
+    if not args.no_extra:
+        line["single_seq"] = bench_single_seq(args, dev, peaks)
+        line["kcp_million"] = bench_kcp_million(args, dev, peaks)
     if not args.no_e2e:
         line["e2e"] = bench_e2e(args, inp, dev, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -389,6 +392,78 @@ def bench_decode(args, dev, peaks, peak_kind, rank):
             "roofline": {"bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": gbs / peaks["hbm_gbs"], "peak_kind": peak_kind,
                          "frac_of_nominal_8tbs": gbs / 8000.0}}
+
+
+def _time_calls(fn, warm: int, steps: int, stream) -> float:
+    """Mean ms per call of fn() on `stream`, CUDA events, after `warm` untimed calls."""
+    import torch
+    for _ in range(warm):
+        fn()
+    torch.cuda.synchronize()
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    s.record(stream)
+    for _ in range(steps):
+        fn()
+    e.record(stream)
+    torch.cuda.synchronize()
+    return s.elapsed_time(e) / steps
+
+
+def bench_single_seq(args, dev, peaks):
+    """One sequence of 8,192 tokens, H=32, d=128, N(0, 0.1) initial state: only 32
+    serial chains, so this measures the latency of the chunk-to-chunk state path."""
+    import torch
+
+    import decode_kda_chunked_b200 as kda
+    from decode_kda_chunked_b200 import inputs as I
+    x = I.single_seq(device=dev)
+    T, H, d = x.total_tokens, 32, 128
+    o = torch.empty(T, H, d, device=dev)
+    fin = torch.empty(1, H, d, d, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    cu_host = torch.tensor([0, T], dtype=torch.int32)
+    ms = _time_calls(lambda: kda.kda_prefill_chunked(
+        x.q, x.k, x.v, x.g, x.beta, x.cu_seqlens, o, x.initial_state, fin,
+        cu_seqlens_host=cu_host, stream=stream), 3, max(args.steps, 5), stream)
+    b = prefill_bytes(T, H, d, d, 1, initial=True, final=True)
+    return {"workload": "B=1, H=32, T=8192, d=128, bf16, N(0,0.1) initial state, final state out",
+            "value": T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
+            "tflops": prefill_flops_per_token_head(d, d) * T * H / (ms * 1e-3) / 1e12,
+            "roofline": {"bound": "hbm", "achieved": b / (ms * 1e-3) / 1e9,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": b / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}}
+
+
+def bench_kcp_million(args, dev, peaks):
+    """B=1, H=16, T=1,048,576, d=128: 16 segments of 65,536 tokens through local
+    states + transitions, the exact combine, and the segment-wise prefill with
+    snapshots every 512 tokens; the unsplit single-chain-per-head run is timed once
+    beside it."""
+    import torch
+
+    import decode_kda_chunked_b200 as kda
+    from decode_kda_chunked_b200 import inputs as I
+    x = I.million(device=dev)
+    T, H, d = x.total_tokens, 16, 128
+    stream = torch.cuda.current_stream(dev)
+    ms = _time_calls(lambda: kda.long_context_prefill(x.q, x.k, x.v, x.g, x.beta, 65536, 512,
+                                                      stream=stream), 1, 2, stream)
+    ms_unsplit = _time_calls(lambda: kda.prefill(x.q, x.k, x.v, x.g, x.beta, x.cu_seqlens,
+                                                 snapshot_stride=512, cu_seqlens_host=[0, T],
+                                                 stream=stream), 0, 1, stream)
+    # two passes over the inputs (pass 1 reads k, v, g, beta twice: state and transition)
+    b = (T * H * (2 * (2 * d * 2 + 4 * d + 4))       # pass 1, two CTAs per segment-head
+         + prefill_bytes(T, H, d, d, 16, initial=True, final=True)
+         + (T // 512) * H * d * d * 4)               # snapshots
+    return {"workload": "B=1, H=16, T=1,048,576, d=128, bf16; 16 segments x 65,536 tokens: "
+                        "local state + transition, exact combine, segment prefill with fp32 "
+                        "snapshots every 512 tokens",
+            "value": T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
+            "unsplit_ms": ms_unsplit, "speedup_vs_unsplit": ms_unsplit / ms,
+            "roofline": {"bound": "hbm", "achieved": b / (ms * 1e-3) / 1e9,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": b / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}}
 
 
 def bench_e2e(args, inp, dev, world):
@@ -446,6 +521,8 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--no-extra", action="store_true",
+                    help="skip the single-sequence and million-token measurements")
     ap.add_argument("--prefill-requests", type=int, default=None,
                     help="keep only the first N requests of the varlen workload (profiling)")
     ap.add_argument("--decode-requests", type=int, default=256,

@@ -213,8 +213,12 @@ kda_status kda_chunk_local_state(const kda_local_state_args *a, void *workspace,
   p.validate = env_flag("KDA_VALIDATE");
   p.status = device_status_word();
   if (!p.status) return KDA_ERR_CUDA;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (prefill_tc_supported(a->dk, a->dv, a->in_dtype) && a->total_tokens > 0 &&
+      !env_flag("KDA_FORCE_SIMT"))
+    return from_cuda(launch_prefill_tc(p, a->in_dtype, KDA_F32, s));
   p.n_slices = prefill_simt_slices(a->dk, a->dv, true);
-  return from_cuda(launch_prefill_simt(p, a->in_dtype, KDA_F32, static_cast<cudaStream_t>(stream)));
+  return from_cuda(launch_prefill_simt(p, a->in_dtype, KDA_F32, s));
 }
 
 kda_status kda_state_combine(const float *s_loc, const float *m, const float *s_init,

@@ -65,6 +65,7 @@ constexpr uint32_t RAW_BYTES = 81920;
 __host__ __device__ constexpr uint32_t rp_off(int a) { return 4096u * a * (a + 1); }
 constexpr uint32_t OFF_R = 81920;       // T-solve scratch (two [64 x 65] fp32); then W [64 x 128]
 constexpr int LDT = 65;                 // padded row stride of the T-solve scratch
+constexpr int LDR = 132;                // padded row stride of the fp32 R scratch [64][132]
 constexpr uint32_t OFF_MS = OFF_R;                  // beta*A strict lower
 constexpr uint32_t OFF_TI = OFF_R + 64 * LDT * 4;   // T = (I + beta A)^-1
 constexpr uint32_t OFF_GQ = 115712;     // (gamma*Q) [64 x 128] tf32 B operand
@@ -81,6 +82,7 @@ constexpr uint32_t OFF_BETA = 228352;   // beta[64]
 constexpr uint32_t OFF_BAR = 228608;    // mbarriers + TMEM base + flags
 constexpr uint32_t SMEM_BYTES = 228704;
 static_assert(OFF_TI + 64 * LDT * 4 <= OFF_GQ, "T-solve scratch must fit the R region");
+static_assert(OFF_R + 64 * LDR * 4 <= OFF_GQ, "R scratch must fit the R region");
 constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;  // alignment slack
 
 // ---- TMEM column map (512 columns x 128 lanes of fp32) ----
@@ -154,8 +156,16 @@ __global__ void __launch_bounds__(NT + 32, 1)
   const int g = (warp >> 2) & 3;                   // worker column quarter
   const uint32_t lane = (uint32_t)((warp & 3) * 32) << 16;
   const int H = p.H;
-  const int r = p.order ? p.order[blockIdx.x / H] : blockIdx.x / H;
-  const int h = blockIdx.x % H;
+  // Local-state mode (context-parallel pass 1): CTA part 0 runs the segment from a
+  // zero state with its values (-> S_loc), part 1 from the identity with zero values
+  // (-> M = A_L ... A_1); the two are the column blocks of the augmented state.
+  const int pairs = p.n_req * H;
+  const int part = p.local_mode ? (int)(blockIdx.x / pairs) : 0;
+  const int rem = (int)(blockIdx.x % pairs);
+  const int r = p.order ? p.order[rem / H] : rem / H;
+  const int h = rem % H;
+  const bool load_q = !p.local_mode;
+  const bool zero_v = p.local_mode && part == 1;
   const int bos = p.cu_seqlens[r], eos = p.cu_seqlens[r + 1];
   const int len = eos - bos;
   if (bos < 0 || len < 0 || eos > p.total_tokens) {  // uniform per CTA, before any barrier
@@ -194,12 +204,12 @@ __global__ void __launch_bounds__(NT + 32, 1)
       tma_prefetch_desc(&maps.v);
       tma_prefetch_desc(&maps.g);
       auto issue_tma = [&](int c0) {
-        mbar_expect_tx(bar_tma, RAW_BYTES);
+        mbar_expect_tx(bar_tma, load_q ? RAW_BYTES : RAW_BYTES - 16384u);
         const int y = bos + c0;
         for (int half = 0; half < 2; ++half) {
           const int x = h * DH + 64 * half;
           tma_load_2d(sm + OFF_KRAW + 8192 * half, &maps.k, x, y, bar_tma);
-          tma_load_2d(sm + OFF_QRAW + 8192 * half, &maps.q, x, y, bar_tma);
+          if (load_q) tma_load_2d(sm + OFF_QRAW + 8192 * half, &maps.q, x, y, bar_tma);
           tma_load_2d(sm + OFF_VRAW + 8192 * half, &maps.v, x, y, bar_tma);
         }
         for (int qd = 0; qd < 4; ++qd)
@@ -298,7 +308,9 @@ __global__ void __launch_bounds__(NT + 32, 1)
           p.initial_state ? p.initial_state + ((size_t)(r * H + h)) * DH * DH : nullptr;
       float v[32];
 #pragma unroll
-      for (int j = 0; j < 32; ++j) v[j] = s0 ? s0[(size_t)(32 * g + j) * DH + l] : 0.f;
+      for (int j = 0; j < 32; ++j)
+        v[j] = p.local_mode ? ((part == 1 && 32 * g + j == l) ? 1.f : 0.f)
+                            : (s0 ? s0[(size_t)(32 * g + j) * DH + l] : 0.f);
       tmem_st32(tm + lane + TM_S + 32 * g, v);
       tmem_wait_st();
     }
@@ -352,83 +364,86 @@ __global__ void __launch_bounds__(NT + 32, 1)
       }
 
       // ---- a3 operands (thread = row i, channels 32g..32g+31) -----------------
-      // L*_i = x_i exp(G_i - G_rb) with r_b the last row of i's own block (x = k or q),
-      // into TMEM; R_i = k_i exp(G_rb - G_i) kept for the B operands R'_a below.
+      // L*_i = x_i exp(G_i - G_rb) with r_b the last row of i's own block (x = k or q)
+      // goes to TMEM; K side: R_i = k_i exp(G_rb - G_i) to fp32 scratch (for R'_a);
+      // Q side: gamma*Q = L* exp(G_rb) to its B operand.
       const bool kside = l < C;
       const int i = l & (C - 1);
       const int bi = i >> 4;
-      const bool valid = i < n;
-      float Rv[32];
+      const bool valid = i < n && (kside || load_q);
+      float *Rs = reinterpret_cast<float *>(sm + OFF_R);  // [64][LDR] fp32 scratch
       {
         const unsigned char *xraw = sm + (kside ? OFF_KRAW : OFF_QRAW);
         const int rb = 16 * bi + 15;
 #pragma unroll
         for (int half = 0; half < 2; ++half) {
-        float Lv[16];
+          float Lv[16];
 #pragma unroll
-        for (int c4 = 0; c4 < 4; ++c4) {
-          const int cc = 4 * half + c4;
-          const int c = 32 * g + 4 * cc;
-          const float4 gi = *reinterpret_cast<const float4 *>(sm + OFF_GRAW + g_off(i, c));
-          const float4 grb = *reinterpret_cast<const float4 *>(sm + OFF_GRAW + g_off(rb, c));
-          float x[4];
-          bf16_x4(xraw, i, c, x);
-          const float giv[4] = {gi.x, gi.y, gi.z, gi.w}, grv[4] = {grb.x, grb.y, grb.z, grb.w};
+          for (int c4 = 0; c4 < 4; ++c4) {
+            const int c = 32 * g + 16 * half + 4 * c4;
+            const float4 gi = *reinterpret_cast<const float4 *>(sm + OFF_GRAW + g_off(i, c));
+            const float4 grb = *reinterpret_cast<const float4 *>(sm + OFF_GRAW + g_off(rb, c));
+            float x[4];
+            bf16_x4(xraw, i, c, x);
+            const float giv[4] = {gi.x, gi.y, gi.z, gi.w}, grv[4] = {grb.x, grb.y, grb.z, grb.w};
+            float lst[4];
 #pragma unroll
-          for (int e = 0; e < 4; ++e) {
-            if (!valid) x[e] = 0.f;
-            const float lst = x[e] * ex2(giv[e] - grv[e]);
-            Lv[4 * c4 + e] = tf32_rna(lst);
+            for (int e = 0; e < 4; ++e) {
+              if (!valid) x[e] = 0.f;
+              lst[e] = x[e] * ex2(giv[e] - grv[e]);
+              Lv[4 * c4 + e] = tf32_rna(lst[e]);
+            }
             if (kside) {
-              Rv[4 * cc + e] = x[e] * ex2(grv[e] - giv[e]);
+              float rv[4];
+#pragma unroll
+              for (int e = 0; e < 4; ++e) rv[e] = x[e] * ex2(grv[e] - giv[e]);
+              *reinterpret_cast<float4 *>(&Rs[i * LDR + c]) = make_float4(rv[0], rv[1], rv[2], rv[3]);
             } else {
-              Rv[4 * cc + e] = lst;  // Q side: gamma*Q = L* exp(G_rb)
+              const float4 eg = *reinterpret_cast<const float4 *>(&sEgr[bi * DH + c]);
+              *reinterpret_cast<float4 *>(sm + OFF_GQ + sw128_chunk(C, i, c)) =
+                  make_float4(tf32_rna(lst[0] * eg.x), tf32_rna(lst[1] * eg.y),
+                              tf32_rna(lst[2] * eg.z), tf32_rna(lst[3] * eg.w));
             }
           }
-          if (kside) {
-            // Khat = R * exp(G_63 - G_rb), stored transposed (rows = channels)
-#pragma unroll
-            for (int e = 0; e < 4; ++e)
-              *reinterpret_cast<float *>(sm + OFF_KHT + sw128_offset(DH, c + e, i)) =
-                  tf32_rna(Rv[4 * cc + e] * sE[(bi * 4 + 3) * DH + c + e]);
-          } else {
-            float gq[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) gq[e] = tf32_rna(Rv[4 * cc + e] * sEgr[bi * DH + c + e]);
-            *reinterpret_cast<float4 *>(sm + OFF_GQ + sw128_chunk(C, i, c)) =
-                make_float4(gq[0], gq[1], gq[2], gq[3]);
-          }
-        }
-        tmem_st16(tm + lane + TM_L + 32 * g + 16 * half, Lv);
+          tmem_st16(tm + lane + TM_L + 32 * g + 16 * half, Lv);
         }
       }
-      // V^T and (gamma*K)^T (thread = channel l, tokens 16g..16g+15), held in registers
-      // (v is bf16, so it is exact in tf32 and is kept packed, two values per register)
+      // thread = channel l, tokens 16g..16g+15: V^T and (gamma*K)^T (kept in registers
+      // until L* is free), Khat^T = k exp(G_63 - G) straight to its B operand
       uint32_t vT2[8];
       float gkT[16];
+      {
+        const float G63 = *reinterpret_cast<const float *>(sm + OFF_GRAW + g_off(C - 1, l));
+        float kh[16];
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const int t = 16 * g + j;
-        const float G2 = *reinterpret_cast<const float *>(sm + OFF_GRAW + g_off(t, l));
-        const uint32_t vb = (t < n) ? (uint32_t)*reinterpret_cast<const unsigned short *>(
-                                          sm + OFF_VRAW + bf16_off(t, l))
-                                    : 0u;
-        if (j & 1) vT2[j >> 1] |= vb << 16; else vT2[j >> 1] = vb;
-        gkT[j] = (t < n) ? tf32_rna(bf16_at(sm + OFF_KRAW, t, l) * ex2(G2)) : 0.f;
+        for (int j = 0; j < 16; ++j) {
+          const int t = 16 * g + j;
+          const float G2 = *reinterpret_cast<const float *>(sm + OFF_GRAW + g_off(t, l));
+          const uint32_t vb = (t < n && !zero_v) ? (uint32_t)*reinterpret_cast<const unsigned short *>(
+                                            sm + OFF_VRAW + bf16_off(t, l))
+                                      : 0u;
+          if (j & 1) vT2[j >> 1] |= vb << 16; else vT2[j >> 1] = vb;
+          const float kk = (t < n) ? bf16_at(sm + OFF_KRAW, t, l) : 0.f;
+          gkT[j] = tf32_rna(kk * ex2(G2));
+          kh[j] = tf32_rna(kk * ex2(G63 - G2));
+        }
+#pragma unroll
+        for (int m4 = 0; m4 < 4; ++m4)
+          *reinterpret_cast<float4 *>(sm + OFF_KHT + sw128_chunk(DH, l, 16 * g + 4 * m4)) =
+              make_float4(kh[4 * m4], kh[4 * m4 + 1], kh[4 * m4 + 2], kh[4 * m4 + 3]);
       }
       wsync();  // every raw tile read: the raw region now takes the R'_a operands
-      if (kside) {
-        // R'_a row i = R_i exp(G_ra - G_rb) for every row block a >= bi
-        for (int a = bi; a < 4; ++a) {
-          const int rows = 16 * (a + 1);
+      // R'_a row j = R_j exp(G_ra - G_rb(j)) for j <= r_a, spread over all workers
 #pragma unroll
-          for (int cc = 0; cc < 8; ++cc) {
-            const int c = 32 * g + 4 * cc;
-            const float *ea = sE + (bi * 4 + a) * DH + c;
-            *reinterpret_cast<float4 *>(sm + rp_off(a) + sw128_chunk(rows, i, c)) =
-                make_float4(tf32_rna(Rv[4 * cc] * ea[0]), tf32_rna(Rv[4 * cc + 1] * ea[1]),
-                            tf32_rna(Rv[4 * cc + 2] * ea[2]), tf32_rna(Rv[4 * cc + 3] * ea[3]));
-          }
+      for (int a = 0; a < 4; ++a) {
+        const int rows = 16 * (a + 1);
+        for (int it = tid; it < rows * 32; it += NT) {
+          const int j = it >> 5, c = (it & 31) * 4;
+          const float4 rv = *reinterpret_cast<const float4 *>(&Rs[j * LDR + c]);
+          const float4 ea = *reinterpret_cast<const float4 *>(&sE[((j >> 4) * 4 + a) * DH + c]);
+          *reinterpret_cast<float4 *>(sm + rp_off(a) + sw128_chunk(rows, j, c)) =
+              make_float4(tf32_rna(rv.x * ea.x), tf32_rna(rv.y * ea.y), tf32_rna(rv.z * ea.z),
+                          tf32_rna(rv.w * ea.w));
         }
       }
       tmem_wait_st();
@@ -602,8 +617,9 @@ __global__ void __launch_bounds__(NT + 32, 1)
       wsync();
     }
 
-    if (ok && p.final_state) {
-      float *dst = p.final_state + ((size_t)(r * H + h)) * DH * DH;
+    float *fin = p.local_mode ? (part == 0 ? p.s_loc : p.m) : p.final_state;
+    if (ok && fin) {
+      float *dst = fin + ((size_t)(r * H + h)) * DH * DH;
       tc_fence_after();
       float v[32];
       tmem_ld32(tm + lane + TM_S + 32 * g, v);
@@ -654,22 +670,23 @@ cudaError_t launch_prefill_tc(const PrefillParams &p, kda_dtype in_dtype, kda_dt
   if (p.n_req == 0) return cudaSuccess;
   TcMaps maps;
   const uint64_t T = (uint64_t)p.total_tokens, W = (uint64_t)p.H * DH;
-  if (!encode_map(&maps.q, p.q, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W, T, 64) ||
+  if (!encode_map(&maps.q, p.q ? p.q : p.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W, T, 64) ||
       !encode_map(&maps.k, p.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W, T, 64) ||
       !encode_map(&maps.v, p.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W, T, 64) ||
       !encode_map(&maps.g, p.g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, W, T, 32))
     return cudaErrorInvalidValue;
+  const unsigned grid = (unsigned)(p.n_req * p.H * (p.local_mode ? 2 : 1));
   cudaError_t e;
   if (out_dtype == KDA_BF16) {
     e = cudaFuncSetAttribute(prefill_tc_kernel<__nv_bfloat16>,
                              cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_ALLOC);
     if (e != cudaSuccess) return e;
-    prefill_tc_kernel<__nv_bfloat16><<<(unsigned)(p.n_req * p.H), NT + 32, SMEM_ALLOC, stream>>>(p, maps);
+    prefill_tc_kernel<__nv_bfloat16><<<grid, NT + 32, SMEM_ALLOC, stream>>>(p, maps);
   } else {
     e = cudaFuncSetAttribute(prefill_tc_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                              (int)SMEM_ALLOC);
     if (e != cudaSuccess) return e;
-    prefill_tc_kernel<float><<<(unsigned)(p.n_req * p.H), NT + 32, SMEM_ALLOC, stream>>>(p, maps);
+    prefill_tc_kernel<float><<<grid, NT + 32, SMEM_ALLOC, stream>>>(p, maps);
   }
   return cudaGetLastError();
 }
