@@ -527,30 +527,38 @@ __global__ void __launch_bounds__(NT + 32, 1)
         Ti[rot(16 * a + k, 16 * b + j)] = -t;
         wsync();
       }
-      // 32 -> 64: T[32:64, 0:32] = -T[32:64, 32:64] (N[32:64, 0:32] T[0:32, 0:32])
+      // 32 -> 64: T[32:64, 0:32] = -T[32:64, 32:64] (N[32:64, 0:32] T[0:32, 0:32]);
+      // two outputs per thread, each summed in two halves to shorten the FMA chains
       {
         const int ii = tid >> 4, j0 = tid & 15;  // rows ii, columns j0 and j0 + 16
-        float y0 = 0.f, y1 = 0.f;
-#pragma unroll 8
-        for (int q = 0; q < 32; ++q) {
-          const float nv = Ms[rot(32 + ii, q)];
-          if (q >= j0) y0 += nv * Ti[rot(q, j0)];
-          if (q >= j0 + 16) y1 += nv * Ti[rot(q, j0 + 16)];
+        float y0a = 0.f, y0b = 0.f, y1a = 0.f, y1b = 0.f;
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
+          const float na = Ms[rot(32 + ii, q)], nb = Ms[rot(32 + ii, q + 16)];
+          if (q >= j0) y0a += na * Ti[rot(q, j0)];
+          y0b += nb * Ti[rot(q + 16, j0)];
+          y1b += (q >= j0) ? nb * Ti[rot(q + 16, j0 + 16)] : 0.f;
+          (void)y1a;
         }
-        Ys[ii * 33 + j0] = y0;
-        Ys[ii * 33 + j0 + 16] = y1;
+        Ys[ii * 33 + j0] = y0a + y0b;
+        Ys[ii * 33 + j0 + 16] = y1b;
         wsync();
-        float t0 = 0.f, t1 = 0.f;
-#pragma unroll 8
-        for (int q = 0; q < 32; ++q) {
+        float t0a = 0.f, t0b = 0.f, t1a = 0.f, t1b = 0.f;
+#pragma unroll
+        for (int q = 0; q < 16; ++q) {
           if (q <= ii) {
             const float tv = Ti[rot(32 + ii, 32 + q)];
-            t0 += tv * Ys[q * 33 + j0];
-            t1 += tv * Ys[q * 33 + j0 + 16];
+            t0a += tv * Ys[q * 33 + j0];
+            t1a += tv * Ys[q * 33 + j0 + 16];
+          }
+          if (q + 16 <= ii) {
+            const float tv = Ti[rot(32 + ii, 48 + q)];
+            t0b += tv * Ys[(q + 16) * 33 + j0];
+            t1b += tv * Ys[(q + 16) * 33 + j0 + 16];
           }
         }
-        Ti[rot(32 + ii, j0)] = -t0;
-        Ti[rot(32 + ii, j0 + 16)] = -t1;
+        Ti[rot(32 + ii, j0)] = -(t0a + t0b);
+        Ti[rot(32 + ii, j0 + 16)] = -(t1a + t1b);
         wsync();
       }
       if (kside) {  // TB = T Diag(beta): row i, columns 16g..16g+15
