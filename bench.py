@@ -3,7 +3,7 @@
 
 One step = one chunked prefill (kda_prefill_chunked through the C ABI) of the
 varlen workload: 64 requests with lengths log-uniform on [128, 4096] (seed 0,
-73,490 tokens), H=32, d_k=d_v=128, bf16 q/k/v, fp32 g/beta, fp32 outputs,
+72,585 tokens), H=32, d_k=d_v=128, bf16 q/k/v, fp32 g/beta, fp32 outputs,
 zero initial states, final states returned.  Inputs are generated on the
 device before timing and are larger than L2 (about 2.7 GB per step), so no
 L2 flush is needed between steps.
@@ -110,6 +110,23 @@ class ClockSampler:
         return {"sm_mhz": statistics.median(sm) if sm else None,
                 "sm_max_mhz": max(mx) if mx else None, "reasons": reasons,
                 "samples": len(rows), "power_w_max": max(pw) if pw else None}
+
+
+def measured_traffic(algorithmic_bytes: int):
+    """DRAM bytes per launch of the prefill kernel from the committed ncu capture
+    (profiles/prefill_tc_traffic.json), scaled from the captured case by the
+    algorithmic bytes; None when the kernel source changed since the capture."""
+    import hashlib
+    try:
+        with open(os.path.join(ROOT, "profiles", "prefill_tc_traffic.json")) as f:
+            cap = json.load(f)
+        with open(os.path.join(ROOT, cap["source"]), "rb") as f:
+            sha = hashlib.sha256(f.read()).hexdigest()
+    except (OSError, KeyError, ValueError):
+        return None
+    if sha != cap.get("source_sha256"):
+        return None
+    return cap["traffic_over_algorithmic"] * algorithmic_bytes
 
 
 def load_peaks():
@@ -320,6 +337,7 @@ def run_ours(args, world, rank, local):
     value = world * T * args.steps / (total_ms * 1e-3)
     tc = kda.kda_prefill_uses_tensor_cores(dk, dv)
 
+    traffic = measured_traffic(bytes_)
     line = {"metric": METRIC, "value": value, "unit": "tokens/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": total_ms / args.steps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -328,7 +346,7 @@ def run_ours(args, world, rank, local):
             "tflops": tflops,
             "roofline": {"bound": "hbm", "achieved": achieved_gbs, "peak": peaks["hbm_gbs"],
                          "unit": "GB/s", "frac": achieved_gbs / peaks["hbm_gbs"],
-                         "traffic": None, "peak_kind": peak_kind,
+                         "traffic": traffic, "peak_kind": peak_kind,
                          "algorithmic_bytes_per_launch": bytes_,
                          "launch_ms": launch_ms,
                          "tensor_frac": tflops / peaks["bf16_tflops"],

@@ -63,7 +63,7 @@ def build(verbose: bool = False, jobs: int | None = None, extra=()) -> str:
     with cf.ThreadPoolExecutor(max_workers=jobs or min(8, len(srcs))) as ex:
         objs = list(ex.map(lambda s: _compile(s, verbose, list(extra)), srcs))
     if _stale(LIB, objs) or extra:
-        cmd = [nvcc(), *ARCH, "-shared", "-o", LIB, *objs, "-lcuda"]
+        cmd = [nvcc(), *ARCH, "-shared", "-o", LIB, *objs]
         subprocess.run(cmd, check=True)
     return LIB
 
