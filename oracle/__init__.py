@@ -75,6 +75,10 @@ def _bind(lib):
     lib.oracle_kda_state_combine.argtypes = [
         ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
         _D, _D, _D, _D, _D]
+    lib.oracle_kda_prefill_backward.restype = ctypes.c_int
+    lib.oracle_kda_prefill_backward.argtypes = [
+        ctypes.c_int, _I64, ctypes.c_int, ctypes.c_int, ctypes.c_int,
+        _D, _D, _D, _D, _D, _D, _D, _D, _D, _D, _D, _D, _D, _D, ctypes.c_int]
     lib.oracle_snapshot_count.restype = ctypes.c_long
     lib.oracle_snapshot_count.argtypes = [ctypes.c_long, ctypes.c_long]
     return lib
@@ -148,6 +152,33 @@ def prefill(q, k, v, g, beta, cu_seqlens, initial_state=None, snapshot_stride: i
     return {"o": o, "final_state": fin,
             "snapshots": snaps if snaps is not None else np.zeros((0, H, dk, dv)),
             "cu_snapshots": cu_snap}
+
+
+def prefill_backward(q, k, v, g, beta, cu_seqlens, initial_state=None, d_o=None,
+                     d_final=None, n_threads: int | None = None, lib=None):
+    """Gradients of L = sum(d_o * o) + sum(d_final * final_state) of the prefill
+    map, by reverse mode through the recurrence's defining lines
+    (``oracle_kda_prefill_backward`` in kda_oracle.c).
+
+    Returns dict(dq, dk, dv, dg, dbeta, d_initial) shaped like the inputs
+    (d_initial [n_req, H, dk, dv]).  d_o / d_final / initial_state may be None."""
+    lib = lib or load()
+    q, k, v, g, beta = (_f64(a) for a in (q, k, v, g, beta))
+    s0, do, dfin = _f64(initial_state), _f64(d_o), _f64(d_final)
+    cu = _i64(cu_seqlens)
+    T, H, dk = k.shape
+    dv = v.shape[2]
+    n_req = cu.shape[0] - 1
+    out = {"dq": np.zeros((T, H, dk)), "dk": np.zeros((T, H, dk)), "dv": np.zeros((T, H, dv)),
+           "dg": np.zeros((T, H, dk)), "dbeta": np.zeros((T, H)),
+           "d_initial": np.zeros((n_req, H, dk, dv))}
+    rc = lib.oracle_kda_prefill_backward(
+        n_req, _p(cu, _I64), H, dk, dv, _p(q), _p(k), _p(v), _p(g), _p(beta), _p(s0), _p(do),
+        _p(dfin), _p(out["dq"]), _p(out["dk"]), _p(out["dv"]), _p(out["dg"]), _p(out["dbeta"]),
+        _p(out["d_initial"]), int(n_threads or default_threads()))
+    if rc != 0:
+        raise ValueError(f"oracle_kda_prefill_backward failed with code {rc}")
+    return out
 
 
 def decode_step(q, k, v, g, beta, state, slot=None, n_threads: int | None = None, lib=None):

@@ -341,3 +341,182 @@ int oracle_kda_state_combine(int n_seg, int H, int dk, int dv, const double *s_l
     free(nxt);
     return ORACLE_OK;
 }
+
+/* ------------------------------------------------------------------------- */
+/* Backward (training): the vector-Jacobian product of the prefill map.      */
+/* FlashKDA also "raises training throughput" ("Kimi K3 开源日来了",          */
+/* FlashKDA section), so the derivative of the same map is part of the path. */
+/* Given cotangents dO (of o) and dS_final (of the final state), it returns  */
+/* dq, dk, dv, dg (of g = log alpha), dbeta and dS_0 (of the initial state). */
+/* Snapshots are by-products and take no cotangent.                          */
+/*                                                                           */
+/* The derivative is taken through the four defining lines of kda_step and   */
+/* the read-out, in reverse:                                                 */
+/*     o = S_t^T q          ->  dq = S_t dO,   dS += q dO^T                  */
+/*     S_t = S' + k d^T     ->  dd = dS^T k,   dk = dS d,   dS' = dS         */
+/*     d = beta (v - u)     ->  dv = beta dd,  dbeta = dd . (v - u),         */
+/*                              du = -beta dd                                */
+/*     u = S'^T k           ->  dS' += k du^T, dk += S' du                   */
+/*     S' = Diag(a) S_{t-1} ->  dg_i = a_i sum_j dS'_ij S_{t-1,ij},          */
+/*                              dS_{t-1} = Diag(a) dS'                       */
+/* The forward states S_{t-1} are recomputed, in the forward order, in       */
+/* blocks of 64 tokens from block-start states saved by a first forward      */
+/* pass, so memory stays at (L/64 + 65) states per chain.                    */
+/* ------------------------------------------------------------------------- */
+
+#define ORACLE_BWD_BLOCK 64
+
+typedef struct {
+    int H, dk, dv;
+    const int64_t *cu;
+    const double *q, *k, *v, *g, *beta, *s0, *d_o, *d_final;
+    double *dq, *dk_, *dv_, *dg, *dbeta, *d_init;
+} backward_ctx;
+
+/* One reverse step.  S_prev = S_{t-1}; dS holds dL/dS_t on entry and
+ * dL/dS_{t-1} on exit.  Sp and dSp are dk x dv scratch, u/dd/du dv scratch. */
+static void kda_step_backward(const double *S_prev, double *dS, int dk, int dv,
+                              const double *q, const double *k, const double *v,
+                              const double *g, double beta, const double *dO,
+                              double *dq, double *dk_out, double *dv_out, double *dg,
+                              double *dbeta, double *Sp, double *u, double *dd,
+                              double *du) {
+    int i, j;
+    double s, dq_tail = 0.0;
+    /* recompute the forward line by line: S', u, d */
+    for (i = 0; i < dk; ++i) {
+        const double a = exp(g[i]);
+        for (j = 0; j < dv; ++j) Sp[(size_t)i * dv + j] = a * S_prev[(size_t)i * dv + j];
+    }
+    for (j = 0; j < dv; ++j) {
+        s = 0.0;
+        for (i = 0; i < dk; ++i) s += Sp[(size_t)i * dv + j] * k[i];
+        u[j] = s;
+    }
+    /* d = beta (v - u); d lives in du's slot until du itself is formed below */
+    for (j = 0; j < dv; ++j) du[j] = beta * (v[j] - u[j]);
+    /* o = S_t^T q with S_t = S' + k d^T:  dq = S' dO + k (d . dO) */
+    if (dO) {
+        for (j = 0; j < dv; ++j) dq_tail += du[j] * dO[j];
+        for (i = 0; i < dk; ++i) {
+            s = 0.0;
+            for (j = 0; j < dv; ++j) s += Sp[(size_t)i * dv + j] * dO[j];
+            dq[i] = s + k[i] * dq_tail;
+        }
+        for (i = 0; i < dk; ++i)
+            for (j = 0; j < dv; ++j) dS[(size_t)i * dv + j] += q[i] * dO[j];
+    } else {
+        for (i = 0; i < dk; ++i) dq[i] = 0.0;
+    }
+    /* S_t = S' + k d^T:  dd = dS^T k,  dk = dS d */
+    for (j = 0; j < dv; ++j) {
+        s = 0.0;
+        for (i = 0; i < dk; ++i) s += dS[(size_t)i * dv + j] * k[i];
+        dd[j] = s;
+    }
+    for (i = 0; i < dk; ++i) {
+        s = 0.0;
+        for (j = 0; j < dv; ++j) s += dS[(size_t)i * dv + j] * du[j];
+        dk_out[i] = s;
+    }
+    /* d = beta (v - u):  dv = beta dd,  dbeta = dd . (v - u),  du = -beta dd */
+    s = 0.0;
+    for (j = 0; j < dv; ++j) {
+        dv_out[j] = beta * dd[j];
+        s += dd[j] * (v[j] - u[j]);
+        du[j] = -beta * dd[j];
+    }
+    *dbeta = s;
+    /* u = S'^T k:  dS' = dS + k du^T,  dk += S' du */
+    for (i = 0; i < dk; ++i) {
+        s = 0.0;
+        for (j = 0; j < dv; ++j) s += Sp[(size_t)i * dv + j] * du[j];
+        dk_out[i] += s;
+        for (j = 0; j < dv; ++j) dS[(size_t)i * dv + j] += k[i] * du[j];
+    }
+    /* S' = Diag(a) S_{t-1}:  dg_i = a_i sum_j dS'_ij S_{t-1,ij};  dS_{t-1} = Diag(a) dS' */
+    for (i = 0; i < dk; ++i) {
+        const double a = exp(g[i]);
+        s = 0.0;
+        for (j = 0; j < dv; ++j) s += dS[(size_t)i * dv + j] * S_prev[(size_t)i * dv + j];
+        dg[i] = a * s;
+        for (j = 0; j < dv; ++j) dS[(size_t)i * dv + j] *= a;
+    }
+}
+
+static void backward_job(void *vctx, long job) {
+    const backward_ctx *c = (const backward_ctx *)vctx;
+    const int r = (int)(job / c->H), h = (int)(job % c->H);
+    const int H = c->H, dk = c->dk, dv = c->dv;
+    const size_t ss = (size_t)dk * dv;
+    const int64_t t0 = c->cu[r], L = c->cu[r + 1] - c->cu[r];
+    const int64_t n_blk = (L + ORACLE_BWD_BLOCK - 1) / ORACLE_BWD_BLOCK;
+    double *ck = (double *)malloc((size_t)(n_blk + 1) * ss * sizeof(double));
+    double *blk = (double *)malloc((size_t)(ORACLE_BWD_BLOCK + 1) * ss * sizeof(double));
+    double *dS = (double *)malloc(ss * sizeof(double));
+    double *Sp = (double *)malloc(ss * sizeof(double));
+    double *w = (double *)malloc((size_t)4 * dv * sizeof(double));
+    int64_t b, t;
+    if (!ck || !blk || !dS || !Sp || !w) goto done;
+    /* forward pass: keep the state at every block start */
+    if (c->s0) memcpy(ck, c->s0 + ((size_t)r * H + h) * ss, ss * sizeof(double));
+    else memset(ck, 0, ss * sizeof(double));
+    memcpy(blk, ck, ss * sizeof(double));
+    for (t = 0; t < L; ++t) {
+        const size_t th = (size_t)(t0 + t) * H + h;
+        kda_step(blk, dk, dv, c->k + th * dk, c->v + th * dv, c->g + th * dk, c->beta[th], w);
+        if ((t + 1) % ORACLE_BWD_BLOCK == 0)
+            memcpy(ck + (size_t)((t + 1) / ORACLE_BWD_BLOCK) * ss, blk, ss * sizeof(double));
+    }
+    /* reverse pass */
+    if (c->d_final) memcpy(dS, c->d_final + ((size_t)r * H + h) * ss, ss * sizeof(double));
+    else memset(dS, 0, ss * sizeof(double));
+    for (b = n_blk - 1; b >= 0; --b) {
+        const int64_t lo = b * ORACLE_BWD_BLOCK;
+        const int64_t hi = (lo + ORACLE_BWD_BLOCK < L) ? lo + ORACLE_BWD_BLOCK : L;
+        /* blk[i] = S_{lo + i}, recomputed forward from the saved S_lo */
+        memcpy(blk, ck + (size_t)b * ss, ss * sizeof(double));
+        for (t = lo; t < hi - 1; ++t) {
+            const size_t th = (size_t)(t0 + t) * H + h;
+            memcpy(blk + (size_t)(t - lo + 1) * ss, blk + (size_t)(t - lo) * ss, ss * sizeof(double));
+            kda_step(blk + (size_t)(t - lo + 1) * ss, dk, dv, c->k + th * dk, c->v + th * dv,
+                     c->g + th * dk, c->beta[th], w);
+        }
+        for (t = hi - 1; t >= lo; --t) {
+            const size_t th = (size_t)(t0 + t) * H + h;
+            kda_step_backward(blk + (size_t)(t - lo) * ss, dS, dk, dv, c->q + th * dk,
+                              c->k + th * dk, c->v + th * dv, c->g + th * dk, c->beta[th],
+                              c->d_o ? c->d_o + th * dv : NULL, c->dq + th * dk,
+                              c->dk_ + th * dk, c->dv_ + th * dv, c->dg + th * dk,
+                              c->dbeta + th, Sp, w, w + dv, w + 2 * dv);
+        }
+    }
+    if (c->d_init) memcpy(c->d_init + ((size_t)r * H + h) * ss, dS, ss * sizeof(double));
+done:
+    free(ck); free(blk); free(dS); free(Sp); free(w);
+}
+
+/* Gradients of L = sum(dO * o) + sum(dS_final * S_final) with respect to
+ * q, k, v, g, beta and the initial state, for the same packed requests as
+ * oracle_kda_prefill.  d_o / d_final / initial_state may be NULL (zeros);
+ * d_initial may be NULL (not returned). */
+int oracle_kda_prefill_backward(int n_req, const int64_t *cu_seqlens, int H, int dk, int dv,
+                                const double *q, const double *k, const double *v,
+                                const double *g, const double *beta,
+                                const double *initial_state, const double *d_o,
+                                const double *d_final, double *dq, double *dk_out,
+                                double *dv_out, double *dg, double *dbeta,
+                                double *d_initial, int n_threads) {
+    backward_ctx c;
+    int r;
+    if (n_req < 0 || H <= 0 || dk <= 0 || dv <= 0 || !cu_seqlens) return ORACLE_EINVAL;
+    if (!dq || !dk_out || !dv_out || !dg || !dbeta) return ORACLE_EINVAL;
+    for (r = 0; r < n_req; ++r)
+        if (cu_seqlens[r + 1] < cu_seqlens[r]) return ORACLE_EINVAL;
+    c.H = H; c.dk = dk; c.dv = dv; c.cu = cu_seqlens;
+    c.q = q; c.k = k; c.v = v; c.g = g; c.beta = beta; c.s0 = initial_state;
+    c.d_o = d_o; c.d_final = d_final;
+    c.dq = dq; c.dk_ = dk_out; c.dv_ = dv_out; c.dg = dg; c.dbeta = dbeta; c.d_init = d_initial;
+    run_jobs(backward_job, &c, (long)n_req * H, n_threads);
+    return ORACLE_OK;
+}

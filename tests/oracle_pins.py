@@ -379,7 +379,107 @@ def pin_varlen_isolation(lib):
         assert np.array_equal(alone["snapshots"], packed["snapshots"][cs[r_]:cs[r_ + 1]])
 
 
+# ----------------------------------------------------------------------------
+# Backward (vector-Jacobian product of the prefill map)
+# ----------------------------------------------------------------------------
+
+_GRAD_OF = {"q": "dq", "k": "dk", "v": "dv", "g": "dg", "beta": "dbeta", "s0": "d_initial"}
+
+
+def _loss(lib, x, d_o, d_fin):
+    r = _run(lib, x)
+    return float((r["o"] * d_o).sum() + (r["final_state"] * d_fin).sum())
+
+
+def _backward(lib, x, d_o, d_fin):
+    return oracle.prefill_backward(x["q"], x["k"], x["v"], x["g"], x["beta"], x["cu"], x["s0"],
+                                   d_o, d_fin, n_threads=2, lib=lib)
+
+
+def _fd_check(lib, x, d_o, d_fin, n_sample=None, seed=0, h=1e-6, tol=1e-6):
+    """Central differences of the forward oracle's scalar loss against the
+    backward's gradients, element by element (all, or n_sample per input)."""
+    grads = _backward(lib, x, d_o, d_fin)
+    rng = _rng(seed)
+    for name, gname in _GRAD_OF.items():
+        a = x[name]
+        idx = list(np.ndindex(a.shape))
+        if n_sample is not None:
+            idx = [idx[i] for i in rng.choice(len(idx), size=min(n_sample, len(idx)), replace=False)]
+        scale = max(np.abs(grads[gname]).max(), 1e-12)
+        for ix in idx:
+            keep = a[ix]
+            a[ix] = keep + h
+            lp = _loss(lib, x, d_o, d_fin)
+            a[ix] = keep - h
+            lm = _loss(lib, x, d_o, d_fin)
+            a[ix] = keep
+            fd = (lp - lm) / (2 * h)
+            assert abs(fd - grads[gname][ix]) <= tol * scale, (name, ix, fd, grads[gname][ix])
+
+
+def pin_backward_finite_differences(lib):
+    """Every gradient element of a small varlen case (two requests, an initial
+    state, random cotangents) equals the central difference of the forward."""
+    x = rand_inputs([5, 9], H=2, dk=3, dv=4, seed=71, gate_lo=-1.0, s0_std=1.0)
+    rng = _rng(72)
+    d_o = rng.standard_normal(x["v"].shape)
+    d_fin = rng.standard_normal(x["s0"].shape)
+    _fd_check(lib, x, d_o, d_fin)
+
+
+def pin_backward_across_blocks(lib):
+    """A 150-token chain crosses the backward's 64-token recompute blocks twice;
+    sampled elements of every gradient still match central differences."""
+    x = rand_inputs([150], H=1, dk=3, dv=2, seed=73, gate_lo=-0.5, s0_std=1.0)
+    rng = _rng(74)
+    d_o = rng.standard_normal(x["v"].shape)
+    d_fin = rng.standard_normal(x["s0"].shape)
+    _fd_check(lib, x, d_o, d_fin, n_sample=40, seed=75)
+
+
+def pin_backward_beta0_closed_form(lib):
+    """beta = 0 and dO = 0: S_L = Diag(gamma_L) S_0 with gamma_L = exp(sum_t g_t), so
+    dS_0 = Diag(gamma_L) dS_L, dg_t,i = gamma_L,i sum_j dS_L,ij S_0,ij for every t,
+    dq = dk = dv = 0, and dbeta_t = k_t^T Diag(gamma_L / gamma_t) dS_L
+    (v_t - (Diag(gamma_t) S_0)^T k_t) with gamma_t the decay over tokens 1..t."""
+    x = rand_inputs([11], H=1, dk=4, dv=3, seed=76, s0_std=1.0)
+    x["beta"][:] = 0.0
+    rng = _rng(77)
+    d_fin = rng.standard_normal(x["s0"].shape)
+    r = _backward(lib, x, None, d_fin)
+    g = x["g"][:, 0]
+    S0, dF = x["s0"][0, 0], d_fin[0, 0]
+    gam_L = np.exp(g.sum(0))
+    np.testing.assert_allclose(r["d_initial"][0, 0], gam_L[:, None] * dF, rtol=1e-12, atol=1e-14)
+    for name in ("dq", "dk", "dv"):
+        assert np.array_equal(r[name], np.zeros_like(r[name])), name
+    row = gam_L * (dF * S0).sum(1)
+    for t in range(11):
+        np.testing.assert_allclose(r["dg"][t, 0], row, rtol=1e-12, atol=1e-14)
+        gam_t = np.exp(g[:t + 1].sum(0))
+        kt = x["k"][t, 0]
+        ref = kt @ ((gam_L / gam_t)[:, None] * dF) @ (x["v"][t, 0] - (gam_t[:, None] * S0).T @ kt)
+        np.testing.assert_allclose(r["dbeta"][t, 0], ref, rtol=1e-10, atol=1e-13)
+
+
+def pin_backward_dq_is_state_times_cotangent(lib):
+    """o_t = S_t^T q_t makes dq_t = S_t dO_t exactly; S_t is read from the forward
+    oracle's snapshots at stride 1 (dS_L = 0)."""
+    x = rand_inputs([7, 12], H=2, dk=5, dv=3, seed=78, s0_std=0.5)
+    rng = _rng(79)
+    d_o = rng.standard_normal(x["v"].shape)
+    r = _backward(lib, x, d_o, None)
+    f = _run(lib, x, stride=1)
+    for t in range(19):
+        for h in range(2):
+            np.testing.assert_allclose(r["dq"][t, h], f["snapshots"][t, h] @ d_o[t, h],
+                                       rtol=1e-12, atol=1e-13)
+
+
 ALL_PINS = [pin_identity_beta0, pin_orthonormal_retrieval, pin_self_query,
             pin_decay_closed_form, pin_golden_fixtures, pin_brute_force, pin_chunked_form,
             pin_split_combine, pin_snapshot_tagging, pin_contraction_bound, pin_resume,
-            pin_decode_matches_prefill, pin_decode_slots, pin_varlen_isolation]
+            pin_decode_matches_prefill, pin_decode_slots, pin_varlen_isolation,
+            pin_backward_finite_differences, pin_backward_across_blocks,
+            pin_backward_beta0_closed_form, pin_backward_dq_is_state_times_cotangent]

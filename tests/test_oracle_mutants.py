@@ -46,6 +46,15 @@ MUTANTS = {
     "transition_dropped_beta": ("M[(size_t)i * dk + j] -= bt * kt[i] * w[j];",
                                 "M[(size_t)i * dk + j] -= kt[i] * w[j];"),
     "decode_ignores_slot": ("c->slot ? c->slot[n] : n", "n"),
+    "bwd_dropped_read_term": ("for (j = 0; j < dv; ++j) dS[(size_t)i * dv + j] += k[i] * du[j];",
+                              "for (j = 0; j < dv; ++j) dS[(size_t)i * dv + j] += 0.0 * du[j];"),
+    "bwd_du_sign": ("du[j] = -beta * dd[j];", "du[j] = beta * dd[j];"),
+    "bwd_dg_without_alpha": ("dg[i] = a * s;", "dg[i] = s;"),
+    "bwd_dq_dropped_write": ("dq[i] = s + k[i] * dq_tail;", "dq[i] = s;"),
+    "bwd_dk_transposed_state": ("for (j = 0; j < dv; ++j) s += Sp[(size_t)i * dv + j] * du[j];",
+                                "for (j = 0; j < dv; ++j) s += Sp[(size_t)(j % dk) * dv + i % dv] * du[j];"),
+    "bwd_wrong_checkpoint": ("memcpy(blk, ck + (size_t)b * ss, ss * sizeof(double));",
+                             "memcpy(blk, ck + (size_t)(b > 0 ? b - 1 : 0) * ss, ss * sizeof(double));"),
     "readout_uses_key": ("kda_readout(S, dk, dv, c->q + th * dk, c->o + th * dv);\n    free(u);",
                          "kda_readout(S, dk, dv, c->k + th * dk, c->o + th * dv);\n    free(u);"),
 }
