@@ -117,6 +117,92 @@ def chunked_chain(q, k, v, g, beta, s0, C):
     return O, S
 
 
+def chunked_backward_chain(q, k, v, g, beta, s0, d_o, d_fin, C):
+    """The backward of chunked_chain, derived by reverse mode through its
+    chunk algebra (one chain).  Returns dict(dq, dk, dv, dg, dbeta, d_initial).
+
+    Per chunk, with S its start state, dSn the cotangent of its end state,
+    Gam = gamma at the chunk's last token and Khat = (Gam / gamma) * K:
+      dU  = P^T dO + Khat dSn
+      dS  = Diag(Gam) dSn + (gamma Q)^T dO - W^T dU            (serial, chunks in reverse)
+      dP  = tril(dO U^T),  d(gamma Q) = dO S^T,  dKhat = U dSn^T,  dW = -dU S^T
+      [U~ | W] = T Diag(beta) [V | gamma K]  ->  dV, d(gamma K), dT, dbeta
+      T = (I + Diag(beta) A)^-1  ->  dZ = -T^T dT T^T,  dA = tril_strict(Diag(beta) dZ)
+      A, P gated products -> dK, dQ and the cumulative-gate cotangent dG, every
+      gate factor an exp(G_t - G_s) with t >= s (never above 1);
+      dg = reverse cumulative sum of dG inside the chunk.
+    """
+    L, dk = k.shape
+    dv = v.shape[1]
+    starts = list(range(0, L, C))
+    # forward: chunk-start states and the chunk quantities the backward reuses
+    S = s0.copy()
+    fw = []
+    for c0 in starts:
+        sl = slice(c0, min(c0 + C, L))
+        K, Q, V, b = k[sl], q[sl], v[sl], beta[sl]
+        n = K.shape[0]
+        G = np.cumsum(g[sl], axis=0)
+        ii, jj = np.meshgrid(np.arange(n), np.arange(n), indexing="ij")
+        D = np.where((ii >= jj)[:, :, None], G[:, None, :] - G[None, :, :], -np.inf)
+        E = np.exp(D)                                   # E[t, s, c] = exp(G_tc - G_sc), t >= s
+        A = np.einsum("ic,jc,ijc->ij", K, K, E) * (ii > jj)
+        P = np.einsum("ic,jc,ijc->ij", Q, K, E) * (ii >= jj)
+        gam = np.exp(G)
+        Gam = gam[-1]
+        T = np.linalg.inv(np.eye(n) + b[:, None] * A)
+        Kg, Qg = gam * K, gam * Q
+        W = T @ (b[:, None] * Kg)
+        Ut = T @ (b[:, None] * V)
+        U = Ut - W @ S
+        Kh = (Gam[None, :] / gam) * K
+        fw.append(dict(sl=sl, K=K, Q=Q, V=V, b=b, n=n, G=G, E=E, A=A, P=P, gam=gam, Gam=Gam,
+                       T=T, Kg=Kg, Qg=Qg, W=W, U=U, Kh=Kh, S=S.copy(), ii=ii, jj=jj))
+        S = Gam[:, None] * S + Kh.T @ U
+    out = {"dq": np.zeros_like(q), "dk": np.zeros_like(k), "dv": np.zeros_like(v),
+           "dg": np.zeros_like(g), "dbeta": np.zeros_like(beta)}
+    # serial reverse pass over chunk-end cotangents
+    dS = d_fin.copy()
+    for f in reversed(fw):
+        dO = d_o[f["sl"]]
+        dSn = dS
+        dU = f["P"].T @ dO + f["Kh"] @ dSn
+        dS = f["Gam"][:, None] * dSn + f["Qg"].T @ dO - f["W"].T @ dU
+        f["dSn"], f["dU"] = dSn, dU
+    out["d_initial"] = dS
+    # chunk-parallel gradients
+    for f in fw:
+        sl, K, Q, V, b, E, S = f["sl"], f["K"], f["Q"], f["V"], f["b"], f["E"], f["S"]
+        ii, jj, T, U, dU, dSn = f["ii"], f["jj"], f["T"], f["U"], f["dU"], f["dSn"]
+        dO = d_o[sl]
+        dQg = dO @ S.T
+        dP = (dO @ U.T) * (ii >= jj)
+        dKh = U @ dSn.T
+        dGam = (dSn * S).sum(1)
+        dW = -dU @ S.T
+        TdU, TdW = T.T @ dU, T.T @ dW
+        dV = b[:, None] * TdU
+        dKg = b[:, None] * TdW
+        dbeta = (TdU * V).sum(1) + (TdW * f["Kg"]).sum(1)
+        dT = dU @ (b[:, None] * V).T + dW @ (b[:, None] * f["Kg"]).T
+        dZ = -T.T @ dT @ T.T
+        dA = b[:, None] * dZ * (ii > jj)
+        dbeta += (dZ * f["A"] * (ii > jj)).sum(1)
+        a1 = np.einsum("ts,sc,tsc->tc", dA, K, E)      # sum_{s<t} dA_ts k_s e^{G_t - G_s}
+        a2 = np.einsum("ts,tc,tsc->sc", dA, K, E)      # sum_{t>s} dA_ts k_t e^{G_t - G_s}
+        p1 = np.einsum("ts,sc,tsc->tc", dP, K, E)      # sum_{s<=t} dP_ts k_s e^{G_t - G_s}
+        p2 = np.einsum("ts,tc,tsc->sc", dP, Q, E)      # sum_{t>=s} dP_ts q_t e^{G_t - G_s}
+        gam, Gam, Kh = f["gam"], f["Gam"], f["Kh"]
+        dQ = p1 + dQg * gam
+        dK = a1 + a2 + p2 + dKg * gam + dKh * (Gam[None, :] / gam)
+        dG = K * a1 - K * a2 + Q * p1 - K * p2 + dQg * f["Qg"] + dKg * f["Kg"] - dKh * Kh
+        dG[-1] += (dKh * Kh).sum(0) + dGam * Gam
+        out["dq"][sl], out["dk"][sl], out["dv"][sl] = dQ, dK, dV
+        out["dg"][sl] = np.cumsum(dG[::-1], axis=0)[::-1]
+        out["dbeta"][sl] = dbeta
+    return out
+
+
 def read_golden(name):
     """Parse a fixture: header keys dk/dv/s0, then 'token <inputs> | <S_t> <o_t>'."""
     dk = dv = None
@@ -477,9 +563,34 @@ def pin_backward_dq_is_state_times_cotangent(lib):
                                        rtol=1e-12, atol=1e-13)
 
 
+def pin_backward_chunked_form(lib):
+    """The oracle's backward equals the reverse mode of the chunked form at chunk
+    sizes 1, 16, 64 and the whole sequence, strong and weak decay."""
+    for gate_lo in (-5.0, -0.05):
+        L, H, dk, dv = 150, 2, 8, 6
+        x = rand_inputs([L], H, dk, dv, seed=81, s0_std=0.3, gate_lo=gate_lo)
+        rng = _rng(82)
+        d_o = rng.standard_normal(x["v"].shape)
+        d_fin = rng.standard_normal(x["s0"].shape)
+        r = _backward(lib, x, d_o, d_fin)
+        for C in (1, 16, 64, L):
+            for h in range(H):
+                c = chunked_backward_chain(x["q"][:, h], x["k"][:, h], x["v"][:, h],
+                                           x["g"][:, h], x["beta"][:, h], x["s0"][0, h],
+                                           d_o[:, h], d_fin[0, h], C)
+                for name in ("dq", "dk", "dv", "dg", "dbeta"):
+                    ref = r[name][:, h]
+                    np.testing.assert_allclose(c[name], ref, rtol=0,
+                                               atol=1e-9 * max(1.0, np.abs(ref).max()),
+                                               err_msg=f"{name} C={C} gate_lo={gate_lo}")
+                np.testing.assert_allclose(c["d_initial"], r["d_initial"][0, h], rtol=0,
+                                           atol=1e-9 * max(1.0, np.abs(r["d_initial"]).max()))
+
+
 ALL_PINS = [pin_identity_beta0, pin_orthonormal_retrieval, pin_self_query,
             pin_decay_closed_form, pin_golden_fixtures, pin_brute_force, pin_chunked_form,
             pin_split_combine, pin_snapshot_tagging, pin_contraction_bound, pin_resume,
             pin_decode_matches_prefill, pin_decode_slots, pin_varlen_isolation,
             pin_backward_finite_differences, pin_backward_across_blocks,
-            pin_backward_beta0_closed_form, pin_backward_dq_is_state_times_cotangent]
+            pin_backward_beta0_closed_form, pin_backward_dq_is_state_times_cotangent,
+            pin_backward_chunked_form]
