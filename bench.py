@@ -358,7 +358,7 @@ def run_ours(args, world, rank, local):
         line["decode"] = bench_decode(args, dev, peaks, peak_kind, rank)
     if not args.no_extra:
         line["single_seq"] = bench_single_seq(args, dev, peaks)
-        line["kcp_million"] = bench_kcp_million(args, dev, peaks)
+        line["kcp_million"] = bench_kcp_million(args, dev, peaks, world, rank)
     if not args.no_e2e:
         line["e2e"] = bench_e2e(args, inp, dev, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -465,35 +465,53 @@ def bench_single_seq(args, dev, peaks):
                          "frac": b / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}}
 
 
-def bench_kcp_million(args, dev, peaks):
+def bench_kcp_million(args, dev, peaks, world, rank):
     """B=1, H=16, T=1,048,576, d=128: 16 segments of 65,536 tokens through local
-    states + transitions, the exact combine, and the segment-wise prefill with
-    snapshots every 512 tokens; the unsplit single-chain-per-head run is timed once
-    beside it."""
+    states + transitions, the one exchange of (S_loc, M), the exact combine, and
+    the segment-wise prefill with snapshots every 512 tokens.  With N ranks each
+    holds a contiguous slice of whole segments and the exchange is one NCCL
+    all-gather (total work fixed: strong scaling, time = max over ranks).  On one
+    GPU the unsplit single-chain-per-head run is timed once beside it."""
     import torch
 
-    import decode_kda_chunked_b200 as kda
+    from decode_kda_chunked_b200 import context_parallel as cp
     from decode_kda_chunked_b200 import inputs as I
+    seg = 65536
     x = I.million(device=dev)
     T, H, d = x.total_tokens, 16, 128
+    n_seg = T // seg
+    per = [n_seg // world + (1 if r < n_seg % world else 0) for r in range(world)]
+    rank_tokens = [n * seg for n in per]
+    lo = sum(rank_tokens[:rank])
+    sl = slice(lo, lo + rank_tokens[rank])
+    mine = [t[sl] for t in (x.q, x.k, x.v, x.g, x.beta)]
     stream = torch.cuda.current_stream(dev)
-    ms = _time_calls(lambda: kda.long_context_prefill(x.q, x.k, x.v, x.g, x.beta, 65536, 512,
-                                                      stream=stream), 1, 2, stream)
-    ms_unsplit = _time_calls(lambda: kda.prefill(x.q, x.k, x.v, x.g, x.beta, x.cu_seqlens,
-                                                 snapshot_stride=512, cu_seqlens_host=[0, T],
-                                                 stream=stream), 0, 1, stream)
+    call = lambda: cp.context_parallel_prefill(*mine, rank_tokens, seg, 512, stream=stream)
+    call()
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(_time_calls(call, 1, 2, stream), world)
+    out = {"workload": "B=1, H=16, T=1,048,576, d=128, bf16; 16 segments x 65,536 tokens: "
+                       "local state + transition, one exchange of (S_loc, M), exact combine, "
+                       "segment prefill with fp32 snapshots every 512 tokens",
+           "value": T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
+           "n_gpus": world, "scaling": "strong",
+           "parallelism": f"context parallel x{world}: segments per rank {per}"}
+    if world == 1:
+        import decode_kda_chunked_b200 as kda
+        ms_unsplit = _time_calls(lambda: kda.prefill(x.q, x.k, x.v, x.g, x.beta, x.cu_seqlens,
+                                                     snapshot_stride=512, cu_seqlens_host=[0, T],
+                                                     stream=stream), 0, 1, stream)
+        out["unsplit_ms"] = ms_unsplit
+        out["speedup_vs_unsplit"] = ms_unsplit / ms
     # two passes over the inputs (pass 1 reads k, v, g, beta twice: state and transition)
     b = (T * H * (2 * (2 * d * 2 + 4 * d + 4))       # pass 1, two CTAs per segment-head
-         + prefill_bytes(T, H, d, d, 16, initial=True, final=True)
+         + prefill_bytes(T, H, d, d, n_seg, initial=True, final=False)
          + (T // 512) * H * d * d * 4)               # snapshots
-    return {"workload": "B=1, H=16, T=1,048,576, d=128, bf16; 16 segments x 65,536 tokens: "
-                        "local state + transition, exact combine, segment prefill with fp32 "
-                        "snapshots every 512 tokens",
-            "value": T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
-            "unsplit_ms": ms_unsplit, "speedup_vs_unsplit": ms_unsplit / ms,
-            "roofline": {"bound": "hbm", "achieved": b / (ms * 1e-3) / 1e9,
-                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": b / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}}
+    out["roofline"] = {"bound": "hbm", "achieved": b / (ms * 1e-3) / 1e9,
+                       "peak": peaks["hbm_gbs"] * world, "unit": "GB/s",
+                       "frac": b / (ms * 1e-3) / 1e9 / (peaks["hbm_gbs"] * world)}
+    return out
 
 
 def bench_e2e(args, inp, dev, world):

@@ -31,11 +31,11 @@ SNAP = ("        if (c->snaps && c->stride > 0 && pos % c->stride == 0) {\n"
         "        }\n")
 
 MUTANTS = {
-    "delta_sign": ("u[j] = beta * (v[j] - u[j]);", "u[j] = beta * (v[j] + u[j]);"),
+    "delta_sign": ("u[j] = beta * (v[j] - u[j]);  /* delta", "u[j] = beta * (v[j] + u[j]);  /* delta"),
     "dropped_decay": ("for (j = 0; j < dv; ++j) row[j] *= a;", "for (j = 0; j < dv; ++j) row[j] *= 1.0;"),
     "half_gate": ("const double a = exp(g[i]);\n        double *row",
                   "const double a = exp(0.5 * g[i]);\n        double *row"),
-    "dropped_beta": ("u[j] = beta * (v[j] - u[j]);", "u[j] = (v[j] - u[j]);"),
+    "dropped_beta": ("u[j] = beta * (v[j] - u[j]);  /* delta", "u[j] = (v[j] - u[j]);  /* delta"),
     "transposed_readout": ("o[j] += row[j] * q[i];", "o[j] += S[(size_t)j * dv + i] * q[j];"),
     "transposed_write": ("row[j] += k[i] * u[j];", "row[j] += k[j % dk] * u[i % dv];"),
     "preupdate_output": (STEP + READ, READ + STEP),
