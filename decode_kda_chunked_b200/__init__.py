@@ -13,15 +13,19 @@ from __future__ import annotations
 import torch
 
 from ._lib import (CHUNK, KdaError, kda_chunk_local_state, kda_decode_step,  # noqa: F401
-                   kda_get_device_status, kda_prefill_chunked, kda_prefill_workspace_size,
+                   kda_get_device_status, kda_prefill_backward,
+                   kda_prefill_backward_workspace_size, kda_prefill_chunked,
+                   kda_prefill_workspace_size, make_backward_args,
                    kda_prefill_uses_tensor_cores, kda_snapshot_count, kda_state_combine,
                    kda_status_string, kda_version, load, make_prefill_args)
 
 __all__ = ["kda_prefill_chunked", "kda_chunk_local_state", "kda_state_combine",
            "kda_decode_step", "kda_snapshot_count", "kda_get_device_status",
            "kda_status_string", "kda_version", "kda_prefill_workspace_size", "KdaError",
-           "kda_prefill_uses_tensor_cores",
-           "prefill", "long_context_prefill", "decode_step", "snapshot_offsets", "load"]
+           "kda_prefill_uses_tensor_cores", "kda_prefill_backward",
+           "kda_prefill_backward_workspace_size",
+           "prefill", "prefill_backward", "long_context_prefill", "decode_step",
+           "snapshot_offsets", "load"]
 
 
 def snapshot_offsets(lengths, stride: int) -> list:
@@ -63,6 +67,27 @@ def prefill(q, k, v, g, beta, cu_seqlens, initial_state=None, snapshot_stride: i
     if snaps is not None:
         snaps = snaps[:offs[-1]]
     return {"o": o, "final_state": fin, "snapshots": snaps, "cu_snapshots": cu_snap}
+
+
+def prefill_backward(q, k, v, g, beta, cu_seqlens, d_o=None, d_final=None, initial_state=None,
+                     want_initial: bool = True, cu_seqlens_host=None, stream=None) -> dict:
+    """Gradients of sum(d_o * o) + sum(d_final * final_state) of ``prefill`` for the
+    same inputs; allocates the fp32 gradients and the workspace.
+
+    Returns dict(dq, dk, dv, dg, dbeta, d_initial)."""
+    T, H, dk = k.shape
+    dv = v.shape[2]
+    dev = k.device
+    cu_host, lengths = _host_lengths(cu_seqlens, cu_seqlens_host)
+    f32 = dict(dtype=torch.float32, device=dev)
+    dq, dk_, dg = (torch.empty((T, H, dk), **f32) for _ in range(3))
+    dv_ = torch.empty((T, H, dv), **f32)
+    db = torch.empty((T, H), **f32)
+    d0 = torch.empty((len(lengths), H, dk, dv), **f32) if want_initial else None
+    kda_prefill_backward(q, k, v, g, beta, cu_seqlens, torch.tensor(cu_host, dtype=torch.int32),
+                         dq, dk_, dv_, dg, db, initial_state=initial_state, d_o=d_o,
+                         d_final=d_final, d_initial=d0, stream=stream)
+    return {"dq": dq, "dk": dk_, "dv": dv_, "dg": dg, "dbeta": db, "d_initial": d0}
 
 
 def long_context_prefill(q, k, v, g, beta, seg_len: int, snapshot_stride: int = 512,

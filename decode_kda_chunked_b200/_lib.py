@@ -48,6 +48,14 @@ class DecodeArgs(ctypes.Structure):
                 ("state", _vp), ("n_slots", _i32), ("slot", _vp), ("o", _vp)]
 
 
+class BackwardArgs(ctypes.Structure):
+    _fields_ = [("n_req", _i32), ("total_tokens", _i32), ("H", _i32), ("dk", _i32), ("dv", _i32),
+                ("in_dtype", ctypes.c_int), ("q", _vp), ("k", _vp), ("v", _vp), ("g", _vp),
+                ("beta", _vp), ("cu_seqlens", _vp), ("cu_seqlens_host", _vp),
+                ("initial_state", _vp), ("d_o", _vp), ("d_final", _vp), ("d_q", _vp),
+                ("d_k", _vp), ("d_v", _vp), ("d_g", _vp), ("d_beta", _vp), ("d_initial", _vp)]
+
+
 class KdaError(RuntimeError):
     def __init__(self, fn: str, code: int):
         super().__init__(f"{fn} returned {STATUS_NAMES.get(code, code)}")
@@ -60,7 +68,8 @@ _lock = threading.Lock()
 EXPORTS = ("kda_prefill_workspace_size", "kda_prefill_chunked", "kda_local_state_workspace_size",
            "kda_chunk_local_state", "kda_state_combine", "kda_decode_step", "kda_snapshot_count",
            "kda_get_device_status", "kda_status_string", "kda_version",
-           "kda_prefill_uses_tensor_cores", "kda_prefill_chunked_noalloc")
+           "kda_prefill_uses_tensor_cores", "kda_prefill_chunked_noalloc",
+           "kda_prefill_backward_workspace_size", "kda_prefill_backward")
 
 
 def load(path: str = LIB_PATH):
@@ -97,6 +106,10 @@ def load(path: str = LIB_PATH):
         lib.kda_version.argtypes = []
         lib.kda_prefill_chunked_noalloc.restype = ctypes.c_int
         lib.kda_prefill_chunked_noalloc.argtypes = [P(PrefillArgs), _vp]
+        lib.kda_prefill_backward_workspace_size.restype = ctypes.c_size_t
+        lib.kda_prefill_backward_workspace_size.argtypes = [P(BackwardArgs)]
+        lib.kda_prefill_backward.restype = ctypes.c_int
+        lib.kda_prefill_backward.argtypes = [P(BackwardArgs), _vp, ctypes.c_size_t, _vp]
         lib.kda_prefill_uses_tensor_cores.restype = _i32
         lib.kda_prefill_uses_tensor_cores.argtypes = [_i32, _i32, ctypes.c_int]
         _lib = lib
@@ -196,6 +209,47 @@ def kda_prefill_chunked(q, k, v, g, beta, cu_seqlens, o, initial_state=None, fin
     _check("kda_prefill_chunked",
            lib.kda_prefill_chunked(ctypes.byref(a), ws_ptr, ws_bytes, _stream(stream)))
     return o
+
+
+def make_backward_args(q, k, v, g, beta, cu_seqlens, cu_seqlens_host, d_q, d_k, d_v, d_g, d_beta,
+                       initial_state=None, d_o=None, d_final=None, d_initial=None):
+    T, H, dk = k.shape
+    a = BackwardArgs()
+    a.n_req = cu_seqlens.numel() - 1
+    a.total_tokens = T
+    a.H, a.dk, a.dv = H, dk, v.shape[2]
+    a.in_dtype = _dtype(k)
+    a.q, a.k, a.v, a.g, a.beta = _ptr(q), _ptr(k), _ptr(v), _ptr(g), _ptr(beta)
+    a.cu_seqlens, a.cu_seqlens_host = _ptr(cu_seqlens), _ptr(cu_seqlens_host)
+    a.initial_state, a.d_o, a.d_final = _ptr(initial_state), _ptr(d_o), _ptr(d_final)
+    a.d_q, a.d_k, a.d_v, a.d_g, a.d_beta = _ptr(d_q), _ptr(d_k), _ptr(d_v), _ptr(d_g), _ptr(d_beta)
+    a.d_initial = _ptr(d_initial)
+    return a
+
+
+def kda_prefill_backward_workspace_size(args: BackwardArgs) -> int:
+    return int(load().kda_prefill_backward_workspace_size(ctypes.byref(args)))
+
+
+def kda_prefill_backward(q, k, v, g, beta, cu_seqlens, cu_seqlens_host, d_q, d_k, d_v, d_g,
+                         d_beta, initial_state=None, d_o=None, d_final=None, d_initial=None,
+                         workspace=None, stream=None):
+    """Gradients of sum(d_o * o) + sum(d_final * final_state) of the prefill into
+    caller-provided fp32 outputs (see include/kda.h).  ``cu_seqlens_host`` (CPU
+    int32) is required; ``workspace`` (uint8 CUDA tensor) is allocated through
+    torch when None."""
+    lib = load()
+    host = _host_i32(cu_seqlens_host)
+    a = make_backward_args(q, k, v, g, beta, cu_seqlens, host, d_q, d_k, d_v, d_g, d_beta,
+                           initial_state, d_o, d_final, d_initial)
+    need = int(lib.kda_prefill_backward_workspace_size(ctypes.byref(a)))
+    if workspace is None and need > 0:
+        workspace = torch.empty(need, dtype=torch.uint8, device=k.device)
+    ws_ptr = _ptr(workspace) if workspace is not None else None
+    ws_bytes = workspace.numel() if workspace is not None else 0
+    _check("kda_prefill_backward",
+           lib.kda_prefill_backward(ctypes.byref(a), ws_ptr, ws_bytes, _stream(stream)))
+    return d_q, d_k, d_v, d_g, d_beta, d_initial
 
 
 def kda_chunk_local_state(k, v, g, beta, seg_cu, s_loc, m, seg_cu_host=None, stream=None):

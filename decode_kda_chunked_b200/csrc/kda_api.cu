@@ -7,6 +7,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <vector>
 
 #include "kda_internal.cuh"
 
@@ -354,4 +355,159 @@ extern "C" kda_status kda_prefill_chunked_noalloc(const kda_prefill_args *args, 
   int32_t *scratch = kda::noalloc_scratch();
   if (!scratch) return KDA_ERR_CUDA;
   return kda_prefill_chunked(args, scratch, sizeof(kda::g_noalloc_order), stream);
+}
+
+// ---------------------------------------------------------------------------
+// Backward of the prefill: argument checks, the chunk table, the forward pass
+// that leaves the chunk-start states in the workspace, then the backward
+// kernels (kda_backward.cu).
+// ---------------------------------------------------------------------------
+
+namespace kda {
+namespace {
+
+struct BwdShape {
+  int n_chunks = 0, n_snap = 0;
+};
+
+kda_status check_backward(const kda_backward_args *a, BwdShape *sh) {
+  if (!a) return KDA_ERR_INVALID_ARG;
+  if (a->n_req < 0 || a->total_tokens < 0 || a->H <= 0 || a->dk <= 0 || a->dv <= 0)
+    return KDA_ERR_INVALID_ARG;
+  if (!valid_dtype(a->in_dtype)) return KDA_ERR_INVALID_ARG;
+  if (!head_dims_supported(a->dk, a->dv)) return KDA_ERR_UNSUPPORTED;
+  *sh = BwdShape{};
+  if (a->n_req == 0) return KDA_OK;
+  if (!a->cu_seqlens || !a->cu_seqlens_host) return KDA_ERR_INVALID_ARG;
+  const int32_t *cu = a->cu_seqlens_host;
+  if (cu[0] != 0 || cu[a->n_req] != a->total_tokens) return KDA_ERR_INVALID_ARG;
+  long long n_chunks = 0, n_snap = 0;
+  for (int r = 0; r < a->n_req; ++r) {
+    const long long len = (long long)cu[r + 1] - cu[r];
+    if (len < 0) return KDA_ERR_INVALID_ARG;
+    n_chunks += (len + KDA_CHUNK - 1) / KDA_CHUNK;
+    n_snap += len / KDA_CHUNK;
+  }
+  if (n_chunks * a->H > 0x7fffffffLL || (long long)a->n_req * a->H > 0x7fffffffLL)
+    return KDA_ERR_UNSUPPORTED;
+  if (a->total_tokens > 0 && (!a->q || !a->k || !a->v || !a->g || !a->beta || !a->d_q ||
+                              !a->d_k || !a->d_v || !a->d_g || !a->d_beta))
+    return KDA_ERR_INVALID_ARG;
+  const void *ptrs[] = {a->q, a->k, a->v, a->g, a->beta, a->cu_seqlens, a->initial_state,
+                        a->d_o, a->d_final, a->d_q, a->d_k, a->d_v, a->d_g, a->d_beta,
+                        a->d_initial};
+  for (const void *p : ptrs)
+    if (p && !aligned16(p)) return KDA_ERR_INVALID_ARG;
+  const size_t T = (size_t)a->total_tokens, H = (size_t)a->H, dk = (size_t)a->dk,
+               dv = (size_t)a->dv, n = (size_t)a->n_req;
+  Range ins[] = {span(a->q, T * H * dk * dsize(a->in_dtype)),
+                 span(a->k, T * H * dk * dsize(a->in_dtype)),
+                 span(a->v, T * H * dv * dsize(a->in_dtype)), span(a->g, T * H * dk * 4),
+                 span(a->beta, T * H * 4), span(a->cu_seqlens, (n + 1) * 4),
+                 span(a->initial_state, n * H * dk * dv * 4), span(a->d_o, T * H * dv * 4),
+                 span(a->d_final, n * H * dk * dv * 4)};
+  Range outs[] = {span(a->d_q, T * H * dk * 4), span(a->d_k, T * H * dk * 4),
+                  span(a->d_v, T * H * dv * 4), span(a->d_g, T * H * dk * 4),
+                  span(a->d_beta, T * H * 4), span(a->d_initial, n * H * dk * dv * 4)};
+  for (size_t i = 0; i < sizeof(outs) / sizeof(outs[0]); ++i) {
+    for (Range in : ins)
+      if (overlap(outs[i], in)) return KDA_ERR_INVALID_ARG;
+    for (size_t j = i + 1; j < sizeof(outs) / sizeof(outs[0]); ++j)
+      if (overlap(outs[i], outs[j])) return KDA_ERR_INVALID_ARG;
+  }
+  sh->n_chunks = (int)n_chunks;
+  sh->n_snap = (int)n_snap;
+  return KDA_OK;
+}
+
+}  // namespace
+}  // namespace kda
+
+extern "C" size_t kda_prefill_backward_workspace_size(const kda_backward_args *a) {
+  kda::BwdShape sh;
+  if (kda::check_backward(a, &sh) != KDA_OK || a->n_req == 0) return 0;
+  return kda::backward_workspace_bytes(a->n_req, sh.n_chunks, sh.n_snap, a->H, a->dk);
+}
+
+extern "C" kda_status kda_prefill_backward(const kda_backward_args *a, void *workspace,
+                                           size_t workspace_bytes, void *stream) {
+  using namespace kda;
+  BwdShape sh;
+  kda_status st = check_backward(a, &sh);
+  if (st != KDA_OK) return st;
+  if (a->n_req == 0) return KDA_OK;
+  const int D = a->dk, H = a->H, n_req = a->n_req;
+  const size_t need = backward_workspace_bytes(n_req, sh.n_chunks, sh.n_snap, H, D);
+  if (!workspace || workspace_bytes < need || (reinterpret_cast<uintptr_t>(workspace) & 255u))
+    return KDA_ERR_WORKSPACE;
+  {  // outputs must not overlap the workspace
+    const size_t T = (size_t)a->total_tokens, n = (size_t)n_req;
+    Range ws = span(workspace, need);
+    Range outs[] = {span(a->d_q, T * H * D * 4), span(a->d_k, T * H * D * 4),
+                    span(a->d_v, T * H * D * 4), span(a->d_g, T * H * D * 4),
+                    span(a->d_beta, T * H * 4), span(a->d_initial, n * H * D * D * 4)};
+    for (Range o : outs)
+      if (overlap(o, ws)) return KDA_ERR_INVALID_ARG;
+  }
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  size_t o_chunks, o_cu_chunks, o_cu_snap, o_snaps, o_zero;
+  backward_offsets(n_req, sh.n_chunks, sh.n_snap, H, D, &o_chunks, &o_cu_chunks, &o_cu_snap,
+                   &o_snaps, &o_zero);
+  char *ws = static_cast<char *>(workspace);
+
+  // chunk table (request, chunk index, first token, rows), chunk and snapshot offsets
+  std::vector<unsigned char> host(o_snaps, 0);
+  int32_t *chunks = reinterpret_cast<int32_t *>(host.data() + o_chunks);
+  int32_t *cu_chunks = reinterpret_cast<int32_t *>(host.data() + o_cu_chunks);
+  int32_t *cu_snap = reinterpret_cast<int32_t *>(host.data() + o_cu_snap);
+  const int32_t *cu = a->cu_seqlens_host;
+  int jc = 0;
+  cu_chunks[0] = 0;
+  cu_snap[0] = 0;
+  for (int r = 0; r < n_req; ++r) {
+    const int len = cu[r + 1] - cu[r];
+    for (int c = 0; c * KDA_CHUNK < len; ++c, ++jc) {
+      chunks[4 * jc + 0] = r;
+      chunks[4 * jc + 1] = c;
+      chunks[4 * jc + 2] = cu[r] + c * KDA_CHUNK;
+      chunks[4 * jc + 3] = len - c * KDA_CHUNK < KDA_CHUNK ? len - c * KDA_CHUNK : KDA_CHUNK;
+    }
+    cu_chunks[r + 1] = jc;
+    cu_snap[r + 1] = cu_snap[r] + len / KDA_CHUNK;
+  }
+  cudaError_t e = cudaMemcpyAsync(ws, host.data(), o_snaps, cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess) e = cudaMemsetAsync(ws + o_zero, 0, (size_t)D * D * sizeof(float), s);
+  if (e != cudaSuccess) return from_cuda(e);
+
+  // forward pass: the state at every 64-token boundary is a chunk's start state
+  if (sh.n_chunks > 0) {
+    PrefillParams p{};
+    p.q = a->q; p.k = a->k; p.v = a->v; p.g = a->g; p.beta = a->beta;
+    p.cu_seqlens = a->cu_seqlens;
+    p.initial_state = a->initial_state;
+    p.cu_snapshots = reinterpret_cast<const int32_t *>(ws + o_cu_snap);
+    p.snapshots = reinterpret_cast<float *>(ws + o_snaps);
+    p.n_req = n_req; p.total_tokens = a->total_tokens;
+    p.H = H; p.dk = D; p.dv = D;
+    p.snapshot_stride = KDA_CHUNK;
+    p.validate = env_flag("KDA_VALIDATE");
+    p.status = device_status_word();
+    if (!p.status) return KDA_ERR_CUDA;
+    if (prefill_tc_supported(D, D, a->in_dtype) && !env_flag("KDA_FORCE_SIMT")) {
+      e = launch_prefill_tc(p, a->in_dtype, KDA_F32, s);
+    } else {
+      p.n_slices = prefill_simt_slices(D, D, false);
+      e = launch_prefill_simt(p, a->in_dtype, KDA_F32, s);
+    }
+    if (e != cudaSuccess) return from_cuda(e);
+  }
+  BackwardLaunch b{};
+  b.q = a->q; b.k = a->k; b.v = a->v; b.g = a->g; b.beta = a->beta;
+  b.initial_state = a->initial_state; b.d_o = a->d_o; b.d_final = a->d_final;
+  b.dq = a->d_q; b.dk = a->d_k; b.dv = a->d_v; b.dg = a->d_g; b.dbeta = a->d_beta;
+  b.d_initial = a->d_initial;
+  b.workspace = workspace;
+  b.n_req = n_req; b.n_chunks = sh.n_chunks; b.n_snap = sh.n_snap; b.H = H; b.D = D;
+  b.in_dtype = a->in_dtype;
+  return from_cuda(launch_backward(b, s));
 }

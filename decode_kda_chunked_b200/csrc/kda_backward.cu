@@ -1,0 +1,815 @@
+// KDA backward (training) on sm_100a: gradients of the chunked prefill.
+//
+// FlashKDA also speeds up training ("Kimi K3 开源日来了", FlashKDA section), so
+// the path carries the derivative of the prefill map: given cotangents dO of o
+// and dS_L of the final state, the gradients of q, k, v, g (= log alpha),
+// beta and the initial state.
+//
+// Reverse mode through the forward's chunk algebra (one chain; chunk start
+// state S, chunk-end cotangent dSn, G the chunk-local cumsum of g,
+// gamma = exp(G), Gam = gamma at the chunk's last row, Khat = (Gam/gamma) K,
+// [U~ | W] = T Diag(beta) [V | gamma K], U = U~ - W S, T = (I + Diag(beta) A)^-1):
+//
+//   serial over chunks, last to first:
+//     dU = P^T dO + Khat dSn
+//     dS = Diag(Gam) dSn + (gamma Q)^T dO - W^T dU
+//   per chunk, all chunks in parallel:
+//     d(gamma Q) = dO S^T      dP = tril(dO U^T)      dKhat = U dSn^T      dW = -dU S^T
+//     dV = Diag(beta) T^T dU   d(gamma K) = Diag(beta) T^T dW
+//     dT = dU (Diag(beta) V)^T + dW (Diag(beta) gamma K)^T
+//     dZ = -T^T dT T^T         dA = tril_strict(Diag(beta) dZ)
+//     dbeta_t = (T^T dU)_t . v_t + (T^T dW)_t . (gamma k)_t + sum_s dZ_ts A_ts
+//     A and P are gated Gram products; their cotangents reach K, Q and the
+//     cumulative gate through sums  sum_s M_ts x_s exp(G_t - G_s)  (t >= s),
+//     each taken with the 16-row block factorisation
+//     exp(G_t - G_s) = exp(G_t - G_r) exp(G_r - G_s), r a block boundary, so
+//     every factor is a finite fp32 number (log alpha >= -5, the lower-bounded
+//     decay of KDA, CSDN post on the Kimi K3 technical report, section 一.1).
+//     dg = reverse cumulative sum of dG over the chunk.
+//
+// Launches: the forward kernel with a snapshot every 64 tokens (the chunk
+// start states), then
+//   bwd_prep  (CTA per chunk and head): A, T, W, U~, Khat, Gam, X = P^T dO, Y = (gamma Q)^T dO
+//   bwd_state (CTA per request and head): the serial pass; dU overwrites X, dSn overwrites Y
+//   bwd_grad  (CTA per chunk and head): every token gradient of the chunk
+// All backward arithmetic is fp32 on the CUDA cores.  A CTA's 256 threads
+// form a 16 x 16 grid; thread (ty, tx) owns rows ty + 16 i and columns
+// tx + 16 j of every tile it produces, so per-element folds stay in registers.
+#include "kda_internal.cuh"
+
+namespace kda {
+
+namespace {
+
+constexpr int NTH = 256;
+constexpr int C = kChunk;  // 64
+constexpr float LOG2E = 1.4426950408889634f;
+
+struct BwdParams {
+  const void *q, *k, *v;
+  const float *g, *beta;
+  const float *initial_state;  // NULL = zeros
+  const float *d_o;            // NULL = zeros
+  const float *d_final;        // NULL = zeros
+  float *dq, *dk, *dv, *dg, *dbeta;
+  float *d_initial;            // NULL = not returned
+  const int4 *chunks;          // per chunk: request, chunk index in the request, first token, rows
+  const int32_t *cu_chunks;    // [n_req + 1]
+  const int32_t *cu_snap;      // [n_req + 1]: chunk-start snapshots of the forward pass
+  const float *snaps;          // [n_snap, H, D, D]
+  const float *zero_state;     // D x D zeros
+  float *wA, *wT, *wW, *wU, *wKh, *wX, *wY, *wGam;
+  int n_req, n_chunks, H;
+};
+
+// acc[i][j] += sum_k A(m_i, k) B(k, n_j) for k < K (a multiple of 16), where
+// the calling thread's rows are m_i = ty + 16 i and columns n_j = tx + 16 j;
+// A(m, k) = A[m am + k ak], B(k, n) = B[k bk + n bn], in any memory space.
+// Slices of 16 along k are staged through shared memory `stage`
+// (16 (16 MI + 1) + 16 (16 NJ + 1) floats) so the inner loop reads
+// conflict-free shared memory.  Every thread of the CTA must call it.
+template <int MI, int NJ>
+__device__ void mm_acc(float (&acc)[MI][NJ], const float *A, int am, int ak, const float *B,
+                       int bk, int bn, int K, float *stage) {
+  constexpr int M = 16 * MI, N = 16 * NJ, LA = M + 1, LB = N + 1;
+  float *As = stage, *Bs = stage + 16 * LA;
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  for (int k0 = 0; k0 < K; k0 += 16) {
+    __syncthreads();
+    if (ak == 1) {
+      for (int e = tid; e < 16 * M; e += NTH) {
+        const int kk = e & 15, m = e >> 4;
+        As[kk * LA + m] = A[(size_t)m * am + k0 + kk];
+      }
+    } else {
+      for (int e = tid; e < 16 * M; e += NTH) {
+        const int m = e % M, kk = e / M;
+        As[kk * LA + m] = A[(size_t)m * am + (size_t)(k0 + kk) * ak];
+      }
+    }
+    if (bn == 1) {
+      for (int e = tid; e < 16 * N; e += NTH) {
+        const int n = e % N, kk = e / N;
+        Bs[kk * LB + n] = B[(size_t)(k0 + kk) * bk + n];
+      }
+    } else {
+      for (int e = tid; e < 16 * N; e += NTH) {
+        const int kk = e & 15, n = e >> 4;
+        Bs[kk * LB + n] = B[(size_t)(k0 + kk) * bk + (size_t)n * bn];
+      }
+    }
+    __syncthreads();
+#pragma unroll 4
+    for (int kk = 0; kk < 16; ++kk) {
+      float a[MI], b[NJ];
+#pragma unroll
+      for (int i = 0; i < MI; ++i) a[i] = As[kk * LA + ty + 16 * i];
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) b[j] = Bs[kk * LB + tx + 16 * j];
+#pragma unroll
+      for (int i = 0; i < MI; ++i)
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) acc[i][j] = fmaf(a[i], b[j], acc[i][j]);
+    }
+  }
+  __syncthreads();
+}
+
+template <int MI, int NJ>
+__device__ __forceinline__ void zero(float (&acc)[MI][NJ]) {
+#pragma unroll
+  for (int i = 0; i < MI; ++i)
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) acc[i][j] = 0.f;
+}
+
+constexpr int stage_floats(int M, int N) { return 16 * (M + 1) + 16 * (N + 1); }
+
+// Rows tok0 .. tok0 + n - 1 of a token-major [T, H, D] tensor into a [64][ld]
+// fp32 tile (rows >= n are zero: the exact no-op padding of the chunk form).
+template <int D, typename TIn>
+__device__ void stage_rows(float *dst, int ld, const TIn *src, int tok0, int n, int H, int h) {
+  for (int e = threadIdx.x; e < C * D; e += NTH) {
+    const int t = e / D, c = e % D;
+    dst[t * ld + c] = (src && t < n) ? load_elem(src, ((size_t)(tok0 + t) * H + h) * D + c) : 0.f;
+  }
+}
+
+// g rows into sG, then the in-place chunk-local cumsum scaled by log2(e)
+// (thread = channel); beta into sB.  Padded rows have g = 0 and beta = 0.
+template <int D>
+__device__ void stage_gate(float *sG, float *sB, const BwdParams &p, int tok0, int n, int h) {
+  stage_rows<D, float>(sG, D, p.g, tok0, n, p.H, h);
+  if (threadIdx.x < C)
+    sB[threadIdx.x] = threadIdx.x < n ? p.beta[(size_t)(tok0 + threadIdx.x) * p.H + h] : 0.f;
+  __syncthreads();
+  if (threadIdx.x < D) {
+    const int c = threadIdx.x;
+    float run = 0.f;
+    for (int t = 0; t < C; ++t) {
+      run += sG[t * D + c];
+      sG[t * D + c] = run * LOG2E;
+    }
+  }
+  __syncthreads();
+}
+
+// Sum over the 16 lanes that share a row (lanes tx = 0..15 of one half-warp).
+__device__ __forceinline__ float row_sum16(float x) {
+#pragma unroll
+  for (int off = 8; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+  return x;
+}
+
+// ---------------------------------------------------------------------------
+// bwd_prep: the state-independent chunk quantities
+// ---------------------------------------------------------------------------
+template <int D>
+struct PrepLayout {
+  static constexpr int LDP = D + 1;
+  static constexpr int oK = 0, oQ = oK + C * D, oG = oQ + C * D, oA = oG + C * D;
+  static constexpr int oP = oA + C * C, oT = oP + C * C, oBuf = oT + C * C;
+  static constexpr int oKL = oBuf + C * LDP, oQL = oKL + 16 * LDP, oStage = oQL + 16 * LDP;
+  static constexpr int oB = oStage + stage_floats(D, D);
+  static constexpr int total = oB + C;
+  static constexpr size_t bytes = sizeof(float) * total;
+};
+
+template <int D, typename TIn>
+__global__ void __launch_bounds__(NTH, 1) bwd_prep_kernel(const BwdParams p) {
+  using L = PrepLayout<D>;
+  constexpr int NJ = D / 16, LDP = L::LDP;
+  extern __shared__ float4 smem_f4[];
+  float *sm = reinterpret_cast<float *>(smem_f4);
+  float *sK = sm + L::oK, *sQ = sm + L::oQ, *sG = sm + L::oG, *sA = sm + L::oA;
+  float *sP = sm + L::oP, *sT = sm + L::oT, *sBuf = sm + L::oBuf, *sKL = sm + L::oKL;
+  float *sQL = sm + L::oQL, *sStage = sm + L::oStage, *sB = sm + L::oB;
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  const int H = p.H;
+  const int jc = blockIdx.x / H, h = blockIdx.x % H;
+  const int4 cd = p.chunks[jc];
+  const int tok0 = cd.z, n = cd.w;
+  const size_t ch = (size_t)jc * H + h;
+
+  stage_rows<D, TIn>(sK, D, static_cast<const TIn *>(p.k), tok0, n, H, h);
+  stage_rows<D, TIn>(sQ, D, static_cast<const TIn *>(p.q), tok0, n, H, h);
+  stage_gate<D>(sG, sB, p, tok0, n, h);
+
+  // A (strict lower) and P (inclusive lower), row block b at a time:
+  // A_ts = sum_c [k_tc exp(G_tc - G_rc)] [k_sc exp(G_rc - G_sc)], r = 16 b.
+  for (int b = 0; b < 4; ++b) {
+    const int r0 = 16 * b, rows = r0 + 16;
+    __syncthreads();
+    for (int e = tid; e < rows * D; e += NTH) {
+      const int s = e / D, c = e % D;
+      sBuf[s * LDP + c] = sK[s * D + c] * exp2f(sG[r0 * D + c] - sG[s * D + c]);
+    }
+    for (int e = tid; e < 16 * D; e += NTH) {
+      const int t = e / D, c = e % D;
+      const float f = exp2f(sG[(r0 + t) * D + c] - sG[r0 * D + c]);
+      sKL[t * LDP + c] = sK[(r0 + t) * D + c] * f;
+      sQL[t * LDP + c] = sQ[(r0 + t) * D + c] * f;
+    }
+    __syncthreads();
+    float a[4] = {0.f, 0.f, 0.f, 0.f}, pp[4] = {0.f, 0.f, 0.f, 0.f};
+    for (int c = 0; c < D; ++c) {
+      const float kl = sKL[ty * LDP + c], ql = sQL[ty * LDP + c];
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        const int s = tx + 16 * jj;
+        if (s < rows) {
+          const float tv = sBuf[s * LDP + c];
+          a[jj] = fmaf(kl, tv, a[jj]);
+          pp[jj] = fmaf(ql, tv, pp[jj]);
+        }
+      }
+    }
+    const int t = r0 + ty;
+#pragma unroll
+    for (int jj = 0; jj < 4; ++jj) {
+      const int s = tx + 16 * jj;
+      sA[t * C + s] = s < t ? a[jj] : 0.f;
+      sP[t * C + s] = s <= t ? pp[jj] : 0.f;
+    }
+  }
+  __syncthreads();
+
+  // T = (I + Diag(beta) A)^-1 by forward substitution, one column per thread
+  if (tid < C) {
+    const int j = tid;
+    for (int i = 0; i < C; ++i) {
+      float tv;
+      if (i < j) {
+        tv = 0.f;
+      } else if (i == j) {
+        tv = 1.f;
+      } else {
+        float acc = 0.f;
+        for (int s = j; s < i; ++s) acc = fmaf(sA[i * C + s], sT[s * C + j], acc);
+        tv = -sB[i] * acc;
+      }
+      sT[i * C + j] = tv;
+    }
+  }
+  __syncthreads();
+
+  float acc[4][NJ];
+  // W = T Diag(beta) (gamma K)
+  for (int e = tid; e < C * D; e += NTH) {
+    const int t = e / D, c = e % D;
+    sBuf[t * LDP + c] = sB[t] * exp2f(sG[t * D + c]) * sK[t * D + c];
+  }
+  zero(acc);
+  mm_acc<4, NJ>(acc, sT, C, 1, sBuf, LDP, 1, C, sStage);
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) p.wW[ch * C * D + (ty + 16 * i) * D + tx + 16 * j] = acc[i][j];
+  // U~ = T Diag(beta) V
+  stage_rows<D, TIn>(sBuf, LDP, static_cast<const TIn *>(p.v), tok0, n, H, h);
+  __syncthreads();
+  for (int e = tid; e < C * D; e += NTH) sBuf[(e / D) * LDP + e % D] *= sB[e / D];
+  zero(acc);
+  mm_acc<4, NJ>(acc, sT, C, 1, sBuf, LDP, 1, C, sStage);
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) p.wU[ch * C * D + (ty + 16 * i) * D + tx + 16 * j] = acc[i][j];
+  // X = P^T dO
+  stage_rows<D, float>(sBuf, LDP, p.d_o, tok0, n, H, h);
+  zero(acc);
+  mm_acc<4, NJ>(acc, sP, 1, C, sBuf, LDP, 1, C, sStage);
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) p.wX[ch * C * D + (ty + 16 * i) * D + tx + 16 * j] = acc[i][j];
+  // Y = (gamma Q)^T dO
+  for (int e = tid; e < C * D; e += NTH) sQ[e] *= exp2f(sG[e]);
+  {
+    float y[NJ][NJ];
+    zero(y);
+    mm_acc<NJ, NJ>(y, sQ, 1, D, sBuf, LDP, 1, C, sStage);
+#pragma unroll
+    for (int i = 0; i < NJ; ++i)
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) p.wY[ch * D * D + (ty + 16 * i) * D + tx + 16 * j] = y[i][j];
+  }
+  // Khat = exp(G_last - G) K, Gam = exp(G_last); A and T for the gradient pass
+  for (int e = tid; e < C * D; e += NTH) {
+    const int t = e / D, c = e % D;
+    p.wKh[ch * C * D + e] = sK[e] * exp2f(sG[(C - 1) * D + c] - sG[t * D + c]);
+  }
+  if (tid < D) p.wGam[ch * D + tid] = exp2f(sG[(C - 1) * D + tid]);
+  for (int e = tid; e < C * C; e += NTH) {
+    p.wA[ch * C * C + e] = sA[e];
+    p.wT[ch * C * C + e] = sT[e];
+  }
+}
+
+// ---------------------------------------------------------------------------
+// bwd_state: the serial pass over chunk-end cotangents, last chunk first
+// ---------------------------------------------------------------------------
+template <int D>
+struct StateLayout {
+  static constexpr int oS = 0, oU = oS + D * D, oStage = oU + C * D;
+  static constexpr int total = oStage + stage_floats(D, D);
+  static constexpr size_t bytes = sizeof(float) * total;
+};
+
+template <int D>
+__global__ void __launch_bounds__(NTH, 1) bwd_state_kernel(const BwdParams p) {
+  using L = StateLayout<D>;
+  constexpr int NJ = D / 16;
+  extern __shared__ float4 smem_f4[];
+  float *sm = reinterpret_cast<float *>(smem_f4);
+  float *sdS = sm + L::oS, *sdU = sm + L::oU, *sStage = sm + L::oStage;
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  const int H = p.H;
+  const int r = blockIdx.x / H, h = blockIdx.x % H;
+  const float *dfin = p.d_final ? p.d_final + ((size_t)r * H + h) * D * D : nullptr;
+  for (int e = tid; e < D * D; e += NTH) sdS[e] = dfin ? dfin[e] : 0.f;
+
+  for (int jc = p.cu_chunks[r + 1] - 1; jc >= p.cu_chunks[r]; --jc) {
+    const size_t ch = (size_t)jc * H + h;
+    // dU = X + Khat dSn  (overwrites X)
+    float u[4][NJ];
+    zero(u);
+    mm_acc<4, NJ>(u, p.wKh + ch * C * D, D, 1, sdS, D, 1, D, sStage);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) {
+        const int e = (ty + 16 * i) * D + tx + 16 * j;
+        const float x = p.wX[ch * C * D + e] + u[i][j];
+        p.wX[ch * C * D + e] = x;
+        sdU[e] = x;
+      }
+    // dS = Diag(Gam) dSn + Y - W^T dU;  dSn overwrites Y for the gradient pass
+    float s[NJ][NJ];
+    zero(s);
+    mm_acc<NJ, NJ>(s, p.wW + ch * C * D, 1, D, sdU, D, 1, C, sStage);
+#pragma unroll
+    for (int i = 0; i < NJ; ++i) {
+      const float gam = p.wGam[ch * D + ty + 16 * i];
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) {
+        const int e = (ty + 16 * i) * D + tx + 16 * j;
+        const float old = sdS[e];
+        s[i][j] = fmaf(gam, old, p.wY[ch * D * D + e] - s[i][j]);
+        p.wY[ch * D * D + e] = old;
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int i = 0; i < NJ; ++i)
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) sdS[(ty + 16 * i) * D + tx + 16 * j] = s[i][j];
+  }
+  __syncthreads();
+  if (p.d_initial) {
+    float *dst = p.d_initial + ((size_t)r * H + h) * D * D;
+    for (int e = tid; e < D * D; e += NTH) dst[e] = sdS[e];
+  }
+}
+
+// ---------------------------------------------------------------------------
+// bwd_grad: every token gradient of one chunk
+// ---------------------------------------------------------------------------
+template <int D>
+struct GradLayout {
+  static constexpr int oK = 0, oQ = oK + C * D, oV = oQ + C * D, oO = oV + C * D;
+  static constexpr int oG = oO + C * D, oP = oG + C * D, oT = oP + C * C;
+  static constexpr int oStage = oT + C * C, oB = oStage + stage_floats(C, D);
+  static constexpr int oDb = oB + C, oX = oDb + C, oPart = oX + D;
+  static constexpr int total = oPart + 16 * D;
+  static constexpr size_t bytes = sizeof(float) * total;
+};
+
+template <int D, typename TIn>
+__global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
+  using L = GradLayout<D>;
+  constexpr int NJ = D / 16;
+  extern __shared__ float4 smem_f4[];
+  float *sm = reinterpret_cast<float *>(smem_f4);
+  float *sK = sm + L::oK, *sQ = sm + L::oQ, *sV = sm + L::oV, *sO = sm + L::oO;
+  float *sG = sm + L::oG, *sP = sm + L::oP, *sT = sm + L::oT, *sStage = sm + L::oStage;
+  float *sB = sm + L::oB, *sDb = sm + L::oDb, *sExtra = sm + L::oX, *sPart = sm + L::oPart;
+  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  const int H = p.H;
+  const int jc = blockIdx.x / H, h = blockIdx.x % H;
+  const int4 cd = p.chunks[jc];
+  const int r = cd.x, cidx = cd.y, tok0 = cd.z, n = cd.w;
+  const size_t ch = (size_t)jc * H + h;
+  const float *S;
+  if (cidx == 0)
+    S = p.initial_state ? p.initial_state + ((size_t)r * H + h) * D * D : p.zero_state;
+  else
+    S = p.snaps + ((size_t)(p.cu_snap[r] + cidx - 1) * H + h) * D * D;
+  const float *dSn = p.wY + ch * D * D;
+  const float *dU = p.wX + ch * C * D;
+  const float *W = p.wW + ch * C * D;
+  float *U = p.wU + ch * C * D;
+
+  stage_rows<D, TIn>(sK, D, static_cast<const TIn *>(p.k), tok0, n, H, h);
+  stage_rows<D, TIn>(sQ, D, static_cast<const TIn *>(p.q), tok0, n, H, h);
+  stage_rows<D, TIn>(sV, D, static_cast<const TIn *>(p.v), tok0, n, H, h);
+  stage_rows<D, float>(sO, D, p.d_o, tok0, n, H, h);
+  if (tid < C) sDb[tid] = 0.f;
+  stage_gate<D>(sG, sB, p, tok0, n, h);
+
+  // the thread's elements: rows ty + 16 i, columns tx + 16 j
+  float accQ[4][NJ], accK[4][NJ], accG[4][NJ], acc[4][NJ];
+  const float *G63 = sG + (C - 1) * D;
+
+  // U = U~ - W S (in place)
+  zero(acc);
+  mm_acc<4, NJ>(acc, W, D, 1, S, D, 1, D, sStage);
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) {
+      const int e = (ty + 16 * i) * D + tx + 16 * j;
+      U[e] = U[e] - acc[i][j];
+    }
+  // d(gamma Q) = dO S^T  ->  dQ = d(gamma Q) gamma,  dG = d(gamma Q) gamma q
+  zero(acc);
+  mm_acc<4, NJ>(acc, sO, D, 1, S, 1, D, D, sStage);
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) {
+      const int e = (ty + 16 * i) * D + tx + 16 * j;
+      const float gq = acc[i][j] * exp2f(sG[e]);
+      accQ[i][j] = gq;
+      accG[i][j] = gq * sQ[e];
+      accK[i][j] = 0.f;
+    }
+  // dP = tril(dO U^T)
+  {
+    float pp[4][4];
+    zero(pp);
+    mm_acc<4, 4>(pp, sO, D, 1, U, 1, D, D, sStage);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int t = ty + 16 * i, s = tx + 16 * j;
+        sP[t * C + s] = s <= t ? pp[i][j] : 0.f;
+      }
+  }
+  // dKhat = U dSn^T  ->  dK += dKhat Gam/gamma,  dG -= dKhat Khat,  dG_last += sum_t dKhat Khat
+  zero(acc);
+  mm_acc<4, NJ>(acc, U, D, 1, dSn, 1, D, D, sStage);
+#pragma unroll
+  for (int j = 0; j < NJ; ++j) {
+    float colsum = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int c = tx + 16 * j, e = (ty + 16 * i) * D + c;
+      const float f = exp2f(G63[c] - sG[e]);
+      const float kh = sK[e] * f;
+      accK[i][j] = fmaf(acc[i][j], f, accK[i][j]);
+      accG[i][j] = fmaf(-acc[i][j], kh, accG[i][j]);
+      colsum = fmaf(acc[i][j], kh, colsum);
+    }
+    sPart[ty * D + tx + 16 * j] = colsum;
+  }
+  __syncthreads();
+  // dGam = rowsum(dSn * S)  ->  dG_last += dGam Gam;  the partial column sums in a
+  // fixed order, so the result is the same on every run
+  if (tid < D) {
+    float s = 0.f;
+    for (int jj = 0; jj < D; ++jj) s = fmaf(dSn[(size_t)tid * D + jj], S[(size_t)tid * D + jj], s);
+    float e = s * exp2f(G63[tid]);
+    for (int y = 0; y < 16; ++y) e += sPart[y * D + tid];
+    sExtra[tid] = e;
+  }
+
+  // gated products of dP:  P1_t = sum_{s<=t} dP_ts k_s e^{G_t-G_s},  P2_s = sum_{t>=s} dP_ts q_t e^{G_t-G_s}
+  // (the shared-memory dO tile is dead from here on and holds the gate tables)
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    const int r0 = 16 * b, r1 = r0 + 15;
+    __syncthreads();
+    for (int e = tid; e < (r0 + 16) * D; e += NTH) {
+      const int c = e % D;
+      sO[e] = sK[e] * exp2f(sG[r0 * D + c] - sG[e]);
+    }
+    __syncthreads();
+    {
+      const int t = r0 + ty;
+      float o1[NJ];
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) o1[j] = 0.f;
+      for (int s = 0; s <= t; ++s) {
+        const float dp = sP[t * C + s];
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) o1[j] = fmaf(dp, sO[s * D + tx + 16 * j], o1[j]);
+      }
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) {
+        const int c = tx + 16 * j, e = t * D + c;
+        const float p1 = o1[j] * exp2f(sG[e] - sG[r0 * D + c]);
+        accQ[b][j] += p1;
+        accG[b][j] = fmaf(sQ[e], p1, accG[b][j]);
+      }
+    }
+    __syncthreads();
+    for (int e = r0 * D + tid; e < C * D; e += NTH) {
+      const int c = e % D;
+      sO[e] = sQ[e] * exp2f(sG[e] - sG[r1 * D + c]);
+    }
+    __syncthreads();
+    {
+      const int s = r0 + ty;
+      float o2[NJ];
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) o2[j] = 0.f;
+      for (int t = s; t < C; ++t) {
+        const float dp = sP[t * C + s];
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) o2[j] = fmaf(dp, sO[t * D + tx + 16 * j], o2[j]);
+      }
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) {
+        const int c = tx + 16 * j, e = s * D + c;
+        const float p2 = o2[j] * exp2f(sG[r1 * D + c] - sG[e]);
+        accK[b][j] += p2;
+        accG[b][j] = fmaf(-sK[e], p2, accG[b][j]);
+      }
+    }
+  }
+
+  // dW = -dU S^T (into the dO tile)
+  zero(acc);
+  mm_acc<4, NJ>(acc, dU, D, 1, S, 1, D, D, sStage);
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) sO[(ty + 16 * i) * D + tx + 16 * j] = -acc[i][j];
+  for (int e = tid; e < C * C; e += NTH) sT[e] = p.wT[ch * C * C + e];
+  // T^T dU -> dV = Diag(beta) T^T dU, dbeta += (T^T dU) . v
+  zero(acc);
+  mm_acc<4, NJ>(acc, sT, 1, C, dU, D, 1, C, sStage);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int t = ty + 16 * i;
+    float rs = 0.f;
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) {
+      const int c = tx + 16 * j;
+      rs = fmaf(acc[i][j], sV[t * D + c], rs);
+      if (t < n) p.dv[((size_t)(tok0 + t) * H + h) * D + c] = sB[t] * acc[i][j];
+    }
+    rs = row_sum16(rs);
+    if (tx == 0) sDb[t] += rs;
+  }
+  // T^T dW -> d(gamma K) = Diag(beta) T^T dW;  dbeta += (T^T dW) . (gamma k)
+  zero(acc);
+  mm_acc<4, NJ>(acc, sT, 1, C, sO, D, 1, C, sStage);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int t = ty + 16 * i;
+    float rs = 0.f;
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) {
+      const int e = t * D + tx + 16 * j;
+      const float kg = exp2f(sG[e]) * sK[e];
+      const float dkg = sB[t] * acc[i][j];
+      accK[i][j] = fmaf(dkg, exp2f(sG[e]), accK[i][j]);
+      accG[i][j] = fmaf(dkg, kg, accG[i][j]);
+      rs = fmaf(acc[i][j], kg, rs);
+    }
+    rs = row_sum16(rs);
+    if (tx == 0) sDb[t] += rs;
+  }
+  // dT = dU (Diag(beta) V)^T + dW (Diag(beta) gamma K)^T   (into the dP tile)
+  {
+    float tt[4][4];
+    zero(tt);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) sV[(ty + 16 * i) * D + tx + 16 * j] *= sB[ty + 16 * i];
+    mm_acc<4, 4>(tt, dU, D, 1, sV, 1, D, D, sStage);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) {
+        const int e = (ty + 16 * i) * D + tx + 16 * j;
+        sV[e] = sB[ty + 16 * i] * exp2f(sG[e]) * sK[e];
+      }
+    mm_acc<4, 4>(tt, sO, D, 1, sV, 1, D, D, sStage);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) sP[(ty + 16 * i) * C + tx + 16 * j] = tt[i][j];
+  }
+  // dZ = -T^T (dT T^T);  dA = tril_strict(Diag(beta) dZ);  dbeta += sum_s dZ_ts A_ts
+  {
+    float tt[4][4];
+    zero(tt);
+    mm_acc<4, 4>(tt, sP, C, 1, sT, 1, C, C, sStage);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) sV[(ty + 16 * i) * C + tx + 16 * j] = tt[i][j];
+    zero(tt);
+    mm_acc<4, 4>(tt, sT, 1, C, sV, C, 1, C, sStage);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int t = ty + 16 * i;
+      float rs = 0.f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int s = tx + 16 * j;
+        const float dz = -tt[i][j];
+        const bool low = s < t;
+        if (low) rs = fmaf(dz, p.wA[ch * C * C + t * C + s], rs);
+        sP[t * C + s] = low ? sB[t] * dz : 0.f;
+      }
+      rs = row_sum16(rs);
+      if (tx == 0) sDb[t] += rs;
+    }
+  }
+
+  // gated products of dA:  A1_t = sum_{s<t} dA_ts k_s e^{G_t-G_s},  A2_s = sum_{t>s} dA_ts k_t e^{G_t-G_s}
+#pragma unroll
+  for (int b = 0; b < 4; ++b) {
+    const int r0 = 16 * b, r1 = r0 + 15;
+    __syncthreads();
+    for (int e = tid; e < (r0 + 16) * D; e += NTH) {
+      const int c = e % D;
+      sO[e] = sK[e] * exp2f(sG[r0 * D + c] - sG[e]);
+    }
+    __syncthreads();
+    {
+      const int t = r0 + ty;
+      float o1[NJ];
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) o1[j] = 0.f;
+      for (int s = 0; s < t; ++s) {
+        const float da = sP[t * C + s];
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) o1[j] = fmaf(da, sO[s * D + tx + 16 * j], o1[j]);
+      }
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) {
+        const int c = tx + 16 * j, e = t * D + c;
+        const float a1 = o1[j] * exp2f(sG[e] - sG[r0 * D + c]);
+        accK[b][j] += a1;
+        accG[b][j] = fmaf(sK[e], a1, accG[b][j]);
+      }
+    }
+    __syncthreads();
+    for (int e = r0 * D + tid; e < C * D; e += NTH) {
+      const int c = e % D;
+      sO[e] = sK[e] * exp2f(sG[e] - sG[r1 * D + c]);
+    }
+    __syncthreads();
+    {
+      const int s = r0 + ty;
+      float o2[NJ];
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) o2[j] = 0.f;
+      for (int t = s + 1; t < C; ++t) {
+        const float da = sP[t * C + s];
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) o2[j] = fmaf(da, sO[t * D + tx + 16 * j], o2[j]);
+      }
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) {
+        const int c = tx + 16 * j, e = s * D + c;
+        const float a2 = o2[j] * exp2f(sG[r1 * D + c] - sG[e]);
+        accK[b][j] += a2;
+        accG[b][j] = fmaf(-sK[e], a2, accG[b][j]);
+      }
+    }
+  }
+
+  // dg = reverse cumsum of dG (the last-row terms reach every row); write the gradients
+  __syncthreads();
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) {
+      const int t = ty + 16 * i, c = tx + 16 * j;
+      sV[t * D + c] = accG[i][j];
+      if (t < n) {
+        const size_t o = ((size_t)(tok0 + t) * H + h) * D + c;
+        p.dq[o] = accQ[i][j];
+        p.dk[o] = accK[i][j];
+      }
+    }
+  __syncthreads();
+  if (tid < D) {
+    float run = sExtra[tid];
+    for (int t = C - 1; t >= 0; --t) {
+      run += sV[t * D + tid];
+      if (t < n) p.dg[((size_t)(tok0 + t) * H + h) * D + tid] = run;
+    }
+  }
+  if (tid < C && tid < n) p.dbeta[(size_t)(tok0 + tid) * H + h] = sDb[tid];
+}
+
+template <typename K>
+cudaError_t set_smem(K kernel, size_t bytes) {
+  return cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes);
+}
+
+template <int D, typename TIn>
+cudaError_t launch_bwd_d(const BwdParams &p, cudaStream_t stream) {
+  cudaError_t e;
+  const unsigned chunk_grid = (unsigned)((size_t)p.n_chunks * p.H);
+  if (chunk_grid > 0) {
+    if ((e = set_smem(bwd_prep_kernel<D, TIn>, PrepLayout<D>::bytes)) != cudaSuccess) return e;
+    bwd_prep_kernel<D, TIn><<<chunk_grid, NTH, PrepLayout<D>::bytes, stream>>>(p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  if ((e = set_smem(bwd_state_kernel<D>, StateLayout<D>::bytes)) != cudaSuccess) return e;
+  bwd_state_kernel<D><<<(unsigned)(p.n_req * p.H), NTH, StateLayout<D>::bytes, stream>>>(p);
+  if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if (chunk_grid > 0) {
+    if ((e = set_smem(bwd_grad_kernel<D, TIn>, GradLayout<D>::bytes)) != cudaSuccess) return e;
+    bwd_grad_kernel<D, TIn><<<chunk_grid, NTH, GradLayout<D>::bytes, stream>>>(p);
+    if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  }
+  return cudaSuccess;
+}
+
+}  // namespace
+
+// Workspace carve-up shared by the size query and the launch.
+struct BwdWorkspace {
+  size_t off_chunks, off_cu_chunks, off_cu_snap, off_snaps, off_zero;
+  size_t off_A, off_T, off_W, off_U, off_Kh, off_X, off_Y, off_Gam, total;
+};
+
+static size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
+
+BwdWorkspace backward_workspace(int n_req, int n_chunks, int n_snap, int H, int D) {
+  BwdWorkspace w{};
+  const size_t nch = (size_t)n_chunks * H, f = sizeof(float);
+  size_t o = 0;
+  auto take = [&](size_t bytes) { const size_t at = o; o = a256(o + bytes); return at; };
+  w.off_chunks = take((size_t)n_chunks * sizeof(int4));
+  w.off_cu_chunks = take((size_t)(n_req + 1) * sizeof(int32_t));
+  w.off_cu_snap = take((size_t)(n_req + 1) * sizeof(int32_t));
+  w.off_snaps = take((size_t)n_snap * H * D * D * f);
+  w.off_zero = take((size_t)D * D * f);
+  w.off_A = take(nch * C * C * f);
+  w.off_T = take(nch * C * C * f);
+  w.off_W = take(nch * C * D * f);
+  w.off_U = take(nch * C * D * f);
+  w.off_Kh = take(nch * C * D * f);
+  w.off_X = take(nch * C * D * f);
+  w.off_Y = take(nch * (size_t)D * D * f);
+  w.off_Gam = take(nch * D * f);
+  w.total = o;
+  return w;
+}
+
+cudaError_t launch_backward(const BackwardLaunch &b, cudaStream_t stream) {
+  const BwdWorkspace w = backward_workspace(b.n_req, b.n_chunks, b.n_snap, b.H, b.D);
+  char *ws = static_cast<char *>(b.workspace);
+  BwdParams p{};
+  p.q = b.q; p.k = b.k; p.v = b.v; p.g = b.g; p.beta = b.beta;
+  p.initial_state = b.initial_state; p.d_o = b.d_o; p.d_final = b.d_final;
+  p.dq = b.dq; p.dk = b.dk; p.dv = b.dv; p.dg = b.dg; p.dbeta = b.dbeta;
+  p.d_initial = b.d_initial;
+  p.chunks = reinterpret_cast<const int4 *>(ws + w.off_chunks);
+  p.cu_chunks = reinterpret_cast<const int32_t *>(ws + w.off_cu_chunks);
+  p.cu_snap = reinterpret_cast<const int32_t *>(ws + w.off_cu_snap);
+  p.snaps = reinterpret_cast<const float *>(ws + w.off_snaps);
+  p.zero_state = reinterpret_cast<const float *>(ws + w.off_zero);
+  p.wA = reinterpret_cast<float *>(ws + w.off_A);
+  p.wT = reinterpret_cast<float *>(ws + w.off_T);
+  p.wW = reinterpret_cast<float *>(ws + w.off_W);
+  p.wU = reinterpret_cast<float *>(ws + w.off_U);
+  p.wKh = reinterpret_cast<float *>(ws + w.off_Kh);
+  p.wX = reinterpret_cast<float *>(ws + w.off_X);
+  p.wY = reinterpret_cast<float *>(ws + w.off_Y);
+  p.wGam = reinterpret_cast<float *>(ws + w.off_Gam);
+  p.n_req = b.n_req; p.n_chunks = b.n_chunks; p.H = b.H;
+  if (b.D == 128)
+    return b.in_dtype == KDA_BF16 ? launch_bwd_d<128, __nv_bfloat16>(p, stream)
+                                  : launch_bwd_d<128, float>(p, stream);
+  return b.in_dtype == KDA_BF16 ? launch_bwd_d<64, __nv_bfloat16>(p, stream)
+                                : launch_bwd_d<64, float>(p, stream);
+}
+
+size_t backward_workspace_bytes(int n_req, int n_chunks, int n_snap, int H, int D) {
+  return backward_workspace(n_req, n_chunks, n_snap, H, D).total;
+}
+
+void backward_offsets(int n_req, int n_chunks, int n_snap, int H, int D, size_t *chunks,
+                      size_t *cu_chunks, size_t *cu_snap, size_t *snaps, size_t *zero) {
+  const BwdWorkspace w = backward_workspace(n_req, n_chunks, n_snap, H, D);
+  *chunks = w.off_chunks;
+  *cu_chunks = w.off_cu_chunks;
+  *cu_snap = w.off_cu_snap;
+  *snaps = w.off_snaps;
+  *zero = w.off_zero;
+}
+
+}  // namespace kda

@@ -77,6 +77,23 @@ cudaError_t launch_combine(const float *s_loc, const float *m, const float *s_in
                            cudaStream_t stream);
 unsigned int *device_status_word();  // address of the current device's status word
 
+// Backward of the prefill (kda_backward.cu).  The workspace holds, in order,
+// the chunk table, the chunk-start snapshots of a forward pass, a zero state
+// and the per-(chunk, head) intermediates; backward_offsets() gives the first
+// five regions so the host can fill the tables and run the forward pass.
+struct BackwardLaunch {
+  const void *q, *k, *v;
+  const float *g, *beta, *initial_state, *d_o, *d_final;
+  float *dq, *dk, *dv, *dg, *dbeta, *d_initial;
+  void *workspace;
+  int n_req, n_chunks, n_snap, H, D;
+  kda_dtype in_dtype;
+};
+cudaError_t launch_backward(const BackwardLaunch &b, cudaStream_t stream);
+size_t backward_workspace_bytes(int n_req, int n_chunks, int n_snap, int H, int D);
+void backward_offsets(int n_req, int n_chunks, int n_snap, int H, int D, size_t *chunks,
+                      size_t *cu_chunks, size_t *cu_snap, size_t *snaps, size_t *zero);
+
 // Element loads/stores shared by the kernels.
 __device__ __forceinline__ float load_elem(const float *p, size_t i) { return p[i]; }
 __device__ __forceinline__ float load_elem(const __nv_bfloat16 *p, size_t i) {

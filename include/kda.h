@@ -288,6 +288,62 @@ typedef struct kda_decode_args {
 kda_status kda_decode_step(const kda_decode_args *args, void *stream);
 
 /* ------------------------------------------------------------------------ */
+/* Backward (training): gradients of the chunked prefill.                   */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Arguments of kda_prefill_backward.
+ *
+ * Source: FlashKDA also speeds up training ("Kimi K3 开源日来了", FlashKDA
+ * section), which needs the derivative of the same prefill map.  For the
+ * inputs of a kda_prefill_chunked call, this computes the gradients of
+ *
+ *     L = sum(d_o * o) + sum(d_final * final_state)
+ *
+ * with respect to q, k, v, g (= log alpha), beta and the initial state, where
+ * (o, final_state) is what kda_prefill_chunked returns for those inputs.
+ * Snapshots take no cotangent.  The chunk-start states are recomputed by a
+ * forward pass inside the call; nothing from an earlier forward is needed.
+ *
+ *   n_req, total_tokens, H, dk, dv, in_dtype, q, k, v, g, beta, cu_seqlens,
+ *   initial_state   as in kda_prefill_args (dk == dv in {64, 128}).
+ *   cu_seqlens_host HOST int32 [n_req + 1], REQUIRED: it sizes the workspace
+ *                   and the chunk table.  Same values as cu_seqlens.
+ *   d_o             fp32 [total_tokens, H, dv] or NULL (zero cotangent).
+ *   d_final         fp32 [n_req, H, dk, dv] or NULL (zero cotangent).
+ *   d_q, d_k, d_g   fp32 [total_tokens, H, dk] outputs: gradients of q, k, g.
+ *   d_v             fp32 [total_tokens, H, dv] output: gradient of v.
+ *   d_beta          fp32 [total_tokens, H] output: gradient of beta.
+ *   d_initial       fp32 [n_req, H, dk, dv] output, or NULL (not returned).
+ * Outputs must not overlap each other, the inputs or the workspace.  The
+ * workspace (kda_prefill_backward_workspace_size bytes, 256-byte aligned) is
+ * scratch owned by the caller for the duration of the call.  The host tables
+ * are copied into the workspace before the call returns, so cu_seqlens_host
+ * may be freed afterwards.
+ */
+typedef struct kda_backward_args {
+  int32_t n_req;
+  int32_t total_tokens;
+  int32_t H, dk, dv;
+  kda_dtype in_dtype;
+  const void *q, *k, *v;
+  const float *g;
+  const float *beta;
+  const int32_t *cu_seqlens;
+  const int32_t *cu_seqlens_host;
+  const float *initial_state;
+  const float *d_o;
+  const float *d_final;
+  float *d_q, *d_k, *d_v, *d_g, *d_beta;
+  float *d_initial;
+} kda_backward_args;
+
+/* Workspace bytes for kda_prefill_backward (0 if the arguments are invalid). */
+size_t kda_prefill_backward_workspace_size(const kda_backward_args *args);
+kda_status kda_prefill_backward(const kda_backward_args *args, void *workspace,
+                                size_t workspace_bytes, void *stream);
+
+/* ------------------------------------------------------------------------ */
 /* Helpers.                                                                 */
 /* ------------------------------------------------------------------------ */
 

@@ -148,3 +148,52 @@ def test_missing_library_fails_loudly(tmp_path):
             _lib.load(str(tmp_path / "nope.so"))
     finally:
         _lib._lib = saved
+
+
+_CU_BWD = (ctypes.c_int32 * 3)(0, 64, 128)
+
+
+def _bwd_args(**over):
+    a = _lib.BackwardArgs()
+    a.n_req, a.total_tokens, a.H, a.dk, a.dv, a.in_dtype = 2, 128, 2, 128, 128, 0
+    names = ("q", "k", "v", "g", "beta", "cu_seqlens", "d_o", "d_q", "d_k", "d_v", "d_g",
+             "d_beta")
+    for i, n in enumerate(names):
+        setattr(a, n, FAKE + (i << 24))
+    a.cu_seqlens_host = ctypes.addressof(_CU_BWD)
+    for k_, v_ in over.items():
+        setattr(a, k_, v_)
+    return a
+
+
+def _backward(a, ws=None, ws_bytes=0):
+    return _lib.load().kda_prefill_backward(ctypes.byref(a), ws, ws_bytes, None)
+
+
+@pytest.mark.parametrize("over,code", [
+    ({"cu_seqlens_host": None}, 1),                # the host offsets are required
+    ({"dk": 96, "dv": 96}, 2), ({"H": 0}, 1), ({"in_dtype": 7}, 1),
+    ({"d_q": None}, 1), ({"d_k": FAKE + 4}, 1),
+    ({"d_v": FAKE + (2 << 24)}, 1),                # d_v overlaps v
+    ({"d_g": FAKE + (7 << 24)}, 1),                # d_g overlaps d_q
+    ({"total_tokens": 100}, 1),                    # host offsets end elsewhere
+])
+def test_backward_rejects_invalid_args(over, code):
+    assert _backward(_bwd_args(**over)) == code
+
+
+def test_backward_workspace_contract():
+    lib = _lib.load()
+    a = _bwd_args()
+    need = lib.kda_prefill_backward_workspace_size(ctypes.byref(a))
+    assert need > 0 and need % 256 == 0
+    assert _backward(a, None, 0) == 6
+    assert _backward(a, FAKE + (20 << 24) + 16, need) == 6
+    assert _backward(a, FAKE + (20 << 24), need - 1) == 6
+    assert _backward(a, FAKE + (7 << 24), need) == 1      # workspace overlaps d_q
+    # one more chunk (65 tokens in the second request) needs more workspace
+    cu = (ctypes.c_int32 * 3)(0, 64, 129)
+    b = _bwd_args(total_tokens=129, cu_seqlens_host=ctypes.addressof(cu))
+    assert lib.kda_prefill_backward_workspace_size(ctypes.byref(b)) > need
+    assert lib.kda_prefill_backward_workspace_size(ctypes.byref(_bwd_args(dk=96, dv=96))) == 0
+    assert _backward(_bwd_args(n_req=0, total_tokens=0)) == 0
