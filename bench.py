@@ -22,6 +22,7 @@ collective; only the timing uses a max over ranks).
 from __future__ import annotations
 
 import argparse
+import itertools
 import json
 import os
 import statistics
@@ -359,6 +360,7 @@ def run_ours(args, world, rank, local):
     if not args.no_extra:
         line["single_seq"] = bench_single_seq(args, dev, peaks)
         line["kcp_million"] = bench_kcp_million(args, dev, peaks, world, rank)
+        line["backward"] = bench_backward(args, inp, dev, peaks, world)
     if not args.no_e2e:
         line["e2e"] = bench_e2e(args, inp, dev, world)
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
@@ -438,6 +440,54 @@ def _time_calls(fn, warm: int, steps: int, stream) -> float:
     e.record(stream)
     torch.cuda.synchronize()
     return s.elapsed_time(e) / steps
+
+
+def backward_bytes(T: int, H: int, d: int, n_req: int) -> int:
+    """Algorithmic bytes of one backward call: q, k, v (bf16), g, beta and dO read
+    once, dq, dk, dv, dg (fp32) and dbeta written once, plus per chain the
+    initial state and dS_final read and dS_0 written."""
+    per_th = 2 * 3 * d + 4 * d + 4 + 4 * d + 4 * 4 * d + 4
+    return T * H * per_th + 3 * n_req * H * d * d * 4
+
+
+def bench_backward(args, inp, dev, peaks, world):
+    """The backward of the headline workload: gradients of q, k, v, g, beta and the
+    initial state for random fp32 cotangents of o and the final states, one
+    kda_prefill_backward call per step (forward recompute included)."""
+    import torch
+
+    import decode_kda_chunked_b200 as kda
+    T, H, d, n = inp.total_tokens, 32, 128, inp.n_req
+    gen = torch.Generator(device=dev).manual_seed(7)
+    d_o = torch.randn((T, H, d), generator=gen, device=dev)
+    d_fin = torch.randn((n, H, d, d), generator=gen, device=dev)
+    s0 = torch.zeros((n, H, d, d), device=dev)
+    cu_h = torch.tensor([0] + list(itertools.accumulate(inp.lengths)), dtype=torch.int32)
+    f32 = dict(dtype=torch.float32, device=dev)
+    dq, dk, dv, dg = (torch.empty((T, H, d), **f32) for _ in range(4))
+    db = torch.empty((T, H), **f32)
+    d0 = torch.empty((n, H, d, d), **f32)
+    a = kda.make_backward_args(inp.q, inp.k, inp.v, inp.g, inp.beta, inp.cu_seqlens, cu_h,
+                               dq, dk, dv, dg, db, s0, d_o, d_fin, d0)
+    ws = torch.empty(kda.kda_prefill_backward_workspace_size(a), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    call = lambda: kda.kda_prefill_backward(inp.q, inp.k, inp.v, inp.g, inp.beta, inp.cu_seqlens,
+                                            cu_h, dq, dk, dv, dg, db, s0, d_o, d_fin, d0, ws,
+                                            stream=stream)
+    call()
+    torch.cuda.synchronize()
+    barrier(world)
+    ms = max_over_ranks(_time_calls(call, 1, 3, stream), world)
+    b = backward_bytes(T, H, d, n)
+    return {"workload": "backward of the headline varlen prefill (64 requests, H=32, d=128, "
+                        "bf16 inputs, fp32 gradients); random fp32 cotangents of o and the "
+                        "final states",
+            "value": world * T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
+            "workspace_bytes": ws.numel(), "gpu_launches_per_step": 4,
+            "roofline": {"bound": "hbm", "achieved": b / (ms * 1e-3) / 1e9,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": b / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+                         "algorithmic_bytes_per_launch": b}}
 
 
 def bench_single_seq(args, dev, peaks):

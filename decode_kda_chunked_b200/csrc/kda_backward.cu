@@ -30,7 +30,8 @@
 // Launches: the forward kernel with a snapshot every 64 tokens (the chunk
 // start states), then
 //   bwd_prep  (CTA per chunk and head): A, T, W, U~, Khat, Gam, X = P^T dO, Y = (gamma Q)^T dO
-//   bwd_state (CTA per request and head): the serial pass; dU overwrites X, dSn overwrites Y
+//   bwd_state (CTA per request, head and 16 state columns): the serial pass;
+//             dU overwrites X, dSn overwrites Y
 //   bwd_grad  (CTA per chunk and head): every token gradient of the chunk
 // All backward arithmetic is fp32 on the CUDA cores.  A CTA's 256 threads
 // form a 16 x 16 grid; thread (ty, tx) owns rows ty + 16 i and columns
@@ -67,38 +68,55 @@ struct BwdParams {
 // A(m, k) = A[m am + k ak], B(k, n) = B[k bk + n bn], in any memory space.
 // Slices of 16 along k are staged through shared memory `stage`
 // (16 (16 MI + 1) + 16 (16 NJ + 1) floats) so the inner loop reads
-// conflict-free shared memory.  Every thread of the CTA must call it.
+// conflict-free shared memory; the next slice is loaded into registers while
+// the current one is multiplied.  Every thread of the CTA must call it.
 template <int MI, int NJ>
 __device__ void mm_acc(float (&acc)[MI][NJ], const float *A, int am, int ak, const float *B,
                        int bk, int bn, int K, float *stage) {
   constexpr int M = 16 * MI, N = 16 * NJ, LA = M + 1, LB = N + 1;
   float *As = stage, *Bs = stage + 16 * LA;
   const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  // each thread moves MI elements of the A slice and NJ of the B slice; the
+  // walk order puts consecutive threads on the operand's contiguous axis
+  const bool a_k_inner = ak == 1, b_n_inner = bn == 1;
+  auto a_at = [&](int e, int &kk, int &m) {
+    if (a_k_inner) { kk = e & 15; m = e >> 4; } else { m = e % M; kk = e / M; }
+  };
+  auto b_at = [&](int e, int &kk, int &n) {
+    if (b_n_inner) { n = e % N; kk = e / N; } else { kk = e & 15; n = e >> 4; }
+  };
+  float ra[MI], rb[NJ];
+  auto fetch = [&](int k0) {
+#pragma unroll
+    for (int q = 0; q < MI; ++q) {
+      int kk, m;
+      a_at(tid + q * NTH, kk, m);
+      ra[q] = A[(size_t)m * am + (size_t)(k0 + kk) * ak];
+    }
+#pragma unroll
+    for (int q = 0; q < NJ; ++q) {
+      int kk, n;
+      b_at(tid + q * NTH, kk, n);
+      rb[q] = B[(size_t)(k0 + kk) * bk + (size_t)n * bn];
+    }
+  };
+  fetch(0);
   for (int k0 = 0; k0 < K; k0 += 16) {
-    __syncthreads();
-    if (ak == 1) {
-      for (int e = tid; e < 16 * M; e += NTH) {
-        const int kk = e & 15, m = e >> 4;
-        As[kk * LA + m] = A[(size_t)m * am + k0 + kk];
-      }
-    } else {
-      for (int e = tid; e < 16 * M; e += NTH) {
-        const int m = e % M, kk = e / M;
-        As[kk * LA + m] = A[(size_t)m * am + (size_t)(k0 + kk) * ak];
-      }
+    __syncthreads();  // the previous slice has been consumed
+#pragma unroll
+    for (int q = 0; q < MI; ++q) {
+      int kk, m;
+      a_at(tid + q * NTH, kk, m);
+      As[kk * LA + m] = ra[q];
     }
-    if (bn == 1) {
-      for (int e = tid; e < 16 * N; e += NTH) {
-        const int n = e % N, kk = e / N;
-        Bs[kk * LB + n] = B[(size_t)(k0 + kk) * bk + n];
-      }
-    } else {
-      for (int e = tid; e < 16 * N; e += NTH) {
-        const int kk = e & 15, n = e >> 4;
-        Bs[kk * LB + n] = B[(size_t)(k0 + kk) * bk + (size_t)n * bn];
-      }
+#pragma unroll
+    for (int q = 0; q < NJ; ++q) {
+      int kk, n;
+      b_at(tid + q * NTH, kk, n);
+      Bs[kk * LB + n] = rb[q];
     }
     __syncthreads();
+    if (k0 + 16 < K) fetch(k0 + 16);  // next slice in flight during this one's FMAs
 #pragma unroll 4
     for (int kk = 0; kk < 16; ++kk) {
       float a[MI], b[NJ];
@@ -307,68 +325,103 @@ __global__ void __launch_bounds__(NTH, 1) bwd_prep_kernel(const BwdParams p) {
 }
 
 // ---------------------------------------------------------------------------
-// bwd_state: the serial pass over chunk-end cotangents, last chunk first
+// bwd_state: the serial pass over chunk-end cotangents, last chunk first.  The
+// recurrence acts on every value column of dS on its own (as the forward acts
+// on the columns of S), so one CTA owns a 16-column slice of one chain; the
+// chunk's Khat and W tiles are copied to shared memory with cp.async.
 // ---------------------------------------------------------------------------
+constexpr int SC = 16;  // state columns per CTA
+
 template <int D>
 struct StateLayout {
-  static constexpr int oS = 0, oU = oS + D * D, oStage = oU + C * D;
-  static constexpr int total = oStage + stage_floats(D, D);
+  static constexpr int oKh = 0, oW = oKh + C * D, oS = oW + C * D, oU = oS + D * SC;
+  static constexpr int total = oU + C * SC;
   static constexpr size_t bytes = sizeof(float) * total;
 };
 
+__device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
+  const uint32_t a = (uint32_t)__cvta_generic_to_shared(smem);
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(a), "l"(gmem) : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+}
+
 template <int D>
-__global__ void __launch_bounds__(NTH, 1) bwd_state_kernel(const BwdParams p) {
+__global__ void __launch_bounds__(NTH) bwd_state_kernel(const BwdParams p) {
   using L = StateLayout<D>;
-  constexpr int NJ = D / 16;
+  constexpr int NSL = D / SC, MI = D / 16;
   extern __shared__ float4 smem_f4[];
   float *sm = reinterpret_cast<float *>(smem_f4);
-  float *sdS = sm + L::oS, *sdU = sm + L::oU, *sStage = sm + L::oStage;
+  float *sKh = sm + L::oKh, *sW = sm + L::oW, *sdS = sm + L::oS, *sdU = sm + L::oU;
   const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
   const int H = p.H;
-  const int r = blockIdx.x / H, h = blockIdx.x % H;
+  const int sl = blockIdx.x % NSL, rh = blockIdx.x / NSL;
+  const int r = rh / H, h = rh % H;
+  const int col = SC * sl + tx;  // the thread's state column; its rows are ty + 16 i
   const float *dfin = p.d_final ? p.d_final + ((size_t)r * H + h) * D * D : nullptr;
-  for (int e = tid; e < D * D; e += NTH) sdS[e] = dfin ? dfin[e] : 0.f;
-
+  float ds[MI];
+#pragma unroll
+  for (int i = 0; i < MI; ++i) {
+    ds[i] = dfin ? dfin[(size_t)(ty + 16 * i) * D + col] : 0.f;
+    sdS[(ty + 16 * i) * SC + tx] = ds[i];
+  }
   for (int jc = p.cu_chunks[r + 1] - 1; jc >= p.cu_chunks[r]; --jc) {
     const size_t ch = (size_t)jc * H + h;
-    // dU = X + Khat dSn  (overwrites X)
-    float u[4][NJ];
-    zero(u);
-    mm_acc<4, NJ>(u, p.wKh + ch * C * D, D, 1, sdS, D, 1, D, sStage);
+    const float4 *gK = reinterpret_cast<const float4 *>(p.wKh + ch * C * D);
+    const float4 *gW = reinterpret_cast<const float4 *>(p.wW + ch * C * D);
+    for (int e = tid; e < C * D / 4; e += NTH) {
+      cp_async16(sKh + 4 * e, gK + e);
+      cp_async16(sW + 4 * e, gW + e);
+    }
+    float u[4], y[MI], gam[MI];
 #pragma unroll
-    for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 4; ++i) u[i] = p.wX[ch * C * D + (size_t)(ty + 16 * i) * D + col];
 #pragma unroll
-      for (int j = 0; j < NJ; ++j) {
-        const int e = (ty + 16 * i) * D + tx + 16 * j;
-        const float x = p.wX[ch * C * D + e] + u[i][j];
-        p.wX[ch * C * D + e] = x;
-        sdU[e] = x;
-      }
-    // dS = Diag(Gam) dSn + Y - W^T dU;  dSn overwrites Y for the gradient pass
-    float s[NJ][NJ];
-    zero(s);
-    mm_acc<NJ, NJ>(s, p.wW + ch * C * D, 1, D, sdU, D, 1, C, sStage);
+    for (int i = 0; i < MI; ++i) {
+      y[i] = p.wY[ch * D * D + (size_t)(ty + 16 * i) * D + col];
+      gam[i] = p.wGam[ch * D + ty + 16 * i];
+    }
+    cp_async_wait_all();
+    __syncthreads();
+    // dU = X + Khat dSn   (overwrites X)
+    for (int k = 0; k < D; k += 4) {
+      const float d0 = sdS[k * SC + tx], d1 = sdS[(k + 1) * SC + tx];
+      const float d2 = sdS[(k + 2) * SC + tx], d3 = sdS[(k + 3) * SC + tx];
 #pragma unroll
-    for (int i = 0; i < NJ; ++i) {
-      const float gam = p.wGam[ch * D + ty + 16 * i];
-#pragma unroll
-      for (int j = 0; j < NJ; ++j) {
-        const int e = (ty + 16 * i) * D + tx + 16 * j;
-        const float old = sdS[e];
-        s[i][j] = fmaf(gam, old, p.wY[ch * D * D + e] - s[i][j]);
-        p.wY[ch * D * D + e] = old;
+      for (int i = 0; i < 4; ++i) {
+        const float4 kh = *reinterpret_cast<const float4 *>(sKh + (ty + 16 * i) * D + k);
+        u[i] = fmaf(kh.x, d0, fmaf(kh.y, d1, fmaf(kh.z, d2, fmaf(kh.w, d3, u[i]))));
       }
     }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      sdU[(ty + 16 * i) * SC + tx] = u[i];
+      p.wX[ch * C * D + (size_t)(ty + 16 * i) * D + col] = u[i];
+    }
     __syncthreads();
+    // dS = Diag(Gam) dSn + Y - W^T dU;  dSn overwrites Y for the gradient pass
+    float acc[MI];
 #pragma unroll
-    for (int i = 0; i < NJ; ++i)
+    for (int i = 0; i < MI; ++i) acc[i] = 0.f;
+    for (int t = 0; t < C; ++t) {
+      const float du = sdU[t * SC + tx];
 #pragma unroll
-      for (int j = 0; j < NJ; ++j) sdS[(ty + 16 * i) * D + tx + 16 * j] = s[i][j];
+      for (int i = 0; i < MI; ++i) acc[i] = fmaf(sW[t * D + ty + 16 * i], du, acc[i]);
+    }
+#pragma unroll
+    for (int i = 0; i < MI; ++i) {
+      p.wY[ch * D * D + (size_t)(ty + 16 * i) * D + col] = ds[i];
+      ds[i] = fmaf(gam[i], ds[i], y[i] - acc[i]);
+    }
+    __syncthreads();  // every read of sdS, sKh and sW of this chunk is done
+#pragma unroll
+    for (int i = 0; i < MI; ++i) sdS[(ty + 16 * i) * SC + tx] = ds[i];
   }
-  __syncthreads();
   if (p.d_initial) {
     float *dst = p.d_initial + ((size_t)r * H + h) * D * D;
-    for (int e = tid; e < D * D; e += NTH) dst[e] = sdS[e];
+#pragma unroll
+    for (int i = 0; i < MI; ++i) dst[(size_t)(ty + 16 * i) * D + col] = ds[i];
   }
 }
 
@@ -727,7 +780,8 @@ cudaError_t launch_bwd_d(const BwdParams &p, cudaStream_t stream) {
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if ((e = set_smem(bwd_state_kernel<D>, StateLayout<D>::bytes)) != cudaSuccess) return e;
-  bwd_state_kernel<D><<<(unsigned)(p.n_req * p.H), NTH, StateLayout<D>::bytes, stream>>>(p);
+  bwd_state_kernel<D>
+      <<<(unsigned)(p.n_req * p.H * (D / SC)), NTH, StateLayout<D>::bytes, stream>>>(p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if (chunk_grid > 0) {
     if ((e = set_smem(bwd_grad_kernel<D, TIn>, GradLayout<D>::bytes)) != cudaSuccess) return e;
