@@ -9,11 +9,12 @@
 // channels, columns = key channels or tokens):
 //
 //   A | P   [128 x 16] per 16-column block b:  [L_b ; Lq_b] R_b^T           (A from TMEM)
-//   W^T     = (gamma*K)^T (T Diag(b))^T                                      (A from TMEM)
-//   U~^T    = V^T (T Diag(b))^T                                              (A from TMEM)
-//   U^T     = U~^T - S^T W^T                                                 (A = S^T in TMEM)
+//   Y^T     = V^T - S^T (gamma*K)^T                                          (A = S^T in TMEM)
+//   U^T     = Y^T (T Diag(b))^T                                              (A = Y^T in TMEM)
 //   O^T     = S^T (gamma*Q)^T + U^T P^T                                      (A = S^T, U^T in TMEM)
 //   S^T    <- S^T Diag(gamma_63) + U^T Khat                                  (A = U^T in TMEM)
+// U = T Diag(b) (V - (gamma*K) S) is the chunk form's U~ - W S with W never formed:
+// Y needs only the state and the chunk's inputs, so it runs while the workers solve T.
 //
 // Gate factorisation for A and P: for the 16-token column block b with last
 // row r_b, exp(G_i - G_j) = exp(G_i - G_rb) * exp(G_rb - G_j).  The right
@@ -63,12 +64,13 @@ constexpr uint32_t RAW_BYTES = 81920;
 // Once every raw tile is read, the raw region holds the B operands R'_a of
 // the A|P products: row block a has 16(a+1) rows at byte 8192 a(a+1)/2.
 __host__ __device__ constexpr uint32_t rp_off(int a) { return 4096u * a * (a + 1); }
-constexpr uint32_t OFF_R = 81920;       // T-solve scratch (two [64 x 65] fp32); then W [64 x 128]
+constexpr uint32_t OFF_R = 81920;       // R scratch [64 x 132] fp32, then T-solve scratch
 constexpr int LDT = 65;                 // padded row stride of the T-solve scratch
 constexpr int LDR = 132;                // padded row stride of the fp32 R scratch [64][132]
 constexpr uint32_t OFF_MS = OFF_R;                  // beta*A strict lower
 constexpr uint32_t OFF_TI = OFF_R + 64 * LDT * 4;   // T = (I + beta A)^-1
-constexpr uint32_t OFF_GQ = 115712;     // (gamma*Q) [64 x 128] tf32 B operand
+constexpr uint32_t OFF_GQ = 115712;     // (gamma*Q) [64 x 128] tf32 B operand; once the O^T
+                                        // product has read it, (gamma*K) [64 x 128]
 constexpr uint32_t OFF_KHT = 148480;    // Khat^T [128 x 64] tf32 B operand
 constexpr uint32_t OFF_TB = 181248;     // T Diag(beta) [64 x 64] tf32 B operand
 constexpr uint32_t OFF_P = 197632;      // P [64 x 64] tf32 B operand
@@ -87,12 +89,11 @@ constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;  // alignment slack
 
 // ---- TMEM column map (512 columns x 128 lanes of fp32) ----
 constexpr uint32_t TM_S = 0;     // S^T (lane = value channel, col = key channel)
-constexpr uint32_t TM_L = 128;   // L* (A operand of A|P); later V^T [0,64), (gK)^T [64,128)
+constexpr uint32_t TM_L = 128;   // L* (A operand of A|P); later V^T -> Y^T in [0,64)
 // A (lanes 0..63) | P (lanes 64..127) of rows in block a: 16(a+1) columns at TM_AP + 8a(a+1)
 constexpr uint32_t TM_AP = 256;  // up to column 416
 __host__ __device__ constexpr uint32_t ap_col(int a) { return TM_AP + 8u * a * (a + 1); }
-constexpr uint32_t TM_X1 = 256;  // W^T             (alias A|P once the solve has read it)
-constexpr uint32_t TM_X2 = 320;  // U~^T -> U^T      (alias A|P)
+constexpr uint32_t TM_X2 = 320;  // U^T (alias A|P once the solve has read it)
 constexpr uint32_t TM_O = 416;   // O^T (own columns: issued right after the A|P products)
 constexpr uint32_t TM_COLS = 512;
 
@@ -144,10 +145,12 @@ __global__ void __launch_bounds__(NT + 32, 1)
   uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
   uint64_t *bar_tma = bars + 0;      // TMA -> workers: raw tiles landed
   uint64_t *bar_raw = bars + 1;      // workers -> control: raw tiles consumed (16 warps)
-  uint64_t *bar_opsap = bars + 2;    // workers -> control: two L_b buffers built (16 warps)
-  uint64_t *bar_ops = bars + 4;      // workers -> control: next MMA group's operands ready
-  uint64_t *bar_ap = bars + 5;       // control -> workers: A/P MMAs of a round done
-  uint64_t *bar_mma = bars + 7;      // control -> workers: MMA group done
+  uint64_t *bar_opsap = bars + 2;    // workers -> control: A|P operands built (16 warps)
+  uint64_t *bar_y = bars + 3;        // control -> workers: Y^T product done (S^T read)
+  uint64_t *bar_ops = bars + 4;      // workers -> control: T Diag(beta) ready, S^T scaled
+  uint64_t *bar_ap = bars + 5;       // control -> workers: A|P and O^T products done
+  uint64_t *bar_u = bars + 6;        // control -> control: U^T product done
+  uint64_t *bar_mma = bars + 7;      // control -> workers: chunk's last products done
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bars + 8);
   volatile int *s_abort = reinterpret_cast<volatile int *>(s_tmem + 1);
 
@@ -187,6 +190,8 @@ __global__ void __launch_bounds__(NT + 32, 1)
     mbar_init(bar_opsap, NT / 32);
     mbar_init(bar_ops, NT / 32);
     mbar_init(bar_ap, 1);
+    mbar_init(bar_y, 1);
+    mbar_init(bar_u, 1);
     mbar_init(bar_mma, 1);
     *s_abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
@@ -216,7 +221,7 @@ __global__ void __launch_bounds__(NT + 32, 1)
         for (int qd = 0; qd < 4; ++qd)
           tma_load_2d(sm + OFF_GRAW + 8192 * qd, &maps.g, h * DH + 32 * qd, y, bar_tma);
       };
-      uint32_t ph_raw = 0, ph_opsap[1] = {0}, ph_ops = 0;
+      uint32_t ph_raw = 0, ph_opsap[1] = {0}, ph_ops = 0, ph_u = 0;
       auto cwait = [&](uint64_t *bar, uint32_t &ph) -> bool {
         const bool good = *s_abort == 0 && mbar_wait(bar, ph);
         ph ^= 1u;
@@ -229,9 +234,9 @@ __global__ void __launch_bounds__(NT + 32, 1)
       };
       if (n_chunks > 0) issue_tma(0);
       for (int ci = 0; ci < n_chunks; ++ci) {
-        bool good = true;
-        // A | P: row block a against its R'_a (N = 16(a+1)); four interleaved chains
-        if (!(good = cwait(bar_opsap, ph_opsap[0]))) break;
+        // A | P: row block a against its R'_a (N = 16(a+1)); four interleaved chains;
+        // then O^T = S^T (gamma Q)^T, which needs only the state and gamma*Q
+        if (!cwait(bar_opsap, ph_opsap[0])) break;
         {
           const uint32_t rp = smem_u32(sm);
 #pragma unroll
@@ -241,38 +246,35 @@ __global__ void __launch_bounds__(NT + 32, 1)
               mma_tf32_ts(tm + ap_col(a), tm + TM_L + 8 * s, sw128_desc(rp + rp_off(a), 16 * (a + 1), s),
                           idesc_tf32(16 * (a + 1)), s > 0);
           }
-          mma_commit(bar_ap);
-          // O^T = S^T (gamma Q)^T needs only the state and gamma*Q: issue it now, so it
-          // runs while the workers solve T (its completion rides on the next commit)
           const uint32_t id = idesc_tf32(64);
           const uint32_t qb = smem_u32(sm + OFF_GQ);
 #pragma unroll
           for (int s = 0; s < DH / 8; ++s)
             mma_tf32_ts(tm + TM_O, tm + TM_S + 8 * s, sw128_desc(qb, C, s), id, s > 0);
+          mma_commit(bar_ap);  // gamma*Q and the R'_a operands are free after this
         }
-        if (!good || !cwait(bar_raw, ph_raw)) break;
+        // raw tiles consumed, V^T in TMEM, gamma*K in shared memory
+        if (!cwait(bar_raw, ph_raw)) break;
         if (ci + 1 < n_chunks) issue_tma((ci + 1) * C);
-        if (!cwait(bar_ops, ph_ops)) break;  // T Diag(beta), V^T, (gK)^T ready
-        {
+        {  // Y^T = V^T - S^T (gamma K)^T, while the workers solve T
+          const uint32_t idn = idesc_tf32(64, true);
+          const uint32_t kb = smem_u32(sm + OFF_GQ);
+#pragma unroll
+          for (int s = 0; s < DH / 8; ++s)
+            mma_tf32_ts(tm + TM_L, tm + TM_S + 8 * s, sw128_desc(kb, C, s), idn, true);
+          mma_commit(bar_y);
+        }
+        if (!cwait(bar_ops, ph_ops)) break;  // T Diag(beta) ready, S^T scaled by gamma_63
+        {  // U^T = Y^T (T Diag(beta))^T
           const uint32_t id = idesc_tf32(64);
           const uint32_t tb = smem_u32(sm + OFF_TB);
 #pragma unroll
-          for (int s = 0; s < C / 8; ++s) {
+          for (int s = 0; s < C / 8; ++s)
             mma_tf32_ts(tm + TM_X2, tm + TM_L + 8 * s, sw128_desc(tb, C, s), id, s > 0);
-            mma_tf32_ts(tm + TM_X1, tm + TM_L + 64 + 8 * s, sw128_desc(tb, C, s), id, s > 0);
-          }
-          mma_commit(bar_mma);
+          mma_commit(bar_u);
         }
-        if (!cwait(bar_ops, ph_ops)) break;  // W operand ready
-        {
-          const uint32_t idn = idesc_tf32(64, true);
-          const uint32_t wb = smem_u32(sm + OFF_R);
-#pragma unroll
-          for (int s = 0; s < DH / 8; ++s)
-            mma_tf32_ts(tm + TM_X2, tm + TM_S + 8 * s, sw128_desc(wb, C, s), idn, true);
-          mma_commit(bar_mma);
-        }
-        if (!cwait(bar_ops, ph_ops)) break;  // S^T scaled by gamma_63
+        // U^T is the A operand of the last two products: wait for it to land
+        if (!cwait(bar_u, ph_u)) break;
         {
           const uint32_t id64 = idesc_tf32(64), id128 = idesc_tf32(128);
           const uint32_t pb = smem_u32(sm + OFF_P), kb = smem_u32(sm + OFF_KHT);
@@ -287,7 +289,7 @@ __global__ void __launch_bounds__(NT + 32, 1)
     }
   } else {
     // ======================= 16 worker warps =======================
-    uint32_t ph_tma = 0, ph_ap[1] = {0}, ph_mma = 0;
+    uint32_t ph_tma = 0, ph_ap[1] = {0}, ph_y = 0, ph_mma = 0;
     auto wsync = [&]() { named_sync(1, NT); };
     // every worker waits, then the workers synchronise so an abort is seen by all
     auto wwait = [&](uint64_t *bar, uint32_t &ph) -> bool {
@@ -425,8 +427,8 @@ __global__ void __launch_bounds__(NT + 32, 1)
       const bool kside = l < C;
       const int i = l & (C - 1);
       float *Rs = reinterpret_cast<float *>(sm + OFF_R);  // [64][LDR] fp32 scratch
-      // thread = channel l, tokens 16g..16g+15: V^T and (gamma*K)^T (kept in registers
-      // until L* is free), Khat^T = k exp(G_63 - G) straight to its B operand
+      // thread = channel l, tokens 16g..16g+15: V^T and gamma*K (kept in registers until
+      // L* and gamma*Q are free), Khat^T = k exp(G_63 - G) straight to its B operand
       uint32_t vT2[8];
       float gkT[16];
       {
@@ -471,11 +473,14 @@ __global__ void __launch_bounds__(NT + 32, 1)
 #pragma unroll
         for (int j = 0; j < 16; ++j)
           vT[j] = __uint_as_float((j & 1) ? (vT2[j >> 1] & 0xFFFF0000u) : (vT2[j >> 1] << 16));
-        tmem_st16(tm + lane + TM_L + 16 * g, vT);  // L* is dead: the W / U~ A operands
+        tmem_st16(tm + lane + TM_L + 16 * g, vT);  // L* is dead: V^T starts Y^T
       }
-      tmem_st16(tm + lane + TM_L + 64 + 16 * g, gkT);
+      // gamma*Q has been read by the O^T product: its tile takes gamma*K (rows = tokens)
+#pragma unroll
+      for (int j = 0; j < 16; ++j)
+        *reinterpret_cast<float *>(sm + OFF_GQ + sw128_offset(C, 16 * g + j, l)) = gkT[j];
       tmem_wait_st();
-      warp_arrive(bar_raw);  // R'_a consumed: the next chunk's TMA may start
+      warp_arrive(bar_raw);  // R'_a consumed (next TMA may start); V^T and gamma*K ready
 
       // ---- a4: T = (I + Diag(beta) A)^-1 (blocked, fp32), P operand ------------
       float *Ms = reinterpret_cast<float *>(sm + OFF_MS);
@@ -590,22 +595,8 @@ __global__ void __launch_bounds__(NT + 32, 1)
               make_float4(v4[0], v4[1], v4[2], v4[3]);
         }
       }
-      warp_arrive(bar_ops);  // -> W^T, U~^T MMAs
-      if (!(ok = wwait(bar_mma, ph_mma))) break;
-
-      // ---- W operand (rows = tokens, K = key channels) from W^T ---------------
-      {
-        float w[16];
-        tmem_ld16(tm + lane + TM_X1 + 16 * g, w);
-        tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 16; ++j)
-          *reinterpret_cast<float *>(sm + OFF_R + sw128_offset(C, 16 * g + j, l)) = tf32_rna(w[j]);
-      }
-      warp_arrive(bar_ops);  // -> U^T -= S^T W^T, O^T = S^T (gQ)^T
-      if (!(ok = wwait(bar_mma, ph_mma))) break;
-
-      // ---- S^T <- S^T Diag(gamma_63): column c scaled by exp(G_63,c) -----------
+      // ---- S^T <- S^T Diag(gamma_63) once the O^T and Y^T products have read S^T ----
+      if (!(ok = wwait(bar_y, ph_y))) break;
       {
         float v[32];
         tmem_ld32(tm + lane + TM_S + 32 * g, v);
@@ -615,7 +606,7 @@ __global__ void __launch_bounds__(NT + 32, 1)
         tmem_st32(tm + lane + TM_S + 32 * g, v);
         tmem_wait_st();
       }
-      warp_arrive(bar_ops);  // -> O^T += U^T P^T, S^T += U^T Khat
+      warp_arrive(bar_ops);  // -> U^T, then O^T += U^T P^T, S^T += U^T Khat
       if (ci + 1 < n_chunks && !(ok = stage(ci + 1))) break;  // overlaps those MMAs
       if (!(ok = wwait(bar_mma, ph_mma))) break;
 
@@ -661,6 +652,10 @@ __global__ void __launch_bounds__(NT + 32, 1)
     // the CTA gave up: give in-flight copies and MMAs a bounded chance to land
     mbar_wait(bar_tma, 0, 100000000ull);
     mbar_wait(bar_tma, 1, 100000000ull);
+    mbar_wait(bar_y, 0, 100000000ull);
+    mbar_wait(bar_y, 1, 100000000ull);
+    mbar_wait(bar_u, 0, 100000000ull);
+    mbar_wait(bar_u, 1, 100000000ull);
     mbar_wait(bar_mma, 0, 100000000ull);
     mbar_wait(bar_mma, 1, 100000000ull);
   }
