@@ -148,10 +148,11 @@ __global__ void __launch_bounds__(NT + 32, 1)
   uint64_t *bar_opsap = bars + 2;    // workers -> control: A|P operands built (16 warps)
   uint64_t *bar_y = bars + 3;        // control -> workers: Y^T product done (S^T read)
   uint64_t *bar_ops = bars + 4;      // workers -> control: T Diag(beta) ready, S^T scaled
-  uint64_t *bar_ap = bars + 5;       // control -> workers: A|P and O^T products done
+  uint64_t *bar_ap = bars + 5;       // control -> workers: O^T and A|P products done
   uint64_t *bar_u = bars + 6;        // control -> control: U^T product done
   uint64_t *bar_mma = bars + 7;      // control -> workers: chunk's last products done
-  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bars + 8);
+  uint64_t *bar_st = bars + 8;       // workers -> control: chunk staged, previous O^T stored
+  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bars + 9);
   volatile int *s_abort = reinterpret_cast<volatile int *>(s_tmem + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane_id = tid & 31;
@@ -193,6 +194,7 @@ __global__ void __launch_bounds__(NT + 32, 1)
     mbar_init(bar_y, 1);
     mbar_init(bar_u, 1);
     mbar_init(bar_mma, 1);
+    mbar_init(bar_st, NT / 32);
     *s_abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -221,7 +223,7 @@ __global__ void __launch_bounds__(NT + 32, 1)
         for (int qd = 0; qd < 4; ++qd)
           tma_load_2d(sm + OFF_GRAW + 8192 * qd, &maps.g, h * DH + 32 * qd, y, bar_tma);
       };
-      uint32_t ph_raw = 0, ph_opsap[1] = {0}, ph_ops = 0, ph_u = 0;
+      uint32_t ph_raw = 0, ph_opsap[1] = {0}, ph_ops = 0, ph_u = 0, ph_st = 0;
       auto cwait = [&](uint64_t *bar, uint32_t &ph) -> bool {
         const bool good = *s_abort == 0 && mbar_wait(bar, ph);
         ph ^= 1u;
@@ -234,8 +236,17 @@ __global__ void __launch_bounds__(NT + 32, 1)
       };
       if (n_chunks > 0) issue_tma(0);
       for (int ci = 0; ci < n_chunks; ++ci) {
-        // A | P: row block a against its R'_a (N = 16(a+1)); four interleaved chains;
-        // then O^T = S^T (gamma Q)^T, which needs only the state and gamma*Q
+        // O^T = S^T (gamma Q)^T needs only the state and gamma*Q: issue it as soon as the
+        // chunk is staged, so it runs while the workers build the A|P operands
+        if (!cwait(bar_st, ph_st)) break;
+        {
+          const uint32_t id = idesc_tf32(64);
+          const uint32_t qb = smem_u32(sm + OFF_GQ);
+#pragma unroll
+          for (int s = 0; s < DH / 8; ++s)
+            mma_tf32_ts(tm + TM_O, tm + TM_S + 8 * s, sw128_desc(qb, C, s), id, s > 0);
+        }
+        // A | P: row block a against its R'_a (N = 16(a+1)); four interleaved chains
         if (!cwait(bar_opsap, ph_opsap[0])) break;
         {
           const uint32_t rp = smem_u32(sm);
@@ -246,11 +257,6 @@ __global__ void __launch_bounds__(NT + 32, 1)
               mma_tf32_ts(tm + ap_col(a), tm + TM_L + 8 * s, sw128_desc(rp + rp_off(a), 16 * (a + 1), s),
                           idesc_tf32(16 * (a + 1)), s > 0);
           }
-          const uint32_t id = idesc_tf32(64);
-          const uint32_t qb = smem_u32(sm + OFF_GQ);
-#pragma unroll
-          for (int s = 0; s < DH / 8; ++s)
-            mma_tf32_ts(tm + TM_O, tm + TM_S + 8 * s, sw128_desc(qb, C, s), id, s > 0);
           mma_commit(bar_ap);  // gamma*Q and the R'_a operands are free after this
         }
         // raw tiles consumed, V^T in TMEM, gamma*K in shared memory
@@ -427,6 +433,7 @@ __global__ void __launch_bounds__(NT + 32, 1)
       const bool kside = l < C;
       const int i = l & (C - 1);
       float *Rs = reinterpret_cast<float *>(sm + OFF_R);  // [64][LDR] fp32 scratch
+      warp_arrive(bar_st);  // gamma*Q built, the previous chunk's O^T read: -> O^T
       // thread = channel l, tokens 16g..16g+15: V^T and gamma*K (kept in registers until
       // L* and gamma*Q are free), Khat^T = k exp(G_63 - G) straight to its B operand
       uint32_t vT2[8];
