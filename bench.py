@@ -290,6 +290,12 @@ def run_ours(args, world, rank, local):
     inp = workload_inputs(dev, seed=rank, n_req=args.prefill_requests)
     T, H, dk, dv = inp.total_tokens, 32, 128, 128
     n_req = inp.n_req
+    if args.backward_only:  # the backward leg alone (for a launch list of its kernels)
+        peaks, _ = load_peaks()
+        out = bench_backward(args, inp, dev, peaks, world)
+        if rank == 0:
+            print(json.dumps({"impl": "ours", "backward": out}), flush=True)
+        return
     cu_host = torch.tensor([0] + list(__import__("itertools").accumulate(inp.lengths)),
                            dtype=torch.int32)
     o = torch.empty(T, H, dv, device=dev)
@@ -619,6 +625,8 @@ def main():
     ap.add_argument("--no-decode", action="store_true")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--backward-only", action="store_true",
+                    help="run only the backward leg of the headline workload and print it")
     ap.add_argument("--no-extra", action="store_true",
                     help="skip the single-sequence and million-token measurements")
     ap.add_argument("--prefill-requests", type=int, default=None,
