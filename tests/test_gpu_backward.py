@@ -104,3 +104,52 @@ def test_backward_through_the_simt_forward(monkeypatch):
     got = _run_gpu(inp, d_o, d_fin)
     for name in GRADS + ("d_initial",):
         assert rel_err(got[name], ref[name]) <= TOL_BF16, name
+
+
+@pytest.mark.slow
+def test_backward_varlen_full_size():
+    """The headline workload (64 requests, lengths log-uniform on [128, 4096], H=32,
+    d=128) at full size, in the launch configuration bench.py times; the oracle's
+    derivative on 6 sampled chains (the longest and shortest request and 4 random
+    (request, head) pairs), each packed as a one-head request."""
+    import random
+    inp = I.varlen(device=DEV)
+    T, H, d, n = inp.total_tokens, 32, 128, inp.n_req
+    gen = torch.Generator().manual_seed(61)
+    d_o = torch.randn((T, H, d), generator=gen)
+    d_fin = torch.randn((n, H, d, d), generator=gen)
+    got = kda.prefill_backward(inp.q, inp.k, inp.v, inp.g, inp.beta, inp.cu_seqlens,
+                               d_o=d_o.to(DEV), d_final=d_fin.to(DEV),
+                               cu_seqlens_host=inp.cu_seqlens.cpu())
+    torch.cuda.synchronize()
+    lens = inp.lengths
+    rng = random.Random(1)
+    pairs = [(int(np.argmax(lens)), 3), (int(np.argmin(lens)), 17)]
+    pairs += [(rng.randrange(n), rng.randrange(H)) for _ in range(4)]
+    cu = [int(c) for c in inp.cu_seqlens.cpu().tolist()]
+    parts = {k: [] for k in ("q", "k", "v", "g", "beta", "d_o")}
+    for (r, h) in pairs:
+        lo, hi = cu[r], cu[r + 1]
+        for name in ("q", "k", "v", "g"):
+            parts[name].append(getattr(inp, name)[lo:hi, h:h + 1].cpu())
+        parts["beta"].append(inp.beta[lo:hi, h:h + 1].cpu())
+        parts["d_o"].append(d_o[lo:hi, h:h + 1])
+    cat = {k: torch.cat(v, 0) for k, v in parts.items()}
+    pcu = np.concatenate([[0], np.cumsum([cu[r + 1] - cu[r] for r, _ in pairs])])
+    dfin = torch.stack([d_fin[r, h:h + 1] for r, h in pairs], 0)
+    ref = oracle.prefill_backward(cat["q"], cat["k"], cat["v"], cat["g"], cat["beta"], pcu,
+                                  None, cat["d_o"], dfin)
+    for c, (r, h) in enumerate(pairs):
+        lo, hi = cu[r], cu[r + 1]
+        plo, phi = int(pcu[c]), int(pcu[c + 1])
+        for name in GRADS:
+            g_gpu = got[name][lo:hi, h]
+            g_ref = ref[name][plo:phi, 0]
+            assert rel_err(g_gpu, g_ref) <= TOL_BF16, (name, r, h, rel_err(g_gpu, g_ref))
+        # with strong decay a whole request's decay can take dS_0 below the fp32 range
+        d0_ref = np.asarray(ref["d_initial"][c, 0])
+        d0 = got["d_initial"][r, h].double().cpu().numpy()
+        if np.abs(d0_ref).max() < 1e-30:
+            assert np.abs(d0).max() < 1e-30, (r, h)
+        else:
+            assert rel_err(d0, d0_ref) <= TOL_BF16, (r, h)
