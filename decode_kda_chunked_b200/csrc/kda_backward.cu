@@ -69,7 +69,9 @@ struct BwdParams {
 // Slices of 16 along k are staged through shared memory `stage`
 // (16 (16 MI + 1) + 16 (16 NJ + 1) floats) so the inner loop reads
 // conflict-free shared memory; the next slice is loaded into registers while
-// the current one is multiplied.  Every thread of the CTA must call it.
+// the current one is multiplied.  Every thread of the CTA must call it; it
+// synchronises the CTA before its first load, so operands written by the CTA
+// just before the call are complete.
 template <int MI, int NJ>
 __device__ void mm_acc(float (&acc)[MI][NJ], const float *A, int am, int ak, const float *B,
                        int bk, int bn, int K, float *stage) {
@@ -100,6 +102,7 @@ __device__ void mm_acc(float (&acc)[MI][NJ], const float *A, int am, int ak, con
       rb[q] = B[(size_t)(k0 + kk) * bk + (size_t)n * bn];
     }
   };
+  __syncthreads();  // operands the CTA has just written are complete before the first fetch
   fetch(0);
   for (int k0 = 0; k0 < K; k0 += 16) {
     __syncthreads();  // the previous slice has been consumed
@@ -145,11 +148,39 @@ constexpr int stage_floats(int M, int N) { return 16 * (M + 1) + 16 * (N + 1); }
 
 // Rows tok0 .. tok0 + n - 1 of a token-major [T, H, D] tensor into a [64][ld]
 // fp32 tile (rows >= n are zero: the exact no-op padding of the chunk form).
+// 16-byte loads, all of a thread's loads issued before any of its stores.
+__device__ __forceinline__ void unpack16(const uint4 &u, const float *, float (&x)[4]) {
+  x[0] = __uint_as_float(u.x); x[1] = __uint_as_float(u.y);
+  x[2] = __uint_as_float(u.z); x[3] = __uint_as_float(u.w);
+}
+__device__ __forceinline__ void unpack16(const uint4 &u, const __nv_bfloat16 *, float (&x)[8]) {
+  const uint32_t w[4] = {u.x, u.y, u.z, u.w};
+#pragma unroll
+  for (int q = 0; q < 4; ++q) {
+    x[2 * q] = __uint_as_float(w[q] << 16);
+    x[2 * q + 1] = __uint_as_float(w[q] & 0xFFFF0000u);
+  }
+}
 template <int D, typename TIn>
 __device__ void stage_rows(float *dst, int ld, const TIn *src, int tok0, int n, int H, int h) {
-  for (int e = threadIdx.x; e < C * D; e += NTH) {
-    const int t = e / D, c = e % D;
-    dst[t * ld + c] = (src && t < n) ? load_elem(src, ((size_t)(tok0 + t) * H + h) * D + c) : 0.f;
+  constexpr int VEC = 16 / (int)sizeof(TIn);  // elements per 16-byte load
+  constexpr int PER_ROW = D / VEC, ITER = C * PER_ROW / NTH;
+  static_assert(ITER * NTH == C * PER_ROW, "tile must split evenly over the CTA");
+  uint4 buf[ITER];
+#pragma unroll
+  for (int it = 0; it < ITER; ++it) {
+    const int e = threadIdx.x + it * NTH, t = e / PER_ROW, cv = e % PER_ROW;
+    buf[it] = (src && t < n)
+                  ? *reinterpret_cast<const uint4 *>(src + ((size_t)(tok0 + t) * H + h) * D + cv * VEC)
+                  : make_uint4(0u, 0u, 0u, 0u);
+  }
+#pragma unroll
+  for (int it = 0; it < ITER; ++it) {
+    const int e = threadIdx.x + it * NTH, t = e / PER_ROW, cv = e % PER_ROW;
+    float x[VEC];
+    unpack16(buf[it], src, x);
+#pragma unroll
+    for (int q = 0; q < VEC; ++q) dst[t * ld + cv * VEC + q] = x[q];
   }
 }
 
@@ -252,21 +283,18 @@ __global__ void __launch_bounds__(NTH, 1) bwd_prep_kernel(const BwdParams p) {
   }
   __syncthreads();
 
-  // T = (I + Diag(beta) A)^-1 by forward substitution, one column per thread
-  if (tid < C) {
-    const int j = tid;
+  // T = (I + Diag(beta) A)^-1 by forward substitution: column j = tid / 4, its four
+  // threads split each row's sum (s = j + part, j + part + 4, ...) and combine it
+  // with two shuffles inside their aligned group of four lanes
+  {
+    const int j = tid >> 2, part = tid & 3;
     for (int i = 0; i < C; ++i) {
-      float tv;
-      if (i < j) {
-        tv = 0.f;
-      } else if (i == j) {
-        tv = 1.f;
-      } else {
-        float acc = 0.f;
-        for (int s = j; s < i; ++s) acc = fmaf(sA[i * C + s], sT[s * C + j], acc);
-        tv = -sB[i] * acc;
-      }
-      sT[i * C + j] = tv;
+      float acc = 0.f;
+      for (int s = j + part; s < i; s += 4) acc = fmaf(sA[i * C + s], sT[s * C + j], acc);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+      acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+      if (part == 0) sT[i * C + j] = i < j ? 0.f : (i == j ? 1.f : -sB[i] * acc);
+      __syncwarp();
     }
   }
   __syncthreads();
@@ -433,8 +461,8 @@ struct GradLayout {
   static constexpr int oK = 0, oQ = oK + C * D, oV = oQ + C * D, oO = oV + C * D;
   static constexpr int oG = oO + C * D, oP = oG + C * D, oT = oP + C * C;
   static constexpr int oStage = oT + C * C, oB = oStage + stage_floats(C, D);
-  static constexpr int oDb = oB + C, oX = oDb + C, oPart = oX + D;
-  static constexpr int total = oPart + 16 * D;
+  static constexpr int oDb = oB + C, oX = oDb + C, oPart = oX + D, oGam = oPart + 16 * D;
+  static constexpr int total = oGam + D;
   static constexpr size_t bytes = sizeof(float) * total;
 };
 
@@ -447,6 +475,7 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
   float *sK = sm + L::oK, *sQ = sm + L::oQ, *sV = sm + L::oV, *sO = sm + L::oO;
   float *sG = sm + L::oG, *sP = sm + L::oP, *sT = sm + L::oT, *sStage = sm + L::oStage;
   float *sB = sm + L::oB, *sDb = sm + L::oDb, *sExtra = sm + L::oX, *sPart = sm + L::oPart;
+  float *sGam = sm + L::oGam;
   const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
   const int H = p.H;
   const int jc = blockIdx.x / H, h = blockIdx.x % H;
@@ -527,13 +556,29 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
     }
     sPart[ty * D + tx + 16 * j] = colsum;
   }
+  // dGam = rowsum(dSn * S): warp w takes rows w, w + 8, ...; lanes walk the row
+  {
+    const int w = tid >> 5, ln = tid & 31;
+#pragma unroll 4
+    for (int row = w; row < D; row += NTH / 32) {
+      float a[D / 32], b[D / 32];
+#pragma unroll
+      for (int q = 0; q < D / 32; ++q) {
+        a[q] = dSn[(size_t)row * D + ln + 32 * q];
+        b[q] = S[(size_t)row * D + ln + 32 * q];
+      }
+      float v = 0.f;
+#pragma unroll
+      for (int q = 0; q < D / 32; ++q) v = fmaf(a[q], b[q], v);
+#pragma unroll
+      for (int off = 16; off > 0; off >>= 1) v += __shfl_xor_sync(0xffffffffu, v, off);
+      if (ln == 0) sGam[row] = v;
+    }
+  }
   __syncthreads();
-  // dGam = rowsum(dSn * S)  ->  dG_last += dGam Gam;  the partial column sums in a
-  // fixed order, so the result is the same on every run
+  // dG_last += dGam Gam + the partial column sums, in a fixed order (same on every run)
   if (tid < D) {
-    float s = 0.f;
-    for (int jj = 0; jj < D; ++jj) s = fmaf(dSn[(size_t)tid * D + jj], S[(size_t)tid * D + jj], s);
-    float e = s * exp2f(G63[tid]);
+    float e = sGam[tid] * exp2f(G63[tid]);
     for (int y = 0; y < 16; ++y) e += sPart[y * D + tid];
     sExtra[tid] = e;
   }
@@ -600,7 +645,15 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
   for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int j = 0; j < NJ; ++j) sO[(ty + 16 * i) * D + tx + 16 * j] = -acc[i][j];
-  for (int e = tid; e < C * C; e += NTH) sT[e] = p.wT[ch * C * C + e];
+  {
+    float4 tv[C * C / 4 / NTH];
+#pragma unroll
+    for (int q = 0; q < C * C / 4 / NTH; ++q)
+      tv[q] = reinterpret_cast<const float4 *>(p.wT + ch * C * C)[tid + q * NTH];
+#pragma unroll
+    for (int q = 0; q < C * C / 4 / NTH; ++q)
+      reinterpret_cast<float4 *>(sT)[tid + q * NTH] = tv[q];
+  }
   // T^T dU -> dV = Diag(beta) T^T dU, dbeta += (T^T dU) . v
   zero(acc);
   mm_acc<4, NJ>(acc, sT, 1, C, dU, D, 1, C, sStage);
@@ -660,6 +713,11 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
   }
   // dZ = -T^T (dT T^T);  dA = tril_strict(Diag(beta) dZ);  dbeta += sum_s dZ_ts A_ts
   {
+    float av[4][4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < 4; ++j) av[i][j] = p.wA[ch * C * C + (ty + 16 * i) * C + tx + 16 * j];
     float tt[4][4];
     zero(tt);
     mm_acc<4, 4>(tt, sP, C, 1, sT, 1, C, C, sStage);
@@ -678,7 +736,7 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
         const int s = tx + 16 * j;
         const float dz = -tt[i][j];
         const bool low = s < t;
-        if (low) rs = fmaf(dz, p.wA[ch * C * C + t * C + s], rs);
+        if (low) rs = fmaf(dz, av[i][j], rs);
         sP[t * C + s] = low ? sB[t] * dz : 0.f;
       }
       rs = row_sum16(rs);
