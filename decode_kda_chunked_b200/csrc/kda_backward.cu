@@ -16,8 +16,8 @@
 //   per chunk, all chunks in parallel:
 //     d(gamma Q) = dO S^T      dP = tril(dO U^T)      dKhat = U dSn^T      dW = -dU S^T
 //     dV = Diag(beta) T^T dU   d(gamma K) = Diag(beta) T^T dW
-//     dT = dU (Diag(beta) V)^T + dW (Diag(beta) gamma K)^T
-//     dZ = -T^T dT T^T         dA = tril_strict(Diag(beta) dZ)
+//     dT = dU (Diag(beta) V)^T + dW (Diag(beta) gamma K)^T, which T^-1 maps to
+//     dZ = -T^T dT T^T = -[(T^T dU) U~^T + (T^T dW) W^T]   dA = tril_strict(Diag(beta) dZ)
 //     dbeta_t = (T^T dU)_t . v_t + (T^T dW)_t . (gamma k)_t + sum_s dZ_ts A_ts
 //     A and P are gated Gram products; their cotangents reach K, Q and the
 //     cumulative gate through sums  sum_s M_ts x_s exp(G_t - G_s)  (t >= s),
@@ -60,6 +60,7 @@ struct BwdParams {
   const float *snaps;          // [n_snap, H, D, D]
   const float *zero_state;     // D x D zeros
   float *wA, *wT, *wW, *wU, *wKh, *wX, *wY, *wGam;
+  float *wU2;                  // U = U~ - W S per (chunk, head), written by the gradient pass
   int n_req, n_chunks, H;
 };
 
@@ -490,7 +491,8 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
   const float *dSn = p.wY + ch * D * D;
   const float *dU = p.wX + ch * C * D;
   const float *W = p.wW + ch * C * D;
-  float *U = p.wU + ch * C * D;
+  const float *Ut = p.wU + ch * C * D;
+  float *U = p.wU2 + ch * C * D;
 
   stage_rows<D, TIn>(sK, D, static_cast<const TIn *>(p.k), tok0, n, H, h);
   stage_rows<D, TIn>(sQ, D, static_cast<const TIn *>(p.q), tok0, n, H, h);
@@ -503,7 +505,12 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
   float accQ[4][NJ], accK[4][NJ], accG[4][NJ], acc[4][NJ];
   const float *G63 = sG + (C - 1) * D;
 
-  // U = U~ - W S (in place)
+  // U = U~ - W S  (U~ loaded before the product so its latency hides under it)
+  float ut[4][NJ];
+#pragma unroll
+  for (int i = 0; i < 4; ++i)
+#pragma unroll
+    for (int j = 0; j < NJ; ++j) ut[i][j] = Ut[(ty + 16 * i) * D + tx + 16 * j];
   zero(acc);
   mm_acc<4, NJ>(acc, W, D, 1, S, D, 1, D, sStage);
 #pragma unroll
@@ -511,7 +518,7 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
 #pragma unroll
     for (int j = 0; j < NJ; ++j) {
       const int e = (ty + 16 * i) * D + tx + 16 * j;
-      U[e] = U[e] - acc[i][j];
+      U[e] = ut[i][j] - acc[i][j];
     }
   // d(gamma Q) = dO S^T  ->  dQ = d(gamma Q) gamma,  dG = d(gamma Q) gamma q
   zero(acc);
@@ -583,61 +590,6 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
     sExtra[tid] = e;
   }
 
-  // gated products of dP:  P1_t = sum_{s<=t} dP_ts k_s e^{G_t-G_s},  P2_s = sum_{t>=s} dP_ts q_t e^{G_t-G_s}
-  // (the shared-memory dO tile is dead from here on and holds the gate tables)
-#pragma unroll
-  for (int b = 0; b < 4; ++b) {
-    const int r0 = 16 * b, r1 = r0 + 15;
-    __syncthreads();
-    for (int e = tid; e < (r0 + 16) * D; e += NTH) {
-      const int c = e % D;
-      sO[e] = sK[e] * exp2f(sG[r0 * D + c] - sG[e]);
-    }
-    __syncthreads();
-    {
-      const int t = r0 + ty;
-      float o1[NJ];
-#pragma unroll
-      for (int j = 0; j < NJ; ++j) o1[j] = 0.f;
-      for (int s = 0; s <= t; ++s) {
-        const float dp = sP[t * C + s];
-#pragma unroll
-        for (int j = 0; j < NJ; ++j) o1[j] = fmaf(dp, sO[s * D + tx + 16 * j], o1[j]);
-      }
-#pragma unroll
-      for (int j = 0; j < NJ; ++j) {
-        const int c = tx + 16 * j, e = t * D + c;
-        const float p1 = o1[j] * exp2f(sG[e] - sG[r0 * D + c]);
-        accQ[b][j] += p1;
-        accG[b][j] = fmaf(sQ[e], p1, accG[b][j]);
-      }
-    }
-    __syncthreads();
-    for (int e = r0 * D + tid; e < C * D; e += NTH) {
-      const int c = e % D;
-      sO[e] = sQ[e] * exp2f(sG[e] - sG[r1 * D + c]);
-    }
-    __syncthreads();
-    {
-      const int s = r0 + ty;
-      float o2[NJ];
-#pragma unroll
-      for (int j = 0; j < NJ; ++j) o2[j] = 0.f;
-      for (int t = s; t < C; ++t) {
-        const float dp = sP[t * C + s];
-#pragma unroll
-        for (int j = 0; j < NJ; ++j) o2[j] = fmaf(dp, sO[t * D + tx + 16 * j], o2[j]);
-      }
-#pragma unroll
-      for (int j = 0; j < NJ; ++j) {
-        const int c = tx + 16 * j, e = s * D + c;
-        const float p2 = o2[j] * exp2f(sG[r1 * D + c] - sG[e]);
-        accK[b][j] += p2;
-        accG[b][j] = fmaf(-sK[e], p2, accG[b][j]);
-      }
-    }
-  }
-
   // dW = -dU S^T (into the dO tile)
   zero(acc);
   mm_acc<4, NJ>(acc, dU, D, 1, S, 1, D, D, sStage);
@@ -665,6 +617,7 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
     for (int j = 0; j < NJ; ++j) {
       const int c = tx + 16 * j;
       rs = fmaf(acc[i][j], sV[t * D + c], rs);
+      sV[t * D + c] = acc[i][j];  // the V tile now holds T^T dU (own elements only)
       if (t < n) p.dv[((size_t)(tok0 + t) * H + h) * D + c] = sB[t] * acc[i][j];
     }
     rs = row_sum16(rs);
@@ -685,33 +638,13 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
       accK[i][j] = fmaf(dkg, exp2f(sG[e]), accK[i][j]);
       accG[i][j] = fmaf(dkg, kg, accG[i][j]);
       rs = fmaf(acc[i][j], kg, rs);
+      sO[e] = acc[i][j];  // the dO tile (dW) now holds T^T dW (own elements only)
     }
     rs = row_sum16(rs);
     if (tx == 0) sDb[t] += rs;
   }
-  // dT = dU (Diag(beta) V)^T + dW (Diag(beta) gamma K)^T   (into the dP tile)
-  {
-    float tt[4][4];
-    zero(tt);
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < NJ; ++j) sV[(ty + 16 * i) * D + tx + 16 * j] *= sB[ty + 16 * i];
-    mm_acc<4, 4>(tt, dU, D, 1, sV, 1, D, D, sStage);
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < NJ; ++j) {
-        const int e = (ty + 16 * i) * D + tx + 16 * j;
-        sV[e] = sB[ty + 16 * i] * exp2f(sG[e]) * sK[e];
-      }
-    mm_acc<4, 4>(tt, sO, D, 1, sV, 1, D, D, sStage);
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) sP[(ty + 16 * i) * C + tx + 16 * j] = tt[i][j];
-  }
-  // dZ = -T^T (dT T^T);  dA = tril_strict(Diag(beta) dZ);  dbeta += sum_s dZ_ts A_ts
+  // dZ = -[(T^T dU) U~^T + (T^T dW) W^T];  dA = tril_strict(Diag(beta) dZ) into the T tile;
+  // dbeta += sum_{s<t} dZ_ts A_ts
   {
     float av[4][4];
 #pragma unroll
@@ -720,13 +653,8 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
       for (int j = 0; j < 4; ++j) av[i][j] = p.wA[ch * C * C + (ty + 16 * i) * C + tx + 16 * j];
     float tt[4][4];
     zero(tt);
-    mm_acc<4, 4>(tt, sP, C, 1, sT, 1, C, C, sStage);
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < 4; ++j) sV[(ty + 16 * i) * C + tx + 16 * j] = tt[i][j];
-    zero(tt);
-    mm_acc<4, 4>(tt, sT, 1, C, sV, C, 1, C, sStage);
+    mm_acc<4, 4>(tt, sV, D, 1, Ut, 1, D, D, sStage);
+    mm_acc<4, 4>(tt, sO, D, 1, W, 1, D, D, sStage);
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int t = ty + 16 * i;
@@ -737,14 +665,21 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
         const float dz = -tt[i][j];
         const bool low = s < t;
         if (low) rs = fmaf(dz, av[i][j], rs);
-        sP[t * C + s] = low ? sB[t] * dz : 0.f;
+        sT[t * C + s] = low ? sB[t] * dz : 0.f;  // dA (T is no longer needed)
       }
       rs = row_sum16(rs);
       if (tx == 0) sDb[t] += rs;
     }
   }
 
-  // gated products of dA:  A1_t = sum_{s<t} dA_ts k_s e^{G_t-G_s},  A2_s = sum_{t>s} dA_ts k_t e^{G_t-G_s}
+  // Gated Gram cotangents of P (dP in the P tile) and A (dA in the T tile), one row
+  // block at a time, with the block factorisation of exp(G_t - G_s), t >= s:
+  //   lower (row t of block b, reference r0 = 16 b):
+  //     P1_t = sum_{s<=t} dP_ts k_s e^{G_t-G_s}  -> dq, dG += q P1
+  //     A1_t = sum_{s<t}  dA_ts k_s e^{G_t-G_s}  -> dk, dG += k A1     (one k table)
+  //   upper (row s of block b, reference r1 = 16 b + 15):
+  //     P2_s + A2_s = sum_{t>=s} (dP_ts q_t + dA_ts k_t) e^{G_t-G_s}  -> dk, dG -= k (P2 + A2)
+  // The dO and V tiles are dead here and hold the gate tables.
 #pragma unroll
   for (int b = 0; b < 4; ++b) {
     const int r0 = 16 * b, r1 = r0 + 15;
@@ -756,44 +691,53 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
     __syncthreads();
     {
       const int t = r0 + ty;
-      float o1[NJ];
+      float op[NJ], oa[NJ];
 #pragma unroll
-      for (int j = 0; j < NJ; ++j) o1[j] = 0.f;
-      for (int s = 0; s < t; ++s) {
-        const float da = sP[t * C + s];
+      for (int j = 0; j < NJ; ++j) op[j] = oa[j] = 0.f;
+      for (int s2 = 0; s2 <= t; ++s2) {
+        const float dp = sP[t * C + s2], da = sT[t * C + s2];
 #pragma unroll
-        for (int j = 0; j < NJ; ++j) o1[j] = fmaf(da, sO[s * D + tx + 16 * j], o1[j]);
+        for (int j = 0; j < NJ; ++j) {
+          const float tb = sO[s2 * D + tx + 16 * j];
+          op[j] = fmaf(dp, tb, op[j]);
+          oa[j] = fmaf(da, tb, oa[j]);
+        }
       }
 #pragma unroll
       for (int j = 0; j < NJ; ++j) {
         const int c = tx + 16 * j, e = t * D + c;
-        const float a1 = o1[j] * exp2f(sG[e] - sG[r0 * D + c]);
+        const float f = exp2f(sG[e] - sG[r0 * D + c]);
+        const float p1 = op[j] * f, a1 = oa[j] * f;
+        accQ[b][j] += p1;
         accK[b][j] += a1;
-        accG[b][j] = fmaf(sK[e], a1, accG[b][j]);
+        accG[b][j] = fmaf(sQ[e], p1, fmaf(sK[e], a1, accG[b][j]));
       }
     }
     __syncthreads();
     for (int e = r0 * D + tid; e < C * D; e += NTH) {
       const int c = e % D;
-      sO[e] = sK[e] * exp2f(sG[e] - sG[r1 * D + c]);
+      const float f = exp2f(sG[e] - sG[r1 * D + c]);
+      sO[e] = sQ[e] * f;
+      sV[e] = sK[e] * f;
     }
     __syncthreads();
     {
-      const int s = r0 + ty;
+      const int s2 = r0 + ty;
       float o2[NJ];
 #pragma unroll
       for (int j = 0; j < NJ; ++j) o2[j] = 0.f;
-      for (int t = s + 1; t < C; ++t) {
-        const float da = sP[t * C + s];
+      for (int t = s2; t < C; ++t) {
+        const float dp = sP[t * C + s2], da = sT[t * C + s2];
 #pragma unroll
-        for (int j = 0; j < NJ; ++j) o2[j] = fmaf(da, sO[t * D + tx + 16 * j], o2[j]);
+        for (int j = 0; j < NJ; ++j)
+          o2[j] = fmaf(dp, sO[t * D + tx + 16 * j], fmaf(da, sV[t * D + tx + 16 * j], o2[j]));
       }
 #pragma unroll
       for (int j = 0; j < NJ; ++j) {
-        const int c = tx + 16 * j, e = s * D + c;
-        const float a2 = o2[j] * exp2f(sG[r1 * D + c] - sG[e]);
-        accK[b][j] += a2;
-        accG[b][j] = fmaf(-sK[e], a2, accG[b][j]);
+        const int c = tx + 16 * j, e = s2 * D + c;
+        const float v2 = o2[j] * exp2f(sG[r1 * D + c] - sG[e]);
+        accK[b][j] += v2;
+        accG[b][j] = fmaf(-sK[e], v2, accG[b][j]);
       }
     }
   }
@@ -854,7 +798,7 @@ cudaError_t launch_bwd_d(const BwdParams &p, cudaStream_t stream) {
 // Workspace carve-up shared by the size query and the launch.
 struct BwdWorkspace {
   size_t off_chunks, off_cu_chunks, off_cu_snap, off_snaps, off_zero;
-  size_t off_A, off_T, off_W, off_U, off_Kh, off_X, off_Y, off_Gam, total;
+  size_t off_A, off_T, off_W, off_U, off_Kh, off_X, off_Y, off_Gam, off_U2, total;
 };
 
 static size_t a256(size_t x) { return (x + 255) & ~size_t(255); }
@@ -877,6 +821,7 @@ BwdWorkspace backward_workspace(int n_req, int n_chunks, int n_snap, int H, int 
   w.off_X = take(nch * C * D * f);
   w.off_Y = take(nch * (size_t)D * D * f);
   w.off_Gam = take(nch * D * f);
+  w.off_U2 = take(nch * C * D * f);
   w.total = o;
   return w;
 }
@@ -902,6 +847,7 @@ cudaError_t launch_backward(const BackwardLaunch &b, cudaStream_t stream) {
   p.wX = reinterpret_cast<float *>(ws + w.off_X);
   p.wY = reinterpret_cast<float *>(ws + w.off_Y);
   p.wGam = reinterpret_cast<float *>(ws + w.off_Gam);
+  p.wU2 = reinterpret_cast<float *>(ws + w.off_U2);
   p.n_req = b.n_req; p.n_chunks = b.n_chunks; p.H = b.H;
   if (b.D == 128)
     return b.in_dtype == KDA_BF16 ? launch_bwd_d<128, __nv_bfloat16>(p, stream)
