@@ -284,18 +284,40 @@ __global__ void __launch_bounds__(NTH, 1) bwd_prep_kernel(const BwdParams p) {
   }
   __syncthreads();
 
-  // T = (I + Diag(beta) A)^-1 by forward substitution: column j = tid / 4, its four
-  // threads split each row's sum (s = j + part, j + part + 4, ...) and combine it
-  // with two shuffles inside their aligned group of four lanes
+  // T = (I + Diag(beta) A)^-1, blocked.  (1) The four 16x16 diagonal blocks by forward
+  // substitution: column task j = tid / 4 (block j / 16), its four threads split each
+  // row's sum and combine it with two shuffles inside their aligned group of four.
+  // (2) The blocks below the diagonal, one block diagonal d at a time:
+  //     T_ab = -T_aa sum_{c=b}^{a-1} N_ac T_cb,  N = Diag(beta) A,  b = a - d.
   {
-    const int j = tid >> 2, part = tid & 3;
-    for (int i = 0; i < C; ++i) {
+    const int task = tid >> 2, part = tid & 3;
+    const int o = 16 * (task >> 4), j = o + (task & 15);
+    for (int i = o; i < o + 16; ++i) {
       float acc = 0.f;
       for (int s = j + part; s < i; s += 4) acc = fmaf(sA[i * C + s], sT[s * C + j], acc);
       acc += __shfl_xor_sync(0xffffffffu, acc, 1);
       acc += __shfl_xor_sync(0xffffffffu, acc, 2);
       if (part == 0) sT[i * C + j] = i < j ? 0.f : (i == j ? 1.f : -sB[i] * acc);
       __syncwarp();
+    }
+    for (int e = tid; e < C * C; e += NTH)  // blocks above the diagonal
+      if ((e / C) >> 4 < (e % C) >> 4) sT[e] = 0.f;
+    float *Ys = sBuf;  // [3][16][17] scratch: N_a. T_.b of one block diagonal
+    for (int d = 1; d < 4; ++d) {
+      __syncthreads();
+      for (int a = d; a < 4; ++a) {
+        const int bb = a - d, i = 16 * a + ty, jc = 16 * bb + tx;
+        float y = 0.f;
+        for (int s2 = 16 * bb; s2 < 16 * a; ++s2) y = fmaf(sA[i * C + s2], sT[s2 * C + jc], y);
+        Ys[(bb * 16 + ty) * 17 + tx] = sB[i] * y;
+      }
+      __syncthreads();
+      for (int a = d; a < 4; ++a) {
+        const int bb = a - d, i = 16 * a + ty, jc = 16 * bb + tx;
+        float t = 0.f;
+        for (int r = 16 * a; r <= i; ++r) t = fmaf(sT[i * C + r], Ys[(bb * 16 + r - 16 * a) * 17 + tx], t);
+        sT[i * C + jc] = -t;
+      }
     }
   }
   __syncthreads();
