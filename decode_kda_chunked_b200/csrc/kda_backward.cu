@@ -247,6 +247,8 @@ __global__ void __launch_bounds__(NTH, 1) bwd_prep_kernel(const BwdParams p) {
 
   // A (strict lower) and P (inclusive lower), row block b at a time:
   // A_ts = sum_c [k_tc exp(G_tc - G_rc)] [k_sc exp(G_rc - G_sc)], r = 16 b.
+  // Unrolled over b, so the thread's valid column groups (jj <= b) are fixed.
+#pragma unroll
   for (int b = 0; b < 4; ++b) {
     const int r0 = 16 * b, rows = r0 + 16;
     __syncthreads();
@@ -262,16 +264,14 @@ __global__ void __launch_bounds__(NTH, 1) bwd_prep_kernel(const BwdParams p) {
     }
     __syncthreads();
     float a[4] = {0.f, 0.f, 0.f, 0.f}, pp[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
     for (int c = 0; c < D; ++c) {
       const float kl = sKL[ty * LDP + c], ql = sQL[ty * LDP + c];
 #pragma unroll
-      for (int jj = 0; jj < 4; ++jj) {
-        const int s = tx + 16 * jj;
-        if (s < rows) {
-          const float tv = sBuf[s * LDP + c];
-          a[jj] = fmaf(kl, tv, a[jj]);
-          pp[jj] = fmaf(ql, tv, pp[jj]);
-        }
+      for (int jj = 0; jj <= b; ++jj) {
+        const float tv = sBuf[(tx + 16 * jj) * LDP + c];
+        a[jj] = fmaf(kl, tv, a[jj]);
+        pp[jj] = fmaf(ql, tv, pp[jj]);
       }
     }
     const int t = r0 + ty;
