@@ -76,7 +76,14 @@ struct BwdParams {
 template <int MI, int NJ>
 __device__ void mm_acc(float (&acc)[MI][NJ], const float *A, int am, int ak, const float *B,
                        int bk, int bn, int K, float *stage) {
-  constexpr int M = 16 * MI, N = 16 * NJ, LA = M + 1, LB = N + 1;
+  static_assert(MI % 4 == 0 && NJ % 4 == 0, "rows and columns load as float4 runs");
+  constexpr int M = 16 * MI, N = 16 * NJ;
+  // Staged slices are stored permuted so a thread's MI rows (ty + 16 i) and NJ columns
+  // (tx + 16 j) sit side by side: row m at MI (m % 16) + m / 16; column n at
+  // NJ (n % 16) + n / 16, plus 4 floats per group of four threads when NJ = 8, which
+  // keeps every quarter-warp's 16-byte loads on distinct banks.
+  constexpr int PADB = NJ >= 8 ? 4 : 0;
+  constexpr int LA = M + 4, LB = N + 4 * PADB + 4;
   float *As = stage, *Bs = stage + 16 * LA;
   const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
   // each thread moves MI elements of the A slice and NJ of the B slice; the
@@ -88,6 +95,8 @@ __device__ void mm_acc(float (&acc)[MI][NJ], const float *A, int am, int ak, con
   auto b_at = [&](int e, int &kk, int &n) {
     if (b_n_inner) { n = e % N; kk = e / N; } else { kk = e & 15; n = e >> 4; }
   };
+  auto a_pos = [&](int m) { return MI * (m & 15) + (m >> 4); };
+  auto b_pos = [&](int n) { return NJ * (n & 15) + (n >> 4) + PADB * ((n & 15) >> 2); };
   float ra[MI], rb[NJ];
   auto fetch = [&](int k0) {
 #pragma unroll
@@ -103,6 +112,7 @@ __device__ void mm_acc(float (&acc)[MI][NJ], const float *A, int am, int ak, con
       rb[q] = B[(size_t)(k0 + kk) * bk + (size_t)n * bn];
     }
   };
+  const int a_base = MI * ty, b_base = NJ * tx + PADB * (tx >> 2);
   __syncthreads();  // operands the CTA has just written are complete before the first fetch
   fetch(0);
   for (int k0 = 0; k0 < K; k0 += 16) {
@@ -111,13 +121,13 @@ __device__ void mm_acc(float (&acc)[MI][NJ], const float *A, int am, int ak, con
     for (int q = 0; q < MI; ++q) {
       int kk, m;
       a_at(tid + q * NTH, kk, m);
-      As[kk * LA + m] = ra[q];
+      As[kk * LA + a_pos(m)] = ra[q];
     }
 #pragma unroll
     for (int q = 0; q < NJ; ++q) {
       int kk, n;
       b_at(tid + q * NTH, kk, n);
-      Bs[kk * LB + n] = rb[q];
+      Bs[kk * LB + b_pos(n)] = rb[q];
     }
     __syncthreads();
     if (k0 + 16 < K) fetch(k0 + 16);  // next slice in flight during this one's FMAs
@@ -125,9 +135,13 @@ __device__ void mm_acc(float (&acc)[MI][NJ], const float *A, int am, int ak, con
     for (int kk = 0; kk < 16; ++kk) {
       float a[MI], b[NJ];
 #pragma unroll
-      for (int i = 0; i < MI; ++i) a[i] = As[kk * LA + ty + 16 * i];
+      for (int q = 0; q < MI / 4; ++q)
+        *reinterpret_cast<float4 *>(&a[4 * q]) =
+            *reinterpret_cast<const float4 *>(As + kk * LA + a_base + 4 * q);
 #pragma unroll
-      for (int j = 0; j < NJ; ++j) b[j] = Bs[kk * LB + tx + 16 * j];
+      for (int q = 0; q < NJ / 4; ++q)
+        *reinterpret_cast<float4 *>(&b[4 * q]) =
+            *reinterpret_cast<const float4 *>(Bs + kk * LB + b_base + 4 * q);
 #pragma unroll
       for (int i = 0; i < MI; ++i)
 #pragma unroll
@@ -145,7 +159,8 @@ __device__ __forceinline__ void zero(float (&acc)[MI][NJ]) {
     for (int j = 0; j < NJ; ++j) acc[i][j] = 0.f;
 }
 
-constexpr int stage_floats(int M, int N) { return 16 * (M + 1) + 16 * (N + 1); }
+// shared floats mm_acc stages for an M x N output (the padded A and B slices)
+constexpr int stage_floats(int M, int N) { return 16 * (M + 4) + 16 * (N + 4 * (N >= 128 ? 4 : 0) + 4); }
 
 // Rows tok0 .. tok0 + n - 1 of a token-major [T, H, D] tensor into a [64][ld]
 // fp32 tile (rows >= n are zero: the exact no-op padding of the chunk form).
