@@ -219,6 +219,21 @@ __device__ void stage_gate(float *sG, float *sB, const BwdParams &p, int tok0, i
   __syncthreads();
 }
 
+// Gate tables store a row's column c at a permuted position so the thread that owns
+// columns tx + 16 j (j < NJ) reads them as NJ / 4 float4 chunks (2 tx, 2 tx + 1 for
+// NJ = 8, with chunk bit 0 flipped by tx bit 2 so every quarter-warp covers all 32
+// banks; chunk tx for NJ = 4).
+template <int NJ>
+__device__ __forceinline__ int gate_pos(int c) {
+  const int tx = c & 15, j = c >> 4;
+  if (NJ == 8) return 4 * ((2 * tx + (j >> 2)) ^ ((tx >> 2) & 1)) + (j & 3);
+  return 4 * tx + j;
+}
+template <int NJ>
+__device__ __forceinline__ int gate_chunk(int tx, int q) {
+  return NJ == 8 ? ((2 * tx + q) ^ ((tx >> 2) & 1)) : tx;
+}
+
 // Sum over the 16 lanes that share a row (lanes tx = 0..15 of one half-warp).
 __device__ __forceinline__ float row_sum16(float x) {
 #pragma unroll
@@ -723,7 +738,7 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
     __syncthreads();
     for (int e = tid; e < (r0 + 16) * D; e += NTH) {
       const int c = e % D;
-      sO[e] = sK[e] * exp2f(sG[r0 * D + c] - sG[e]);
+      sO[e - c + gate_pos<NJ>(c)] = sK[e] * exp2f(sG[r0 * D + c] - sG[e]);
     }
     __syncthreads();
     {
@@ -731,13 +746,18 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
       float op[NJ], oa[NJ];
 #pragma unroll
       for (int j = 0; j < NJ; ++j) op[j] = oa[j] = 0.f;
+#pragma unroll 4
       for (int s2 = 0; s2 <= t; ++s2) {
         const float dp = sP[t * C + s2], da = sT[t * C + s2];
+        float tb[NJ];
+#pragma unroll
+        for (int q = 0; q < NJ / 4; ++q)
+          *reinterpret_cast<float4 *>(&tb[4 * q]) =
+              *reinterpret_cast<const float4 *>(sO + s2 * D + 4 * gate_chunk<NJ>(tx, q));
 #pragma unroll
         for (int j = 0; j < NJ; ++j) {
-          const float tb = sO[s2 * D + tx + 16 * j];
-          op[j] = fmaf(dp, tb, op[j]);
-          oa[j] = fmaf(da, tb, oa[j]);
+          op[j] = fmaf(dp, tb[j], op[j]);
+          oa[j] = fmaf(da, tb[j], oa[j]);
         }
       }
 #pragma unroll
@@ -752,10 +772,10 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
     }
     __syncthreads();
     for (int e = r0 * D + tid; e < C * D; e += NTH) {
-      const int c = e % D;
+      const int c = e % D, at = e - c + gate_pos<NJ>(c);
       const float f = exp2f(sG[e] - sG[r1 * D + c]);
-      sO[e] = sQ[e] * f;
-      sV[e] = sK[e] * f;
+      sO[at] = sQ[e] * f;
+      sV[at] = sK[e] * f;
     }
     __syncthreads();
     {
@@ -763,11 +783,19 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
       float o2[NJ];
 #pragma unroll
       for (int j = 0; j < NJ; ++j) o2[j] = 0.f;
+#pragma unroll 4
       for (int t = s2; t < C; ++t) {
         const float dp = sP[t * C + s2], da = sT[t * C + s2];
+        float qb[NJ], kb[NJ];
 #pragma unroll
-        for (int j = 0; j < NJ; ++j)
-          o2[j] = fmaf(dp, sO[t * D + tx + 16 * j], fmaf(da, sV[t * D + tx + 16 * j], o2[j]));
+        for (int q = 0; q < NJ / 4; ++q) {
+          *reinterpret_cast<float4 *>(&qb[4 * q]) =
+              *reinterpret_cast<const float4 *>(sO + t * D + 4 * gate_chunk<NJ>(tx, q));
+          *reinterpret_cast<float4 *>(&kb[4 * q]) =
+              *reinterpret_cast<const float4 *>(sV + t * D + 4 * gate_chunk<NJ>(tx, q));
+        }
+#pragma unroll
+        for (int j = 0; j < NJ; ++j) o2[j] = fmaf(dp, qb[j], fmaf(da, kb[j], o2[j]));
       }
 #pragma unroll
       for (int j = 0; j < NJ; ++j) {
