@@ -413,9 +413,13 @@ __global__ void __launch_bounds__(NTH, 1) bwd_prep_kernel(const BwdParams p) {
 // ---------------------------------------------------------------------------
 constexpr int SC = 16;  // state columns per CTA
 
+// Shared layout: the chunk's Khat and W tiles (as copied), the CTA's 16-column slice of
+// dS held transposed (row stride LT, so a thread reads four consecutive k of its
+// column as one float4 on distinct banks), and the dU slice.
 template <int D>
 struct StateLayout {
-  static constexpr int oKh = 0, oW = oKh + C * D, oS = oW + C * D, oU = oS + D * SC;
+  static constexpr int LT = D + 4;
+  static constexpr int oKh = 0, oW = oKh + C * D, oS = oW + C * D, oU = oS + SC * LT;
   static constexpr int total = oU + C * SC;
   static constexpr size_t bytes = sizeof(float) * total;
 };
@@ -431,22 +435,25 @@ __device__ __forceinline__ void cp_async_wait_all() {
 template <int D>
 __global__ void __launch_bounds__(NTH) bwd_state_kernel(const BwdParams p) {
   using L = StateLayout<D>;
-  constexpr int NSL = D / SC, MI = D / 16;
+  constexpr int NSL = D / SC, MI = D / 16, LT = L::LT;
   extern __shared__ float4 smem_f4[];
   float *sm = reinterpret_cast<float *>(smem_f4);
-  float *sKh = sm + L::oKh, *sW = sm + L::oW, *sdS = sm + L::oS, *sdU = sm + L::oU;
+  float *sKh = sm + L::oKh, *sW = sm + L::oW, *sdST = sm + L::oS, *sdU = sm + L::oU;
   const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
   const int H = p.H;
   const int sl = blockIdx.x % NSL, rh = blockIdx.x / NSL;
   const int r = rh / H, h = rh % H;
-  const int col = SC * sl + tx;  // the thread's state column; its rows are ty + 16 i
+  // the thread's state column; its dS rows are MI ty + i (side by side), its dU rows
+  // ty + 16 i
+  const int col = SC * sl + tx;
   const float *dfin = p.d_final ? p.d_final + ((size_t)r * H + h) * D * D : nullptr;
   float ds[MI];
 #pragma unroll
-  for (int i = 0; i < MI; ++i) {
-    ds[i] = dfin ? dfin[(size_t)(ty + 16 * i) * D + col] : 0.f;
-    sdS[(ty + 16 * i) * SC + tx] = ds[i];
-  }
+  for (int i = 0; i < MI; ++i) ds[i] = dfin ? dfin[(size_t)(MI * ty + i) * D + col] : 0.f;
+#pragma unroll
+  for (int q = 0; q < MI / 4; ++q)
+    *reinterpret_cast<float4 *>(sdST + tx * LT + MI * ty + 4 * q) =
+        make_float4(ds[4 * q], ds[4 * q + 1], ds[4 * q + 2], ds[4 * q + 3]);
   for (int jc = p.cu_chunks[r + 1] - 1; jc >= p.cu_chunks[r]; --jc) {
     const size_t ch = (size_t)jc * H + h;
     const float4 *gK = reinterpret_cast<const float4 *>(p.wKh + ch * C * D);
@@ -460,19 +467,19 @@ __global__ void __launch_bounds__(NTH) bwd_state_kernel(const BwdParams p) {
     for (int i = 0; i < 4; ++i) u[i] = p.wX[ch * C * D + (size_t)(ty + 16 * i) * D + col];
 #pragma unroll
     for (int i = 0; i < MI; ++i) {
-      y[i] = p.wY[ch * D * D + (size_t)(ty + 16 * i) * D + col];
-      gam[i] = p.wGam[ch * D + ty + 16 * i];
+      y[i] = p.wY[ch * D * D + (size_t)(MI * ty + i) * D + col];
+      gam[i] = p.wGam[ch * D + MI * ty + i];
     }
     cp_async_wait_all();
     __syncthreads();
     // dU = X + Khat dSn   (overwrites X)
+#pragma unroll 4
     for (int k = 0; k < D; k += 4) {
-      const float d0 = sdS[k * SC + tx], d1 = sdS[(k + 1) * SC + tx];
-      const float d2 = sdS[(k + 2) * SC + tx], d3 = sdS[(k + 3) * SC + tx];
+      const float4 d4 = *reinterpret_cast<const float4 *>(sdST + tx * LT + k);
 #pragma unroll
       for (int i = 0; i < 4; ++i) {
         const float4 kh = *reinterpret_cast<const float4 *>(sKh + (ty + 16 * i) * D + k);
-        u[i] = fmaf(kh.x, d0, fmaf(kh.y, d1, fmaf(kh.z, d2, fmaf(kh.w, d3, u[i]))));
+        u[i] = fmaf(kh.x, d4.x, fmaf(kh.y, d4.y, fmaf(kh.z, d4.z, fmaf(kh.w, d4.w, u[i]))));
       }
     }
 #pragma unroll
@@ -485,24 +492,33 @@ __global__ void __launch_bounds__(NTH) bwd_state_kernel(const BwdParams p) {
     float acc[MI];
 #pragma unroll
     for (int i = 0; i < MI; ++i) acc[i] = 0.f;
+#pragma unroll 4
     for (int t = 0; t < C; ++t) {
       const float du = sdU[t * SC + tx];
 #pragma unroll
-      for (int i = 0; i < MI; ++i) acc[i] = fmaf(sW[t * D + ty + 16 * i], du, acc[i]);
+      for (int q = 0; q < MI / 4; ++q) {
+        const float4 w4 = *reinterpret_cast<const float4 *>(sW + t * D + MI * ty + 4 * q);
+        acc[4 * q] = fmaf(w4.x, du, acc[4 * q]);
+        acc[4 * q + 1] = fmaf(w4.y, du, acc[4 * q + 1]);
+        acc[4 * q + 2] = fmaf(w4.z, du, acc[4 * q + 2]);
+        acc[4 * q + 3] = fmaf(w4.w, du, acc[4 * q + 3]);
+      }
     }
 #pragma unroll
     for (int i = 0; i < MI; ++i) {
-      p.wY[ch * D * D + (size_t)(ty + 16 * i) * D + col] = ds[i];
+      p.wY[ch * D * D + (size_t)(MI * ty + i) * D + col] = ds[i];
       ds[i] = fmaf(gam[i], ds[i], y[i] - acc[i]);
     }
-    __syncthreads();  // every read of sdS, sKh and sW of this chunk is done
+    __syncthreads();  // every read of sdST, sKh and sW of this chunk is done
 #pragma unroll
-    for (int i = 0; i < MI; ++i) sdS[(ty + 16 * i) * SC + tx] = ds[i];
+    for (int q = 0; q < MI / 4; ++q)
+      *reinterpret_cast<float4 *>(sdST + tx * LT + MI * ty + 4 * q) =
+          make_float4(ds[4 * q], ds[4 * q + 1], ds[4 * q + 2], ds[4 * q + 3]);
   }
   if (p.d_initial) {
     float *dst = p.d_initial + ((size_t)r * H + h) * D * D;
 #pragma unroll
-    for (int i = 0; i < MI; ++i) dst[(size_t)(ty + 16 * i) * D + col] = ds[i];
+    for (int i = 0; i < MI; ++i) dst[(size_t)(MI * ty + i) * D + col] = ds[i];
   }
 }
 
