@@ -42,7 +42,10 @@ def _run_oracle(inp, d_o, d_fin):
 
 
 @pytest.mark.parametrize("d,dtype,tol", [(128, torch.bfloat16, TOL_BF16),
-                                         (64, torch.float32, TOL_F32)], ids=["bf16", "fp32"])
+                                         (64, torch.float32, TOL_F32),
+                                         (64, torch.bfloat16, TOL_BF16),
+                                         (128, torch.float32, TOL_F32)],
+                         ids=["bf16-d128", "fp32-d64", "bf16-d64", "fp32-d128"])
 @pytest.mark.parametrize("gate_scale", [5.0, 0.05], ids=["strong_decay", "weak_decay"])
 def test_backward_matches_oracle(d, dtype, tol, gate_scale):
     # ragged tails, a one-token request and several chunks per request
