@@ -456,6 +456,20 @@ def backward_bytes(T: int, H: int, d: int, n_req: int) -> int:
     return T * H * per_th + 3 * n_req * H * d * d * 4
 
 
+def backward_flops_per_token_head(d: int, C: int = 64) -> int:
+    """Algorithmic FLOPs of the backward per token-head (d = dk = dv, triangular
+    C x C tiles counted as half): per chunk the dense C d^2 products Y, dU, dS, U,
+    d(gamma Q), dKhat and dW (7), the C^2 d products A, P, W, U~, X, dP, T^T dU,
+    T^T dW (half each), dZ (1) and the four gated Gram cotangents (2 in all), i.e.
+    7 C d^2 + 7 C^2 d multiply-adds; plus the forward recompute."""
+    return 2 * (7 * d * d + 7 * C * d) + prefill_flops_per_token_head(d, d)
+
+
+def simt_fp32_peak_tflops(sm_mhz: float = 1965.0) -> float:
+    """fp32 FMA peak of the CUDA cores: 148 SMs x 128 fp32 lanes x 2 FLOP per clock."""
+    return 148 * 128 * 2 * sm_mhz * 1e6 / 1e12
+
+
 def bench_backward(args, inp, dev, peaks, world):
     """The backward of the headline workload: gradients of q, k, v, g, beta and the
     initial state for random fp32 cotangents of o and the final states, one
@@ -485,14 +499,20 @@ def bench_backward(args, inp, dev, peaks, world):
     barrier(world)
     ms = max_over_ranks(_time_calls(call, 1, 3, stream), world)
     b = backward_bytes(T, H, d, n)
+    fl = backward_flops_per_token_head(d) * T * H
+    tf = fl / (ms * 1e-3) / 1e12
+    peak_tf = simt_fp32_peak_tflops()
     return {"workload": "backward of the headline varlen prefill (64 requests, H=32, d=128, "
                         "bf16 inputs, fp32 gradients); random fp32 cotangents of o and the "
                         "final states",
             "value": world * T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
             "workspace_bytes": ws.numel(), "gpu_launches_per_step": 4,
-            "roofline": {"bound": "hbm", "achieved": b / (ms * 1e-3) / 1e9,
-                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
-                         "frac": b / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
+            "roofline": {"bound": "alu", "achieved": tf, "peak": peak_tf, "unit": "TFLOP/s",
+                         "frac": tf / peak_tf,
+                         "peak_kind": "derived: 148 SMs x 128 fp32 lanes x 2 FLOP x 1,965 MHz",
+                         "algorithmic_flops_per_launch": fl,
+                         "hbm_achieved_gbs": b / (ms * 1e-3) / 1e9,
+                         "hbm_frac": b / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"],
                          "algorithmic_bytes_per_launch": b}}
 
 
