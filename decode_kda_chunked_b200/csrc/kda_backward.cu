@@ -37,10 +37,15 @@
 // form a 16 x 16 grid; thread (ty, tx) owns rows ty + 16 i and columns
 // tx + 16 j of every tile it produces, so per-element folds stay in registers.
 #include "kda_internal.cuh"
+#include "kda_sm100.cuh"
+
+#include <type_traits>
 
 namespace kda {
 
 namespace {
+
+using namespace sm100;
 
 constexpr int NTH = 256;
 constexpr int C = kChunk;  // 64
@@ -62,6 +67,7 @@ struct BwdParams {
   float *wA, *wT, *wW, *wU, *wKh, *wX, *wY, *wGam;
   float *wU2;                  // U = U~ - W S per (chunk, head), written by the gradient pass
   int n_req, n_chunks, H;
+  unsigned int *status;        // device status word (a bounded wait that gave up)
 };
 
 // acc[i][j] += sum_k A(m_i, k) B(k, n_j) for k < K (a multiple of 16), where
@@ -251,16 +257,31 @@ struct PrepLayout {
   static constexpr int oP = oA + C * C, oT = oP + C * C, oBuf = oT + C * C;
   static constexpr int oKL = oBuf + C * LDP, oQL = oKL + 16 * LDP, oStage = oQL + 16 * LDP;
   static constexpr int oB = oStage + stage_floats(D, D);
-  static constexpr int total = oB + C;
-  static constexpr size_t bytes = sizeof(float) * total;
+  static constexpr int oMisc = oB + C;  // mbarrier (8 bytes) and the TMEM base address
+  static constexpr int total = oMisc + 4;
+  // + alignment slack: the tensor-core operand tiles need a 1024-byte aligned base
+  static constexpr size_t bytes = sizeof(float) * total + 1024;
 };
+
+// The products of the prep pass run on the tensor cores (tf32, like the forward's)
+// for bf16 inputs at d = 128; fp32 inputs keep fp32 products (their 1e-5 tolerance
+// rules out tf32 operands).
+template <int D, typename TIn>
+constexpr bool kPrepTensorCores = D == 128 && std::is_same<TIn, __nv_bfloat16>::value;
+
+__device__ __forceinline__ float tf32_round(float x) {
+  uint32_t r;
+  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  return __uint_as_float(r);
+}
 
 template <int D, typename TIn>
 __global__ void __launch_bounds__(NTH, 1) bwd_prep_kernel(const BwdParams p) {
   using L = PrepLayout<D>;
   constexpr int NJ = D / 16, LDP = L::LDP;
   extern __shared__ float4 smem_f4[];
-  float *sm = reinterpret_cast<float *>(smem_f4);
+  float *sm = reinterpret_cast<float *>(
+      (reinterpret_cast<uintptr_t>(smem_f4) + 1023) & ~uintptr_t(1023));
   float *sK = sm + L::oK, *sQ = sm + L::oQ, *sG = sm + L::oG, *sA = sm + L::oA;
   float *sP = sm + L::oP, *sT = sm + L::oT, *sBuf = sm + L::oBuf, *sKL = sm + L::oKL;
   float *sQL = sm + L::oQL, *sStage = sm + L::oStage, *sB = sm + L::oB;
@@ -270,6 +291,18 @@ __global__ void __launch_bounds__(NTH, 1) bwd_prep_kernel(const BwdParams p) {
   const int4 cd = p.chunks[jc];
   const int tok0 = cd.z, n = cd.w;
   const size_t ch = (size_t)jc * H + h;
+  uint64_t *bar = reinterpret_cast<uint64_t *>(sm + L::oMisc);
+  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + L::oMisc + 2);
+  if constexpr (kPrepTensorCores<D, TIn>) {
+    if ((tid >> 5) == 0) {
+      tmem_alloc(s_tmem, 512);
+      tmem_relinquish();
+    }
+    if (tid == 0) {
+      mbar_init(bar, 1);
+      asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+  }
 
   stage_rows<D, TIn>(sK, D, static_cast<const TIn *>(p.k), tok0, n, H, h);
   stage_rows<D, TIn>(sQ, D, static_cast<const TIn *>(p.q), tok0, n, H, h);
@@ -352,47 +385,152 @@ __global__ void __launch_bounds__(NTH, 1) bwd_prep_kernel(const BwdParams p) {
   }
   __syncthreads();
 
+  if constexpr (kPrepTensorCores<D, TIn>) {
+    // Transposed, so every product has M = 128 TMEM lanes (one per channel):
+    //   W^T = (beta gamma K)^T T^T,  U~^T = (beta V)^T T^T,  X^T = dO^T P,  Y^T = dO^T (gamma Q)
+    // A operands in TMEM (lane = channel, column = token), B operands K-major with the
+    // 128-byte swizzle in shared memory: T and P^T in the scratch tile, (gamma Q)^T in
+    // the (now unused) row-factor / staging region.
+    constexpr uint32_t TA1 = 0, TA2 = 64, TA3 = 128, TD1 = 192, TD2 = 256, TD3 = 320, TD4 = 384;
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    const uint32_t tm = *s_tmem;
+    const int w = tid >> 5, ln = tid & 31, c = 32 * (w & 3) + ln, j0 = 32 * (w >> 2);
+    const uint32_t lane = (uint32_t)(32 * (w & 3)) << 16;
+    stage_rows<D, TIn>(sBuf, LDP, static_cast<const TIn *>(p.v), tok0, n, H, h);
+    __syncthreads();
+    {
+      float v1[32], v2[32];
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj) {
+        const int j = j0 + jj;
+        v1[jj] = tf32_round(sB[j] * exp2f(sG[j * D + c]) * sK[j * D + c]);
+        v2[jj] = tf32_round(sB[j] * sBuf[j * LDP + c]);
+      }
+      tmem_st32(tm + lane + TA1 + j0, v1);
+      tmem_st32(tm + lane + TA2 + j0, v2);
+    }
+    __syncthreads();  // V read out of the scratch tile
+    stage_rows<D, float>(sBuf, LDP, p.d_o, tok0, n, H, h);
+    __syncthreads();
+    {
+      float v3[32];
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj) v3[jj] = tf32_round(sBuf[(j0 + jj) * LDP + c]);
+      tmem_st32(tm + lane + TA3 + j0, v3);
+    }
+    tmem_wait_st();
+    __syncthreads();  // dO read out of the scratch tile: it takes the B tiles now
+    unsigned char *bT = reinterpret_cast<unsigned char *>(sBuf);
+    unsigned char *bP = bT + 64 * 64 * 4;
+    unsigned char *bQ = reinterpret_cast<unsigned char *>(
+        (reinterpret_cast<uintptr_t>(sKL) + 1023) & ~uintptr_t(1023));
+    // consecutive threads walk each source's contiguous axis (conflict-free reads)
+    for (int e = tid; e < C * C; e += NTH) {
+      const int a = e >> 6, b = e & 63;
+      *reinterpret_cast<float *>(bT + sw128_offset(C, a, b)) = tf32_round(sT[a * C + b]);
+      *reinterpret_cast<float *>(bP + sw128_offset(C, b, a)) = tf32_round(sP[a * C + b]);
+    }
+    for (int e = tid; e < D * C; e += NTH) {
+      const int j = e / D, nn = e % D;
+      *reinterpret_cast<float *>(bQ + sw128_offset(D, nn, j)) =
+          tf32_round(exp2f(sG[j * D + nn]) * sQ[j * D + nn]);
+    }
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (tid == 0) {
+      const uint32_t id64 = idesc_tf32(64), id128 = idesc_tf32(128);
+      const uint32_t tb = smem_u32(bT), pb = smem_u32(bP), qb = smem_u32(bQ);
+#pragma unroll
+      for (int s = 0; s < C / 8; ++s) {
+        mma_tf32_ts(tm + TD1, tm + TA1 + 8 * s, sw128_desc(tb, C, s), id64, s > 0);
+        mma_tf32_ts(tm + TD2, tm + TA2 + 8 * s, sw128_desc(tb, C, s), id64, s > 0);
+        mma_tf32_ts(tm + TD3, tm + TA3 + 8 * s, sw128_desc(pb, C, s), id64, s > 0);
+        mma_tf32_ts(tm + TD4, tm + TA3 + 8 * s, sw128_desc(qb, D, s), id128, s > 0);
+      }
+      mma_commit(bar);
+    }
+    const bool done = mbar_wait(bar, 0);
+    if (!done && tid == 0) set_status(p.status, STATUS_TIMEOUT);
+    tc_fence_after();
+    if (done) {
+      float v[32];
+      tmem_ld32(tm + lane + TD1 + j0, v);  // W[token][channel]
+      tmem_wait_ld();
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj) p.wW[ch * C * D + (size_t)(j0 + jj) * D + c] = v[jj];
+      tmem_ld32(tm + lane + TD2 + j0, v);  // U~
+      tmem_wait_ld();
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj) p.wU[ch * C * D + (size_t)(j0 + jj) * D + c] = v[jj];
+      tmem_ld32(tm + lane + TD3 + j0, v);  // X
+      tmem_wait_ld();
+#pragma unroll
+      for (int jj = 0; jj < 32; ++jj) p.wX[ch * C * D + (size_t)(j0 + jj) * D + c] = v[jj];
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {  // Y[dk][dv] from Y^T (lane = dv)
+        const int c0 = 64 * (w >> 2) + 32 * half;
+        tmem_ld32(tm + lane + TD4 + c0, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) p.wY[ch * D * D + (size_t)(c0 + jj) * D + c] = v[jj];
+      }
+    }
+    tc_fence_before();
+    __syncthreads();
+    if (!done && tid == 0) mbar_wait(bar, 0, 100000000ull);  // give the products a last chance
+    __syncthreads();
+    if (w == 0) {
+      tc_fence_after();
+      tmem_dealloc(tm, 512);
+    }
+  } else {
   float acc[4][NJ];
-  // W = T Diag(beta) (gamma K)
-  for (int e = tid; e < C * D; e += NTH) {
-    const int t = e / D, c = e % D;
-    sBuf[t * LDP + c] = sB[t] * exp2f(sG[t * D + c]) * sK[t * D + c];
+    // W = T Diag(beta) (gamma K)
+    for (int e = tid; e < C * D; e += NTH) {
+      const int t = e / D, c = e % D;
+      sBuf[t * LDP + c] = sB[t] * exp2f(sG[t * D + c]) * sK[t * D + c];
+    }
+    zero(acc);
+    mm_acc<4, NJ>(acc, sT, C, 1, sBuf, LDP, 1, C, sStage);
+  #pragma unroll
+    for (int i = 0; i < 4; ++i)
+  #pragma unroll
+      for (int j = 0; j < NJ; ++j) p.wW[ch * C * D + (ty + 16 * i) * D + tx + 16 * j] = acc[i][j];
+    // U~ = T Diag(beta) V
+    stage_rows<D, TIn>(sBuf, LDP, static_cast<const TIn *>(p.v), tok0, n, H, h);
+    __syncthreads();
+    for (int e = tid; e < C * D; e += NTH) sBuf[(e / D) * LDP + e % D] *= sB[e / D];
+    zero(acc);
+    mm_acc<4, NJ>(acc, sT, C, 1, sBuf, LDP, 1, C, sStage);
+  #pragma unroll
+    for (int i = 0; i < 4; ++i)
+  #pragma unroll
+      for (int j = 0; j < NJ; ++j) p.wU[ch * C * D + (ty + 16 * i) * D + tx + 16 * j] = acc[i][j];
+    // X = P^T dO
+    stage_rows<D, float>(sBuf, LDP, p.d_o, tok0, n, H, h);
+    zero(acc);
+    mm_acc<4, NJ>(acc, sP, 1, C, sBuf, LDP, 1, C, sStage);
+  #pragma unroll
+    for (int i = 0; i < 4; ++i)
+  #pragma unroll
+      for (int j = 0; j < NJ; ++j) p.wX[ch * C * D + (ty + 16 * i) * D + tx + 16 * j] = acc[i][j];
+    // Y = (gamma Q)^T dO
+    for (int e = tid; e < C * D; e += NTH) sQ[e] *= exp2f(sG[e]);
+    {
+      float y[NJ][NJ];
+      zero(y);
+      mm_acc<NJ, NJ>(y, sQ, 1, D, sBuf, LDP, 1, C, sStage);
+  #pragma unroll
+      for (int i = 0; i < NJ; ++i)
+  #pragma unroll
+        for (int j = 0; j < NJ; ++j) p.wY[ch * D * D + (ty + 16 * i) * D + tx + 16 * j] = y[i][j];
+    }
   }
-  zero(acc);
-  mm_acc<4, NJ>(acc, sT, C, 1, sBuf, LDP, 1, C, sStage);
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < NJ; ++j) p.wW[ch * C * D + (ty + 16 * i) * D + tx + 16 * j] = acc[i][j];
-  // U~ = T Diag(beta) V
-  stage_rows<D, TIn>(sBuf, LDP, static_cast<const TIn *>(p.v), tok0, n, H, h);
-  __syncthreads();
-  for (int e = tid; e < C * D; e += NTH) sBuf[(e / D) * LDP + e % D] *= sB[e / D];
-  zero(acc);
-  mm_acc<4, NJ>(acc, sT, C, 1, sBuf, LDP, 1, C, sStage);
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < NJ; ++j) p.wU[ch * C * D + (ty + 16 * i) * D + tx + 16 * j] = acc[i][j];
-  // X = P^T dO
-  stage_rows<D, float>(sBuf, LDP, p.d_o, tok0, n, H, h);
-  zero(acc);
-  mm_acc<4, NJ>(acc, sP, 1, C, sBuf, LDP, 1, C, sStage);
-#pragma unroll
-  for (int i = 0; i < 4; ++i)
-#pragma unroll
-    for (int j = 0; j < NJ; ++j) p.wX[ch * C * D + (ty + 16 * i) * D + tx + 16 * j] = acc[i][j];
-  // Y = (gamma Q)^T dO
-  for (int e = tid; e < C * D; e += NTH) sQ[e] *= exp2f(sG[e]);
-  {
-    float y[NJ][NJ];
-    zero(y);
-    mm_acc<NJ, NJ>(y, sQ, 1, D, sBuf, LDP, 1, C, sStage);
-#pragma unroll
-    for (int i = 0; i < NJ; ++i)
-#pragma unroll
-      for (int j = 0; j < NJ; ++j) p.wY[ch * D * D + (ty + 16 * i) * D + tx + 16 * j] = y[i][j];
-  }
+
   // Khat = exp(G_last - G) K, Gam = exp(G_last); A and T for the gradient pass
   for (int e = tid; e < C * D; e += NTH) {
     const int t = e / D, c = e % D;
@@ -930,6 +1068,7 @@ cudaError_t launch_backward(const BackwardLaunch &b, cudaStream_t stream) {
   p.wGam = reinterpret_cast<float *>(ws + w.off_Gam);
   p.wU2 = reinterpret_cast<float *>(ws + w.off_U2);
   p.n_req = b.n_req; p.n_chunks = b.n_chunks; p.H = b.H;
+  p.status = device_status_word();
   if (b.D == 128)
     return b.in_dtype == KDA_BF16 ? launch_bwd_d<128, __nv_bfloat16>(p, stream)
                                   : launch_bwd_d<128, float>(p, stream);
