@@ -33,9 +33,12 @@
 //   bwd_state (CTA per request, head and 16 state columns): the serial pass;
 //             dU overwrites X, dSn overwrites Y
 //   bwd_grad  (CTA per chunk and head): every token gradient of the chunk
-// All backward arithmetic is fp32 on the CUDA cores.  A CTA's 256 threads
-// form a 16 x 16 grid; thread (ty, tx) owns rows ty + 16 i and columns
+// The state and gradient passes are fp32 on the CUDA cores: a CTA's 256 threads
+// form a 16 x 16 grid, and thread (ty, tx) owns rows ty + 16 i and columns
 // tx + 16 j of every tile it produces, so per-element folds stay in registers.
+// For bf16 inputs at d = 128 the prep pass runs its four products as tcgen05
+// tf32 MMAs (transposed to M = 128 TMEM lanes, as in the forward); fp32 inputs
+// keep fp32 products there too.
 #include "kda_internal.cuh"
 #include "kda_sm100.cuh"
 
