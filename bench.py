@@ -506,7 +506,9 @@ def bench_backward(args, inp, dev, peaks, world):
                         "bf16 inputs, fp32 gradients); random fp32 cotangents of o and the "
                         "final states",
             "value": world * T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
-            "workspace_bytes": ws.numel(), "gpu_launches_per_step": 4,
+            "workspace_bytes": ws.numel(),
+            # forward recompute, prep, state pass, state products, gradient pass
+            "gpu_launches_per_step": 5,
             "roofline": {"bound": "alu", "achieved": tf, "peak": peak_tf, "unit": "TFLOP/s",
                          "frac": tf / peak_tf,
                          "peak_kind": "derived: 148 SMs x 128 fp32 lanes x 2 FLOP x 1,965 MHz",

@@ -32,13 +32,16 @@
 //   bwd_prep  (CTA per chunk and head): A, T, W, U~, Khat, Gam, X = P^T dO, Y = (gamma Q)^T dO
 //   bwd_state (CTA per request, head and 16 state columns): the serial pass;
 //             dU overwrites X, dSn overwrites Y
+//   bwd_sprod (CTA per chunk and head; bf16 inputs at d = 128): U, d(gamma Q),
+//             dKhat, dW and dGam, the products with the state, on the tensor cores
 //   bwd_grad  (CTA per chunk and head): every token gradient of the chunk
 // The state and gradient passes are fp32 on the CUDA cores: a CTA's 256 threads
 // form a 16 x 16 grid, and thread (ty, tx) owns rows ty + 16 i and columns
 // tx + 16 j of every tile it produces, so per-element folds stay in registers.
 // For bf16 inputs at d = 128 the prep pass runs its four products as tcgen05
-// tf32 MMAs (transposed to M = 128 TMEM lanes, as in the forward); fp32 inputs
-// keep fp32 products there too.
+// tf32 MMAs (transposed to M = 128 TMEM lanes, as in the forward), and so does
+// bwd_sprod with the four products of the state; fp32 inputs keep fp32 products
+// throughout.
 #include "kda_internal.cuh"
 #include "kda_sm100.cuh"
 
@@ -664,6 +667,204 @@ __global__ void __launch_bounds__(NTH) bwd_state_kernel(const BwdParams p) {
 }
 
 // ---------------------------------------------------------------------------
+// bwd_sprod (bf16 inputs, d = 128): the four state products of the gradient pass
+// on the tensor cores.  Transposed, as in the forward, so each has M = 128 TMEM
+// lanes; A operands in TMEM, B operands K-major with the 128-byte swizzle in
+// shared memory, tf32 operands rounded to nearest, fp32 accumulation:
+//   U^T          = U~^T - S^T W^T    A = S^T (lane = value column), D starts as U~^T
+//   d(gamma Q)^T = S dO^T            A = S (lane = key row)
+//   dW^T         = -S dU^T           A = S
+//   dKhat^T      = dSn U^T           A = dSn (lane = key row), B = U from the first product
+// and dGam_i = sum_j dSn_ij S_ij (fp32 on the CUDA cores, from the unrounded values).
+// The results go to workspace tiles the gradient pass no longer needs: U to its own
+// tile, d(gamma Q) and dKhat over dSn, dW over Khat (both read only by the state
+// pass), dGam over Gam.
+// ---------------------------------------------------------------------------
+constexpr int SP_NTH = 512;
+
+struct SprodLayout {
+  static constexpr int D = 128;
+  // B operand tiles (64 rows x 128 tf32 each, 1024-byte aligned), then the dGam partials
+  static constexpr int oW = 0, oO = oW + C * D, oDU = oO + C * D, oU = oDU + C * D;
+  static constexpr int oPart = oU + C * D;     // [4][128]
+  static constexpr int oMisc = oPart + 4 * D;  // two mbarriers and the TMEM base address
+  static constexpr int total = oMisc + 8;
+  static constexpr size_t bytes = sizeof(float) * total + 1024;
+};
+
+__device__ __forceinline__ float4 tf32_round4(float4 x) {
+  return make_float4(tf32_round(x.x), tf32_round(x.y), tf32_round(x.z), tf32_round(x.w));
+}
+
+__global__ void __launch_bounds__(SP_NTH, 1) bwd_sprod_kernel(const BwdParams p) {
+  using L = SprodLayout;
+  constexpr int D = L::D;
+  // TMEM columns: S^T, then dW^T | dKhat^T once the first product is done; U~^T -> U^T;
+  // S; dSn; d(gamma Q)^T
+  constexpr uint32_t TST = 0, TDW = 0, TDK = 64, TU = 128, TS = 192, TDS = 320, TGQ = 448;
+  extern __shared__ float4 smem_f4[];
+  float *sm = reinterpret_cast<float *>(
+      (reinterpret_cast<uintptr_t>(smem_f4) + 1023) & ~uintptr_t(1023));
+  unsigned char *bW = reinterpret_cast<unsigned char *>(sm + L::oW);
+  unsigned char *bO = reinterpret_cast<unsigned char *>(sm + L::oO);
+  unsigned char *bDU = reinterpret_cast<unsigned char *>(sm + L::oDU);
+  unsigned char *bU = reinterpret_cast<unsigned char *>(sm + L::oU);
+  float *sPart = sm + L::oPart;
+  uint64_t *bar = reinterpret_cast<uint64_t *>(sm + L::oMisc);  // [0]: U^T, [1]: the rest
+  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + L::oMisc + 4);
+  const int tid = threadIdx.x, w = tid >> 5, ln = tid & 31;
+  const int H = p.H;
+  const int jc = blockIdx.x / H, h = blockIdx.x % H;
+  const int4 cd = p.chunks[jc];
+  const int r = cd.x, cidx = cd.y, tok0 = cd.z, n = cd.w;
+  const size_t ch = (size_t)jc * H + h;
+  const float *S;
+  if (cidx == 0)
+    S = p.initial_state ? p.initial_state + ((size_t)r * H + h) * D * D : p.zero_state;
+  else
+    S = p.snaps + ((size_t)(p.cu_snap[r] + cidx - 1) * H + h) * D * D;
+  const float *dSn = p.wY + ch * D * D;
+  if (w == 0) {
+    tmem_alloc(s_tmem, 512);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    mbar_init(bar + 1, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+
+  // B operands: W, dO (rows past the chunk's end are zero) and dU, rows = tokens
+  for (int e = tid; e < C * D / 4; e += SP_NTH) {
+    const int t = e >> 5, k = (e & 31) * 4;
+    const float4 wv = *reinterpret_cast<const float4 *>(p.wW + ch * C * D + t * D + k);
+    const float4 uv = *reinterpret_cast<const float4 *>(p.wX + ch * C * D + t * D + k);
+    const float4 ov = (p.d_o && t < n) ? *reinterpret_cast<const float4 *>(
+                                             p.d_o + ((size_t)(tok0 + t) * H + h) * D + k)
+                                       : make_float4(0.f, 0.f, 0.f, 0.f);
+    *reinterpret_cast<float4 *>(bW + sw128_chunk(C, t, k)) = tf32_round4(wv);
+    *reinterpret_cast<float4 *>(bDU + sw128_chunk(C, t, k)) = tf32_round4(uv);
+    *reinterpret_cast<float4 *>(bO + sw128_chunk(C, t, k)) = tf32_round4(ov);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tm = *s_tmem;
+  // warp w reaches TMEM lanes 32 (w % 4) .. + 31 and takes the 32-column part w / 4
+  const int qd = w & 3, part = w >> 2, lrow = 32 * qd + ln;
+  const uint32_t lane = (uint32_t)(32 * qd) << 16;
+  {  // S^T: lane = value column, columns = key rows (consecutive lanes read one row)
+    float v[32];
+#pragma unroll
+    for (int jj = 0; jj < 32; ++jj) v[jj] = tf32_round(S[(size_t)(32 * part + jj) * D + lrow]);
+    tmem_st32(tm + lane + TST + 32 * part, v);
+  }
+  {  // S and dSn: lane = key row, columns = value columns; the dGam partial sums
+    float a[32], b[32];
+    const float4 *sr = reinterpret_cast<const float4 *>(S + (size_t)lrow * D + 32 * part);
+    const float4 *dr = reinterpret_cast<const float4 *>(dSn + (size_t)lrow * D + 32 * part);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      *reinterpret_cast<float4 *>(&a[4 * q]) = sr[q];
+      *reinterpret_cast<float4 *>(&b[4 * q]) = dr[q];
+    }
+    float gs = 0.f;
+#pragma unroll
+    for (int jj = 0; jj < 32; ++jj) {
+      gs = fmaf(a[jj], b[jj], gs);
+      a[jj] = tf32_round(a[jj]);
+      b[jj] = tf32_round(b[jj]);
+    }
+    sPart[part * D + lrow] = gs;
+    tmem_st32(tm + lane + TS + 32 * part, a);
+    tmem_st32(tm + lane + TDS + 32 * part, b);
+  }
+  {  // U~^T (the first product's accumulator, fp32): lane = value column, columns = tokens
+    float v[16];
+#pragma unroll
+    for (int tt = 0; tt < 16; ++tt) v[tt] = p.wU[ch * C * D + (size_t)(16 * part + tt) * D + lrow];
+    tmem_st16(tm + lane + TU + 16 * part, v);
+  }
+  tmem_wait_st();
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t id64 = idesc_tf32(64), id64n = idesc_tf32(64, true);
+  if (tid == 0) {
+    const uint32_t wb = smem_u32(bW), ob = smem_u32(bO);
+#pragma unroll
+    for (int s = 0; s < D / 8; ++s)
+      mma_tf32_ts(tm + TU, tm + TST + 8 * s, sw128_desc(wb, C, s), id64n, true);
+    mma_commit(bar);
+#pragma unroll
+    for (int s = 0; s < D / 8; ++s)
+      mma_tf32_ts(tm + TGQ, tm + TS + 8 * s, sw128_desc(ob, C, s), id64, s > 0);
+  }
+  if (tid < D)  // dGam in a fixed order
+    p.wGam[ch * D + tid] = (sPart[tid] + sPart[D + tid]) + (sPart[2 * D + tid] + sPart[3 * D + tid]);
+  const bool ok = mbar_wait(bar, 0);
+  tc_fence_after();
+  if (tid == 0 && ok) {  // S^T is consumed: dW^T = -S dU^T goes over its first half
+    const uint32_t db = smem_u32(bDU);
+#pragma unroll
+    for (int s = 0; s < D / 8; ++s)
+      mma_tf32_ts(tm + TDW, tm + TS + 8 * s, sw128_desc(db, C, s), id64n, s > 0);
+  }
+  if (ok) {  // U: to its workspace tile (fp32) and, rounded, to the B tile of dKhat^T
+    float v[16];
+    tmem_ld16(tm + lane + TU + 16 * part, v);
+    tmem_wait_ld();
+#pragma unroll
+    for (int tt = 0; tt < 16; ++tt) {
+      const int t = 16 * part + tt;
+      p.wU2[ch * C * D + (size_t)t * D + lrow] = v[tt];
+      *reinterpret_cast<float *>(bU + sw128_offset(C, t, lrow)) = tf32_round(v[tt]);
+    }
+  }
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (tid == 0) {
+    if (ok) {
+      const uint32_t ub = smem_u32(bU);
+#pragma unroll
+      for (int s = 0; s < D / 8; ++s)
+        mma_tf32_ts(tm + TDK, tm + TDS + 8 * s, sw128_desc(ub, C, s), id64, s > 0);
+    }
+    mma_commit(bar + 1);  // covers every product issued, whatever happened above
+  }
+  const bool done = ok && mbar_wait(bar + 1, 0);
+  if (!done && tid == 0) set_status(p.status, STATUS_TIMEOUT);
+  tc_fence_after();
+  if (done) {
+    float v[16];
+    tmem_ld16(tm + lane + TGQ + 16 * part, v);  // d(gamma Q)[token][key]
+    tmem_wait_ld();
+#pragma unroll
+    for (int tt = 0; tt < 16; ++tt) p.wY[ch * D * D + (size_t)(16 * part + tt) * D + lrow] = v[tt];
+    tmem_ld16(tm + lane + TDK + 16 * part, v);  // dKhat
+    tmem_wait_ld();
+#pragma unroll
+    for (int tt = 0; tt < 16; ++tt)
+      p.wY[ch * D * D + C * D + (size_t)(16 * part + tt) * D + lrow] = v[tt];
+    tmem_ld16(tm + lane + TDW + 16 * part, v);  // dW
+    tmem_wait_ld();
+#pragma unroll
+    for (int tt = 0; tt < 16; ++tt) p.wKh[ch * C * D + (size_t)(16 * part + tt) * D + lrow] = v[tt];
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (!done && tid == 0) mbar_wait(bar + 1, 0, 100000000ull);  // let issued products finish
+  __syncthreads();
+  if (w == 0) {
+    tc_fence_after();
+    tmem_dealloc(tm, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // bwd_grad: every token gradient of one chunk
 // ---------------------------------------------------------------------------
 template <int D>
@@ -680,6 +881,8 @@ template <int D, typename TIn>
 __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
   using L = GradLayout<D>;
   constexpr int NJ = D / 16;
+  // U, d(gamma Q), dKhat, dW and dGam come from bwd_sprod (tensor cores) when it ran
+  constexpr bool PRE = kPrepTensorCores<D, TIn>;
   extern __shared__ float4 smem_f4[];
   float *sm = reinterpret_cast<float *>(smem_f4);
   float *sK = sm + L::oK, *sQ = sm + L::oQ, *sV = sm + L::oV, *sO = sm + L::oO;
@@ -714,24 +917,37 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
   float accQ[4][NJ], accK[4][NJ], accG[4][NJ], acc[4][NJ];
   const float *G63 = sG + (C - 1) * D;
 
-  // U = U~ - W S  (U~ loaded before the product so its latency hides under it)
-  float ut[4][NJ];
+  // the thread's elements of a precomputed C x D product
+  auto load_own = [&](const float *src) {
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int j = 0; j < NJ; ++j) ut[i][j] = Ut[(ty + 16 * i) * D + tx + 16 * j];
-  zero(acc);
-  mm_acc<4, NJ>(acc, W, D, 1, S, D, 1, D, sStage);
+      for (int j = 0; j < NJ; ++j) acc[i][j] = src[(ty + 16 * i) * D + tx + 16 * j];
+  };
+  if constexpr (!PRE) {
+    // U = U~ - W S  (U~ loaded before the product so its latency hides under it)
+    float ut[4][NJ];
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int j = 0; j < NJ; ++j) {
-      const int e = (ty + 16 * i) * D + tx + 16 * j;
-      U[e] = ut[i][j] - acc[i][j];
-    }
+      for (int j = 0; j < NJ; ++j) ut[i][j] = Ut[(ty + 16 * i) * D + tx + 16 * j];
+    zero(acc);
+    mm_acc<4, NJ>(acc, W, D, 1, S, D, 1, D, sStage);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) {
+        const int e = (ty + 16 * i) * D + tx + 16 * j;
+        U[e] = ut[i][j] - acc[i][j];
+      }
+  }
   // d(gamma Q) = dO S^T  ->  dQ = d(gamma Q) gamma,  dG = d(gamma Q) gamma q
-  zero(acc);
-  mm_acc<4, NJ>(acc, sO, D, 1, S, 1, D, D, sStage);
+  if constexpr (PRE) {
+    load_own(dSn);  // bwd_sprod put d(gamma Q) over the first half of the dSn tile
+  } else {
+    zero(acc);
+    mm_acc<4, NJ>(acc, sO, D, 1, S, 1, D, D, sStage);
+  }
 #pragma unroll
   for (int i = 0; i < 4; ++i)
 #pragma unroll
@@ -756,8 +972,12 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
       }
   }
   // dKhat = U dSn^T  ->  dK += dKhat Gam/gamma,  dG -= dKhat Khat,  dG_last += sum_t dKhat Khat
-  zero(acc);
-  mm_acc<4, NJ>(acc, U, D, 1, dSn, 1, D, D, sStage);
+  if constexpr (PRE) {
+    load_own(dSn + C * D);  // and dKhat over its second half
+  } else {
+    zero(acc);
+    mm_acc<4, NJ>(acc, U, D, 1, dSn, 1, D, D, sStage);
+  }
 #pragma unroll
   for (int j = 0; j < NJ; ++j) {
     float colsum = 0.f;
@@ -773,7 +993,9 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
     sPart[ty * D + tx + 16 * j] = colsum;
   }
   // dGam = rowsum(dSn * S): warp w takes rows w, w + 8, ...; lanes walk the row
-  {
+  if constexpr (PRE) {
+    if (tid < D) sGam[tid] = p.wGam[ch * D + tid];  // from bwd_sprod, over Gam
+  } else {
     const int w = tid >> 5, ln = tid & 31;
 #pragma unroll 4
     for (int row = w; row < D; row += NTH / 32) {
@@ -799,13 +1021,21 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
     sExtra[tid] = e;
   }
 
-  // dW = -dU S^T (into the dO tile)
-  zero(acc);
-  mm_acc<4, NJ>(acc, dU, D, 1, S, 1, D, D, sStage);
+  // dW = -dU S^T (into the dO tile; the sync above ends every read of that tile)
+  if constexpr (PRE) {
+    load_own(p.wKh + ch * C * D);  // from bwd_sprod, over Khat
 #pragma unroll
-  for (int i = 0; i < 4; ++i)
+    for (int i = 0; i < 4; ++i)
 #pragma unroll
-    for (int j = 0; j < NJ; ++j) sO[(ty + 16 * i) * D + tx + 16 * j] = -acc[i][j];
+      for (int j = 0; j < NJ; ++j) sO[(ty + 16 * i) * D + tx + 16 * j] = acc[i][j];
+  } else {
+    zero(acc);
+    mm_acc<4, NJ>(acc, dU, D, 1, S, 1, D, D, sStage);
+#pragma unroll
+    for (int i = 0; i < 4; ++i)
+#pragma unroll
+      for (int j = 0; j < NJ; ++j) sO[(ty + 16 * i) * D + tx + 16 * j] = -acc[i][j];
+  }
   {
     float4 tv[C * C / 4 / NTH];
 #pragma unroll
@@ -1007,6 +1237,13 @@ cudaError_t launch_bwd_d(const BwdParams &p, cudaStream_t stream) {
   bwd_state_kernel<D>
       <<<(unsigned)(p.n_req * p.H * (D / SC)), NTH, StateLayout<D>::bytes, stream>>>(p);
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
+  if constexpr (kPrepTensorCores<D, TIn>) {
+    if (chunk_grid > 0) {
+      if ((e = set_smem(bwd_sprod_kernel, SprodLayout::bytes)) != cudaSuccess) return e;
+      bwd_sprod_kernel<<<chunk_grid, SP_NTH, SprodLayout::bytes, stream>>>(p);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+  }
   if (chunk_grid > 0) {
     if ((e = set_smem(bwd_grad_kernel<D, TIn>, GradLayout<D>::bytes)) != cudaSuccess) return e;
     bwd_grad_kernel<D, TIn><<<chunk_grid, NTH, GradLayout<D>::bytes, stream>>>(p);
