@@ -50,8 +50,11 @@ def prefill_flops_per_token_head(dk: int, dv: int, C: int = CHUNK) -> int:
 
 
 def prefill_bytes(T: int, H: int, dk: int, dv: int, n_req: int, in_bytes: int = 2,
-                  out_bytes: int = 4, initial: bool = False, final: bool = True) -> int:
-    per_th = in_bytes * (2 * dk + dv) + 4 * dk + 4 + out_bytes * dv
+                  out_bytes: int = 4, initial: bool = False, final: bool = True,
+                  gate_bytes: int = 4) -> int:
+    """q, k, v at in_bytes, the gate at gate_bytes (4: fp32 log alpha, 2: bf16 logits),
+    beta fp32, o at out_bytes, per token-head; plus the states read and written."""
+    per_th = in_bytes * (2 * dk + dv) + gate_bytes * dk + 4 + out_bytes * dv
     state = n_req * H * dk * dv * 4
     return T * H * per_th + (state if initial else 0) + (state if final else 0)
 
@@ -365,6 +368,7 @@ def run_ours(args, world, rank, local):
         line["decode"] = bench_decode(args, dev, peaks, peak_kind, rank)
     if not args.no_extra:
         line["single_seq"] = bench_single_seq(args, dev, peaks)
+        line["fused_gate"] = bench_fused_gate(args, inp, dev, peaks, rank)
         line["kcp_million"] = bench_kcp_million(args, dev, peaks, world, rank)
         line["backward"] = bench_backward(args, inp, dev, peaks, world)
     if not args.no_e2e:
@@ -538,6 +542,35 @@ def bench_single_seq(args, dev, peaks):
     return {"workload": "B=1, H=32, T=8192, d=128, bf16, N(0,0.1) initial state, final state out",
             "value": T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
             "tflops": prefill_flops_per_token_head(d, d) * T * H / (ms * 1e-3) / 1e12,
+            "roofline": {"bound": "hbm", "achieved": b / (ms * 1e-3) / 1e9,
+                         "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                         "frac": b / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}}
+
+
+def bench_fused_gate(args, inp, dev, peaks, rank):
+    """The headline varlen workload with the gate given as bf16 logits x (fused gate
+    activation: the kernel computes log alpha = -5 sigmoid(x)), same lengths, same
+    q, k, v and beta draws; 1,540 algorithmic bytes per token-head instead of 1,796."""
+    import torch
+
+    import decode_kda_chunked_b200 as kda
+    from decode_kda_chunked_b200 import inputs as I
+    x = I.make_prefill_inputs(inp.lengths, H=32, dk=128, dv=128, seed=rank, device=dev,
+                              gate_logits=True)
+    T, H, d, n = x.total_tokens, 32, 128, x.n_req
+    o = torch.empty(T, H, d, device=dev)
+    fin = torch.empty(n, H, d, d, device=dev)
+    stream = torch.cuda.current_stream(dev)
+    cu_host = torch.tensor([0] + list(__import__("itertools").accumulate(x.lengths)),
+                           dtype=torch.int32)
+    ms = _time_calls(lambda: kda.kda_prefill_chunked(
+        x.q, x.k, x.v, None, x.beta, x.cu_seqlens, o, None, fin, cu_seqlens_host=cu_host,
+        stream=stream, g_logits=x.g_logits), 3, max(args.steps, 5), stream)
+    assert kda.kda_get_device_status() == 0
+    b = prefill_bytes(T, H, d, d, n, final=True, gate_bytes=2)
+    return {"workload": "the headline varlen prefill with bf16 gate logits instead of fp32 g",
+            "value": T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
+            "algorithmic_bytes_per_launch": b,
             "roofline": {"bound": "hbm", "achieved": b / (ms * 1e-3) / 1e9,
                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
                          "frac": b / (ms * 1e-3) / 1e9 / peaks["hbm_gbs"]}}

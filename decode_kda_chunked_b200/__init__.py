@@ -44,8 +44,10 @@ def _host_lengths(cu_seqlens, cu_seqlens_host):
 
 def prefill(q, k, v, g, beta, cu_seqlens, initial_state=None, snapshot_stride: int = 0,
             out_dtype=torch.float32, want_final: bool = True, cu_seqlens_host=None,
-            stream=None) -> dict:
+            stream=None, g_logits=None) -> dict:
     """Chunked prefill over packed requests; allocates o / final / snapshots.
+    The gate is ``g`` (fp32 log alpha) or, with ``g=None``, ``g_logits`` (bf16
+    logits x, log alpha = -5 sigmoid(x) computed in the kernels).
 
     Returns dict(o, final_state, snapshots, cu_snapshots)."""
     T, H, dk = k.shape
@@ -63,16 +65,18 @@ def prefill(q, k, v, g, beta, cu_seqlens, initial_state=None, snapshot_stride: i
         snaps = torch.empty((max(offs[-1], 1), H, dk, dv), dtype=torch.float32, device=dev)
     kda_prefill_chunked(q, k, v, g, beta, cu_seqlens, o, initial_state, fin, snapshot_stride,
                         cu_snap, snaps, cu_seqlens_host=torch.tensor(cu_host, dtype=torch.int32),
-                        stream=stream)
+                        stream=stream, g_logits=g_logits)
     if snaps is not None:
         snaps = snaps[:offs[-1]]
     return {"o": o, "final_state": fin, "snapshots": snaps, "cu_snapshots": cu_snap}
 
 
 def prefill_backward(q, k, v, g, beta, cu_seqlens, d_o=None, d_final=None, initial_state=None,
-                     want_initial: bool = True, cu_seqlens_host=None, stream=None) -> dict:
+                     want_initial: bool = True, cu_seqlens_host=None, stream=None,
+                     g_logits=None) -> dict:
     """Gradients of sum(d_o * o) + sum(d_final * final_state) of ``prefill`` for the
-    same inputs; allocates the fp32 gradients and the workspace.
+    same inputs; allocates the fp32 gradients and the workspace.  With ``g_logits``
+    (and ``g=None``) the returned ``dg`` is the gradient of the logits.
 
     Returns dict(dq, dk, dv, dg, dbeta, d_initial)."""
     T, H, dk = k.shape
@@ -86,12 +90,13 @@ def prefill_backward(q, k, v, g, beta, cu_seqlens, d_o=None, d_final=None, initi
     d0 = torch.empty((len(lengths), H, dk, dv), **f32) if want_initial else None
     kda_prefill_backward(q, k, v, g, beta, cu_seqlens, torch.tensor(cu_host, dtype=torch.int32),
                          dq, dk_, dv_, dg, db, initial_state=initial_state, d_o=d_o,
-                         d_final=d_final, d_initial=d0, stream=stream)
+                         d_final=d_final, d_initial=d0, stream=stream, g_logits=g_logits)
     return {"dq": dq, "dk": dk_, "dv": dv_, "dg": dg, "dbeta": db, "d_initial": d0}
 
 
 def long_context_prefill(q, k, v, g, beta, seg_len: int, snapshot_stride: int = 512,
-                         initial_state=None, out_dtype=torch.float32, stream=None) -> dict:
+                         initial_state=None, out_dtype=torch.float32, stream=None,
+                         g_logits=None) -> dict:
     """One long sequence split into segments of ``seg_len`` tokens (KDA context
     parallelism on one device): local zero-start states and transitions per
     segment, an exact combine, then the chunked prefill of every segment from
@@ -111,12 +116,13 @@ def long_context_prefill(q, k, v, g, beta, seg_len: int, snapshot_stride: int = 
     s_loc = torch.empty((n_seg, H, dk, dv), dtype=torch.float32, device=dev)
     m = torch.empty((n_seg, H, dk, dk), dtype=torch.float32, device=dev)
     kda_chunk_local_state(k, v, g, beta, seg_cu, s_loc, m,
-                          seg_cu_host=torch.tensor(bounds, dtype=torch.int32), stream=stream)
+                          seg_cu_host=torch.tensor(bounds, dtype=torch.int32), stream=stream,
+                          g_logits=g_logits)
     s_in = torch.empty_like(s_loc)
     kda_state_combine(s_loc, m, initial_state, s_in, None, stream=stream)
     out = prefill(q, k, v, g, beta, seg_cu, initial_state=s_in,
                   snapshot_stride=snapshot_stride, out_dtype=out_dtype,
-                  cu_seqlens_host=bounds, stream=stream)
+                  cu_seqlens_host=bounds, stream=stream, g_logits=g_logits)
     return {"o": out["o"], "final_state": out["final_state"][-1], "snapshots": out["snapshots"],
             "s_in": s_in, "s_loc": s_loc, "m": m}
 

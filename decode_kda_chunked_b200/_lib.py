@@ -32,13 +32,14 @@ class PrefillArgs(ctypes.Structure):
                 ("q", _vp), ("k", _vp), ("v", _vp), ("g", _vp), ("beta", _vp),
                 ("cu_seqlens", _vp), ("cu_seqlens_host", _vp), ("initial_state", _vp),
                 ("o", _vp), ("final_state", _vp), ("snapshot_stride", _i32),
-                ("cu_snapshots", _vp), ("snapshots", _vp)]
+                ("cu_snapshots", _vp), ("snapshots", _vp), ("g_logits", _vp)]
 
 
 class LocalStateArgs(ctypes.Structure):
     _fields_ = [("n_seg", _i32), ("total_tokens", _i32), ("H", _i32), ("dk", _i32), ("dv", _i32),
                 ("in_dtype", ctypes.c_int), ("k", _vp), ("v", _vp), ("g", _vp), ("beta", _vp),
-                ("seg_cu", _vp), ("seg_cu_host", _vp), ("s_loc", _vp), ("m", _vp)]
+                ("seg_cu", _vp), ("seg_cu_host", _vp), ("s_loc", _vp), ("m", _vp),
+                ("g_logits", _vp)]
 
 
 class DecodeArgs(ctypes.Structure):
@@ -53,7 +54,8 @@ class BackwardArgs(ctypes.Structure):
                 ("in_dtype", ctypes.c_int), ("q", _vp), ("k", _vp), ("v", _vp), ("g", _vp),
                 ("beta", _vp), ("cu_seqlens", _vp), ("cu_seqlens_host", _vp),
                 ("initial_state", _vp), ("d_o", _vp), ("d_final", _vp), ("d_q", _vp),
-                ("d_k", _vp), ("d_v", _vp), ("d_g", _vp), ("d_beta", _vp), ("d_initial", _vp)]
+                ("d_k", _vp), ("d_v", _vp), ("d_g", _vp), ("d_beta", _vp), ("d_initial", _vp),
+                ("g_logits", _vp)]
 
 
 class KdaError(RuntimeError):
@@ -164,7 +166,7 @@ def _host_i32(x):
 
 def make_prefill_args(q, k, v, g, beta, cu_seqlens, o, initial_state=None, final_state=None,
                       snapshot_stride=0, cu_snapshots=None, snapshots=None,
-                      cu_seqlens_host=None):
+                      cu_seqlens_host=None, g_logits=None):
     T, H, dk = k.shape
     dv = v.shape[2]
     a = PrefillArgs()
@@ -182,6 +184,7 @@ def make_prefill_args(q, k, v, g, beta, cu_seqlens, o, initial_state=None, final
     a.snapshot_stride = int(snapshot_stride)
     a.cu_snapshots = _ptr(cu_snapshots)
     a.snapshots = _ptr(snapshots)
+    a.g_logits = _ptr(g_logits)
     return a
 
 
@@ -191,7 +194,7 @@ def kda_prefill_workspace_size(args: PrefillArgs) -> int:
 
 def kda_prefill_chunked(q, k, v, g, beta, cu_seqlens, o, initial_state=None, final_state=None,
                         snapshot_stride=0, cu_snapshots=None, snapshots=None,
-                        cu_seqlens_host=None, workspace=None, stream=None):
+                        cu_seqlens_host=None, workspace=None, stream=None, g_logits=None):
     """Chunked prefill into caller-provided outputs (see include/kda.h).
 
     All tensors are CUDA tensors except ``cu_seqlens_host`` (optional CPU int32).
@@ -200,7 +203,7 @@ def kda_prefill_chunked(q, k, v, g, beta, cu_seqlens, o, initial_state=None, fin
     lib = load()
     host = _host_i32(cu_seqlens_host)
     a = make_prefill_args(q, k, v, g, beta, cu_seqlens, o, initial_state, final_state,
-                          snapshot_stride, cu_snapshots, snapshots, host)
+                          snapshot_stride, cu_snapshots, snapshots, host, g_logits)
     need = int(lib.kda_prefill_workspace_size(ctypes.byref(a)))
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=k.device)
@@ -212,7 +215,8 @@ def kda_prefill_chunked(q, k, v, g, beta, cu_seqlens, o, initial_state=None, fin
 
 
 def make_backward_args(q, k, v, g, beta, cu_seqlens, cu_seqlens_host, d_q, d_k, d_v, d_g, d_beta,
-                       initial_state=None, d_o=None, d_final=None, d_initial=None):
+                       initial_state=None, d_o=None, d_final=None, d_initial=None,
+                       g_logits=None):
     T, H, dk = k.shape
     a = BackwardArgs()
     a.n_req = cu_seqlens.numel() - 1
@@ -224,6 +228,7 @@ def make_backward_args(q, k, v, g, beta, cu_seqlens, cu_seqlens_host, d_q, d_k, 
     a.initial_state, a.d_o, a.d_final = _ptr(initial_state), _ptr(d_o), _ptr(d_final)
     a.d_q, a.d_k, a.d_v, a.d_g, a.d_beta = _ptr(d_q), _ptr(d_k), _ptr(d_v), _ptr(d_g), _ptr(d_beta)
     a.d_initial = _ptr(d_initial)
+    a.g_logits = _ptr(g_logits)
     return a
 
 
@@ -233,7 +238,7 @@ def kda_prefill_backward_workspace_size(args: BackwardArgs) -> int:
 
 def kda_prefill_backward(q, k, v, g, beta, cu_seqlens, cu_seqlens_host, d_q, d_k, d_v, d_g,
                          d_beta, initial_state=None, d_o=None, d_final=None, d_initial=None,
-                         workspace=None, stream=None):
+                         workspace=None, stream=None, g_logits=None):
     """Gradients of sum(d_o * o) + sum(d_final * final_state) of the prefill into
     caller-provided fp32 outputs (see include/kda.h).  ``cu_seqlens_host`` (CPU
     int32) is required; ``workspace`` (uint8 CUDA tensor) is allocated through
@@ -241,7 +246,7 @@ def kda_prefill_backward(q, k, v, g, beta, cu_seqlens, cu_seqlens_host, d_q, d_k
     lib = load()
     host = _host_i32(cu_seqlens_host)
     a = make_backward_args(q, k, v, g, beta, cu_seqlens, host, d_q, d_k, d_v, d_g, d_beta,
-                           initial_state, d_o, d_final, d_initial)
+                           initial_state, d_o, d_final, d_initial, g_logits)
     need = int(lib.kda_prefill_backward_workspace_size(ctypes.byref(a)))
     if workspace is None and need > 0:
         workspace = torch.empty(need, dtype=torch.uint8, device=k.device)
@@ -252,7 +257,8 @@ def kda_prefill_backward(q, k, v, g, beta, cu_seqlens, cu_seqlens_host, d_q, d_k
     return d_q, d_k, d_v, d_g, d_beta, d_initial
 
 
-def kda_chunk_local_state(k, v, g, beta, seg_cu, s_loc, m, seg_cu_host=None, stream=None):
+def kda_chunk_local_state(k, v, g, beta, seg_cu, s_loc, m, seg_cu_host=None, stream=None,
+                          g_logits=None):
     lib = load()
     T, H, dk = k.shape
     a = LocalStateArgs()
@@ -265,6 +271,7 @@ def kda_chunk_local_state(k, v, g, beta, seg_cu, s_loc, m, seg_cu_host=None, str
     host = _host_i32(seg_cu_host)
     a.seg_cu_host = _ptr(host)
     a.s_loc, a.m = _ptr(s_loc), _ptr(m)
+    a.g_logits = _ptr(g_logits)
     _check("kda_chunk_local_state",
            lib.kda_chunk_local_state(ctypes.byref(a), None, 0, _stream(stream)))
     return s_loc, m

@@ -49,6 +49,13 @@ bool overlap(Range a, Range b) {
 
 bool head_dims_supported(int dk, int dv) { return dk == dv && (dk == 64 || dk == 128); }
 
+// The gate is given as exactly one of g (fp32 log alpha) and g_logits (bf16 logits of
+// the fused activation); n = elements.
+bool gate_given(const void *g, const void *g_logits) { return (g != nullptr) != (g_logits != nullptr); }
+Range gate_span(const void *g, const void *g_logits, size_t n) {
+  return g ? span(g, n * 4) : span(g_logits, n * 2);
+}
+
 kda_status check_prefill(const kda_prefill_args *a) {
   if (!a) return KDA_ERR_INVALID_ARG;
   if (a->n_req < 0 || a->total_tokens < 0 || a->H <= 0 || a->dk <= 0 || a->dv <= 0)
@@ -58,11 +65,13 @@ kda_status check_prefill(const kda_prefill_args *a) {
   if (a->snapshot_stride < 0 || a->snapshot_stride % KDA_CHUNK != 0) return KDA_ERR_INVALID_ARG;
   if (a->n_req == 0) return KDA_OK;
   if (!a->cu_seqlens) return KDA_ERR_INVALID_ARG;
-  if (a->total_tokens > 0 && (!a->q || !a->k || !a->v || !a->g || !a->beta || !a->o))
+  if (a->g && a->g_logits) return KDA_ERR_INVALID_ARG;
+  if (a->total_tokens > 0 &&
+      (!a->q || !a->k || !a->v || !gate_given(a->g, a->g_logits) || !a->beta || !a->o))
     return KDA_ERR_INVALID_ARG;
   if (a->snapshot_stride > 0 && (!a->cu_snapshots || !a->snapshots)) return KDA_ERR_INVALID_ARG;
-  const void *ptrs[] = {a->q, a->k, a->v, a->g, a->beta, a->cu_seqlens, a->initial_state,
-                        a->o, a->final_state, a->cu_snapshots, a->snapshots};
+  const void *ptrs[] = {a->q, a->k, a->v, a->g, a->g_logits, a->beta, a->cu_seqlens,
+                        a->initial_state, a->o, a->final_state, a->cu_snapshots, a->snapshots};
   for (const void *p : ptrs)
     if (p && !aligned16(p)) return KDA_ERR_INVALID_ARG;
   if (a->cu_seqlens_host) {
@@ -78,8 +87,9 @@ kda_status check_prefill(const kda_prefill_args *a) {
   const size_t st = n * H * dk * dv * 4;
   Range in[] = {span(a->q, T * H * dk * dsize(a->in_dtype)),
                 span(a->k, T * H * dk * dsize(a->in_dtype)),
-                span(a->v, T * H * dv * dsize(a->in_dtype)), span(a->g, T * H * dk * 4),
-                span(a->beta, T * H * 4), span(a->cu_seqlens, (n + 1) * 4)};
+                span(a->v, T * H * dv * dsize(a->in_dtype)),
+                gate_span(a->g, a->g_logits, T * H * dk), span(a->beta, T * H * 4),
+                span(a->cu_seqlens, (n + 1) * 4)};
   Range o = span(a->o, T * H * dv * dsize(a->out_dtype));
   Range fs = span(a->final_state, st);
   Range is = span(a->initial_state, st);
@@ -142,6 +152,7 @@ kda_status kda_prefill_chunked(const kda_prefill_args *a, void *workspace,
 
   PrefillParams p{};
   p.q = a->q; p.k = a->k; p.v = a->v; p.g = a->g; p.beta = a->beta;
+  p.g_logits = static_cast<const __nv_bfloat16 *>(a->g_logits);
   p.cu_seqlens = a->cu_seqlens;
   p.initial_state = a->initial_state;
   p.o = a->o;
@@ -182,8 +193,10 @@ kda_status kda_chunk_local_state(const kda_local_state_args *a, void *workspace,
   if (!valid_dtype(a->in_dtype)) return KDA_ERR_INVALID_ARG;
   if (!head_dims_supported(a->dk, a->dv)) return KDA_ERR_UNSUPPORTED;
   if (!a->seg_cu || !a->s_loc || !a->m) return KDA_ERR_INVALID_ARG;
-  if (a->total_tokens > 0 && (!a->k || !a->v || !a->g || !a->beta)) return KDA_ERR_INVALID_ARG;
-  const void *ptrs[] = {a->k, a->v, a->g, a->beta, a->seg_cu, a->s_loc, a->m};
+  if (a->g && a->g_logits) return KDA_ERR_INVALID_ARG;
+  if (a->total_tokens > 0 && (!a->k || !a->v || !gate_given(a->g, a->g_logits) || !a->beta))
+    return KDA_ERR_INVALID_ARG;
+  const void *ptrs[] = {a->k, a->v, a->g, a->g_logits, a->beta, a->seg_cu, a->s_loc, a->m};
   for (const void *p : ptrs)
     if (p && !aligned16(p)) return KDA_ERR_INVALID_ARG;
   if (a->seg_cu_host) {
@@ -196,8 +209,9 @@ kda_status kda_chunk_local_state(const kda_local_state_args *a, void *workspace,
                dv = (size_t)a->dv, n = (size_t)a->n_seg;
   Range outs[] = {span(a->s_loc, n * H * dk * dv * 4), span(a->m, n * H * dk * dk * 4)};
   Range ins[] = {span(a->k, T * H * dk * dsize(a->in_dtype)),
-                 span(a->v, T * H * dv * dsize(a->in_dtype)), span(a->g, T * H * dk * 4),
-                 span(a->beta, T * H * 4), span(a->seg_cu, (n + 1) * 4)};
+                 span(a->v, T * H * dv * dsize(a->in_dtype)),
+                 gate_span(a->g, a->g_logits, T * H * dk), span(a->beta, T * H * 4),
+                 span(a->seg_cu, (n + 1) * 4)};
   if (overlap(outs[0], outs[1])) return KDA_ERR_INVALID_ARG;
   for (Range o : outs)
     for (Range i : ins)
@@ -205,6 +219,7 @@ kda_status kda_chunk_local_state(const kda_local_state_args *a, void *workspace,
 
   PrefillParams p{};
   p.k = a->k; p.v = a->v; p.g = a->g; p.beta = a->beta;
+  p.g_logits = static_cast<const __nv_bfloat16 *>(a->g_logits);
   p.cu_seqlens = a->seg_cu;
   p.n_req = a->n_seg; p.total_tokens = a->total_tokens;
   p.H = a->H; p.dk = a->dk; p.dv = a->dv;
@@ -390,20 +405,23 @@ kda_status check_backward(const kda_backward_args *a, BwdShape *sh) {
   }
   if (n_chunks * a->H > 0x7fffffffLL || (long long)a->n_req * a->H > 0x7fffffffLL)
     return KDA_ERR_UNSUPPORTED;
-  if (a->total_tokens > 0 && (!a->q || !a->k || !a->v || !a->g || !a->beta || !a->d_q ||
-                              !a->d_k || !a->d_v || !a->d_g || !a->d_beta))
+  if (a->g && a->g_logits) return KDA_ERR_INVALID_ARG;
+  if (a->total_tokens > 0 &&
+      (!a->q || !a->k || !a->v || !gate_given(a->g, a->g_logits) || !a->beta || !a->d_q ||
+       !a->d_k || !a->d_v || !a->d_g || !a->d_beta))
     return KDA_ERR_INVALID_ARG;
-  const void *ptrs[] = {a->q, a->k, a->v, a->g, a->beta, a->cu_seqlens, a->initial_state,
-                        a->d_o, a->d_final, a->d_q, a->d_k, a->d_v, a->d_g, a->d_beta,
-                        a->d_initial};
+  const void *ptrs[] = {a->q, a->k, a->v, a->g, a->g_logits, a->beta, a->cu_seqlens,
+                        a->initial_state, a->d_o, a->d_final, a->d_q, a->d_k, a->d_v, a->d_g,
+                        a->d_beta, a->d_initial};
   for (const void *p : ptrs)
     if (p && !aligned16(p)) return KDA_ERR_INVALID_ARG;
   const size_t T = (size_t)a->total_tokens, H = (size_t)a->H, dk = (size_t)a->dk,
                dv = (size_t)a->dv, n = (size_t)a->n_req;
   Range ins[] = {span(a->q, T * H * dk * dsize(a->in_dtype)),
                  span(a->k, T * H * dk * dsize(a->in_dtype)),
-                 span(a->v, T * H * dv * dsize(a->in_dtype)), span(a->g, T * H * dk * 4),
-                 span(a->beta, T * H * 4), span(a->cu_seqlens, (n + 1) * 4),
+                 span(a->v, T * H * dv * dsize(a->in_dtype)),
+                 gate_span(a->g, a->g_logits, T * H * dk), span(a->beta, T * H * 4),
+                 span(a->cu_seqlens, (n + 1) * 4),
                  span(a->initial_state, n * H * dk * dv * 4), span(a->d_o, T * H * dv * 4),
                  span(a->d_final, n * H * dk * dv * 4)};
   Range outs[] = {span(a->d_q, T * H * dk * 4), span(a->d_k, T * H * dk * 4),
@@ -483,6 +501,7 @@ extern "C" kda_status kda_prefill_backward(const kda_backward_args *a, void *wor
   if (sh.n_chunks > 0) {
     PrefillParams p{};
     p.q = a->q; p.k = a->k; p.v = a->v; p.g = a->g; p.beta = a->beta;
+    p.g_logits = static_cast<const __nv_bfloat16 *>(a->g_logits);
     p.cu_seqlens = a->cu_seqlens;
     p.initial_state = a->initial_state;
     p.cu_snapshots = reinterpret_cast<const int32_t *>(ws + o_cu_snap);
@@ -503,6 +522,7 @@ extern "C" kda_status kda_prefill_backward(const kda_backward_args *a, void *wor
   }
   BackwardLaunch b{};
   b.q = a->q; b.k = a->k; b.v = a->v; b.g = a->g; b.beta = a->beta;
+  b.g_logits = static_cast<const __nv_bfloat16 *>(a->g_logits);
   b.initial_state = a->initial_state; b.d_o = a->d_o; b.d_final = a->d_final;
   b.dq = a->d_q; b.dk = a->d_k; b.dv = a->d_v; b.dg = a->d_g; b.dbeta = a->d_beta;
   b.d_initial = a->d_initial;

@@ -60,6 +60,8 @@ constexpr float LOG2E = 1.4426950408889634f;
 struct BwdParams {
   const void *q, *k, *v;
   const float *g, *beta;
+  const __nv_bfloat16 *g_logits;  // when set (g NULL): log alpha = -5 sigmoid(logit), and dg
+                                  // is the gradient of the logits
   const float *initial_state;  // NULL = zeros
   const float *d_o;            // NULL = zeros
   const float *d_final;        // NULL = zeros
@@ -216,16 +218,26 @@ __device__ void stage_rows(float *dst, int ld, const TIn *src, int tok0, int n, 
 // (thread = channel); beta into sB.  Padded rows have g = 0 and beta = 0.
 template <int D>
 __device__ void stage_gate(float *sG, float *sB, const BwdParams &p, int tok0, int n, int h) {
-  stage_rows<D, float>(sG, D, p.g, tok0, n, p.H, h);
+  if (p.g_logits)
+    stage_rows<D, __nv_bfloat16>(sG, D, p.g_logits, tok0, n, p.H, h);
+  else
+    stage_rows<D, float>(sG, D, p.g, tok0, n, p.H, h);
   if (threadIdx.x < C)
     sB[threadIdx.x] = threadIdx.x < n ? p.beta[(size_t)(tok0 + threadIdx.x) * p.H + h] : 0.f;
   __syncthreads();
   if (threadIdx.x < D) {
     const int c = threadIdx.x;
     float run = 0.f;
-    for (int t = 0; t < C; ++t) {
-      run += sG[t * D + c];
-      sG[t * D + c] = run * LOG2E;
+    if (p.g_logits) {
+      for (int t = 0; t < C; ++t) {
+        run += t < n ? gate_from_logit(sG[t * D + c]) : 0.f;
+        sG[t * D + c] = run * LOG2E;
+      }
+    } else {
+      for (int t = 0; t < C; ++t) {
+        run += sG[t * D + c];
+        sG[t * D + c] = run * LOG2E;
+      }
     }
   }
   __syncthreads();
@@ -1209,12 +1221,18 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
       }
     }
   __syncthreads();
-  if (tid < D) {
+  if (tid < D) {  // dg = reverse cumulative sum of dG over the chunk, in place
     float run = sExtra[tid];
     for (int t = C - 1; t >= 0; --t) {
       run += sV[t * D + tid];
-      if (t < n) p.dg[((size_t)(tok0 + t) * H + h) * D + tid] = run;
+      sV[t * D + tid] = run;
     }
+  }
+  __syncthreads();
+  // stored by the whole CTA; for gate logits x, times d log(alpha) / dx
+  for (int e = tid; e < n * D; e += NTH) {
+    const size_t o = ((size_t)(tok0 + e / D) * H + h) * D + e % D;
+    p.dg[o] = p.g_logits ? sV[e] * gate_logit_slope(__bfloat162float(p.g_logits[o])) : sV[e];
   }
   if (tid < C && tid < n) p.dbeta[(size_t)(tok0 + tid) * H + h] = sDb[tid];
 }
@@ -1289,7 +1307,7 @@ cudaError_t launch_backward(const BackwardLaunch &b, cudaStream_t stream) {
   const BwdWorkspace w = backward_workspace(b.n_req, b.n_chunks, b.n_snap, b.H, b.D);
   char *ws = static_cast<char *>(b.workspace);
   BwdParams p{};
-  p.q = b.q; p.k = b.k; p.v = b.v; p.g = b.g; p.beta = b.beta;
+  p.q = b.q; p.k = b.k; p.v = b.v; p.g = b.g; p.beta = b.beta; p.g_logits = b.g_logits;
   p.initial_state = b.initial_state; p.d_o = b.d_o; p.d_final = b.d_final;
   p.dq = b.dq; p.dk = b.dk; p.dv = b.dv; p.dg = b.dg; p.dbeta = b.dbeta;
   p.d_initial = b.d_initial;

@@ -31,6 +31,7 @@ __device__ __forceinline__ void set_status(unsigned int *status, unsigned int bi
 struct PrefillParams {
   const void *q, *k, *v;
   const float *g, *beta;
+  const __nv_bfloat16 *g_logits;  // when set (g NULL): log(alpha) = -5 sigmoid(logit)
   const int32_t *cu_seqlens;
   const int32_t *order;          // work order over requests (longest first) or NULL
   const float *initial_state;    // NULL = zeros
@@ -84,6 +85,7 @@ unsigned int *device_status_word();  // address of the current device's status w
 struct BackwardLaunch {
   const void *q, *k, *v;
   const float *g, *beta, *initial_state, *d_o, *d_final;
+  const __nv_bfloat16 *g_logits;  // when set (g NULL), dg is the gradient of the logits
   float *dq, *dk, *dv, *dg, *dbeta, *d_initial;
   void *workspace;
   int n_req, n_chunks, n_snap, H, D;
@@ -93,6 +95,24 @@ cudaError_t launch_backward(const BackwardLaunch &b, cudaStream_t stream);
 size_t backward_workspace_bytes(int n_req, int n_chunks, int n_snap, int H, int D);
 void backward_offsets(int n_req, int n_chunks, int n_snap, int H, int D, size_t *chunks,
                       size_t *cu_chunks, size_t *cu_snap, size_t *snaps, size_t *zero);
+
+// Fused gate activation: the lower-bounded decay log(alpha) = -5 sigmoid(x) of a
+// gate logit x, which lies in [-5, 0] for every x (alpha >= exp(-5)), and its
+// derivative d log(alpha) / dx = -5 sigmoid(x) (1 - sigmoid(x)).  The sigmoid is
+// 1 / (1 + 2^(-x log2 e)) with the approximate ex2 and rcp instructions (relative
+// error a few 1e-7); for x below about -88 the power is +inf and the gate is 0, the
+// limit.
+__device__ __forceinline__ float gate_sigmoid(float x) {
+  float e, r;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(e) : "f"(-1.4426950408889634f * x));
+  asm("rcp.approx.ftz.f32 %0, %1;" : "=f"(r) : "f"(1.f + e));
+  return r;
+}
+__device__ __forceinline__ float gate_from_logit(float x) { return kGateLower * gate_sigmoid(x); }
+__device__ __forceinline__ float gate_logit_slope(float x) {
+  const float s = gate_sigmoid(x);
+  return kGateLower * s * (1.f - s);
+}
 
 // Element loads/stores shared by the kernels.
 __device__ __forceinline__ float load_elem(const float *p, size_t i) { return p[i]; }

@@ -111,8 +111,12 @@ __global__ void __launch_bounds__(kThreads, 1) prefill_simt_kernel(const Prefill
         const size_t off = ((size_t)(bos + c0 + i) * H + h) * DK + c;
         kk = load_elem(gk, off);
         if (go) qq = load_elem(gq, off);
-        gg = p.g[off];
-        if (p.validate && !(gg >= kGateLower && gg <= 0.f)) set_status(p.status, STATUS_GATE_RANGE);
+        if (p.g_logits) {
+          gg = gate_from_logit(__bfloat162float(p.g_logits[off]));
+        } else {
+          gg = p.g[off];
+          if (p.validate && !(gg >= kGateLower && gg <= 0.f)) set_status(p.status, STATUS_GATE_RANGE);
+        }
       }
       sK[idx] = kk;
       sQ[idx] = qq;

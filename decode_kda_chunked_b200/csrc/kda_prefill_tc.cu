@@ -58,8 +58,10 @@ constexpr float LOG2E = 1.4426950408889634f;
 constexpr uint32_t OFF_KRAW = 0;        // bf16 [64 x 128]: 2 TMA boxes of 64 cols (SW128)
 constexpr uint32_t OFF_QRAW = 16384;
 constexpr uint32_t OFF_VRAW = 32768;
-constexpr uint32_t OFF_GRAW = 49152;    // fp32 [64 x 128]: 4 TMA boxes of 32 cols (SW128);
-                                        // rewritten in place with log2(e) * cumsum(g)
+constexpr uint32_t OFF_GRAW = 49152;    // fp32 [64 x 128]: 4 TMA boxes of 32 cols (SW128), or
+                                        // bf16 gate logits in its first half (2 boxes of 64
+                                        // cols, as q/k/v); rewritten in place with
+                                        // log2(e) * cumsum(g)
 constexpr uint32_t RAW_BYTES = 81920;
 // Once every raw tile is read, the raw region holds the B operands R'_a of
 // the A|P products: row block a has 16(a+1) rows at byte 8192 a(a+1)/2.
@@ -131,7 +133,8 @@ __device__ __forceinline__ float tf32_rna(float x) {
 // walk on 32 distinct banks and keeps addresses affine in the loop indices.
 __device__ __forceinline__ int rot(int r, int c) { return r * LDT + c; }
 
-template <typename TOut>
+// LOGITS: the gate arrives as bf16 logits (fused gate activation) instead of fp32 g.
+template <typename TOut, bool LOGITS>
 __global__ void __launch_bounds__(NT + 32, 1)
     prefill_tc_kernel(const PrefillParams p, const __grid_constant__ TcMaps maps) {
   extern __shared__ unsigned char smem_raw[];
@@ -170,6 +173,7 @@ __global__ void __launch_bounds__(NT + 32, 1)
   const int r = p.order ? p.order[rem / H] : rem / H;
   const int h = rem % H;
   const bool load_q = !p.local_mode;
+  constexpr bool logits = LOGITS;
   const bool zero_v = p.local_mode && part == 1;
   const int bos = p.cu_seqlens[r], eos = p.cu_seqlens[r + 1];
   const int len = eos - bos;
@@ -212,7 +216,7 @@ __global__ void __launch_bounds__(NT + 32, 1)
       tma_prefetch_desc(&maps.v);
       tma_prefetch_desc(&maps.g);
       auto issue_tma = [&](int c0) {
-        mbar_expect_tx(bar_tma, load_q ? RAW_BYTES : RAW_BYTES - 16384u);
+        mbar_expect_tx(bar_tma, RAW_BYTES - (load_q ? 0u : 16384u) - (logits ? 16384u : 0u));
         const int y = bos + c0;
         for (int half = 0; half < 2; ++half) {
           const int x = h * DH + 64 * half;
@@ -220,8 +224,13 @@ __global__ void __launch_bounds__(NT + 32, 1)
           if (load_q) tma_load_2d(sm + OFF_QRAW + 8192 * half, &maps.q, x, y, bar_tma);
           tma_load_2d(sm + OFF_VRAW + 8192 * half, &maps.v, x, y, bar_tma);
         }
-        for (int qd = 0; qd < 4; ++qd)
-          tma_load_2d(sm + OFF_GRAW + 8192 * qd, &maps.g, h * DH + 32 * qd, y, bar_tma);
+        if (logits) {
+          for (int half = 0; half < 2; ++half)
+            tma_load_2d(sm + OFF_GRAW + 8192 * half, &maps.g, h * DH + 64 * half, y, bar_tma);
+        } else {
+          for (int qd = 0; qd < 4; ++qd)
+            tma_load_2d(sm + OFF_GRAW + 8192 * qd, &maps.g, h * DH + 32 * qd, y, bar_tma);
+        }
       };
       uint32_t ph_raw = 0, ph_opsap[1] = {0}, ph_ops = 0, ph_u = 0, ph_st = 0;
       auto cwait = [&](uint64_t *bar, uint32_t &ph) -> bool {
@@ -350,14 +359,24 @@ __global__ void __launch_bounds__(NT + 32, 1)
       beta_next = load_beta(c0 + C);
 
       // ---- a2: cumulative gate (thread = channel l, tokens 16g..16g+15) --------
+      // Every thread reads its raw gates before the first worker sync and writes the
+      // cumulative ones only after it, so the bf16 logits can share the region.
       {
         float gv[16];
+        if (logits) {
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int t = 16 * g + j;
-          gv[j] = (t < n) ? *reinterpret_cast<const float *>(sm + OFF_GRAW + g_off(t, l)) : 0.f;
+          for (int j = 0; j < 16; ++j) {
+            const int t = 16 * g + j;
+            gv[j] = (t < n) ? gate_from_logit(bf16_at(sm + OFF_GRAW, t, l)) : 0.f;
+          }
+        } else {
+#pragma unroll
+          for (int j = 0; j < 16; ++j) {
+            const int t = 16 * g + j;
+            gv[j] = (t < n) ? *reinterpret_cast<const float *>(sm + OFF_GRAW + g_off(t, l)) : 0.f;
+          }
         }
-        if (p.validate)
+        if (p.validate && !logits)
 #pragma unroll
           for (int j = 0; j < 16; ++j)
             if (!(gv[j] >= kGateLower && gv[j] <= 0.f)) set_status(p.status, STATUS_GATE_RANGE);
@@ -722,22 +741,22 @@ cudaError_t launch_prefill_tc(const PrefillParams &p, kda_dtype in_dtype, kda_dt
   if (!encode_map(&maps.q, p.q ? p.q : p.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W, T, 64) ||
       !encode_map(&maps.k, p.k, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W, T, 64) ||
       !encode_map(&maps.v, p.v, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W, T, 64) ||
-      !encode_map(&maps.g, p.g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, W, T, 32))
+      !(p.g_logits ? encode_map(&maps.g, p.g_logits, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W, T, 64)
+                   : encode_map(&maps.g, p.g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, W, T, 32)))
     return cudaErrorInvalidValue;
   const unsigned grid = (unsigned)(p.n_req * p.H * (p.local_mode ? 2 : 1));
-  cudaError_t e;
-  if (out_dtype == KDA_BF16) {
-    e = cudaFuncSetAttribute(prefill_tc_kernel<__nv_bfloat16>,
-                             cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_ALLOC);
+  auto run = [&](auto kernel) -> cudaError_t {
+    const cudaError_t e =
+        cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_ALLOC);
     if (e != cudaSuccess) return e;
-    prefill_tc_kernel<__nv_bfloat16><<<grid, NT + 32, SMEM_ALLOC, stream>>>(p, maps);
-  } else {
-    e = cudaFuncSetAttribute(prefill_tc_kernel<float>, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                             (int)SMEM_ALLOC);
-    if (e != cudaSuccess) return e;
-    prefill_tc_kernel<float><<<grid, NT + 32, SMEM_ALLOC, stream>>>(p, maps);
-  }
-  return cudaGetLastError();
+    kernel<<<grid, NT + 32, SMEM_ALLOC, stream>>>(p, maps);
+    return cudaGetLastError();
+  };
+  const bool logits = p.g_logits != nullptr;
+  if (out_dtype == KDA_BF16)
+    return logits ? run(prefill_tc_kernel<__nv_bfloat16, true>)
+                  : run(prefill_tc_kernel<__nv_bfloat16, false>);
+  return logits ? run(prefill_tc_kernel<float, true>) : run(prefill_tc_kernel<float, false>);
 }
 
 }  // namespace kda

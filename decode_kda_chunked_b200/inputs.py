@@ -14,6 +14,10 @@ Distributions (the five standard workloads below):
     so alpha >= exp(-5) (the lower-bounded decay of KDA, CSDN post on the
     Kimi K3 technical report, section 一.1);
   * initial states ~ N(0, std) fp32 where a workload asks for one.
+
+With ``gate_logits=True`` the gate's N(0, 1) draw is kept as bf16 logits
+``g_logits`` instead (for the fused gate activation, which applies
+-5 * sigmoid itself) and ``g`` is None; every other draw is unchanged.
 """
 from __future__ import annotations
 
@@ -36,6 +40,7 @@ class PrefillInputs:
     lengths: list              # host copy of the request lengths
     initial_state: torch.Tensor | None  # [n_req, H, dk, dv] fp32 or None
     meta: dict = field(default_factory=dict)
+    g_logits: torch.Tensor | None = None  # [T, H, dk] bf16 gate logits (g is None then)
 
     @property
     def total_tokens(self) -> int:
@@ -49,7 +54,7 @@ class PrefillInputs:
         mv = lambda t: None if t is None else t.to(device)
         return PrefillInputs(mv(self.q), mv(self.k), mv(self.v), mv(self.g), mv(self.beta),
                              mv(self.cu_seqlens), list(self.lengths), mv(self.initial_state),
-                             dict(self.meta))
+                             dict(self.meta), mv(self.g_logits))
 
 
 def _gen(seed: int, device) -> torch.Generator:
@@ -66,7 +71,8 @@ def _unit_rows(shape, gen, device, dtype):
 
 def make_prefill_inputs(lengths, H: int, dk: int, dv: int, dtype=torch.bfloat16,
                         seed: int = 0, s0_std: float | None = None, device="cpu",
-                        gate_scale: float = -GATE_LOWER) -> PrefillInputs:
+                        gate_scale: float = -GATE_LOWER,
+                        gate_logits: bool = False) -> PrefillInputs:
     """Packed varlen inputs for ``len(lengths)`` requests of the given lengths."""
     lengths = [int(x) for x in lengths]
     T = sum(lengths)
@@ -74,16 +80,17 @@ def make_prefill_inputs(lengths, H: int, dk: int, dv: int, dtype=torch.bfloat16,
     q = _unit_rows((T, H, dk), gen, device, dtype)
     k = _unit_rows((T, H, dk), gen, device, dtype)
     v = torch.randn((T, H, dv), generator=gen, device=device, dtype=torch.float32).to(dtype)
-    g = -gate_scale * torch.sigmoid(
-        torch.randn((T, H, dk), generator=gen, device=device, dtype=torch.float32))
+    z = torch.randn((T, H, dk), generator=gen, device=device, dtype=torch.float32)
+    x = z.to(torch.bfloat16).contiguous() if gate_logits else None
+    g = None if gate_logits else (-gate_scale * torch.sigmoid(z)).contiguous()
     beta = torch.sigmoid(torch.randn((T, H), generator=gen, device=device, dtype=torch.float32))
     s0 = None
     if s0_std is not None:
         s0 = s0_std * torch.randn((len(lengths), H, dk, dv), generator=gen, device=device,
                                   dtype=torch.float32)
     cu = torch.tensor([0] + list(_cumsum(lengths)), dtype=torch.int32, device=device)
-    return PrefillInputs(q, k, v, g.contiguous(), beta.contiguous(), cu, lengths, s0,
-                         {"seed": seed, "dtype": str(dtype).replace("torch.", "")})
+    return PrefillInputs(q, k, v, g, beta.contiguous(), cu, lengths, s0,
+                         {"seed": seed, "dtype": str(dtype).replace("torch.", "")}, x)
 
 
 def _cumsum(xs):
@@ -135,9 +142,10 @@ def varlen_lengths(seed: int = 0) -> list:
     return loguniform_lengths(VARLEN_N, VARLEN_LO, VARLEN_HI, seed)
 
 
-def varlen(device="cpu", seed: int = 0) -> PrefillInputs:
+def varlen(device="cpu", seed: int = 0, gate_logits: bool = False) -> PrefillInputs:
     return make_prefill_inputs(varlen_lengths(seed), H=32, dk=128, dv=128,
-                               dtype=torch.bfloat16, seed=seed, s0_std=None, device=device)
+                               dtype=torch.bfloat16, seed=seed, s0_std=None, device=device,
+                               gate_logits=gate_logits)
 
 
 MILLION_T, MILLION_SEGMENTS, SNAPSHOT_STRIDE = 1 << 20, 16, 512

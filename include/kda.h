@@ -90,6 +90,7 @@ typedef enum { KDA_BF16 = 0, KDA_F32 = 1 } kda_dtype;
  *                  Precondition -5 <= g <= 0 (alpha >= exp(-5)): the
  *                  lower-bounded decay that keeps the chunked form's
  *                  exponentials finite.  Checked only when KDA_VALIDATE=1.
+ *                  NULL when g_logits is given (exactly one of the two).
  *   beta           [T_total, H] fp32, precondition 0 <= beta <= 1.
  *   cu_seqlens     DEVICE int32 [n_req + 1]; cu_seqlens[0] == 0, non-decreasing.
  *                  Request r owns tokens cu_seqlens[r] .. cu_seqlens[r+1]-1.
@@ -114,6 +115,13 @@ typedef enum { KDA_BF16 = 0, KDA_F32 = 1 } kda_dtype;
  *                  tokens, stored at row cu_snapshots[r] + j - 1.  When L_r is
  *                  a multiple of the stride the last snapshot equals the
  *                  final state.
+ *   g_logits       fused gate activation: NULL, or bf16 [T_total, H, dk] gate
+ *                  logits x with g == NULL.  The kernels then use
+ *                  log(alpha) = -5 * sigmoid(x), computed in fp32 as the tiles
+ *                  are loaded: the lower-bounded decay (CSDN post on the Kimi
+ *                  K3 technical report, section 一.1), alpha >= exp(-5) for
+ *                  every x, with half the gate bytes of fp32 g and no range
+ *                  precondition.
  */
 typedef struct kda_prefill_args {
   int32_t n_req;
@@ -132,6 +140,7 @@ typedef struct kda_prefill_args {
   int32_t snapshot_stride;
   const int32_t *cu_snapshots;
   float *snapshots;
+  const void *g_logits;
 } kda_prefill_args;
 
 /* Bytes of device workspace kda_prefill_chunked needs for these arguments
@@ -209,6 +218,8 @@ kda_status kda_prefill_chunked_noalloc(const kda_prefill_args *args, void *strea
  *   seg_cu_host    optional HOST copy (may be NULL), used only for validation.
  *   s_loc          [n_seg, H, dk, dv] fp32 output.
  *   m              [n_seg, H, dk, dk] fp32 output (row-major: m[.., i, j]).
+ *   g_logits       as in kda_prefill_args: bf16 gate logits instead of g
+ *                  (then g == NULL).
  */
 typedef struct kda_local_state_args {
   int32_t n_seg;
@@ -222,6 +233,7 @@ typedef struct kda_local_state_args {
   const int32_t *seg_cu_host;
   float *s_loc;
   float *m;
+  const void *g_logits;
 } kda_local_state_args;
 
 size_t kda_local_state_workspace_size(const kda_local_state_args *args);
@@ -315,6 +327,9 @@ kda_status kda_decode_step(const kda_decode_args *args, void *stream);
  *   d_v             fp32 [total_tokens, H, dv] output: gradient of v.
  *   d_beta          fp32 [total_tokens, H] output: gradient of beta.
  *   d_initial       fp32 [n_req, H, dk, dv] output, or NULL (not returned).
+ *   g_logits        as in kda_prefill_args: bf16 gate logits x instead of g
+ *                   (then g == NULL).  d_g then receives dL/dx, the gradient
+ *                   of the logits: dL/dg * (-5) sigmoid(x) (1 - sigmoid(x)).
  * Outputs must not overlap each other, the inputs or the workspace.  The
  * workspace (kda_prefill_backward_workspace_size bytes, 256-byte aligned) is
  * scratch owned by the caller for the duration of the call.  The host tables
@@ -336,6 +351,7 @@ typedef struct kda_backward_args {
   const float *d_final;
   float *d_q, *d_k, *d_v, *d_g, *d_beta;
   float *d_initial;
+  const void *g_logits;
 } kda_backward_args;
 
 /* Workspace bytes for kda_prefill_backward (0 if the arguments are invalid). */

@@ -122,16 +122,44 @@ def snapshot_counts(cu_seqlens, stride: int) -> np.ndarray:
     return lens // stride if stride > 0 else np.zeros_like(lens)
 
 
+def gate_from_logits(x):
+    """log(alpha) = -5 sigmoid(x) of gate logits x, in fp64.
+
+    The lower-bounded decay of KDA (CSDN post on the Kimi K3 technical report,
+    section 一.1): alpha >= exp(-5) for every logit, the bound every workload's
+    gate is drawn under.  The pages give the bound, not the squashing function;
+    the logistic sigmoid scaled to [-5, 0] is the plainest map onto that range."""
+    x = _f64(x)
+    with np.errstate(over="ignore"):
+        return -5.0 / (1.0 + np.exp(-x))
+
+
+def gate_logit_slope(x):
+    """d log(alpha) / dx of ``gate_from_logits``: -5 sigmoid(x) (1 - sigmoid(x))."""
+    x = _f64(x)
+    with np.errstate(over="ignore"):
+        s = 1.0 / (1.0 + np.exp(-x))
+    return -5.0 * s * (1.0 - s)
+
+
+def _gate(g, g_logits):
+    if (g is None) == (g_logits is None):
+        raise ValueError("give exactly one of g and g_logits")
+    return _f64(g) if g is not None else gate_from_logits(g_logits)
+
+
 def prefill(q, k, v, g, beta, cu_seqlens, initial_state=None, snapshot_stride: int = 0,
-            want_o: bool = True, n_threads: int | None = None, lib=None):
+            want_o: bool = True, n_threads: int | None = None, lib=None, g_logits=None):
     """Token-by-token KDA over packed varlen requests.
 
     q, k, g: [T, H, dk]; v: [T, H, dv]; beta: [T, H]; cu_seqlens: [n_req + 1];
-    initial_state: [n_req, H, dk, dv] or None (zeros).
+    initial_state: [n_req, H, dk, dv] or None (zeros).  With ``g=None``, the gate
+    is ``gate_from_logits(g_logits)``.
     Returns dict(o=[T,H,dv] or None, final_state=[n_req,H,dk,dv],
     snapshots=[n_snap,H,dk,dv], cu_snapshots=[n_req+1]).
     """
     lib = lib or load()
+    g = _gate(g, g_logits)
     q, k, v, g, beta = (_f64(a) for a in (q, k, v, g, beta))
     s0 = _f64(initial_state)
     cu = _i64(cu_seqlens)
@@ -155,14 +183,17 @@ def prefill(q, k, v, g, beta, cu_seqlens, initial_state=None, snapshot_stride: i
 
 
 def prefill_backward(q, k, v, g, beta, cu_seqlens, initial_state=None, d_o=None,
-                     d_final=None, n_threads: int | None = None, lib=None):
+                     d_final=None, n_threads: int | None = None, lib=None, g_logits=None):
     """Gradients of L = sum(d_o * o) + sum(d_final * final_state) of the prefill
     map, by reverse mode through the recurrence's defining lines
     (``oracle_kda_prefill_backward`` in kda_oracle.c).
 
     Returns dict(dq, dk, dv, dg, dbeta, d_initial) shaped like the inputs
-    (d_initial [n_req, H, dk, dv]).  d_o / d_final / initial_state may be None."""
+    (d_initial [n_req, H, dk, dv]).  d_o / d_final / initial_state may be None.
+    With ``g=None`` the gate is ``gate_from_logits(g_logits)`` and ``dg`` is the
+    gradient of the logits (the chain rule through ``gate_logit_slope``)."""
     lib = lib or load()
+    g = _gate(g, g_logits)
     q, k, v, g, beta = (_f64(a) for a in (q, k, v, g, beta))
     s0, do, dfin = _f64(initial_state), _f64(d_o), _f64(d_final)
     cu = _i64(cu_seqlens)
@@ -178,6 +209,8 @@ def prefill_backward(q, k, v, g, beta, cu_seqlens, initial_state=None, d_o=None,
         _p(out["d_initial"]), int(n_threads or default_threads()))
     if rc != 0:
         raise ValueError(f"oracle_kda_prefill_backward failed with code {rc}")
+    if g_logits is not None:
+        out["dg"] = out["dg"] * gate_logit_slope(g_logits)
     return out
 
 
@@ -201,9 +234,12 @@ def decode_step(q, k, v, g, beta, state, slot=None, n_threads: int | None = None
     return o
 
 
-def chunk_local_state(k, v, g, beta, seg_cu, n_threads: int | None = None, lib=None):
-    """Per segment and head: (S_loc [n_seg,H,dk,dv], M [n_seg,H,dk,dk])."""
+def chunk_local_state(k, v, g, beta, seg_cu, n_threads: int | None = None, lib=None,
+                      g_logits=None):
+    """Per segment and head: (S_loc [n_seg,H,dk,dv], M [n_seg,H,dk,dk]).  With
+    ``g=None`` the gate is ``gate_from_logits(g_logits)``."""
     lib = lib or load()
+    g = _gate(g, g_logits)
     k, v, g, beta = (_f64(a) for a in (k, v, g, beta))
     seg = _i64(seg_cu)
     _, H, dk = k.shape

@@ -24,6 +24,12 @@ post on the Kimi K3 technical report, section 一.1):
   * pin_decode_matches_prefill L decode steps == a prefill of L tokens
   * pin_decode_slots          decode writes the slot it is told to and no other
   * pin_varlen_isolation      a packed request equals the same request run alone
+  * pin_gate_logit_map        the fused gate activation log(alpha) = -5 sigmoid(x):
+                              exact values, the reflection g(x) + g(-x) = -5, the
+                              range, and its slope against central differences
+  * pin_gate_logit_decay      beta = 0 with zero logits: S_t = exp(-2.5 t) S_0
+  * pin_gate_logit_backward   the logits' gradient against central differences of
+                              the forward loss in the logits
 """
 from __future__ import annotations
 
@@ -587,10 +593,82 @@ def pin_backward_chunked_form(lib):
                                            atol=1e-9 * max(1.0, np.abs(r["d_initial"]).max()))
 
 
+# ----------------------------------------------------------------------------
+# Fused gate activation: log(alpha) = -5 sigmoid(x) of bf16 logits x (the
+# lower-bounded decay, CSDN post on the Kimi K3 technical report, section 一.1)
+# ----------------------------------------------------------------------------
+
+def pin_gate_logit_map(lib):
+    """Values fixed by the sigmoid itself: g(0) = -2.5, g(x) + g(-x) = -5 (as
+    sigmoid(x) + sigmoid(-x) = 1), g in [-5, 0] and decreasing, the limits -0 and
+    -5 at the ends of the range, and the slope equal to central differences."""
+    del lib
+    assert oracle.gate_from_logits(np.array([0.0]))[0] == -2.5
+    x = np.linspace(-30.0, 30.0, 601)
+    gx = oracle.gate_from_logits(x)
+    np.testing.assert_allclose(gx + oracle.gate_from_logits(-x), -5.0, rtol=0, atol=1e-14)
+    assert np.all(gx <= 0.0) and np.all(gx >= -5.0) and np.all(np.diff(gx) < 0.0)
+    ends = oracle.gate_from_logits(np.array([-800.0, 800.0]))
+    assert ends[0] == 0.0 and ends[1] == -5.0
+    h = 1e-5
+    fd = (oracle.gate_from_logits(x + h) - oracle.gate_from_logits(x - h)) / (2 * h)
+    np.testing.assert_allclose(oracle.gate_logit_slope(x), fd, rtol=0, atol=1e-9)
+
+
+def pin_gate_logit_decay(lib):
+    """beta = 0 and every logit 0: alpha = exp(-2.5) on every channel, so
+    S_t = exp(-2.5 t) S_0 and o_t = S_t^T q_t (the decay closed form)."""
+    x = rand_inputs([6, 9], H=2, dk=4, dv=3, seed=83, s0_std=1.0)
+    x["beta"][:] = 0.0
+    logits = np.zeros_like(x["g"])
+    r = oracle.prefill(x["q"], x["k"], x["v"], None, x["beta"], x["cu"], x["s0"],
+                       n_threads=2, lib=lib, g_logits=logits)
+    for req in range(2):
+        lo, hi = x["cu"][req], x["cu"][req + 1]
+        for h in range(2):
+            for i, t in enumerate(range(lo, hi)):
+                St = np.exp(-2.5 * (i + 1)) * x["s0"][req, h]
+                np.testing.assert_allclose(r["o"][t, h], St.T @ x["q"][t, h], rtol=1e-12,
+                                           atol=1e-15)
+            np.testing.assert_allclose(r["final_state"][req, h],
+                                       np.exp(-2.5 * (hi - lo)) * x["s0"][req, h],
+                                       rtol=1e-12, atol=1e-15)
+
+
+def pin_gate_logit_backward(lib):
+    """The gradient the backward returns for logits equals central differences of
+    the forward loss taken in the logits themselves."""
+    x = rand_inputs([5, 8], H=2, dk=3, dv=2, seed=84, s0_std=1.0)
+    rng = _rng(85)
+    logits = rng.standard_normal(x["g"].shape)
+    d_o = rng.standard_normal(x["v"].shape)
+    d_fin = rng.standard_normal(x["s0"].shape)
+
+    def loss(lg):
+        r = oracle.prefill(x["q"], x["k"], x["v"], None, x["beta"], x["cu"], x["s0"],
+                           n_threads=2, lib=lib, g_logits=lg)
+        return float((r["o"] * d_o).sum() + (r["final_state"] * d_fin).sum())
+
+    grads = oracle.prefill_backward(x["q"], x["k"], x["v"], None, x["beta"], x["cu"], x["s0"],
+                                    d_o, d_fin, n_threads=2, lib=lib, g_logits=logits)
+    scale = max(np.abs(grads["dg"]).max(), 1e-12)
+    h = 1e-6
+    for ix in np.ndindex(logits.shape):
+        keep = logits[ix]
+        logits[ix] = keep + h
+        lp = loss(logits)
+        logits[ix] = keep - h
+        lm = loss(logits)
+        logits[ix] = keep
+        fd = (lp - lm) / (2 * h)
+        assert abs(fd - grads["dg"][ix]) <= 1e-6 * scale, (ix, fd, grads["dg"][ix])
+
+
 ALL_PINS = [pin_identity_beta0, pin_orthonormal_retrieval, pin_self_query,
             pin_decay_closed_form, pin_golden_fixtures, pin_brute_force, pin_chunked_form,
             pin_split_combine, pin_snapshot_tagging, pin_contraction_bound, pin_resume,
             pin_decode_matches_prefill, pin_decode_slots, pin_varlen_isolation,
             pin_backward_finite_differences, pin_backward_across_blocks,
             pin_backward_beta0_closed_form, pin_backward_dq_is_state_times_cotangent,
-            pin_backward_chunked_form]
+            pin_backward_chunked_form, pin_gate_logit_map, pin_gate_logit_decay,
+            pin_gate_logit_backward]

@@ -67,9 +67,25 @@ def _prefill(a, ws=None, ws_bytes=0):
     ({"snapshot_stride": 100}, 1), ({"snapshot_stride": 512}, 1),  # no snapshot buffers
     ({"q": FAKE + 4}, 1), ({"o": None}, 1), ({"in_dtype": 7}, 1),
     ({"o": FAKE + (2 << 24)}, 1),  # o overlaps v
+    ({"g_logits": FAKE + (9 << 24)}, 1),                          # both gate forms
+    ({"g": None}, 1),                                             # no gate at all
+    ({"g": None, "g_logits": FAKE + (9 << 24) + 2}, 1),           # logits misaligned
+    ({"g": None, "g_logits": FAKE + (6 << 24) - 4096}, 1),        # o overlaps the logits
 ])
 def test_prefill_rejects_invalid_args(over, code):
     assert _prefill(_args(**over)) == code
+
+
+def test_gate_logits_are_an_accepted_gate():
+    """With g NULL and bf16 logits given, the arguments are valid (the size query
+    succeeds, as it does for fp32 g)."""
+    lib = _lib.load()
+    a = _args(g=None, g_logits=FAKE + (9 << 24))
+    assert lib.kda_prefill_workspace_size(ctypes.byref(a)) > 0
+    b = _bwd_args(g=None, g_logits=FAKE + (21 << 24))
+    assert lib.kda_prefill_backward_workspace_size(ctypes.byref(b)) > 0
+    assert lib.kda_prefill_backward_workspace_size(
+        ctypes.byref(_bwd_args(g_logits=FAKE + (21 << 24)))) == 0   # both gate forms
 
 
 def test_prefill_rejects_bad_host_seqlens():
@@ -130,6 +146,9 @@ def test_combine_and_local_state_reject_invalid_args():
     a.seg_cu_host = ctypes.addressof(bad)
     assert lib.kda_chunk_local_state(ctypes.byref(a), None, 0, None) == 1
     a.seg_cu_host = None
+    a.g_logits = FAKE + (9 << 24)                          # both gate forms
+    assert lib.kda_chunk_local_state(ctypes.byref(a), None, 0, None) == 1
+    a.g_logits = None
     a.m = a.s_loc
     assert lib.kda_chunk_local_state(ctypes.byref(a), None, 0, None) == 1
 
@@ -177,6 +196,9 @@ def _backward(a, ws=None, ws_bytes=0):
     ({"d_v": FAKE + (2 << 24)}, 1),                # d_v overlaps v
     ({"d_g": FAKE + (7 << 24)}, 1),                # d_g overlaps d_q
     ({"total_tokens": 100}, 1),                    # host offsets end elsewhere
+    ({"g": None}, 1),                              # no gate at all
+    ({"g": None, "g_logits": FAKE + (21 << 24) + 8}, 1),   # logits misaligned
+    ({"g": None, "g_logits": FAKE + (10 << 24)}, 1),       # d_g overlaps the logits
 ])
 def test_backward_rejects_invalid_args(over, code):
     assert _backward(_bwd_args(**over)) == code

@@ -102,3 +102,35 @@ def test_unmutated_source_builds_and_passes(workdir):
     for pin in P.ALL_PINS:
         pin(lib)
 
+
+
+# Mistakes planted in the fused gate activation (Python side of the oracle): each
+# must fail at least one of the gate-logit pins.
+_GATE_PINS = [P.pin_gate_logit_map, P.pin_gate_logit_decay, P.pin_gate_logit_backward]
+
+
+def _sig(x):
+    import numpy as np
+    return 1.0 / (1.0 + np.exp(-oracle._f64(x)))
+
+
+_GATE_MUTANTS = {
+    "flipped_logit": ("gate_from_logits", lambda x: -5.0 * _sig(-oracle._f64(x))),
+    "wrong_scale": ("gate_from_logits", lambda x: -4.0 * _sig(x)),
+    "slope_dropped_factor": ("gate_logit_slope", lambda x: -5.0 * _sig(x)),
+    "slope_sign": ("gate_logit_slope", lambda x: 5.0 * _sig(x) * (1.0 - _sig(x))),
+}
+
+
+@pytest.mark.parametrize("name", sorted(_GATE_MUTANTS))
+def test_gate_mutant_is_caught(name, monkeypatch, oracle_lib):
+    attr, fn = _GATE_MUTANTS[name]
+    monkeypatch.setattr(oracle, attr, fn)
+    caught = False
+    for pin in _GATE_PINS:
+        try:
+            pin(oracle_lib)
+        except AssertionError:
+            caught = True
+            break
+    assert caught, f"gate mutant {name} passed every gate pin"
