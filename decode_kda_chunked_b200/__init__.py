@@ -25,7 +25,7 @@ __all__ = ["kda_prefill_chunked", "kda_chunk_local_state", "kda_state_combine",
            "kda_prefill_uses_tensor_cores", "kda_prefill_backward",
            "kda_prefill_backward_workspace_size",
            "prefill", "prefill_backward", "long_context_prefill", "decode_step",
-           "snapshot_offsets", "load"]
+           "snapshot_offsets", "load", "PrefixCache"]
 
 
 def snapshot_offsets(lengths, stride: int) -> list:
@@ -131,3 +131,6 @@ def decode_step(q, k, v, g, beta, state, slot=None, out_dtype=torch.float32, str
     """One token per request; ``state`` is updated in place.  Returns o [N, H, dv]."""
     o = torch.empty((k.shape[0], k.shape[1], v.shape[2]), dtype=out_dtype, device=k.device)
     return kda_decode_step(q, k, v, g, beta, state, o, slot, stream=stream)
+
+
+from .prefix_cache import PrefixCache  # noqa: E402  (needs prefill above)

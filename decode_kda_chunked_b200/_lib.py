@@ -71,7 +71,10 @@ EXPORTS = ("kda_prefill_workspace_size", "kda_prefill_chunked", "kda_local_state
            "kda_chunk_local_state", "kda_state_combine", "kda_decode_step", "kda_snapshot_count",
            "kda_get_device_status", "kda_status_string", "kda_version",
            "kda_prefill_uses_tensor_cores", "kda_prefill_chunked_noalloc",
-           "kda_prefill_backward_workspace_size", "kda_prefill_backward")
+           "kda_prefill_backward_workspace_size", "kda_prefill_backward",
+           "kda_prefix_cache_create", "kda_prefix_cache_destroy", "kda_prefix_cache_lookup",
+           "kda_prefix_cache_insert", "kda_prefix_cache_size", "kda_state_gather",
+           "kda_state_scatter")
 
 
 def load(path: str = LIB_PATH):
@@ -114,6 +117,20 @@ def load(path: str = LIB_PATH):
         lib.kda_prefill_backward.argtypes = [P(BackwardArgs), _vp, ctypes.c_size_t, _vp]
         lib.kda_prefill_uses_tensor_cores.restype = _i32
         lib.kda_prefill_uses_tensor_cores.argtypes = [_i32, _i32, ctypes.c_int]
+        lib.kda_prefix_cache_create.restype = _vp
+        lib.kda_prefix_cache_create.argtypes = [_i32, _i32]
+        lib.kda_prefix_cache_destroy.restype = None
+        lib.kda_prefix_cache_destroy.argtypes = [_vp]
+        lib.kda_prefix_cache_lookup.restype = _i32
+        lib.kda_prefix_cache_lookup.argtypes = [_vp, _vp, _i32, _i32, P(_i32)]
+        lib.kda_prefix_cache_insert.restype = _i32
+        lib.kda_prefix_cache_insert.argtypes = [_vp, _vp, _i32, _i32, _vp]
+        lib.kda_prefix_cache_size.restype = _i32
+        lib.kda_prefix_cache_size.argtypes = [_vp]
+        lib.kda_state_gather.restype = ctypes.c_int
+        lib.kda_state_gather.argtypes = [_vp, _i32, _vp, _i32, _i32, _i32, _i32, _vp, _vp]
+        lib.kda_state_scatter.restype = ctypes.c_int
+        lib.kda_state_scatter.argtypes = [_vp, _vp, _i32, _i32, _i32, _i32, _vp, _i32, _vp]
         _lib = lib
         return lib
 
@@ -327,3 +344,66 @@ def kda_version() -> int:
 
 def kda_prefill_uses_tensor_cores(dk: int, dv: int, in_dtype: int = KDA_BF16) -> bool:
     return bool(load().kda_prefill_uses_tensor_cores(int(dk), int(dv), int(in_dtype)))
+
+
+# ----------------------------------------------------------------------------
+# prefix cache over state snapshots (host index + device pool copies)
+# ----------------------------------------------------------------------------
+
+def kda_prefix_cache_create(block_tokens: int, n_slots: int) -> int:
+    h = load().kda_prefix_cache_create(int(block_tokens), int(n_slots))
+    if not h:
+        raise ValueError("kda_prefix_cache_create: block_tokens and n_slots must be > 0")
+    return h
+
+
+def kda_prefix_cache_destroy(handle: int) -> None:
+    load().kda_prefix_cache_destroy(handle)
+
+
+def _host_ids(tokens):
+    t = torch.as_tensor(tokens, dtype=torch.int32).contiguous().cpu()
+    return t, (t.data_ptr() if t.numel() else None)
+
+
+def kda_prefix_cache_lookup(handle: int, tokens, max_tokens: int | None = None):
+    """(cached prefix length in tokens, slot or -1) for host token ids."""
+    t, p = _host_ids(tokens)
+    n = t.numel()
+    slot = _i32(-1)
+    m = load().kda_prefix_cache_lookup(handle, p, n, n if max_tokens is None else int(max_tokens),
+                                       ctypes.byref(slot))
+    if m < 0:
+        raise ValueError("kda_prefix_cache_lookup: invalid arguments")
+    return int(m), int(slot.value)
+
+
+def kda_prefix_cache_insert(handle: int, tokens, first_block: int = 0):
+    """(leading blocks cached afterwards, slots to fill per block: list, -1 = none)."""
+    t, p = _host_ids(tokens)
+    n = t.numel()
+    out = torch.full((max(n, 1),), -1, dtype=torch.int32)
+    k = load().kda_prefix_cache_insert(handle, p, n, int(first_block), out.data_ptr())
+    if k < 0:
+        raise ValueError("kda_prefix_cache_insert: invalid arguments")
+    return int(k), out
+
+
+def kda_prefix_cache_size(handle: int) -> int:
+    return int(load().kda_prefix_cache_size(handle))
+
+
+def kda_state_gather(pool, slots, dst, stream=None):
+    """dst[i] = pool[slots[i]] (zeros for slots[i] < 0); slots: CUDA int32."""
+    n_slots, H, dk, dv = pool.shape
+    _check("kda_state_gather", load().kda_state_gather(
+        _ptr(pool), n_slots, _ptr(slots), slots.numel(), H, dk, dv, _ptr(dst), _stream(stream)))
+    return dst
+
+
+def kda_state_scatter(src, slots, pool, stream=None):
+    """pool[slots[i]] = src[i] where slots[i] >= 0; slots: CUDA int32."""
+    n_slots, H, dk, dv = pool.shape
+    _check("kda_state_scatter", load().kda_state_scatter(
+        _ptr(src), _ptr(slots), slots.numel(), H, dk, dv, _ptr(pool), n_slots, _stream(stream)))
+    return pool

@@ -181,3 +181,28 @@ def decode(steps: int, N: int = 256, H: int = 32, d: int = 128, device="cpu", se
     state = state_std * torch.randn((N, H, d, d), generator=gen, device=device,
                                     dtype=torch.float32)
     return DecodeInputs(q, k, v, g, beta, state)
+
+
+# --------------------------------------------------------------------------
+# Prompts as token ids (prefix-cache workloads): the inputs of a token are a
+# fixed row per id, so prompts that share a prefix share its inputs.
+# --------------------------------------------------------------------------
+
+def token_table(vocab: int, H: int, dk: int, dv: int, dtype=torch.bfloat16, seed: int = 0,
+                device="cpu", gate_logits: bool = False) -> PrefillInputs:
+    """Per token id t < vocab, the inputs of one token (row t of every tensor),
+    drawn like any workload; a stand-in for a model's per-token projections."""
+    return make_prefill_inputs([vocab], H, dk, dv, dtype=dtype, seed=seed, device=device,
+                               gate_logits=gate_logits)
+
+
+def prompt_inputs(table: PrefillInputs, prompts) -> PrefillInputs:
+    """Packed inputs of the given prompts (sequences of token ids): rows of ``table``."""
+    lengths = [len(p) for p in prompts]
+    dev = table.k.device
+    ids = torch.tensor([int(t) for p in prompts for t in p], dtype=torch.long, device=dev)
+    pick = lambda x: None if x is None else x[ids].contiguous()
+    cu = torch.tensor([0] + list(_cumsum(lengths)), dtype=torch.int32, device=dev)
+    return PrefillInputs(pick(table.q), pick(table.k), pick(table.v), pick(table.g),
+                         pick(table.beta), cu, lengths, None, dict(table.meta),
+                         pick(table.g_logits))

@@ -360,6 +360,81 @@ kda_status kda_prefill_backward(const kda_backward_args *args, void *workspace,
                                 size_t workspace_bytes, void *stream);
 
 /* ------------------------------------------------------------------------ */
+/* Prefix cache over state snapshots (serving).                             */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Source: the serving cache keeps sparse state snapshots at 512-token block
+ * boundaries, and a request whose prompt starts with a cached prefix resumes
+ * from the longest one ("Kimi K3 开源日来了", Infra section, second layer).
+ * The state after a prefix depends only on the prefix, so the cache maps
+ * prompt prefixes that end on a block boundary to states.
+ *
+ * kda_prefix_cache is a HOST index (no device memory of its own): the chained
+ * 64-bit FNV-1a hash of a prompt's first j blocks of token ids (block j hashed
+ * over the hash of block j-1, 0 before the first, and its ids, little-endian)
+ * maps to a slot of a caller-owned device state pool [n_slots, H, dk, dv]
+ * fp32.  Each entry keeps its parent's hash and its block's ids, and lookups
+ * compare both, so a hash collision cannot return another prompt's state.
+ * When every slot is taken, an insert evicts the least recently used entry;
+ * lookups and inserts refresh the blocks they walk, deepest first, so a
+ * chain's leading blocks are evicted last.  Calls on one cache are serialised
+ * by an internal lock.  A slot returned by a lookup holds its state until a
+ * later insert evicts it: enqueue the copy out of the pool (kda_state_gather)
+ * before the next insert's copies into it, on the same stream.
+ *
+ * Typical resume of one request with prompt ids t[0..n):
+ *   m = kda_prefix_cache_lookup(c, t, n, n - 1, &slot);   (keep >= 1 token)
+ *   kda_state_gather(pool, n_slots, &slot, 1, ...) -> initial state;
+ *   prefill tokens m..n from it with snapshot_stride = block_tokens;
+ *   kda_prefix_cache_insert(c, t, n, m / block_tokens, slots_out), then
+ *   kda_state_scatter of snapshot j - m / block_tokens into slots_out[j].
+ */
+typedef struct kda_prefix_cache kda_prefix_cache;
+
+/* New empty cache of n_slots states, keyed by blocks of block_tokens ids
+ * (512 in the standard workloads).  NULL if an argument is <= 0 or memory runs
+ * out.  Release it with kda_prefix_cache_destroy. */
+kda_prefix_cache *kda_prefix_cache_create(int32_t block_tokens, int32_t n_slots);
+void kda_prefix_cache_destroy(kda_prefix_cache *cache);
+
+/* Longest cached prefix of tokens[0..n_tokens) that ends on a block boundary
+ * and is at most max_tokens long.  Returns its length in tokens (a multiple of
+ * block_tokens, 0 for none) and writes the slot holding the state after it
+ * to *slot (-1 for none); -1 on invalid arguments.  tokens: HOST int32. */
+int32_t kda_prefix_cache_lookup(kda_prefix_cache *cache, const int32_t *tokens,
+                                int32_t n_tokens, int32_t max_tokens, int32_t *slot);
+
+/* Registers the complete blocks of tokens[0..n_tokens) (HOST int32).
+ * slots_out (HOST int32 [n_tokens / block_tokens]) receives, for block j
+ * (0-based), the slot the caller must fill with the state after tokens
+ * [0, (j+1) * block_tokens), or -1 when nothing is to be written (the block
+ * was cached already, or was not registered).  Blocks before first_block must
+ * be cached already (their states are not at hand): the walk stops at the
+ * first one that is not.  The walk also stops when the only slot left to
+ * evict belongs to this prompt.  Returns how many leading blocks are cached
+ * afterwards, or -1 on invalid arguments. */
+int32_t kda_prefix_cache_insert(kda_prefix_cache *cache, const int32_t *tokens,
+                                int32_t n_tokens, int32_t first_block, int32_t *slots_out);
+
+/* Number of cached blocks (-1 for a NULL cache). */
+int32_t kda_prefix_cache_size(const kda_prefix_cache *cache);
+
+/* Device copies between the state pool [n_slots, H, dk, dv] fp32 and dense
+ * states [n, H, dk, dv] fp32.  slots: DEVICE int32 [n].
+ *   gather:  dst[i] = pool[slots[i]], zeros where slots[i] < 0;
+ *   scatter: pool[slots[i]] = src[i] where slots[i] >= 0.
+ * All pointers 16-byte aligned; the pool must not overlap dst / src.  A slot
+ * >= n_slots copies nothing and is reported through the device status word
+ * (KDA_ERR_INVALID_ARG from kda_get_device_status).  Asynchronous on stream. */
+kda_status kda_state_gather(const float *pool, int32_t n_slots, const int32_t *slots,
+                            int32_t n, int32_t H, int32_t dk, int32_t dv, float *dst,
+                            void *stream);
+kda_status kda_state_scatter(const float *src, const int32_t *slots, int32_t n, int32_t H,
+                             int32_t dk, int32_t dv, float *pool, int32_t n_slots,
+                             void *stream);
+
+/* ------------------------------------------------------------------------ */
 /* Helpers.                                                                 */
 /* ------------------------------------------------------------------------ */
 
