@@ -373,6 +373,12 @@ def run_ours(args, world, rank, local):
         line["backward"] = bench_backward(args, inp, dev, peaks, world)
     if not args.no_e2e:
         line["e2e"] = bench_e2e(args, inp, dev, world)
+        xl = I.make_prefill_inputs(inp.lengths, H=32, dk=128, dv=128, seed=rank, device=dev,
+                                   gate_logits=True)
+        line["e2e"]["fused_gate"] = bench_e2e(args, xl, dev, world, gate_logits=True)
+        line["e2e"]["fused_gate"]["workload"] = ("the same requests with bf16 gate logits in "
+                                                 "place of fp32 g (fused gate activation)")
+        del xl
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         r = time_oracle(inp, sample_chains(inp.lengths, H))
         line["cpu_baseline"] = {"value": r["token_heads"] / H / r["seconds"], "unit": "tokens/s",
@@ -625,18 +631,20 @@ def bench_kcp_million(args, dev, peaks, world, rank):
     return out
 
 
-def bench_e2e(args, inp, dev, world):
+def bench_e2e(args, inp, dev, world, gate_logits: bool = False):
     """Same metric through the public entry point with host buffers: every step
     copies that step's inputs from pinned host memory and reads o and the final
     states back to pinned host memory inside the timed region.  Steps are double
     buffered on three streams, as a serving loop runs them: step k's inputs are
     copied in and step k-1's outputs copied out while step k-1 / k computes, so the
-    time per step is set by the busier PCIe direction, not by the sum."""
+    time per step is set by the busier PCIe direction, not by the sum.  With
+    ``gate_logits`` the gate travels as bf16 logits (fused gate activation)."""
     import torch
 
     import decode_kda_chunked_b200 as kda
     T, H, dv, dk = inp.total_tokens, 32, 128, 128
-    names = ("q", "k", "v", "g", "beta", "cu_seqlens")
+    gname = "g_logits" if gate_logits else "g"
+    names = ("q", "k", "v", gname, "beta", "cu_seqlens")
     host = {n: getattr(inp, n).cpu().pin_memory() for n in names}
     devb = [{n: torch.empty_like(getattr(inp, n)) for n in names} for _ in range(2)]
     o = [torch.empty(T, H, dv, device=dev) for _ in range(2)]
@@ -647,7 +655,7 @@ def bench_e2e(args, inp, dev, world):
     s_in, s_cmp, s_out = (torch.cuda.Stream(dev) for _ in range(3))
     # the prefill's workspace is allocated once per buffer (not per call on another stream)
     a = kda.make_prefill_args(inp.q, inp.k, inp.v, inp.g, inp.beta, inp.cu_seqlens, o[0], None,
-                              fin[0], 0, None, None, cu_host)
+                              fin[0], 0, None, None, cu_host, g_logits=inp.g_logits)
     ws_bytes = max(kda.kda_prefill_workspace_size(a), 256)
     ws = [torch.empty(ws_bytes, dtype=torch.uint8, device=dev) for _ in range(2)]
     ev = {k: [torch.cuda.Event() for _ in range(2)] for k in ("in", "cmp", "out")}
@@ -664,10 +672,12 @@ def bench_e2e(args, inp, dev, world):
             ev["in"][b].record(s_in)
         s_cmp.wait_event(ev["in"][b])
         s_cmp.wait_event(ev["out"][b])             # step k-2's outputs have been read out
-        kda.kda_prefill_chunked(devb[b]["q"], devb[b]["k"], devb[b]["v"], devb[b]["g"],
+        kda.kda_prefill_chunked(devb[b]["q"], devb[b]["k"], devb[b]["v"],
+                                None if gate_logits else devb[b]["g"],
                                 devb[b]["beta"], devb[b]["cu_seqlens"], o[b], None, fin[b], 0,
                                 None, None, cu_seqlens_host=cu_host, workspace=ws[b],
-                                stream=s_cmp)
+                                stream=s_cmp,
+                                g_logits=devb[b]["g_logits"] if gate_logits else None)
         ev["cmp"][b].record(s_cmp)
         with torch.cuda.stream(s_out):
             s_out.wait_event(ev["cmp"][b])

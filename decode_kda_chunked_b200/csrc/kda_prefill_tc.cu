@@ -8,7 +8,7 @@
 // one TMEM lane per feature channel (S^T, U^T, O^T have lanes = value
 // channels, columns = key channels or tokens):
 //
-//   A | P   [128 x 16] per 16-column block b:  [L_b ; Lq_b] R_b^T           (A from TMEM)
+//   A | P   [128 x 32(b+1)] per 32-row block b: [L ; Lq] R'_b^T             (A from TMEM)
 //   Y^T     = V^T - S^T (gamma*K)^T                                          (A = S^T in TMEM)
 //   U^T     = Y^T (T Diag(b))^T                                              (A = Y^T in TMEM)
 //   O^T     = S^T (gamma*Q)^T + U^T P^T                                      (A = S^T, U^T in TMEM)
@@ -16,15 +16,17 @@
 // U = T Diag(b) (V - (gamma*K) S) is the chunk form's U~ - W S with W never formed:
 // Y needs only the state and the chunk's inputs, so it runs while the workers solve T.
 //
-// Gate factorisation for A and P: for the 16-token column block b with last
-// row r_b, exp(G_i - G_j) = exp(G_i - G_rb) * exp(G_rb - G_j).  The right
-// factor is <= 1 for j <= r_b; the left factor is <= exp(5 * 15) for rows i
-// of block b and <= 1 below it, and rows above block b (masked anyway) are
-// set to zero.  Because log alpha >= -5 (the lower-bounded decay of KDA, CSDN
-// post on the Kimi K3 technical report, section 一.1) every factor is a
-// finite fp32 number.  Row i's left factors for earlier blocks follow from
-// its own block's factor times the per-channel block-to-block decays
-// exp(G_ra - G_rb), so each row needs one exponential per channel.
+// Gate factorisation for A and P: rows come in two 32-row blocks b with reference
+// rows m_b = 32 b + 15, and exp(G_i - G_j) = exp(G_i - G_mb) * exp(G_mb - G_j) for a
+// row i of block b and a column j <= i.  The left factor is <= exp(5 * 15) (rows
+// i < m_b) or <= 1; the right factor is <= exp(5 * 16) (columns j > m_b) or <= 1.
+// Because log alpha >= -5 (the lower-bounded decay of KDA, CSDN post on the Kimi K3
+// technical report, section 一.1) every factor is a finite fp32 number, and only
+// masked products (j > i) can overflow; they are dropped by selection, never
+// multiplied.  Column j's right factor for block b follows from its own block's
+// factor times the block-to-block decay exp(G_mb - G_m(j)) <= 1, so each row
+// needs one exponential per channel.  Each block's product runs as two 8-step
+// accumulation chains over the halves of the key channels, summed on read-out.
 //
 // All tensor-core operands are tf32 (B operands K-major with the 128-byte
 // swizzle in shared memory): bf16 operands for the gate-scaled products would
@@ -63,9 +65,9 @@ constexpr uint32_t OFF_GRAW = 49152;    // fp32 [64 x 128]: 4 TMA boxes of 32 co
                                         // cols, as q/k/v); rewritten in place with
                                         // log2(e) * cumsum(g)
 constexpr uint32_t RAW_BYTES = 81920;
-// Once every raw tile is read, the raw region holds the B operands R'_a of
-// the A|P products: row block a has 16(a+1) rows at byte 8192 a(a+1)/2.
-__host__ __device__ constexpr uint32_t rp_off(int a) { return 4096u * a * (a + 1); }
+// Once every raw tile is read, the raw region holds the B operands R'_b of
+// the A|P products: row block b (32 rows) has 32(b+1) rows at byte 16384 b.
+__host__ __device__ constexpr uint32_t rp_off(int b) { return 16384u * b; }
 constexpr uint32_t OFF_R = 81920;       // R scratch [64 x 132] fp32, then T-solve scratch
 constexpr int LDT = 65;                 // padded row stride of the T-solve scratch
 constexpr int LDR = 132;                // padded row stride of the fp32 R scratch [64][132]
@@ -76,12 +78,10 @@ constexpr uint32_t OFF_GQ = 115712;     // (gamma*Q) [64 x 128] tf32 B operand; 
 constexpr uint32_t OFF_KHT = 148480;    // Khat^T [128 x 64] tf32 B operand
 constexpr uint32_t OFF_TB = 181248;     // T Diag(beta) [64 x 64] tf32 B operand
 constexpr uint32_t OFF_P = 197632;      // P [64 x 64] tf32 B operand
-constexpr uint32_t OFF_E = 214016;      // E[b*4+a][128] = exp(G_ra - G_rb), b <= a; then
-                                        // the T-solve products ([2][16][17], then [32][33])
-constexpr uint32_t OFF_Y = OFF_E;
-constexpr uint32_t OFF_EGR = 222208;    // exp(G_rb)[4][128]
+constexpr uint32_t OFF_Y = 214016;      // the T-solve products ([2][16][17], then [32][33])
+constexpr uint32_t OFF_EGR = 222208;    // exp(G_rb)[4][128], r_b = 16 b + 15
 constexpr uint32_t OFF_SEG = 224256;    // cumsum segment totals [4][128]
-constexpr uint32_t OFF_GR2 = 226304;    // log2(e) * G at block ends [4][128]
+constexpr uint32_t OFF_GR2 = 226304;    // log2(e) * G at rows 16 b + 15 [4][128]
 constexpr uint32_t OFF_BETA = 228352;   // beta[64]
 constexpr uint32_t OFF_BAR = 228608;    // mbarriers + TMEM base + flags
 constexpr uint32_t SMEM_BYTES = 228704;
@@ -92,11 +92,14 @@ constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;  // alignment slack
 // ---- TMEM column map (512 columns x 128 lanes of fp32) ----
 constexpr uint32_t TM_S = 0;     // S^T (lane = value channel, col = key channel)
 constexpr uint32_t TM_L = 128;   // L* (A operand of A|P); later V^T -> Y^T in [0,64)
-// A (lanes 0..63) | P (lanes 64..127) of rows in block a: 16(a+1) columns at TM_AP + 8a(a+1)
-constexpr uint32_t TM_AP = 256;  // up to column 416
-__host__ __device__ constexpr uint32_t ap_col(int a) { return TM_AP + 8u * a * (a + 1); }
+// A (lanes 0..63) | P (lanes 64..127) of the rows of 32-row block b: 32(b+1) columns,
+// summed over two halves of the key channels held apart (two accumulators each)
+constexpr uint32_t TM_AP = 256;  // up to column 448
+__host__ __device__ constexpr uint32_t ap_col(int b, int half) {
+  return TM_AP + (b == 0 ? 32u * half : 64u + 64u * half);
+}
 constexpr uint32_t TM_X2 = 320;  // U^T (alias A|P once the solve has read it)
-constexpr uint32_t TM_O = 416;   // O^T (own columns: issued right after the A|P products)
+constexpr uint32_t TM_O = 448;   // O^T (own columns: issued right after the A|P products)
 constexpr uint32_t TM_COLS = 512;
 
 struct TcMaps {
@@ -140,7 +143,6 @@ __global__ void __launch_bounds__(NT + 32, 1)
   extern __shared__ unsigned char smem_raw[];
   unsigned char *sm = reinterpret_cast<unsigned char *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float *sE = reinterpret_cast<float *>(sm + OFF_E);
   float *sEgr = reinterpret_cast<float *>(sm + OFF_EGR);
   float *sSeg = reinterpret_cast<float *>(sm + OFF_SEG);
   float *sGr2 = reinterpret_cast<float *>(sm + OFF_GR2);
@@ -255,18 +257,24 @@ __global__ void __launch_bounds__(NT + 32, 1)
           for (int s = 0; s < DH / 8; ++s)
             mma_tf32_ts(tm + TM_O, tm + TM_S + 8 * s, sw128_desc(qb, C, s), id, s > 0);
         }
-        // A | P: row block a against its R'_a (N = 16(a+1)); four interleaved chains
+        // A | P: row block b against its R'_b (N = 32(b+1)), each over the two halves of
+        // the key channels into its own accumulator: four interleaved chains of 8 steps
         if (!cwait(bar_opsap, ph_opsap[0])) break;
         {
           const uint32_t rp = smem_u32(sm);
 #pragma unroll
-          for (int s = 0; s < DH / 8; ++s) {
+          for (int s = 0; s < DH / 16; ++s) {
 #pragma unroll
-            for (int a = 0; a < 4; ++a)
-              mma_tf32_ts(tm + ap_col(a), tm + TM_L + 8 * s, sw128_desc(rp + rp_off(a), 16 * (a + 1), s),
-                          idesc_tf32(16 * (a + 1)), s > 0);
+            for (int half = 0; half < 2; ++half)
+#pragma unroll
+              for (int b = 0; b < 2; ++b) {
+                const int ks = (DH / 16) * half + s;
+                mma_tf32_ts(tm + ap_col(b, half), tm + TM_L + 8 * ks,
+                            sw128_desc(rp + rp_off(b), 32 * (b + 1), ks), idesc_tf32(32 * (b + 1)),
+                            s > 0);
+              }
           }
-          mma_commit(bar_ap);  // gamma*Q and the R'_a operands are free after this
+          mma_commit(bar_ap);  // gamma*Q and the R'_b operands are free after this
         }
         // raw tiles consumed, V^T in TMEM, gamma*K in shared memory
         if (!cwait(bar_raw, ph_raw)) break;
@@ -392,19 +400,17 @@ __global__ void __launch_bounds__(NT + 32, 1)
           *reinterpret_cast<float *>(sm + OFF_GRAW + g_off(16 * g + j, l)) = gv[j];
         }
         sGr2[g * DH + l] = gv[15];
-        wsync();
         sEgr[g * DH + l] = ex2(gv[15]);
-        for (int b = 0; b <= g; ++b) sE[(b * 4 + g) * DH + l] = ex2(gv[15] - sGr2[b * DH + l]);
         wsync();
       }
 
       // ---- a3 operands (thread = row i, channels 32g..32g+31) -----------------
-      // L*_i = x_i exp(G_i - G_rb) with r_b the last row of i's own block (x = k or q)
-      // goes to TMEM; K side: R_i = k_i exp(G_rb - G_i) to fp32 scratch (for R'_a);
-      // Q side: gamma*Q = L* exp(G_rb) to its B operand.
+      // L*_i = x_i exp(G_i - G_m) with m = 32 b + 15 the reference row of i's 32-row block
+      // (x = k or q) goes to TMEM; K side: k_i to fp32 scratch (for R'_b); Q side:
+      // gamma*Q = L* exp(G_m) to its B operand.
       const bool kside = l < C;
       const int i = l & (C - 1);
-      const int bi = i >> 4;
+      const int bi = 2 * (i >> 5);  // the 16-row group ending at the reference row of i's block
       const bool valid = i < n && (kside || load_q);
       float *Rs = reinterpret_cast<float *>(sm + OFF_R);  // [64][LDR] fp32 scratch
       {
@@ -428,11 +434,8 @@ __global__ void __launch_bounds__(NT + 32, 1)
               lst[e] = x[e] * ex2(giv[e] - grv[e]);
               Lv[4 * c4 + e] = tf32_rna(lst[e]);
             }
-            if (kside) {
-              float rv[4];
-#pragma unroll
-              for (int e = 0; e < 4; ++e) rv[e] = x[e] * ex2(grv[e] - giv[e]);
-              *reinterpret_cast<float4 *>(&Rs[i * LDR + c]) = make_float4(rv[0], rv[1], rv[2], rv[3]);
+            if (kside) {  // k itself: R'_b takes its block factor in one exponential
+              *reinterpret_cast<float4 *>(&Rs[i * LDR + c]) = make_float4(x[0], x[1], x[2], x[3]);
             } else {
               const float4 eg = *reinterpret_cast<const float4 *>(&sEgr[bi * DH + c]);
               *reinterpret_cast<float4 *>(sm + OFF_GQ + sw128_chunk(C, i, c)) =
@@ -478,17 +481,21 @@ __global__ void __launch_bounds__(NT + 32, 1)
               make_float4(kh[4 * m4], kh[4 * m4 + 1], kh[4 * m4 + 2], kh[4 * m4 + 3]);
       }
       wsync();  // every raw tile read: the raw region now takes the R'_a operands
-      // R'_a row j = R_j exp(G_ra - G_rb(j)) for j <= r_a, spread over all workers
+      // R'_b row j = k_j exp(G_mb - G_j) for the rows j of blocks up to b, m_b = 32 b + 15
+      // (the 16-row group end 2b of the G table), spread over all workers.  One exponential
+      // of the exponent difference: a factor underflows only where the true factor is
+      // below FLT_MIN, and then its product with an L* factor (<= exp(75)) is < exp(-12).
 #pragma unroll
-      for (int a = 0; a < 4; ++a) {
-        const int rows = 16 * (a + 1);
+      for (int b = 0; b < 2; ++b) {
+        const int rows = 32 * (b + 1);
         for (int it = tid; it < rows * 32; it += NT) {
           const int j = it >> 5, c = (it & 31) * 4;
-          const float4 rv = *reinterpret_cast<const float4 *>(&Rs[j * LDR + c]);
-          const float4 ea = *reinterpret_cast<const float4 *>(&sE[((j >> 4) * 4 + a) * DH + c]);
-          *reinterpret_cast<float4 *>(sm + rp_off(a) + sw128_chunk(rows, j, c)) =
-              make_float4(tf32_rna(rv.x * ea.x), tf32_rna(rv.y * ea.y), tf32_rna(rv.z * ea.z),
-                          tf32_rna(rv.w * ea.w));
+          const float4 kv = *reinterpret_cast<const float4 *>(&Rs[j * LDR + c]);
+          const float4 gj = *reinterpret_cast<const float4 *>(sm + OFF_GRAW + g_off(j, c));
+          const float4 gm = *reinterpret_cast<const float4 *>(&sGr2[(2 * b) * DH + c]);
+          *reinterpret_cast<float4 *>(sm + rp_off(b) + sw128_chunk(rows, j, c)) =
+              make_float4(tf32_rna(kv.x * ex2(gm.x - gj.x)), tf32_rna(kv.y * ex2(gm.y - gj.y)),
+                          tf32_rna(kv.z * ex2(gm.z - gj.z)), tf32_rna(kv.w * ex2(gm.w - gj.w)));
         }
       }
       tmem_wait_st();
@@ -513,15 +520,15 @@ __global__ void __launch_bounds__(NT + 32, 1)
       float *Ti = reinterpret_cast<float *>(sm + OFF_TI);
       float *Ys = reinterpret_cast<float *>(sm + OFF_Y);
       {
-        // this warp's 32 rows span two row blocks; load both blocks' columns
-        const int a_lo = 2 * (warp & 1);
+        // this warp's 32 rows are one row block: the sum of its two accumulators (columns
+        // past the block's width belong to other accumulators and are masked below)
+        const int blk = warp & 1;
         float a[16], a_hi[16];
-        tmem_ld16(tm + lane + ap_col(a_lo) + 16 * g, a);
-        tmem_ld16(tm + lane + ap_col(a_lo + 1) + 16 * g, a_hi);
+        tmem_ld16(tm + lane + ap_col(blk, 0) + 16 * g, a);
+        tmem_ld16(tm + lane + ap_col(blk, 1) + 16 * g, a_hi);
         tmem_wait_ld();
-        if (lane_id >= 16)
 #pragma unroll
-          for (int j = 0; j < 16; ++j) a[j] = a_hi[j];
+        for (int j = 0; j < 16; ++j) a[j] += a_hi[j];
         if (kside) {
           const float bi_ = sB[i];
 #pragma unroll
