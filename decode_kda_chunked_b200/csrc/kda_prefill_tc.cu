@@ -356,6 +356,10 @@ __global__ void __launch_bounds__(NT + 32, 1)
       return b;
     };
     float beta_next = load_beta(0);
+    // T Diag(beta) is lower triangular: its blocks above the diagonal stay zero, so they
+    // are written once here; the solve below stores every other element as it finalises it
+    for (int e = tid; e < C * C / 4; e += NT)
+      reinterpret_cast<float4 *>(sm + OFF_TB)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
     // Stage a chunk: its beta, wait for its tiles, cumulative gate, row operands
     // (L* into TMEM, R into scratch, gamma*Q).  Chunk n+1 is staged while chunk n's
     // last MMAs run.
@@ -519,6 +523,10 @@ __global__ void __launch_bounds__(NT + 32, 1)
       float *Ms = reinterpret_cast<float *>(sm + OFF_MS);
       float *Ti = reinterpret_cast<float *>(sm + OFF_TI);
       float *Ys = reinterpret_cast<float *>(sm + OFF_Y);
+      // element (r, c) of T Diag(beta), the B operand of U^T, once T_rc is final
+      auto put_tb = [&](int r, int c, float t) {
+        *reinterpret_cast<float *>(sm + OFF_TB + sw128_offset(C, r, c)) = tf32_rna(t * sB[c]);
+      };
       {
         // this warp's 32 rows are one row block: the sum of its two accumulators (columns
         // past the block's width belong to other accumulators and are masked below)
@@ -563,6 +571,7 @@ __global__ void __launch_bounds__(NT + 32, 1)
           if (q >= jj && k > q) x -= m[q] * xq;
         }
         Ti[rot(o + k, o + jj)] = (k >= jj) ? x : 0.f;
+        put_tb(o + k, o + jj, (k >= jj) ? x : 0.f);
       }
       wsync();
       // 16 -> 32: T_ab = -T_aa (N_ab T_bb) for (a, b) = (1, 0) and (3, 2); T lower triangular
@@ -580,6 +589,7 @@ __global__ void __launch_bounds__(NT + 32, 1)
         for (int q = 0; q < 16; ++q)
           if (q <= k) t += Ti[rot(16 * a + k, 16 * a + q)] * Ys[(blk * 16 + q) * 17 + j];
         Ti[rot(16 * a + k, 16 * b + j)] = -t;
+        put_tb(16 * a + k, 16 * b + j, -t);
         wsync();
       }
       // 32 -> 64: T[32:64, 0:32] = -T[32:64, 32:64] (N[32:64, 0:32] T[0:32, 0:32]);
@@ -612,21 +622,8 @@ __global__ void __launch_bounds__(NT + 32, 1)
             t1b += tv * Ys[(q + 16) * 33 + j0 + 16];
           }
         }
-        Ti[rot(32 + ii, j0)] = -(t0a + t0b);
-        Ti[rot(32 + ii, j0 + 16)] = -(t1a + t1b);
-        wsync();
-      }
-      if (kside) {  // TB = T Diag(beta): row i, columns 16g..16g+15
-#pragma unroll
-        for (int j = 0; j < 16; j += 4) {
-          const int c = 16 * g + j;
-          float v4[4];
-#pragma unroll
-          for (int e = 0; e < 4; ++e)
-            v4[e] = (c + e <= i) ? tf32_rna(Ti[rot(i, c + e)] * sB[c + e]) : 0.f;
-          *reinterpret_cast<float4 *>(sm + OFF_TB + sw128_chunk(C, i, c)) =
-              make_float4(v4[0], v4[1], v4[2], v4[3]);
-        }
+        put_tb(32 + ii, j0, -(t0a + t0b));
+        put_tb(32 + ii, j0 + 16, -(t1a + t1b));
       }
       // ---- S^T <- S^T Diag(gamma_63) once the O^T and Y^T products have read S^T ----
       if (!(ok = wwait(bar_y, ph_y))) break;
