@@ -556,42 +556,38 @@ __global__ void __launch_bounds__(NT + 32, 1)
         }
       }
       wsync();
-      // diagonal 16x16 blocks: forward substitution, one column per 16 lanes, shuffles
+      // diagonal 32x32 blocks: forward substitution, x_k = [k == j] - sum_{q<k} N_kq x_q for
+      // column j.  Warp w takes block w / 8 and its columns w % 8 + 8 c (c < 4) as four
+      // chains over the same rows, so the one value N_kq of a step (lane k) feeds all four
+      // and the chains' shuffles overlap; the next step's N_kq is loaded a step ahead.
+      {
+        const int o = 32 * (warp >> 3), k = lane_id;
+        int jj[4];
+        float x[4];
 #pragma unroll
-      for (int rho = 0; rho < 2; ++rho) {
-        const int task = 4 * warp + 2 * rho + (lane_id >> 4);
-        const int o = 16 * (task >> 4), jj = task & 15, k = lane_id & 15;
-        float m[16];
-#pragma unroll
-        for (int q = 0; q < 16; ++q) m[q] = Ms[rot(o + k, o + q)];
-        float x = (k == jj) ? 1.f : 0.f;
-#pragma unroll
-        for (int q = 0; q < 15; ++q) {
-          const float xq = __shfl_sync(0xffffffffu, x, (lane_id & 16) | q);
-          if (q >= jj && k > q) x -= m[q] * xq;
+        for (int c = 0; c < 4; ++c) {
+          jj[c] = (warp & 7) + 8 * c;
+          x[c] = (k == jj[c]) ? 1.f : 0.f;
         }
-        Ti[rot(o + k, o + jj)] = (k >= jj) ? x : 0.f;
-        put_tb(o + k, o + jj, (k >= jj) ? x : 0.f);
+        float m_next = Ms[rot(o + k, o)];
+#pragma unroll
+        for (int q = 0; q < 31; ++q) {
+          const float m = m_next;
+          if (q < 30) m_next = Ms[rot(o + k, o + q + 1)];
+#pragma unroll
+          for (int c = 0; c < 4; ++c) {
+            const float xq = __shfl_sync(0xffffffffu, x[c], q);
+            if (q >= jj[c] && k > q) x[c] -= m * xq;
+          }
+        }
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const float t = (k >= jj[c]) ? x[c] : 0.f;
+          Ti[rot(o + k, o + jj[c])] = t;
+          put_tb(o + k, o + jj[c], t);
+        }
       }
       wsync();
-      // 16 -> 32: T_ab = -T_aa (N_ab T_bb) for (a, b) = (1, 0) and (3, 2); T lower triangular
-      {
-        const int blk = tid >> 8, k = (tid >> 4) & 15, j = tid & 15;
-        const int a = 2 * blk + 1, b = 2 * blk;
-        float acc = 0.f;
-#pragma unroll
-        for (int q = 0; q < 16; ++q)
-          if (q >= j) acc += Ms[rot(16 * a + k, 16 * b + q)] * Ti[rot(16 * b + q, 16 * b + j)];
-        Ys[(blk * 16 + k) * 17 + j] = acc;
-        wsync();
-        float t = 0.f;
-#pragma unroll
-        for (int q = 0; q < 16; ++q)
-          if (q <= k) t += Ti[rot(16 * a + k, 16 * a + q)] * Ys[(blk * 16 + q) * 17 + j];
-        Ti[rot(16 * a + k, 16 * b + j)] = -t;
-        put_tb(16 * a + k, 16 * b + j, -t);
-        wsync();
-      }
       // 32 -> 64: T[32:64, 0:32] = -T[32:64, 32:64] (N[32:64, 0:32] T[0:32, 0:32]);
       // two outputs per thread, each summed in two halves to shorten the FMA chains
       {
