@@ -275,8 +275,8 @@ struct PrepLayout {
   static constexpr int oP = oA + C * C, oT = oP + C * C, oBuf = oT + C * C;
   static constexpr int oKL = oBuf + C * LDP, oQL = oKL + 16 * LDP, oStage = oQL + 16 * LDP;
   static constexpr int oB = oStage + stage_floats(D, D);
-  static constexpr int oMisc = oB + C;  // mbarrier (8 bytes) and the TMEM base address
-  static constexpr int total = oMisc + 4;
+  static constexpr int oMisc = oB + C;  // two mbarriers (8 bytes each) and the TMEM base address
+  static constexpr int total = oMisc + 6;
   // + alignment slack: the tensor-core operand tiles need a 1024-byte aligned base
   static constexpr size_t bytes = sizeof(float) * total + 1024;
 };
@@ -309,8 +309,8 @@ __global__ void __launch_bounds__(NTH, 1) bwd_prep_kernel(const BwdParams p) {
   const int4 cd = p.chunks[jc];
   const int tok0 = cd.z, n = cd.w;
   const size_t ch = (size_t)jc * H + h;
-  uint64_t *bar = reinterpret_cast<uint64_t *>(sm + L::oMisc);
-  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + L::oMisc + 2);
+  uint64_t *bar = reinterpret_cast<uint64_t *>(sm + L::oMisc);  // [0]: products, [1]: A|P
+  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + L::oMisc + 4);
   if constexpr (kPrepTensorCores<D, TIn>) {
     if ((tid >> 5) == 0) {
       tmem_alloc(s_tmem, 512);
@@ -318,53 +318,140 @@ __global__ void __launch_bounds__(NTH, 1) bwd_prep_kernel(const BwdParams p) {
     }
     if (tid == 0) {
       mbar_init(bar, 1);
+      mbar_init(bar + 1, 1);
       asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
     }
   }
+  bool ap_done = true;
 
   stage_rows<D, TIn>(sK, D, static_cast<const TIn *>(p.k), tok0, n, H, h);
   stage_rows<D, TIn>(sQ, D, static_cast<const TIn *>(p.q), tok0, n, H, h);
   stage_gate<D>(sG, sB, p, tok0, n, h);
 
-  // A (strict lower) and P (inclusive lower), row block b at a time:
-  // A_ts = sum_c [k_tc exp(G_tc - G_rc)] [k_sc exp(G_rc - G_sc)], r = 16 b.
-  // Unrolled over b, so the thread's valid column groups (jj <= b) are fixed.
-#pragma unroll
-  for (int b = 0; b < 4; ++b) {
-    const int r0 = 16 * b, rows = r0 + 16;
+  if constexpr (kPrepTensorCores<D, TIn>) {
+    // A and P on the tensor cores, as in the forward: two 32-row blocks b with reference
+    // rows m_b = 32 b + 15; L*_i = x_i exp(G_i - G_mb) (<= e^75) in TMEM, lanes 0..63 the
+    // k rows and 64..127 the q rows; R'_b row j = k_j exp(G_mb - G_j) (<= e^80, rows
+    // j < 32 (b + 1)) as B operands in the scratch region; each block's product runs as two
+    // 8-step chains over the key-channel halves, summed on read-out.  Masked entries
+    // (s > t) may overflow and are dropped by selection.
+    constexpr uint32_t TL = 0, TAP = 128;
+    auto apc = [](int b, int hh) { return TAP + (b == 0 ? 32u * hh : 64u + 64u * hh); };
+    tc_fence_before();
     __syncthreads();
-    for (int e = tid; e < rows * D; e += NTH) {
-      const int s = e / D, c = e % D;
-      sBuf[s * LDP + c] = sK[s * D + c] * exp2f(sG[r0 * D + c] - sG[s * D + c]);
-    }
-    for (int e = tid; e < 16 * D; e += NTH) {
-      const int t = e / D, c = e % D;
-      const float f = exp2f(sG[(r0 + t) * D + c] - sG[r0 * D + c]);
-      sKL[t * LDP + c] = sK[(r0 + t) * D + c] * f;
-      sQL[t * LDP + c] = sQ[(r0 + t) * D + c] * f;
-    }
-    __syncthreads();
-    float a[4] = {0.f, 0.f, 0.f, 0.f}, pp[4] = {0.f, 0.f, 0.f, 0.f};
-#pragma unroll 8
-    for (int c = 0; c < D; ++c) {
-      const float kl = sKL[ty * LDP + c], ql = sQL[ty * LDP + c];
+    tc_fence_after();
+    const uint32_t tm = *s_tmem;
+    const int w = tid >> 5, ln = tid & 31;
+    const uint32_t lane = (uint32_t)(32 * (w & 3)) << 16;
+    const int lr = 32 * (w & 3) + ln, i = lr & 63, m = 32 * (i >> 5) + 15;
+    unsigned char *rp = reinterpret_cast<unsigned char *>(sBuf);  // 1024-byte aligned
+    {
+      const float *x = lr < C ? sK : sQ;
 #pragma unroll
-      for (int jj = 0; jj <= b; ++jj) {
-        const float tv = sBuf[(tx + 16 * jj) * LDP + c];
-        a[jj] = fmaf(kl, tv, a[jj]);
-        pp[jj] = fmaf(ql, tv, pp[jj]);
+      for (int hh = 0; hh < 2; ++hh) {  // warp w % 4 ... w / 4 takes channels 64 (w / 4) + 32 hh..
+        const int c0 = 64 * (w >> 2) + 32 * hh;
+        float v[32];
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) {
+          const int c = c0 + jj;
+          v[jj] = tf32_round(x[i * D + c] * exp2f(sG[i * D + c] - sG[m * D + c]));
+        }
+        tmem_st32(tm + lane + TL + c0, v);
       }
     }
-    const int t = r0 + ty;
 #pragma unroll
-    for (int jj = 0; jj < 4; ++jj) {
-      const int s = tx + 16 * jj;
-      sA[t * C + s] = s < t ? a[jj] : 0.f;
-      sP[t * C + s] = s <= t ? pp[jj] : 0.f;
+    for (int b = 0; b < 2; ++b) {
+      const int rows = 32 * (b + 1), mb = 32 * b + 15;
+      for (int e = tid; e < rows * (D / 4); e += NTH) {
+        const int j = e / (D / 4), c = (e % (D / 4)) * 4;
+        float4 r;
+        r.x = tf32_round(sK[j * D + c] * exp2f(sG[mb * D + c] - sG[j * D + c]));
+        r.y = tf32_round(sK[j * D + c + 1] * exp2f(sG[mb * D + c + 1] - sG[j * D + c + 1]));
+        r.z = tf32_round(sK[j * D + c + 2] * exp2f(sG[mb * D + c + 2] - sG[j * D + c + 2]));
+        r.w = tf32_round(sK[j * D + c + 3] * exp2f(sG[mb * D + c + 3] - sG[j * D + c + 3]));
+        *reinterpret_cast<float4 *>(rp + 16384 * b + sw128_chunk(rows, j, c)) = r;
+      }
     }
+    tmem_wait_st();
+    fence_async_smem();
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+    if (tid == 0) {
+      const uint32_t rb = smem_u32(rp);
+#pragma unroll
+      for (int st = 0; st < D / 16; ++st)
+#pragma unroll
+        for (int hh = 0; hh < 2; ++hh)
+#pragma unroll
+          for (int b = 0; b < 2; ++b) {
+            const int ks = (D / 16) * hh + st;
+            mma_tf32_ts(tm + apc(b, hh), tm + TL + 8 * ks,
+                        sw128_desc(rb + 16384 * b, 32 * (b + 1), ks), idesc_tf32(32 * (b + 1)),
+                        st > 0);
+          }
+      mma_commit(bar + 1);
+    }
+    ap_done = mbar_wait(bar + 1, 0);
+    if (!ap_done && tid == 0) set_status(p.status, STATUS_TIMEOUT);
+    tc_fence_after();
+    {  // row i (lane lr), columns 32 (w / 4) .. + 31: A for k rows, P for q rows
+      const int b = i >> 5, cb = 32 * (w >> 2);
+      float a0[32], a1[32];
+      tmem_ld32(tm + lane + apc(b, 0) + cb, a0);
+      tmem_ld32(tm + lane + apc(b, 1) + cb, a1);
+      tmem_wait_ld();
+      if (lr < C) {
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) sA[i * C + cb + jj] = (cb + jj < i) ? a0[jj] + a1[jj] : 0.f;
+      } else {
+#pragma unroll
+        for (int jj = 0; jj < 32; ++jj) sP[i * C + cb + jj] = (cb + jj <= i) ? a0[jj] + a1[jj] : 0.f;
+      }
+    }
+    tc_fence_before();
+    __syncthreads();
+    tc_fence_after();
+  } else {
+    // A (strict lower) and P (inclusive lower), row block b at a time:
+    // A_ts = sum_c [k_tc exp(G_tc - G_rc)] [k_sc exp(G_rc - G_sc)], r = 16 b.
+    // Unrolled over b, so the thread's valid column groups (jj <= b) are fixed.
+#pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const int r0 = 16 * b, rows = r0 + 16;
+      __syncthreads();
+      for (int e = tid; e < rows * D; e += NTH) {
+        const int s = e / D, c = e % D;
+        sBuf[s * LDP + c] = sK[s * D + c] * exp2f(sG[r0 * D + c] - sG[s * D + c]);
+      }
+      for (int e = tid; e < 16 * D; e += NTH) {
+        const int t = e / D, c = e % D;
+        const float f = exp2f(sG[(r0 + t) * D + c] - sG[r0 * D + c]);
+        sKL[t * LDP + c] = sK[(r0 + t) * D + c] * f;
+        sQL[t * LDP + c] = sQ[(r0 + t) * D + c] * f;
+      }
+      __syncthreads();
+      float a[4] = {0.f, 0.f, 0.f, 0.f}, pp[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+      for (int c = 0; c < D; ++c) {
+        const float kl = sKL[ty * LDP + c], ql = sQL[ty * LDP + c];
+#pragma unroll
+        for (int jj = 0; jj <= b; ++jj) {
+          const float tv = sBuf[(tx + 16 * jj) * LDP + c];
+          a[jj] = fmaf(kl, tv, a[jj]);
+          pp[jj] = fmaf(ql, tv, pp[jj]);
+        }
+      }
+      const int t = r0 + ty;
+#pragma unroll
+      for (int jj = 0; jj < 4; ++jj) {
+        const int s = tx + 16 * jj;
+        sA[t * C + s] = s < t ? a[jj] : 0.f;
+        sP[t * C + s] = s <= t ? pp[jj] : 0.f;
+      }
+    }
+    __syncthreads();
   }
-  __syncthreads();
-
   // T = (I + Diag(beta) A)^-1, blocked.  (1) The four 16x16 diagonal blocks by forward
   // substitution: column task j = tid / 4 (block j / 16), its four threads split each
   // row's sum and combine it with two shuffles inside their aligned group of four.
@@ -500,6 +587,7 @@ __global__ void __launch_bounds__(NTH, 1) bwd_prep_kernel(const BwdParams p) {
     tc_fence_before();
     __syncthreads();
     if (!done && tid == 0) mbar_wait(bar, 0, 100000000ull);  // give the products a last chance
+    if (!ap_done && tid == 0) mbar_wait(bar + 1, 0, 100000000ull);  // and the A|P products
     __syncthreads();
     if (w == 0) {
       tc_fence_after();
