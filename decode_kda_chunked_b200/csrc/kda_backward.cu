@@ -38,10 +38,10 @@
 // The state and gradient passes are fp32 on the CUDA cores: a CTA's 256 threads
 // form a 16 x 16 grid, and thread (ty, tx) owns rows ty + 16 i and columns
 // tx + 16 j of every tile it produces, so per-element folds stay in registers.
-// For bf16 inputs at d = 128 the prep pass runs its four products as tcgen05
-// tf32 MMAs (transposed to M = 128 TMEM lanes, as in the forward), and so does
-// bwd_sprod with the four products of the state; fp32 inputs keep fp32 products
-// throughout.
+// For bf16 inputs at d = 128 the prep pass forms A and P and runs its four
+// products as tcgen05 tf32 MMAs (transposed to M = 128 TMEM lanes, as in the
+// forward), and so does bwd_sprod with the four products of the state; fp32
+// inputs keep fp32 products throughout.
 #include "kda_internal.cuh"
 #include "kda_sm100.cuh"
 
