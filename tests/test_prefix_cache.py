@@ -39,7 +39,10 @@ def test_model_never_evicts_its_own_prompt():
 
 
 class Native:
+    """The libkda.so index behind the model's interface."""
+
     def __init__(self, block, n_slots):
+        self.block = block
         self.h = _lib.kda_prefix_cache_create(block, n_slots)
 
     def lookup(self, ids, max_tokens=None):
@@ -47,7 +50,7 @@ class Native:
 
     def insert(self, ids, first_block=0):
         k, out = _lib.kda_prefix_cache_insert(self.h, ids, first_block)
-        return k, [int(x) for x in out[:len(ids) // _BLOCK[0]]]
+        return k, [int(x) for x in out[:len(ids) // self.block]]
 
     def __len__(self):
         return _lib.kda_prefix_cache_size(self.h)
@@ -56,12 +59,8 @@ class Native:
         _lib.kda_prefix_cache_destroy(self.h)
 
 
-_BLOCK = [0]
-
-
 @pytest.mark.parametrize("block,n_slots,seed", [(2, 3, 0), (4, 5, 1), (3, 16, 2), (512, 6, 3)])
 def test_native_index_matches_model(block, n_slots, seed):
-    _BLOCK[0] = block
     rng = np.random.default_rng(seed)
     model, native = PrefixCacheModel(block, n_slots), Native(block, n_slots)
     # a few stems that prompts extend, so prefixes are shared and partly diverge
