@@ -484,7 +484,7 @@ __global__ void __launch_bounds__(NT + 32, 1)
           *reinterpret_cast<float4 *>(sm + OFF_KHT + sw128_chunk(DH, l, 16 * g + 4 * m4)) =
               make_float4(kh[4 * m4], kh[4 * m4 + 1], kh[4 * m4 + 2], kh[4 * m4 + 3]);
       }
-      wsync();  // every raw tile read: the raw region now takes the R'_a operands
+      wsync();  // every raw tile read: the raw region now takes the R'_b operands
       // R'_b row j = k_j exp(G_mb - G_j) for the rows j of blocks up to b, m_b = 32 b + 15
       // (the 16-row group end 2b of the G table), spread over all workers.  One exponential
       // of the exponent difference: a factor underflows only where the true factor is
@@ -517,7 +517,7 @@ __global__ void __launch_bounds__(NT + 32, 1)
       for (int j = 0; j < 16; ++j)
         *reinterpret_cast<float *>(sm + OFF_GQ + sw128_offset(C, 16 * g + j, l)) = gkT[j];
       tmem_wait_st();
-      warp_arrive(bar_raw);  // R'_a consumed (next TMA may start); V^T and gamma*K ready
+      warp_arrive(bar_raw);  // R'_b consumed (next TMA may start); V^T and gamma*K ready
 
       // ---- a4: T = (I + Diag(beta) A)^-1 (blocked, fp32), P operand ------------
       float *Ms = reinterpret_cast<float *>(sm + OFF_MS);
