@@ -146,19 +146,60 @@ def load_peaks():
 # distributed plumbing (timing only; the workload has no collective)
 # ---------------------------------------------------------------------------
 
-def dist_setup():
+def torchrun_command(n: int, argv, port: int) -> list:
+    """The one-node launch of this script on n ranks (one process per GPU)."""
+    return [sys.executable, "-m", "torch.distributed.run", "--nnodes=1",
+            f"--nproc-per-node={n}", "--master-addr=127.0.0.1", f"--master-port={port}",
+            os.path.abspath(__file__), *argv]
+
+
+def free_port() -> int:
+    import socket
+    with socket.socket() as s:
+        s.bind(("127.0.0.1", 0))
+        return s.getsockname()[1]
+
+
+def launch_ranks(n: int, argv) -> int:
+    """``--gpus N`` with N > 1 and no launcher around this process: start the N
+    ranks through torchrun and return its exit status.  The outer bound is well
+    above the process group's own timeout, so ranks that wait on one another end
+    with an error first."""
+    cmd = ["timeout", "-k", "60", "3600", *torchrun_command(n, argv, free_port())]
+    return subprocess.call(cmd)
+
+
+def dist_setup(expect: int, backend: str = "nccl"):
+    """Rank, world and local rank from the launcher's environment; joins the
+    process group when world > 1.  ``expect`` is the --gpus value: a world of
+    another size is an error, so a run never reports N GPUs it did not use."""
     import torch
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
     local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != expect:
+        raise SystemExit(f"bench.py: --gpus {expect} but the launcher started {world} rank(s)")
     if world > 1:
         import datetime
 
         import torch.distributed as dist
-        torch.cuda.set_device(local)
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                device_id=torch.device("cuda", local))
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+            dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                    device_id=torch.device("cuda", local))
+        else:
+            dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+        if dist.get_world_size() != world:
+            raise SystemExit("bench.py: the process group size differs from WORLD_SIZE")
     return world, rank, local
+
+
+def process_group_info(world: int) -> dict:
+    """Backend and size of the communicator the ranks share (none at one rank)."""
+    if world == 1:
+        return {"backend": None, "size": 1}
+    import torch.distributed as dist
+    return {"backend": dist.get_backend(), "size": dist.get_world_size()}
 
 
 def barrier(world):
@@ -168,13 +209,26 @@ def barrier(world):
 
 
 def max_over_ranks(x: float, world: int) -> float:
+    """The largest x over all ranks (every rank gets it)."""
     if world == 1:
         return x
     import torch
     import torch.distributed as dist
-    t = torch.tensor([x], dtype=torch.float64, device="cuda")
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
     return float(t.item())
+
+
+def run_dist_check(args, world, rank):
+    """Launcher check without a GPU (gloo): every rank reports its own rank as a
+    stand-in time, and rank 0 prints the rank count and the max over ranks."""
+    barrier(world)
+    m = max_over_ranks(float(rank), world)
+    if rank == 0:
+        print(json.dumps({"dist_check": True, "n_gpus": world,
+                          "process_group": process_group_info(world),
+                          "max_over_ranks": m}), flush=True)
 
 
 # ---------------------------------------------------------------------------
@@ -360,8 +414,12 @@ def run_ours(args, world, rank, local):
                          "algorithmic_bytes_per_launch": bytes_,
                          "launch_ms": launch_ms,
                          "tensor_frac": tflops / peaks["bf16_tflops"],
+                         "tensor_frac_of": "the measured bf16 dense peak; the MMAs are "
+                                           "kind::tf32, whose nominal rate is half of bf16",
+                         "tensor_frac_of_tf32": tflops / (0.5 * peaks["bf16_tflops"]),
                          "kernel": "prefill (schedule + chunked prefill launches)"},
             "gpu_launches": 2 * args.steps,
+            "process_group": process_group_info(world),
             "clocks": clocks}
 
     if not args.no_decode:
@@ -621,14 +679,21 @@ def bench_kcp_million(args, dev, peaks, world, rank):
                                                      stream=stream), 0, 1, stream)
         out["unsplit_ms"] = ms_unsplit
         out["speedup_vs_unsplit"] = ms_unsplit / ms
-    # two passes over the inputs (pass 1 reads k, v, g, beta twice: state and transition)
-    b = (T * H * (2 * (2 * d * 2 + 4 * d + 4))       # pass 1, two CTAs per segment-head
-         + prefill_bytes(T, H, d, d, n_seg, initial=True, final=False)
-         + (T // 512) * H * d * d * 4)               # snapshots
+    b = kcp_bytes(T, H, d, n_seg)
     out["roofline"] = {"bound": "hbm", "achieved": b / (ms * 1e-3) / 1e9,
                        "peak": peaks["hbm_gbs"] * world, "unit": "GB/s",
                        "frac": b / (ms * 1e-3) / 1e9 / (peaks["hbm_gbs"] * world)}
     return out
+
+
+def kcp_bytes(T: int, H: int, d: int, n_seg: int, stride: int = 512) -> int:
+    """Algorithmic bytes of the split run: pass 1 reads k, v (bf16), g and beta once
+    per token-head (1,028 B at d = 128) and writes (S_loc, M) per segment-head; pass 2
+    is the chunked prefill with fp32 o from the recovered start states; plus the fp32
+    snapshots every ``stride`` tokens."""
+    pass1 = T * H * (2 * d * 2 + 4 * d + 4) + 2 * n_seg * H * d * d * 4
+    pass2 = prefill_bytes(T, H, d, d, n_seg, initial=True, final=False)
+    return pass1 + pass2 + (T // stride) * H * d * d * 4
 
 
 def bench_e2e(args, inp, dev, world, gate_logits: bool = False):
@@ -722,18 +787,27 @@ def main():
                     help="keep only the first N requests of the varlen workload (profiling)")
     ap.add_argument("--decode-requests", type=int, default=256,
                     help="requests in the decode step (256 in the standard workload)")
+    ap.add_argument("--dist-check", action="store_true",
+                    help="launcher check on CPU (gloo): rank count and max over ranks only")
     args = ap.parse_args()
     if args.warmup < 3:
         args.warmup = 3  # the timing rules ask for at least 3 warm-up steps
-    world, rank, local = dist_setup() if args.impl == "ours" else (
-        int(os.environ.get("WORLD_SIZE", "1")), int(os.environ.get("RANK", "0")), 0)
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(launch_ranks(args.gpus, sys.argv[1:]))
+    if args.impl == "reference":
+        # the oracle runs on rank 0's host cores; the other ranks exit without work
+        world = int(os.environ.get("WORLD_SIZE", "1"))
+        rank = int(os.environ.get("RANK", "0"))
+        run_reference(args, world, rank)
+        return
+    world, rank, local = dist_setup(args.gpus, "gloo" if args.dist_check else "nccl")
     try:
-        if args.impl == "reference":
-            run_reference(args, world, rank)
+        if args.dist_check:
+            run_dist_check(args, world, rank)
         else:
             run_ours(args, world, rank, local)
     finally:
-        if world > 1 and args.impl == "ours":
+        if world > 1:
             import torch.distributed as dist
             dist.destroy_process_group()
 

@@ -7,6 +7,7 @@
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
+#include <mutex>
 #include <vector>
 
 #include "kda_internal.cuh"
@@ -20,9 +21,12 @@ __device__ unsigned int g_device_status;
 namespace {
 
 constexpr int kMaxDevices = 64;
-unsigned int *g_status_addr[kMaxDevices];  // cached device address per ordinal
 
-constexpr int kMaxScheduledRequests = 16384;  // longer lists run in index order
+// Longer request lists run in index order (no workspace).  The allocation-free
+// entry point's scratch holds exactly one order of this many requests.
+constexpr int kMaxScheduledRequests = KDA_NOALLOC_MAX_REQUESTS;
+static_assert(kMaxScheduledRequests == KDA_NOALLOC_MAX_REQUESTS,
+              "the allocation-free scratch must hold every order the workspace path writes");
 
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
@@ -115,17 +119,49 @@ kda_status from_cuda(cudaError_t e) {
   return KDA_ERR_CUDA;
 }
 
+// The current thread's CUDA context, through the driver entry point the
+// runtime exposes (the library does not link libcuda).  NULL if unavailable.
+CUcontext current_context() {
+  using Fn = CUresult (*)(CUcontext *);
+  static Fn fn = [] {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    return (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) ==
+                cudaSuccess &&
+            q == cudaDriverEntryPointSuccess)
+               ? reinterpret_cast<Fn>(ptr)
+               : nullptr;
+  }();
+  CUcontext ctx = nullptr;
+  if (!fn || fn(&ctx) != CUDA_SUCCESS) return nullptr;
+  return ctx;
+}
+
 }  // namespace
 
-unsigned int *device_status_word() {
+// Device addresses of this library's __device__ arrays, looked up with
+// cudaGetSymbolAddress once per device and context: a device reset (or any
+// new primary context) gives the module new addresses, so an entry is reused
+// only while the context it was taken in is still current.  The lock makes a
+// first call from two host threads at once safe.
+SymbolAddressCache::SymbolAddressCache(const void *symbol) : symbol_(symbol) {}
+
+void *SymbolAddressCache::get() {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  if (!g_status_addr[dev]) {
-    void *addr = nullptr;
-    if (cudaGetSymbolAddress(&addr, g_device_status) != cudaSuccess) return nullptr;
-    g_status_addr[dev] = static_cast<unsigned int *>(addr);
-  }
-  return g_status_addr[dev];
+  std::lock_guard<std::mutex> hold(mu_);
+  CUcontext ctx = current_context();
+  if (ctx && ctx == ctx_[dev] && addr_[dev]) return addr_[dev];
+  void *addr = nullptr;  // also makes the device's primary context current
+  if (cudaGetSymbolAddress(&addr, symbol_) != cudaSuccess) return nullptr;
+  ctx_[dev] = current_context();
+  addr_[dev] = addr;
+  return addr;
+}
+
+unsigned int *device_status_word() {
+  static SymbolAddressCache cache(reinterpret_cast<const void *>(&g_device_status));
+  return static_cast<unsigned int *>(cache.get());
 }
 
 }  // namespace kda
@@ -344,21 +380,13 @@ namespace {
 
 // Scratch of kda_prefill_chunked_noalloc.  Host code must not use this name
 // as a device address: it is a host-side stand-in.  The device address comes
-// from cudaGetSymbolAddress, looked up once per device.
+// from cudaGetSymbolAddress, looked up on the first call with a device (and
+// context) current and reused after that.
 static __device__ __align__(256) int32_t g_noalloc_order[KDA_NOALLOC_MAX_REQUESTS];
 
-int32_t *g_noalloc_addr[kMaxDevices];  // device address of g_noalloc_order per ordinal
-
-// Per-device set-up on the first call with that device current.
 int32_t *noalloc_scratch() {
-  int dev = 0;
-  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return nullptr;
-  if (!g_noalloc_addr[dev]) {
-    int32_t *ptr = nullptr;
-    if (cudaGetSymbolAddress((void **)&ptr, g_noalloc_order) != cudaSuccess) return nullptr;
-    g_noalloc_addr[dev] = ptr;
-  }
-  return g_noalloc_addr[dev];
+  static SymbolAddressCache cache(reinterpret_cast<const void *>(&g_noalloc_order));
+  return static_cast<int32_t *>(cache.get());
 }
 
 }  // namespace

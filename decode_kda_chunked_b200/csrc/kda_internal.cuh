@@ -2,9 +2,12 @@
 // Nothing here is part of the public C ABI (include/kda.h).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_bf16.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
+
+#include <mutex>
 
 #include "kda.h"
 
@@ -77,6 +80,20 @@ cudaError_t launch_combine(const float *s_loc, const float *m, const float *s_in
                            int H, int dk, int dv, float *s_in, float *s_final,
                            cudaStream_t stream);
 unsigned int *device_status_word();  // address of the current device's status word
+
+// Device address of a __device__ symbol of this library on the current device,
+// cached per device and context under a lock (kda_api.cu).
+class SymbolAddressCache {
+ public:
+  explicit SymbolAddressCache(const void *symbol);
+  void *get();  // NULL if no device is usable
+
+ private:
+  const void *symbol_;
+  std::mutex mu_;
+  CUcontext ctx_[64] = {};
+  void *addr_[64] = {};
+};
 
 // Backward of the prefill (kda_backward.cu).  The workspace holds, in order,
 // the chunk table, the chunk-start snapshots of a forward pass, a zero state

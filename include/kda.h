@@ -177,8 +177,10 @@ kda_status kda_prefill_chunked(const kda_prefill_args *args, void *workspace,
  *   - n_req > KDA_NOALLOC_MAX_REQUESTS returns KDA_ERR_WORKSPACE and launches
  *     nothing;
  *   - the first call on each device looks up the array's device address
- *     (cudaGetSymbolAddress) with that device current; make that first call
- *     before any stream capture;
+ *     (cudaGetSymbolAddress) with that device current, and so does the first
+ *     call after the device's context changes (cudaDeviceReset); make that
+ *     first call before any stream capture.  The lookup is guarded by a
+ *     lock, so first calls from several host threads are safe;
  *   - every call on a device shares the one array, which keeps the last
  *     call's contents.  Nothing in it needs to start at zero: each call
  *     rewrites entries 0 .. n_req-1 before reading them.  Calls that overlap

@@ -56,3 +56,51 @@ def test_traffic_record_matches_the_kernel_source():
     the bench reports its traffic instead of null."""
     t = bench.measured_traffic(1_000_000)
     assert t is not None and 0.9e6 < t < 1.1e6
+
+
+def test_kcp_bytes_count_each_input_once():
+    # pass 1 reads k, v (bf16), g and beta once per token-head: 1,028 B at d = 128, and
+    # writes (S_loc, M) per segment-head; pass 2 is the prefill with fp32 o from the
+    # recovered start states; snapshots every 512 tokens
+    T, H, n_seg = 65536, 1, 1
+    pass1 = T * H * 1_028 + 2 * n_seg * H * D * D * 4
+    pass2 = T * H * 1_796 + n_seg * H * D * D * 4
+    snaps = (T // 512) * H * D * D * 4
+    assert bench.kcp_bytes(T, H, D, n_seg) == pass1 + pass2 + snaps
+    # the million-token workload: about 17.2 GB + 30.1 GB + 2.15 GB
+    assert 49.4e9 < bench.kcp_bytes(1 << 20, 16, D, 16) < 49.6e9
+
+
+def test_launcher_command_is_one_node_torchrun():
+    cmd = bench.torchrun_command(4, ["--gpus", "4", "--steps", "2"], 29511)
+    assert cmd[1:4] == ["-m", "torch.distributed.run", "--nnodes=1"]
+    assert "--nproc-per-node=4" in cmd and "--master-addr=127.0.0.1" in cmd
+    assert "--master-port=29511" in cmd
+    assert cmd[-4:] == ["--gpus", "4", "--steps", "2"]
+
+
+def test_gpus_flag_starts_that_many_ranks():
+    """`bench.py --gpus 2` outside any launcher starts two ranks itself; the ranks
+    join one process group (gloo here, NCCL on GPUs) and rank 0 reports the group
+    size and the max over ranks of a per-rank value."""
+    import json
+    import subprocess
+    env = {k: v for k, v in os.environ.items()
+           if k not in ("WORLD_SIZE", "RANK", "LOCAL_RANK", "MASTER_ADDR", "MASTER_PORT")}
+    out = subprocess.run([sys.executable, bench.__file__, "--gpus", "2", "--dist-check"],
+                         env=env, capture_output=True, text=True, timeout=300)
+    assert out.returncode == 0, out.stderr[-2000:]
+    lines = [json.loads(x) for x in out.stdout.splitlines() if x.startswith("{")]
+    assert len(lines) == 1
+    rec = lines[0]
+    assert rec["n_gpus"] == 2
+    assert rec["process_group"] == {"backend": "gloo", "size": 2}
+    assert rec["max_over_ranks"] == 1.0
+
+
+def test_world_size_must_match_the_gpus_flag():
+    import subprocess
+    env = dict(os.environ, WORLD_SIZE="1", RANK="0", LOCAL_RANK="0")
+    out = subprocess.run([sys.executable, bench.__file__, "--gpus", "3", "--dist-check"],
+                         env=env, capture_output=True, text=True, timeout=120)
+    assert out.returncode != 0 and "--gpus 3" in out.stderr
