@@ -37,6 +37,15 @@ bool env_flag(const char *name) {
   return v && v[0] && std::strcmp(v, "0") != 0;
 }
 
+// Limit of the bounded waits inside the tensor-core kernels, in ns; 0 keeps the
+// kernels' 2 s.  KDA_TEST_WAIT_LIMIT_NS exists for tests that make a wait run out
+// on purpose (to exercise the timeout path); nothing else should set it.
+unsigned long long wait_limit_ns() {
+  const char *v = std::getenv("KDA_TEST_WAIT_LIMIT_NS");
+  if (!v || !v[0]) return 0ull;
+  return std::strtoull(v, nullptr, 10);
+}
+
 bool valid_dtype(kda_dtype d) { return d == KDA_BF16 || d == KDA_F32; }
 size_t dsize(kda_dtype d) { return d == KDA_BF16 ? 2 : 4; }
 
@@ -199,6 +208,7 @@ kda_status kda_prefill_chunked(const kda_prefill_args *a, void *workspace,
   p.H = a->H; p.dk = a->dk; p.dv = a->dv;
   p.snapshot_stride = a->snapshot_stride;
   p.validate = env_flag("KDA_VALIDATE");
+  p.wait_ns = wait_limit_ns();
   p.status = device_status_word();
   if (!p.status) return KDA_ERR_CUDA;
   if (need > 0) {
@@ -263,6 +273,7 @@ kda_status kda_chunk_local_state(const kda_local_state_args *a, void *workspace,
   p.s_loc = a->s_loc;
   p.m = a->m;
   p.validate = env_flag("KDA_VALIDATE");
+  p.wait_ns = wait_limit_ns();
   p.status = device_status_word();
   if (!p.status) return KDA_ERR_CUDA;
   cudaStream_t s = static_cast<cudaStream_t>(stream);

@@ -47,6 +47,9 @@ struct PrefillParams {
   int n_slices;                  // column slices per (request, head)
   int validate;
   unsigned int *status;
+  // Limit of every bounded wait inside the tensor-core kernel, in ns (0: 2 s).
+  // Only tests shorten it, to make a wait run out on purpose.
+  unsigned long long wait_ns;
   // local-state mode: columns [0, dv) of the augmented state are S_loc (V,
   // zero start), columns [dv, dv + dk) are M (zero V, identity start).
   int local_mode;

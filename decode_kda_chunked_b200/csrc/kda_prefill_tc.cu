@@ -4,41 +4,45 @@
 //
 // The chunk algebra is that of the chunk-parallel form (tokens of a chunk in
 // parallel, state passed between chunks in order: "Kimi K3 开源日来了",
-// FlashKDA section), written transposed so that every MMA has M = 128 with
-// one TMEM lane per feature channel (S^T, U^T, O^T have lanes = value
-// channels, columns = key channels or tokens):
+// FlashKDA section), here with chunks of 32 tokens, written transposed so that
+// every MMA has M = 128 with one TMEM lane per feature channel (S^T, U^T, O^T
+// have lanes = value channels, columns = key channels or tokens):
 //
-//   A | P   [128 x 32(b+1)] per 32-row block b: [L ; Lq] R'_b^T             (A from TMEM)
-//   Y^T     = V^T - S^T (gamma*K)^T                                          (A = S^T in TMEM)
-//   U^T     = Y^T (T Diag(b))^T                                              (A = Y^T in TMEM)
-//   O^T     = S^T (gamma*Q)^T + U^T P^T                                      (A = S^T, U^T in TMEM)
-//   S^T    <- S^T Diag(gamma_63) + U^T Khat                                  (A = U^T in TMEM)
-// U = T Diag(b) (V - (gamma*K) S) is the chunk form's U~ - W S with W never formed:
-// Y needs only the state and the chunk's inputs, so it runs while the workers solve T.
+//   A | P   [128 x 32] = [L_k ; L_q] R'^T                 (A from TMEM, lanes 0-31 | 32-63)
+//   O^T     = S^T (gamma*Q)^T                            (A = S^T in TMEM)
+//   Y^T     = V^T - S^T (gamma*K)^T                      (A = S^T in TMEM, D starts as V^T)
+//   U^T     = Y^T (T Diag(b))^T                          (A = Y^T in TMEM)
+//   O^T    += U^T P^T,   S^T <- S^T Diag(gamma_31) + U^T Khat      (A = U^T in TMEM)
+// U = T Diag(b) (V - (gamma*K) S) is the chunk form's U~ - W S with W never formed.
 //
-// Gate factorisation for A and P: rows come in two 32-row blocks b with reference
-// rows m_b = 32 b + 15, and exp(G_i - G_j) = exp(G_i - G_mb) * exp(G_mb - G_j) for a
-// row i of block b and a column j <= i.  The left factor is <= exp(5 * 15) (rows
-// i < m_b) or <= 1; the right factor is <= exp(5 * 16) (columns j > m_b) or <= 1.
-// Because log alpha >= -5 (the lower-bounded decay of KDA, CSDN post on the Kimi K3
-// technical report, section 一.1) every factor is a finite fp32 number, and only
-// masked products (j > i) can overflow; they are dropped by selection, never
-// multiplied.  Column j's right factor for block b follows from its own block's
-// factor times the block-to-block decay exp(G_mb - G_m(j)) <= 1, so each row
-// needs one exponential per channel.  Each block's product runs as two 8-step
-// accumulation chains over the halves of the key channels, summed on read-out.
+// Gate factorisation for A and P: exp(G_i - G_j) = exp(G_i - G_15) exp(G_15 - G_j) with
+// the chunk's row 15 as reference.  The left factor is <= exp(5 * 15) (rows i < 15) or
+// <= 1, the right factor <= exp(5 * 16) (columns j > 15) or <= 1.  Because
+// log alpha >= -5 (the lower-bounded decay of KDA, CSDN post on the Kimi K3 technical
+// report, section 一.1) every factor is a finite fp32 number; only masked products
+// (j > i) can overflow, and they are dropped by selection, never multiplied.
 //
-// All tensor-core operands are tf32 (B operands K-major with the 128-byte
-// swizzle in shared memory): bf16 operands for the gate-scaled products would
-// cost about 2e-3 of relative accuracy, tf32 stays near 5e-4.
+// All tensor-core operands are tf32 (B operands K-major with the 128-byte swizzle in
+// shared memory, rounded to nearest): bf16 operands for the gate-scaled products
+// would cost about 2e-3 of relative accuracy, tf32 stays near 5e-4.
 //
-// One CTA runs one (request, head) chain with 16 worker warps and one control
-// warp.  Worker warp w reaches the TMEM lane quarter w % 4, and the four warps
-// sharing a quarter split the columns.  The control warp issues the TMA loads
-// and every tcgen05.mma; workers and control hand off through mbarriers
-// (operands ready / MMA done / raw tiles consumed), so MMA issue never stalls
-// a worker warp.  Every wait is bounded; a timeout is reported through the
-// status word.
+// Pipeline.  One CTA runs one (request, head) chain with 16 worker warps and one
+// control warp; the control warp issues every TMA load and tcgen05.mma, the workers
+// do the SIMT work, and they hand off through mbarriers.  Iteration n of the worker
+// loop finishes chunk n's state products while it prepares chunk n+1:
+//
+//   gate(n+1)  cumulative gate of chunk n+1              (raw tiles loaded long before)
+//   scale(n)   S^T *= gamma_31(n) once O^T, Y^T(n) read S^T   -> control: last products(n)
+//   rows(n+1)  L_k, L_q -> TMEM, R', gamma*Q, gamma*K -> smem  -> control: A|P(n+1)
+//   out(n)     after last products(n): Khat^T(n+1), O^T(n) -> o, snapshot(n)
+//   read(n+1)  after A|P(n+1): Diag(b) A, P, V^T(n+1) -> TMEM  -> control: O^T, Y^T(n+1)
+//   solve(n+1) T Diag(b)                                        -> control: U^T(n+1)
+//
+// so every product runs while the workers do other work, and every buffer is
+// rewritten only after the product that reads it has completed.  Raw tiles are
+// double buffered: chunk m+2 is loaded as soon as chunk m's tiles are read.
+// Every wait is bounded; a wait that runs out ends the CTA with KDA_ERR_TIMEOUT in
+// the status word, after the CTA has let every copy and product it issued land.
 #include "kda_internal.cuh"
 #include "kda_sm100.cuh"
 
@@ -47,84 +51,85 @@ namespace {
 
 using namespace sm100;
 
-constexpr int C = 64;     // chunk
+constexpr int C = 32;     // tokens per chunk of this kernel
 constexpr int DH = 128;   // head dim (dk = dv)
 constexpr int NT = 512;   // worker threads per CTA: 16 warps (plus one control warp)
+constexpr int MREF = 15;  // reference row of the gate factorisation
 constexpr float LOG2E = 1.4426950408889634f;
 
-// Thread (g, l): warp w = tid / 32 owns TMEM lane quarter w % 4, so
-// l = 32 (w % 4) + tid % 32 is the thread's TMEM lane, and g = w / 4 picks a
-// quarter of the columns (32 of 128, or 16 of 64).
-
 // ---- shared memory map (byte offsets from a 1024-aligned base) ----
-constexpr uint32_t OFF_KRAW = 0;        // bf16 [64 x 128]: 2 TMA boxes of 64 cols (SW128)
-constexpr uint32_t OFF_QRAW = 16384;
-constexpr uint32_t OFF_VRAW = 32768;
-constexpr uint32_t OFF_GRAW = 49152;    // fp32 [64 x 128]: 4 TMA boxes of 32 cols (SW128), or
-                                        // bf16 gate logits in its first half (2 boxes of 64
-                                        // cols, as q/k/v); rewritten in place with
-                                        // log2(e) * cumsum(g)
-constexpr uint32_t RAW_BYTES = 81920;
-// Once every raw tile is read, the raw region holds the B operands R'_b of
-// the A|P products: row block b (32 rows) has 32(b+1) rows at byte 16384 b.
-__host__ __device__ constexpr uint32_t rp_off(int b) { return 16384u * b; }
-constexpr uint32_t OFF_R = 81920;       // R scratch [64 x 132] fp32, then T-solve scratch
-constexpr int LDT = 65;                 // padded row stride of the T-solve scratch
-constexpr int LDR = 132;                // padded row stride of the fp32 R scratch [64][132]
-constexpr uint32_t OFF_MS = OFF_R;                  // beta*A strict lower
-constexpr uint32_t OFF_TI = OFF_R + 64 * LDT * 4;   // T = (I + beta A)^-1
-constexpr uint32_t OFF_GQ = 115712;     // (gamma*Q) [64 x 128] tf32 B operand; once the O^T
-                                        // product has read it, (gamma*K) [64 x 128]
-constexpr uint32_t OFF_KHT = 148480;    // Khat^T [128 x 64] tf32 B operand
-constexpr uint32_t OFF_TB = 181248;     // T Diag(beta) [64 x 64] tf32 B operand
-constexpr uint32_t OFF_P = 197632;      // P [64 x 64] tf32 B operand
-constexpr uint32_t OFF_Y = 214016;      // the T-solve products ([2][16][17], then [32][33])
-constexpr uint32_t OFF_EGR = 222208;    // exp(G_rb)[4][128], r_b = 16 b + 15
-constexpr uint32_t OFF_SEG = 224256;    // cumsum segment totals [4][128]
-constexpr uint32_t OFF_GR2 = 226304;    // log2(e) * G at rows 16 b + 15 [4][128]
-constexpr uint32_t OFF_BETA = 228352;   // beta[64]
-constexpr uint32_t OFF_BAR = 228608;    // mbarriers + TMEM base + flags
-constexpr uint32_t SMEM_BYTES = 228704;
-static_assert(OFF_TI + 64 * LDT * 4 <= OFF_GQ, "T-solve scratch must fit the R region");
-static_assert(OFF_R + 64 * LDR * 4 <= OFF_GQ, "R scratch must fit the R region");
+// Raw tiles of one chunk: q, k, v bf16 [32 x 128] as two 64-column 128B-swizzled TMA
+// boxes each; g fp32 [32 x 128] as four 32-column boxes (bf16 gate logits: two
+// 64-column boxes).  Chunk m uses buffer m & 1.
+constexpr uint32_t RAW_BYTES = 40960;
+constexpr uint32_t R_K = 0, R_Q = 8192, R_V = 16384, R_G = 24576;
+constexpr uint32_t OFF_RAW = 0;
+constexpr uint32_t OFF_GT = 81920;   // log2(e) * G (chunk-local cumulative gate), fp32 [32][LDG]
+constexpr int LDG = 132;             // padded so that row-wise float4 reads hit distinct banks
+constexpr uint32_t OFF_GQ = 99328;   // gamma*Q  tf32 B operand [32 x 128]
+constexpr uint32_t OFF_GK = 115712;  // gamma*K  tf32 B operand [32 x 128]
+constexpr uint32_t OFF_KH = 132096;  // Khat^T   tf32 B operand [128 x 32]
+constexpr uint32_t OFF_RP = 148480;  // R'       tf32 B operand [32 x 128]
+constexpr uint32_t OFF_PP = 164864;  // P        tf32 B operand [32 x 32]
+constexpr uint32_t OFF_TB = 168960;  // T Diag(beta) tf32 B operand [32 x 32]
+constexpr uint32_t OFF_NS = 173056;  // Diag(beta) A, strict lower, fp32 [32][LDN]
+constexpr int LDN = 36;
+constexpr uint32_t OFF_TS = 177664;  // the two diagonal 16x16 blocks of T, fp32 [32][LDN]
+constexpr uint32_t OFF_XS = 182272;  // N10 T00, fp32 [16][LDX]
+constexpr int LDX = 20;
+constexpr uint32_t OFF_GC = 183552;  // exp(G_31) per key channel, [2][128] by chunk parity
+constexpr uint32_t OFF_BT = 184576;  // beta of the chunk being prepared [32]
+constexpr uint32_t OFF_SEG = 184704; // cumulative-gate segment totals [4][128]
+constexpr uint32_t OFF_BAR = 186752; // mbarriers, TMEM base, flags
+constexpr uint32_t SMEM_BYTES = 187008;
 constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;  // alignment slack
+static_assert(OFF_RAW + 2 * RAW_BYTES <= OFF_GT, "raw buffers");
+static_assert(OFF_GT + C * LDG * 4 <= OFF_GQ, "gate table");
+static_assert(OFF_GQ % 1024 == 0 && OFF_GK % 1024 == 0 && OFF_KH % 1024 == 0 &&
+                  OFF_RP % 1024 == 0 && OFF_PP % 1024 == 0 && OFF_TB % 1024 == 0,
+              "swizzled operands need 1024-byte alignment");
+static_assert(OFF_GQ + 16384 == OFF_GK && OFF_GK + 16384 == OFF_KH && OFF_KH + 16384 == OFF_RP &&
+                  OFF_RP + 16384 == OFF_PP && OFF_PP + 4096 == OFF_TB && OFF_TB + 4096 == OFF_NS,
+              "operand tiles");
+static_assert(OFF_NS + C * LDN * 4 == OFF_TS && OFF_TS + C * LDN * 4 == OFF_XS &&
+                  OFF_XS + 16 * LDX * 4 == OFF_GC && OFF_GC + 2 * DH * 4 == OFF_BT &&
+                  OFF_BT + C * 4 == OFF_SEG && OFF_SEG + 4 * DH * 4 == OFF_BAR,
+              "scratch tiles");
 
 // ---- TMEM column map (512 columns x 128 lanes of fp32) ----
 constexpr uint32_t TM_S = 0;     // S^T (lane = value channel, col = key channel)
-constexpr uint32_t TM_L = 128;   // L* (A operand of A|P); later V^T -> Y^T in [0,64)
-// A (lanes 0..63) | P (lanes 64..127) of the rows of 32-row block b: 32(b+1) columns,
-// summed over two halves of the key channels held apart (two accumulators each)
-constexpr uint32_t TM_AP = 256;  // up to column 448
-__host__ __device__ constexpr uint32_t ap_col(int b, int half) {
-  return TM_AP + (b == 0 ? 32u * half : 64u + 64u * half);
-}
-constexpr uint32_t TM_X2 = 320;  // U^T (alias A|P once the solve has read it)
-constexpr uint32_t TM_O = 448;   // O^T (own columns: issued right after the A|P products)
+constexpr uint32_t TM_L = 128;   // [L_k ; L_q]: A operand of A|P (lanes 0-31 | 32-63)
+constexpr uint32_t TM_AP = 256;  // A (lanes 0-31) | P (lanes 32-63), 32 columns
+constexpr uint32_t TM_Y = 288;   // V^T -> Y^T
+constexpr uint32_t TM_U = 320;   // U^T
+constexpr uint32_t TM_O = 352;   // O^T
 constexpr uint32_t TM_COLS = 512;
 
 struct TcMaps {
   CUtensorMap q, k, v, g;
 };
 
+// bf16 [32 x 128] tile: byte offset of the 16-byte chunk with channels c..c+7 (c % 8 == 0)
+// of row t, and of one element
+__device__ __forceinline__ uint32_t bf16_chunk(int t, int c) {
+  return (uint32_t)(c >> 6) * 4096u + (uint32_t)t * 128u +
+         ((uint32_t)(((c & 63) >> 3) ^ (t & 7)) << 4);
+}
 __device__ __forceinline__ uint32_t bf16_off(int t, int c) {
-  // bf16 [64 x 128] as two 64-column SW128 boxes
-  return (uint32_t)(c >> 6) * 8192u + (uint32_t)t * 128u +
-         ((uint32_t)(((c & 63) >> 3) ^ (t & 7)) << 4) + (uint32_t)(c & 7) * 2u;
+  return bf16_chunk(t, c & ~7) + (uint32_t)(c & 7) * 2u;
+}
+__device__ __forceinline__ float bf16_lo(uint32_t u) { return __uint_as_float(u << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t u) { return __uint_as_float(u & 0xFFFF0000u); }
+__device__ __forceinline__ void bf16_x8(const uint4 u, float *x) {
+  x[0] = bf16_lo(u.x); x[1] = bf16_hi(u.x); x[2] = bf16_lo(u.y); x[3] = bf16_hi(u.y);
+  x[4] = bf16_lo(u.z); x[5] = bf16_hi(u.z); x[6] = bf16_lo(u.w); x[7] = bf16_hi(u.w);
 }
 __device__ __forceinline__ float bf16_at(const unsigned char *tile, int t, int c) {
-  return __bfloat162float(*reinterpret_cast<const __nv_bfloat16 *>(tile + bf16_off(t, c)));
+  return bf16_lo(*reinterpret_cast<const unsigned short *>(tile + bf16_off(t, c)));
 }
-// four consecutive channels c..c+3 (c % 4 == 0) of row t
-__device__ __forceinline__ void bf16_x4(const unsigned char *tile, int t, int c, float *x) {
-  const uint2 u = *reinterpret_cast<const uint2 *>(tile + bf16_off(t, c));
-  x[0] = __uint_as_float(u.x << 16);
-  x[1] = __uint_as_float(u.x & 0xFFFF0000u);
-  x[2] = __uint_as_float(u.y << 16);
-  x[3] = __uint_as_float(u.y & 0xFFFF0000u);
-}
-__device__ __forceinline__ uint32_t g_off(int t, int c) {
-  // fp32 [64 x 128] as four 32-column SW128 boxes
-  return (uint32_t)(c >> 5) * 8192u + (uint32_t)t * 128u +
+// fp32 [32 x 128] tile as four 32-column boxes
+__device__ __forceinline__ uint32_t f32_off(int t, int c) {
+  return (uint32_t)(c >> 5) * 4096u + (uint32_t)t * 128u +
          ((uint32_t)(((c & 31) >> 2) ^ (t & 7)) << 4) + (uint32_t)(c & 3) * 4u;
 }
 __device__ __forceinline__ float tf32_rna(float x) {
@@ -132,9 +137,32 @@ __device__ __forceinline__ float tf32_rna(float x) {
   asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
   return __uint_as_float(r);
 }
-// [64 x 65] fp32 scratch: the padded stride puts a warp's row walk and column
-// walk on 32 distinct banks and keeps addresses affine in the loop indices.
-__device__ __forceinline__ int rot(int r, int c) { return r * LDT + c; }
+__device__ __forceinline__ void ld8f(const float *p, float *x) {
+  const float4 a = reinterpret_cast<const float4 *>(p)[0];
+  const float4 b = reinterpret_cast<const float4 *>(p)[1];
+  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
+
+#ifdef KDA_PHASE_PROFILE
+// Cycles of worker thread 0 per phase of the loop, summed over every CTA (profiling
+// builds only), in the order of the loop: 0 chunk 0's operands, 1 wait for the next
+// chunk's tiles, 2 gate, 3 wait for O^T/Y^T, 4 scale, 5 rows, 6 wait for the last
+// products, 7 Khat^T, 8 out, 9 wait for A|P, 10 read, 11 solve, 12 final state;
+// entry 15 counts the chunks.
+__device__ unsigned long long g_phase_cycles[16];
+#define KDA_PHASE(k)                                              \
+  do {                                                            \
+    if (prof) {                                                   \
+      const long long now_ = clock64();                           \
+      phase_acc[k] += (unsigned long long)(now_ - phase_t);       \
+      phase_t = now_;                                             \
+    }                                                             \
+  } while (0)
+#else
+#define KDA_PHASE(k) \
+  do {               \
+  } while (0)
+#endif
 
 // LOGITS: the gate arrives as bf16 logits (fused gate activation) instead of fp32 g.
 template <typename TOut, bool LOGITS>
@@ -143,28 +171,33 @@ __global__ void __launch_bounds__(NT + 32, 1)
   extern __shared__ unsigned char smem_raw[];
   unsigned char *sm = reinterpret_cast<unsigned char *>(
       (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  float *sEgr = reinterpret_cast<float *>(sm + OFF_EGR);
-  float *sSeg = reinterpret_cast<float *>(sm + OFF_SEG);
-  float *sGr2 = reinterpret_cast<float *>(sm + OFF_GR2);
-  float *sB = reinterpret_cast<float *>(sm + OFF_BETA);
+  float *GT = reinterpret_cast<float *>(sm + OFF_GT);
+  float *NS = reinterpret_cast<float *>(sm + OFF_NS);
+  float *TS = reinterpret_cast<float *>(sm + OFF_TS);
+  float *XS = reinterpret_cast<float *>(sm + OFF_XS);
+  float *GC = reinterpret_cast<float *>(sm + OFF_GC);
+  float *BT = reinterpret_cast<float *>(sm + OFF_BT);
+  float *SEG = reinterpret_cast<float *>(sm + OFF_SEG);
   uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
-  uint64_t *bar_tma = bars + 0;      // TMA -> workers: raw tiles landed
-  uint64_t *bar_raw = bars + 1;      // workers -> control: raw tiles consumed (16 warps)
-  uint64_t *bar_opsap = bars + 2;    // workers -> control: A|P operands built (16 warps)
-  uint64_t *bar_y = bars + 3;        // control -> workers: Y^T product done (S^T read)
-  uint64_t *bar_ops = bars + 4;      // workers -> control: T Diag(beta) ready, S^T scaled
-  uint64_t *bar_ap = bars + 5;       // control -> workers: O^T and A|P products done
-  uint64_t *bar_u = bars + 6;        // control -> control: U^T product done
-  uint64_t *bar_mma = bars + 7;      // control -> workers: chunk's last products done
-  uint64_t *bar_st = bars + 8;       // workers -> control: chunk staged, previous O^T stored
-  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bars + 9);
+  uint64_t *bar_tma = bars + 0;   // [2] TMA -> workers: raw buffer b landed
+  uint64_t *bar_ap = bars + 2;    // commit: A|P products done
+  uint64_t *bar_oy = bars + 3;    // commit: O^T and Y^T products done (S^T read)
+  uint64_t *bar_u = bars + 4;     // commit: U^T product done (control only)
+  uint64_t *bar_fin = bars + 5;   // commit: the chunk's last products done
+  uint64_t *ops_ap = bars + 6;    // workers -> control: A|P operands built
+  uint64_t *raw_free = bars + 7;  // workers -> control: a raw buffer fully read
+  uint64_t *ops_oy = bars + 8;    // workers -> control: V^T, gamma*Q/K, Khat^T, P ready
+  uint64_t *ops_tb = bars + 9;    // workers -> control: T Diag(beta) ready
+  uint64_t *ops_sc = bars + 10;   // workers -> control: S^T scaled by gamma_31
+  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bars + 11);
   volatile int *s_abort = reinterpret_cast<volatile int *>(s_tmem + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane_id = tid & 31;
   const bool control = warp == NT / 32;            // warp 16: TMA and MMA issue
-  const int l = ((warp & 3) << 5) | lane_id;       // TMEM lane of a worker thread
-  const int g = (warp >> 2) & 3;                   // worker column quarter
-  const uint32_t lane = (uint32_t)((warp & 3) * 32) << 16;
+  const int qd = warp & 3;                         // TMEM lane quarter of a worker warp
+  const int cg = (warp >> 2) & 3;                  // its column group
+  const int l = 32 * qd + lane_id;                 // its TMEM lane / channel
+  const uint32_t lane_base = (uint32_t)(32 * qd) << 16;
   const int H = p.H;
   // Local-state mode (context-parallel pass 1): CTA part 0 runs the segment from a
   // zero state with its values (-> S_loc), part 1 from the identity with zero values
@@ -174,9 +207,9 @@ __global__ void __launch_bounds__(NT + 32, 1)
   const int rem = (int)(blockIdx.x % pairs);
   const int r = p.order ? p.order[rem / H] : rem / H;
   const int h = rem % H;
-  const bool load_q = !p.local_mode;
-  constexpr bool logits = LOGITS;
+  const bool has_q = !p.local_mode;
   const bool zero_v = p.local_mode && part == 1;
+  const uint64_t wait_ns = p.wait_ns ? p.wait_ns : 2000000000ull;
   const int bos = p.cu_seqlens[r], eos = p.cu_seqlens[r + 1];
   const int len = eos - bos;
   if (bos < 0 || len < 0 || eos > p.total_tokens) {  // uniform per CTA, before any barrier
@@ -193,14 +226,16 @@ __global__ void __launch_bounds__(NT + 32, 1)
   if (warp == 0) tmem_alloc(s_tmem, TM_COLS);
   if (tid == 0) {
     mbar_init(bar_tma, 1);
-    mbar_init(bar_raw, NT / 32);
-    mbar_init(bar_opsap, NT / 32);
-    mbar_init(bar_ops, NT / 32);
+    mbar_init(bar_tma + 1, 1);
     mbar_init(bar_ap, 1);
-    mbar_init(bar_y, 1);
+    mbar_init(bar_oy, 1);
     mbar_init(bar_u, 1);
-    mbar_init(bar_mma, 1);
-    mbar_init(bar_st, NT / 32);
+    mbar_init(bar_fin, 1);
+    mbar_init(ops_ap, NT / 32);
+    mbar_init(raw_free, NT / 32);
+    mbar_init(ops_oy, NT / 32);
+    mbar_init(ops_tb, NT / 32);
+    mbar_init(ops_sc, NT / 32);
     *s_abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -210,6 +245,12 @@ __global__ void __launch_bounds__(NT + 32, 1)
   const uint32_t tm = *s_tmem;
   const int n_chunks = (len + C - 1) / C;
 
+  // What the control thread issued, so that a CTA that gives up can let it land: the
+  // TMA loads per raw buffer, and the barrier and phase parity of the last commit.
+  uint32_t tma_n0 = 0u, tma_n1 = 0u;
+  uint64_t *last_bar = nullptr;
+  uint32_t last_par = 0u;
+
   if (control) {
     // ======================= control warp: TMA + MMA issue =======================
     if (lane_id == 0) {
@@ -217,26 +258,37 @@ __global__ void __launch_bounds__(NT + 32, 1)
       tma_prefetch_desc(&maps.k);
       tma_prefetch_desc(&maps.v);
       tma_prefetch_desc(&maps.g);
-      auto issue_tma = [&](int c0) {
-        mbar_expect_tx(bar_tma, RAW_BYTES - (load_q ? 0u : 16384u) - (logits ? 16384u : 0u));
-        const int y = bos + c0;
+      const uint32_t tx = (has_q ? 3u : 2u) * 8192u + (LOGITS ? 8192u : 16384u);
+      auto issue_tma = [&](int m) {
+        const int b = m & 1;
+        unsigned char *raw = sm + OFF_RAW + b * RAW_BYTES;
+        mbar_expect_tx(bar_tma + b, tx);
+        const int y = bos + m * C;
         for (int half = 0; half < 2; ++half) {
           const int x = h * DH + 64 * half;
-          tma_load_2d(sm + OFF_KRAW + 8192 * half, &maps.k, x, y, bar_tma);
-          if (load_q) tma_load_2d(sm + OFF_QRAW + 8192 * half, &maps.q, x, y, bar_tma);
-          tma_load_2d(sm + OFF_VRAW + 8192 * half, &maps.v, x, y, bar_tma);
+          tma_load_2d(raw + R_K + 4096 * half, &maps.k, x, y, bar_tma + b);
+          if (has_q) tma_load_2d(raw + R_Q + 4096 * half, &maps.q, x, y, bar_tma + b);
+          tma_load_2d(raw + R_V + 4096 * half, &maps.v, x, y, bar_tma + b);
         }
-        if (logits) {
+        if (LOGITS) {
           for (int half = 0; half < 2; ++half)
-            tma_load_2d(sm + OFF_GRAW + 8192 * half, &maps.g, h * DH + 64 * half, y, bar_tma);
+            tma_load_2d(raw + R_G + 4096 * half, &maps.g, h * DH + 64 * half, y, bar_tma + b);
         } else {
-          for (int qd = 0; qd < 4; ++qd)
-            tma_load_2d(sm + OFF_GRAW + 8192 * qd, &maps.g, h * DH + 32 * qd, y, bar_tma);
+          for (int q4 = 0; q4 < 4; ++q4)
+            tma_load_2d(raw + R_G + 4096 * q4, &maps.g, h * DH + 32 * q4, y, bar_tma + b);
         }
+        if (b) ++tma_n1; else ++tma_n0;
       };
-      uint32_t ph_raw = 0, ph_opsap[1] = {0}, ph_ops = 0, ph_u = 0, ph_st = 0;
+      // one commit per chunk on each barrier: phase m of a barrier belongs to chunk m
+      auto commit = [&](uint64_t *bar, int m) {
+        mma_commit(bar);
+        last_bar = bar;
+        last_par = (uint32_t)m & 1u;
+      };
+      uint32_t ph_ops_ap = 0, ph_raw = 0, ph_ops_oy = 0, ph_tb = 0, ph_sc = 0, ph_oy = 0,
+               ph_u = 0;
       auto cwait = [&](uint64_t *bar, uint32_t &ph) -> bool {
-        const bool good = *s_abort == 0 && mbar_wait(bar, ph);
+        const bool good = *s_abort == 0 && mbar_wait(bar, ph, wait_ns, s_abort);
         ph ^= 1u;
         if (!good) {
           *s_abort = 1;
@@ -245,85 +297,93 @@ __global__ void __launch_bounds__(NT + 32, 1)
         tc_fence_after();
         return good;
       };
+      // A | P: [L_k ; L_q] R'^T, N = 32 over the 128 key channels
+      auto mma_ap = [&](int m) {
+        const uint32_t rp = smem_u32(sm + OFF_RP);
+        const uint32_t id = idesc_tf32(C);
+#pragma unroll
+        for (int s = 0; s < DH / 8; ++s)
+          mma_tf32_ts(tm + TM_AP, tm + TM_L + 8 * s, sw128_desc(rp, C, s), id, s > 0);
+        commit(bar_ap, m);
+      };
+      // O^T = S^T (gamma Q)^T and Y^T = V^T - S^T (gamma K)^T
+      auto mma_oy = [&](int m) {
+        const uint32_t id = idesc_tf32(C), idn = idesc_tf32(C, true);
+        const uint32_t gq = smem_u32(sm + OFF_GQ), gk = smem_u32(sm + OFF_GK);
+#pragma unroll
+        for (int s = 0; s < DH / 8; ++s) {
+          if (has_q) mma_tf32_ts(tm + TM_O, tm + TM_S + 8 * s, sw128_desc(gq, C, s), id, s > 0);
+          mma_tf32_ts(tm + TM_Y, tm + TM_S + 8 * s, sw128_desc(gk, C, s), idn, true);
+        }
+        commit(bar_oy, m);
+      };
+      // U^T = Y^T (T Diag(beta))^T
+      auto mma_u = [&](int m) {
+        const uint32_t tb = smem_u32(sm + OFF_TB);
+        const uint32_t id = idesc_tf32(C);
+#pragma unroll
+        for (int s = 0; s < C / 8; ++s)
+          mma_tf32_ts(tm + TM_U, tm + TM_Y + 8 * s, sw128_desc(tb, C, s), id, s > 0);
+        commit(bar_u, m);
+      };
+      // O^T += U^T P^T and S^T += U^T Khat (S^T already scaled by gamma_31)
+      auto mma_fin = [&](int m) {
+        const uint32_t pp = smem_u32(sm + OFF_PP), kh = smem_u32(sm + OFF_KH);
+        const uint32_t id32 = idesc_tf32(C), id128 = idesc_tf32(DH);
+#pragma unroll
+        for (int s = 0; s < C / 8; ++s) {
+          if (has_q) mma_tf32_ts(tm + TM_O, tm + TM_U + 8 * s, sw128_desc(pp, C, s), id32, true);
+          mma_tf32_ts(tm + TM_S, tm + TM_U + 8 * s, sw128_desc(kh, DH, s), id128, true);
+        }
+        commit(bar_fin, m);
+      };
+      // the products of chunk m that need only its own operands and the current state
+      auto prepare = [&](int m) -> bool {
+        if (!cwait(ops_ap, ph_ops_ap)) return false;
+        mma_ap(m);
+        if (!cwait(raw_free, ph_raw)) return false;
+        if (m + 2 < n_chunks) issue_tma(m + 2);
+        if (!cwait(ops_oy, ph_ops_oy)) return false;
+        mma_oy(m);
+        if (!cwait(ops_tb, ph_tb)) return false;
+        if (!cwait(bar_oy, ph_oy)) return false;  // Y^T is U^T's A operand
+        mma_u(m);
+        return true;
+      };
+      bool ok = true;
       if (n_chunks > 0) issue_tma(0);
-      for (int ci = 0; ci < n_chunks; ++ci) {
-        // O^T = S^T (gamma Q)^T needs only the state and gamma*Q: issue it as soon as the
-        // chunk is staged, so it runs while the workers build the A|P operands
-        if (!cwait(bar_st, ph_st)) break;
-        {
-          const uint32_t id = idesc_tf32(64);
-          const uint32_t qb = smem_u32(sm + OFF_GQ);
-#pragma unroll
-          for (int s = 0; s < DH / 8; ++s)
-            mma_tf32_ts(tm + TM_O, tm + TM_S + 8 * s, sw128_desc(qb, C, s), id, s > 0);
-        }
-        // A | P: row block b against its R'_b (N = 32(b+1)), each over the two halves of
-        // the key channels into its own accumulator: four interleaved chains of 8 steps
-        if (!cwait(bar_opsap, ph_opsap[0])) break;
-        {
-          const uint32_t rp = smem_u32(sm);
-#pragma unroll
-          for (int s = 0; s < DH / 16; ++s) {
-#pragma unroll
-            for (int half = 0; half < 2; ++half)
-#pragma unroll
-              for (int b = 0; b < 2; ++b) {
-                const int ks = (DH / 16) * half + s;
-                mma_tf32_ts(tm + ap_col(b, half), tm + TM_L + 8 * ks,
-                            sw128_desc(rp + rp_off(b), 32 * (b + 1), ks), idesc_tf32(32 * (b + 1)),
-                            s > 0);
-              }
-          }
-          mma_commit(bar_ap);  // gamma*Q and the R'_b operands are free after this
-        }
-        // raw tiles consumed, V^T in TMEM, gamma*K in shared memory
-        if (!cwait(bar_raw, ph_raw)) break;
-        if (ci + 1 < n_chunks) issue_tma((ci + 1) * C);
-        {  // Y^T = V^T - S^T (gamma K)^T, while the workers solve T
-          const uint32_t idn = idesc_tf32(64, true);
-          const uint32_t kb = smem_u32(sm + OFF_GQ);
-#pragma unroll
-          for (int s = 0; s < DH / 8; ++s)
-            mma_tf32_ts(tm + TM_L, tm + TM_S + 8 * s, sw128_desc(kb, C, s), idn, true);
-          mma_commit(bar_y);
-        }
-        if (!cwait(bar_ops, ph_ops)) break;  // T Diag(beta) ready, S^T scaled by gamma_63
-        {  // U^T = Y^T (T Diag(beta))^T
-          const uint32_t id = idesc_tf32(64);
-          const uint32_t tb = smem_u32(sm + OFF_TB);
-#pragma unroll
-          for (int s = 0; s < C / 8; ++s)
-            mma_tf32_ts(tm + TM_X2, tm + TM_L + 8 * s, sw128_desc(tb, C, s), id, s > 0);
-          mma_commit(bar_u);
-        }
-        // U^T is the A operand of the last two products: wait for it to land
-        if (!cwait(bar_u, ph_u)) break;
-        {
-          const uint32_t id64 = idesc_tf32(64), id128 = idesc_tf32(128);
-          const uint32_t pb = smem_u32(sm + OFF_P), kb = smem_u32(sm + OFF_KHT);
-#pragma unroll
-          for (int s = 0; s < C / 8; ++s) {
-            mma_tf32_ts(tm + TM_O, tm + TM_X2 + 8 * s, sw128_desc(pb, C, s), id64, true);
-            mma_tf32_ts(tm + TM_S, tm + TM_X2 + 8 * s, sw128_desc(kb, DH, s), id128, true);
-          }
-          mma_commit(bar_mma);
-        }
+      if (n_chunks > 1) issue_tma(1);
+      if (n_chunks > 0) ok = prepare(0);
+      for (int n = 0; ok && n < n_chunks; ++n) {
+        if (!(ok = cwait(ops_sc, ph_sc))) break;
+        if (!(ok = cwait(bar_u, ph_u))) break;  // U^T is the A operand of the last products
+        mma_fin(n);
+        if (n + 1 < n_chunks) ok = prepare(n + 1);
       }
     }
   } else {
     // ======================= 16 worker warps =======================
-    uint32_t ph_tma = 0, ph_ap[1] = {0}, ph_y = 0, ph_mma = 0;
+    uint32_t ph_tma = 0u, ph_ap = 0, ph_oy = 0, ph_fin = 0;  // ph_tma: bit b for buffer b
+#ifdef KDA_PHASE_PROFILE
+    // thread 0's per-phase sums live in the spare bytes after the barriers
+    const bool prof = tid == 0;
+    unsigned long long *phase_acc = reinterpret_cast<unsigned long long *>(sm + OFF_BAR + 128);
+    if (prof)
+      for (int k = 0; k < 16; ++k) phase_acc[k] = 0ull;
+    long long phase_t = clock64();
+#endif
     auto wsync = [&]() { named_sync(1, NT); };
-    // every worker waits, then the workers synchronise so an abort is seen by all
+    // every worker waits, then all of them vote, so an abort is taken by all together
     auto wwait = [&](uint64_t *bar, uint32_t &ph) -> bool {
-      if (!(*s_abort == 0 && mbar_wait(bar, ph))) {
-        *s_abort = 1;
-        set_status(p.status, STATUS_TIMEOUT);
-      }
+      const bool got = mbar_wait(bar, ph, wait_ns, s_abort);
       ph ^= 1u;
-      wsync();
+      const bool bad = named_sync_or(1, NT, !got || *s_abort != 0);
+      if (bad) {
+        if (!got) set_status(p.status, STATUS_TIMEOUT);
+        *s_abort = 1;
+      }
       tc_fence_after();
-      return *s_abort == 0;
+      return !bad;
     };
     // one arrival per warp once all its lanes' writes are visible to the async proxy
     auto warp_arrive = [&](uint64_t *bar) {
@@ -340,324 +400,331 @@ __global__ void __launch_bounds__(NT + 32, 1)
       float v[32];
 #pragma unroll
       for (int j = 0; j < 32; ++j)
-        v[j] = p.local_mode ? ((part == 1 && 32 * g + j == l) ? 1.f : 0.f)
-                            : (s0 ? s0[(size_t)(32 * g + j) * DH + l] : 0.f);
-      tmem_st32(tm + lane + TM_S + 32 * g, v);
+        v[j] = p.local_mode ? ((part == 1 && 32 * cg + j == l) ? 1.f : 0.f)
+                            : (s0 ? s0[(size_t)(32 * cg + j) * DH + l] : 0.f);
+      tmem_st32(tm + lane_base + TM_S + 32 * cg, v);
       tmem_wait_st();
     }
+    // T Diag(beta) is lower triangular: its block above the diagonal stays zero
+    if (tid < 64)
+      *reinterpret_cast<float4 *>(sm + OFF_TB + sw128_chunk(C, tid >> 2, 16 + 4 * (tid & 3))) =
+          make_float4(0.f, 0.f, 0.f, 0.f);
 
-    // beta of the chunk about to start, loaded one chunk ahead (threads 0..63)
-    auto load_beta = [&](int c0) -> float {
+    // beta of chunk m, row tid (warp 0), loaded a chunk ahead
+    auto load_beta = [&](int m) -> float {
       float b = 0.f;
-      if (tid < C && c0 + tid < len) {
-        b = p.beta[(size_t)(bos + c0 + tid) * H + h];
+      const int t = m * C + tid;
+      if (tid < C && m < n_chunks && t < len) {
+        b = p.beta[(size_t)(bos + t) * H + h];
         if (p.validate && !(b >= 0.f && b <= 1.f)) set_status(p.status, STATUS_GATE_RANGE);
       }
       return b;
     };
-    float beta_next = load_beta(0);
-    // T Diag(beta) is lower triangular: its blocks above the diagonal stay zero, so they
-    // are written once here; the solve below stores every other element as it finalises it
-    for (int e = tid; e < C * C / 4; e += NT)
-      reinterpret_cast<float4 *>(sm + OFF_TB)[e] = make_float4(0.f, 0.f, 0.f, 0.f);
-    // Stage a chunk: its beta, wait for its tiles, cumulative gate, row operands
-    // (L* into TMEM, R into scratch, gamma*Q).  Chunk n+1 is staged while chunk n's
-    // last MMAs run.
-    auto stage = [&](int cs) -> bool {
-      const int c0 = cs * C;
-      const int n = min(C, len - c0);
-      if (tid < C) sB[tid] = beta_next;
-      if (!wwait(bar_tma, ph_tma)) return false;
-      beta_next = load_beta(c0 + C);
+    float beta_pref = load_beta(0);
 
-      // ---- a2: cumulative gate (thread = channel l, tokens 16g..16g+15) --------
-      // Every thread reads its raw gates before the first worker sync and writes the
-      // cumulative ones only after it, so the bf16 logits can share the region.
-      {
-        float gv[16];
-        if (logits) {
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int t = 16 * g + j;
-            gv[j] = (t < n) ? gate_from_logit(bf16_at(sm + OFF_GRAW, t, l)) : 0.f;
-          }
-        } else {
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int t = 16 * g + j;
-            gv[j] = (t < n) ? *reinterpret_cast<const float *>(sm + OFF_GRAW + g_off(t, l)) : 0.f;
-          }
-        }
-        if (p.validate && !logits)
-#pragma unroll
-          for (int j = 0; j < 16; ++j)
-            if (!(gv[j] >= kGateLower && gv[j] <= 0.f)) set_status(p.status, STATUS_GATE_RANGE);
-#pragma unroll
-        for (int j = 1; j < 16; ++j) gv[j] += gv[j - 1];
-        sSeg[g * DH + l] = gv[15];
-        wsync();
-        float off = 0.f;
-        for (int gg = 0; gg < g; ++gg) off += sSeg[gg * DH + l];
-#pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          gv[j] = (gv[j] + off) * LOG2E;
-          *reinterpret_cast<float *>(sm + OFF_GRAW + g_off(16 * g + j, l)) = gv[j];
-        }
-        sGr2[g * DH + l] = gv[15];
-        sEgr[g * DH + l] = ex2(gv[15]);
-        wsync();
-      }
-
-      // ---- a3 operands (thread = row i, channels 32g..32g+31) -----------------
-      // L*_i = x_i exp(G_i - G_m) with m = 32 b + 15 the reference row of i's 32-row block
-      // (x = k or q) goes to TMEM; K side: k_i to fp32 scratch (for R'_b); Q side:
-      // gamma*Q = L* exp(G_m) to its B operand.
-      const bool kside = l < C;
-      const int i = l & (C - 1);
-      const int bi = 2 * (i >> 5);  // the 16-row group ending at the reference row of i's block
-      const bool valid = i < n && (kside || load_q);
-      float *Rs = reinterpret_cast<float *>(sm + OFF_R);  // [64][LDR] fp32 scratch
-      {
-        const unsigned char *xraw = sm + (kside ? OFF_KRAW : OFF_QRAW);
-        const int rb = 16 * bi + 15;
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          float Lv[16];
-#pragma unroll
-          for (int c4 = 0; c4 < 4; ++c4) {
-            const int c = 32 * g + 16 * half + 4 * c4;
-            const float4 gi = *reinterpret_cast<const float4 *>(sm + OFF_GRAW + g_off(i, c));
-            const float4 grb = *reinterpret_cast<const float4 *>(sm + OFF_GRAW + g_off(rb, c));
-            float x[4];
-            bf16_x4(xraw, i, c, x);
-            const float giv[4] = {gi.x, gi.y, gi.z, gi.w}, grv[4] = {grb.x, grb.y, grb.z, grb.w};
-            float lst[4];
-#pragma unroll
-            for (int e = 0; e < 4; ++e) {
-              if (!valid) x[e] = 0.f;
-              lst[e] = x[e] * ex2(giv[e] - grv[e]);
-              Lv[4 * c4 + e] = tf32_rna(lst[e]);
-            }
-            if (kside) {  // k itself: R'_b takes its block factor in one exponential
-              *reinterpret_cast<float4 *>(&Rs[i * LDR + c]) = make_float4(x[0], x[1], x[2], x[3]);
-            } else {
-              const float4 eg = *reinterpret_cast<const float4 *>(&sEgr[bi * DH + c]);
-              *reinterpret_cast<float4 *>(sm + OFF_GQ + sw128_chunk(C, i, c)) =
-                  make_float4(tf32_rna(lst[0] * eg.x), tf32_rna(lst[1] * eg.y),
-                              tf32_rna(lst[2] * eg.z), tf32_rna(lst[3] * eg.w));
-            }
-          }
-          tmem_st16(tm + lane + TM_L + 32 * g + 16 * half, Lv);
-        }
-      }
-      return true;
+    // ---- gate(m): cumulative gate (thread = channel l, tokens 8 cg .. 8 cg + 7) ----
+    auto wait_tma = [&](int m) -> bool {
+      uint32_t ph = (ph_tma >> (m & 1)) & 1u;
+      const bool got = wwait(bar_tma + (m & 1), ph);
+      ph_tma ^= 1u << (m & 1);
+      return got;
     };
-    bool ok = n_chunks > 0 ? stage(0) : true;
-    for (int ci = 0; ci < n_chunks && ok; ++ci) {
-      const int c0 = ci * C;
-      const int n = min(C, len - c0);
-      const bool kside = l < C;
-      const int i = l & (C - 1);
-      float *Rs = reinterpret_cast<float *>(sm + OFF_R);  // [64][LDR] fp32 scratch
-      warp_arrive(bar_st);  // gamma*Q built, the previous chunk's O^T read: -> O^T
-      // thread = channel l, tokens 16g..16g+15: V^T and gamma*K (kept in registers until
-      // L* and gamma*Q are free), Khat^T = k exp(G_63 - G) straight to its B operand
-      uint32_t vT2[8];
-      float gkT[16];
-      {
-        const float G63 = *reinterpret_cast<const float *>(sm + OFF_GRAW + g_off(C - 1, l));
-        float kh[16];
+    auto w_gate = [&](int m) {
+      const int nr = min(C, len - m * C);
+      const unsigned char *raw = sm + OFF_RAW + (m & 1) * RAW_BYTES;
+      if (tid < C) BT[tid] = beta_pref;
+      beta_pref = load_beta(m + 1);
+      float gv[8];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int t = 16 * g + j;
-          const float G2 = *reinterpret_cast<const float *>(sm + OFF_GRAW + g_off(t, l));
-          const uint32_t vb = (t < n && !zero_v) ? (uint32_t)*reinterpret_cast<const unsigned short *>(
-                                            sm + OFF_VRAW + bf16_off(t, l))
-                                      : 0u;
-          if (j & 1) vT2[j >> 1] |= vb << 16; else vT2[j >> 1] = vb;
-          const float kk = (t < n) ? bf16_at(sm + OFF_KRAW, t, l) : 0.f;
-          gkT[j] = tf32_rna(kk * ex2(G2));
-          kh[j] = tf32_rna(kk * ex2(G63 - G2));
-        }
-#pragma unroll
-        for (int m4 = 0; m4 < 4; ++m4)
-          *reinterpret_cast<float4 *>(sm + OFF_KHT + sw128_chunk(DH, l, 16 * g + 4 * m4)) =
-              make_float4(kh[4 * m4], kh[4 * m4 + 1], kh[4 * m4 + 2], kh[4 * m4 + 3]);
-      }
-      wsync();  // every raw tile read: the raw region now takes the R'_b operands
-      // R'_b row j = k_j exp(G_mb - G_j) for the rows j of blocks up to b, m_b = 32 b + 15
-      // (the 16-row group end 2b of the G table), spread over all workers.  One exponential
-      // of the exponent difference: a factor underflows only where the true factor is
-      // below FLT_MIN, and then its product with an L* factor (<= exp(75)) is < exp(-12).
-#pragma unroll
-      for (int b = 0; b < 2; ++b) {
-        const int rows = 32 * (b + 1);
-        for (int it = tid; it < rows * 32; it += NT) {
-          const int j = it >> 5, c = (it & 31) * 4;
-          const float4 kv = *reinterpret_cast<const float4 *>(&Rs[j * LDR + c]);
-          const float4 gj = *reinterpret_cast<const float4 *>(sm + OFF_GRAW + g_off(j, c));
-          const float4 gm = *reinterpret_cast<const float4 *>(&sGr2[(2 * b) * DH + c]);
-          *reinterpret_cast<float4 *>(sm + rp_off(b) + sw128_chunk(rows, j, c)) =
-              make_float4(tf32_rna(kv.x * ex2(gm.x - gj.x)), tf32_rna(kv.y * ex2(gm.y - gj.y)),
-                          tf32_rna(kv.z * ex2(gm.z - gj.z)), tf32_rna(kv.w * ex2(gm.w - gj.w)));
-        }
-      }
-      tmem_wait_st();
-      warp_arrive(bar_opsap);  // -> A|P MMAs
-      if (!(ok = wwait(bar_ap, ph_ap[0]))) break;
-      {
-        float vT[16];
-#pragma unroll
-        for (int j = 0; j < 16; ++j)
-          vT[j] = __uint_as_float((j & 1) ? (vT2[j >> 1] & 0xFFFF0000u) : (vT2[j >> 1] << 16));
-        tmem_st16(tm + lane + TM_L + 16 * g, vT);  // L* is dead: V^T starts Y^T
-      }
-      // gamma*Q has been read by the O^T product: its tile takes gamma*K (rows = tokens)
-#pragma unroll
-      for (int j = 0; j < 16; ++j)
-        *reinterpret_cast<float *>(sm + OFF_GQ + sw128_offset(C, 16 * g + j, l)) = gkT[j];
-      tmem_wait_st();
-      warp_arrive(bar_raw);  // R'_b consumed (next TMA may start); V^T and gamma*K ready
-
-      // ---- a4: T = (I + Diag(beta) A)^-1 (blocked, fp32), P operand ------------
-      float *Ms = reinterpret_cast<float *>(sm + OFF_MS);
-      float *Ti = reinterpret_cast<float *>(sm + OFF_TI);
-      float *Ys = reinterpret_cast<float *>(sm + OFF_Y);
-      // element (r, c) of T Diag(beta), the B operand of U^T, once T_rc is final
-      auto put_tb = [&](int r, int c, float t) {
-        *reinterpret_cast<float *>(sm + OFF_TB + sw128_offset(C, r, c)) = tf32_rna(t * sB[c]);
-      };
-      {
-        // this warp's 32 rows are one row block: the sum of its two accumulators (columns
-        // past the block's width belong to other accumulators and are masked below)
-        const int blk = warp & 1;
-        float a[16], a_hi[16];
-        tmem_ld16(tm + lane + ap_col(blk, 0) + 16 * g, a);
-        tmem_ld16(tm + lane + ap_col(blk, 1) + 16 * g, a_hi);
-        tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 16; ++j) a[j] += a_hi[j];
-        if (kside) {
-          const float bi_ = sB[i];
-#pragma unroll
-          for (int j = 0; j < 16; ++j) {
-            const int c = 16 * g + j;
-            Ms[rot(i, c)] = (c < i) ? bi_ * a[j] : 0.f;
-          }
-        } else {
-#pragma unroll
-          for (int j = 0; j < 16; j += 4) {
-            const int c = 16 * g + j;
-            *reinterpret_cast<float4 *>(sm + OFF_P + sw128_chunk(C, i, c)) =
-                make_float4(c + 0 <= i ? tf32_rna(a[j]) : 0.f, c + 1 <= i ? tf32_rna(a[j + 1]) : 0.f,
-                            c + 2 <= i ? tf32_rna(a[j + 2]) : 0.f,
-                            c + 3 <= i ? tf32_rna(a[j + 3]) : 0.f);
+      for (int j = 0; j < 8; ++j) {
+        const int t = 8 * cg + j;
+        float x = 0.f;
+        if (t < nr) {
+          if (LOGITS) {
+            x = gate_from_logit(bf16_at(raw + R_G, t, l));
+          } else {
+            x = *reinterpret_cast<const float *>(raw + R_G + f32_off(t, l));
+            if (p.validate && !(x >= kGateLower && x <= 0.f)) set_status(p.status, STATUS_GATE_RANGE);
           }
         }
+        gv[j] = x;
+      }
+#pragma unroll
+      for (int j = 1; j < 8; ++j) gv[j] += gv[j - 1];
+      SEG[cg * DH + l] = gv[7];
+      wsync();
+      float off = 0.f;
+      for (int gg = 0; gg < cg; ++gg) off += SEG[gg * DH + l];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const float g2 = (gv[j] + off) * LOG2E;
+        GT[(8 * cg + j) * LDG + l] = g2;
+        if (cg == 3 && j == 7) GC[(m & 1) * DH + l] = ex2(g2);
       }
       wsync();
-      // diagonal 32x32 blocks: forward substitution, x_k = [k == j] - sum_{q<k} N_kq x_q for
-      // column j.  Warp w takes block w / 8 and its columns w % 8 + 8 c (c < 4) as four
-      // chains over the same rows, so the one value N_kq of a step (lane k) feeds all four
-      // and the chains' shuffles overlap; the next step's N_kq is loaded a step ahead.
-      {
-        const int o = 32 * (warp >> 3), k = lane_id;
-        int jj[4];
-        float x[4];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          jj[c] = (warp & 7) + 8 * c;
-          x[c] = (k == jj[c]) ? 1.f : 0.f;
-        }
-        float m_next = Ms[rot(o + k, o)];
-#pragma unroll
-        for (int q = 0; q < 31; ++q) {
-          const float m = m_next;
-          if (q < 30) m_next = Ms[rot(o + k, o + q + 1)];
-#pragma unroll
-          for (int c = 0; c < 4; ++c) {
-            const float xq = __shfl_sync(0xffffffffu, x[c], q);
-            if (q >= jj[c] && k > q) x[c] -= m * xq;
-          }
-        }
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const float t = (k >= jj[c]) ? x[c] : 0.f;
-          Ti[rot(o + k, o + jj[c])] = t;
-          put_tb(o + k, o + jj[c], t);
-        }
-      }
-      wsync();
-      // 32 -> 64: T[32:64, 0:32] = -T[32:64, 32:64] (N[32:64, 0:32] T[0:32, 0:32]);
-      // two outputs per thread, each summed in two halves to shorten the FMA chains
-      {
-        const int ii = tid >> 4, j0 = tid & 15;  // rows ii, columns j0 and j0 + 16
-        float y0a = 0.f, y0b = 0.f, y1a = 0.f, y1b = 0.f;
-#pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          const float na = Ms[rot(32 + ii, q)], nb = Ms[rot(32 + ii, q + 16)];
-          if (q >= j0) y0a += na * Ti[rot(q, j0)];
-          y0b += nb * Ti[rot(q + 16, j0)];
-          y1b += (q >= j0) ? nb * Ti[rot(q + 16, j0 + 16)] : 0.f;
-          (void)y1a;
-        }
-        Ys[ii * 33 + j0] = y0a + y0b;
-        Ys[ii * 33 + j0 + 16] = y1b;
-        wsync();
-        float t0a = 0.f, t0b = 0.f, t1a = 0.f, t1b = 0.f;
-#pragma unroll
-        for (int q = 0; q < 16; ++q) {
-          if (q <= ii) {
-            const float tv = Ti[rot(32 + ii, 32 + q)];
-            t0a += tv * Ys[q * 33 + j0];
-            t1a += tv * Ys[q * 33 + j0 + 16];
-          }
-          if (q + 16 <= ii) {
-            const float tv = Ti[rot(32 + ii, 48 + q)];
-            t0b += tv * Ys[(q + 16) * 33 + j0];
-            t1b += tv * Ys[(q + 16) * 33 + j0 + 16];
-          }
-        }
-        put_tb(32 + ii, j0, -(t0a + t0b));
-        put_tb(32 + ii, j0 + 16, -(t1a + t1b));
-      }
-      // ---- S^T <- S^T Diag(gamma_63) once the O^T and Y^T products have read S^T ----
-      if (!(ok = wwait(bar_y, ph_y))) break;
-      {
-        float v[32];
-        tmem_ld32(tm + lane + TM_S + 32 * g, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 32; ++j) v[j] *= sEgr[3 * DH + 32 * g + j];
-        tmem_st32(tm + lane + TM_S + 32 * g, v);
-        tmem_wait_st();
-      }
-      warp_arrive(bar_ops);  // -> U^T, then O^T += U^T P^T, S^T += U^T Khat
-      if (ci + 1 < n_chunks && !(ok = stage(ci + 1))) break;  // overlaps those MMAs
-      if (!(ok = wwait(bar_mma, ph_mma))) break;
+    };
 
-      // ---- a6: outputs (lane = value channel, tokens 16g..) and snapshots -------
+    // ---- scale(n): S^T <- S^T Diag(gamma_31) once the O^T and Y^T products read S^T ----
+    auto w_scale = [&](int n) {
+      float v[32];
+      tmem_ld32(tm + lane_base + TM_S + 32 * cg, v);
+      tmem_wait_ld();
+      const float *gc = GC + (n & 1) * DH + 32 * cg;
+#pragma unroll
+      for (int j = 0; j < 32; j += 8) {
+        float f[8];
+        ld8f(gc + j, f);
+#pragma unroll
+        for (int e = 0; e < 8; ++e) v[j + e] *= f[e];
+      }
+      tmem_st32(tm + lane_base + TM_S + 32 * cg, v);
+      tmem_wait_st();
+      warp_arrive(ops_sc);
+    };
+
+    // ---- rows(m): the row operands (thread = row i, channels 32 cg .. 32 cg + 31) ----
+    // lane quarter 0: L_k = k exp(G_i - G_15) -> TMEM lanes 0-31
+    // lane quarter 1: L_q = q exp(G_i - G_15) -> TMEM lanes 32-63
+    // lane quarter 2: R'  = k exp(G_15 - G_i) -> smem
+    // lane quarter 3: gamma*K, gamma*Q = (k, q) exp(G_i)  -> smem
+    auto w_rows = [&](int m) {
+      const int nr = min(C, len - m * C);
+      const unsigned char *raw = sm + OFF_RAW + (m & 1) * RAW_BYTES;
+      const int i = lane_id;
+      const bool valid = i < nr;
+      const float *gi = GT + i * LDG + 32 * cg;
+      const float *gm = GT + MREF * LDG + 32 * cg;
+      const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
+      if (qd <= 1) {
+        if (qd == 0 || has_q) {
+          const unsigned char *xr = raw + (qd == 0 ? R_K : R_Q);
+#pragma unroll
+          for (int jj = 0; jj < 4; ++jj) {
+            const int c = 32 * cg + 8 * jj;
+            float x[8], g[8], gr[8], lv[8];
+            bf16_x8(valid ? *reinterpret_cast<const uint4 *>(xr + bf16_chunk(i, c)) : z4, x);
+            ld8f(gi + 8 * jj, g);
+            ld8f(gm + 8 * jj, gr);
+#pragma unroll
+            for (int e = 0; e < 8; ++e) lv[e] = tf32_rna(x[e] * ex2(g[e] - gr[e]));
+            tmem_st8(tm + lane_base + TM_L + c, lv);
+          }
+          tmem_wait_st();
+        }
+      } else if (qd == 2) {
+        unsigned char *rp = sm + OFF_RP;
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          const int c = 32 * cg + 8 * jj;
+          float x[8], g[8], gr[8];
+          bf16_x8(valid ? *reinterpret_cast<const uint4 *>(raw + R_K + bf16_chunk(i, c)) : z4, x);
+          ld8f(gi + 8 * jj, g);
+          ld8f(gm + 8 * jj, gr);
+          float y[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) y[e] = tf32_rna(x[e] * ex2(gr[e] - g[e]));
+          *reinterpret_cast<float4 *>(rp + sw128_chunk(C, i, c)) = make_float4(y[0], y[1], y[2], y[3]);
+          *reinterpret_cast<float4 *>(rp + sw128_chunk(C, i, c + 4)) = make_float4(y[4], y[5], y[6], y[7]);
+        }
+      } else {
+        unsigned char *gk = sm + OFF_GK, *gq = sm + OFF_GQ;
+#pragma unroll
+        for (int jj = 0; jj < 4; ++jj) {
+          const int c = 32 * cg + 8 * jj;
+          float xk[8], xq[8], g[8];
+          bf16_x8(valid ? *reinterpret_cast<const uint4 *>(raw + R_K + bf16_chunk(i, c)) : z4, xk);
+          bf16_x8(valid && has_q ? *reinterpret_cast<const uint4 *>(raw + R_Q + bf16_chunk(i, c)) : z4, xq);
+          ld8f(gi + 8 * jj, g);
+          float yk[8], yq[8];
+#pragma unroll
+          for (int e = 0; e < 8; ++e) {
+            const float gam = ex2(g[e]);
+            yk[e] = tf32_rna(xk[e] * gam);
+            yq[e] = tf32_rna(xq[e] * gam);
+          }
+          *reinterpret_cast<float4 *>(gk + sw128_chunk(C, i, c)) = make_float4(yk[0], yk[1], yk[2], yk[3]);
+          *reinterpret_cast<float4 *>(gk + sw128_chunk(C, i, c + 4)) = make_float4(yk[4], yk[5], yk[6], yk[7]);
+          if (has_q) {
+            *reinterpret_cast<float4 *>(gq + sw128_chunk(C, i, c)) = make_float4(yq[0], yq[1], yq[2], yq[3]);
+            *reinterpret_cast<float4 *>(gq + sw128_chunk(C, i, c + 4)) = make_float4(yq[4], yq[5], yq[6], yq[7]);
+          }
+        }
+      }
+      warp_arrive(ops_ap);
+    };
+
+    // ---- khat(m): Khat^T = (k exp(G_31 - G))^T (thread = row i, channels 8 warp ..) ----
+    auto w_khat = [&](int m) {
+      const int nr = min(C, len - m * C);
+      const unsigned char *raw = sm + OFF_RAW + (m & 1) * RAW_BYTES;
+      const int i = lane_id, c = 8 * warp;
+      float x[8], g[8], ge[8];
+      bf16_x8(i < nr ? *reinterpret_cast<const uint4 *>(raw + R_K + bf16_chunk(i, c))
+                     : make_uint4(0u, 0u, 0u, 0u),
+              x);
+      ld8f(GT + i * LDG + c, g);
+      ld8f(GT + (C - 1) * LDG + c, ge);
+#pragma unroll
+      for (int e = 0; e < 8; ++e)
+        *reinterpret_cast<float *>(sm + OFF_KH + sw128_offset(DH, c + e, i)) =
+            tf32_rna(x[e] * ex2(ge[e] - g[e]));
+    };
+
+    // ---- out(n): O^T -> o (lane = value channel, tokens 8 cg ..), snapshot ----
+    auto w_out = [&](int n) {
+      const int c0 = n * C, nr = min(C, len - c0);
       if (go) {
-        float o[16];
-        tmem_ld16(tm + lane + TM_O + 16 * g, o);
+        float o8[8];
+        tmem_ld8(tm + lane_base + TM_O + 8 * cg, o8);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int t = 16 * g + j;
-          if (t < n) store_elem(go, ((size_t)(bos + c0 + t) * H + h) * DH + l, o[j]);
+        for (int j = 0; j < 8; ++j) {
+          const int t = 8 * cg + j;
+          if (t < nr) store_elem(go, ((size_t)(bos + c0 + t) * H + h) * DH + l, o8[j]);
         }
       }
-      if (snaps_ok && n == C && (c0 + C) % p.snapshot_stride == 0) {
+      if (snaps_ok && nr == C && (c0 + C) % p.snapshot_stride == 0) {
         const size_t row = (size_t)p.cu_snapshots[r] + (c0 + C) / p.snapshot_stride - 1;
         float *dst = p.snapshots + (row * H + h) * (size_t)DH * DH;
         float v[32];
-        tmem_ld32(tm + lane + TM_S + 32 * g, v);
+        tmem_ld32(tm + lane_base + TM_S + 32 * cg, v);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) dst[(size_t)(32 * g + j) * DH + l] = v[j];
+        for (int j = 0; j < 32; ++j) dst[(size_t)(32 * cg + j) * DH + l] = v[j];
       }
-      tc_fence_before();
-      wsync();
+    };
+
+    // ---- read(m): Diag(beta) A and P out of TMEM (after the A|P products), V^T into TMEM ----
+    auto w_read = [&](int m) {
+      const int nr = min(C, len - m * C);
+      const unsigned char *raw = sm + OFF_RAW + (m & 1) * RAW_BYTES;
+      const int i = lane_id;
+      if (qd == 0) {  // row i of A, columns 8 cg ..: N = beta_i A_ij for j < i
+        float a8[8];
+        tmem_ld8(tm + lane_base + TM_AP + 8 * cg, a8);
+        tmem_wait_ld();
+        const float bi = BT[i];
+        float n8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) n8[e] = (8 * cg + e < i) ? bi * a8[e] : 0.f;
+        float4 *dst = reinterpret_cast<float4 *>(NS + i * LDN + 8 * cg);
+        dst[0] = make_float4(n8[0], n8[1], n8[2], n8[3]);
+        dst[1] = make_float4(n8[4], n8[5], n8[6], n8[7]);
+      } else if (qd == 1 && has_q) {  // row i of P, inclusive lower, tf32 B operand
+        float a8[8];
+        tmem_ld8(tm + lane_base + TM_AP + 8 * cg, a8);
+        tmem_wait_ld();
+        float p8[8];
+#pragma unroll
+        for (int e = 0; e < 8; ++e) p8[e] = (8 * cg + e <= i) ? tf32_rna(a8[e]) : 0.f;
+        *reinterpret_cast<float4 *>(sm + OFF_PP + sw128_chunk(C, i, 8 * cg)) =
+            make_float4(p8[0], p8[1], p8[2], p8[3]);
+        *reinterpret_cast<float4 *>(sm + OFF_PP + sw128_chunk(C, i, 8 * cg + 4)) =
+            make_float4(p8[4], p8[5], p8[6], p8[7]);
+      }
+      float v8[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int t = 8 * cg + j;
+        v8[j] = (t < nr && !zero_v) ? bf16_at(raw + R_V, t, l) : 0.f;
+      }
+      tmem_st8(tm + lane_base + TM_Y + 8 * cg, v8);
+      tmem_wait_st();
+      warp_arrive(raw_free);
+      warp_arrive(ops_oy);
+    };
+
+    // ---- solve(m): T = (I + Diag(beta) A)^-1 by 16 x 16 blocks, then T Diag(beta) ----
+    auto w_solve = [&]() {
+      wsync();  // Diag(beta) A complete
+      if (warp == 2) {
+        // the two diagonal blocks, row by row: t_i = e_i - sum_{j<i} N_ij t_j, one
+        // column per lane (lanes 0-15: block 0, lanes 16-31: block 1)
+        const int o = 16 * (lane_id >> 4), c = lane_id & 15;
+        float t[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const float4 *nrow = reinterpret_cast<const float4 *>(NS + (o + i) * LDN + o);
+          float acc = (i == c) ? 1.f : 0.f;
+#pragma unroll
+          for (int j4 = 0; 4 * j4 < i; ++j4) {
+            const float4 n4 = nrow[j4];
+            const float nv[4] = {n4.x, n4.y, n4.z, n4.w};
+#pragma unroll
+            for (int e = 0; e < 4; ++e)
+              if (4 * j4 + e < i) acc -= nv[e] * t[4 * j4 + e];
+          }
+          t[i] = acc;
+        }
+        const float bc = BT[o + c];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          TS[(o + i) * LDN + o + c] = t[i];
+          *reinterpret_cast<float *>(sm + OFF_TB + sw128_offset(C, o + i, o + c)) =
+              tf32_rna(t[i] * bc);
+        }
+      }
+      wsync();  // diagonal blocks ready
+      if (warp >= 8) {  // T10 = -T11 (N10 T00): one element (i, c) per thread
+        const int tt = tid - 256, i = tt >> 4, c = tt & 15;
+        float x = 0.f;
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          if (j >= c) x += NS[(16 + i) * LDN + j] * TS[j * LDN + c];
+        XS[i * LDX + c] = x;
+        named_sync(2, 256);
+        float y = 0.f;
+#pragma unroll
+        for (int j = 0; j < 16; ++j)
+          if (j <= i) y += TS[(16 + i) * LDN + 16 + j] * XS[j * LDX + c];
+        *reinterpret_cast<float *>(sm + OFF_TB + sw128_offset(C, 16 + i, c)) =
+            tf32_rna(-y * BT[c]);
+      }
+      warp_arrive(ops_tb);
+    };
+
+    // chunk 0's operands, then the pipelined loop (phase numbers: profiling builds)
+    bool ok = true;
+    if (n_chunks > 0) {
+      if ((ok = wait_tma(0))) {
+        w_gate(0);
+        w_rows(0);
+        w_khat(0);
+        if ((ok = wwait(bar_ap, ph_ap))) {
+          w_read(0);
+          w_solve();
+        }
+      }
+    }
+    KDA_PHASE(0);
+    for (int n = 0; ok && n < n_chunks; ++n) {
+      const bool more = n + 1 < n_chunks;
+      if (more) {
+        if (!(ok = wait_tma(n + 1))) break;
+        KDA_PHASE(1);
+        w_gate(n + 1);
+        KDA_PHASE(2);
+      }
+      if (!(ok = wwait(bar_oy, ph_oy))) break;
+      KDA_PHASE(3);
+      w_scale(n);
+      KDA_PHASE(4);
+      if (more) w_rows(n + 1);
+      KDA_PHASE(5);
+      if (!(ok = wwait(bar_fin, ph_fin))) break;
+      KDA_PHASE(6);
+      if (more) w_khat(n + 1);
+      KDA_PHASE(7);
+      w_out(n);
+      KDA_PHASE(8);
+      if (more) {
+        if (!(ok = wwait(bar_ap, ph_ap))) break;
+        KDA_PHASE(9);
+        w_read(n + 1);
+        KDA_PHASE(10);
+        w_solve();
+        KDA_PHASE(11);
+      }
     }
 
     float *fin = p.local_mode ? (part == 0 ? p.s_loc : p.m) : p.final_state;
@@ -665,25 +732,29 @@ __global__ void __launch_bounds__(NT + 32, 1)
       float *dst = fin + ((size_t)(r * H + h)) * DH * DH;
       tc_fence_after();
       float v[32];
-      tmem_ld32(tm + lane + TM_S + 32 * g, v);
+      tmem_ld32(tm + lane_base + TM_S + 32 * cg, v);
       tmem_wait_ld();
 #pragma unroll
-      for (int j = 0; j < 32; ++j) dst[(size_t)(32 * g + j) * DH + l] = v[j];
+      for (int j = 0; j < 32; ++j) dst[(size_t)(32 * cg + j) * DH + l] = v[j];
     }
+#ifdef KDA_PHASE_PROFILE
+    KDA_PHASE(12);
+    if (prof) {
+      for (int k = 0; k < 13; ++k) atomicAdd(&g_phase_cycles[k], phase_acc[k]);
+      atomicAdd(&g_phase_cycles[15], (unsigned long long)n_chunks);
+    }
+#endif
   }
 
   tc_fence_before();
   __syncthreads();
-  if (*s_abort && tid == 0) {
-    // the CTA gave up: give in-flight copies and MMAs a bounded chance to land
-    mbar_wait(bar_tma, 0, 100000000ull);
-    mbar_wait(bar_tma, 1, 100000000ull);
-    mbar_wait(bar_y, 0, 100000000ull);
-    mbar_wait(bar_y, 1, 100000000ull);
-    mbar_wait(bar_u, 0, 100000000ull);
-    mbar_wait(bar_u, 1, 100000000ull);
-    mbar_wait(bar_mma, 0, 100000000ull);
-    mbar_wait(bar_mma, 1, 100000000ull);
+  if (*s_abort && control && lane_id == 0) {
+    // the CTA gave up: let the copies and products it issued land before it releases
+    // its shared and tensor memory (at most one load per buffer and, the products
+    // completing in order, the last commit are outstanding)
+    if (tma_n0) mbar_wait(bar_tma, (tma_n0 - 1u) & 1u, 100000000ull);
+    if (tma_n1) mbar_wait(bar_tma + 1, (tma_n1 - 1u) & 1u, 100000000ull);
+    if (last_bar) mbar_wait(last_bar, last_par, 100000000ull);
   }
   __syncthreads();
   if (warp == 0) {
@@ -712,13 +783,15 @@ EncodeTiledFn encode_tiled_fn() {
   return fn;
 }
 
+// A [rows, inner] row-major tensor read as boxes of [C rows, box_inner elements]
+// (box_inner * esize = 128 bytes, the swizzle span); rows past the end read as zero.
 bool encode_map(CUtensorMap *m, const void *ptr, CUtensorMapDataType dt, uint64_t esize,
                 uint64_t inner, uint64_t rows, uint32_t box_inner) {
   const EncodeTiledFn encode = encode_tiled_fn();
   if (!encode) return false;
   cuuint64_t dims[2] = {inner, rows};
   cuuint64_t strides[1] = {inner * esize};
-  cuuint32_t box[2] = {box_inner, 64};
+  cuuint32_t box[2] = {box_inner, (cuuint32_t)C};
   cuuint32_t es[2] = {1, 1};
   return encode(m, dt, 2, const_cast<void *>(ptr), dims, strides, box, es,
                 CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
@@ -760,3 +833,19 @@ cudaError_t launch_prefill_tc(const PrefillParams &p, kda_dtype in_dtype, kda_dt
 }
 
 }  // namespace kda
+
+#ifdef KDA_PHASE_PROFILE
+// Profiling builds only: copy (and optionally clear) the per-phase cycle sums of
+// the tensor-core prefill; entry 15 is the number of chunks they cover.
+extern "C" int kda_phase_cycles(unsigned long long *out, int n, int clear) {
+  if (n > 16) n = 16;
+  if (cudaMemcpyFromSymbol(out, kda::g_phase_cycles, n * sizeof(unsigned long long)) !=
+      cudaSuccess)
+    return 1;
+  if (clear) {
+    const unsigned long long zero[16] = {};
+    if (cudaMemcpyToSymbol(kda::g_phase_cycles, zero, sizeof(zero)) != cudaSuccess) return 1;
+  }
+  return 0;
+}
+#endif

@@ -147,6 +147,24 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float *v) {
       : "memory");
 }
 
+// 32 lanes x 8 columns.
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, float *v) {
+  uint32_t *r = reinterpret_cast<uint32_t *>(v);
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]),
+        "=r"(r[7])
+      : "r"(taddr));
+}
+__device__ __forceinline__ void tmem_st8(uint32_t taddr, const float *v) {
+  const uint32_t *r = reinterpret_cast<const uint32_t *>(v);
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(
+          taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
+      : "memory");
+}
+
 // 2^x on the special-function unit (ex2.approx, flush-to-zero; relative error
 // about 2^-22 over the range used here).
 __device__ __forceinline__ float ex2(float x) {
@@ -205,27 +223,34 @@ __device__ __forceinline__ uint64_t global_ns() {
   asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t));
   return t;
 }
-// try_wait that lets the hardware suspend the thread (up to ~20 us) until the
-// phase completes, so waiting warps do not take issue slots from working ones.
-__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t *bar, uint32_t parity) {
+// try_wait that lets the hardware suspend the thread (up to hint_ns, at most
+// ~20 us here) until the phase completes, so waiting warps do not take issue
+// slots from working ones.
+__device__ __forceinline__ bool mbar_try_wait_suspend(uint64_t *bar, uint32_t parity,
+                                                      uint32_t hint_ns = 20000u) {
   uint32_t ok;
   asm volatile(
       "{\n\t.reg .pred p;\n\t"
       "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n\t"
       "selp.u32 %0, 1, 0, p;\n\t}"
       : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity), "r"(20000u)
+      : "r"(smem_u32(bar)), "r"(parity), "r"(hint_ns)
       : "memory");
   return ok != 0;
 }
 // Wait for the phase with the given parity to complete; gives up after
-// timeout_ns and returns false (the caller reports KDA_ERR_TIMEOUT).
+// timeout_ns and returns false (the caller reports KDA_ERR_TIMEOUT).  The
+// suspend hint never exceeds the limit, so a short limit does run out.  When
+// `abort_flag` is given, the wait also gives up as soon as it reads non-zero.
 __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
-                                          uint64_t timeout_ns = 2000000000ull) {
+                                          uint64_t timeout_ns = 2000000000ull,
+                                          const volatile int *abort_flag = nullptr) {
   if (mbar_try_wait(bar, parity)) return true;
+  const uint32_t hint = timeout_ns < 20000ull ? (uint32_t)timeout_ns : 20000u;
   const uint64_t t0 = global_ns();
   for (;;) {
-    if (mbar_try_wait_suspend(bar, parity)) return true;
+    if (mbar_try_wait_suspend(bar, parity, hint)) return true;
+    if (abort_flag && *abort_flag) return false;
     if (global_ns() - t0 > timeout_ns) return false;
   }
 }
@@ -238,6 +263,21 @@ __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
 // Named barrier over the first `count` threads (a multiple of 32).
 __device__ __forceinline__ void named_sync(uint32_t id, uint32_t count) {
   asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(count) : "memory");
+}
+
+// Named barrier over the first `count` threads that also returns the OR of
+// every participant's predicate, so all of them take the same branch after it.
+__device__ __forceinline__ bool named_sync_or(uint32_t id, uint32_t count, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n\t.reg .pred p, q;\n\t"
+      "setp.ne.u32 p, %1, 0;\n\t"
+      "bar.red.or.pred q, %2, %3, p;\n\t"
+      "selp.u32 %0, 1, 0, q;\n\t}"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(count)
+      : "memory");
+  return r != 0;
 }
 
 // Make generic-proxy shared-memory writes visible to the async proxy (MMA, TMA).

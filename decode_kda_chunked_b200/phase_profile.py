@@ -1,0 +1,66 @@
+"""Per-phase cycle profile of the tensor-core chunked prefill.
+
+    python -m decode_kda_chunked_b200.phase_profile [--requests N] [--steps K]
+
+Builds the diagnostic library libkda_phase.so (the same sources compiled with
+KDA_PHASE_PROFILE: worker thread 0 of every CTA reads clock64 at each step of the
+chunk loop), runs the varlen prefill workload (64 requests, lengths log-uniform on
+[128, 4096], H=32, d=128, bf16 q/k/v, fp32 g, beta and o) through it, and prints
+the mean cycles per 32-token chunk of each step with its share.  The counters
+perturb the timing slightly; the table shows where a chunk's time goes, the
+bench measures how long it takes.  Needs a CUDA device.
+"""
+from __future__ import annotations
+
+import argparse
+import ctypes
+import json
+
+PHASES = ("chunk 0 operands", "wait: next tiles", "gate (cumulative)", "wait: O^T, Y^T",
+          "scale S^T", "rows (L, R', gamma Q/K)", "wait: last products", "Khat^T",
+          "out (o, snapshots)", "wait: A|P", "read (A, P, V^T)", "solve (T Diag(beta))",
+          "final state")
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--requests", type=int, default=None, help="first N requests only")
+    ap.add_argument("--steps", type=int, default=3)
+    args = ap.parse_args()
+
+    import torch
+
+    from . import _lib, build
+    from . import inputs as I
+    path = build.build(phase_profile=True)
+    lib = _lib.load(path)
+    lib.kda_phase_cycles.restype = ctypes.c_int
+    lib.kda_phase_cycles.argtypes = [ctypes.POINTER(ctypes.c_ulonglong), ctypes.c_int, ctypes.c_int]
+    dev = torch.device("cuda", 0)
+    if args.requests is None:
+        x = I.varlen(device=dev)
+    else:
+        x = I.make_prefill_inputs(I.varlen_lengths(0)[:args.requests], H=32, dk=128, dv=128,
+                                  seed=0, device=dev)
+    from . import prefill
+    buf = (ctypes.c_ulonglong * 16)()
+    prefill(x.q, x.k, x.v, x.g, x.beta, x.cu_seqlens, cu_seqlens_host=x.cu_seqlens.cpu())
+    torch.cuda.synchronize()
+    assert lib.kda_phase_cycles(buf, 16, 1) == 0  # clear after the warm-up call
+    for _ in range(args.steps):
+        prefill(x.q, x.k, x.v, x.g, x.beta, x.cu_seqlens, cu_seqlens_host=x.cu_seqlens.cpu())
+    torch.cuda.synchronize()
+    assert lib.kda_phase_cycles(buf, 16, 0) == 0
+    chunks = buf[15]
+    total = sum(buf[k] for k in range(len(PHASES)))
+    rows = [{"phase": name, "cycles_per_chunk": buf[k] / chunks, "share": buf[k] / total}
+            for k, name in enumerate(PHASES)]
+    print(f"{chunks // args.steps} chunks of 32 tokens per call; "
+          f"{total / chunks:.0f} cycles per chunk (worker thread 0)")
+    for rw in rows:
+        print(f"  {rw['phase']:<28} {rw['cycles_per_chunk']:8.0f}  {100 * rw['share']:5.1f} %")
+    print(json.dumps({"cycles_per_chunk": total / chunks, "phases": rows}))
+
+
+if __name__ == "__main__":
+    main()

@@ -74,6 +74,17 @@ def test_ragged_varlen(d, dtype):
     check_all_chains(inp, out, 64, TOL_F32 if dtype == torch.float32 else TOL_BF16)
 
 
+RAGGED_32 = [31, 32, 33, 95, 96, 97, 160, 1, 0, 64]
+
+
+def test_ragged_around_32_token_chunks():
+    """The tensor-core kernel works in 32-token chunks: lengths one short of, at and
+    one past chunk ends, with snapshots every 64 tokens (every second chunk end)."""
+    inp = I.make_prefill_inputs(RAGGED_32, H=2, dk=128, dv=128, seed=8, s0_std=0.1)
+    out = run_prefill(inp, stride=64)
+    check_all_chains(inp, out, 64, TOL_BF16)
+
+
 def test_weak_decay_long_memory():
     """Weak gates keep long-range state alive, so errors carried across many
     chunks show up (the standard -5 sigmoid gates forget within a few tokens)."""
