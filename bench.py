@@ -436,6 +436,10 @@ def run_ours(args, world, rank, local):
         line["e2e"]["fused_gate"] = bench_e2e(args, xl, dev, world, gate_logits=True)
         line["e2e"]["fused_gate"]["workload"] = ("the same requests with bf16 gate logits in "
                                                  "place of fp32 g (fused gate activation)")
+        line["e2e"]["serving"] = bench_e2e(args, xl, dev, world, gate_logits=True,
+                                           out_dtype=torch.bfloat16)
+        line["e2e"]["serving"]["workload"] = ("serving-shaped copies: bf16 gate logits in, "
+                                              "bf16 o and fp32 final states out")
         del xl
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
         r = time_oracle(inp, sample_chains(inp.lengths, H))
@@ -696,15 +700,17 @@ def kcp_bytes(T: int, H: int, d: int, n_seg: int, stride: int = 512) -> int:
     return pass1 + pass2 + (T // stride) * H * d * d * 4
 
 
-def bench_e2e(args, inp, dev, world, gate_logits: bool = False):
+def bench_e2e(args, inp, dev, world, gate_logits: bool = False, out_dtype=None):
     """Same metric through the public entry point with host buffers: every step
     copies that step's inputs from pinned host memory and reads o and the final
     states back to pinned host memory inside the timed region.  Steps are double
     buffered on three streams, as a serving loop runs them: step k's inputs are
     copied in and step k-1's outputs copied out while step k-1 / k computes, so the
     time per step is set by the busier PCIe direction, not by the sum.  With
-    ``gate_logits`` the gate travels as bf16 logits (fused gate activation)."""
+    ``gate_logits`` the gate travels as bf16 logits (fused gate activation); with
+    ``out_dtype`` bfloat16, o is written and copied back in bf16."""
     import torch
+    out_dtype = out_dtype or torch.float32
 
     import decode_kda_chunked_b200 as kda
     T, H, dv, dk = inp.total_tokens, 32, 128, 128
@@ -712,7 +718,7 @@ def bench_e2e(args, inp, dev, world, gate_logits: bool = False):
     names = ("q", "k", "v", gname, "beta", "cu_seqlens")
     host = {n: getattr(inp, n).cpu().pin_memory() for n in names}
     devb = [{n: torch.empty_like(getattr(inp, n)) for n in names} for _ in range(2)]
-    o = [torch.empty(T, H, dv, device=dev) for _ in range(2)]
+    o = [torch.empty(T, H, dv, device=dev, dtype=out_dtype) for _ in range(2)]
     fin = [torch.empty(inp.n_req, H, dk, dv, device=dev) for _ in range(2)]
     o_h = [torch.empty(o[0].shape, dtype=o[0].dtype).pin_memory() for _ in range(2)]
     fin_h = [torch.empty(fin[0].shape, dtype=fin[0].dtype).pin_memory() for _ in range(2)]
@@ -725,7 +731,7 @@ def bench_e2e(args, inp, dev, world, gate_logits: bool = False):
     ws = [torch.empty(ws_bytes, dtype=torch.uint8, device=dev) for _ in range(2)]
     ev = {k: [torch.cuda.Event() for _ in range(2)] for k in ("in", "cmp", "out")}
     h2d = sum(t.numel() * t.element_size() for t in host.values())
-    d2h = o[0].numel() * 4 + fin[0].numel() * 4
+    d2h = o[0].numel() * o[0].element_size() + fin[0].numel() * 4
     steps = max(3, min(args.steps, 10))
 
     def step(k):

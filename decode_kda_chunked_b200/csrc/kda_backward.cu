@@ -298,8 +298,7 @@ __global__ void __launch_bounds__(NTH, 1) bwd_prep_kernel(const BwdParams p) {
   using L = PrepLayout<D>;
   constexpr int NJ = D / 16, LDP = L::LDP;
   extern __shared__ float4 smem_f4[];
-  float *sm = reinterpret_cast<float *>(
-      (reinterpret_cast<uintptr_t>(smem_f4) + 1023) & ~uintptr_t(1023));
+  float *sm = reinterpret_cast<float *>(align1024_shared(smem_f4));
   float *sK = sm + L::oK, *sQ = sm + L::oQ, *sG = sm + L::oG, *sA = sm + L::oA;
   float *sP = sm + L::oP, *sT = sm + L::oT, *sBuf = sm + L::oBuf, *sKL = sm + L::oKL;
   float *sQL = sm + L::oQL, *sStage = sm + L::oStage, *sB = sm + L::oB;
@@ -803,8 +802,7 @@ __global__ void __launch_bounds__(SP_NTH, 1) bwd_sprod_kernel(const BwdParams p)
   // S; dSn; d(gamma Q)^T
   constexpr uint32_t TST = 0, TDW = 0, TDK = 64, TU = 128, TS = 192, TDS = 320, TGQ = 448;
   extern __shared__ float4 smem_f4[];
-  float *sm = reinterpret_cast<float *>(
-      (reinterpret_cast<uintptr_t>(smem_f4) + 1023) & ~uintptr_t(1023));
+  float *sm = reinterpret_cast<float *>(align1024_shared(smem_f4));
   unsigned char *bW = reinterpret_cast<unsigned char *>(sm + L::oW);
   unsigned char *bO = reinterpret_cast<unsigned char *>(sm + L::oO);
   unsigned char *bDU = reinterpret_cast<unsigned char *>(sm + L::oDU);

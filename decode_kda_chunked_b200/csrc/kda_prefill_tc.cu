@@ -21,28 +21,32 @@
 // log alpha >= -5 (the lower-bounded decay of KDA, CSDN post on the Kimi K3 technical
 // report, section 一.1) every factor is a finite fp32 number; only masked products
 // (j > i) can overflow, and they are dropped by selection, never multiplied.
+// gamma_i = exp(G_i) is exp(G_i - G_15) exp(G_15), a product of two finite factors
+// that is flushed to zero only where the true value is below FLT_MIN.
 //
 // All tensor-core operands are tf32 (B operands K-major with the 128-byte swizzle in
 // shared memory, rounded to nearest): bf16 operands for the gate-scaled products
 // would cost about 2e-3 of relative accuracy, tf32 stays near 5e-4.
 //
-// Pipeline.  One CTA runs one (request, head) chain with 16 worker warps and one
-// control warp; the control warp issues every TMA load and tcgen05.mma, the workers
-// do the SIMT work, and they hand off through mbarriers.  Iteration n of the worker
-// loop finishes chunk n's state products while it prepares chunk n+1:
+// Warp roles.  One CTA runs one (request, head) chain: two control warps issue every
+// TMA load and tcgen05.mma, and two groups of 8 worker warps run side by side,
+// handing off through mbarriers (intra-chunk work in parallel with the state
+// passing, as the FlashKDA section of "Kimi K3 开源日来了" describes):
 //
-//   gate(n+1)  cumulative gate of chunk n+1              (raw tiles loaded long before)
-//   scale(n)   S^T *= gamma_31(n) once O^T, Y^T(n) read S^T   -> control: last products(n)
-//   rows(n+1)  L_k, L_q -> TMEM, R', gamma*Q, gamma*K -> smem  -> control: A|P(n+1)
-//   out(n)     after last products(n): Khat^T(n+1), O^T(n) -> o, snapshot(n)
-//   read(n+1)  after A|P(n+1): Diag(b) A, P, V^T(n+1) -> TMEM  -> control: O^T, Y^T(n+1)
-//   solve(n+1) T Diag(b)                                        -> control: U^T(n+1)
+//   group A (warps 0-7), chunk m:  gate(m): cumulative gate;  rows(m): L_k, L_q -> TMEM,
+//       R', gamma*Q, gamma*K -> smem  [-> A|P(m)];  read(m): Diag(b) A, P;
+//       solve(m): T Diag(b)  [-> U^T(m)]
+//   group B (warps 8-15), chunk n:  scale(n): S^T *= gamma_31 once O^T, Y^T(n) read S^T
+//       [-> last products(n)];  khat(n+1): Khat^T;  out(n): O^T -> o, snapshot;
+//       vt(n+1): V^T -> TMEM  [with group A's read(n+1): -> O^T, Y^T(n+1)]
 //
-// so every product runs while the workers do other work, and every buffer is
-// rewritten only after the product that reads it has completed.  Raw tiles are
-// double buffered: chunk m+2 is loaded as soon as chunk m's tiles are read.
-// Every wait is bounded; a wait that runs out ends the CTA with KDA_ERR_TIMEOUT in
-// the status word, after the CTA has let every copy and product it issued land.
+// so group A prepares chunk n+1 while group B finishes chunk n, and every product
+// runs while the workers do other work.  Khat^T, P and T Diag(b) are double
+// buffered by chunk parity, raw tiles too (chunk m+2 loads as soon as chunk m's
+// tiles are read); every other buffer is rewritten only after the product that
+// reads it has completed (group A starts chunk m after O^T, Y^T(m-1)).  Every wait
+// is bounded; a wait that runs out ends the CTA with KDA_ERR_TIMEOUT in the status
+// word, after the CTA has let every copy and product it issued land.
 #include "kda_internal.cuh"
 #include "kda_sm100.cuh"
 
@@ -54,6 +58,7 @@ using namespace sm100;
 constexpr int C = 32;     // tokens per chunk of this kernel
 constexpr int DH = 128;   // head dim (dk = dv)
 constexpr int NT = 512;   // worker threads per CTA: 16 warps (plus one control warp)
+constexpr int NA = 256;   // group A threads (warps 0-7); group B is warps 8-15
 constexpr int MREF = 15;  // reference row of the gate factorisation
 constexpr float LOG2E = 1.4426950408889634f;
 
@@ -68,33 +73,39 @@ constexpr uint32_t OFF_GT = 81920;   // log2(e) * G (chunk-local cumulative gate
 constexpr int LDG = 132;             // padded so that row-wise float4 reads hit distinct banks
 constexpr uint32_t OFF_GQ = 99328;   // gamma*Q  tf32 B operand [32 x 128]
 constexpr uint32_t OFF_GK = 115712;  // gamma*K  tf32 B operand [32 x 128]
-constexpr uint32_t OFF_KH = 132096;  // Khat^T   tf32 B operand [128 x 32]
-constexpr uint32_t OFF_RP = 148480;  // R'       tf32 B operand [32 x 128]
-constexpr uint32_t OFF_PP = 164864;  // P        tf32 B operand [32 x 32]
-constexpr uint32_t OFF_TB = 168960;  // T Diag(beta) tf32 B operand [32 x 32]
-constexpr uint32_t OFF_NS = 173056;  // Diag(beta) A, strict lower, fp32 [32][LDN]
+constexpr uint32_t OFF_KH = 132096;  // Khat^T   tf32 B operand [128 x 32], x2 (chunk parity)
+constexpr uint32_t OFF_RP = 164864;  // R'       tf32 B operand [32 x 128]
+constexpr uint32_t OFF_PP = 181248;  // P        tf32 B operand [32 x 32], x2
+constexpr uint32_t OFF_TB = 189440;  // T Diag(beta) tf32 B operand [32 x 32], x2
+constexpr uint32_t OFF_NS = 197632;  // Diag(beta) A, strict lower, fp32 [32][LDN]
 constexpr int LDN = 36;
-constexpr uint32_t OFF_TS = 177664;  // the two diagonal 16x16 blocks of T, fp32 [32][LDN]
-constexpr uint32_t OFF_XS = 182272;  // N10 T00, fp32 [16][LDX]
+constexpr uint32_t OFF_TS = 202240;  // the two diagonal 16x16 blocks of T, fp32 [32][LDN]
+constexpr uint32_t OFF_XS = 206848;  // N10 T00, fp32 [16][LDX]
 constexpr int LDX = 20;
-constexpr uint32_t OFF_GC = 183552;  // exp(G_31) per key channel, [2][128] by chunk parity
-constexpr uint32_t OFF_BT = 184576;  // beta of the chunk being prepared [32]
-constexpr uint32_t OFF_SEG = 184704; // cumulative-gate segment totals [4][128]
-constexpr uint32_t OFF_BAR = 186752; // mbarriers, TMEM base, flags
-constexpr uint32_t SMEM_BYTES = 187008;
+constexpr uint32_t OFF_GC = 208128;  // exp(G_31) per key channel, [2][128] (chunk parity)
+constexpr uint32_t OFF_E15 = 209152; // exp(G_15) per key channel [128]
+constexpr uint32_t OFF_BT = 209664;  // beta of the chunk group A prepares [32]
+constexpr uint32_t OFF_SEG = 209792; // cumulative-gate segment totals [2][128]
+constexpr uint32_t OFF_BAR = 210816; // mbarriers, TMEM base, flags (+ phase counters)
+constexpr uint32_t SMEM_BYTES = 211072;
 constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;  // alignment slack
 static_assert(OFF_RAW + 2 * RAW_BYTES <= OFF_GT, "raw buffers");
 static_assert(OFF_GT + C * LDG * 4 <= OFF_GQ, "gate table");
 static_assert(OFF_GQ % 1024 == 0 && OFF_GK % 1024 == 0 && OFF_KH % 1024 == 0 &&
                   OFF_RP % 1024 == 0 && OFF_PP % 1024 == 0 && OFF_TB % 1024 == 0,
               "swizzled operands need 1024-byte alignment");
-static_assert(OFF_GQ + 16384 == OFF_GK && OFF_GK + 16384 == OFF_KH && OFF_KH + 16384 == OFF_RP &&
-                  OFF_RP + 16384 == OFF_PP && OFF_PP + 4096 == OFF_TB && OFF_TB + 4096 == OFF_NS,
+static_assert(OFF_GQ + 16384 == OFF_GK && OFF_GK + 16384 == OFF_KH &&
+                  OFF_KH + 2 * 16384 == OFF_RP && OFF_RP + 16384 == OFF_PP &&
+                  OFF_PP + 2 * 4096 == OFF_TB && OFF_TB + 2 * 4096 == OFF_NS,
               "operand tiles");
 static_assert(OFF_NS + C * LDN * 4 == OFF_TS && OFF_TS + C * LDN * 4 == OFF_XS &&
-                  OFF_XS + 16 * LDX * 4 == OFF_GC && OFF_GC + 2 * DH * 4 == OFF_BT &&
-                  OFF_BT + C * 4 == OFF_SEG && OFF_SEG + 4 * DH * 4 == OFF_BAR,
+                  OFF_XS + 16 * LDX * 4 == OFF_GC && OFF_GC + 2 * DH * 4 == OFF_E15 &&
+                  OFF_E15 + DH * 4 == OFF_BT && OFF_BT + C * 4 == OFF_SEG &&
+                  OFF_SEG + 2 * DH * 4 == OFF_BAR,
               "scratch tiles");
+__host__ __device__ constexpr uint32_t kh_off(int m) { return OFF_KH + 16384u * (m & 1); }
+__host__ __device__ constexpr uint32_t pp_off(int m) { return OFF_PP + 4096u * (m & 1); }
+__host__ __device__ constexpr uint32_t tb_off(int m) { return OFF_TB + 4096u * (m & 1); }
 
 // ---- TMEM column map (512 columns x 128 lanes of fp32) ----
 constexpr uint32_t TM_S = 0;     // S^T (lane = value channel, col = key channel)
@@ -142,13 +153,19 @@ __device__ __forceinline__ void ld8f(const float *p, float *x) {
   const float4 b = reinterpret_cast<const float4 *>(p)[1];
   x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
 }
+// eight operand values as two 16-byte shared-memory stores (see st_shared_f4)
+__device__ __forceinline__ void st8f(unsigned char *base, uint32_t off_lo, uint32_t off_hi,
+                                     const float *y) {
+  st_shared_f4(base + off_lo, y[0], y[1], y[2], y[3]);
+  st_shared_f4(base + off_hi, y[4], y[5], y[6], y[7]);
+}
 
 #ifdef KDA_PHASE_PROFILE
-// Cycles of worker thread 0 per phase of the loop, summed over every CTA (profiling
-// builds only), in the order of the loop: 0 chunk 0's operands, 1 wait for the next
-// chunk's tiles, 2 gate, 3 wait for O^T/Y^T, 4 scale, 5 rows, 6 wait for the last
-// products, 7 Khat^T, 8 out, 9 wait for A|P, 10 read, 11 solve, 12 final state;
-// entry 15 counts the chunks.
+// Cycles per step of the loops, summed over every CTA (profiling builds only):
+// group A (thread 0): 0 wait for O^T/Y^T(m-1), 1 wait for the tiles, 2 gate, 3 rows,
+// 4 wait for A|P, 5 read, 6 solve;  group B (thread 256): 8 wait for O^T/Y^T(n),
+// 9 scale, 10 wait for the next gate, 11 Khat^T, 12 wait for the last products,
+// 13 out, 14 V^T.  Entry 15 counts the chunks.
 __device__ unsigned long long g_phase_cycles[16];
 #define KDA_PHASE(k)                                              \
   do {                                                            \
@@ -166,36 +183,38 @@ __device__ unsigned long long g_phase_cycles[16];
 
 // LOGITS: the gate arrives as bf16 logits (fused gate activation) instead of fp32 g.
 template <typename TOut, bool LOGITS>
-__global__ void __launch_bounds__(NT + 32, 1)
+__global__ void __launch_bounds__(NT + 64, 1)
     prefill_tc_kernel(const PrefillParams p, const __grid_constant__ TcMaps maps) {
   extern __shared__ unsigned char smem_raw[];
-  unsigned char *sm = reinterpret_cast<unsigned char *>(
-      (reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  unsigned char *sm = align1024_shared(smem_raw);
   float *GT = reinterpret_cast<float *>(sm + OFF_GT);
   float *NS = reinterpret_cast<float *>(sm + OFF_NS);
   float *TS = reinterpret_cast<float *>(sm + OFF_TS);
   float *XS = reinterpret_cast<float *>(sm + OFF_XS);
   float *GC = reinterpret_cast<float *>(sm + OFF_GC);
+  float *E15 = reinterpret_cast<float *>(sm + OFF_E15);
   float *BT = reinterpret_cast<float *>(sm + OFF_BT);
   float *SEG = reinterpret_cast<float *>(sm + OFF_SEG);
   uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
-  uint64_t *bar_tma = bars + 0;   // [2] TMA -> workers: raw buffer b landed
+  uint64_t *bar_tma = bars + 0;   // [2] TMA -> group A: raw buffer b landed
   uint64_t *bar_ap = bars + 2;    // commit: A|P products done
   uint64_t *bar_oy = bars + 3;    // commit: O^T and Y^T products done (S^T read)
   uint64_t *bar_u = bars + 4;     // commit: U^T product done (control only)
   uint64_t *bar_fin = bars + 5;   // commit: the chunk's last products done
-  uint64_t *ops_ap = bars + 6;    // workers -> control: A|P operands built
-  uint64_t *raw_free = bars + 7;  // workers -> control: a raw buffer fully read
-  uint64_t *ops_oy = bars + 8;    // workers -> control: V^T, gamma*Q/K, Khat^T, P ready
-  uint64_t *ops_tb = bars + 9;    // workers -> control: T Diag(beta) ready
-  uint64_t *ops_sc = bars + 10;   // workers -> control: S^T scaled by gamma_31
-  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bars + 11);
+  uint64_t *ops_ap = bars + 6;    // group A -> control: A|P operands built
+  uint64_t *raw_free = bars + 7;  // A and B -> control: a raw buffer fully read
+  uint64_t *ops_oy = bars + 8;    // A (P, gamma*Q/K) and B (Khat^T, V^T) -> control
+  uint64_t *ops_tb = bars + 9;    // group A -> control: T Diag(beta) ready
+  uint64_t *ops_sc = bars + 10;   // group B -> control: S^T scaled by gamma_31
+  uint64_t *gate_ok = bars + 11;  // group A -> group B: cumulative gate of a chunk ready
+  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bars + 12);
   volatile int *s_abort = reinterpret_cast<volatile int *>(s_tmem + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane_id = tid & 31;
-  const bool control = warp == NT / 32;            // warp 16: TMA and MMA issue
+  const bool control = warp >= NT / 32;            // warps 16, 17: TMA and MMA issue
+  const bool group_a = warp < NA / 32;
   const int qd = warp & 3;                         // TMEM lane quarter of a worker warp
-  const int cg = (warp >> 2) & 3;                  // its column group
+  const int cg = (warp >> 2) & 1;                  // its half of the columns / tokens
   const int l = 32 * qd + lane_id;                 // its TMEM lane / channel
   const uint32_t lane_base = (uint32_t)(32 * qd) << 16;
   const int H = p.H;
@@ -231,11 +250,12 @@ __global__ void __launch_bounds__(NT + 32, 1)
     mbar_init(bar_oy, 1);
     mbar_init(bar_u, 1);
     mbar_init(bar_fin, 1);
-    mbar_init(ops_ap, NT / 32);
+    mbar_init(ops_ap, NA / 32);
     mbar_init(raw_free, NT / 32);
     mbar_init(ops_oy, NT / 32);
-    mbar_init(ops_tb, NT / 32);
-    mbar_init(ops_sc, NT / 32);
+    mbar_init(ops_tb, NA / 32);
+    mbar_init(ops_sc, (NT - NA) / 32);
+    mbar_init(gate_ok, NA / 32);
     *s_abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -245,14 +265,47 @@ __global__ void __launch_bounds__(NT + 32, 1)
   const uint32_t tm = *s_tmem;
   const int n_chunks = (len + C - 1) / C;
 
-  // What the control thread issued, so that a CTA that gives up can let it land: the
-  // TMA loads per raw buffer, and the barrier and phase parity of the last commit.
+  // What each issuing thread of the control warp issued, so that a CTA that gives up
+  // can let it land: the TMA loads per raw buffer, and the barrier and phase parity of
+  // the thread's last commit (a commit covers every earlier product of its thread).
   uint32_t tma_n0 = 0u, tma_n1 = 0u;
   uint64_t *last_bar = nullptr;
   uint32_t last_par = 0u;
 
+#ifdef KDA_PHASE_PROFILE
+  // thread 0's (group A) and thread 256's (group B) per-step sums, in spare bytes
+  const bool prof = tid == 0 || tid == NA;
+  unsigned long long *phase_acc = reinterpret_cast<unsigned long long *>(sm + OFF_BAR + 128);
+  if (tid == 0)
+    for (int k = 0; k < 16; ++k) phase_acc[k] = 0ull;
+  __syncthreads();
+  long long phase_t = clock64();
+#endif
+
+  // One arrival per warp.  warp_arrive hands shared-memory operands to the tensor
+  // cores, so its lanes' generic writes are first made visible to the async proxy;
+  // warp_signal orders only ordinary shared-memory and TMEM accesses (the arrival's
+  // release and the waiter's acquire), as for tables read by other warps, tiles
+  // that were only read, and TMEM written with tcgen05.st.
+  auto warp_signal = [&](uint64_t *bar) {
+    tc_fence_before();
+    __syncwarp();
+    if (lane_id == 0) mbar_arrive(bar);
+  };
+  auto warp_arrive = [&](uint64_t *bar) {
+    fence_async_smem();
+    warp_signal(bar);
+  };
+
   if (control) {
-    // ======================= control warp: TMA + MMA issue =======================
+    // ==================== control warp: TMA and MMA issue ====================
+    // Two threads in two warps issue independently, so that neither group's products
+    // wait for the other's (and a waiting thread never holds up the other's warp):
+    // warp 16 the TMA loads, A|P and U^T (group A's chain), warp 17 O^T, Y^T and the
+    // last products (the state chain).  Products of the two threads that depend on
+    // each other are ordered by the barriers below: U^T(m) waits for O^T, Y^T(m)
+    // (whose commit also covers warp 17's earlier products of chunk m-1), the last
+    // products of chunk m for U^T(m).
     if (lane_id == 0) {
       tma_prefetch_desc(&maps.q);
       tma_prefetch_desc(&maps.k);
@@ -319,7 +372,7 @@ __global__ void __launch_bounds__(NT + 32, 1)
       };
       // U^T = Y^T (T Diag(beta))^T
       auto mma_u = [&](int m) {
-        const uint32_t tb = smem_u32(sm + OFF_TB);
+        const uint32_t tb = smem_u32(sm + tb_off(m));
         const uint32_t id = idesc_tf32(C);
 #pragma unroll
         for (int s = 0; s < C / 8; ++s)
@@ -328,7 +381,7 @@ __global__ void __launch_bounds__(NT + 32, 1)
       };
       // O^T += U^T P^T and S^T += U^T Khat (S^T already scaled by gamma_31)
       auto mma_fin = [&](int m) {
-        const uint32_t pp = smem_u32(sm + OFF_PP), kh = smem_u32(sm + OFF_KH);
+        const uint32_t pp = smem_u32(sm + pp_off(m)), kh = smem_u32(sm + kh_off(m));
         const uint32_t id32 = idesc_tf32(C), id128 = idesc_tf32(DH);
 #pragma unroll
         for (int s = 0; s < C / 8; ++s) {
@@ -337,47 +390,39 @@ __global__ void __launch_bounds__(NT + 32, 1)
         }
         commit(bar_fin, m);
       };
-      // the products of chunk m that need only its own operands and the current state
-      auto prepare = [&](int m) -> bool {
-        if (!cwait(ops_ap, ph_ops_ap)) return false;
-        mma_ap(m);
-        if (!cwait(raw_free, ph_raw)) return false;
-        if (m + 2 < n_chunks) issue_tma(m + 2);
-        if (!cwait(ops_oy, ph_ops_oy)) return false;
-        mma_oy(m);
-        if (!cwait(ops_tb, ph_tb)) return false;
-        if (!cwait(bar_oy, ph_oy)) return false;  // Y^T is U^T's A operand
-        mma_u(m);
-        return true;
-      };
-      bool ok = true;
-      if (n_chunks > 0) issue_tma(0);
-      if (n_chunks > 1) issue_tma(1);
-      if (n_chunks > 0) ok = prepare(0);
-      for (int n = 0; ok && n < n_chunks; ++n) {
-        if (!(ok = cwait(ops_sc, ph_sc))) break;
-        if (!(ok = cwait(bar_u, ph_u))) break;  // U^T is the A operand of the last products
-        mma_fin(n);
-        if (n + 1 < n_chunks) ok = prepare(n + 1);
+      if (warp == NT / 32) {
+        if (n_chunks > 0) issue_tma(0);
+        if (n_chunks > 1) issue_tma(1);
+        for (int m = 0; m < n_chunks; ++m) {
+          if (!cwait(ops_ap, ph_ops_ap)) break;
+          mma_ap(m);
+          if (!cwait(ops_tb, ph_tb)) break;
+          if (!cwait(bar_oy, ph_oy)) break;  // Y^T is U^T's A operand
+          mma_u(m);
+          // chunk m's tiles are read by both groups: chunk m + 2 may load
+          if (!cwait(raw_free, ph_raw)) break;
+          if (m + 2 < n_chunks) issue_tma(m + 2);
+        }
+      } else {
+        for (int m = 0; m < n_chunks; ++m) {
+          if (!cwait(ops_oy, ph_ops_oy)) break;
+          mma_oy(m);
+          if (!cwait(ops_sc, ph_sc)) break;
+          if (!cwait(bar_u, ph_u)) break;  // U^T is the A operand of the last products
+          mma_fin(m);
+        }
       }
     }
-  } else {
-    // ======================= 16 worker warps =======================
-    uint32_t ph_tma = 0u, ph_ap = 0, ph_oy = 0, ph_fin = 0;  // ph_tma: bit b for buffer b
-#ifdef KDA_PHASE_PROFILE
-    // thread 0's per-phase sums live in the spare bytes after the barriers
-    const bool prof = tid == 0;
-    unsigned long long *phase_acc = reinterpret_cast<unsigned long long *>(sm + OFF_BAR + 128);
-    if (prof)
-      for (int k = 0; k < 16; ++k) phase_acc[k] = 0ull;
-    long long phase_t = clock64();
-#endif
-    auto wsync = [&]() { named_sync(1, NT); };
-    // every worker waits, then all of them vote, so an abort is taken by all together
+  } else if (group_a) {
+    // ============ group A (warps 0-7): gate, row operands, read-out, solve ============
+    uint32_t ph_tma = 0u, ph_ap = 0, ph_oy = 0;  // ph_tma: bit b for buffer b
+    auto wsync = [&]() { named_sync(1, NA); };
+    // every thread of the group waits, then all of them vote, so an abort is taken
+    // by all together
     auto wwait = [&](uint64_t *bar, uint32_t &ph) -> bool {
       const bool got = mbar_wait(bar, ph, wait_ns, s_abort);
       ph ^= 1u;
-      const bool bad = named_sync_or(1, NT, !got || *s_abort != 0);
+      const bool bad = named_sync_or(1, NA, !got || *s_abort != 0);
       if (bad) {
         if (!got) set_status(p.status, STATUS_TIMEOUT);
         *s_abort = 1;
@@ -385,373 +430,414 @@ __global__ void __launch_bounds__(NT + 32, 1)
       tc_fence_after();
       return !bad;
     };
-    // one arrival per warp once all its lanes' writes are visible to the async proxy
-    auto warp_arrive = [&](uint64_t *bar) {
-      fence_async_smem();
-      tc_fence_before();
-      __syncwarp();
-      if (lane_id == 0) mbar_arrive(bar);
-    };
-
-    // initial state -> S^T in TMEM (lane v holds S[:, v])
-    {
-      const float *s0 =
-          p.initial_state ? p.initial_state + ((size_t)(r * H + h)) * DH * DH : nullptr;
-      float v[32];
-#pragma unroll
-      for (int j = 0; j < 32; ++j)
-        v[j] = p.local_mode ? ((part == 1 && 32 * cg + j == l) ? 1.f : 0.f)
-                            : (s0 ? s0[(size_t)(32 * cg + j) * DH + l] : 0.f);
-      tmem_st32(tm + lane_base + TM_S + 32 * cg, v);
-      tmem_wait_st();
-    }
-    // T Diag(beta) is lower triangular: its block above the diagonal stays zero
-    if (tid < 64)
-      *reinterpret_cast<float4 *>(sm + OFF_TB + sw128_chunk(C, tid >> 2, 16 + 4 * (tid & 3))) =
-          make_float4(0.f, 0.f, 0.f, 0.f);
-
-    // beta of chunk m, row tid (warp 0), loaded a chunk ahead
-    auto load_beta = [&](int m) -> float {
-      float b = 0.f;
-      const int t = m * C + tid;
-      if (tid < C && m < n_chunks && t < len) {
-        b = p.beta[(size_t)(bos + t) * H + h];
-        if (p.validate && !(b >= 0.f && b <= 1.f)) set_status(p.status, STATUS_GATE_RANGE);
-      }
-      return b;
-    };
-    float beta_pref = load_beta(0);
-
-    // ---- gate(m): cumulative gate (thread = channel l, tokens 8 cg .. 8 cg + 7) ----
     auto wait_tma = [&](int m) -> bool {
       uint32_t ph = (ph_tma >> (m & 1)) & 1u;
       const bool got = wwait(bar_tma + (m & 1), ph);
       ph_tma ^= 1u << (m & 1);
       return got;
     };
+    // T Diag(beta) is lower triangular: its block above the diagonal stays zero
+    if (tid < 128)
+      *reinterpret_cast<float4 *>(sm + tb_off(tid >> 6) +
+                                  sw128_chunk(C, (tid >> 2) & 15, 16 + 4 * (tid & 3))) =
+          make_float4(0.f, 0.f, 0.f, 0.f);
+
+    // beta of chunk m, row tid (warp 0), loaded a chunk ahead and checked when stored;
+    // a predicated load, so that nothing waits for it before its use a chunk later
+    auto load_beta = [&](int m) -> float {
+      const int t = m * C + tid;
+      const bool in = tid < C && m < n_chunks && t < len;
+      const float *src = p.beta + (in ? (size_t)(bos + t) * H + h : 0);
+      float b = 0.f;
+      asm volatile(
+          "{\n\t.reg .pred q;\n\tsetp.ne.u32 q, %2, 0;\n\t@q ld.global.nc.f32 %0, [%1];\n\t}"
+          : "+f"(b)
+          : "l"(src), "r"((uint32_t)in));
+      return b;
+    };
+    float beta_pref = load_beta(0);
+
+    // ---- gate(m): cumulative gate (thread = channel l, tokens 16 cg .. 16 cg + 15) ----
     auto w_gate = [&](int m) {
       const int nr = min(C, len - m * C);
       const unsigned char *raw = sm + OFF_RAW + (m & 1) * RAW_BYTES;
-      if (tid < C) BT[tid] = beta_pref;
+      if (tid < C) {
+        if (p.validate && !(beta_pref >= 0.f && beta_pref <= 1.f))
+          set_status(p.status, STATUS_GATE_RANGE);
+        BT[tid] = beta_pref;
+      }
       beta_pref = load_beta(m + 1);
-      float gv[8];
+      // every row of the tile is loaded (rows past the chunk's end hold other data or the
+      // zero fill) and masked afterwards, so that the 16 loads issue back to back
+      float gv[16];
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int t = 8 * cg + j;
-        float x = 0.f;
-        if (t < nr) {
-          if (LOGITS) {
-            x = gate_from_logit(bf16_at(raw + R_G, t, l));
-          } else {
-            x = *reinterpret_cast<const float *>(raw + R_G + f32_off(t, l));
-            if (p.validate && !(x >= kGateLower && x <= 0.f)) set_status(p.status, STATUS_GATE_RANGE);
-          }
-        }
-        gv[j] = x;
+      for (int j = 0; j < 16; ++j) {
+        const int t = 16 * cg + j;
+        gv[j] = LOGITS ? gate_from_logit(bf16_at(raw + R_G, t, l))
+                       : *reinterpret_cast<const float *>(raw + R_G + f32_off(t, l));
       }
 #pragma unroll
-      for (int j = 1; j < 8; ++j) gv[j] += gv[j - 1];
-      SEG[cg * DH + l] = gv[7];
-      wsync();
-      float off = 0.f;
-      for (int gg = 0; gg < cg; ++gg) off += SEG[gg * DH + l];
+      for (int j = 0; j < 16; ++j) gv[j] = (16 * cg + j < nr) ? gv[j] : 0.f;
+      if (!LOGITS && p.validate) {
+        bool bad = false;
 #pragma unroll
-      for (int j = 0; j < 8; ++j) {
+        for (int j = 0; j < 16; ++j) bad |= !(gv[j] >= kGateLower && gv[j] <= 0.f);
+        if (bad) set_status(p.status, STATUS_GATE_RANGE);
+      }
+#pragma unroll
+      for (int j = 1; j < 16; ++j) gv[j] += gv[j - 1];
+      if (cg == 0) SEG[l] = gv[15];
+      wsync();
+      const float off = cg ? SEG[l] : 0.f;
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
         const float g2 = (gv[j] + off) * LOG2E;
-        GT[(8 * cg + j) * LDG + l] = g2;
-        if (cg == 3 && j == 7) GC[(m & 1) * DH + l] = ex2(g2);
+        GT[(16 * cg + j) * LDG + l] = g2;
+        if (j == 15) (cg ? GC + (m & 1) * DH : E15)[l] = ex2(g2);
       }
       wsync();
+      warp_signal(gate_ok);
     };
 
-    // ---- scale(n): S^T <- S^T Diag(gamma_31) once the O^T and Y^T products read S^T ----
-    auto w_scale = [&](int n) {
-      float v[32];
-      tmem_ld32(tm + lane_base + TM_S + 32 * cg, v);
-      tmem_wait_ld();
-      const float *gc = GC + (n & 1) * DH + 32 * cg;
-#pragma unroll
-      for (int j = 0; j < 32; j += 8) {
-        float f[8];
-        ld8f(gc + j, f);
-#pragma unroll
-        for (int e = 0; e < 8; ++e) v[j + e] *= f[e];
-      }
-      tmem_st32(tm + lane_base + TM_S + 32 * cg, v);
-      tmem_wait_st();
-      warp_arrive(ops_sc);
-    };
-
-    // ---- rows(m): the row operands (thread = row i, channels 32 cg .. 32 cg + 31) ----
+    // ---- rows(m): the row operands (thread = row i, channels 64 cg .. 64 cg + 63) ----
     // lane quarter 0: L_k = k exp(G_i - G_15) -> TMEM lanes 0-31
-    // lane quarter 1: L_q = q exp(G_i - G_15) -> TMEM lanes 32-63
+    // lane quarter 1: L_q = q exp(G_i - G_15) -> TMEM lanes 32-63, gamma*Q = L_q exp(G_15)
     // lane quarter 2: R'  = k exp(G_15 - G_i) -> smem
-    // lane quarter 3: gamma*K, gamma*Q = (k, q) exp(G_i)  -> smem
+    // lane quarter 3: gamma*K = k exp(G_i)    -> smem
     auto w_rows = [&](int m) {
       const int nr = min(C, len - m * C);
       const unsigned char *raw = sm + OFF_RAW + (m & 1) * RAW_BYTES;
       const int i = lane_id;
       const bool valid = i < nr;
-      const float *gi = GT + i * LDG + 32 * cg;
-      const float *gm = GT + MREF * LDG + 32 * cg;
       const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
-      if (qd <= 1) {
-        if (qd == 0 || has_q) {
-          const unsigned char *xr = raw + (qd == 0 ? R_K : R_Q);
+      if (qd == 1 && !has_q) return;
+      const unsigned char *xr = raw + (qd == 1 ? R_Q : R_K);
+      unsigned char *dst = sm + (qd == 1 ? OFF_GQ : qd == 2 ? OFF_RP : OFF_GK);
+#pragma unroll 2
+      for (int jj = 0; jj < 8; ++jj) {
+        const int c = 64 * cg + 8 * jj;
+        float x[8], g[8], y[8];
+        bf16_x8(valid ? *reinterpret_cast<const uint4 *>(xr + bf16_chunk(i, c)) : z4, x);
+        ld8f(GT + i * LDG + c, g);
+        if (qd == 3) {
 #pragma unroll
-          for (int jj = 0; jj < 4; ++jj) {
-            const int c = 32 * cg + 8 * jj;
-            float x[8], g[8], gr[8], lv[8];
-            bf16_x8(valid ? *reinterpret_cast<const uint4 *>(xr + bf16_chunk(i, c)) : z4, x);
-            ld8f(gi + 8 * jj, g);
-            ld8f(gm + 8 * jj, gr);
+          for (int e = 0; e < 8; ++e) y[e] = tf32_rna(x[e] * ex2(g[e]));
+        } else {
+          float gr[8];
+          ld8f(GT + MREF * LDG + c, gr);
+          if (qd == 2) {
 #pragma unroll
-            for (int e = 0; e < 8; ++e) lv[e] = tf32_rna(x[e] * ex2(g[e] - gr[e]));
+            for (int e = 0; e < 8; ++e) y[e] = tf32_rna(x[e] * ex2(gr[e] - g[e]));
+          } else {
+            float lv[8];
+#pragma unroll
+            for (int e = 0; e < 8; ++e) {
+              const float a = x[e] * ex2(g[e] - gr[e]);
+              lv[e] = tf32_rna(a);
+              y[e] = a;
+            }
             tmem_st8(tm + lane_base + TM_L + c, lv);
-          }
-          tmem_wait_st();
-        }
-      } else if (qd == 2) {
-        unsigned char *rp = sm + OFF_RP;
+            if (qd == 1) {
+              float e15[8];
+              ld8f(E15 + c, e15);
 #pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-          const int c = 32 * cg + 8 * jj;
-          float x[8], g[8], gr[8];
-          bf16_x8(valid ? *reinterpret_cast<const uint4 *>(raw + R_K + bf16_chunk(i, c)) : z4, x);
-          ld8f(gi + 8 * jj, g);
-          ld8f(gm + 8 * jj, gr);
-          float y[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) y[e] = tf32_rna(x[e] * ex2(gr[e] - g[e]));
-          *reinterpret_cast<float4 *>(rp + sw128_chunk(C, i, c)) = make_float4(y[0], y[1], y[2], y[3]);
-          *reinterpret_cast<float4 *>(rp + sw128_chunk(C, i, c + 4)) = make_float4(y[4], y[5], y[6], y[7]);
-        }
-      } else {
-        unsigned char *gk = sm + OFF_GK, *gq = sm + OFF_GQ;
-#pragma unroll
-        for (int jj = 0; jj < 4; ++jj) {
-          const int c = 32 * cg + 8 * jj;
-          float xk[8], xq[8], g[8];
-          bf16_x8(valid ? *reinterpret_cast<const uint4 *>(raw + R_K + bf16_chunk(i, c)) : z4, xk);
-          bf16_x8(valid && has_q ? *reinterpret_cast<const uint4 *>(raw + R_Q + bf16_chunk(i, c)) : z4, xq);
-          ld8f(gi + 8 * jj, g);
-          float yk[8], yq[8];
-#pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            const float gam = ex2(g[e]);
-            yk[e] = tf32_rna(xk[e] * gam);
-            yq[e] = tf32_rna(xq[e] * gam);
-          }
-          *reinterpret_cast<float4 *>(gk + sw128_chunk(C, i, c)) = make_float4(yk[0], yk[1], yk[2], yk[3]);
-          *reinterpret_cast<float4 *>(gk + sw128_chunk(C, i, c + 4)) = make_float4(yk[4], yk[5], yk[6], yk[7]);
-          if (has_q) {
-            *reinterpret_cast<float4 *>(gq + sw128_chunk(C, i, c)) = make_float4(yq[0], yq[1], yq[2], yq[3]);
-            *reinterpret_cast<float4 *>(gq + sw128_chunk(C, i, c + 4)) = make_float4(yq[4], yq[5], yq[6], yq[7]);
+              for (int e = 0; e < 8; ++e) y[e] = tf32_rna(y[e] * e15[e]);
+            }
           }
         }
+        if (qd != 0) st8f(dst, sw128_chunk(C, i, c), sw128_chunk(C, i, c + 4), y);
       }
-      warp_arrive(ops_ap);
+      if (qd <= 1) tmem_wait_st();
     };
 
-    // ---- khat(m): Khat^T = (k exp(G_31 - G))^T (thread = row i, channels 8 warp ..) ----
-    auto w_khat = [&](int m) {
-      const int nr = min(C, len - m * C);
-      const unsigned char *raw = sm + OFF_RAW + (m & 1) * RAW_BYTES;
-      const int i = lane_id, c = 8 * warp;
-      float x[8], g[8], ge[8];
-      bf16_x8(i < nr ? *reinterpret_cast<const uint4 *>(raw + R_K + bf16_chunk(i, c))
-                     : make_uint4(0u, 0u, 0u, 0u),
-              x);
-      ld8f(GT + i * LDG + c, g);
-      ld8f(GT + (C - 1) * LDG + c, ge);
-#pragma unroll
-      for (int e = 0; e < 8; ++e)
-        *reinterpret_cast<float *>(sm + OFF_KH + sw128_offset(DH, c + e, i)) =
-            tf32_rna(x[e] * ex2(ge[e] - g[e]));
-    };
-
-    // ---- out(n): O^T -> o (lane = value channel, tokens 8 cg ..), snapshot ----
-    auto w_out = [&](int n) {
-      const int c0 = n * C, nr = min(C, len - c0);
-      if (go) {
-        float o8[8];
-        tmem_ld8(tm + lane_base + TM_O + 8 * cg, o8);
-        tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          const int t = 8 * cg + j;
-          if (t < nr) store_elem(go, ((size_t)(bos + c0 + t) * H + h) * DH + l, o8[j]);
-        }
-      }
-      if (snaps_ok && nr == C && (c0 + C) % p.snapshot_stride == 0) {
-        const size_t row = (size_t)p.cu_snapshots[r] + (c0 + C) / p.snapshot_stride - 1;
-        float *dst = p.snapshots + (row * H + h) * (size_t)DH * DH;
-        float v[32];
-        tmem_ld32(tm + lane_base + TM_S + 32 * cg, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int j = 0; j < 32; ++j) dst[(size_t)(32 * cg + j) * DH + l] = v[j];
-      }
-    };
-
-    // ---- read(m): Diag(beta) A and P out of TMEM (after the A|P products), V^T into TMEM ----
+    // ---- read(m): Diag(beta) A and P out of TMEM (after the A|P products) ----
     auto w_read = [&](int m) {
-      const int nr = min(C, len - m * C);
-      const unsigned char *raw = sm + OFF_RAW + (m & 1) * RAW_BYTES;
       const int i = lane_id;
-      if (qd == 0) {  // row i of A, columns 8 cg ..: N = beta_i A_ij for j < i
-        float a8[8];
-        tmem_ld8(tm + lane_base + TM_AP + 8 * cg, a8);
+      if (qd == 0) {  // row i of A, columns 16 cg ..: N = beta_i A_ij for j < i
+        float a[16];
+        tmem_ld16(tm + lane_base + TM_AP + 16 * cg, a);
         tmem_wait_ld();
         const float bi = BT[i];
-        float n8[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) n8[e] = (8 * cg + e < i) ? bi * a8[e] : 0.f;
-        float4 *dst = reinterpret_cast<float4 *>(NS + i * LDN + 8 * cg);
-        dst[0] = make_float4(n8[0], n8[1], n8[2], n8[3]);
-        dst[1] = make_float4(n8[4], n8[5], n8[6], n8[7]);
+        for (int e = 0; e < 16; ++e) a[e] = (16 * cg + e < i) ? bi * a[e] : 0.f;
+        float4 *nd = reinterpret_cast<float4 *>(NS + i * LDN + 16 * cg);
+#pragma unroll
+        for (int e = 0; e < 4; ++e) nd[e] = make_float4(a[4 * e], a[4 * e + 1], a[4 * e + 2], a[4 * e + 3]);
       } else if (qd == 1 && has_q) {  // row i of P, inclusive lower, tf32 B operand
-        float a8[8];
-        tmem_ld8(tm + lane_base + TM_AP + 8 * cg, a8);
+        float a[16];
+        tmem_ld16(tm + lane_base + TM_AP + 16 * cg, a);
         tmem_wait_ld();
-        float p8[8];
 #pragma unroll
-        for (int e = 0; e < 8; ++e) p8[e] = (8 * cg + e <= i) ? tf32_rna(a8[e]) : 0.f;
-        *reinterpret_cast<float4 *>(sm + OFF_PP + sw128_chunk(C, i, 8 * cg)) =
-            make_float4(p8[0], p8[1], p8[2], p8[3]);
-        *reinterpret_cast<float4 *>(sm + OFF_PP + sw128_chunk(C, i, 8 * cg + 4)) =
-            make_float4(p8[4], p8[5], p8[6], p8[7]);
+        for (int e = 0; e < 16; ++e) a[e] = (16 * cg + e <= i) ? tf32_rna(a[e]) : 0.f;
+        unsigned char *pp = sm + pp_off(m);
+        st8f(pp, sw128_chunk(C, i, 16 * cg), sw128_chunk(C, i, 16 * cg + 4), a);
+        st8f(pp, sw128_chunk(C, i, 16 * cg + 8), sw128_chunk(C, i, 16 * cg + 12), a + 8);
       }
-      float v8[8];
-#pragma unroll
-      for (int j = 0; j < 8; ++j) {
-        const int t = 8 * cg + j;
-        v8[j] = (t < nr && !zero_v) ? bf16_at(raw + R_V, t, l) : 0.f;
-      }
-      tmem_st8(tm + lane_base + TM_Y + 8 * cg, v8);
-      tmem_wait_st();
-      warp_arrive(raw_free);
-      warp_arrive(ops_oy);
     };
 
     // ---- solve(m): T = (I + Diag(beta) A)^-1 by 16 x 16 blocks, then T Diag(beta) ----
-    auto w_solve = [&]() {
+    auto w_solve = [&](int m) {
+      unsigned char *tb = sm + tb_off(m);
       wsync();  // Diag(beta) A complete
       if (warp == 2) {
         // the two diagonal blocks, row by row: t_i = e_i - sum_{j<i} N_ij t_j, one
-        // column per lane (lanes 0-15: block 0, lanes 16-31: block 1)
+        // column per lane (lanes 0-15: block 0, lanes 16-31: block 1); the sum runs
+        // in two halves to shorten the dependent chain
         const int o = 16 * (lane_id >> 4), c = lane_id & 15;
         float t[16];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           const float4 *nrow = reinterpret_cast<const float4 *>(NS + (o + i) * LDN + o);
-          float acc = (i == c) ? 1.f : 0.f;
+          float acc0 = (i == c) ? 1.f : 0.f, acc1 = 0.f;
 #pragma unroll
-          for (int j4 = 0; 4 * j4 < i; ++j4) {
+          for (int j4 = 0; j4 < 4; ++j4) {
+            if (4 * j4 >= i) break;
             const float4 n4 = nrow[j4];
             const float nv[4] = {n4.x, n4.y, n4.z, n4.w};
 #pragma unroll
-            for (int e = 0; e < 4; ++e)
-              if (4 * j4 + e < i) acc -= nv[e] * t[4 * j4 + e];
+            for (int e = 0; e < 4; ++e) {
+              const int j = 4 * j4 + e;
+              if (j < i) {
+                if (j & 1) acc1 -= nv[e] * t[j];
+                else acc0 -= nv[e] * t[j];
+              }
+            }
           }
-          t[i] = acc;
+          t[i] = acc0 + acc1;
         }
         const float bc = BT[o + c];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           TS[(o + i) * LDN + o + c] = t[i];
-          *reinterpret_cast<float *>(sm + OFF_TB + sw128_offset(C, o + i, o + c)) =
-              tf32_rna(t[i] * bc);
+          st_shared_f1(tb + sw128_offset(C, o + i, o + c), tf32_rna(t[i] * bc));
         }
       }
       wsync();  // diagonal blocks ready
-      if (warp >= 8) {  // T10 = -T11 (N10 T00): one element (i, c) per thread
-        const int tt = tid - 256, i = tt >> 4, c = tt & 15;
-        float x = 0.f;
+      {  // T10 = -T11 (N10 T00): one element (i, c) per thread of the group
+        // the T00 entries above the diagonal and the T11 entries past row i are zero, so
+        // the sums run over all 16 terms without branches, in two halves each
+        const int i = tid >> 4, c = tid & 15;
+        float x0 = 0.f, x1 = 0.f;
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-          if (j >= c) x += NS[(16 + i) * LDN + j] * TS[j * LDN + c];
-        XS[i * LDX + c] = x;
-        named_sync(2, 256);
-        float y = 0.f;
+        for (int j = 0; j < 8; ++j) {
+          x0 += NS[(16 + i) * LDN + j] * TS[j * LDN + c];
+          x1 += NS[(16 + i) * LDN + 8 + j] * TS[(8 + j) * LDN + c];
+        }
+        XS[i * LDX + c] = x0 + x1;
+        wsync();
+        float y0 = 0.f, y1 = 0.f;
 #pragma unroll
-        for (int j = 0; j < 16; ++j)
-          if (j <= i) y += TS[(16 + i) * LDN + 16 + j] * XS[j * LDX + c];
-        *reinterpret_cast<float *>(sm + OFF_TB + sw128_offset(C, 16 + i, c)) =
-            tf32_rna(-y * BT[c]);
+        for (int j = 0; j < 8; ++j) {
+          y0 += TS[(16 + i) * LDN + 16 + j] * XS[j * LDX + c];
+          y1 += TS[(16 + i) * LDN + 24 + j] * XS[(8 + j) * LDX + c];
+        }
+        st_shared_f1(tb + sw128_offset(C, 16 + i, c), tf32_rna(-(y0 + y1) * BT[c]));
       }
-      warp_arrive(ops_tb);
     };
 
-    // chunk 0's operands, then the pipelined loop (phase numbers: profiling builds)
     bool ok = true;
-    if (n_chunks > 0) {
-      if ((ok = wait_tma(0))) {
-        w_gate(0);
-        w_rows(0);
-        w_khat(0);
-        if ((ok = wwait(bar_ap, ph_ap))) {
-          w_read(0);
-          w_solve();
+    for (int m = 0; ok && m < n_chunks; ++m) {
+      // chunk m-1's O^T and Y^T products are done: gamma*Q/K and the gate tables are free
+      // (and, through group B, chunk m-2's last products are done too)
+      if (m > 0 && !(ok = wwait(bar_oy, ph_oy))) break;
+      KDA_PHASE(0);
+      if (!(ok = wait_tma(m))) break;
+      KDA_PHASE(1);
+      w_gate(m);
+      KDA_PHASE(2);
+      w_rows(m);
+      warp_signal(raw_free);
+      warp_arrive(ops_ap);
+      KDA_PHASE(3);
+      if (!(ok = wwait(bar_ap, ph_ap))) break;
+      KDA_PHASE(4);
+      w_read(m);
+      warp_arrive(ops_oy);
+      KDA_PHASE(5);
+      w_solve(m);
+      warp_arrive(ops_tb);
+      KDA_PHASE(6);
+    }
+  } else {
+    // ====== group B (warps 8-15): state scaling, Khat^T, outputs, V^T, states ======
+    uint32_t ph_oy = 0, ph_gate = 0, ph_fin = 0;
+    // every thread of the group waits, then all of them vote at the group's barrier
+    auto bwait = [&](uint64_t *bar, uint32_t &ph) -> bool {
+      const bool got = mbar_wait(bar, ph, wait_ns, s_abort);
+      ph ^= 1u;
+      const bool bad = named_sync_or(2, NT - NA, !got || *s_abort != 0);
+      if (bad) {
+        if (!got) set_status(p.status, STATUS_TIMEOUT);
+        *s_abort = 1;
+      }
+      tc_fence_after();
+      return !bad;
+    };
+    const int w8 = warp - NA / 32;  // 0..7
+
+    // initial state -> S^T in TMEM (lane v holds S[:, v]), columns 64 cg ..
+    {
+      const float *s0 =
+          p.initial_state ? p.initial_state + ((size_t)(r * H + h)) * DH * DH : nullptr;
+#pragma unroll
+      for (int half = 0; half < 2; ++half) {
+        const int c0 = 64 * cg + 32 * half;
+        float v[32];
+#pragma unroll
+        for (int j = 0; j < 32; ++j)
+          v[j] = p.local_mode ? ((part == 1 && c0 + j == l) ? 1.f : 0.f)
+                              : (s0 ? s0[(size_t)(c0 + j) * DH + l] : 0.f);
+        tmem_st32(tm + lane_base + TM_S + c0, v);
+      }
+      tmem_wait_st();
+    }
+
+    // ---- scale(n): S^T <- S^T Diag(gamma_31) once the O^T and Y^T products read S^T ----
+    auto w_scale = [&](int n) {
+      const float *gc = GC + (n & 1) * DH;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int c0 = 64 * cg + 16 * q;
+        float v[16];
+        tmem_ld16(tm + lane_base + TM_S + c0, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 16; j += 8) {
+          float f[8];
+          ld8f(gc + c0 + j, f);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) v[j + e] *= f[e];
+        }
+        tmem_st16(tm + lane_base + TM_S + c0, v);
+      }
+      tmem_wait_st();
+    };
+
+    // ---- khat(m): Khat^T = (k exp(G_31 - G))^T (thread = row i, channels 16 w8 ..) ----
+    auto w_khat = [&](int m) {
+      const int nr = min(C, len - m * C);
+      const unsigned char *raw = sm + OFF_RAW + (m & 1) * RAW_BYTES;
+      unsigned char *kh = sm + kh_off(m);
+      const int i = lane_id;
+#pragma unroll
+      for (int u = 0; u < 2; ++u) {
+        const int c = 16 * w8 + 8 * u;
+        float x[8], g[8], ge[8];
+        bf16_x8(i < nr ? *reinterpret_cast<const uint4 *>(raw + R_K + bf16_chunk(i, c))
+                       : make_uint4(0u, 0u, 0u, 0u),
+                x);
+        ld8f(GT + i * LDG + c, g);
+        ld8f(GT + (C - 1) * LDG + c, ge);
+#pragma unroll
+        for (int e = 0; e < 8; ++e)
+          st_shared_f1(kh + sw128_offset(DH, c + e, i), tf32_rna(x[e] * ex2(ge[e] - g[e])));
+      }
+    };
+
+    // ---- out(n): O^T -> o (lane = value channel, tokens 16 cg ..), snapshot ----
+    auto w_out = [&](int n) {
+      const int c0 = n * C, nr = min(C, len - c0);
+      if (go) {
+        float o16[16];
+        tmem_ld16(tm + lane_base + TM_O + 16 * cg, o16);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int t = 16 * cg + j;
+          if (t < nr) store_elem(go, ((size_t)(bos + c0 + t) * H + h) * DH + l, o16[j]);
         }
       }
+      if (snaps_ok && nr == C && (c0 + C) % p.snapshot_stride == 0) {
+        const size_t row = (size_t)p.cu_snapshots[r] + (c0 + C) / p.snapshot_stride - 1;
+        float *dst = p.snapshots + (row * H + h) * (size_t)DH * DH;
+#pragma unroll
+        for (int half = 0; half < 2; ++half) {
+          const int k0 = 64 * cg + 32 * half;
+          float v[32];
+          tmem_ld32(tm + lane_base + TM_S + k0, v);
+          tmem_wait_ld();
+#pragma unroll
+          for (int j = 0; j < 32; ++j) dst[(size_t)(k0 + j) * DH + l] = v[j];
+        }
+      }
+    };
+
+    // ---- vt(m): V^T -> TMEM (lane = value channel, tokens 16 cg ..) ----
+    auto w_vt = [&](int m) {
+      const int nr = min(C, len - m * C);
+      const unsigned char *raw = sm + OFF_RAW + (m & 1) * RAW_BYTES;
+      float v16[16];
+#pragma unroll
+      for (int j = 0; j < 16; ++j) {
+        const int t = 16 * cg + j;
+        v16[j] = (t < nr && !zero_v) ? bf16_at(raw + R_V, t, l) : 0.f;
+      }
+      tmem_st16(tm + lane_base + TM_Y + 16 * cg, v16);
+      tmem_wait_st();
+    };
+
+    bool ok = true;
+    if (n_chunks > 0) {
+      if ((ok = bwait(gate_ok, ph_gate))) {
+        w_khat(0);
+        w_vt(0);
+        warp_signal(raw_free);
+        warp_arrive(ops_oy);
+      }
     }
-    KDA_PHASE(0);
     for (int n = 0; ok && n < n_chunks; ++n) {
       const bool more = n + 1 < n_chunks;
-      if (more) {
-        if (!(ok = wait_tma(n + 1))) break;
-        KDA_PHASE(1);
-        w_gate(n + 1);
-        KDA_PHASE(2);
-      }
-      if (!(ok = wwait(bar_oy, ph_oy))) break;
-      KDA_PHASE(3);
-      w_scale(n);
-      KDA_PHASE(4);
-      if (more) w_rows(n + 1);
-      KDA_PHASE(5);
-      if (!(ok = wwait(bar_fin, ph_fin))) break;
-      KDA_PHASE(6);
-      if (more) w_khat(n + 1);
-      KDA_PHASE(7);
-      w_out(n);
+      if (!(ok = bwait(bar_oy, ph_oy))) break;
       KDA_PHASE(8);
+      w_scale(n);
+      warp_signal(ops_sc);
+      KDA_PHASE(9);
       if (more) {
-        if (!(ok = wwait(bar_ap, ph_ap))) break;
-        KDA_PHASE(9);
-        w_read(n + 1);
+        if (!(ok = bwait(gate_ok, ph_gate))) break;
         KDA_PHASE(10);
-        w_solve();
+        w_khat(n + 1);  // the other Khat^T buffer: chunk n-1's last products are done
         KDA_PHASE(11);
       }
+      if (!(ok = bwait(bar_fin, ph_fin))) break;
+      KDA_PHASE(12);
+      w_out(n);
+      KDA_PHASE(13);
+      if (more) {
+        w_vt(n + 1);
+        warp_signal(raw_free);  // before ops_oy: group A's next arrivals wait for it
+        warp_arrive(ops_oy);
+      }
+      KDA_PHASE(14);
     }
 
     float *fin = p.local_mode ? (part == 0 ? p.s_loc : p.m) : p.final_state;
     if (ok && fin) {
       float *dst = fin + ((size_t)(r * H + h)) * DH * DH;
       tc_fence_after();
-      float v[32];
-      tmem_ld32(tm + lane_base + TM_S + 32 * cg, v);
-      tmem_wait_ld();
 #pragma unroll
-      for (int j = 0; j < 32; ++j) dst[(size_t)(32 * cg + j) * DH + l] = v[j];
+      for (int half = 0; half < 2; ++half) {
+        const int k0 = 64 * cg + 32 * half;
+        float v[32];
+        tmem_ld32(tm + lane_base + TM_S + k0, v);
+        tmem_wait_ld();
+#pragma unroll
+        for (int j = 0; j < 32; ++j) dst[(size_t)(k0 + j) * DH + l] = v[j];
+      }
     }
-#ifdef KDA_PHASE_PROFILE
-    KDA_PHASE(12);
-    if (prof) {
-      for (int k = 0; k < 13; ++k) atomicAdd(&g_phase_cycles[k], phase_acc[k]);
-      atomicAdd(&g_phase_cycles[15], (unsigned long long)n_chunks);
-    }
-#endif
   }
+#ifdef KDA_PHASE_PROFILE
+  if (tid == 0) atomicAdd(&g_phase_cycles[15], (unsigned long long)n_chunks);
+  __syncthreads();
+  if (tid == 0)
+    for (int k = 0; k < 15; ++k) atomicAdd(&g_phase_cycles[k], phase_acc[k]);
+#endif
 
   tc_fence_before();
   __syncthreads();
   if (*s_abort && control && lane_id == 0) {
     // the CTA gave up: let the copies and products it issued land before it releases
-    // its shared and tensor memory (at most one load per buffer and, the products
-    // completing in order, the last commit are outstanding)
+    // its shared and tensor memory (at most one load per buffer and, the products of
+    // a thread completing in order, its last commit are outstanding)
     if (tma_n0) mbar_wait(bar_tma, (tma_n0 - 1u) & 1u, 100000000ull);
     if (tma_n1) mbar_wait(bar_tma + 1, (tma_n1 - 1u) & 1u, 100000000ull);
     if (last_bar) mbar_wait(last_bar, last_par, 100000000ull);
@@ -822,7 +908,7 @@ cudaError_t launch_prefill_tc(const PrefillParams &p, kda_dtype in_dtype, kda_dt
     const cudaError_t e =
         cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_ALLOC);
     if (e != cudaSuccess) return e;
-    kernel<<<grid, NT + 32, SMEM_ALLOC, stream>>>(p, maps);
+    kernel<<<grid, NT + 64, SMEM_ALLOC, stream>>>(p, maps);
     return cudaGetLastError();
   };
   const bool logits = p.g_logits != nullptr;

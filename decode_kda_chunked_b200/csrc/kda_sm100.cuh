@@ -23,6 +23,17 @@ __device__ __forceinline__ uint32_t smem_u32(const void *p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
 }
 
+// The first 1024-byte-aligned byte of a dynamic shared-memory block (TMA boxes and
+// MMA operands with the 128-byte swizzle need that alignment).  The offset is
+// added to the __shared__ array itself, never through an integer round trip, so
+// that the compiler still knows every derived pointer addresses shared memory and
+// emits shared-memory loads and stores instead of generic ones.
+template <typename T>
+__device__ __forceinline__ unsigned char *align1024_shared(T *smem) {
+  unsigned char *p = reinterpret_cast<unsigned char *>(smem);
+  return p + ((1024u - (smem_u32(p) & 1023u)) & 1023u);
+}
+
 // --------------------------------------------------------------------------
 // Shared-memory layout of a K-major, 128B-swizzled tf32 B operand.
 // --------------------------------------------------------------------------
@@ -95,6 +106,11 @@ __device__ __forceinline__ void tmem_wait_st() {
   asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory");
 }
 
+// tcgen05.st writes only tensor memory, so its asm carries no memory clobber: the
+// compiler may then move shared-memory loads across it (a TMEM store orders with
+// later tensor-core reads through tcgen05.wait::st and the tcgen05 fences, which
+// keep theirs).
+//
 // 32 lanes x 32 columns: thread t of the warp gets columns c..c+31 of lane
 // (warp's lane quarter) + t.  taddr carries the lane offset in bits 16-31.
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, float *v) {
@@ -122,7 +138,7 @@ __device__ __forceinline__ void tmem_st32(uint32_t taddr, const float *v) {
       "r"(r[15]), "r"(r[16]), "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]),
       "r"(r[22]), "r"(r[23]), "r"(r[24]), "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]),
       "r"(r[29]), "r"(r[30]), "r"(r[31])
-      : "memory");
+      );
 }
 
 // 32 lanes x 16 columns.
@@ -144,7 +160,7 @@ __device__ __forceinline__ void tmem_st16(uint32_t taddr, const float *v) {
       "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]),
       "r"(r[8]), "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]),
       "r"(r[15])
-      : "memory");
+      );
 }
 
 // 32 lanes x 8 columns.
@@ -162,7 +178,7 @@ __device__ __forceinline__ void tmem_st8(uint32_t taddr, const float *v) {
       "tcgen05.st.sync.aligned.32x32b.x8.b32 [%0], {%1, %2, %3, %4, %5, %6, %7, %8};" ::"r"(
           taddr),
       "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7])
-      : "memory");
+      );
 }
 
 // 2^x on the special-function unit (ex2.approx, flush-to-zero; relative error
@@ -255,9 +271,57 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
   }
 }
 
+// Non-blocking test of a phase (no suspension).
+__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// The bounded wait for a thread that waits on behalf of others (its group then
+// learns the outcome at a named barrier, where waiting costs no instructions):
+// non-blocking tests with a short sleep between them (32 ns doubling up to
+// max_sleep_ns), the abort flag and the clock read only every 8 tries.
+__device__ __forceinline__ bool mbar_wait_lean(uint64_t *bar, uint32_t parity,
+                                               uint64_t timeout_ns,
+                                               const volatile int *abort_flag,
+                                               uint32_t max_sleep_ns = 128u) {
+  if (mbar_test_wait(bar, parity)) return true;
+  const uint64_t t0 = global_ns();
+  uint32_t ns = 32u;
+  for (uint32_t i = 1;; ++i) {
+    __nanosleep(ns);
+    if (mbar_test_wait(bar, parity)) return true;
+    if ((i & 7u) == 0u) {
+      if (abort_flag && *abort_flag) return false;
+      if (global_ns() - t0 > timeout_ns) return false;
+    }
+    ns = ns < max_sleep_ns ? 2u * ns : max_sleep_ns;
+  }
+}
+
 // Plain arrive (count 1) on an mbarrier.
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+
+// Shared-memory stores of operand tiles inside a phase, written as asm that the
+// compiler does not treat as aliasing later loads, so that the next loads of a loop
+// can be issued before the current stores.  Only for data no load of the same
+// phase reads back: across phases, the named barriers and mbarrier arrivals (whose
+// asm clobbers memory) order them.
+__device__ __forceinline__ void st_shared_f4(const void *p, float a, float b, float c, float d) {
+  asm volatile("st.shared.v4.f32 [%0], {%1, %2, %3, %4};" ::"r"(smem_u32(p)), "f"(a), "f"(b),
+               "f"(c), "f"(d));
+}
+__device__ __forceinline__ void st_shared_f1(const void *p, float a) {
+  asm volatile("st.shared.f32 [%0], %1;" ::"r"(smem_u32(p)), "f"(a));
 }
 
 // Named barrier over the first `count` threads (a multiple of 32).

@@ -6,7 +6,9 @@ Builds the diagnostic library libkda_phase.so (the same sources compiled with
 KDA_PHASE_PROFILE: worker thread 0 of every CTA reads clock64 at each step of the
 chunk loop), runs the varlen prefill workload (64 requests, lengths log-uniform on
 [128, 4096], H=32, d=128, bf16 q/k/v, fp32 g, beta and o) through it, and prints
-the mean cycles per 32-token chunk of each step with its share.  The counters
+the mean cycles per 32-token chunk of each step of both worker groups (group A:
+gate, row operands, A|P read-out, solve; group B: state scaling, Khat^T, outputs,
+V^T), each with its share of the group's time.  The counters
 perturb the timing slightly; the table shows where a chunk's time goes, the
 bench measures how long it takes.  Needs a CUDA device.
 """
@@ -16,10 +18,12 @@ import argparse
 import ctypes
 import json
 
-PHASES = ("chunk 0 operands", "wait: next tiles", "gate (cumulative)", "wait: O^T, Y^T",
-          "scale S^T", "rows (L, R', gamma Q/K)", "wait: last products", "Khat^T",
-          "out (o, snapshots)", "wait: A|P", "read (A, P, V^T)", "solve (T Diag(beta))",
-          "final state")
+# group A (worker thread 0) and group B (worker thread 256) steps, by counter slot
+PHASES = {0: "A wait: O^T, Y^T of chunk m-1", 1: "A wait: tiles", 2: "A gate (cumulative)",
+          3: "A rows (L, R', gamma Q/K)", 4: "A wait: A|P", 5: "A read (A, P)",
+          6: "A solve (T Diag(beta))",
+          8: "B wait: O^T, Y^T", 9: "B scale S^T", 10: "B wait: next gate", 11: "B Khat^T",
+          12: "B wait: last products", 13: "B out (o, snapshots)", 14: "B V^T"}
 
 
 def main():
@@ -52,14 +56,17 @@ def main():
     torch.cuda.synchronize()
     assert lib.kda_phase_cycles(buf, 16, 0) == 0
     chunks = buf[15]
-    total = sum(buf[k] for k in range(len(PHASES)))
-    rows = [{"phase": name, "cycles_per_chunk": buf[k] / chunks, "share": buf[k] / total}
-            for k, name in enumerate(PHASES)]
-    print(f"{chunks // args.steps} chunks of 32 tokens per call; "
-          f"{total / chunks:.0f} cycles per chunk (worker thread 0)")
-    for rw in rows:
-        print(f"  {rw['phase']:<28} {rw['cycles_per_chunk']:8.0f}  {100 * rw['share']:5.1f} %")
-    print(json.dumps({"cycles_per_chunk": total / chunks, "phases": rows}))
+    out = {}
+    print(f"{chunks // args.steps} chunks of 32 tokens per call")
+    for grp, slots in (("A", range(0, 7)), ("B", range(8, 15))):
+        total = sum(buf[k] for k in slots)
+        print(f"group {grp}: {total / chunks:.0f} cycles per chunk")
+        rows = [{"phase": PHASES[k], "cycles_per_chunk": buf[k] / chunks,
+                 "share": buf[k] / total if total else 0.0} for k in slots]
+        for rw in rows:
+            print(f"  {rw['phase']:<32} {rw['cycles_per_chunk']:8.0f}  {100 * rw['share']:5.1f} %")
+        out[grp] = {"cycles_per_chunk": total / chunks, "phases": rows}
+    print(json.dumps(out))
 
 
 if __name__ == "__main__":
