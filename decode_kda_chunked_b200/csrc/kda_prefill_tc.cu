@@ -55,6 +55,7 @@ namespace {
 
 using namespace sm100;
 
+
 constexpr int C = 32;     // tokens per chunk of this kernel
 constexpr int DH = 128;   // head dim (dk = dv)
 constexpr int NT = 512;   // worker threads per CTA: 16 warps (plus one control warp)
@@ -417,8 +418,8 @@ __global__ void __launch_bounds__(NT + 64, 1)
     // ============ group A (warps 0-7): gate, row operands, read-out, solve ============
     uint32_t ph_tma = 0u, ph_ap = 0, ph_oy = 0;  // ph_tma: bit b for buffer b
     auto wsync = [&]() { named_sync(1, NA); };
-    // every thread of the group waits, then all of them vote, so an abort is taken
-    // by all together
+    // thread 0 waits for the group while the others block at the named barrier; the
+    // vote there gives every thread the outcome, so an abort is taken by all together
     auto wwait = [&](uint64_t *bar, uint32_t &ph) -> bool {
       const bool got = mbar_wait(bar, ph, wait_ns, s_abort);
       ph ^= 1u;
@@ -504,50 +505,67 @@ __global__ void __launch_bounds__(NT + 64, 1)
     // lane quarter 1: L_q = q exp(G_i - G_15) -> TMEM lanes 32-63, gamma*Q = L_q exp(G_15)
     // lane quarter 2: R'  = k exp(G_15 - G_i) -> smem
     // lane quarter 3: gamma*K = k exp(G_i)    -> smem
+    // (one straight-line loop per quarter, so that loads issue ahead of the stores)
     auto w_rows = [&](int m) {
       const int nr = min(C, len - m * C);
       const unsigned char *raw = sm + OFF_RAW + (m & 1) * RAW_BYTES;
       const int i = lane_id;
       const bool valid = i < nr;
       const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
-      if (qd == 1 && !has_q) return;
-      const unsigned char *xr = raw + (qd == 1 ? R_Q : R_K);
-      unsigned char *dst = sm + (qd == 1 ? OFF_GQ : qd == 2 ? OFF_RP : OFF_GK);
-#pragma unroll 2
-      for (int jj = 0; jj < 8; ++jj) {
-        const int c = 64 * cg + 8 * jj;
-        float x[8], g[8], y[8];
-        bf16_x8(valid ? *reinterpret_cast<const uint4 *>(xr + bf16_chunk(i, c)) : z4, x);
-        ld8f(GT + i * LDG + c, g);
-        if (qd == 3) {
+      const float *gi = GT + i * LDG + 64 * cg;
+      const float *gm = GT + MREF * LDG + 64 * cg;
+      auto load_x = [&](uint32_t tile, int c) {
+        return valid ? *reinterpret_cast<const uint4 *>(raw + tile + bf16_chunk(i, c)) : z4;
+      };
+      if (qd <= 1) {  // L = x exp(G_i - G_15) -> TMEM; lane quarter 1 also gamma*Q
+        if (qd == 1 && !has_q) return;
+        const uint32_t tile = qd == 0 ? R_K : R_Q;
+#pragma unroll 1
+        for (int jj = 0; jj < 8; ++jj) {
+          const int c = 64 * cg + 8 * jj;
+          float x[8], g[8], gr[8], lv[8];
+          bf16_x8(load_x(tile, c), x);
+          ld8f(gi + 8 * jj, g);
+          ld8f(gm + 8 * jj, gr);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) y[e] = tf32_rna(x[e] * ex2(g[e]));
-        } else {
-          float gr[8];
-          ld8f(GT + MREF * LDG + c, gr);
-          if (qd == 2) {
+          for (int e = 0; e < 8; ++e) {
+            x[e] *= ex2(g[e] - gr[e]);
+            lv[e] = tf32_rna(x[e]);
+          }
+          tmem_st8(tm + lane_base + TM_L + c, lv);
+          if (qd == 1) {
+            float e15[8];
+            ld8f(E15 + c, e15);
 #pragma unroll
-            for (int e = 0; e < 8; ++e) y[e] = tf32_rna(x[e] * ex2(gr[e] - g[e]));
-          } else {
-            float lv[8];
-#pragma unroll
-            for (int e = 0; e < 8; ++e) {
-              const float a = x[e] * ex2(g[e] - gr[e]);
-              lv[e] = tf32_rna(a);
-              y[e] = a;
-            }
-            tmem_st8(tm + lane_base + TM_L + c, lv);
-            if (qd == 1) {
-              float e15[8];
-              ld8f(E15 + c, e15);
-#pragma unroll
-              for (int e = 0; e < 8; ++e) y[e] = tf32_rna(y[e] * e15[e]);
-            }
+            for (int e = 0; e < 8; ++e) x[e] = tf32_rna(x[e] * e15[e]);
+            st8f(sm + OFF_GQ, sw128_chunk(C, i, c), sw128_chunk(C, i, c + 4), x);
           }
         }
-        if (qd != 0) st8f(dst, sw128_chunk(C, i, c), sw128_chunk(C, i, c + 4), y);
+        tmem_wait_st();
+      } else if (qd == 2) {  // R' = k exp(G_15 - G_i)
+#pragma unroll 1
+        for (int jj = 0; jj < 8; ++jj) {
+          const int c = 64 * cg + 8 * jj;
+          float x[8], g[8], gr[8];
+          bf16_x8(load_x(R_K, c), x);
+          ld8f(gi + 8 * jj, g);
+          ld8f(gm + 8 * jj, gr);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) x[e] = tf32_rna(x[e] * ex2(gr[e] - g[e]));
+          st8f(sm + OFF_RP, sw128_chunk(C, i, c), sw128_chunk(C, i, c + 4), x);
+        }
+      } else {  // gamma*K = k exp(G_i)
+#pragma unroll 1
+        for (int jj = 0; jj < 8; ++jj) {
+          const int c = 64 * cg + 8 * jj;
+          float x[8], g[8];
+          bf16_x8(load_x(R_K, c), x);
+          ld8f(gi + 8 * jj, g);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) x[e] = tf32_rna(x[e] * ex2(g[e]));
+          st8f(sm + OFF_GK, sw128_chunk(C, i, c), sw128_chunk(C, i, c + 4), x);
+        }
       }
-      if (qd <= 1) tmem_wait_st();
     };
 
     // ---- read(m): Diag(beta) A and P out of TMEM (after the A|P products) ----
@@ -661,7 +679,7 @@ __global__ void __launch_bounds__(NT + 64, 1)
   } else {
     // ====== group B (warps 8-15): state scaling, Khat^T, outputs, V^T, states ======
     uint32_t ph_oy = 0, ph_gate = 0, ph_fin = 0;
-    // every thread of the group waits, then all of them vote at the group's barrier
+    // thread 256 waits for the group while the others block at the group's barrier
     auto bwait = [&](uint64_t *bar, uint32_t &ph) -> bool {
       const bool got = mbar_wait(bar, ph, wait_ns, s_abort);
       ph ^= 1u;

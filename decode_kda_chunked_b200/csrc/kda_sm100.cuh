@@ -271,41 +271,6 @@ __device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t parity,
   }
 }
 
-// Non-blocking test of a phase (no suspension).
-__device__ __forceinline__ bool mbar_test_wait(uint64_t *bar, uint32_t parity) {
-  uint32_t ok;
-  asm volatile(
-      "{\n\t.reg .pred p;\n\t"
-      "mbarrier.test_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-      "selp.u32 %0, 1, 0, p;\n\t}"
-      : "=r"(ok)
-      : "r"(smem_u32(bar)), "r"(parity)
-      : "memory");
-  return ok != 0;
-}
-
-// The bounded wait for a thread that waits on behalf of others (its group then
-// learns the outcome at a named barrier, where waiting costs no instructions):
-// non-blocking tests with a short sleep between them (32 ns doubling up to
-// max_sleep_ns), the abort flag and the clock read only every 8 tries.
-__device__ __forceinline__ bool mbar_wait_lean(uint64_t *bar, uint32_t parity,
-                                               uint64_t timeout_ns,
-                                               const volatile int *abort_flag,
-                                               uint32_t max_sleep_ns = 128u) {
-  if (mbar_test_wait(bar, parity)) return true;
-  const uint64_t t0 = global_ns();
-  uint32_t ns = 32u;
-  for (uint32_t i = 1;; ++i) {
-    __nanosleep(ns);
-    if (mbar_test_wait(bar, parity)) return true;
-    if ((i & 7u) == 0u) {
-      if (abort_flag && *abort_flag) return false;
-      if (global_ns() - t0 > timeout_ns) return false;
-    }
-    ns = ns < max_sleep_ns ? 2u * ns : max_sleep_ns;
-  }
-}
-
 // Plain arrive (count 1) on an mbarrier.
 __device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
