@@ -70,28 +70,26 @@ constexpr float LOG2E = 1.4426950408889634f;
 constexpr uint32_t RAW_BYTES = 40960;
 constexpr uint32_t R_K = 0, R_Q = 8192, R_V = 16384, R_G = 24576;
 constexpr uint32_t OFF_RAW = 0;
-constexpr uint32_t OFF_GT = 81920;   // log2(e) * G (chunk-local cumulative gate), fp32 [32][LDG]
-constexpr int LDG = 132;             // padded so that row-wise float4 reads hit distinct banks
-constexpr uint32_t OFF_GQ = 99328;   // gamma*Q  tf32 B operand [32 x 128]
-constexpr uint32_t OFF_GK = 115712;  // gamma*K  tf32 B operand [32 x 128]
-constexpr uint32_t OFF_KH = 132096;  // Khat^T   tf32 B operand [128 x 32], x2 (chunk parity)
-constexpr uint32_t OFF_RP = 164864;  // R'       tf32 B operand [32 x 128]
-constexpr uint32_t OFF_PP = 181248;  // P        tf32 B operand [32 x 32], x2
-constexpr uint32_t OFF_TB = 189440;  // T Diag(beta) tf32 B operand [32 x 32], x2
-constexpr uint32_t OFF_NS = 197632;  // Diag(beta) A, strict lower, fp32 [32][LDN]
+// The chunk-local cumulative gate, log2(e) * G, replaces the raw g tile in place (fp32,
+// the same four swizzled boxes), so each raw buffer carries its chunk's gate table.
+constexpr uint32_t OFF_GQ = 81920;   // gamma*Q  tf32 B operand [32 x 128]
+constexpr uint32_t OFF_GK = 98304;   // gamma*K  tf32 B operand [32 x 128]
+constexpr uint32_t OFF_KH = 114688;  // Khat^T   tf32 B operand [128 x 32], x2 (chunk parity)
+constexpr uint32_t OFF_RP = 147456;  // R'       tf32 B operand [32 x 128]
+constexpr uint32_t OFF_PP = 163840;  // P        tf32 B operand [32 x 32], x2
+constexpr uint32_t OFF_TB = 172032;  // T Diag(beta) tf32 B operand [32 x 32], x2
+constexpr uint32_t OFF_NS = 180224;  // Diag(beta) A, strict lower, fp32 [32][LDN]
 constexpr int LDN = 36;
-constexpr uint32_t OFF_TS = 202240;  // the two diagonal 16x16 blocks of T, fp32 [32][LDN]
-constexpr uint32_t OFF_XS = 206848;  // N10 T00, fp32 [16][LDX]
+constexpr uint32_t OFF_TS = 184832;  // the two diagonal 16x16 blocks of T, fp32 [32][LDN]
+constexpr uint32_t OFF_XS = 189440;  // N10 T00, fp32 [16][LDX]
 constexpr int LDX = 20;
-constexpr uint32_t OFF_GC = 208128;  // exp(G_31) per key channel, [2][128] (chunk parity)
-constexpr uint32_t OFF_E15 = 209152; // exp(G_15) per key channel [128]
-constexpr uint32_t OFF_BT = 209664;  // beta of the chunk group A prepares [32]
-constexpr uint32_t OFF_SEG = 209792; // cumulative-gate segment totals [2][128]
-constexpr uint32_t OFF_BAR = 210816; // mbarriers, TMEM base, flags (+ phase counters)
-constexpr uint32_t SMEM_BYTES = 211072;
+constexpr uint32_t OFF_GC = 190720;  // exp(G_31) per key channel, [4][128] (chunk index mod 4)
+constexpr uint32_t OFF_BT = 192768;  // beta [2][32] (chunk parity)
+constexpr uint32_t OFF_SEG = 193024; // cumulative-gate segment totals [2][128]
+constexpr uint32_t OFF_BAR = 194048; // mbarriers, TMEM base, flags (+ phase counters)
+constexpr uint32_t SMEM_BYTES = 194304;
 constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;  // alignment slack
-static_assert(OFF_RAW + 2 * RAW_BYTES <= OFF_GT, "raw buffers");
-static_assert(OFF_GT + C * LDG * 4 <= OFF_GQ, "gate table");
+static_assert(OFF_RAW + 2 * RAW_BYTES == OFF_GQ, "raw buffers");
 static_assert(OFF_GQ % 1024 == 0 && OFF_GK % 1024 == 0 && OFF_KH % 1024 == 0 &&
                   OFF_RP % 1024 == 0 && OFF_PP % 1024 == 0 && OFF_TB % 1024 == 0,
               "swizzled operands need 1024-byte alignment");
@@ -100,8 +98,8 @@ static_assert(OFF_GQ + 16384 == OFF_GK && OFF_GK + 16384 == OFF_KH &&
                   OFF_PP + 2 * 4096 == OFF_TB && OFF_TB + 2 * 4096 == OFF_NS,
               "operand tiles");
 static_assert(OFF_NS + C * LDN * 4 == OFF_TS && OFF_TS + C * LDN * 4 == OFF_XS &&
-                  OFF_XS + 16 * LDX * 4 == OFF_GC && OFF_GC + 2 * DH * 4 == OFF_E15 &&
-                  OFF_E15 + DH * 4 == OFF_BT && OFF_BT + C * 4 == OFF_SEG &&
+                  OFF_XS + 16 * LDX * 4 == OFF_GC && OFF_GC + 4 * DH * 4 == OFF_BT &&
+                  OFF_BT + 2 * C * 4 == OFF_SEG &&
                   OFF_SEG + 2 * DH * 4 == OFF_BAR,
               "scratch tiles");
 __host__ __device__ constexpr uint32_t kh_off(int m) { return OFF_KH + 16384u * (m & 1); }
@@ -144,6 +142,12 @@ __device__ __forceinline__ uint32_t f32_off(int t, int c) {
   return (uint32_t)(c >> 5) * 4096u + (uint32_t)t * 128u +
          ((uint32_t)(((c & 31) >> 2) ^ (t & 7)) << 4) + (uint32_t)(c & 3) * 4u;
 }
+// eight consecutive channels c..c+7 (c % 8 == 0) of row t of an fp32 tile in that layout
+__device__ __forceinline__ void ld8g(const unsigned char *tile, int t, int c, float *x) {
+  const float4 a = *reinterpret_cast<const float4 *>(tile + f32_off(t, c));
+  const float4 b = *reinterpret_cast<const float4 *>(tile + f32_off(t, c + 4));
+  x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
+}
 __device__ __forceinline__ float tf32_rna(float x) {
   uint32_t r;
   asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
@@ -163,10 +167,10 @@ __device__ __forceinline__ void st8f(unsigned char *base, uint32_t off_lo, uint3
 
 #ifdef KDA_PHASE_PROFILE
 // Cycles per step of the loops, summed over every CTA (profiling builds only):
-// group A (thread 0): 0 wait for O^T/Y^T(m-1), 1 wait for the tiles, 2 gate, 3 rows,
-// 4 wait for A|P, 5 read, 6 solve;  group B (thread 256): 8 wait for O^T/Y^T(n),
-// 9 scale, 10 wait for the next gate, 11 Khat^T, 12 wait for the last products,
-// 13 out, 14 V^T.  Entry 15 counts the chunks.
+// group A (thread 0): 0 wait for O^T/Y^T(m-1), 1 wait for group B's Khat^T(m) and the
+// tiles of chunk m+1, 2 gate(m+1), 3 rows(m), 4 wait for A|P(m), 5 read, 6 solve;
+// group B (thread 256): 8 wait for O^T/Y^T(n), 9 scale, 10 wait for the next gate,
+// 11 Khat^T, 12 wait for the last products, 13 out, 14 V^T.  Entry 15 counts the chunks.
 __device__ unsigned long long g_phase_cycles[16];
 #define KDA_PHASE(k)                                              \
   do {                                                            \
@@ -188,12 +192,10 @@ __global__ void __launch_bounds__(NT + 64, 1)
     prefill_tc_kernel(const PrefillParams p, const __grid_constant__ TcMaps maps) {
   extern __shared__ unsigned char smem_raw[];
   unsigned char *sm = align1024_shared(smem_raw);
-  float *GT = reinterpret_cast<float *>(sm + OFF_GT);
   float *NS = reinterpret_cast<float *>(sm + OFF_NS);
   float *TS = reinterpret_cast<float *>(sm + OFF_TS);
   float *XS = reinterpret_cast<float *>(sm + OFF_XS);
   float *GC = reinterpret_cast<float *>(sm + OFF_GC);
-  float *E15 = reinterpret_cast<float *>(sm + OFF_E15);
   float *BT = reinterpret_cast<float *>(sm + OFF_BT);
   float *SEG = reinterpret_cast<float *>(sm + OFF_SEG);
   uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
@@ -208,7 +210,8 @@ __global__ void __launch_bounds__(NT + 64, 1)
   uint64_t *ops_tb = bars + 9;    // group A -> control: T Diag(beta) ready
   uint64_t *ops_sc = bars + 10;   // group B -> control: S^T scaled by gamma_31
   uint64_t *gate_ok = bars + 11;  // group A -> group B: cumulative gate of a chunk ready
-  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bars + 12);
+  uint64_t *khat_done = bars + 12;  // group B -> group A: a chunk's gate table read
+  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bars + 13);
   volatile int *s_abort = reinterpret_cast<volatile int *>(s_tmem + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane_id = tid & 31;
@@ -257,6 +260,7 @@ __global__ void __launch_bounds__(NT + 64, 1)
     mbar_init(ops_tb, NA / 32);
     mbar_init(ops_sc, (NT - NA) / 32);
     mbar_init(gate_ok, NA / 32);
+    mbar_init(khat_done, (NT - NA) / 32);
     *s_abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -416,7 +420,7 @@ __global__ void __launch_bounds__(NT + 64, 1)
     }
   } else if (group_a) {
     // ============ group A (warps 0-7): gate, row operands, read-out, solve ============
-    uint32_t ph_tma = 0u, ph_ap = 0, ph_oy = 0;  // ph_tma: bit b for buffer b
+    uint32_t ph_tma = 0u, ph_ap = 0, ph_oy = 0, ph_kd = 0;  // ph_tma: bit b for buffer b
     auto wsync = [&]() { named_sync(1, NA); };
     // thread 0 waits for the group while the others block at the named barrier; the
     // vote there gives every thread the outcome, so an abort is taken by all together
@@ -461,11 +465,11 @@ __global__ void __launch_bounds__(NT + 64, 1)
     // ---- gate(m): cumulative gate (thread = channel l, tokens 16 cg .. 16 cg + 15) ----
     auto w_gate = [&](int m) {
       const int nr = min(C, len - m * C);
-      const unsigned char *raw = sm + OFF_RAW + (m & 1) * RAW_BYTES;
+      unsigned char *raw = sm + OFF_RAW + (m & 1) * RAW_BYTES;
       if (tid < C) {
         if (p.validate && !(beta_pref >= 0.f && beta_pref <= 1.f))
           set_status(p.status, STATUS_GATE_RANGE);
-        BT[tid] = beta_pref;
+        BT[(m & 1) * C + tid] = beta_pref;
       }
       beta_pref = load_beta(m + 1);
       // every row of the tile is loaded (rows past the chunk's end hold other data or the
@@ -493,8 +497,8 @@ __global__ void __launch_bounds__(NT + 64, 1)
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
         const float g2 = (gv[j] + off) * LOG2E;
-        GT[(16 * cg + j) * LDG + l] = g2;
-        if (j == 15) (cg ? GC + (m & 1) * DH : E15)[l] = ex2(g2);
+        *reinterpret_cast<float *>(raw + R_G + f32_off(16 * cg + j, l)) = g2;
+        if (cg == 1 && j == 15) GC[(m & 3) * DH + l] = ex2(g2);
       }
       wsync();
       warp_signal(gate_ok);
@@ -502,9 +506,9 @@ __global__ void __launch_bounds__(NT + 64, 1)
 
     // ---- rows(m): the row operands (thread = row i, channels 64 cg .. 64 cg + 63) ----
     // lane quarter 0: L_k = k exp(G_i - G_15) -> TMEM lanes 0-31
-    // lane quarter 1: L_q = q exp(G_i - G_15) -> TMEM lanes 32-63, gamma*Q = L_q exp(G_15)
+    // lane quarter 1: L_q = q exp(G_i - G_15) -> TMEM lanes 32-63
     // lane quarter 2: R'  = k exp(G_15 - G_i) -> smem
-    // lane quarter 3: gamma*K = k exp(G_i)    -> smem
+    // lane quarter 3: gamma*Q = q exp(G_i)    -> smem  (gamma*K: group B, with Khat^T)
     // (one straight-line loop per quarter, so that loads issue ahead of the stores)
     auto w_rows = [&](int m) {
       const int nr = min(C, len - m * C);
@@ -512,34 +516,23 @@ __global__ void __launch_bounds__(NT + 64, 1)
       const int i = lane_id;
       const bool valid = i < nr;
       const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
-      const float *gi = GT + i * LDG + 64 * cg;
-      const float *gm = GT + MREF * LDG + 64 * cg;
+      const unsigned char *gt = raw + R_G;  // the chunk's gate table (see gate)
       auto load_x = [&](uint32_t tile, int c) {
         return valid ? *reinterpret_cast<const uint4 *>(raw + tile + bf16_chunk(i, c)) : z4;
       };
-      if (qd <= 1) {  // L = x exp(G_i - G_15) -> TMEM; lane quarter 1 also gamma*Q
+      if (qd <= 1) {  // L = x exp(G_i - G_15) -> TMEM lanes 32 qd + i
         if (qd == 1 && !has_q) return;
         const uint32_t tile = qd == 0 ? R_K : R_Q;
 #pragma unroll 1
         for (int jj = 0; jj < 8; ++jj) {
           const int c = 64 * cg + 8 * jj;
-          float x[8], g[8], gr[8], lv[8];
+          float x[8], g[8], gr[8];
           bf16_x8(load_x(tile, c), x);
-          ld8f(gi + 8 * jj, g);
-          ld8f(gm + 8 * jj, gr);
+          ld8g(gt, i, c, g);
+          ld8g(gt, MREF, c, gr);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) {
-            x[e] *= ex2(g[e] - gr[e]);
-            lv[e] = tf32_rna(x[e]);
-          }
-          tmem_st8(tm + lane_base + TM_L + c, lv);
-          if (qd == 1) {
-            float e15[8];
-            ld8f(E15 + c, e15);
-#pragma unroll
-            for (int e = 0; e < 8; ++e) x[e] = tf32_rna(x[e] * e15[e]);
-            st8f(sm + OFF_GQ, sw128_chunk(C, i, c), sw128_chunk(C, i, c + 4), x);
-          }
+          for (int e = 0; e < 8; ++e) x[e] = tf32_rna(x[e] * ex2(g[e] - gr[e]));
+          tmem_st8(tm + lane_base + TM_L + c, x);
         }
         tmem_wait_st();
       } else if (qd == 2) {  // R' = k exp(G_15 - G_i)
@@ -548,22 +541,22 @@ __global__ void __launch_bounds__(NT + 64, 1)
           const int c = 64 * cg + 8 * jj;
           float x[8], g[8], gr[8];
           bf16_x8(load_x(R_K, c), x);
-          ld8f(gi + 8 * jj, g);
-          ld8f(gm + 8 * jj, gr);
+          ld8g(gt, i, c, g);
+          ld8g(gt, MREF, c, gr);
 #pragma unroll
           for (int e = 0; e < 8; ++e) x[e] = tf32_rna(x[e] * ex2(gr[e] - g[e]));
           st8f(sm + OFF_RP, sw128_chunk(C, i, c), sw128_chunk(C, i, c + 4), x);
         }
-      } else {  // gamma*K = k exp(G_i)
+      } else if (has_q) {  // gamma*Q = q exp(G_i)
 #pragma unroll 1
         for (int jj = 0; jj < 8; ++jj) {
           const int c = 64 * cg + 8 * jj;
           float x[8], g[8];
-          bf16_x8(load_x(R_K, c), x);
-          ld8f(gi + 8 * jj, g);
+          bf16_x8(load_x(R_Q, c), x);
+          ld8g(gt, i, c, g);
 #pragma unroll
           for (int e = 0; e < 8; ++e) x[e] = tf32_rna(x[e] * ex2(g[e]));
-          st8f(sm + OFF_GK, sw128_chunk(C, i, c), sw128_chunk(C, i, c + 4), x);
+          st8f(sm + OFF_GQ, sw128_chunk(C, i, c), sw128_chunk(C, i, c + 4), x);
         }
       }
     };
@@ -575,7 +568,7 @@ __global__ void __launch_bounds__(NT + 64, 1)
         float a[16];
         tmem_ld16(tm + lane_base + TM_AP + 16 * cg, a);
         tmem_wait_ld();
-        const float bi = BT[i];
+        const float bi = BT[(m & 1) * C + i];
 #pragma unroll
         for (int e = 0; e < 16; ++e) a[e] = (16 * cg + e < i) ? bi * a[e] : 0.f;
         float4 *nd = reinterpret_cast<float4 *>(NS + i * LDN + 16 * cg);
@@ -623,7 +616,7 @@ __global__ void __launch_bounds__(NT + 64, 1)
           }
           t[i] = acc0 + acc1;
         }
-        const float bc = BT[o + c];
+        const float bc = BT[(m & 1) * C + o + c];
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           TS[(o + i) * LDN + o + c] = t[i];
@@ -649,24 +642,31 @@ __global__ void __launch_bounds__(NT + 64, 1)
           y0 += TS[(16 + i) * LDN + 16 + j] * XS[j * LDX + c];
           y1 += TS[(16 + i) * LDN + 24 + j] * XS[(8 + j) * LDX + c];
         }
-        st_shared_f1(tb + sw128_offset(C, 16 + i, c), tf32_rna(-(y0 + y1) * BT[c]));
+        st_shared_f1(tb + sw128_offset(C, 16 + i, c), tf32_rna(-(y0 + y1) * BT[(m & 1) * C + c]));
       }
     };
 
+    // The gate of chunk m+1 runs while the A|P products of chunk m do (its table sits in
+    // chunk m+1's own raw buffer); it waits until group B has read chunk m's table, so
+    // that group A is never two gates ahead.
     bool ok = true;
+    if (n_chunks > 0 && (ok = wait_tma(0))) w_gate(0);
     for (int m = 0; ok && m < n_chunks; ++m) {
-      // chunk m-1's O^T and Y^T products are done: gamma*Q/K and the gate tables are free
-      // (and, through group B, chunk m-2's last products are done too)
+      // chunk m-1's O^T and Y^T products are done: gamma*Q/K are free (and, through
+      // group B, chunk m-2's last products are done too)
       if (m > 0 && !(ok = wwait(bar_oy, ph_oy))) break;
       KDA_PHASE(0);
-      if (!(ok = wait_tma(m))) break;
-      KDA_PHASE(1);
-      w_gate(m);
-      KDA_PHASE(2);
       w_rows(m);
       warp_signal(raw_free);
       warp_arrive(ops_ap);
       KDA_PHASE(3);
+      if (m + 1 < n_chunks) {
+        if (!(ok = wwait(khat_done, ph_kd))) break;
+        if (!(ok = wait_tma(m + 1))) break;
+        KDA_PHASE(1);
+        w_gate(m + 1);
+        KDA_PHASE(2);
+      }
       if (!(ok = wwait(bar_ap, ph_ap))) break;
       KDA_PHASE(4);
       w_read(m);
@@ -712,7 +712,7 @@ __global__ void __launch_bounds__(NT + 64, 1)
 
     // ---- scale(n): S^T <- S^T Diag(gamma_31) once the O^T and Y^T products read S^T ----
     auto w_scale = [&](int n) {
-      const float *gc = GC + (n & 1) * DH;
+      const float *gc = GC + (n & 3) * DH;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
         const int c0 = 64 * cg + 16 * q;
@@ -731,7 +731,9 @@ __global__ void __launch_bounds__(NT + 64, 1)
       tmem_wait_st();
     };
 
-    // ---- khat(m): Khat^T = (k exp(G_31 - G))^T (thread = row i, channels 16 w8 ..) ----
+    // ---- khat(m): Khat^T = (k exp(G_31 - G))^T and gamma*K = k exp(G), one pass over k
+    // (thread = row i, channels 16 w8 ..); gamma*K's tile is free once O^T, Y^T(m-1)
+    // are done, which precedes this ----
     auto w_khat = [&](int m) {
       const int nr = min(C, len - m * C);
       const unsigned char *raw = sm + OFF_RAW + (m & 1) * RAW_BYTES;
@@ -740,15 +742,18 @@ __global__ void __launch_bounds__(NT + 64, 1)
 #pragma unroll
       for (int u = 0; u < 2; ++u) {
         const int c = 16 * w8 + 8 * u;
-        float x[8], g[8], ge[8];
+        float x[8], g[8], ge[8], gk[8];
         bf16_x8(i < nr ? *reinterpret_cast<const uint4 *>(raw + R_K + bf16_chunk(i, c))
                        : make_uint4(0u, 0u, 0u, 0u),
                 x);
-        ld8f(GT + i * LDG + c, g);
-        ld8f(GT + (C - 1) * LDG + c, ge);
+        ld8g(raw + R_G, i, c, g);
+        ld8g(raw + R_G, C - 1, c, ge);
 #pragma unroll
-        for (int e = 0; e < 8; ++e)
+        for (int e = 0; e < 8; ++e) {
           st_shared_f1(kh + sw128_offset(DH, c + e, i), tf32_rna(x[e] * ex2(ge[e] - g[e])));
+          gk[e] = tf32_rna(x[e] * ex2(g[e]));
+        }
+        st8f(sm + OFF_GK, sw128_chunk(C, i, c), sw128_chunk(C, i, c + 4), gk);
       }
     };
 
@@ -798,6 +803,7 @@ __global__ void __launch_bounds__(NT + 64, 1)
     if (n_chunks > 0) {
       if ((ok = bwait(gate_ok, ph_gate))) {
         w_khat(0);
+        warp_signal(khat_done);
         w_vt(0);
         warp_signal(raw_free);
         warp_arrive(ops_oy);
@@ -814,6 +820,7 @@ __global__ void __launch_bounds__(NT + 64, 1)
         if (!(ok = bwait(gate_ok, ph_gate))) break;
         KDA_PHASE(10);
         w_khat(n + 1);  // the other Khat^T buffer: chunk n-1's last products are done
+        warp_signal(khat_done);
         KDA_PHASE(11);
       }
       if (!(ok = bwait(bar_fin, ph_fin))) break;

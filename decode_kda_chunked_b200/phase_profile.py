@@ -19,7 +19,8 @@ import ctypes
 import json
 
 # group A (worker thread 0) and group B (worker thread 256) steps, by counter slot
-PHASES = {0: "A wait: O^T, Y^T of chunk m-1", 1: "A wait: tiles", 2: "A gate (cumulative)",
+PHASES = {0: "A wait: O^T, Y^T of chunk m-1", 1: "A wait: Khat^T(m), tiles(m+1)",
+          2: "A gate (cumulative) of m+1",
           3: "A rows (L, R', gamma Q/K)", 4: "A wait: A|P", 5: "A read (A, P)",
           6: "A solve (T Diag(beta))",
           8: "B wait: O^T, Y^T", 9: "B scale S^T", 10: "B wait: next gate", 11: "B Khat^T",
