@@ -287,9 +287,10 @@ struct PrepLayout {
 template <int D, typename TIn>
 constexpr bool kPrepTensorCores = D == 128 && std::is_same<TIn, __nv_bfloat16>::value;
 
+// fp32 -> tf32, round to nearest even (the tensor cores read the 19 leading bits)
 __device__ __forceinline__ float tf32_round(float x) {
   uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  asm("cvt.rn.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
   return __uint_as_float(r);
 }
 

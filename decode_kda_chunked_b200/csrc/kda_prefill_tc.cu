@@ -25,7 +25,7 @@
 // that is flushed to zero only where the true value is below FLT_MIN.
 //
 // All tensor-core operands are tf32 (B operands K-major with the 128-byte swizzle in
-// shared memory, rounded to nearest): bf16 operands for the gate-scaled products
+// shared memory, rounded to nearest even): bf16 operands for the gate-scaled products
 // would cost about 2e-3 of relative accuracy, tf32 stays near 5e-4.
 //
 // Warp roles.  One CTA runs one (request, head) chain: two control warps issue every
@@ -148,9 +148,10 @@ __device__ __forceinline__ void ld8g(const unsigned char *tile, int t, int c, fl
   const float4 b = *reinterpret_cast<const float4 *>(tile + f32_off(t, c + 4));
   x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
 }
-__device__ __forceinline__ float tf32_rna(float x) {
+// fp32 -> tf32, round to nearest even (the tensor cores read the 19 leading bits)
+__device__ __forceinline__ float tf32_rn(float x) {
   uint32_t r;
-  asm("cvt.rna.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
+  asm("cvt.rn.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
   return __uint_as_float(r);
 }
 __device__ __forceinline__ void ld8f(const float *p, float *x) {
@@ -206,7 +207,7 @@ __global__ void __launch_bounds__(NT + 64, 1)
   uint64_t *bar_fin = bars + 5;   // commit: the chunk's last products done
   uint64_t *ops_ap = bars + 6;    // group A -> control: A|P operands built
   uint64_t *raw_free = bars + 7;  // A and B -> control: a raw buffer fully read
-  uint64_t *ops_oy = bars + 8;    // A (P, gamma*Q/K) and B (Khat^T, V^T) -> control
+  uint64_t *ops_oy = bars + 8;    // A (gamma*Q) and B (gamma*K, V^T) -> control
   uint64_t *ops_tb = bars + 9;    // group A -> control: T Diag(beta) ready
   uint64_t *ops_sc = bars + 10;   // group B -> control: S^T scaled by gamma_31
   uint64_t *gate_ok = bars + 11;  // group A -> group B: cumulative gate of a chunk ready
@@ -531,7 +532,7 @@ __global__ void __launch_bounds__(NT + 64, 1)
           ld8g(gt, i, c, g);
           ld8g(gt, MREF, c, gr);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) x[e] = tf32_rna(x[e] * ex2(g[e] - gr[e]));
+          for (int e = 0; e < 8; ++e) x[e] = tf32_rn(x[e] * ex2(g[e] - gr[e]));
           tmem_st8(tm + lane_base + TM_L + c, x);
         }
         tmem_wait_st();
@@ -544,7 +545,7 @@ __global__ void __launch_bounds__(NT + 64, 1)
           ld8g(gt, i, c, g);
           ld8g(gt, MREF, c, gr);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) x[e] = tf32_rna(x[e] * ex2(gr[e] - g[e]));
+          for (int e = 0; e < 8; ++e) x[e] = tf32_rn(x[e] * ex2(gr[e] - g[e]));
           st8f(sm + OFF_RP, sw128_chunk(C, i, c), sw128_chunk(C, i, c + 4), x);
         }
       } else if (has_q) {  // gamma*Q = q exp(G_i)
@@ -555,7 +556,7 @@ __global__ void __launch_bounds__(NT + 64, 1)
           bf16_x8(load_x(R_Q, c), x);
           ld8g(gt, i, c, g);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) x[e] = tf32_rna(x[e] * ex2(g[e]));
+          for (int e = 0; e < 8; ++e) x[e] = tf32_rn(x[e] * ex2(g[e]));
           st8f(sm + OFF_GQ, sw128_chunk(C, i, c), sw128_chunk(C, i, c + 4), x);
         }
       }
@@ -579,7 +580,7 @@ __global__ void __launch_bounds__(NT + 64, 1)
         tmem_ld16(tm + lane_base + TM_AP + 16 * cg, a);
         tmem_wait_ld();
 #pragma unroll
-        for (int e = 0; e < 16; ++e) a[e] = (16 * cg + e <= i) ? tf32_rna(a[e]) : 0.f;
+        for (int e = 0; e < 16; ++e) a[e] = (16 * cg + e <= i) ? tf32_rn(a[e]) : 0.f;
         unsigned char *pp = sm + pp_off(m);
         st8f(pp, sw128_chunk(C, i, 16 * cg), sw128_chunk(C, i, 16 * cg + 4), a);
         st8f(pp, sw128_chunk(C, i, 16 * cg + 8), sw128_chunk(C, i, 16 * cg + 12), a + 8);
@@ -620,7 +621,7 @@ __global__ void __launch_bounds__(NT + 64, 1)
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           TS[(o + i) * LDN + o + c] = t[i];
-          st_shared_f1(tb + sw128_offset(C, o + i, o + c), tf32_rna(t[i] * bc));
+          st_shared_f1(tb + sw128_offset(C, o + i, o + c), tf32_rn(t[i] * bc));
         }
       }
       wsync();  // diagonal blocks ready
@@ -642,7 +643,7 @@ __global__ void __launch_bounds__(NT + 64, 1)
           y0 += TS[(16 + i) * LDN + 16 + j] * XS[j * LDX + c];
           y1 += TS[(16 + i) * LDN + 24 + j] * XS[(8 + j) * LDX + c];
         }
-        st_shared_f1(tb + sw128_offset(C, 16 + i, c), tf32_rna(-(y0 + y1) * BT[(m & 1) * C + c]));
+        st_shared_f1(tb + sw128_offset(C, 16 + i, c), tf32_rn(-(y0 + y1) * BT[(m & 1) * C + c]));
       }
     };
 
@@ -659,6 +660,7 @@ __global__ void __launch_bounds__(NT + 64, 1)
       w_rows(m);
       warp_signal(raw_free);
       warp_arrive(ops_ap);
+      warp_signal(ops_oy);  // gamma*Q made visible by the fence of the arrival above
       KDA_PHASE(3);
       if (m + 1 < n_chunks) {
         if (!(ok = wwait(khat_done, ph_kd))) break;
@@ -669,8 +671,7 @@ __global__ void __launch_bounds__(NT + 64, 1)
       }
       if (!(ok = wwait(bar_ap, ph_ap))) break;
       KDA_PHASE(4);
-      w_read(m);
-      warp_arrive(ops_oy);
+      w_read(m);  // P reaches the tensor cores after the solve's arrival (fence there)
       KDA_PHASE(5);
       w_solve(m);
       warp_arrive(ops_tb);
@@ -750,8 +751,8 @@ __global__ void __launch_bounds__(NT + 64, 1)
         ld8g(raw + R_G, C - 1, c, ge);
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          st_shared_f1(kh + sw128_offset(DH, c + e, i), tf32_rna(x[e] * ex2(ge[e] - g[e])));
-          gk[e] = tf32_rna(x[e] * ex2(g[e]));
+          st_shared_f1(kh + sw128_offset(DH, c + e, i), tf32_rn(x[e] * ex2(ge[e] - g[e])));
+          gk[e] = tf32_rn(x[e] * ex2(g[e]));
         }
         st8f(sm + OFF_GK, sw128_chunk(C, i, c), sw128_chunk(C, i, c + 4), gk);
       }
