@@ -55,6 +55,19 @@ namespace {
 
 using namespace sm100;
 
+// The bounded wait with its slow path (suspend, clock and abort checks) out of line:
+// one copy in the kernel's code instead of one per wait site, since the kernel's
+// speed depends on how much of its code the instruction caches hold.
+__device__ __noinline__ bool mbar_wait_slow(uint64_t *bar, uint32_t parity, uint64_t timeout_ns,
+                                            const volatile int *abort_flag) {
+  return mbar_wait(bar, parity, timeout_ns, abort_flag);
+}
+__device__ __forceinline__ bool mbar_wait_ni(uint64_t *bar, uint32_t parity, uint64_t timeout_ns,
+                                             const volatile int *abort_flag) {
+  if (mbar_try_wait(bar, parity)) return true;
+  return mbar_wait_slow(bar, parity, timeout_ns, abort_flag);
+}
+
 
 constexpr int C = 32;     // tokens per chunk of this kernel
 constexpr int DH = 128;   // head dim (dk = dv)
@@ -154,6 +167,23 @@ __device__ __forceinline__ float tf32_rn(float x) {
   asm("cvt.rn.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
   return __uint_as_float(r);
 }
+// two fp32 lanes per instruction (packed f32x2 arithmetic, round to nearest even, the
+// same results as two scalar operations)
+__device__ __forceinline__ void mul2(float &a0, float &a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 x, y;\n\tmov.b64 x, {%0, %1};\n\tmov.b64 y, {%2, %3};\n\t"
+      "mul.rn.f32x2 x, x, y;\n\tmov.b64 {%0, %1}, x;\n\t}"
+      : "+f"(a0), "+f"(a1) : "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ void sub2(float &a0, float &a1, float b0, float b1) {
+  asm("{\n\t.reg .b64 x, y;\n\tmov.b64 x, {%0, %1};\n\tmov.b64 y, {%2, %3};\n\t"
+      "sub.rn.f32x2 x, x, y;\n\tmov.b64 {%0, %1}, x;\n\t}"
+      : "+f"(a0), "+f"(a1) : "f"(b0), "f"(b1));
+}
+__device__ __forceinline__ void fma2(float &a0, float &a1, float b0, float b1, float c0, float c1) {
+  asm("{\n\t.reg .b64 x, y, z;\n\tmov.b64 x, {%0, %1};\n\tmov.b64 y, {%2, %3};\n\t"
+      "mov.b64 z, {%4, %5};\n\tfma.rn.f32x2 x, y, z, x;\n\tmov.b64 {%0, %1}, x;\n\t}"
+      : "+f"(a0), "+f"(a1) : "f"(b0), "f"(b1), "f"(c0), "f"(c1));
+}
 __device__ __forceinline__ void ld8f(const float *p, float *x) {
   const float4 a = reinterpret_cast<const float4 *>(p)[0];
   const float4 b = reinterpret_cast<const float4 *>(p)[1];
@@ -210,8 +240,7 @@ __global__ void __launch_bounds__(NT + 64, 1)
   uint64_t *ops_oy = bars + 8;    // A (gamma*Q) and B (gamma*K, V^T) -> control
   uint64_t *ops_tb = bars + 9;    // group A -> control: T Diag(beta) ready
   uint64_t *ops_sc = bars + 10;   // group B -> control: S^T scaled by gamma_31
-  uint64_t *gate_ok = bars + 11;  // group A -> group B: cumulative gate of a chunk ready
-  uint64_t *khat_done = bars + 12;  // group B -> group A: a chunk's gate table read
+  uint64_t *gate_ok = bars + 11;  // [2] group A -> group B: cumulative gate of a chunk ready
   uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bars + 13);
   volatile int *s_abort = reinterpret_cast<volatile int *>(s_tmem + 1);
 
@@ -261,7 +290,7 @@ __global__ void __launch_bounds__(NT + 64, 1)
     mbar_init(ops_tb, NA / 32);
     mbar_init(ops_sc, (NT - NA) / 32);
     mbar_init(gate_ok, NA / 32);
-    mbar_init(khat_done, (NT - NA) / 32);
+    mbar_init(gate_ok + 1, NA / 32);
     *s_abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -347,7 +376,7 @@ __global__ void __launch_bounds__(NT + 64, 1)
       uint32_t ph_ops_ap = 0, ph_raw = 0, ph_ops_oy = 0, ph_tb = 0, ph_sc = 0, ph_oy = 0,
                ph_u = 0;
       auto cwait = [&](uint64_t *bar, uint32_t &ph) -> bool {
-        const bool good = *s_abort == 0 && mbar_wait(bar, ph, wait_ns, s_abort);
+        const bool good = *s_abort == 0 && mbar_wait_ni(bar, ph, wait_ns, s_abort);
         ph ^= 1u;
         if (!good) {
           *s_abort = 1;
@@ -421,12 +450,12 @@ __global__ void __launch_bounds__(NT + 64, 1)
     }
   } else if (group_a) {
     // ============ group A (warps 0-7): gate, row operands, read-out, solve ============
-    uint32_t ph_tma = 0u, ph_ap = 0, ph_oy = 0, ph_kd = 0;  // ph_tma: bit b for buffer b
+    uint32_t ph_tma = 0u, ph_ap = 0, ph_oy = 0;  // ph_tma: bit b for buffer b
     auto wsync = [&]() { named_sync(1, NA); };
-    // thread 0 waits for the group while the others block at the named barrier; the
-    // vote there gives every thread the outcome, so an abort is taken by all together
+    // every thread waits, and the vote at the group's named barrier gives every thread
+    // the outcome, so that an abort is taken by all together
     auto wwait = [&](uint64_t *bar, uint32_t &ph) -> bool {
-      const bool got = mbar_wait(bar, ph, wait_ns, s_abort);
+      const bool got = mbar_wait_ni(bar, ph, wait_ns, s_abort);
       ph ^= 1u;
       const bool bad = named_sync_or(1, NA, !got || *s_abort != 0);
       if (bad) {
@@ -502,7 +531,7 @@ __global__ void __launch_bounds__(NT + 64, 1)
         if (cg == 1 && j == 15) GC[(m & 3) * DH + l] = ex2(g2);
       }
       wsync();
-      warp_signal(gate_ok);
+      warp_signal(gate_ok + (m & 1));
     };
 
     // ---- rows(m): the row operands (thread = row i, channels 64 cg .. 64 cg + 63) ----
@@ -532,7 +561,13 @@ __global__ void __launch_bounds__(NT + 64, 1)
           ld8g(gt, i, c, g);
           ld8g(gt, MREF, c, gr);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) x[e] = tf32_rn(x[e] * ex2(g[e] - gr[e]));
+          for (int e = 0; e < 8; e += 2) sub2(g[e], g[e + 1], gr[e], gr[e + 1]);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) g[e] = ex2(g[e]);
+#pragma unroll
+          for (int e = 0; e < 8; e += 2) mul2(x[e], x[e + 1], g[e], g[e + 1]);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) x[e] = tf32_rn(x[e]);
           tmem_st8(tm + lane_base + TM_L + c, x);
         }
         tmem_wait_st();
@@ -545,7 +580,13 @@ __global__ void __launch_bounds__(NT + 64, 1)
           ld8g(gt, i, c, g);
           ld8g(gt, MREF, c, gr);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) x[e] = tf32_rn(x[e] * ex2(gr[e] - g[e]));
+          for (int e = 0; e < 8; e += 2) sub2(gr[e], gr[e + 1], g[e], g[e + 1]);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) gr[e] = ex2(gr[e]);
+#pragma unroll
+          for (int e = 0; e < 8; e += 2) mul2(x[e], x[e + 1], gr[e], gr[e + 1]);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) x[e] = tf32_rn(x[e]);
           st8f(sm + OFF_RP, sw128_chunk(C, i, c), sw128_chunk(C, i, c + 4), x);
         }
       } else if (has_q) {  // gamma*Q = q exp(G_i)
@@ -556,7 +597,11 @@ __global__ void __launch_bounds__(NT + 64, 1)
           bf16_x8(load_x(R_Q, c), x);
           ld8g(gt, i, c, g);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) x[e] = tf32_rn(x[e] * ex2(g[e]));
+          for (int e = 0; e < 8; ++e) g[e] = ex2(g[e]);
+#pragma unroll
+          for (int e = 0; e < 8; e += 2) mul2(x[e], x[e + 1], g[e], g[e + 1]);
+#pragma unroll
+          for (int e = 0; e < 8; ++e) x[e] = tf32_rn(x[e]);
           st8f(sm + OFF_GQ, sw128_chunk(C, i, c), sw128_chunk(C, i, c + 4), x);
         }
       }
@@ -631,25 +676,24 @@ __global__ void __launch_bounds__(NT + 64, 1)
         const int i = tid >> 4, c = tid & 15;
         float x0 = 0.f, x1 = 0.f;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          x0 += NS[(16 + i) * LDN + j] * TS[j * LDN + c];
-          x1 += NS[(16 + i) * LDN + 8 + j] * TS[(8 + j) * LDN + c];
-        }
+        for (int j = 0; j < 8; ++j)
+          fma2(x0, x1, NS[(16 + i) * LDN + j], NS[(16 + i) * LDN + 8 + j], TS[j * LDN + c],
+               TS[(8 + j) * LDN + c]);
         XS[i * LDX + c] = x0 + x1;
         wsync();
         float y0 = 0.f, y1 = 0.f;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          y0 += TS[(16 + i) * LDN + 16 + j] * XS[j * LDX + c];
-          y1 += TS[(16 + i) * LDN + 24 + j] * XS[(8 + j) * LDX + c];
-        }
+        for (int j = 0; j < 8; ++j)
+          fma2(y0, y1, TS[(16 + i) * LDN + 16 + j], TS[(16 + i) * LDN + 24 + j], XS[j * LDX + c],
+               XS[(8 + j) * LDX + c]);
         st_shared_f1(tb + sw128_offset(C, 16 + i, c), tf32_rn(-(y0 + y1) * BT[(m & 1) * C + c]));
       }
     };
 
     // The gate of chunk m+1 runs while the A|P products of chunk m do (its table sits in
-    // chunk m+1's own raw buffer); it waits until group B has read chunk m's table, so
-    // that group A is never two gates ahead.
+    // chunk m+1's own raw buffer, which group B has read for chunk m-1 before the tiles
+    // of chunk m+1 could load).  Its barrier is one of a pair, by chunk parity, so group
+    // A may finish a gate before group B has taken the previous one.
     bool ok = true;
     if (n_chunks > 0 && (ok = wait_tma(0))) w_gate(0);
     for (int m = 0; ok && m < n_chunks; ++m) {
@@ -663,7 +707,6 @@ __global__ void __launch_bounds__(NT + 64, 1)
       warp_signal(ops_oy);  // gamma*Q made visible by the fence of the arrival above
       KDA_PHASE(3);
       if (m + 1 < n_chunks) {
-        if (!(ok = wwait(khat_done, ph_kd))) break;
         if (!(ok = wait_tma(m + 1))) break;
         KDA_PHASE(1);
         w_gate(m + 1);
@@ -679,10 +722,11 @@ __global__ void __launch_bounds__(NT + 64, 1)
     }
   } else {
     // ====== group B (warps 8-15): state scaling, Khat^T, outputs, V^T, states ======
-    uint32_t ph_oy = 0, ph_gate = 0, ph_fin = 0;
-    // thread 256 waits for the group while the others block at the group's barrier
+    uint32_t ph_oy = 0, ph_fin = 0;
+    // every thread waits, and the vote at the group's named barrier gives every thread
+    // the outcome, so that an abort is taken by all together
     auto bwait = [&](uint64_t *bar, uint32_t &ph) -> bool {
-      const bool got = mbar_wait(bar, ph, wait_ns, s_abort);
+      const bool got = mbar_wait_ni(bar, ph, wait_ns, s_abort);
       ph ^= 1u;
       const bool bad = named_sync_or(2, NT - NA, !got || *s_abort != 0);
       if (bad) {
@@ -698,15 +742,15 @@ __global__ void __launch_bounds__(NT + 64, 1)
     {
       const float *s0 =
           p.initial_state ? p.initial_state + ((size_t)(r * H + h)) * DH * DH : nullptr;
+#pragma unroll 1
+      for (int q8 = 0; q8 < 8; ++q8) {
+        const int c0 = 64 * cg + 8 * q8;
+        float v[8];
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int c0 = 64 * cg + 32 * half;
-        float v[32];
-#pragma unroll
-        for (int j = 0; j < 32; ++j)
+        for (int j = 0; j < 8; ++j)
           v[j] = p.local_mode ? ((part == 1 && c0 + j == l) ? 1.f : 0.f)
                               : (s0 ? s0[(size_t)(c0 + j) * DH + l] : 0.f);
-        tmem_st32(tm + lane_base + TM_S + c0, v);
+        tmem_st8(tm + lane_base + TM_S + c0, v);
       }
       tmem_wait_st();
     }
@@ -725,7 +769,7 @@ __global__ void __launch_bounds__(NT + 64, 1)
           float f[8];
           ld8f(gc + c0 + j, f);
 #pragma unroll
-          for (int e = 0; e < 8; ++e) v[j + e] *= f[e];
+          for (int e = 0; e < 8; e += 2) mul2(v[j + e], v[j + e + 1], f[e], f[e + 1]);
         }
         tmem_st16(tm + lane_base + TM_S + c0, v);
       }
@@ -740,7 +784,7 @@ __global__ void __launch_bounds__(NT + 64, 1)
       const unsigned char *raw = sm + OFF_RAW + (m & 1) * RAW_BYTES;
       unsigned char *kh = sm + kh_off(m);
       const int i = lane_id;
-#pragma unroll
+#pragma unroll 1  // rolled: smaller code (see mbar_wait_slow)
       for (int u = 0; u < 2; ++u) {
         const int c = 16 * w8 + 8 * u;
         float x[8], g[8], ge[8], gk[8];
@@ -750,9 +794,21 @@ __global__ void __launch_bounds__(NT + 64, 1)
         ld8g(raw + R_G, i, c, g);
         ld8g(raw + R_G, C - 1, c, ge);
 #pragma unroll
+        for (int e = 0; e < 8; e += 2) sub2(ge[e], ge[e + 1], g[e], g[e + 1]);
+#pragma unroll
         for (int e = 0; e < 8; ++e) {
-          st_shared_f1(kh + sw128_offset(DH, c + e, i), tf32_rn(x[e] * ex2(ge[e] - g[e])));
-          gk[e] = tf32_rn(x[e] * ex2(g[e]));
+          ge[e] = ex2(ge[e]);
+          gk[e] = ex2(g[e]);
+        }
+#pragma unroll
+        for (int e = 0; e < 8; e += 2) {
+          mul2(ge[e], ge[e + 1], x[e], x[e + 1]);
+          mul2(gk[e], gk[e + 1], x[e], x[e + 1]);
+        }
+#pragma unroll
+        for (int e = 0; e < 8; ++e) {
+          st_shared_f1(kh + sw128_offset(DH, c + e, i), tf32_rn(ge[e]));
+          gk[e] = tf32_rn(gk[e]);
         }
         st8f(sm + OFF_GK, sw128_chunk(C, i, c), sw128_chunk(C, i, c + 4), gk);
       }
@@ -765,23 +821,28 @@ __global__ void __launch_bounds__(NT + 64, 1)
         float o16[16];
         tmem_ld16(tm + lane_base + TM_O + 16 * cg, o16);
         tmem_wait_ld();
+        // one pointer stepped by a token's row (64-bit index arithmetic per store was a
+        // large part of this step, which lies on the state chain)
+        TOut *dst = go + ((size_t)(bos + c0 + 16 * cg) * H + h) * DH + l;
+        const size_t step = (size_t)H * DH;
+        const int nt = nr - 16 * cg;
 #pragma unroll
         for (int j = 0; j < 16; ++j) {
-          const int t = 16 * cg + j;
-          if (t < nr) store_elem(go, ((size_t)(bos + c0 + t) * H + h) * DH + l, o16[j]);
+          if (j < nt) store_elem(dst, 0, o16[j]);
+          dst += step;
         }
       }
       if (snaps_ok && nr == C && (c0 + C) % p.snapshot_stride == 0) {
         const size_t row = (size_t)p.cu_snapshots[r] + (c0 + C) / p.snapshot_stride - 1;
         float *dst = p.snapshots + (row * H + h) * (size_t)DH * DH;
-#pragma unroll
-        for (int half = 0; half < 2; ++half) {
-          const int k0 = 64 * cg + 32 * half;
-          float v[32];
-          tmem_ld32(tm + lane_base + TM_S + k0, v);
+#pragma unroll 1
+        for (int q8 = 0; q8 < 8; ++q8) {
+          const int k0 = 64 * cg + 8 * q8;
+          float v[8];
+          tmem_ld8(tm + lane_base + TM_S + k0, v);
           tmem_wait_ld();
 #pragma unroll
-          for (int j = 0; j < 32; ++j) dst[(size_t)(k0 + j) * DH + l] = v[j];
+          for (int j = 0; j < 8; ++j) dst[(size_t)(k0 + j) * DH + l] = v[j];
         }
       }
     };
@@ -802,9 +863,9 @@ __global__ void __launch_bounds__(NT + 64, 1)
 
     bool ok = true;
     if (n_chunks > 0) {
-      if ((ok = bwait(gate_ok, ph_gate))) {
+      uint32_t ph = 0;
+      if ((ok = bwait(gate_ok, ph))) {
         w_khat(0);
-        warp_signal(khat_done);
         w_vt(0);
         warp_signal(raw_free);
         warp_arrive(ops_oy);
@@ -818,10 +879,10 @@ __global__ void __launch_bounds__(NT + 64, 1)
       warp_signal(ops_sc);
       KDA_PHASE(9);
       if (more) {
-        if (!(ok = bwait(gate_ok, ph_gate))) break;
+        uint32_t ph = ((n + 1) >> 1) & 1u;
+        if (!(ok = bwait(gate_ok + ((n + 1) & 1), ph))) break;
         KDA_PHASE(10);
         w_khat(n + 1);  // the other Khat^T buffer: chunk n-1's last products are done
-        warp_signal(khat_done);
         KDA_PHASE(11);
       }
       if (!(ok = bwait(bar_fin, ph_fin))) break;
@@ -840,14 +901,14 @@ __global__ void __launch_bounds__(NT + 64, 1)
     if (ok && fin) {
       float *dst = fin + ((size_t)(r * H + h)) * DH * DH;
       tc_fence_after();
-#pragma unroll
-      for (int half = 0; half < 2; ++half) {
-        const int k0 = 64 * cg + 32 * half;
-        float v[32];
-        tmem_ld32(tm + lane_base + TM_S + k0, v);
+#pragma unroll 1
+      for (int q8 = 0; q8 < 8; ++q8) {
+        const int k0 = 64 * cg + 8 * q8;
+        float v[8];
+        tmem_ld8(tm + lane_base + TM_S + k0, v);
         tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 32; ++j) dst[(size_t)(k0 + j) * DH + l] = v[j];
+        for (int j = 0; j < 8; ++j) dst[(size_t)(k0 + j) * DH + l] = v[j];
       }
     }
   }
