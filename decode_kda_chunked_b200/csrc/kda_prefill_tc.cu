@@ -83,8 +83,6 @@ constexpr float LOG2E = 1.4426950408889634f;
 constexpr uint32_t RAW_BYTES = 40960;
 constexpr uint32_t R_K = 0, R_Q = 8192, R_V = 16384, R_G = 24576;
 constexpr uint32_t OFF_RAW = 0;
-// The chunk-local cumulative gate, log2(e) * G, replaces the raw g tile in place (fp32,
-// the same four swizzled boxes), so each raw buffer carries its chunk's gate table.
 constexpr uint32_t OFF_GQ = 81920;   // gamma*Q  tf32 B operand [32 x 128]
 constexpr uint32_t OFF_GK = 98304;   // gamma*K  tf32 B operand [32 x 128]
 constexpr uint32_t OFF_KH = 114688;  // Khat^T   tf32 B operand [128 x 32], x2 (chunk parity)
@@ -98,9 +96,16 @@ constexpr uint32_t OFF_XS = 189440;  // N10 T00, fp32 [16][LDX]
 constexpr int LDX = 20;
 constexpr uint32_t OFF_GC = 190720;  // exp(G_31) per key channel, [4][128] (chunk index mod 4)
 constexpr uint32_t OFF_BT = 192768;  // beta [2][32] (chunk parity)
-constexpr uint32_t OFF_SEG = 193024; // cumulative-gate segment totals [2][128]
+constexpr uint32_t OFF_SEG = 193024; // spare [2][128]
 constexpr uint32_t OFF_BAR = 194048; // mbarriers, TMEM base, flags (+ phase counters)
-constexpr uint32_t SMEM_BYTES = 194304;
+// Cumulative gate log2(e) G of a chunk, fp32 [32 tokens][LDG], x2 (chunk parity): rows
+// padded to LDG = 132 floats, so that eight consecutive channels of a token are one
+// 16-byte aligned pair of loads at a plain offset, and lanes reading eight rows hit
+// eight distinct bank quads.
+constexpr uint32_t OFF_GT = 194304;
+constexpr int LDG = 132;
+constexpr uint32_t GT_BYTES = C * LDG * 4;
+constexpr uint32_t SMEM_BYTES = OFF_GT + 2 * GT_BYTES;
 constexpr uint32_t SMEM_ALLOC = SMEM_BYTES + 1024;  // alignment slack
 static_assert(OFF_RAW + 2 * RAW_BYTES == OFF_GQ, "raw buffers");
 static_assert(OFF_GQ % 1024 == 0 && OFF_GK % 1024 == 0 && OFF_KH % 1024 == 0 &&
@@ -113,8 +118,9 @@ static_assert(OFF_GQ + 16384 == OFF_GK && OFF_GK + 16384 == OFF_KH &&
 static_assert(OFF_NS + C * LDN * 4 == OFF_TS && OFF_TS + C * LDN * 4 == OFF_XS &&
                   OFF_XS + 16 * LDX * 4 == OFF_GC && OFF_GC + 4 * DH * 4 == OFF_BT &&
                   OFF_BT + 2 * C * 4 == OFF_SEG &&
-                  OFF_SEG + 2 * DH * 4 == OFF_BAR,
+                  OFF_SEG + 2 * DH * 4 == OFF_BAR && OFF_BAR + 256 == OFF_GT,
               "scratch tiles");
+static_assert(SMEM_BYTES + 1024 <= 232448, "227 KB of shared memory per CTA");
 __host__ __device__ constexpr uint32_t kh_off(int m) { return OFF_KH + 16384u * (m & 1); }
 __host__ __device__ constexpr uint32_t pp_off(int m) { return OFF_PP + 4096u * (m & 1); }
 __host__ __device__ constexpr uint32_t tb_off(int m) { return OFF_TB + 4096u * (m & 1); }
@@ -155,10 +161,10 @@ __device__ __forceinline__ uint32_t f32_off(int t, int c) {
   return (uint32_t)(c >> 5) * 4096u + (uint32_t)t * 128u +
          ((uint32_t)(((c & 31) >> 2) ^ (t & 7)) << 4) + (uint32_t)(c & 3) * 4u;
 }
-// eight consecutive channels c..c+7 (c % 8 == 0) of row t of an fp32 tile in that layout
-__device__ __forceinline__ void ld8g(const unsigned char *tile, int t, int c, float *x) {
-  const float4 a = *reinterpret_cast<const float4 *>(tile + f32_off(t, c));
-  const float4 b = *reinterpret_cast<const float4 *>(tile + f32_off(t, c + 4));
+// eight consecutive channels c..c+7 (c % 8 == 0) of token t of a gate table (row stride LDG)
+__device__ __forceinline__ void ld8g(const float *table, int t, int c, float *x) {
+  const float4 *q = reinterpret_cast<const float4 *>(table + t * LDG + c);
+  const float4 a = q[0], b = q[1];
   x[0] = a.x; x[1] = a.y; x[2] = a.z; x[3] = a.w; x[4] = b.x; x[5] = b.y; x[6] = b.z; x[7] = b.w;
 }
 // fp32 -> tf32, round to nearest even (the tensor cores read the 19 leading bits)
@@ -198,10 +204,11 @@ __device__ __forceinline__ void st8f(unsigned char *base, uint32_t off_lo, uint3
 
 #ifdef KDA_PHASE_PROFILE
 // Cycles per step of the loops, summed over every CTA (profiling builds only):
-// group A (thread 0): 0 wait for O^T/Y^T(m-1), 1 wait for group B's Khat^T(m) and the
-// tiles of chunk m+1, 2 gate(m+1), 3 rows(m), 4 wait for A|P(m), 5 read, 6 solve;
-// group B (thread 256): 8 wait for O^T/Y^T(n), 9 scale, 10 wait for the next gate,
-// 11 Khat^T, 12 wait for the last products, 13 out, 14 V^T.  Entry 15 counts the chunks.
+// group A (thread 0): 0 wait for O^T/Y^T(m-1), 1 wait for the tiles of chunk m+1,
+// 2 gate(m+1), 3 rows(m), 4 wait for A|P(m), 5 read, 7 solve up to the diagonal blocks,
+// 6 the rest of the solve; group B (thread 256): 8 wait for O^T/Y^T(n), 9 scale, 10 wait
+// for the next gate, 11 Khat^T, 12 wait for the last products, 13 out, 14 V^T.
+// Entry 15 counts the chunks.
 __device__ unsigned long long g_phase_cycles[16];
 #define KDA_PHASE(k)                                              \
   do {                                                            \
@@ -228,7 +235,6 @@ __global__ void __launch_bounds__(NT + 64, 1)
   float *XS = reinterpret_cast<float *>(sm + OFF_XS);
   float *GC = reinterpret_cast<float *>(sm + OFF_GC);
   float *BT = reinterpret_cast<float *>(sm + OFF_BT);
-  float *SEG = reinterpret_cast<float *>(sm + OFF_SEG);
   uint64_t *bars = reinterpret_cast<uint64_t *>(sm + OFF_BAR);
   uint64_t *bar_tma = bars + 0;   // [2] TMA -> group A: raw buffer b landed
   uint64_t *bar_ap = bars + 2;    // commit: A|P products done
@@ -431,12 +437,13 @@ __global__ void __launch_bounds__(NT + 64, 1)
         for (int m = 0; m < n_chunks; ++m) {
           if (!cwait(ops_ap, ph_ops_ap)) break;
           mma_ap(m);
+          // chunk m's tiles are read (group A signs with the A|P operands, group B with
+          // V^T(m), a chunk earlier): chunk m + 2 may load, a whole chunk before its gate
+          if (!cwait(raw_free, ph_raw)) break;
+          if (m + 2 < n_chunks) issue_tma(m + 2);
           if (!cwait(ops_tb, ph_tb)) break;
           if (!cwait(bar_oy, ph_oy)) break;  // Y^T is U^T's A operand
           mma_u(m);
-          // chunk m's tiles are read by both groups: chunk m + 2 may load
-          if (!cwait(raw_free, ph_raw)) break;
-          if (m + 2 < n_chunks) issue_tma(m + 2);
         }
       } else {
         for (int m = 0; m < n_chunks; ++m) {
@@ -492,7 +499,9 @@ __global__ void __launch_bounds__(NT + 64, 1)
     };
     float beta_pref = load_beta(0);
 
-    // ---- gate(m): cumulative gate (thread = channel l, tokens 16 cg .. 16 cg + 15) ----
+    // ---- gate(m): cumulative gate (thread = key channel gc, tokens 16 gh .. 16 gh + 15:
+    // the two halves of a channel sit in one warp, lanes 16 apart) ----
+    const int gc = 16 * warp + (lane_id & 15), gh = lane_id >> 4;
     auto w_gate = [&](int m) {
       const int nr = min(C, len - m * C);
       unsigned char *raw = sm + OFF_RAW + (m & 1) * RAW_BYTES;
@@ -507,12 +516,12 @@ __global__ void __launch_bounds__(NT + 64, 1)
       float gv[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
-        const int t = 16 * cg + j;
-        gv[j] = LOGITS ? gate_from_logit(bf16_at(raw + R_G, t, l))
-                       : *reinterpret_cast<const float *>(raw + R_G + f32_off(t, l));
+        const int t = 16 * gh + j;
+        gv[j] = LOGITS ? gate_from_logit(bf16_at(raw + R_G, t, gc))
+                       : *reinterpret_cast<const float *>(raw + R_G + f32_off(t, gc));
       }
 #pragma unroll
-      for (int j = 0; j < 16; ++j) gv[j] = (16 * cg + j < nr) ? gv[j] : 0.f;
+      for (int j = 0; j < 16; ++j) gv[j] = (16 * gh + j < nr) ? gv[j] : 0.f;
       if (!LOGITS && p.validate) {
         bool bad = false;
 #pragma unroll
@@ -521,16 +530,13 @@ __global__ void __launch_bounds__(NT + 64, 1)
       }
 #pragma unroll
       for (int j = 1; j < 16; ++j) gv[j] += gv[j - 1];
-      if (cg == 0) SEG[l] = gv[15];
-      wsync();
-      const float off = cg ? SEG[l] : 0.f;
+      const float first = __shfl_sync(0xffffffffu, gv[15], lane_id & 15);
+      const float off = gh ? first : 0.f;
+      float *gtab = reinterpret_cast<float *>(sm + OFF_GT + (m & 1) * GT_BYTES) +
+                    16 * gh * LDG + gc;
 #pragma unroll
-      for (int j = 0; j < 16; ++j) {
-        const float g2 = (gv[j] + off) * LOG2E;
-        *reinterpret_cast<float *>(raw + R_G + f32_off(16 * cg + j, l)) = g2;
-        if (cg == 1 && j == 15) GC[(m & 3) * DH + l] = ex2(g2);
-      }
-      wsync();
+      for (int j = 0; j < 16; ++j) gtab[j * LDG] = (gv[j] + off) * LOG2E;
+      if (gh) GC[(m & 3) * DH + gc] = ex2((gv[15] + off) * LOG2E);
       warp_signal(gate_ok + (m & 1));
     };
 
@@ -546,7 +552,7 @@ __global__ void __launch_bounds__(NT + 64, 1)
       const int i = lane_id;
       const bool valid = i < nr;
       const uint4 z4 = make_uint4(0u, 0u, 0u, 0u);
-      const unsigned char *gt = raw + R_G;  // the chunk's gate table (see gate)
+      const float *gt = reinterpret_cast<const float *>(sm + OFF_GT + (m & 1) * GT_BYTES);
       auto load_x = [&](uint32_t tile, int c) {
         return valid ? *reinterpret_cast<const uint4 *>(raw + tile + bf16_chunk(i, c)) : z4;
       };
@@ -670,6 +676,7 @@ __global__ void __launch_bounds__(NT + 64, 1)
         }
       }
       wsync();  // diagonal blocks ready
+      KDA_PHASE(7);
       {  // T10 = -T11 (N10 T00): one element (i, c) per thread of the group
         // the T00 entries above the diagonal and the T11 entries past row i are zero, so
         // the sums run over all 16 terms without branches, in two halves each
@@ -782,8 +789,14 @@ __global__ void __launch_bounds__(NT + 64, 1)
     auto w_khat = [&](int m) {
       const int nr = min(C, len - m * C);
       const unsigned char *raw = sm + OFF_RAW + (m & 1) * RAW_BYTES;
-      unsigned char *kh = sm + kh_off(m);
+      const float *gtab = reinterpret_cast<const float *>(sm + OFF_GT + (m & 1) * GT_BYTES);
       const int i = lane_id;
+      // element (channel c + e, token i) of the Khat^T tile: row c + e, 16-byte chunk
+      // (i >> 2) ^ e (c % 8 == 0), so eight offsets serve both channel groups
+      unsigned char *kh = sm + kh_off(m) + (i & 3) * 4;
+      uint32_t koff[8];
+#pragma unroll
+      for (int e = 0; e < 8; ++e) koff[e] = e * 128 + (((i >> 2) ^ e) << 4);
 #pragma unroll 1  // rolled: smaller code (see mbar_wait_slow)
       for (int u = 0; u < 2; ++u) {
         const int c = 16 * w8 + 8 * u;
@@ -791,8 +804,8 @@ __global__ void __launch_bounds__(NT + 64, 1)
         bf16_x8(i < nr ? *reinterpret_cast<const uint4 *>(raw + R_K + bf16_chunk(i, c))
                        : make_uint4(0u, 0u, 0u, 0u),
                 x);
-        ld8g(raw + R_G, i, c, g);
-        ld8g(raw + R_G, C - 1, c, ge);
+        ld8g(gtab, i, c, g);
+        ld8g(gtab, C - 1, c, ge);
 #pragma unroll
         for (int e = 0; e < 8; e += 2) sub2(ge[e], ge[e + 1], g[e], g[e + 1]);
 #pragma unroll
@@ -807,7 +820,7 @@ __global__ void __launch_bounds__(NT + 64, 1)
         }
 #pragma unroll
         for (int e = 0; e < 8; ++e) {
-          st_shared_f1(kh + sw128_offset(DH, c + e, i), tf32_rn(ge[e]));
+          st_shared_f1(kh + c * 128 + koff[e], tf32_rn(ge[e]));
           gk[e] = tf32_rn(gk[e]);
         }
         st8f(sm + OFF_GK, sw128_chunk(C, i, c), sw128_chunk(C, i, c + 4), gk);
@@ -850,12 +863,17 @@ __global__ void __launch_bounds__(NT + 64, 1)
     // ---- vt(m): V^T -> TMEM (lane = value channel, tokens 16 cg ..) ----
     auto w_vt = [&](int m) {
       const int nr = min(C, len - m * C);
-      const unsigned char *raw = sm + OFF_RAW + (m & 1) * RAW_BYTES;
+      // row t = 16 cg + j of the swizzled v tile: the 16-byte chunk of channel l sits at
+      // chunk index ((l & 63) >> 3) ^ (j & 7), so eight offsets serve all sixteen rows
+      const unsigned char *row0 = sm + OFF_RAW + (m & 1) * RAW_BYTES + R_V + (l >> 6) * 4096 +
+                                  16 * cg * 128 + (l & 7) * 2;
+      const int c8 = (l & 63) >> 3, nv = zero_v ? 0 : nr - 16 * cg;
       float v16[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
-        const int t = 16 * cg + j;
-        v16[j] = (t < nr && !zero_v) ? bf16_at(raw + R_V, t, l) : 0.f;
+        const unsigned short u =
+            *reinterpret_cast<const unsigned short *>(row0 + j * 128 + ((c8 ^ (j & 7)) << 4));
+        v16[j] = j < nv ? bf16_lo(u) : 0.f;
       }
       tmem_st16(tm + lane_base + TM_Y + 16 * cg, v16);
       tmem_wait_st();

@@ -19,12 +19,14 @@ import ctypes
 import json
 
 # group A (worker thread 0) and group B (worker thread 256) steps, by counter slot
-PHASES = {0: "A wait: O^T, Y^T of chunk m-1", 1: "A wait: Khat^T(m), tiles(m+1)",
+PHASES = {0: "A wait: O^T, Y^T of chunk m-1", 1: "A wait: tiles of m+1",
           2: "A gate (cumulative) of m+1",
           3: "A rows (L, R', gamma Q/K)", 4: "A wait: A|P", 5: "A read (A, P)",
-          6: "A solve (T Diag(beta))",
+          7: "A solve: diagonal blocks", 6: "A solve: block below the diagonal",
           8: "B wait: O^T, Y^T", 9: "B scale S^T", 10: "B wait: next gate", 11: "B Khat^T",
           12: "B wait: last products", 13: "B out (o, snapshots)", 14: "B V^T"}
+# group A (worker thread 0) and group B (worker thread 256), slots in loop order
+GROUPS = (("A", (0, 1, 2, 3, 4, 5, 7, 6)), ("B", range(8, 15)))
 
 
 def main():
@@ -59,7 +61,7 @@ def main():
     chunks = buf[15]
     out = {}
     print(f"{chunks // args.steps} chunks of 32 tokens per call")
-    for grp, slots in (("A", range(0, 7)), ("B", range(8, 15))):
+    for grp, slots in GROUPS:
         total = sum(buf[k] for k in slots)
         print(f"group {grp}: {total / chunks:.0f} cycles per chunk")
         rows = [{"phase": PHASES[k], "cycles_per_chunk": buf[k] / chunks,
