@@ -592,7 +592,8 @@ def bench_backward(args, inp, dev, peaks, world):
 
 def bench_single_seq(args, dev, peaks):
     """One sequence of 8,192 tokens, H=32, d=128, N(0, 0.1) initial state: only 32
-    serial chains, so this measures the latency of the chunk-to-chunk state path."""
+    serial chains, which kda_prefill_chunked splits into segments (local states, exact
+    combine, segment prefill) to occupy more SMs; the unsplit call is timed beside it."""
     import torch
 
     import decode_kda_chunked_b200 as kda
@@ -603,12 +604,21 @@ def bench_single_seq(args, dev, peaks):
     fin = torch.empty(1, H, d, d, device=dev)
     stream = torch.cuda.current_stream(dev)
     cu_host = torch.tensor([0, T], dtype=torch.int32)
-    ms = _time_calls(lambda: kda.kda_prefill_chunked(
+    call = lambda: kda.kda_prefill_chunked(
         x.q, x.k, x.v, x.g, x.beta, x.cu_seqlens, o, x.initial_state, fin,
-        cu_seqlens_host=cu_host, stream=stream), 3, max(args.steps, 5), stream)
+        cu_seqlens_host=cu_host, stream=stream)
+    segments = kda.kda_prefill_split_segments(x.q, x.k, x.v, x.g, x.beta, x.cu_seqlens, o,
+                                              x.initial_state, fin, cu_seqlens_host=cu_host)
+    ms = _time_calls(call, 3, max(args.steps, 5), stream)
+    os.environ["KDA_NO_SPLIT"] = "1"
+    try:
+        ms_unsplit = _time_calls(call, 3, max(args.steps, 5), stream)
+    finally:
+        del os.environ["KDA_NO_SPLIT"]
     b = prefill_bytes(T, H, d, d, 1, initial=True, final=True)
     return {"workload": "B=1, H=32, T=8192, d=128, bf16, N(0,0.1) initial state, final state out",
             "value": T / (ms * 1e-3), "unit": "tokens/s", "ms_per_step": ms,
+            "split_segments": segments, "unsplit_ms": ms_unsplit,
             "tflops": prefill_flops_per_token_head(d, d) * T * H / (ms * 1e-3) / 1e12,
             "roofline": {"bound": "hbm", "achieved": b / (ms * 1e-3) / 1e9,
                          "peak": peaks["hbm_gbs"], "unit": "GB/s",
@@ -678,9 +688,15 @@ def bench_kcp_million(args, dev, peaks, world, rank):
            "parallelism": f"context parallel x{world}: segments per rank {per}"}
     if world == 1:
         import decode_kda_chunked_b200 as kda
-        ms_unsplit = _time_calls(lambda: kda.prefill(x.q, x.k, x.v, x.g, x.beta, x.cu_seqlens,
-                                                     snapshot_stride=512, cu_seqlens_host=[0, T],
-                                                     stream=stream), 0, 1, stream)
+        unsplit = lambda: kda.prefill(x.q, x.k, x.v, x.g, x.beta, x.cu_seqlens,
+                                      snapshot_stride=512, cu_seqlens_host=[0, T], stream=stream)
+        # the library's own split of few-chain calls, and the 16 chains left unsplit
+        out["library_split_ms"] = _time_calls(unsplit, 0, 1, stream)
+        os.environ["KDA_NO_SPLIT"] = "1"
+        try:
+            ms_unsplit = _time_calls(unsplit, 0, 1, stream)
+        finally:
+            del os.environ["KDA_NO_SPLIT"]
         out["unsplit_ms"] = ms_unsplit
         out["speedup_vs_unsplit"] = ms_unsplit / ms
     b = kcp_bytes(T, H, d, n_seg)

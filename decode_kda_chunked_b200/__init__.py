@@ -15,7 +15,7 @@ import torch
 from ._lib import (CHUNK, KdaError, kda_chunk_local_state, kda_decode_step,  # noqa: F401
                    kda_get_device_status, kda_prefill_backward,
                    kda_prefill_backward_workspace_size, kda_prefill_chunked,
-                   kda_prefill_workspace_size, make_backward_args,
+                   kda_prefill_workspace_size, kda_prefill_split_segments, make_backward_args,
                    kda_prefill_uses_tensor_cores, kda_snapshot_count, kda_state_combine,
                    kda_status_string, kda_version, load, make_prefill_args)
 
@@ -23,7 +23,7 @@ __all__ = ["kda_prefill_chunked", "kda_chunk_local_state", "kda_state_combine",
            "kda_decode_step", "kda_snapshot_count", "kda_get_device_status",
            "kda_status_string", "kda_version", "kda_prefill_workspace_size", "KdaError",
            "kda_prefill_uses_tensor_cores", "kda_prefill_backward",
-           "kda_prefill_backward_workspace_size",
+           "kda_prefill_backward_workspace_size", "kda_prefill_split_segments",
            "prefill", "prefill_backward", "long_context_prefill", "decode_step",
            "snapshot_offsets", "load", "PrefixCache"]
 

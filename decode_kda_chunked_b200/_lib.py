@@ -74,7 +74,7 @@ EXPORTS = ("kda_prefill_workspace_size", "kda_prefill_chunked", "kda_local_state
            "kda_prefill_backward_workspace_size", "kda_prefill_backward",
            "kda_prefix_cache_create", "kda_prefix_cache_destroy", "kda_prefix_cache_lookup",
            "kda_prefix_cache_insert", "kda_prefix_cache_size", "kda_state_gather",
-           "kda_state_scatter")
+           "kda_state_scatter", "kda_prefill_split_segments")
 
 
 def load(path: str = LIB_PATH):
@@ -93,6 +93,8 @@ def load(path: str = LIB_PATH):
         lib.kda_prefill_workspace_size.argtypes = [P(PrefillArgs)]
         lib.kda_prefill_chunked.restype = ctypes.c_int
         lib.kda_prefill_chunked.argtypes = [P(PrefillArgs), _vp, ctypes.c_size_t, _vp]
+        lib.kda_prefill_split_segments.restype = _i32
+        lib.kda_prefill_split_segments.argtypes = [P(PrefillArgs)]
         lib.kda_local_state_workspace_size.restype = ctypes.c_size_t
         lib.kda_local_state_workspace_size.argtypes = [P(LocalStateArgs)]
         lib.kda_chunk_local_state.restype = ctypes.c_int
@@ -229,6 +231,17 @@ def kda_prefill_chunked(q, k, v, g, beta, cu_seqlens, o, initial_state=None, fin
     _check("kda_prefill_chunked",
            lib.kda_prefill_chunked(ctypes.byref(a), ws_ptr, ws_bytes, _stream(stream)))
     return o
+
+
+def kda_prefill_split_segments(q, k, v, g, beta, cu_seqlens, o, initial_state=None,
+                               final_state=None, snapshot_stride=0, cu_snapshots=None,
+                               snapshots=None, cu_seqlens_host=None, g_logits=None) -> int:
+    """Segments kda_prefill_chunked would run for these arguments after its
+    context-parallel split of few-chain calls; 0 when it would not split."""
+    host = _host_i32(cu_seqlens_host)
+    a = make_prefill_args(q, k, v, g, beta, cu_seqlens, o, initial_state, final_state,
+                          snapshot_stride, cu_snapshots, snapshots, host, g_logits)
+    return int(load().kda_prefill_split_segments(ctypes.byref(a)))
 
 
 def make_backward_args(q, k, v, g, beta, cu_seqlens, cu_seqlens_host, d_q, d_k, d_v, d_g, d_beta,

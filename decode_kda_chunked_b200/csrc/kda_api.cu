@@ -4,6 +4,7 @@
 // code before launching anything; it allocates no device memory (scratch is
 // the caller's workspace) and never synchronises except in
 // kda_get_device_status().
+#include <algorithm>
 #include <cstdio>
 #include <cstdlib>
 #include <cstring>
@@ -121,11 +122,232 @@ size_t prefill_ws(int n_req) {
   return align256((size_t)n_req * sizeof(int32_t));
 }
 
+// ---------------------------------------------------------------------------
+// Context-parallel split of long requests when few chains are live.
+//
+// A (request, head) chain is one CTA of the tensor-core kernel, and its chunks run
+// in order, so a call with fewer chains than SMs leaves most of the GPU idle.  Such a
+// call is run as KDA context parallelism inside one device ("Kimi K3 开源日来了",
+// Infra section, first layer): long requests are cut into segments; a local-state
+// pass gives each non-final segment its zero-start state S_loc and transition M (two
+// CTAs per segment and head, all in one wave); an exact combine per request recovers
+// every segment's start state; and one prefill over all segments, each from its
+// start state, writes o, the snapshots and (through the last segment) the final
+// state.  The results equal the unsplit call's up to rounding.
+// ---------------------------------------------------------------------------
+struct SplitPlan {
+  int n_seg = 0;                    // segments over all requests; 0: no split
+  std::vector<int32_t> seg_cu;      // [n_seg + 1] token bounds of the segments
+  std::vector<int32_t> first_seg;   // [n_req + 1] first segment of each request
+  std::vector<int32_t> pass1;       // the non-final segments of split requests
+  std::vector<int32_t> seg_snap;    // [n_seg + 1] snapshot rows before each segment
+  // workspace layout (byte offsets, 256-aligned)
+  size_t off_cu = 0, off_p1 = 0, off_snap = 0, off_sloc = 0, off_m = 0, off_sin = 0, bytes = 0;
+};
+
+// SMs of the current device.  KDA_TEST_SM_COUNT overrides it, so that host tests
+// (which may run without a GPU) can check the split plan; nothing else should set it.
+int device_sm_count() {
+  if (const char *v = std::getenv("KDA_TEST_SM_COUNT"))
+    if (v[0]) return std::atoi(v);
+  int dev = 0, n = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess ||
+      cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();  // no device here: never split
+    return 0;
+  }
+  return n;
+}
+
+// Plans the split from the host lengths; false (no split) unless it pays:
+//   - the tensor-core kernel runs, the host lengths are given, KDA_NO_SPLIT is unset;
+//   - the chains fill at most half of the SMs;
+//   - every segment holds at least 1,024 tokens and starts on a multiple of 32 (of
+//     the snapshot stride when snapshots are taken), so that snapshots tile it;
+//   - the local-state pass (two CTAs per non-final segment and head) and the
+//     segment prefill (one CTA per segment and head) each fit in one wave;
+//   - the estimated time, in tokens of one chain, drops by 15 % or more: the longest
+//     non-final segment at 0.8 (the local-state pass skips q, P and O), plus the
+//     longest segment, plus 256 for the extra launches and the combine, against the
+//     longest request unsplit.  (So a two-way split never pays.)
+// Extra segments go, one at a time, to the request whose longest segment is longest.
+bool plan_split(const kda_prefill_args *a, SplitPlan *pl) {
+  if (!a->cu_seqlens_host || a->n_req <= 0 || a->total_tokens <= 0) return false;
+  if (!prefill_tc_supported(a->dk, a->dv, a->in_dtype) || env_flag("KDA_FORCE_SIMT") ||
+      env_flag("KDA_NO_SPLIT"))
+    return false;
+  const int sms = device_sm_count();
+  const long chains = (long)a->n_req * a->H;
+  if (sms <= 0 || 2 * chains > sms) return false;
+  const int max_total = sms / a->H, max_extra = sms / (2 * a->H);
+  const int align = a->snapshot_stride > 0 ? a->snapshot_stride : 32;  // stride % 64 == 0
+  const int min_len = align > 1024 ? align : 1024;
+  const int32_t *cu = a->cu_seqlens_host;
+  std::vector<int> parts(a->n_req, 1);
+  // segment length of request r cut in s parts (the last one takes the rest)
+  auto piece = [&](int r, int s) -> long {
+    const long len = cu[r + 1] - cu[r];
+    const long p = (len + s - 1) / s;
+    return (p + align - 1) / align * align;
+  };
+  // the next part count of request r with every segment but the last at least
+  // min_len tokens and a non-empty last one (alignment may skip a count); 0 if none
+  auto next_parts = [&](int r) -> int {
+    const long len = cu[r + 1] - cu[r];
+    for (int s = parts[r] + 1; s <= parts[r] + max_extra; ++s) {
+      const long p = piece(r, s);
+      if (p < min_len) return 0;
+      if ((s - 1) * p < len) return s;
+    }
+    return 0;
+  };
+  int total = a->n_req, extra = 0;
+  for (;;) {
+    int best = -1, best_parts = 0;
+    long best_len = 0;
+    for (int r = 0; r < a->n_req; ++r) {
+      const int s = next_parts(r);
+      if (s == 0 || total + (s - parts[r]) > max_total || extra + (s - parts[r]) > max_extra)
+        continue;
+      const long len = cu[r + 1] - cu[r];
+      const long longest = parts[r] == 1 ? len : piece(r, parts[r]);
+      if (longest > best_len) {
+        best_len = longest;
+        best = r;
+        best_parts = s;
+      }
+    }
+    if (best < 0) break;
+    total += best_parts - parts[best];
+    extra += best_parts - parts[best];
+    parts[best] = best_parts;
+  }
+  if (extra == 0) return false;
+  long longest = 0, longest_seg = 0, longest_nonfinal = 0;
+  for (int r = 0; r < a->n_req; ++r) {
+    const long len = cu[r + 1] - cu[r];
+    longest = len > longest ? len : longest;
+    const long p = parts[r] > 1 ? piece(r, parts[r]) : len;
+    const long last = len - (parts[r] - 1) * p;
+    longest_seg = std::max(longest_seg, std::max(parts[r] > 1 ? p : 0L, last));
+    if (parts[r] > 1) longest_nonfinal = std::max(longest_nonfinal, p);
+  }
+  if (0.8 * longest_nonfinal + longest_seg + 256.0 > 0.85 * longest) return false;
+
+  pl->n_seg = total;
+  pl->seg_cu.assign(1, 0);
+  pl->first_seg.assign(1, 0);
+  pl->pass1.clear();
+  pl->seg_snap.assign(1, 0);
+  int32_t snaps_before = 0;
+  for (int r = 0; r < a->n_req; ++r) {
+    const int32_t bos = cu[r], eos = cu[r + 1];
+    const long p = parts[r] > 1 ? piece(r, parts[r]) : (long)(eos - bos);
+    for (int k = 0; k < parts[r]; ++k) {
+      const int32_t end = k + 1 < parts[r] ? bos + (int32_t)((k + 1) * p) : eos;
+      if (k + 1 < parts[r]) pl->pass1.push_back((int32_t)pl->seg_cu.size() - 1);
+      pl->seg_cu.push_back(end);
+      if (a->snapshot_stride > 0)
+        pl->seg_snap.push_back(snaps_before + (end - bos) / a->snapshot_stride);
+    }
+    pl->first_seg.push_back((int32_t)pl->seg_cu.size() - 1);
+    if (a->snapshot_stride > 0) snaps_before += (eos - bos) / a->snapshot_stride;
+  }
+  const size_t n = (size_t)pl->n_seg, state = (size_t)a->H * a->dk * a->dv * sizeof(float);
+  size_t off = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = off;
+    off += align256(bytes);
+    return at;
+  };
+  pl->off_cu = take((n + 1) * sizeof(int32_t));
+  pl->off_p1 = take(pl->pass1.size() * sizeof(int32_t));
+  pl->off_snap = take((n + 1) * sizeof(int32_t));
+  pl->off_sloc = take(n * state);
+  pl->off_m = take(n * (size_t)a->H * a->dk * a->dk * sizeof(float));
+  pl->off_sin = take(n * state);
+  pl->bytes = off;
+  return true;
+}
+
 // A failed CUDA call becomes KDA_ERR_CUDA; with KDA_VERBOSE=1 its message goes to stderr.
 kda_status from_cuda(cudaError_t e) {
   if (e == cudaSuccess) return KDA_OK;
   if (env_flag("KDA_VERBOSE")) std::fprintf(stderr, "libkda: CUDA error: %s\n", cudaGetErrorString(e));
   return KDA_ERR_CUDA;
+}
+
+// The split call (see plan_split): local states, combine, segment prefill, final states.
+kda_status run_split(const kda_prefill_args *a, const SplitPlan &pl, char *ws,
+                     const PrefillParams &base, cudaStream_t s) {
+  int32_t *seg_cu = reinterpret_cast<int32_t *>(ws + pl.off_cu);
+  int32_t *p1 = reinterpret_cast<int32_t *>(ws + pl.off_p1);
+  int32_t *seg_snap = reinterpret_cast<int32_t *>(ws + pl.off_snap);
+  float *sloc = reinterpret_cast<float *>(ws + pl.off_sloc);
+  float *m = reinterpret_cast<float *>(ws + pl.off_m);
+  float *s_start = reinterpret_cast<float *>(ws + pl.off_sin);
+  const size_t state = (size_t)a->H * a->dk * a->dv, trans = (size_t)a->H * a->dk * a->dk;
+  // the plan's small tables (pageable host memory: each copy has left the host
+  // buffer when it returns)
+  cudaError_t e = cudaMemcpyAsync(seg_cu, pl.seg_cu.data(), pl.seg_cu.size() * sizeof(int32_t),
+                                  cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess)
+    e = cudaMemcpyAsync(p1, pl.pass1.data(), pl.pass1.size() * sizeof(int32_t),
+                        cudaMemcpyHostToDevice, s);
+  if (e == cudaSuccess && a->snapshot_stride > 0)
+    e = cudaMemcpyAsync(seg_snap, pl.seg_snap.data(), pl.seg_snap.size() * sizeof(int32_t),
+                        cudaMemcpyHostToDevice, s);
+  if (e != cudaSuccess) return from_cuda(e);
+
+  // local states and transitions of the non-final segments
+  PrefillParams lp = base;
+  lp.q = nullptr;
+  lp.o = nullptr;
+  lp.initial_state = nullptr;
+  lp.final_state = nullptr;
+  lp.snapshot_stride = 0;
+  lp.cu_snapshots = nullptr;
+  lp.snapshots = nullptr;
+  lp.cu_seqlens = seg_cu;
+  lp.n_req = (int)pl.pass1.size();
+  lp.order = p1;
+  lp.local_mode = 1;
+  lp.s_loc = sloc;
+  lp.m = m;
+  if ((e = launch_prefill_tc(lp, a->in_dtype, KDA_F32, s)) != cudaSuccess) return from_cuda(e);
+
+  // start states of every segment: the request's initial state, then the combine
+  for (int r = 0; r < a->n_req; ++r) {
+    const int row0 = pl.first_seg[r], n = pl.first_seg[r + 1] - row0;
+    const float *s_init = a->initial_state ? a->initial_state + (size_t)r * state : nullptr;
+    if (n == 1)
+      e = s_init ? cudaMemcpyAsync(s_start + row0 * state, s_init, state * sizeof(float),
+                                   cudaMemcpyDeviceToDevice, s)
+                 : cudaMemsetAsync(s_start + row0 * state, 0, state * sizeof(float), s);
+    else
+      e = launch_combine(sloc + row0 * state, m + row0 * trans, s_init, n - 1, a->H, a->dk,
+                         a->dv, s_start + row0 * state, s_start + (row0 + n - 1) * state, s);
+    if (e != cudaSuccess) return from_cuda(e);
+  }
+
+  // every segment from its start state; the final states land in place
+  PrefillParams sp = base;
+  sp.cu_seqlens = seg_cu;
+  sp.n_req = pl.n_seg;
+  sp.order = nullptr;
+  sp.initial_state = s_start;
+  sp.final_state = s_start;
+  sp.cu_snapshots = a->snapshot_stride > 0 ? seg_snap : nullptr;
+  if ((e = launch_prefill_tc(sp, a->in_dtype, a->out_dtype, s)) != cudaSuccess)
+    return from_cuda(e);
+  if (a->final_state)
+    for (int r = 0; r < a->n_req; ++r) {
+      const int last = pl.first_seg[r + 1] - 1;
+      e = cudaMemcpyAsync(a->final_state + (size_t)r * state, s_start + last * state,
+                          state * sizeof(float), cudaMemcpyDeviceToDevice, s);
+      if (e != cudaSuccess) return from_cuda(e);
+    }
+  return KDA_OK;
 }
 
 // The current thread's CUDA context, through the driver entry point the
@@ -177,18 +399,43 @@ unsigned int *device_status_word() {
 
 using namespace kda;
 
+namespace kda {
+// kda_prefill_chunked, with the context-parallel split allowed or not
+kda_status prefill_call(const kda_prefill_args *a, void *workspace, size_t workspace_bytes,
+                        void *stream, bool allow_split);
+}  // namespace kda
+
 extern "C" {
 
 size_t kda_prefill_workspace_size(const kda_prefill_args *args) {
   if (check_prefill(args) != KDA_OK) return 0;
+  kda::SplitPlan plan;
+  if (kda::plan_split(args, &plan)) return plan.bytes;
   return prefill_ws(args->n_req);
+}
+
+int32_t kda_prefill_split_segments(const kda_prefill_args *args) {
+  if (check_prefill(args) != KDA_OK) return 0;
+  kda::SplitPlan plan;
+  return kda::plan_split(args, &plan) ? plan.n_seg : 0;
 }
 
 kda_status kda_prefill_chunked(const kda_prefill_args *a, void *workspace,
                                size_t workspace_bytes, void *stream) {
+  return kda::prefill_call(a, workspace, workspace_bytes, stream, true);
+}
+
+}  // extern "C"
+
+namespace kda {
+
+kda_status prefill_call(const kda_prefill_args *a, void *workspace, size_t workspace_bytes,
+                        void *stream, bool allow_split) {
   kda_status st = check_prefill(a);
   if (st != KDA_OK) return st;
   if (a->n_req == 0) return KDA_OK;
+  // the unsplit call's workspace (the split asks for more, and falls back to the
+  // unsplit call when it does not get it)
   const size_t need = prefill_ws(a->n_req);
   if (need > 0 && (!workspace || workspace_bytes < need ||
                    (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0))
@@ -211,19 +458,29 @@ kda_status kda_prefill_chunked(const kda_prefill_args *a, void *workspace,
   p.wait_ns = wait_limit_ns();
   p.status = device_status_word();
   if (!p.status) return KDA_ERR_CUDA;
+  // the tensor-core kernel needs at least one token to build its TMA maps
+  const bool use_tc = prefill_tc_supported(a->dk, a->dv, a->in_dtype) && a->total_tokens > 0 &&
+                      !env_flag("KDA_FORCE_SIMT");
+  // few chains: the context-parallel split, when the workspace holds it
+  if (use_tc && allow_split && workspace && (reinterpret_cast<uintptr_t>(workspace) & 255u) == 0) {
+    SplitPlan plan;
+    if (plan_split(a, &plan) && workspace_bytes >= plan.bytes)
+      return run_split(a, plan, static_cast<char *>(workspace), p, s);
+  }
   if (need > 0) {
     int32_t *order = static_cast<int32_t *>(workspace);
     cudaError_t e = launch_schedule(a->cu_seqlens, a->n_req, order, s);
     if (e != cudaSuccess) return KDA_ERR_CUDA;
     p.order = order;
   }
-  // the tensor-core kernel needs at least one token to build its TMA maps
-  const bool use_tc = prefill_tc_supported(a->dk, a->dv, a->in_dtype) && a->total_tokens > 0 &&
-                      !env_flag("KDA_FORCE_SIMT");
   if (use_tc) return from_cuda(launch_prefill_tc(p, a->in_dtype, a->out_dtype, s));
   p.n_slices = prefill_simt_slices(a->dk, a->dv, false);
   return from_cuda(launch_prefill_simt(p, a->in_dtype, a->out_dtype, s));
 }
+
+}  // namespace kda
+
+extern "C" {
 
 size_t kda_local_state_workspace_size(const kda_local_state_args *a) {
   (void)a;
@@ -408,7 +665,8 @@ extern "C" kda_status kda_prefill_chunked_noalloc(const kda_prefill_args *args, 
   if (args->n_req > KDA_NOALLOC_MAX_REQUESTS) return KDA_ERR_WORKSPACE;
   int32_t *scratch = kda::noalloc_scratch();
   if (!scratch) return KDA_ERR_CUDA;
-  return kda_prefill_chunked(args, scratch, sizeof(kda::g_noalloc_order), stream);
+  // no context-parallel split: its states would need more than the fixed scratch
+  return kda::prefill_call(args, scratch, sizeof(kda::g_noalloc_order), stream, false);
 }
 
 // ---------------------------------------------------------------------------

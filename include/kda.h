@@ -144,16 +144,40 @@ typedef struct kda_prefill_args {
 } kda_prefill_args;
 
 /* Bytes of device workspace kda_prefill_chunked needs for these arguments
- * (a multiple of 256; 0 is possible).  Pure host computation; returns 0 for
- * invalid arguments (kda_prefill_chunked then reports the error). */
+ * (a multiple of 256; 0 is possible).  Host computation (it reads the current
+ * device's SM count); returns 0 for invalid arguments (kda_prefill_chunked then
+ * reports the error).  When the call would be split (see below) this is the
+ * split's workspace: the segment tables and three fp32 states per segment and
+ * head, for example 19 MB for one 8,192-token request with H = 32, d = 128. */
 size_t kda_prefill_workspace_size(const kda_prefill_args *args);
 
 /* Run chunked prefill.  workspace: device memory of at least
  * kda_prefill_workspace_size(args) bytes, 256-byte aligned, owned by the
  * caller and not used concurrently by another call; workspace_bytes: its
- * size.  Returns KDA_OK once the work is enqueued on `stream`. */
+ * size.  Returns KDA_OK once the work is enqueued on `stream`.
+ *
+ * Few chains.  A (request, head) chain runs its chunks in order on one SM, so
+ * a call with few chains leaves most SMs idle.  When the tensor-core kernel
+ * runs, cu_seqlens_host is given, the chains fill at most half of the SMs and
+ * some request is long enough (segments of at least 1,024 tokens, starting on
+ * multiples of 32 or of snapshot_stride), the call is split the way KDA
+ * context parallelism splits a sequence ("Kimi K3 开源日来了", Infra section,
+ * first layer): the local states and transitions of every non-final segment
+ * (kda_chunk_local_state), an exact combine per request (kda_state_combine),
+ * then every segment from its start state.  o, the snapshots and the final
+ * states equal the unsplit call's up to rounding (not bit for bit); the call
+ * then also makes small host-to-device copies of its segment tables from
+ * pageable memory, which a CUDA graph capture does not accept.  The split is
+ * skipped when the workspace is smaller than kda_prefill_workspace_size asks
+ * for (the call then needs only the unsplit workspace), and when the
+ * environment variable KDA_NO_SPLIT is set to a non-zero value. */
 kda_status kda_prefill_chunked(const kda_prefill_args *args, void *workspace,
                                size_t workspace_bytes, void *stream);
+
+/* Segments the call would run after the context-parallel split described
+ * above, 0 when it would not be split.  Host computation, like
+ * kda_prefill_workspace_size. */
+int32_t kda_prefill_split_segments(const kda_prefill_args *args);
 
 /* Largest n_req that kda_prefill_chunked_noalloc accepts. */
 #define KDA_NOALLOC_MAX_REQUESTS 16384
@@ -169,7 +193,8 @@ kda_status kda_prefill_chunked(const kda_prefill_args *args, void *workspace,
  *   - latency-critical code that cannot call cudaMalloc, which may
  *     synchronise the device and take milliseconds.
  *
- * Same arguments, results and error codes as kda_prefill_chunked, except
+ * Same arguments, results and error codes as kda_prefill_chunked, never
+ * split (its scratch has no room for segment states), and except
  * that the scratch (one int32 per request: the longest-first work order)
  * lives in a fixed array inside libkda.so instead of a caller workspace:
  *   - the array holds KDA_NOALLOC_MAX_REQUESTS int32 (64 KiB) and is resident
