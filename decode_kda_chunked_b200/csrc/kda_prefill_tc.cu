@@ -702,7 +702,10 @@ __global__ void __launch_bounds__(NT + 64, 1)
     // of chunk m+1 could load).  Its barrier is one of a pair, by chunk parity, so group
     // A may finish a gate before group B has taken the previous one.
     bool ok = true;
-    if (n_chunks > 0 && (ok = wait_tma(0))) w_gate(0);
+    if (n_chunks > 0 && (ok = wait_tma(0))) {
+      w_gate(0);
+      wsync();  // every warp's channels of the table before any row operand reads them
+    }
     for (int m = 0; ok && m < n_chunks; ++m) {
       // chunk m-1's O^T and Y^T products are done: gamma*Q/K are free (and, through
       // group B, chunk m-2's last products are done too)
