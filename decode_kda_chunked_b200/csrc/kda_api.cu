@@ -167,9 +167,10 @@ int device_sm_count() {
 //   - the local-state pass (two CTAs per non-final segment and head) and the
 //     segment prefill (one CTA per segment and head) each fit in one wave;
 //   - the estimated time, in tokens of one chain, drops by 15 % or more: the longest
-//     non-final segment at 0.8 (the local-state pass skips q, P and O), plus the
-//     longest segment, plus 256 for the extra launches and the combine, against the
-//     longest request unsplit.  (So a two-way split never pays.)
+//     non-final segment at 0.95 (the local-state pass skips q, P and O but keeps the
+//     gate, the row operands and the solve: measured 4.0 against 4.3 us per chunk),
+//     plus the longest segment, plus 256 for the extra launches and the combine,
+//     against the longest request unsplit.  (So a two-way split never pays.)
 // Extra segments go, one at a time, to the request whose longest segment is longest.
 bool plan_split(const kda_prefill_args *a, SplitPlan *pl) {
   if (!a->cu_seqlens_host || a->n_req <= 0 || a->total_tokens <= 0) return false;
@@ -232,7 +233,7 @@ bool plan_split(const kda_prefill_args *a, SplitPlan *pl) {
     longest_seg = std::max(longest_seg, std::max(parts[r] > 1 ? p : 0L, last));
     if (parts[r] > 1) longest_nonfinal = std::max(longest_nonfinal, p);
   }
-  if (0.8 * longest_nonfinal + longest_seg + 256.0 > 0.85 * longest) return false;
+  if (0.95 * longest_nonfinal + longest_seg + 256.0 > 0.85 * longest) return false;
 
   pl->n_seg = total;
   pl->seg_cu.assign(1, 0);
