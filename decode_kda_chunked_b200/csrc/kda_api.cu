@@ -129,8 +129,8 @@ size_t prefill_ws(int n_req) {
 // in order, so a call with fewer chains than SMs leaves most of the GPU idle.  Such a
 // call is run as KDA context parallelism inside one device ("Kimi K3 开源日来了",
 // Infra section, first layer): long requests are cut into segments; a local-state
-// pass gives each non-final segment its zero-start state S_loc and transition M (two
-// CTAs per segment and head, all in one wave); an exact combine per request recovers
+// pass gives each non-final segment its zero-start state S_loc and transition M (one
+// CTA per segment and head, all in one wave); an exact combine per request recovers
 // every segment's start state; and one prefill over all segments, each from its
 // start state, writes o, the snapshots and (through the last segment) the final
 // state.  The results equal the unsplit call's up to rounding.
@@ -164,11 +164,12 @@ int device_sm_count() {
 //   - the chains fill at most half of the SMs;
 //   - every segment holds at least 1,024 tokens and starts on a multiple of 32 (of
 //     the snapshot stride when snapshots are taken), so that snapshots tile it;
-//   - the local-state pass (two CTAs per non-final segment and head) and the
-//     segment prefill (one CTA per segment and head) each fit in one wave;
+//   - the local-state pass (one CTA per non-final segment and head) and the segment
+//     prefill (one CTA per segment and head) each fit in one wave;
 //   - the estimated time, in tokens of one chain, drops by 15 % or more: the longest
-//     non-final segment at 0.95 (the local-state pass skips q, P and O but keeps the
-//     gate, the row operands and the solve: measured 4.0 against 4.3 us per chunk),
+//     non-final segment at 0.9 (the local-state pass skips q, P and O but keeps the
+//     gate, the row operands and the solve, and adds the transition's columns:
+//     measured 4.25 against 4.7 us per chunk),
 //     plus the longest segment, plus 256 for the extra launches and the combine,
 //     against the longest request unsplit.  (So a two-way split never pays.)
 // Extra segments go, one at a time, to the request whose longest segment is longest.
@@ -180,7 +181,7 @@ bool plan_split(const kda_prefill_args *a, SplitPlan *pl) {
   const int sms = device_sm_count();
   const long chains = (long)a->n_req * a->H;
   if (sms <= 0 || 2 * chains > sms) return false;
-  const int max_total = sms / a->H, max_extra = sms / (2 * a->H);
+  const int max_total = sms / a->H, max_extra = max_total;
   const int align = a->snapshot_stride > 0 ? a->snapshot_stride : 32;  // stride % 64 == 0
   const int min_len = align > 1024 ? align : 1024;
   const int32_t *cu = a->cu_seqlens_host;
@@ -233,7 +234,7 @@ bool plan_split(const kda_prefill_args *a, SplitPlan *pl) {
     longest_seg = std::max(longest_seg, std::max(parts[r] > 1 ? p : 0L, last));
     if (parts[r] > 1) longest_nonfinal = std::max(longest_nonfinal, p);
   }
-  if (0.95 * longest_nonfinal + longest_seg + 256.0 > 0.85 * longest) return false;
+  if (0.9 * longest_nonfinal + longest_seg + 256.0 > 0.85 * longest) return false;
 
   pl->n_seg = total;
   pl->seg_cu.assign(1, 0);

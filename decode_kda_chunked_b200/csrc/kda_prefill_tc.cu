@@ -131,7 +131,8 @@ constexpr uint32_t TM_L = 128;   // [L_k ; L_q]: A operand of A|P (lanes 0-31 | 
 constexpr uint32_t TM_AP = 256;  // A (lanes 0-31) | P (lanes 32-63), 32 columns
 constexpr uint32_t TM_Y = 288;   // V^T -> Y^T
 constexpr uint32_t TM_U = 320;   // U^T
-constexpr uint32_t TM_O = 352;   // O^T
+constexpr uint32_t TM_O = 352;   // O^T (local state: Y_M^T)
+constexpr uint32_t TM_M = 384;   // local state: M^T, the segment's transition
 constexpr uint32_t TM_COLS = 512;
 
 struct TcMaps {
@@ -225,7 +226,13 @@ __device__ unsigned long long g_phase_cycles[16];
 #endif
 
 // LOGITS: the gate arrives as bf16 logits (fused gate activation) instead of fp32 g.
-template <typename TOut, bool LOGITS>
+// LOCAL: the local state of a segment (context-parallel pass 1): S_loc from a zero state
+// with the segment's values, and, in the same pass over the chunks, the transition M
+// from the identity with zero values (the augmented columns [V | 0] from [0 | I]), both
+// sharing the chunk's gate, row operands, A, T and Khat.  M^T lives in TMEM columns the
+// local state leaves free: Y_M^T where O^T would be, U_M^T over Y_S^T once U_S^T has
+// read it.
+template <typename TOut, bool LOGITS, bool LOCAL>
 __global__ void __launch_bounds__(NT + 64, 1)
     prefill_tc_kernel(const PrefillParams p, const __grid_constant__ TcMaps maps) {
   extern __shared__ unsigned char smem_raw[];
@@ -247,7 +254,8 @@ __global__ void __launch_bounds__(NT + 64, 1)
   uint64_t *ops_tb = bars + 9;    // group A -> control: T Diag(beta) ready
   uint64_t *ops_sc = bars + 10;   // group B -> control: S^T scaled by gamma_31
   uint64_t *gate_ok = bars + 11;  // [2] group A -> group B: cumulative gate of a chunk ready
-  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bars + 13);
+  uint64_t *bar_us = bars + 13;   // local state: commit of U_S^T (before U_M^T overwrites Y_S^T)
+  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(bars + 14);
   volatile int *s_abort = reinterpret_cast<volatile int *>(s_tmem + 1);
 
   const int tid = threadIdx.x, warp = tid >> 5, lane_id = tid & 31;
@@ -258,16 +266,12 @@ __global__ void __launch_bounds__(NT + 64, 1)
   const int l = 32 * qd + lane_id;                 // its TMEM lane / channel
   const uint32_t lane_base = (uint32_t)(32 * qd) << 16;
   const int H = p.H;
-  // Local-state mode (context-parallel pass 1): CTA part 0 runs the segment from a
-  // zero state with its values (-> S_loc), part 1 from the identity with zero values
-  // (-> M = A_L ... A_1); the two are the column blocks of the augmented state.
+  // one CTA per (request or segment, head)
   const int pairs = p.n_req * H;
-  const int part = p.local_mode ? (int)(blockIdx.x / pairs) : 0;
   const int rem = (int)(blockIdx.x % pairs);
   const int r = p.order ? p.order[rem / H] : rem / H;
   const int h = rem % H;
-  const bool has_q = !p.local_mode;
-  const bool zero_v = p.local_mode && part == 1;
+  const bool has_q = !p.local_mode;  // (a runtime flag keeps the register allocation tight)
   const uint64_t wait_ns = p.wait_ns ? p.wait_ns : 2000000000ull;
   const int bos = p.cu_seqlens[r], eos = p.cu_seqlens[r + 1];
   const int len = eos - bos;
@@ -297,6 +301,7 @@ __global__ void __launch_bounds__(NT + 64, 1)
     mbar_init(ops_sc, (NT - NA) / 32);
     mbar_init(gate_ok, NA / 32);
     mbar_init(gate_ok + 1, NA / 32);
+    mbar_init(bar_us, 1);
     *s_abort = 0;
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
@@ -408,17 +413,29 @@ __global__ void __launch_bounds__(NT + 64, 1)
         for (int s = 0; s < DH / 8; ++s) {
           if (has_q) mma_tf32_ts(tm + TM_O, tm + TM_S + 8 * s, sw128_desc(gq, C, s), id, s > 0);
           mma_tf32_ts(tm + TM_Y, tm + TM_S + 8 * s, sw128_desc(gk, C, s), idn, true);
+          // local state: Y_M^T = -M^T (gamma K)^T (zero values)
+          if (LOCAL) mma_tf32_ts(tm + TM_O, tm + TM_M + 8 * s, sw128_desc(gk, C, s), idn, s > 0);
         }
         commit(bar_oy, m);
       };
-      // U^T = Y^T (T Diag(beta))^T
-      auto mma_u = [&](int m) {
+      // U^T = Y^T (T Diag(beta))^T; local state: then U_M^T = Y_M^T (T Diag(beta))^T over
+      // Y_S^T, once U_S^T is done reading it
+      uint32_t ph_us = 0;
+      auto mma_u = [&](int m) -> bool {
         const uint32_t tb = smem_u32(sm + tb_off(m));
         const uint32_t id = idesc_tf32(C);
 #pragma unroll
         for (int s = 0; s < C / 8; ++s)
           mma_tf32_ts(tm + TM_U, tm + TM_Y + 8 * s, sw128_desc(tb, C, s), id, s > 0);
+        if constexpr (LOCAL) {
+          commit(bar_us, m);
+          if (!cwait(bar_us, ph_us)) return false;
+#pragma unroll
+          for (int s = 0; s < C / 8; ++s)
+            mma_tf32_ts(tm + TM_Y, tm + TM_O + 8 * s, sw128_desc(tb, C, s), id, s > 0);
+        }
         commit(bar_u, m);
+        return true;
       };
       // O^T += U^T P^T and S^T += U^T Khat (S^T already scaled by gamma_31)
       auto mma_fin = [&](int m) {
@@ -428,6 +445,8 @@ __global__ void __launch_bounds__(NT + 64, 1)
         for (int s = 0; s < C / 8; ++s) {
           if (has_q) mma_tf32_ts(tm + TM_O, tm + TM_U + 8 * s, sw128_desc(pp, C, s), id32, true);
           mma_tf32_ts(tm + TM_S, tm + TM_U + 8 * s, sw128_desc(kh, DH, s), id128, true);
+          // local state: M^T += U_M^T Khat
+          if (LOCAL) mma_tf32_ts(tm + TM_M, tm + TM_Y + 8 * s, sw128_desc(kh, DH, s), id128, true);
         }
         commit(bar_fin, m);
       };
@@ -443,7 +462,7 @@ __global__ void __launch_bounds__(NT + 64, 1)
           if (m + 2 < n_chunks) issue_tma(m + 2);
           if (!cwait(ops_tb, ph_tb)) break;
           if (!cwait(bar_oy, ph_oy)) break;  // Y^T is U^T's A operand
-          mma_u(m);
+          if (!mma_u(m)) break;
         }
       } else {
         for (int m = 0; m < n_chunks; ++m) {
@@ -757,10 +776,13 @@ __global__ void __launch_bounds__(NT + 64, 1)
         const int c0 = 64 * cg + 8 * q8;
         float v[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j)
-          v[j] = p.local_mode ? ((part == 1 && c0 + j == l) ? 1.f : 0.f)
-                              : (s0 ? s0[(size_t)(c0 + j) * DH + l] : 0.f);
+        for (int j = 0; j < 8; ++j) v[j] = (!LOCAL && s0) ? s0[(size_t)(c0 + j) * DH + l] : 0.f;
         tmem_st8(tm + lane_base + TM_S + c0, v);
+        if constexpr (LOCAL) {  // M^T = I
+#pragma unroll
+          for (int j = 0; j < 8; ++j) v[j] = c0 + j == l ? 1.f : 0.f;
+          tmem_st8(tm + lane_base + TM_M + c0, v);
+        }
       }
       tmem_wait_st();
     }
@@ -768,21 +790,25 @@ __global__ void __launch_bounds__(NT + 64, 1)
     // ---- scale(n): S^T <- S^T Diag(gamma_31) once the O^T and Y^T products read S^T ----
     auto w_scale = [&](int n) {
       const float *gc = GC + (n & 3) * DH;
+      auto scale_cols = [&](uint32_t base) {
 #pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int c0 = 64 * cg + 16 * q;
-        float v[16];
-        tmem_ld16(tm + lane_base + TM_S + c0, v);
-        tmem_wait_ld();
+        for (int q = 0; q < 4; ++q) {
+          const int c0 = 64 * cg + 16 * q;
+          float v[16];
+          tmem_ld16(tm + lane_base + base + c0, v);
+          tmem_wait_ld();
 #pragma unroll
-        for (int j = 0; j < 16; j += 8) {
-          float f[8];
-          ld8f(gc + c0 + j, f);
+          for (int j = 0; j < 16; j += 8) {
+            float f[8];
+            ld8f(gc + c0 + j, f);
 #pragma unroll
-          for (int e = 0; e < 8; e += 2) mul2(v[j + e], v[j + e + 1], f[e], f[e + 1]);
+            for (int e = 0; e < 8; e += 2) mul2(v[j + e], v[j + e + 1], f[e], f[e + 1]);
+          }
+          tmem_st16(tm + lane_base + base + c0, v);
         }
-        tmem_st16(tm + lane_base + TM_S + c0, v);
-      }
+      };
+      scale_cols(TM_S);
+      if constexpr (LOCAL) scale_cols(TM_M);  // the transition scales like the state
       tmem_wait_st();
     };
 
@@ -870,7 +896,7 @@ __global__ void __launch_bounds__(NT + 64, 1)
       // chunk index ((l & 63) >> 3) ^ (j & 7), so eight offsets serve all sixteen rows
       const unsigned char *row0 = sm + OFF_RAW + (m & 1) * RAW_BYTES + R_V + (l >> 6) * 4096 +
                                   16 * cg * 128 + (l & 7) * 2;
-      const int c8 = (l & 63) >> 3, nv = zero_v ? 0 : nr - 16 * cg;
+      const int c8 = (l & 63) >> 3, nv = nr - 16 * cg;
       float v16[16];
 #pragma unroll
       for (int j = 0; j < 16; ++j) {
@@ -918,19 +944,24 @@ __global__ void __launch_bounds__(NT + 64, 1)
       KDA_PHASE(14);
     }
 
-    float *fin = p.local_mode ? (part == 0 ? p.s_loc : p.m) : p.final_state;
-    if (ok && fin) {
-      float *dst = fin + ((size_t)(r * H + h)) * DH * DH;
-      tc_fence_after();
+    // the final state (local state: S_loc and the transition M)
+    auto write_state = [&](float *dst_base, uint32_t col) {
+      float *dst = dst_base + ((size_t)(r * H + h)) * DH * DH;
 #pragma unroll 1
       for (int q8 = 0; q8 < 8; ++q8) {
         const int k0 = 64 * cg + 8 * q8;
         float v[8];
-        tmem_ld8(tm + lane_base + TM_S + k0, v);
+        tmem_ld8(tm + lane_base + col + k0, v);
         tmem_wait_ld();
 #pragma unroll
         for (int j = 0; j < 8; ++j) dst[(size_t)(k0 + j) * DH + l] = v[j];
       }
+    };
+    float *fin = LOCAL ? p.s_loc : p.final_state;
+    if (ok && fin) {
+      tc_fence_after();
+      write_state(fin, TM_S);
+      if constexpr (LOCAL) write_state(p.m, TM_M);
     }
   }
 #ifdef KDA_PHASE_PROFILE
@@ -1011,7 +1042,7 @@ cudaError_t launch_prefill_tc(const PrefillParams &p, kda_dtype in_dtype, kda_dt
       !(p.g_logits ? encode_map(&maps.g, p.g_logits, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, W, T, 64)
                    : encode_map(&maps.g, p.g, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 4, W, T, 32)))
     return cudaErrorInvalidValue;
-  const unsigned grid = (unsigned)(p.n_req * p.H * (p.local_mode ? 2 : 1));
+  const unsigned grid = (unsigned)(p.n_req * p.H);
   auto run = [&](auto kernel) -> cudaError_t {
     const cudaError_t e =
         cudaFuncSetAttribute(kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)SMEM_ALLOC);
@@ -1020,10 +1051,14 @@ cudaError_t launch_prefill_tc(const PrefillParams &p, kda_dtype in_dtype, kda_dt
     return cudaGetLastError();
   };
   const bool logits = p.g_logits != nullptr;
+  if (p.local_mode)  // S_loc and M in one pass (no o)
+    return logits ? run(prefill_tc_kernel<float, true, true>)
+                  : run(prefill_tc_kernel<float, false, true>);
   if (out_dtype == KDA_BF16)
-    return logits ? run(prefill_tc_kernel<__nv_bfloat16, true>)
-                  : run(prefill_tc_kernel<__nv_bfloat16, false>);
-  return logits ? run(prefill_tc_kernel<float, true>) : run(prefill_tc_kernel<float, false>);
+    return logits ? run(prefill_tc_kernel<__nv_bfloat16, true, false>)
+                  : run(prefill_tc_kernel<__nv_bfloat16, false, false>);
+  return logits ? run(prefill_tc_kernel<float, true, false>)
+                : run(prefill_tc_kernel<float, false, false>);
 }
 
 }  // namespace kda

@@ -53,10 +53,10 @@ def _check_oracle(inp, out, stride, pairs):
 
 
 def test_single_sequence_is_split_and_matches_the_oracle():
-    """B=1, H=32, T=8,192 (32 chains): three segments of the one sequence."""
+    """B=1, H=32, T=8,192 (32 chains): four segments of the one sequence."""
     inp = I.single_seq()
     x = inp.to(DEV)
-    assert _segments(x, 512) == 3
+    assert _segments(x, 512) == 4
     out = _run(x, 512)
     _check_oracle(inp, out, 512, [(0, h) for h in (0, 9, 21, 31)])
 

@@ -39,12 +39,12 @@ def _segments(monkeypatch, lengths, H, stride=0, sms=148, dk=128):
 
 
 def test_single_sequence_fills_one_wave_per_pass(monkeypatch):
-    # 32 chains on 148 SMs: at most 148 // 32 = 4 segments per head in the segment
-    # prefill and 148 // 64 = 2 non-final segments in the local-state pass -> 3
+    # 32 chains on 148 SMs: at most 148 // 32 = 4 segments per head, in the local-state
+    # pass (one CTA per non-final segment and head) and in the segment prefill
     n, ws = _segments(monkeypatch, [8192], H=32)
-    assert n == 3
+    assert n == 4
     state = 32 * 128 * 128 * 4
-    assert ws >= 3 * 3 * state  # S_loc, M and start states of every segment
+    assert ws >= 3 * 4 * state  # S_loc, M and start states of every segment
 
 
 def test_split_switch_and_unsupported_calls(monkeypatch):
@@ -78,19 +78,19 @@ def test_few_heads_split_down_to_the_minimum_segment(monkeypatch):
 
 
 def test_longest_request_is_split_first(monkeypatch):
-    # 32 chains: up to 148 // 32 = 4 extra segments; the 9,000-token request takes the
-    # first three (pieces 4,512, 3,008, 2,272), then the 3,000-token one is longest
-    assert _segments(monkeypatch, [3000, 9000], H=16)[0] == 6
-    # the wave limits allow 148 // (2 * 32) = 2 extra segments: two requests cut in
-    # two each would not pay
+    # 16 heads: up to 148 // 16 = 9 segments.  The 9,000-token request takes the first
+    # three extra ones (pieces 4,512, 3,008, 2,272), the 3,000-token one the next (1,504),
+    # then 9,000 again (1,824, 1,504), and at a tie the first request (3 x 1,024)
+    assert _segments(monkeypatch, [3000, 9000], H=16)[0] == 9
+    # 32 heads: 4 segments in all; two requests cut in two each would not pay
     assert _segments(monkeypatch, [9000, 9000], H=32)[0] == 0
-    assert _segments(monkeypatch, [9000], H=32)[0] == 3
+    assert _segments(monkeypatch, [9000], H=32)[0] == 4
     # too many chains for any split
     assert _segments(monkeypatch, [3000, 9000], H=64)[0] == 0
 
 
 def test_snapshot_stride_aligns_segments(monkeypatch):
     # segments start on multiples of the stride; with 4,096 they must hold 4,096 tokens
-    assert _segments(monkeypatch, [8192], H=32, stride=512)[0] == 3  # 3,072 x 2 + 2,048
+    assert _segments(monkeypatch, [8192], H=32, stride=512)[0] == 4  # 2,048 each
     assert _segments(monkeypatch, [8192], H=32, stride=4096)[0] == 0  # only two parts
     assert _segments(monkeypatch, [16384], H=16, stride=4096)[0] == 4
