@@ -640,7 +640,9 @@ __global__ void __launch_bounds__(NTH, 1) bwd_prep_kernel(const BwdParams p) {
   // Khat = exp(G_last - G) K, Gam = exp(G_last); A and T for the gradient pass
   for (int e = tid; e < C * D; e += NTH) {
     const int t = e / D, c = e % D;
-    p.wKh[ch * C * D + e] = sK[e] * exp2f(sG[(C - 1) * D + c] - sG[t * D + c]);
+    const float kh = sK[e] * exp2f(sG[(C - 1) * D + c] - sG[t * D + c]);
+    // the tensor-core state pass reads Khat as a tf32 operand, copied as it is
+    p.wKh[ch * C * D + e] = kPrepTensorCores<D, TIn> ? tf32_round(kh) : kh;
   }
   if (tid < D) p.wGam[ch * D + tid] = exp2f(sG[(C - 1) * D + tid]);
   for (int e = tid; e < C * C; e += NTH) {
@@ -652,18 +654,23 @@ __global__ void __launch_bounds__(NTH, 1) bwd_prep_kernel(const BwdParams p) {
 // ---------------------------------------------------------------------------
 // bwd_state: the serial pass over chunk-end cotangents, last chunk first.  The
 // recurrence acts on every value column of dS on its own (as the forward acts
-// on the columns of S), so one CTA owns a 16-column slice of one chain; the
-// chunk's Khat and W tiles are copied to shared memory with cp.async.
+// on the columns of S), so one CTA owns a 32-column slice of one chain.  The
+// chunk's Khat and W tiles are copied to shared memory with cp.async one chunk
+// ahead (two buffers), and the thread's X, Y and Gam entries of the next chunk are
+// loaded into registers while the current chunk is computed, so the serial chain
+// waits on no memory latency of its own operands.
 // ---------------------------------------------------------------------------
-constexpr int SC = 16;  // state columns per CTA
+constexpr int SC = 32;             // state columns per CTA
+constexpr int ST_NTH = 16 * SC;    // threads (ty, tx): 16 x SC
 
-// Shared layout: the chunk's Khat and W tiles (as copied), the CTA's 16-column slice of
-// dS held transposed (row stride LT, so a thread reads four consecutive k of its
-// column as one float4 on distinct banks), and the dU slice.
+// Shared layout: two buffers of the chunk's Khat and W tiles (as copied), the CTA's
+// 32-column slice of dS held transposed (row stride LT, so a thread reads four
+// consecutive k of its column as one float4 on distinct banks), and the dU slice.
 template <int D>
 struct StateLayout {
   static constexpr int LT = D + 4;
-  static constexpr int oKh = 0, oW = oKh + C * D, oS = oW + C * D, oU = oS + SC * LT;
+  static constexpr int oBuf = 0, BUF = 2 * C * D;  // Khat tile, then the W tile
+  static constexpr int oS = oBuf + 2 * BUF, oU = oS + SC * LT;
   static constexpr int total = oU + C * SC;
   static constexpr size_t bytes = sizeof(float) * total;
 };
@@ -672,24 +679,61 @@ __device__ __forceinline__ void cp_async16(void *smem, const void *gmem) {
   const uint32_t a = (uint32_t)__cvta_generic_to_shared(smem);
   asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(a), "l"(gmem) : "memory");
 }
-__device__ __forceinline__ void cp_async_wait_all() {
-  asm volatile("cp.async.commit_group;\n\tcp.async.wait_group 0;" ::: "memory");
+__device__ __forceinline__ void cp_async_commit() {
+  asm volatile("cp.async.commit_group;" ::: "memory");
+}
+// wait until at most N of this thread's committed groups are still in flight
+template <int N>
+__device__ __forceinline__ void cp_async_wait() {
+  asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
 
 template <int D>
-__global__ void __launch_bounds__(NTH) bwd_state_kernel(const BwdParams p) {
+__global__ void __launch_bounds__(ST_NTH, 1) bwd_state_kernel(const BwdParams p) {
   using L = StateLayout<D>;
   constexpr int NSL = D / SC, MI = D / 16, LT = L::LT;
+  static_assert(NSL >= 1 && D % SC == 0 && MI % 4 == 0, "state slices");
   extern __shared__ float4 smem_f4[];
   float *sm = reinterpret_cast<float *>(smem_f4);
-  float *sKh = sm + L::oKh, *sW = sm + L::oW, *sdST = sm + L::oS, *sdU = sm + L::oU;
-  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  float *sdST = sm + L::oS, *sdU = sm + L::oU;
+  const int tid = threadIdx.x, ty = tid / SC, tx = tid % SC;
   const int H = p.H;
   const int sl = blockIdx.x % NSL, rh = blockIdx.x / NSL;
   const int r = rh / H, h = rh % H;
   // the thread's state column; its dS rows are MI ty + i (side by side), its dU rows
   // ty + 16 i
   const int col = SC * sl + tx;
+  const int jlo = p.cu_chunks[r], jhi = p.cu_chunks[r + 1];
+  // copies chunk jc's Khat and W tiles into buffer b (one commit group)
+  auto fetch = [&](int jc, int b) {
+    const size_t ch = (size_t)jc * H + h;
+    const float4 *gK = reinterpret_cast<const float4 *>(p.wKh + ch * C * D);
+    const float4 *gW = reinterpret_cast<const float4 *>(p.wW + ch * C * D);
+    float *dK = sm + L::oBuf + b * L::BUF, *dW = dK + C * D;
+    for (int e = tid; e < C * D / 4; e += ST_NTH) {
+      cp_async16(dK + 4 * e, gK + e);
+      cp_async16(dW + 4 * e, gW + e);
+    }
+    cp_async_commit();
+  };
+  // the thread's X, Y and Gam entries of chunk jc
+  float u[4], y[MI], gam[MI];
+  auto load_own = [&](int jc, float *u_, float *y_, float *gam_) {
+    const size_t ch = (size_t)jc * H + h;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) u_[i] = p.wX[ch * C * D + (size_t)(ty + 16 * i) * D + col];
+#pragma unroll
+    for (int i = 0; i < MI; ++i) y_[i] = p.wY[ch * D * D + (size_t)(MI * ty + i) * D + col];
+#pragma unroll
+    for (int q = 0; q < MI / 4; ++q) {
+      const float4 g4 = *reinterpret_cast<const float4 *>(p.wGam + ch * D + MI * ty + 4 * q);
+      gam_[4 * q] = g4.x, gam_[4 * q + 1] = g4.y, gam_[4 * q + 2] = g4.z, gam_[4 * q + 3] = g4.w;
+    }
+  };
+  if (jhi > jlo) {
+    fetch(jhi - 1, 0);
+    load_own(jhi - 1, u, y, gam);
+  }
   const float *dfin = p.d_final ? p.d_final + ((size_t)r * H + h) * D * D : nullptr;
   float ds[MI];
 #pragma unroll
@@ -698,26 +742,17 @@ __global__ void __launch_bounds__(NTH) bwd_state_kernel(const BwdParams p) {
   for (int q = 0; q < MI / 4; ++q)
     *reinterpret_cast<float4 *>(sdST + tx * LT + MI * ty + 4 * q) =
         make_float4(ds[4 * q], ds[4 * q + 1], ds[4 * q + 2], ds[4 * q + 3]);
-  for (int jc = p.cu_chunks[r + 1] - 1; jc >= p.cu_chunks[r]; --jc) {
+  for (int jc = jhi - 1, b = 0; jc >= jlo; --jc, b ^= 1) {
     const size_t ch = (size_t)jc * H + h;
-    const float4 *gK = reinterpret_cast<const float4 *>(p.wKh + ch * C * D);
-    const float4 *gW = reinterpret_cast<const float4 *>(p.wW + ch * C * D);
-    for (int e = tid; e < C * D / 4; e += NTH) {
-      cp_async16(sKh + 4 * e, gK + e);
-      cp_async16(sW + 4 * e, gW + e);
-    }
-    float u[4], y[MI], gam[MI];
-#pragma unroll
-    for (int i = 0; i < 4; ++i) u[i] = p.wX[ch * C * D + (size_t)(ty + 16 * i) * D + col];
-#pragma unroll
-    for (int i = 0; i < MI; ++i) {
-      y[i] = p.wY[ch * D * D + (size_t)(MI * ty + i) * D + col];
-      gam[i] = p.wGam[ch * D + MI * ty + i];
-    }
-    cp_async_wait_all();
-    __syncthreads();
+    const bool more = jc > jlo;
+    // the next chunk's tiles go to the other buffer, whose reads ended at the last
+    // barrier of the previous chunk
+    if (more) fetch(jc - 1, b ^ 1);
+    if (more) cp_async_wait<1>(); else cp_async_wait<0>();
+    __syncthreads();  // this chunk's tiles and the dS slice are complete
+    const float *sKh = sm + L::oBuf + b * L::BUF, *sW = sKh + C * D;
     // dU = X + Khat dSn   (overwrites X)
-#pragma unroll 4
+#pragma unroll 2
     for (int k = 0; k < D; k += 4) {
       const float4 d4 = *reinterpret_cast<const float4 *>(sdST + tx * LT + k);
 #pragma unroll
@@ -732,6 +767,9 @@ __global__ void __launch_bounds__(NTH) bwd_state_kernel(const BwdParams p) {
       p.wX[ch * C * D + (size_t)(ty + 16 * i) * D + col] = u[i];
     }
     __syncthreads();
+    // the next chunk's own entries, in flight while dS is formed
+    float nu[4], ny[MI], ngam[MI];
+    if (more) load_own(jc - 1, nu, ny, ngam);
     // dS = Diag(Gam) dSn + Y - W^T dU;  dSn overwrites Y for the gradient pass
     float acc[MI];
 #pragma unroll
@@ -753,16 +791,223 @@ __global__ void __launch_bounds__(NTH) bwd_state_kernel(const BwdParams p) {
       p.wY[ch * D * D + (size_t)(MI * ty + i) * D + col] = ds[i];
       ds[i] = fmaf(gam[i], ds[i], y[i] - acc[i]);
     }
-    __syncthreads();  // every read of sdST, sKh and sW of this chunk is done
+    __syncthreads();  // every read of sdST, sdU and this chunk's buffer is done
 #pragma unroll
     for (int q = 0; q < MI / 4; ++q)
       *reinterpret_cast<float4 *>(sdST + tx * LT + MI * ty + 4 * q) =
           make_float4(ds[4 * q], ds[4 * q + 1], ds[4 * q + 2], ds[4 * q + 3]);
+    if (more) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i) u[i] = nu[i];
+#pragma unroll
+      for (int i = 0; i < MI; ++i) y[i] = ny[i], gam[i] = ngam[i];
+    }
   }
   if (p.d_initial) {
     float *dst = p.d_initial + ((size_t)r * H + h) * D * D;
 #pragma unroll
     for (int i = 0; i < MI; ++i) dst[(size_t)(MI * ty + i) * D + col] = ds[i];
+  }
+}
+
+// ---------------------------------------------------------------------------
+// bwd_state_tc (bf16 inputs, d = 128): the serial pass on the tensor cores.  One CTA
+// per (request, head) holds dS^T in TMEM (lane = value column j, columns = key rows
+// i) and takes the chunks last first:
+//   dU^T = X^T + dSn^T Khat^T                 A = dSn^T (TMEM), B = Khat (rows = tokens)
+//   dS^T = dSn^T Diag(Gam) + Y^T - dU^T W     A = dU^T (TMEM), B = W^T (rows = keys)
+// The CUDA cores add X^T to the first product and write dU out, then write dSn out
+// and form dSn^T Diag(Gam) + Y^T in place as the second product's accumulator.  Khat
+// arrives tf32-rounded from the prep pass and is copied with cp.async two chunks
+// ahead; W is transposed and rounded through registers one chunk ahead.  Products
+// accumulate in fp32; their tf32 operands are the state (as TMEM holds it), dU
+// (rounded to nearest), Khat and W.
+// ---------------------------------------------------------------------------
+constexpr int STC_NTH = 512;
+
+struct StateTcLayout {
+  static constexpr int D = 128;
+  static constexpr int KB = C * D * 4;  // one Khat operand: 64 rows x 128 tf32 (32 KiB)
+  static constexpr int WB = D * C * 4;  // one W^T operand: 128 rows x 64 tf32 (32 KiB)
+  static constexpr int oK = 0, oW = 2 * KB, oGam = oW + 2 * WB;  // byte offsets
+  static constexpr int oBar = oGam + 2 * D * 4;  // three mbarriers, then the TMEM address
+  static constexpr size_t bytes = oBar + 32 + 1024;
+};
+
+__global__ void __launch_bounds__(STC_NTH, 1) bwd_state_tc_kernel(const BwdParams p) {
+  using L = StateTcLayout;
+  constexpr int D = L::D;
+  constexpr uint32_t TS = 0, TU = 128;  // TMEM columns: dS^T, then dU^T
+  extern __shared__ float4 smem_f4[];
+  unsigned char *sb = align1024_shared(smem_f4);
+  float *sGam = reinterpret_cast<float *>(sb + L::oGam);         // [2][128]
+  uint64_t *bar = reinterpret_cast<uint64_t *>(sb + L::oBar);    // first, second, drain
+  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sb + L::oBar + 24);
+  const int tid = threadIdx.x, w = tid >> 5, ln = tid & 31;
+  // warp w reaches TMEM lanes 32 (w % 4) .. + 31 (value columns j) and takes part w / 4
+  // of the columns: tokens 16 part .. + 15 of dU^T, keys 32 part .. + 31 of dS^T
+  const int qd = w & 3, part = w >> 2, j = 32 * qd + ln;
+  const uint32_t lane = (uint32_t)(32 * qd) << 16;
+  const int H = p.H, r = blockIdx.x / H, h = blockIdx.x % H;
+  const int jlo = p.cu_chunks[r], jhi = p.cu_chunks[r + 1];
+  if (w == 0) {
+    tmem_alloc(s_tmem, 256);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    mbar_init(bar + 1, 1);
+    mbar_init(bar + 2, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  // Khat of chunk jc into operand buffer b (rows = tokens, K = keys); one commit group
+  auto fetch_k = [&](int jc, int b) {
+    const float4 *g = reinterpret_cast<const float4 *>(p.wKh + ((size_t)jc * H + h) * C * D);
+    unsigned char *dst = sb + L::oK + b * L::KB;
+#pragma unroll
+    for (int q = 0; q < C * D / 4 / STC_NTH; ++q) {
+      const int e = tid + q * STC_NTH, t = e >> 5, k = (e & 31) * 4;
+      cp_async16(dst + sw128_chunk(C, t, k), g + e);
+    }
+    cp_async_commit();
+  };
+  // W of chunk jc, transposed (rows = keys, K = tokens): element e of the thread's four
+  // takes key e % 128 and tokens 4 (e / 128) .. + 3 (a warp reads 128 bytes per token)
+  float wv[4][4];
+  auto load_w = [&](int jc) {
+    const float *g = p.wW + ((size_t)jc * H + h) * C * D;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int e = tid + q * STC_NTH, i = e & (D - 1), t0 = (e >> 7) * 4;
+#pragma unroll
+      for (int u = 0; u < 4; ++u) wv[q][u] = g[(size_t)(t0 + u) * D + i];
+    }
+  };
+  auto store_w = [&](int b) {
+    unsigned char *dst = sb + L::oW + b * L::WB;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      const int e = tid + q * STC_NTH, i = e & (D - 1), t0 = (e >> 7) * 4;
+      *reinterpret_cast<float4 *>(dst + sw128_chunk(D, i, t0)) =
+          make_float4(tf32_round(wv[q][0]), tf32_round(wv[q][1]), tf32_round(wv[q][2]),
+                      tf32_round(wv[q][3]));
+    }
+  };
+  auto load_gam = [&](int jc, int b) {
+    if (tid < D / 4)
+      reinterpret_cast<float4 *>(sGam + b * D)[tid] =
+          reinterpret_cast<const float4 *>(p.wGam + ((size_t)jc * H + h) * D)[tid];
+  };
+
+  const float *dfin = p.d_final ? p.d_final + ((size_t)r * H + h) * D * D : nullptr;
+  float sv[32];
+#pragma unroll
+  for (int c = 0; c < 32; ++c) sv[c] = dfin ? dfin[(size_t)(32 * part + c) * D + j] : 0.f;
+  if (jhi > jlo) {
+    fetch_k(jhi - 1, 0);
+    if (jhi - 1 > jlo) fetch_k(jhi - 2, 1);
+    load_w(jhi - 1);
+    load_gam(jhi - 1, 0);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tm = *s_tmem;
+  tmem_st32(tm + lane + TS + 32 * part, sv);  // dS^T of the last chunk's end
+  if (jhi > jlo) store_w(0);
+  if (jhi - 1 > jlo) cp_async_wait<1>(); else cp_async_wait<0>();
+  tmem_wait_st();
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+
+  bool ok = true;
+  uint32_t ph1 = 0, ph2 = 0;
+  const uint32_t id64 = idesc_tf32(C), id128n = idesc_tf32(D, true);
+  for (int jc = jhi - 1, b = 0; jc >= jlo; --jc, b ^= 1) {
+    const size_t ch = (size_t)jc * H + h;
+    if (tid == 0 && ok) {
+      const uint32_t kb = smem_u32(sb + L::oK + b * L::KB);
+#pragma unroll
+      for (int s = 0; s < D / 8; ++s)
+        mma_tf32_ts(tm + TU, tm + TS + 8 * s, sw128_desc(kb, C, s), id64, s > 0);
+      mma_commit(bar);
+    }
+    // this chunk's X and Y entries, in flight under the first product
+    float x[16], y[32];
+#pragma unroll
+    for (int tt = 0; tt < 16; ++tt) x[tt] = p.wX[ch * C * D + (size_t)(16 * part + tt) * D + j];
+#pragma unroll
+    for (int c = 0; c < 32; ++c) y[c] = p.wY[ch * D * D + (size_t)(32 * part + c) * D + j];
+    ok = ok && mbar_wait(bar, ph1);
+    ph1 ^= 1;
+    tc_fence_after();
+    // the first product is done with buffer b and with dSn^T
+    if (jc - 2 >= jlo) fetch_k(jc - 2, b);
+    if (jc - 1 >= jlo) {
+      load_w(jc - 1);
+      load_gam(jc - 1, b ^ 1);
+    }
+    if (ok) {
+      float u[16];
+      tmem_ld16(tm + lane + TU + 16 * part, u);
+      tmem_wait_ld();
+#pragma unroll
+      for (int tt = 0; tt < 16; ++tt) {
+        u[tt] += x[tt];
+        p.wX[ch * C * D + (size_t)(16 * part + tt) * D + j] = u[tt];  // dU over X
+        u[tt] = tf32_round(u[tt]);
+      }
+      tmem_st16(tm + lane + TU + 16 * part, u);
+      tmem_ld32(tm + lane + TS + 32 * part, sv);
+      tmem_wait_ld();
+      const float *gam = sGam + b * D + 32 * part;
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        p.wY[ch * D * D + (size_t)(32 * part + c) * D + j] = sv[c];  // dSn over Y
+        sv[c] = fmaf(gam[c], sv[c], y[c]);
+      }
+      tmem_st32(tm + lane + TS + 32 * part, sv);
+    }
+    if (jc - 1 >= jlo) store_w(b ^ 1);
+    tmem_wait_st();
+    if (jc - 2 >= jlo) cp_async_wait<1>(); else cp_async_wait<0>();  // Khat of jc - 1
+    fence_async_smem();
+    tc_fence_before();
+    ok = __syncthreads_and(ok);
+    tc_fence_after();
+    if (!ok) break;
+    if (tid == 0) {
+      const uint32_t wb = smem_u32(sb + L::oW + b * L::WB);
+#pragma unroll
+      for (int s = 0; s < C / 8; ++s)
+        mma_tf32_ts(tm + TS, tm + TU + 8 * s, sw128_desc(wb, D, s), id128n, true);
+      mma_commit(bar + 1);
+    }
+    ok = mbar_wait(bar + 1, ph2);
+    ph2 ^= 1;
+    tc_fence_after();
+  }
+  cp_async_wait<0>();
+  if (!__syncthreads_and(ok)) {
+    if (tid == 0) {
+      set_status(p.status, STATUS_TIMEOUT);
+      mma_commit(bar + 2);  // covers every product issued
+      mbar_wait(bar + 2, 0, 100000000ull);
+    }
+  } else if (p.d_initial) {
+    tmem_ld32(tm + lane + TS + 32 * part, sv);
+    tmem_wait_ld();
+    float *dst = p.d_initial + ((size_t)r * H + h) * D * D;
+#pragma unroll
+    for (int c = 0; c < 32; ++c) dst[(size_t)(32 * part + c) * D + j] = sv[c];
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (w == 0) {
+    tc_fence_after();
+    tmem_dealloc(tm, 256);
   }
 }
 
@@ -1338,9 +1583,14 @@ cudaError_t launch_bwd_d(const BwdParams &p, cudaStream_t stream) {
     bwd_prep_kernel<D, TIn><<<chunk_grid, NTH, PrepLayout<D>::bytes, stream>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
-  if ((e = set_smem(bwd_state_kernel<D>, StateLayout<D>::bytes)) != cudaSuccess) return e;
-  bwd_state_kernel<D>
-      <<<(unsigned)(p.n_req * p.H * (D / SC)), NTH, StateLayout<D>::bytes, stream>>>(p);
+  if constexpr (kPrepTensorCores<D, TIn>) {
+    if ((e = set_smem(bwd_state_tc_kernel, StateTcLayout::bytes)) != cudaSuccess) return e;
+    bwd_state_tc_kernel<<<(unsigned)(p.n_req * p.H), STC_NTH, StateTcLayout::bytes, stream>>>(p);
+  } else {
+    if ((e = set_smem(bwd_state_kernel<D>, StateLayout<D>::bytes)) != cudaSuccess) return e;
+    bwd_state_kernel<D>
+        <<<(unsigned)(p.n_req * p.H * (D / SC)), ST_NTH, StateLayout<D>::bytes, stream>>>(p);
+  }
   if ((e = cudaGetLastError()) != cudaSuccess) return e;
   if constexpr (kPrepTensorCores<D, TIn>) {
     if (chunk_grid > 0) {
