@@ -1209,6 +1209,174 @@ __global__ void __launch_bounds__(SP_NTH, 1) bwd_sprod_kernel(const BwdParams p)
 }
 
 // ---------------------------------------------------------------------------
+// bwd_tprod (bf16 inputs, d = 128): the gradient pass's products of chunk-sized tiles
+// on the tensor cores, with M = 128 TMEM lanes of which the chunk's 64 tokens t use
+// the first 64:
+//   dP   = dO U^T                                 A = dO (lanes t), B = U (rows s)
+//   [T^T dU | T^T dW] = T^T [dU | dW]             A = T^T (lanes t), B = [dU^T ; dW^T]
+//                                                   (rows = 256 value columns, K = s)
+//   dZ   = -[(T^T dU) U~^T + (T^T dW) W^T]        A = the product above (K = 256),
+//                                                   B = [U~ | W] (rows s, K = 256)
+// tf32 operands rounded to nearest (the middle product is read from TMEM as it
+// stands), fp32 accumulation.  The results replace tiles the gradient pass no
+// longer reads: dP over T, T^T dU over dU, T^T dW over dW, dZ over U.
+// ---------------------------------------------------------------------------
+constexpr int TP_NTH = 512;
+
+struct TprodLayout {
+  static constexpr int D = 128;
+  // B operands (byte offsets, 1024-byte aligned): U (64 rows x 128), [dU^T ; dW^T]
+  // (256 rows x 64), [U~ | W] (64 rows x 256); then two mbarriers and the TMEM address
+  static constexpr int oU = 0, oDUW = oU + C * D * 4, oUtW = oDUW + 2 * D * C * 4;
+  static constexpr int oBar = oUtW + C * 2 * D * 4;
+  static constexpr size_t bytes = oBar + 32 + 1024;
+};
+
+__global__ void __launch_bounds__(TP_NTH, 1) bwd_tprod_kernel(const BwdParams p) {
+  using L = TprodLayout;
+  constexpr int D = L::D;
+  // TMEM columns: dO (A of the first product), later dZ; dP; T^T; [T^T dU | T^T dW]
+  constexpr uint32_t TDO = 0, TZ = 0, TP = 128, TT = 192, TB = 256;
+  extern __shared__ float4 smem_f4[];
+  unsigned char *sb = align1024_shared(smem_f4);
+  uint64_t *bar = reinterpret_cast<uint64_t *>(sb + L::oBar);
+  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sb + L::oBar + 16);
+  const int tid = threadIdx.x, w = tid >> 5, ln = tid & 31;
+  const int H = p.H;
+  const int jc = blockIdx.x / H, h = blockIdx.x % H;
+  const int4 cd = p.chunks[jc];
+  const int tok0 = cd.z, n = cd.w;
+  const size_t ch = (size_t)jc * H + h;
+  const float *U = p.wU2 + ch * C * D, *dU = p.wX + ch * C * D, *dW = p.wKh + ch * C * D;
+  const float *Ut = p.wU + ch * C * D, *W = p.wW + ch * C * D, *T = p.wT + ch * C * C;
+  if (w == 0) {
+    tmem_alloc(s_tmem, 512);
+    tmem_relinquish();
+  }
+  if (tid == 0) {
+    mbar_init(bar, 1);
+    mbar_init(bar + 1, 1);
+    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+  }
+  // B operands, rounded to tf32
+  unsigned char *bU = sb + L::oU, *bDUW = sb + L::oDUW, *bUtW = sb + L::oUtW;
+#pragma unroll
+  for (int q = 0; q < C * D / 4 / TP_NTH; ++q) {  // U: rows s, K = value columns
+    const int e = tid + q * TP_NTH, t = e >> 5, k = (e & 31) * 4;
+    const float4 u = *reinterpret_cast<const float4 *>(U + t * D + k);
+    *reinterpret_cast<float4 *>(bU + sw128_chunk(C, t, k)) = tf32_round4(u);
+  }
+#pragma unroll 2
+  for (int q = 0; q < 2 * D * C / 4 / TP_NTH; ++q) {  // [dU^T ; dW^T]: rows c', K = s
+    const int e = tid + q * TP_NTH, c2 = e & (2 * D - 1), s0 = (e >> 8) * 4;
+    const float *src = c2 < D ? dU + c2 : dW + (c2 - D);
+    float4 v;
+    v.x = src[(size_t)s0 * D];
+    v.y = src[(size_t)(s0 + 1) * D];
+    v.z = src[(size_t)(s0 + 2) * D];
+    v.w = src[(size_t)(s0 + 3) * D];
+    *reinterpret_cast<float4 *>(bDUW + sw128_chunk(2 * D, c2, s0)) = tf32_round4(v);
+  }
+#pragma unroll 2
+  for (int q = 0; q < C * 2 * D / 4 / TP_NTH; ++q) {  // [U~ | W]: rows s, K = c'
+    const int e = tid + q * TP_NTH, t = e >> 6, k = (e & 63) * 4;
+    const float4 v = k < D ? *reinterpret_cast<const float4 *>(Ut + t * D + k)
+                           : *reinterpret_cast<const float4 *>(W + t * D + (k - D));
+    *reinterpret_cast<float4 *>(bUtW + sw128_chunk(C, t, k)) = tf32_round4(v);
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tm = *s_tmem;
+  // A operands: warps of lane quarters 0 and 1 hold tokens t = 32 (w % 4) + lane; part
+  // w / 4 takes a quarter of the columns.  Lanes 64..127 are left as they are: they
+  // only reach accumulator lanes that nothing reads.
+  const int qd = w & 3, part = w >> 2;
+  const uint32_t lane = (uint32_t)(32 * qd) << 16;
+  const int t = 32 * qd + ln;
+  if (qd < 2) {
+    float v[32];  // dO row t, value columns 32 part .. + 31 (rows past the chunk: zero)
+    const bool live = p.d_o && t < n;
+    const float4 *src =
+        reinterpret_cast<const float4 *>(p.d_o + ((size_t)(tok0 + (live ? t : 0)) * H + h) * D);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) {
+      const float4 x = live ? src[8 * part + q] : make_float4(0.f, 0.f, 0.f, 0.f);
+      v[4 * q] = tf32_round(x.x), v[4 * q + 1] = tf32_round(x.y);
+      v[4 * q + 2] = tf32_round(x.z), v[4 * q + 3] = tf32_round(x.w);
+    }
+    tmem_st32(tm + lane + TDO + 32 * part, v);
+    float tv[16];  // T^T row t: T[s][t] for s = 16 part .. + 15
+#pragma unroll
+    for (int ss = 0; ss < 16; ++ss) tv[ss] = tf32_round(T[(16 * part + ss) * C + t]);
+    tmem_st16(tm + lane + TT + 16 * part, tv);
+  }
+  tmem_wait_st();
+  fence_async_smem();
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  bool ok = true;
+  if (tid == 0) {
+    const uint32_t ub = smem_u32(bU), dwb = smem_u32(bDUW), uwb = smem_u32(bUtW);
+#pragma unroll
+    for (int s = 0; s < D / 8; ++s)
+      mma_tf32_ts(tm + TP, tm + TDO + 8 * s, sw128_desc(ub, C, s), idesc_tf32(C), s > 0);
+#pragma unroll
+    for (int s = 0; s < C / 8; ++s)
+      mma_tf32_ts(tm + TB, tm + TT + 8 * s, sw128_desc(dwb, 2 * D, s), idesc_tf32(2 * D),
+                  s > 0);
+    mma_commit(bar);
+    ok = mbar_wait(bar, 0);  // the middle product is the next one's A; dO's columns free
+    tc_fence_after();
+    if (ok) {
+#pragma unroll
+      for (int s = 0; s < 2 * D / 8; ++s)
+        mma_tf32_ts(tm + TZ, tm + TB + 8 * s, sw128_desc(uwb, C, s), idesc_tf32(C, true),
+                    s > 0);
+    }
+    mma_commit(bar + 1);  // covers every product issued
+  }
+  const bool done = __syncthreads_and(ok) && mbar_wait(bar + 1, 0);
+  if (!done && tid == 0) set_status(p.status, STATUS_TIMEOUT);
+  tc_fence_after();
+  if (done && qd < 2) {
+    float v[32];
+    // dP row t over T, columns 16 part .. + 15
+    tmem_ld16(tm + lane + TP + 16 * part, v);
+    tmem_wait_ld();
+    float4 *dst = reinterpret_cast<float4 *>(p.wT + ch * C * C + (size_t)t * C + 16 * part);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+    // dZ row t over U, columns 16 part .. + 15
+    tmem_ld16(tm + lane + TZ + 16 * part, v);
+    tmem_wait_ld();
+    dst = reinterpret_cast<float4 *>(p.wU2 + ch * C * D + (size_t)t * C + 16 * part);
+#pragma unroll
+    for (int q = 0; q < 4; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+    // [T^T dU | T^T dW] row t: part p takes columns 64 p .. + 63 (parts 0, 1: T^T dU over
+    // dU; parts 2, 3: T^T dW over dW)
+    float *row = (part < 2 ? p.wX : p.wKh) + ch * C * D + (size_t)t * D + 64 * (part & 1);
+#pragma unroll
+    for (int hh = 0; hh < 2; ++hh) {
+      tmem_ld32(tm + lane + TB + 64 * part + 32 * hh, v);
+      tmem_wait_ld();
+      float4 *d4 = reinterpret_cast<float4 *>(row + 32 * hh);
+#pragma unroll
+      for (int q = 0; q < 8; ++q) d4[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+    }
+  }
+  tc_fence_before();
+  __syncthreads();
+  if (!done && tid == 0) mbar_wait(bar + 1, 0, 100000000ull);  // let issued products finish
+  __syncthreads();
+  if (w == 0) {
+    tc_fence_after();
+    tmem_dealloc(tm, 512);
+  }
+}
+
+// ---------------------------------------------------------------------------
 // bwd_grad: every token gradient of one chunk
 // ---------------------------------------------------------------------------
 template <int D>
@@ -1253,7 +1421,7 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
   stage_rows<D, TIn>(sK, D, static_cast<const TIn *>(p.k), tok0, n, H, h);
   stage_rows<D, TIn>(sQ, D, static_cast<const TIn *>(p.q), tok0, n, H, h);
   stage_rows<D, TIn>(sV, D, static_cast<const TIn *>(p.v), tok0, n, H, h);
-  stage_rows<D, float>(sO, D, p.d_o, tok0, n, H, h);
+  if constexpr (!PRE) stage_rows<D, float>(sO, D, p.d_o, tok0, n, H, h);  // PRE: not read
   if (tid < C) sDb[tid] = 0.f;
   stage_gate<D>(sG, sB, p, tok0, n, h);
 
@@ -1302,11 +1470,18 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
       accG[i][j] = gq * sQ[e];
       accK[i][j] = 0.f;
     }
-  // dP = tril(dO U^T)
+  // dP = tril(dO U^T)  (from bwd_tprod, over T, when it ran)
   {
     float pp[4][4];
-    zero(pp);
-    mm_acc<4, 4>(pp, sO, D, 1, U, 1, D, D, sStage);
+    if constexpr (PRE) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j) pp[i][j] = p.wT[ch * C * C + (ty + 16 * i) * C + tx + 16 * j];
+    } else {
+      zero(pp);
+      mm_acc<4, 4>(pp, sO, D, 1, U, 1, D, D, sStage);
+    }
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
@@ -1365,14 +1540,9 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
     sExtra[tid] = e;
   }
 
-  // dW = -dU S^T (into the dO tile; the sync above ends every read of that tile)
-  if constexpr (PRE) {
-    load_own(p.wKh + ch * C * D);  // from bwd_sprod, over Khat
-#pragma unroll
-    for (int i = 0; i < 4; ++i)
-#pragma unroll
-      for (int j = 0; j < NJ; ++j) sO[(ty + 16 * i) * D + tx + 16 * j] = acc[i][j];
-  } else {
+  // dW = -dU S^T (into the dO tile; the sync above ends every read of that tile);
+  // with the tensor cores, bwd_tprod has already taken every product with dW
+  if constexpr (!PRE) {
     zero(acc);
     mm_acc<4, NJ>(acc, dU, D, 1, S, 1, D, D, sStage);
 #pragma unroll
@@ -1380,7 +1550,7 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
 #pragma unroll
       for (int j = 0; j < NJ; ++j) sO[(ty + 16 * i) * D + tx + 16 * j] = -acc[i][j];
   }
-  {
+  if constexpr (!PRE) {
     float4 tv[C * C / 4 / NTH];
 #pragma unroll
     for (int q = 0; q < C * C / 4 / NTH; ++q)
@@ -1389,9 +1559,14 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
     for (int q = 0; q < C * C / 4 / NTH; ++q)
       reinterpret_cast<float4 *>(sT)[tid + q * NTH] = tv[q];
   }
-  // T^T dU -> dV = Diag(beta) T^T dU, dbeta += (T^T dU) . v
-  zero(acc);
-  mm_acc<4, NJ>(acc, sT, 1, C, dU, D, 1, C, sStage);
+  // T^T dU -> dV = Diag(beta) T^T dU, dbeta += (T^T dU) . v  (T^T dU from bwd_tprod, over
+  // dU, when it ran)
+  if constexpr (PRE) {
+    load_own(dU);
+  } else {
+    zero(acc);
+    mm_acc<4, NJ>(acc, sT, 1, C, dU, D, 1, C, sStage);
+  }
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int t = ty + 16 * i;
@@ -1406,9 +1581,14 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
     rs = row_sum16(rs);
     if (tx == 0) sDb[t] += rs;
   }
-  // T^T dW -> d(gamma K) = Diag(beta) T^T dW;  dbeta += (T^T dW) . (gamma k)
-  zero(acc);
-  mm_acc<4, NJ>(acc, sT, 1, C, sO, D, 1, C, sStage);
+  // T^T dW -> d(gamma K) = Diag(beta) T^T dW;  dbeta += (T^T dW) . (gamma k)  (from
+  // bwd_tprod, over dW, when it ran)
+  if constexpr (PRE) {
+    load_own(p.wKh + ch * C * D);
+  } else {
+    zero(acc);
+    mm_acc<4, NJ>(acc, sT, 1, C, sO, D, 1, C, sStage);
+  }
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int t = ty + 16 * i;
@@ -1434,10 +1614,18 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
     for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j) av[i][j] = p.wA[ch * C * C + (ty + 16 * i) * C + tx + 16 * j];
-    float tt[4][4];
-    zero(tt);
-    mm_acc<4, 4>(tt, sV, D, 1, Ut, 1, D, D, sStage);
-    mm_acc<4, 4>(tt, sO, D, 1, W, 1, D, D, sStage);
+    float tt[4][4];  // -dZ  (dZ from bwd_tprod, over U, when it ran)
+    if constexpr (PRE) {
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+#pragma unroll
+        for (int j = 0; j < 4; ++j)
+          tt[i][j] = -p.wU2[ch * C * D + (ty + 16 * i) * C + tx + 16 * j];
+    } else {
+      zero(tt);
+      mm_acc<4, 4>(tt, sV, D, 1, Ut, 1, D, D, sStage);
+      mm_acc<4, 4>(tt, sO, D, 1, W, 1, D, D, sStage);
+    }
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int t = ty + 16 * i;
@@ -1596,6 +1784,13 @@ cudaError_t launch_bwd_d(const BwdParams &p, cudaStream_t stream) {
     if (chunk_grid > 0) {
       if ((e = set_smem(bwd_sprod_kernel, SprodLayout::bytes)) != cudaSuccess) return e;
       bwd_sprod_kernel<<<chunk_grid, SP_NTH, SprodLayout::bytes, stream>>>(p);
+      if ((e = cudaGetLastError()) != cudaSuccess) return e;
+    }
+  }
+  if constexpr (kPrepTensorCores<D, TIn>) {
+    if (chunk_grid > 0) {
+      if ((e = set_smem(bwd_tprod_kernel, TprodLayout::bytes)) != cudaSuccess) return e;
+      bwd_tprod_kernel<<<chunk_grid, TP_NTH, TprodLayout::bytes, stream>>>(p);
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
   }
