@@ -1012,29 +1012,39 @@ __global__ void __launch_bounds__(STC_NTH, 1) bwd_state_tc_kernel(const BwdParam
 }
 
 // ---------------------------------------------------------------------------
-// bwd_sprod (bf16 inputs, d = 128): the four state products of the gradient pass
-// on the tensor cores.  Transposed, as in the forward, so each has M = 128 TMEM
-// lanes; A operands in TMEM, B operands K-major with the 128-byte swizzle in
-// shared memory, tf32 operands rounded to nearest, fp32 accumulation:
+// bwd_sprod (bf16 inputs, d = 128): the gradient pass's tile products on the tensor
+// cores, in two stages per (chunk, head).  Each product has M = 128 TMEM lanes, its A
+// operand in TMEM and its B operand K-major with the 128-byte swizzle in shared
+// memory; tf32 operands rounded to nearest, fp32 accumulation.
+// Stage 1, the products with the state (transposed, as in the forward):
 //   U^T          = U~^T - S^T W^T    A = S^T (lane = value column), D starts as U~^T
 //   d(gamma Q)^T = S dO^T            A = S (lane = key row)
 //   dW^T         = -S dU^T           A = S
 //   dKhat^T      = dSn U^T           A = dSn (lane = key row), B = U from the first product
 // and dGam_i = sum_j dSn_ij S_ij (fp32 on the CUDA cores, from the unrounded values).
-// The results go to workspace tiles the gradient pass no longer needs: U to its own
-// tile, d(gamma Q) and dKhat over dSn, dW over Khat (both read only by the state
-// pass), dGam over Gam.
+// Stage 2, the products of chunk-sized tiles, on lanes t = the chunk's 64 tokens (the
+// other 64 lanes compute nothing anyone reads):
+//   dP   = dO U^T                                 A = dO, B = U (rows s)
+//   [T^T dU | T^T dW] = T^T [dU | dW]             A = T^T, B = [dU^T ; dW^T]
+//                                                   (rows = 256 value columns, K = s)
+//   dZ   = -[(T^T dU) U~^T + (T^T dW) W^T]        A = the product above (K = 256, read
+//                                                   from TMEM as it stands), B = [U~ | W]
+// U and dW stay on chip between the stages.  The results replace workspace tiles the
+// gradient pass no longer reads: d(gamma Q) and dKhat over dSn, dGam over Gam, dP over
+// T, dZ over U, T^T dU over dU, T^T dW over Khat.
 // ---------------------------------------------------------------------------
 constexpr int SP_NTH = 512;
 
 struct SprodLayout {
   static constexpr int D = 128;
-  // B operand tiles (64 rows x 128 tf32 each, 1024-byte aligned), then the dGam partials
-  static constexpr int oW = 0, oO = oW + C * D, oDU = oO + C * D, oU = oDU + C * D;
-  static constexpr int oPart = oU + C * D;     // [4][128]
-  static constexpr int oMisc = oPart + 4 * D;  // two mbarriers and the TMEM base address
-  static constexpr int total = oMisc + 8;
-  static constexpr size_t bytes = sizeof(float) * total + 1024;
+  // B operand tiles (byte offsets, 1024-byte aligned): U~ and W back to back (together
+  // the K = 256 operand [U~ | W] of dZ), dO, dU and U (64 rows x 128 tf32 each), then
+  // [dU^T ; dW^T] (256 rows x 64 tf32), whose space first holds the dGam partials
+  static constexpr int TILE = C * D * 4;
+  static constexpr int oUt = 0, oW = TILE, oO = 2 * TILE, oDU = 3 * TILE, oU = 4 * TILE;
+  static constexpr int oDUW = 5 * TILE, oPart = oDUW;
+  static constexpr int oMisc = oDUW + 2 * TILE;  // four mbarriers, then the TMEM address
+  static constexpr size_t bytes = oMisc + 48 + 1024;
 };
 
 __device__ __forceinline__ float4 tf32_round4(float4 x) {
@@ -1044,18 +1054,17 @@ __device__ __forceinline__ float4 tf32_round4(float4 x) {
 __global__ void __launch_bounds__(SP_NTH, 1) bwd_sprod_kernel(const BwdParams p) {
   using L = SprodLayout;
   constexpr int D = L::D;
-  // TMEM columns: S^T, then dW^T | dKhat^T once the first product is done; U~^T -> U^T;
-  // S; dSn; d(gamma Q)^T
+  // TMEM columns, stage 1: S^T, then dW^T | dKhat^T once the first product is done;
+  // U~^T -> U^T; S; dSn; d(gamma Q)^T.  Stage 2: dO, then dZ; dP; T^T; [T^T dU | T^T dW].
   constexpr uint32_t TST = 0, TDW = 0, TDK = 64, TU = 128, TS = 192, TDS = 320, TGQ = 448;
+  constexpr uint32_t TDO = 0, TZ = 0, TP = 128, TT = 192, TB = 256;
   extern __shared__ float4 smem_f4[];
-  float *sm = reinterpret_cast<float *>(align1024_shared(smem_f4));
-  unsigned char *bW = reinterpret_cast<unsigned char *>(sm + L::oW);
-  unsigned char *bO = reinterpret_cast<unsigned char *>(sm + L::oO);
-  unsigned char *bDU = reinterpret_cast<unsigned char *>(sm + L::oDU);
-  unsigned char *bU = reinterpret_cast<unsigned char *>(sm + L::oU);
-  float *sPart = sm + L::oPart;
-  uint64_t *bar = reinterpret_cast<uint64_t *>(sm + L::oMisc);  // [0]: U^T, [1]: the rest
-  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sm + L::oMisc + 4);
+  unsigned char *sb = align1024_shared(smem_f4);
+  unsigned char *bUt = sb + L::oUt, *bW = sb + L::oW, *bO = sb + L::oO, *bDU = sb + L::oDU;
+  unsigned char *bU = sb + L::oU, *bDUW = sb + L::oDUW;
+  float *sPart = reinterpret_cast<float *>(sb + L::oPart);
+  uint64_t *bar = reinterpret_cast<uint64_t *>(sb + L::oMisc);  // U^T, stage 1, 2a, 2b
+  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sb + L::oMisc + 32);
   const int tid = threadIdx.x, w = tid >> 5, ln = tid & 31;
   const int H = p.H;
   const int jc = blockIdx.x / H, h = blockIdx.x % H;
@@ -1068,24 +1077,27 @@ __global__ void __launch_bounds__(SP_NTH, 1) bwd_sprod_kernel(const BwdParams p)
   else
     S = p.snaps + ((size_t)(p.cu_snap[r] + cidx - 1) * H + h) * D * D;
   const float *dSn = p.wY + ch * D * D;
+  const float *Ut = p.wU + ch * C * D, *T = p.wT + ch * C * C;
   if (w == 0) {
     tmem_alloc(s_tmem, 512);
     tmem_relinquish();
   }
   if (tid == 0) {
-    mbar_init(bar, 1);
-    mbar_init(bar + 1, 1);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) mbar_init(bar + i, 1);
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
 
-  // B operands: W, dO (rows past the chunk's end are zero) and dU, rows = tokens
+  // B operands: U~, W, dO (rows past the chunk's end are zero) and dU, rows = tokens
   for (int e = tid; e < C * D / 4; e += SP_NTH) {
     const int t = e >> 5, k = (e & 31) * 4;
+    const float4 utv = *reinterpret_cast<const float4 *>(Ut + t * D + k);
     const float4 wv = *reinterpret_cast<const float4 *>(p.wW + ch * C * D + t * D + k);
     const float4 uv = *reinterpret_cast<const float4 *>(p.wX + ch * C * D + t * D + k);
     const float4 ov = (p.d_o && t < n) ? *reinterpret_cast<const float4 *>(
                                              p.d_o + ((size_t)(tok0 + t) * H + h) * D + k)
                                        : make_float4(0.f, 0.f, 0.f, 0.f);
+    *reinterpret_cast<float4 *>(bUt + sw128_chunk(C, t, k)) = tf32_round4(utv);
     *reinterpret_cast<float4 *>(bW + sw128_chunk(C, t, k)) = tf32_round4(wv);
     *reinterpret_cast<float4 *>(bDU + sw128_chunk(C, t, k)) = tf32_round4(uv);
     *reinterpret_cast<float4 *>(bO + sw128_chunk(C, t, k)) = tf32_round4(ov);
@@ -1126,7 +1138,7 @@ __global__ void __launch_bounds__(SP_NTH, 1) bwd_sprod_kernel(const BwdParams p)
   {  // U~^T (the first product's accumulator, fp32): lane = value column, columns = tokens
     float v[16];
 #pragma unroll
-    for (int tt = 0; tt < 16; ++tt) v[tt] = p.wU[ch * C * D + (size_t)(16 * part + tt) * D + lrow];
+    for (int tt = 0; tt < 16; ++tt) v[tt] = Ut[(size_t)(16 * part + tt) * D + lrow];
     tmem_st16(tm + lane + TU + 16 * part, v);
   }
   tmem_wait_st();
@@ -1147,7 +1159,7 @@ __global__ void __launch_bounds__(SP_NTH, 1) bwd_sprod_kernel(const BwdParams p)
   }
   if (tid < D)  // dGam in a fixed order
     p.wGam[ch * D + tid] = (sPart[tid] + sPart[D + tid]) + (sPart[2 * D + tid] + sPart[3 * D + tid]);
-  const bool ok = mbar_wait(bar, 0);
+  bool ok = mbar_wait(bar, 0);
   tc_fence_after();
   if (tid == 0 && ok) {  // S^T is consumed: dW^T = -S dU^T goes over its first half
     const uint32_t db = smem_u32(bDU);
@@ -1155,20 +1167,17 @@ __global__ void __launch_bounds__(SP_NTH, 1) bwd_sprod_kernel(const BwdParams p)
     for (int s = 0; s < D / 8; ++s)
       mma_tf32_ts(tm + TDW, tm + TS + 8 * s, sw128_desc(db, C, s), id64n, s > 0);
   }
-  if (ok) {  // U: to its workspace tile (fp32) and, rounded, to the B tile of dKhat^T
+  if (ok) {  // U, rounded, to the B tile of dKhat^T and of dP
     float v[16];
     tmem_ld16(tm + lane + TU + 16 * part, v);
     tmem_wait_ld();
 #pragma unroll
-    for (int tt = 0; tt < 16; ++tt) {
-      const int t = 16 * part + tt;
-      p.wU2[ch * C * D + (size_t)t * D + lrow] = v[tt];
-      *reinterpret_cast<float *>(bU + sw128_offset(C, t, lrow)) = tf32_round(v[tt]);
-    }
+    for (int tt = 0; tt < 16; ++tt)
+      *reinterpret_cast<float *>(bU + sw128_offset(C, 16 * part + tt, lrow)) = tf32_round(v[tt]);
   }
   fence_async_smem();
   tc_fence_before();
-  __syncthreads();
+  __syncthreads();  // also ends every read of the dGam partials
   tc_fence_after();
   if (tid == 0) {
     if (ok) {
@@ -1179,8 +1188,17 @@ __global__ void __launch_bounds__(SP_NTH, 1) bwd_sprod_kernel(const BwdParams p)
     }
     mma_commit(bar + 1);  // covers every product issued, whatever happened above
   }
-  const bool done = ok && mbar_wait(bar + 1, 0);
-  if (!done && tid == 0) set_status(p.status, STATUS_TIMEOUT);
+  // dU^T rows of [dU^T ; dW^T] (rows = value columns c, K = tokens s) while it runs:
+  // element e takes column e % 128 and tokens 4 (e / 128) .. + 3
+#pragma unroll 1
+  for (int q = 0; q < D * C / 4 / SP_NTH; ++q) {
+    const int e = tid + q * SP_NTH, c = e & (D - 1), s0 = (e >> 7) * 4;
+    const float *src = p.wX + ch * C * D + c;
+    const float4 v = make_float4(src[(size_t)s0 * D], src[(size_t)(s0 + 1) * D],
+                                 src[(size_t)(s0 + 2) * D], src[(size_t)(s0 + 3) * D]);
+    *reinterpret_cast<float4 *>(bDUW + sw128_chunk(2 * D, c, s0)) = tf32_round4(v);
+  }
+  bool done = ok && mbar_wait(bar + 1, 0);
   tc_fence_after();
   if (done) {
     float v[16];
@@ -1193,118 +1211,26 @@ __global__ void __launch_bounds__(SP_NTH, 1) bwd_sprod_kernel(const BwdParams p)
 #pragma unroll
     for (int tt = 0; tt < 16; ++tt)
       p.wY[ch * D * D + C * D + (size_t)(16 * part + tt) * D + lrow] = v[tt];
-    tmem_ld16(tm + lane + TDW + 16 * part, v);  // dW
+    tmem_ld16(tm + lane + TDW + 16 * part, v);  // dW^T: rows 128 + key of [dU^T ; dW^T]
     tmem_wait_ld();
 #pragma unroll
-    for (int tt = 0; tt < 16; ++tt) p.wKh[ch * C * D + (size_t)(16 * part + tt) * D + lrow] = v[tt];
+    for (int tt = 0; tt < 16; ++tt)
+      *reinterpret_cast<float *>(bDUW + sw128_offset(2 * D, D + lrow, 16 * part + tt)) =
+          tf32_round(v[tt]);
   }
+  // stage 2: A operands on lanes t = 32 (w % 4) + lane for lane quarters 0 and 1; part
+  // w / 4 takes a quarter of the columns
+  const int t = lrow;
+  fence_async_smem();
   tc_fence_before();
-  __syncthreads();
-  if (!done && tid == 0) mbar_wait(bar + 1, 0, 100000000ull);  // let issued products finish
-  __syncthreads();
-  if (w == 0) {
-    tc_fence_after();
-    tmem_dealloc(tm, 512);
-  }
-}
-
-// ---------------------------------------------------------------------------
-// bwd_tprod (bf16 inputs, d = 128): the gradient pass's products of chunk-sized tiles
-// on the tensor cores, with M = 128 TMEM lanes of which the chunk's 64 tokens t use
-// the first 64:
-//   dP   = dO U^T                                 A = dO (lanes t), B = U (rows s)
-//   [T^T dU | T^T dW] = T^T [dU | dW]             A = T^T (lanes t), B = [dU^T ; dW^T]
-//                                                   (rows = 256 value columns, K = s)
-//   dZ   = -[(T^T dU) U~^T + (T^T dW) W^T]        A = the product above (K = 256),
-//                                                   B = [U~ | W] (rows s, K = 256)
-// tf32 operands rounded to nearest (the middle product is read from TMEM as it
-// stands), fp32 accumulation.  The results replace tiles the gradient pass no
-// longer reads: dP over T, T^T dU over dU, T^T dW over dW, dZ over U.
-// ---------------------------------------------------------------------------
-constexpr int TP_NTH = 512;
-
-struct TprodLayout {
-  static constexpr int D = 128;
-  // B operands (byte offsets, 1024-byte aligned): U (64 rows x 128), [dU^T ; dW^T]
-  // (256 rows x 64), [U~ | W] (64 rows x 256); then two mbarriers and the TMEM address
-  static constexpr int oU = 0, oDUW = oU + C * D * 4, oUtW = oDUW + 2 * D * C * 4;
-  static constexpr int oBar = oUtW + C * 2 * D * 4;
-  static constexpr size_t bytes = oBar + 32 + 1024;
-};
-
-__global__ void __launch_bounds__(TP_NTH, 1) bwd_tprod_kernel(const BwdParams p) {
-  using L = TprodLayout;
-  constexpr int D = L::D;
-  // TMEM columns: dO (A of the first product), later dZ; dP; T^T; [T^T dU | T^T dW]
-  constexpr uint32_t TDO = 0, TZ = 0, TP = 128, TT = 192, TB = 256;
-  extern __shared__ float4 smem_f4[];
-  unsigned char *sb = align1024_shared(smem_f4);
-  uint64_t *bar = reinterpret_cast<uint64_t *>(sb + L::oBar);
-  uint32_t *s_tmem = reinterpret_cast<uint32_t *>(sb + L::oBar + 16);
-  const int tid = threadIdx.x, w = tid >> 5, ln = tid & 31;
-  const int H = p.H;
-  const int jc = blockIdx.x / H, h = blockIdx.x % H;
-  const int4 cd = p.chunks[jc];
-  const int tok0 = cd.z, n = cd.w;
-  const size_t ch = (size_t)jc * H + h;
-  const float *U = p.wU2 + ch * C * D, *dU = p.wX + ch * C * D, *dW = p.wKh + ch * C * D;
-  const float *Ut = p.wU + ch * C * D, *W = p.wW + ch * C * D, *T = p.wT + ch * C * C;
-  if (w == 0) {
-    tmem_alloc(s_tmem, 512);
-    tmem_relinquish();
-  }
-  if (tid == 0) {
-    mbar_init(bar, 1);
-    mbar_init(bar + 1, 1);
-    asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
-  }
-  // B operands, rounded to tf32
-  unsigned char *bU = sb + L::oU, *bDUW = sb + L::oDUW, *bUtW = sb + L::oUtW;
-#pragma unroll
-  for (int q = 0; q < C * D / 4 / TP_NTH; ++q) {  // U: rows s, K = value columns
-    const int e = tid + q * TP_NTH, t = e >> 5, k = (e & 31) * 4;
-    const float4 u = *reinterpret_cast<const float4 *>(U + t * D + k);
-    *reinterpret_cast<float4 *>(bU + sw128_chunk(C, t, k)) = tf32_round4(u);
-  }
-#pragma unroll 2
-  for (int q = 0; q < 2 * D * C / 4 / TP_NTH; ++q) {  // [dU^T ; dW^T]: rows c', K = s
-    const int e = tid + q * TP_NTH, c2 = e & (2 * D - 1), s0 = (e >> 8) * 4;
-    const float *src = c2 < D ? dU + c2 : dW + (c2 - D);
-    float4 v;
-    v.x = src[(size_t)s0 * D];
-    v.y = src[(size_t)(s0 + 1) * D];
-    v.z = src[(size_t)(s0 + 2) * D];
-    v.w = src[(size_t)(s0 + 3) * D];
-    *reinterpret_cast<float4 *>(bDUW + sw128_chunk(2 * D, c2, s0)) = tf32_round4(v);
-  }
-#pragma unroll 2
-  for (int q = 0; q < C * 2 * D / 4 / TP_NTH; ++q) {  // [U~ | W]: rows s, K = c'
-    const int e = tid + q * TP_NTH, t = e >> 6, k = (e & 63) * 4;
-    const float4 v = k < D ? *reinterpret_cast<const float4 *>(Ut + t * D + k)
-                           : *reinterpret_cast<const float4 *>(W + t * D + (k - D));
-    *reinterpret_cast<float4 *>(bUtW + sw128_chunk(C, t, k)) = tf32_round4(v);
-  }
-  tc_fence_before();
-  __syncthreads();
+  done = __syncthreads_and(done);  // every stage-1 read of TMEM is done
   tc_fence_after();
-  const uint32_t tm = *s_tmem;
-  // A operands: warps of lane quarters 0 and 1 hold tokens t = 32 (w % 4) + lane; part
-  // w / 4 takes a quarter of the columns.  Lanes 64..127 are left as they are: they
-  // only reach accumulator lanes that nothing reads.
-  const int qd = w & 3, part = w >> 2;
-  const uint32_t lane = (uint32_t)(32 * qd) << 16;
-  const int t = 32 * qd + ln;
-  if (qd < 2) {
-    float v[32];  // dO row t, value columns 32 part .. + 31 (rows past the chunk: zero)
-    const bool live = p.d_o && t < n;
-    const float4 *src =
-        reinterpret_cast<const float4 *>(p.d_o + ((size_t)(tok0 + (live ? t : 0)) * H + h) * D);
+  if (done && qd < 2) {
+    float v[32];  // dO row t, value columns 32 part .. + 31, from its B tile (rounded)
 #pragma unroll
-    for (int q = 0; q < 8; ++q) {
-      const float4 x = live ? src[8 * part + q] : make_float4(0.f, 0.f, 0.f, 0.f);
-      v[4 * q] = tf32_round(x.x), v[4 * q + 1] = tf32_round(x.y);
-      v[4 * q + 2] = tf32_round(x.z), v[4 * q + 3] = tf32_round(x.w);
-    }
+    for (int q = 0; q < 8; ++q)
+      *reinterpret_cast<float4 *>(&v[4 * q]) =
+          *reinterpret_cast<const float4 *>(bO + sw128_chunk(C, t, 32 * part + 4 * q));
     tmem_st32(tm + lane + TDO + 32 * part, v);
     float tv[16];  // T^T row t: T[s][t] for s = 16 part .. + 15
 #pragma unroll
@@ -1312,50 +1238,49 @@ __global__ void __launch_bounds__(TP_NTH, 1) bwd_tprod_kernel(const BwdParams p)
     tmem_st16(tm + lane + TT + 16 * part, tv);
   }
   tmem_wait_st();
-  fence_async_smem();
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
-  bool ok = true;
   if (tid == 0) {
-    const uint32_t ub = smem_u32(bU), dwb = smem_u32(bDUW), uwb = smem_u32(bUtW);
+    if (done) {
+      const uint32_t ub = smem_u32(bU), dwb = smem_u32(bDUW), uwb = smem_u32(bUt);
 #pragma unroll
-    for (int s = 0; s < D / 8; ++s)
-      mma_tf32_ts(tm + TP, tm + TDO + 8 * s, sw128_desc(ub, C, s), idesc_tf32(C), s > 0);
+      for (int s = 0; s < D / 8; ++s)
+        mma_tf32_ts(tm + TP, tm + TDO + 8 * s, sw128_desc(ub, C, s), idesc_tf32(C), s > 0);
 #pragma unroll
-    for (int s = 0; s < C / 8; ++s)
-      mma_tf32_ts(tm + TB, tm + TT + 8 * s, sw128_desc(dwb, 2 * D, s), idesc_tf32(2 * D),
-                  s > 0);
-    mma_commit(bar);
-    ok = mbar_wait(bar, 0);  // the middle product is the next one's A; dO's columns free
-    tc_fence_after();
-    if (ok) {
-#pragma unroll
-      for (int s = 0; s < 2 * D / 8; ++s)
-        mma_tf32_ts(tm + TZ, tm + TB + 8 * s, sw128_desc(uwb, C, s), idesc_tf32(C, true),
+      for (int s = 0; s < C / 8; ++s)
+        mma_tf32_ts(tm + TB, tm + TT + 8 * s, sw128_desc(dwb, 2 * D, s), idesc_tf32(2 * D),
                     s > 0);
+      mma_commit(bar + 2);
+      // the middle product is the next one's A, and dO's columns take dZ
+      done = mbar_wait(bar + 2, 0);
+      tc_fence_after();
+      if (done) {
+#pragma unroll
+        for (int s = 0; s < 2 * D / 8; ++s)
+          mma_tf32_ts(tm + TZ, tm + TB + 8 * s, sw128_desc(uwb, C, s), idesc_tf32(C, true),
+                      s > 0);
+      }
     }
-    mma_commit(bar + 1);  // covers every product issued
+    mma_commit(bar + 3);  // covers every product issued
   }
-  const bool done = __syncthreads_and(ok) && mbar_wait(bar + 1, 0);
+  done = __syncthreads_and(done) && mbar_wait(bar + 3, 0);
   if (!done && tid == 0) set_status(p.status, STATUS_TIMEOUT);
   tc_fence_after();
   if (done && qd < 2) {
     float v[32];
-    // dP row t over T, columns 16 part .. + 15
-    tmem_ld16(tm + lane + TP + 16 * part, v);
+    tmem_ld16(tm + lane + TP + 16 * part, v);  // dP row t over T, columns 16 part .. + 15
     tmem_wait_ld();
     float4 *dst = reinterpret_cast<float4 *>(p.wT + ch * C * C + (size_t)t * C + 16 * part);
 #pragma unroll
     for (int q = 0; q < 4; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-    // dZ row t over U, columns 16 part .. + 15
-    tmem_ld16(tm + lane + TZ + 16 * part, v);
+    tmem_ld16(tm + lane + TZ + 16 * part, v);  // dZ row t over U, columns 16 part .. + 15
     tmem_wait_ld();
     dst = reinterpret_cast<float4 *>(p.wU2 + ch * C * D + (size_t)t * C + 16 * part);
 #pragma unroll
     for (int q = 0; q < 4; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
     // [T^T dU | T^T dW] row t: part p takes columns 64 p .. + 63 (parts 0, 1: T^T dU over
-    // dU; parts 2, 3: T^T dW over dW)
+    // dU; parts 2, 3: T^T dW over Khat)
     float *row = (part < 2 ? p.wX : p.wKh) + ch * C * D + (size_t)t * D + 64 * (part & 1);
 #pragma unroll
     for (int hh = 0; hh < 2; ++hh) {
@@ -1368,7 +1293,7 @@ __global__ void __launch_bounds__(TP_NTH, 1) bwd_tprod_kernel(const BwdParams p)
   }
   tc_fence_before();
   __syncthreads();
-  if (!done && tid == 0) mbar_wait(bar + 1, 0, 100000000ull);  // let issued products finish
+  if (!done && tid == 0) mbar_wait(bar + 3, 0, 100000000ull);  // let issued products finish
   __syncthreads();
   if (w == 0) {
     tc_fence_after();
@@ -1470,7 +1395,7 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
       accG[i][j] = gq * sQ[e];
       accK[i][j] = 0.f;
     }
-  // dP = tril(dO U^T)  (from bwd_tprod, over T, when it ran)
+  // dP = tril(dO U^T)  (from bwd_sprod, over T, when it ran)
   {
     float pp[4][4];
     if constexpr (PRE) {
@@ -1541,7 +1466,7 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
   }
 
   // dW = -dU S^T (into the dO tile; the sync above ends every read of that tile);
-  // with the tensor cores, bwd_tprod has already taken every product with dW
+  // with the tensor cores, bwd_sprod has already taken every product with dW
   if constexpr (!PRE) {
     zero(acc);
     mm_acc<4, NJ>(acc, dU, D, 1, S, 1, D, D, sStage);
@@ -1559,7 +1484,7 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
     for (int q = 0; q < C * C / 4 / NTH; ++q)
       reinterpret_cast<float4 *>(sT)[tid + q * NTH] = tv[q];
   }
-  // T^T dU -> dV = Diag(beta) T^T dU, dbeta += (T^T dU) . v  (T^T dU from bwd_tprod, over
+  // T^T dU -> dV = Diag(beta) T^T dU, dbeta += (T^T dU) . v  (T^T dU from bwd_sprod, over
   // dU, when it ran)
   if constexpr (PRE) {
     load_own(dU);
@@ -1582,7 +1507,7 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
     if (tx == 0) sDb[t] += rs;
   }
   // T^T dW -> d(gamma K) = Diag(beta) T^T dW;  dbeta += (T^T dW) . (gamma k)  (from
-  // bwd_tprod, over dW, when it ran)
+  // bwd_sprod, over dW, when it ran)
   if constexpr (PRE) {
     load_own(p.wKh + ch * C * D);
   } else {
@@ -1614,7 +1539,7 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
     for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int j = 0; j < 4; ++j) av[i][j] = p.wA[ch * C * C + (ty + 16 * i) * C + tx + 16 * j];
-    float tt[4][4];  // -dZ  (dZ from bwd_tprod, over U, when it ran)
+    float tt[4][4];  // -dZ  (dZ from bwd_sprod, over U, when it ran)
     if constexpr (PRE) {
 #pragma unroll
       for (int i = 0; i < 4; ++i)
@@ -1784,13 +1709,6 @@ cudaError_t launch_bwd_d(const BwdParams &p, cudaStream_t stream) {
     if (chunk_grid > 0) {
       if ((e = set_smem(bwd_sprod_kernel, SprodLayout::bytes)) != cudaSuccess) return e;
       bwd_sprod_kernel<<<chunk_grid, SP_NTH, SprodLayout::bytes, stream>>>(p);
-      if ((e = cudaGetLastError()) != cudaSuccess) return e;
-    }
-  }
-  if constexpr (kPrepTensorCores<D, TIn>) {
-    if (chunk_grid > 0) {
-      if ((e = set_smem(bwd_tprod_kernel, TprodLayout::bytes)) != cudaSuccess) return e;
-      bwd_tprod_kernel<<<chunk_grid, TP_NTH, TprodLayout::bytes, stream>>>(p);
       if ((e = cudaGetLastError()) != cudaSuccess) return e;
     }
   }
