@@ -191,22 +191,22 @@ __device__ __forceinline__ void unpack16(const uint4 &u, const __nv_bfloat16 *, 
     x[2 * q + 1] = __uint_as_float(w[q] & 0xFFFF0000u);
   }
 }
-template <int D, typename TIn>
+template <int D, typename TIn, int NT = NTH>
 __device__ void stage_rows(float *dst, int ld, const TIn *src, int tok0, int n, int H, int h) {
   constexpr int VEC = 16 / (int)sizeof(TIn);  // elements per 16-byte load
-  constexpr int PER_ROW = D / VEC, ITER = C * PER_ROW / NTH;
-  static_assert(ITER * NTH == C * PER_ROW, "tile must split evenly over the CTA");
+  constexpr int PER_ROW = D / VEC, ITER = C * PER_ROW / NT;
+  static_assert(ITER * NT == C * PER_ROW, "tile must split evenly over the CTA");
   uint4 buf[ITER];
 #pragma unroll
   for (int it = 0; it < ITER; ++it) {
-    const int e = threadIdx.x + it * NTH, t = e / PER_ROW, cv = e % PER_ROW;
+    const int e = threadIdx.x + it * NT, t = e / PER_ROW, cv = e % PER_ROW;
     buf[it] = (src && t < n)
                   ? *reinterpret_cast<const uint4 *>(src + ((size_t)(tok0 + t) * H + h) * D + cv * VEC)
                   : make_uint4(0u, 0u, 0u, 0u);
   }
 #pragma unroll
   for (int it = 0; it < ITER; ++it) {
-    const int e = threadIdx.x + it * NTH, t = e / PER_ROW, cv = e % PER_ROW;
+    const int e = threadIdx.x + it * NT, t = e / PER_ROW, cv = e % PER_ROW;
     float x[VEC];
     unpack16(buf[it], src, x);
 #pragma unroll
@@ -216,12 +216,12 @@ __device__ void stage_rows(float *dst, int ld, const TIn *src, int tok0, int n, 
 
 // g rows into sG, then the in-place chunk-local cumsum scaled by log2(e)
 // (thread = channel); beta into sB.  Padded rows have g = 0 and beta = 0.
-template <int D>
+template <int D, int NT = NTH>
 __device__ void stage_gate(float *sG, float *sB, const BwdParams &p, int tok0, int n, int h) {
   if (p.g_logits)
-    stage_rows<D, __nv_bfloat16>(sG, D, p.g_logits, tok0, n, p.H, h);
+    stage_rows<D, __nv_bfloat16, NT>(sG, D, p.g_logits, tok0, n, p.H, h);
   else
-    stage_rows<D, float>(sG, D, p.g, tok0, n, p.H, h);
+    stage_rows<D, float, NT>(sG, D, p.g, tok0, n, p.H, h);
   if (threadIdx.x < C)
     sB[threadIdx.x] = threadIdx.x < n ? p.beta[(size_t)(tok0 + threadIdx.x) * p.H + h] : 0.f;
   __syncthreads();
@@ -244,24 +244,25 @@ __device__ void stage_gate(float *sG, float *sB, const BwdParams &p, int tok0, i
 }
 
 // Gate tables store a row's column c at a permuted position so the thread that owns
-// columns tx + 16 j (j < NJ) reads them as NJ / 4 float4 chunks (2 tx, 2 tx + 1 for
-// NJ = 8, with chunk bit 0 flipped by tx bit 2 so every quarter-warp covers all 32
-// banks; chunk tx for NJ = 4).
-template <int NJ>
+// columns tx + TX j (j < NJ) reads them as NJ / 4 float4 chunks (2 tx, 2 tx + 1 for
+// NJ = 8 at TX = 16, with chunk bit 0 flipped by tx bit 2 so every quarter-warp covers
+// all 32 banks; chunk tx for NJ = 4).
+template <int TX, int NJ>
 __device__ __forceinline__ int gate_pos(int c) {
-  const int tx = c & 15, j = c >> 4;
+  const int tx = c % TX, j = c / TX;
   if (NJ == 8) return 4 * ((2 * tx + (j >> 2)) ^ ((tx >> 2) & 1)) + (j & 3);
   return 4 * tx + j;
 }
-template <int NJ>
+template <int TX, int NJ>
 __device__ __forceinline__ int gate_chunk(int tx, int q) {
   return NJ == 8 ? ((2 * tx + q) ^ ((tx >> 2) & 1)) : tx;
 }
 
-// Sum over the 16 lanes that share a row (lanes tx = 0..15 of one half-warp).
-__device__ __forceinline__ float row_sum16(float x) {
+// Sum over the TX lanes that share a row (TX = 16: one half-warp; 32: the warp).
+template <int TX>
+__device__ __forceinline__ float row_sum(float x) {
 #pragma unroll
-  for (int off = 8; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
+  for (int off = TX / 2; off > 0; off >>= 1) x += __shfl_xor_sync(0xffffffffu, x, off);
   return x;
 }
 
@@ -286,6 +287,12 @@ struct PrepLayout {
 // rules out tf32 operands).
 template <int D, typename TIn>
 constexpr bool kPrepTensorCores = D == 128 && std::is_same<TIn, __nv_bfloat16>::value;
+
+// Threads of the gradient pass: 512 (16 x 32, four columns of d = 128 per thread) when
+// its dense products come from the tensor cores, else 256 (16 x 16, for the fp32 tile
+// products it then runs itself).
+template <int D, typename TIn>
+__host__ __device__ constexpr int grad_threads() { return kPrepTensorCores<D, TIn> ? 512 : 256; }
 
 // fp32 -> tf32, round to nearest even (the tensor cores read the 19 leading bits)
 __device__ __forceinline__ float tf32_round(float x) {
@@ -1315,18 +1322,19 @@ struct GradLayout {
 };
 
 template <int D, typename TIn>
-__global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
+__global__ void __launch_bounds__(grad_threads<D, TIn>(), 1) bwd_grad_kernel(const BwdParams p) {
   using L = GradLayout<D>;
-  constexpr int NJ = D / 16;
-  // U, d(gamma Q), dKhat, dW and dGam come from bwd_sprod (tensor cores) when it ran
+  // every dense product comes from bwd_sprod (tensor cores) when it ran
   constexpr bool PRE = kPrepTensorCores<D, TIn>;
+  // 16 x TX threads: thread (ty, tx) owns rows ty + 16 i and columns tx + TX j of a tile
+  constexpr int TX = grad_threads<D, TIn>() / 16, GN = 16 * TX, NJ = D / TX, NC = C / TX;
   extern __shared__ float4 smem_f4[];
   float *sm = reinterpret_cast<float *>(smem_f4);
   float *sK = sm + L::oK, *sQ = sm + L::oQ, *sV = sm + L::oV, *sO = sm + L::oO;
   float *sG = sm + L::oG, *sP = sm + L::oP, *sT = sm + L::oT, *sStage = sm + L::oStage;
   float *sB = sm + L::oB, *sDb = sm + L::oDb, *sExtra = sm + L::oX, *sPart = sm + L::oPart;
   float *sGam = sm + L::oGam;
-  const int tid = threadIdx.x, ty = tid >> 4, tx = tid & 15;
+  const int tid = threadIdx.x, ty = tid / TX, tx = tid % TX;
   const int H = p.H;
   const int jc = blockIdx.x / H, h = blockIdx.x % H;
   const int4 cd = p.chunks[jc];
@@ -1343,14 +1351,14 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
   const float *Ut = p.wU + ch * C * D;
   float *U = p.wU2 + ch * C * D;
 
-  stage_rows<D, TIn>(sK, D, static_cast<const TIn *>(p.k), tok0, n, H, h);
-  stage_rows<D, TIn>(sQ, D, static_cast<const TIn *>(p.q), tok0, n, H, h);
-  stage_rows<D, TIn>(sV, D, static_cast<const TIn *>(p.v), tok0, n, H, h);
-  if constexpr (!PRE) stage_rows<D, float>(sO, D, p.d_o, tok0, n, H, h);  // PRE: not read
+  stage_rows<D, TIn, GN>(sK, D, static_cast<const TIn *>(p.k), tok0, n, H, h);
+  stage_rows<D, TIn, GN>(sQ, D, static_cast<const TIn *>(p.q), tok0, n, H, h);
+  stage_rows<D, TIn, GN>(sV, D, static_cast<const TIn *>(p.v), tok0, n, H, h);
+  if constexpr (!PRE) stage_rows<D, float, GN>(sO, D, p.d_o, tok0, n, H, h);  // PRE: not read
   if (tid < C) sDb[tid] = 0.f;
-  stage_gate<D>(sG, sB, p, tok0, n, h);
+  stage_gate<D, GN>(sG, sB, p, tok0, n, h);
 
-  // the thread's elements: rows ty + 16 i, columns tx + 16 j
+  // the thread's elements: rows ty + 16 i, columns tx + TX j
   float accQ[4][NJ], accK[4][NJ], accG[4][NJ], acc[4][NJ];
   const float *G63 = sG + (C - 1) * D;
 
@@ -1359,7 +1367,7 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int j = 0; j < NJ; ++j) acc[i][j] = src[(ty + 16 * i) * D + tx + 16 * j];
+      for (int j = 0; j < NJ; ++j) acc[i][j] = src[(ty + 16 * i) * D + tx + TX * j];
   };
   if constexpr (!PRE) {
     // U = U~ - W S  (U~ loaded before the product so its latency hides under it)
@@ -1367,14 +1375,14 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int j = 0; j < NJ; ++j) ut[i][j] = Ut[(ty + 16 * i) * D + tx + 16 * j];
+      for (int j = 0; j < NJ; ++j) ut[i][j] = Ut[(ty + 16 * i) * D + tx + TX * j];
     zero(acc);
     mm_acc<4, NJ>(acc, W, D, 1, S, D, 1, D, sStage);
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
       for (int j = 0; j < NJ; ++j) {
-        const int e = (ty + 16 * i) * D + tx + 16 * j;
+        const int e = (ty + 16 * i) * D + tx + TX * j;
         U[e] = ut[i][j] - acc[i][j];
       }
   }
@@ -1389,7 +1397,7 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
   for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int j = 0; j < NJ; ++j) {
-      const int e = (ty + 16 * i) * D + tx + 16 * j;
+      const int e = (ty + 16 * i) * D + tx + TX * j;
       const float gq = acc[i][j] * exp2f(sG[e]);
       accQ[i][j] = gq;
       accG[i][j] = gq * sQ[e];
@@ -1397,21 +1405,21 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
     }
   // dP = tril(dO U^T)  (from bwd_sprod, over T, when it ran)
   {
-    float pp[4][4];
+    float pp[4][NC];
     if constexpr (PRE) {
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j) pp[i][j] = p.wT[ch * C * C + (ty + 16 * i) * C + tx + 16 * j];
+        for (int j = 0; j < NC; ++j) pp[i][j] = p.wT[ch * C * C + (ty + 16 * i) * C + tx + TX * j];
     } else {
       zero(pp);
-      mm_acc<4, 4>(pp, sO, D, 1, U, 1, D, D, sStage);
+      mm_acc<4, NC>(pp, sO, D, 1, U, 1, D, D, sStage);
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int t = ty + 16 * i, s = tx + 16 * j;
+      for (int j = 0; j < NC; ++j) {
+        const int t = ty + 16 * i, s = tx + TX * j;
         sP[t * C + s] = s <= t ? pp[i][j] : 0.f;
       }
   }
@@ -1427,14 +1435,14 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
     float colsum = 0.f;
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
-      const int c = tx + 16 * j, e = (ty + 16 * i) * D + c;
+      const int c = tx + TX * j, e = (ty + 16 * i) * D + c;
       const float f = exp2f(G63[c] - sG[e]);
       const float kh = sK[e] * f;
       accK[i][j] = fmaf(acc[i][j], f, accK[i][j]);
       accG[i][j] = fmaf(-acc[i][j], kh, accG[i][j]);
       colsum = fmaf(acc[i][j], kh, colsum);
     }
-    sPart[ty * D + tx + 16 * j] = colsum;
+    sPart[ty * D + tx + TX * j] = colsum;
   }
   // dGam = rowsum(dSn * S): warp w takes rows w, w + 8, ...; lanes walk the row
   if constexpr (PRE) {
@@ -1442,7 +1450,7 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
   } else {
     const int w = tid >> 5, ln = tid & 31;
 #pragma unroll 4
-    for (int row = w; row < D; row += NTH / 32) {
+    for (int row = w; row < D; row += GN / 32) {
       float a[D / 32], b[D / 32];
 #pragma unroll
       for (int q = 0; q < D / 32; ++q) {
@@ -1473,16 +1481,16 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int j = 0; j < NJ; ++j) sO[(ty + 16 * i) * D + tx + 16 * j] = -acc[i][j];
+      for (int j = 0; j < NJ; ++j) sO[(ty + 16 * i) * D + tx + TX * j] = -acc[i][j];
   }
   if constexpr (!PRE) {
-    float4 tv[C * C / 4 / NTH];
+    float4 tv[C * C / 4 / GN];
 #pragma unroll
-    for (int q = 0; q < C * C / 4 / NTH; ++q)
-      tv[q] = reinterpret_cast<const float4 *>(p.wT + ch * C * C)[tid + q * NTH];
+    for (int q = 0; q < C * C / 4 / GN; ++q)
+      tv[q] = reinterpret_cast<const float4 *>(p.wT + ch * C * C)[tid + q * GN];
 #pragma unroll
-    for (int q = 0; q < C * C / 4 / NTH; ++q)
-      reinterpret_cast<float4 *>(sT)[tid + q * NTH] = tv[q];
+    for (int q = 0; q < C * C / 4 / GN; ++q)
+      reinterpret_cast<float4 *>(sT)[tid + q * GN] = tv[q];
   }
   // T^T dU -> dV = Diag(beta) T^T dU, dbeta += (T^T dU) . v  (T^T dU from bwd_sprod, over
   // dU, when it ran)
@@ -1498,12 +1506,12 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
     float rs = 0.f;
 #pragma unroll
     for (int j = 0; j < NJ; ++j) {
-      const int c = tx + 16 * j;
+      const int c = tx + TX * j;
       rs = fmaf(acc[i][j], sV[t * D + c], rs);
       sV[t * D + c] = acc[i][j];  // the V tile now holds T^T dU (own elements only)
       if (t < n) p.dv[((size_t)(tok0 + t) * H + h) * D + c] = sB[t] * acc[i][j];
     }
-    rs = row_sum16(rs);
+    rs = row_sum<TX>(rs);
     if (tx == 0) sDb[t] += rs;
   }
   // T^T dW -> d(gamma K) = Diag(beta) T^T dW;  dbeta += (T^T dW) . (gamma k)  (from
@@ -1520,7 +1528,7 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
     float rs = 0.f;
 #pragma unroll
     for (int j = 0; j < NJ; ++j) {
-      const int e = t * D + tx + 16 * j;
+      const int e = t * D + tx + TX * j;
       const float kg = exp2f(sG[e]) * sK[e];
       const float dkg = sB[t] * acc[i][j];
       accK[i][j] = fmaf(dkg, exp2f(sG[e]), accK[i][j]);
@@ -1528,42 +1536,42 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
       rs = fmaf(acc[i][j], kg, rs);
       sO[e] = acc[i][j];  // the dO tile (dW) now holds T^T dW (own elements only)
     }
-    rs = row_sum16(rs);
+    rs = row_sum<TX>(rs);
     if (tx == 0) sDb[t] += rs;
   }
   // dZ = -[(T^T dU) U~^T + (T^T dW) W^T];  dA = tril_strict(Diag(beta) dZ) into the T tile;
   // dbeta += sum_{s<t} dZ_ts A_ts
   {
-    float av[4][4];
+    float av[4][NC];
 #pragma unroll
     for (int i = 0; i < 4; ++i)
 #pragma unroll
-      for (int j = 0; j < 4; ++j) av[i][j] = p.wA[ch * C * C + (ty + 16 * i) * C + tx + 16 * j];
-    float tt[4][4];  // -dZ  (dZ from bwd_sprod, over U, when it ran)
+      for (int j = 0; j < NC; ++j) av[i][j] = p.wA[ch * C * C + (ty + 16 * i) * C + tx + TX * j];
+    float tt[4][NC];  // -dZ  (dZ from bwd_sprod, over U, when it ran)
     if constexpr (PRE) {
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < 4; ++j)
-          tt[i][j] = -p.wU2[ch * C * D + (ty + 16 * i) * C + tx + 16 * j];
+        for (int j = 0; j < NC; ++j)
+          tt[i][j] = -p.wU2[ch * C * D + (ty + 16 * i) * C + tx + TX * j];
     } else {
       zero(tt);
-      mm_acc<4, 4>(tt, sV, D, 1, Ut, 1, D, D, sStage);
-      mm_acc<4, 4>(tt, sO, D, 1, W, 1, D, D, sStage);
+      mm_acc<4, NC>(tt, sV, D, 1, Ut, 1, D, D, sStage);
+      mm_acc<4, NC>(tt, sO, D, 1, W, 1, D, D, sStage);
     }
 #pragma unroll
     for (int i = 0; i < 4; ++i) {
       const int t = ty + 16 * i;
       float rs = 0.f;
 #pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        const int s = tx + 16 * j;
+      for (int j = 0; j < NC; ++j) {
+        const int s = tx + TX * j;
         const float dz = -tt[i][j];
         const bool low = s < t;
         if (low) rs = fmaf(dz, av[i][j], rs);
         sT[t * C + s] = low ? sB[t] * dz : 0.f;  // dA (T is no longer needed)
       }
-      rs = row_sum16(rs);
+      rs = row_sum<TX>(rs);
       if (tx == 0) sDb[t] += rs;
     }
   }
@@ -1580,9 +1588,9 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
   for (int b = 0; b < 4; ++b) {
     const int r0 = 16 * b, r1 = r0 + 15;
     __syncthreads();
-    for (int e = tid; e < (r0 + 16) * D; e += NTH) {
+    for (int e = tid; e < (r0 + 16) * D; e += GN) {
       const int c = e % D;
-      sO[e - c + gate_pos<NJ>(c)] = sK[e] * exp2f(sG[r0 * D + c] - sG[e]);
+      sO[e - c + gate_pos<TX, NJ>(c)] = sK[e] * exp2f(sG[r0 * D + c] - sG[e]);
     }
     __syncthreads();
     {
@@ -1597,7 +1605,7 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
 #pragma unroll
         for (int q = 0; q < NJ / 4; ++q)
           *reinterpret_cast<float4 *>(&tb[4 * q]) =
-              *reinterpret_cast<const float4 *>(sO + s2 * D + 4 * gate_chunk<NJ>(tx, q));
+              *reinterpret_cast<const float4 *>(sO + s2 * D + 4 * gate_chunk<TX, NJ>(tx, q));
 #pragma unroll
         for (int j = 0; j < NJ; ++j) {
           op[j] = fmaf(dp, tb[j], op[j]);
@@ -1606,7 +1614,7 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
       }
 #pragma unroll
       for (int j = 0; j < NJ; ++j) {
-        const int c = tx + 16 * j, e = t * D + c;
+        const int c = tx + TX * j, e = t * D + c;
         const float f = exp2f(sG[e] - sG[r0 * D + c]);
         const float p1 = op[j] * f, a1 = oa[j] * f;
         accQ[b][j] += p1;
@@ -1615,8 +1623,8 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
       }
     }
     __syncthreads();
-    for (int e = r0 * D + tid; e < C * D; e += NTH) {
-      const int c = e % D, at = e - c + gate_pos<NJ>(c);
+    for (int e = r0 * D + tid; e < C * D; e += GN) {
+      const int c = e % D, at = e - c + gate_pos<TX, NJ>(c);
       const float f = exp2f(sG[e] - sG[r1 * D + c]);
       sO[at] = sQ[e] * f;
       sV[at] = sK[e] * f;
@@ -1634,16 +1642,16 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
 #pragma unroll
         for (int q = 0; q < NJ / 4; ++q) {
           *reinterpret_cast<float4 *>(&qb[4 * q]) =
-              *reinterpret_cast<const float4 *>(sO + t * D + 4 * gate_chunk<NJ>(tx, q));
+              *reinterpret_cast<const float4 *>(sO + t * D + 4 * gate_chunk<TX, NJ>(tx, q));
           *reinterpret_cast<float4 *>(&kb[4 * q]) =
-              *reinterpret_cast<const float4 *>(sV + t * D + 4 * gate_chunk<NJ>(tx, q));
+              *reinterpret_cast<const float4 *>(sV + t * D + 4 * gate_chunk<TX, NJ>(tx, q));
         }
 #pragma unroll
         for (int j = 0; j < NJ; ++j) o2[j] = fmaf(dp, qb[j], fmaf(da, kb[j], o2[j]));
       }
 #pragma unroll
       for (int j = 0; j < NJ; ++j) {
-        const int c = tx + 16 * j, e = s2 * D + c;
+        const int c = tx + TX * j, e = s2 * D + c;
         const float v2 = o2[j] * exp2f(sG[r1 * D + c] - sG[e]);
         accK[b][j] += v2;
         accG[b][j] = fmaf(-sK[e], v2, accG[b][j]);
@@ -1657,7 +1665,7 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
   for (int i = 0; i < 4; ++i)
 #pragma unroll
     for (int j = 0; j < NJ; ++j) {
-      const int t = ty + 16 * i, c = tx + 16 * j;
+      const int t = ty + 16 * i, c = tx + TX * j;
       sV[t * D + c] = accG[i][j];
       if (t < n) {
         const size_t o = ((size_t)(tok0 + t) * H + h) * D + c;
@@ -1675,7 +1683,7 @@ __global__ void __launch_bounds__(NTH, 1) bwd_grad_kernel(const BwdParams p) {
   }
   __syncthreads();
   // stored by the whole CTA; for gate logits x, times d log(alpha) / dx
-  for (int e = tid; e < n * D; e += NTH) {
+  for (int e = tid; e < n * D; e += GN) {
     const size_t o = ((size_t)(tok0 + e / D) * H + h) * D + e % D;
     p.dg[o] = p.g_logits ? sV[e] * gate_logit_slope(__bfloat162float(p.g_logits[o])) : sV[e];
   }
@@ -1714,7 +1722,7 @@ cudaError_t launch_bwd_d(const BwdParams &p, cudaStream_t stream) {
   }
   if (chunk_grid > 0) {
     if ((e = set_smem(bwd_grad_kernel<D, TIn>, GradLayout<D>::bytes)) != cudaSuccess) return e;
-    bwd_grad_kernel<D, TIn><<<chunk_grid, NTH, GradLayout<D>::bytes, stream>>>(p);
+    bwd_grad_kernel<D, TIn><<<chunk_grid, grad_threads<D, TIn>(), GradLayout<D>::bytes, stream>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   return cudaSuccess;
