@@ -294,6 +294,12 @@ constexpr bool kPrepTensorCores = D == 128 && std::is_same<TIn, __nv_bfloat16>::
 template <int D, typename TIn>
 __host__ __device__ constexpr int grad_threads() { return kPrepTensorCores<D, TIn> ? 512 : 256; }
 
+// Threads of the prep pass: 512 when its products run on the tensor cores (16 warps
+// share the operand staging and read-out; the triangular solve runs on the first 256),
+// else 256 (its fp32 tile products assume a 16 x 16 thread grid).
+template <int D, typename TIn>
+__host__ __device__ constexpr int prep_threads() { return kPrepTensorCores<D, TIn> ? 512 : 256; }
+
 // fp32 -> tf32, round to nearest even (the tensor cores read the 19 leading bits)
 __device__ __forceinline__ float tf32_round(float x) {
   uint32_t r;
@@ -302,9 +308,9 @@ __device__ __forceinline__ float tf32_round(float x) {
 }
 
 template <int D, typename TIn>
-__global__ void __launch_bounds__(NTH, 1) bwd_prep_kernel(const BwdParams p) {
+__global__ void __launch_bounds__(prep_threads<D, TIn>(), 1) bwd_prep_kernel(const BwdParams p) {
   using L = PrepLayout<D>;
-  constexpr int NJ = D / 16, LDP = L::LDP;
+  constexpr int NJ = D / 16, LDP = L::LDP, PN = prep_threads<D, TIn>();
   extern __shared__ float4 smem_f4[];
   float *sm = reinterpret_cast<float *>(align1024_shared(smem_f4));
   float *sK = sm + L::oK, *sQ = sm + L::oQ, *sG = sm + L::oG, *sA = sm + L::oA;
@@ -331,9 +337,9 @@ __global__ void __launch_bounds__(NTH, 1) bwd_prep_kernel(const BwdParams p) {
   }
   bool ap_done = true;
 
-  stage_rows<D, TIn>(sK, D, static_cast<const TIn *>(p.k), tok0, n, H, h);
-  stage_rows<D, TIn>(sQ, D, static_cast<const TIn *>(p.q), tok0, n, H, h);
-  stage_gate<D>(sG, sB, p, tok0, n, h);
+  stage_rows<D, TIn, PN>(sK, D, static_cast<const TIn *>(p.k), tok0, n, H, h);
+  stage_rows<D, TIn, PN>(sQ, D, static_cast<const TIn *>(p.q), tok0, n, H, h);
+  stage_gate<D, PN>(sG, sB, p, tok0, n, h);
 
   if constexpr (kPrepTensorCores<D, TIn>) {
     // A and P on the tensor cores, as in the forward: two 32-row blocks b with reference
@@ -352,24 +358,21 @@ __global__ void __launch_bounds__(NTH, 1) bwd_prep_kernel(const BwdParams p) {
     const uint32_t lane = (uint32_t)(32 * (w & 3)) << 16;
     const int lr = 32 * (w & 3) + ln, i = lr & 63, m = 32 * (i >> 5) + 15;
     unsigned char *rp = reinterpret_cast<unsigned char *>(sBuf);  // 1024-byte aligned
-    {
+    {  // warp w: lane quarter w % 4, channels 32 (w / 4) .. + 31
       const float *x = lr < C ? sK : sQ;
+      const int c0 = 32 * (w >> 2);
+      float v[32];
 #pragma unroll
-      for (int hh = 0; hh < 2; ++hh) {  // warp w % 4 ... w / 4 takes channels 64 (w / 4) + 32 hh..
-        const int c0 = 64 * (w >> 2) + 32 * hh;
-        float v[32];
-#pragma unroll
-        for (int jj = 0; jj < 32; ++jj) {
-          const int c = c0 + jj;
-          v[jj] = tf32_round(x[i * D + c] * exp2f(sG[i * D + c] - sG[m * D + c]));
-        }
-        tmem_st32(tm + lane + TL + c0, v);
+      for (int jj = 0; jj < 32; ++jj) {
+        const int c = c0 + jj;
+        v[jj] = tf32_round(x[i * D + c] * exp2f(sG[i * D + c] - sG[m * D + c]));
       }
+      tmem_st32(tm + lane + TL + c0, v);
     }
 #pragma unroll
     for (int b = 0; b < 2; ++b) {
       const int rows = 32 * (b + 1), mb = 32 * b + 15;
-      for (int e = tid; e < rows * (D / 4); e += NTH) {
+      for (int e = tid; e < rows * (D / 4); e += PN) {
         const int j = e / (D / 4), c = (e % (D / 4)) * 4;
         float4 r;
         r.x = tf32_round(sK[j * D + c] * exp2f(sG[mb * D + c] - sG[j * D + c]));
@@ -402,18 +405,18 @@ __global__ void __launch_bounds__(NTH, 1) bwd_prep_kernel(const BwdParams p) {
     ap_done = mbar_wait(bar + 1, 0);
     if (!ap_done && tid == 0) set_status(p.status, STATUS_TIMEOUT);
     tc_fence_after();
-    {  // row i (lane lr), columns 32 (w / 4) .. + 31: A for k rows, P for q rows
-      const int b = i >> 5, cb = 32 * (w >> 2);
-      float a0[32], a1[32];
-      tmem_ld32(tm + lane + apc(b, 0) + cb, a0);
-      tmem_ld32(tm + lane + apc(b, 1) + cb, a1);
+    {  // row i (lane lr), columns 16 (w / 4) .. + 15: A for k rows, P for q rows
+      const int b = i >> 5, cb = 16 * (w >> 2);
+      float a0[16], a1[16];
+      tmem_ld16(tm + lane + apc(b, 0) + cb, a0);
+      tmem_ld16(tm + lane + apc(b, 1) + cb, a1);
       tmem_wait_ld();
       if (lr < C) {
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) sA[i * C + cb + jj] = (cb + jj < i) ? a0[jj] + a1[jj] : 0.f;
+        for (int jj = 0; jj < 16; ++jj) sA[i * C + cb + jj] = (cb + jj < i) ? a0[jj] + a1[jj] : 0.f;
       } else {
 #pragma unroll
-        for (int jj = 0; jj < 32; ++jj) sP[i * C + cb + jj] = (cb + jj <= i) ? a0[jj] + a1[jj] : 0.f;
+        for (int jj = 0; jj < 16; ++jj) sP[i * C + cb + jj] = (cb + jj <= i) ? a0[jj] + a1[jj] : 0.f;
       }
     }
     tc_fence_before();
@@ -427,11 +430,11 @@ __global__ void __launch_bounds__(NTH, 1) bwd_prep_kernel(const BwdParams p) {
     for (int b = 0; b < 4; ++b) {
       const int r0 = 16 * b, rows = r0 + 16;
       __syncthreads();
-      for (int e = tid; e < rows * D; e += NTH) {
+      for (int e = tid; e < rows * D; e += PN) {
         const int s = e / D, c = e % D;
         sBuf[s * LDP + c] = sK[s * D + c] * exp2f(sG[r0 * D + c] - sG[s * D + c]);
       }
-      for (int e = tid; e < 16 * D; e += NTH) {
+      for (int e = tid; e < 16 * D; e += PN) {
         const int t = e / D, c = e % D;
         const float f = exp2f(sG[(r0 + t) * D + c] - sG[r0 * D + c]);
         sKL[t * LDP + c] = sK[(r0 + t) * D + c] * f;
@@ -464,30 +467,33 @@ __global__ void __launch_bounds__(NTH, 1) bwd_prep_kernel(const BwdParams p) {
   // row's sum and combine it with two shuffles inside their aligned group of four.
   // (2) The blocks below the diagonal, one block diagonal d at a time:
   //     T_ab = -T_aa sum_{c=b}^{a-1} N_ac T_cb,  N = Diag(beta) A,  b = a - d.
+  // Both steps run on threads 0..255 (16 x 16 for the second); the others wait at the
+  // CTA barriers.
   {
     const int task = tid >> 2, part = tid & 3;
     const int o = 16 * (task >> 4), j = o + (task & 15);
-    for (int i = o; i < o + 16; ++i) {
-      float acc = 0.f;
-      for (int s = j + part; s < i; s += 4) acc = fmaf(sA[i * C + s], sT[s * C + j], acc);
-      acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-      acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-      if (part == 0) sT[i * C + j] = i < j ? 0.f : (i == j ? 1.f : -sB[i] * acc);
-      __syncwarp();
-    }
-    for (int e = tid; e < C * C; e += NTH)  // blocks above the diagonal
+    if (tid < NTH)
+      for (int i = o; i < o + 16; ++i) {
+        float acc = 0.f;
+        for (int s = j + part; s < i; s += 4) acc = fmaf(sA[i * C + s], sT[s * C + j], acc);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
+        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
+        if (part == 0) sT[i * C + j] = i < j ? 0.f : (i == j ? 1.f : -sB[i] * acc);
+        __syncwarp();
+      }
+    for (int e = tid; e < C * C; e += PN)  // blocks above the diagonal
       if ((e / C) >> 4 < (e % C) >> 4) sT[e] = 0.f;
     float *Ys = sBuf;  // [3][16][17] scratch: N_a. T_.b of one block diagonal
     for (int d = 1; d < 4; ++d) {
       __syncthreads();
-      for (int a = d; a < 4; ++a) {
+      for (int a = d; a < 4 && tid < NTH; ++a) {
         const int bb = a - d, i = 16 * a + ty, jc = 16 * bb + tx;
         float y = 0.f;
         for (int s2 = 16 * bb; s2 < 16 * a; ++s2) y = fmaf(sA[i * C + s2], sT[s2 * C + jc], y);
         Ys[(bb * 16 + ty) * 17 + tx] = sB[i] * y;
       }
       __syncthreads();
-      for (int a = d; a < 4; ++a) {
+      for (int a = d; a < 4 && tid < NTH; ++a) {
         const int bb = a - d, i = 16 * a + ty, jc = 16 * bb + tx;
         float t = 0.f;
         for (int r = 16 * a; r <= i; ++r) t = fmaf(sT[i * C + r], Ys[(bb * 16 + r - 16 * a) * 17 + tx], t);
@@ -508,29 +514,30 @@ __global__ void __launch_bounds__(NTH, 1) bwd_prep_kernel(const BwdParams p) {
     __syncthreads();
     tc_fence_after();
     const uint32_t tm = *s_tmem;
-    const int w = tid >> 5, ln = tid & 31, c = 32 * (w & 3) + ln, j0 = 32 * (w >> 2);
+    // warp w: lane quarter w % 4 (channel c), tokens 16 (w / 4) .. + 15
+    const int w = tid >> 5, ln = tid & 31, c = 32 * (w & 3) + ln, j0 = 16 * (w >> 2);
     const uint32_t lane = (uint32_t)(32 * (w & 3)) << 16;
-    stage_rows<D, TIn>(sBuf, LDP, static_cast<const TIn *>(p.v), tok0, n, H, h);
+    stage_rows<D, TIn, PN>(sBuf, LDP, static_cast<const TIn *>(p.v), tok0, n, H, h);
     __syncthreads();
     {
-      float v1[32], v2[32];
+      float v1[16], v2[16];
 #pragma unroll
-      for (int jj = 0; jj < 32; ++jj) {
+      for (int jj = 0; jj < 16; ++jj) {
         const int j = j0 + jj;
         v1[jj] = tf32_round(sB[j] * exp2f(sG[j * D + c]) * sK[j * D + c]);
         v2[jj] = tf32_round(sB[j] * sBuf[j * LDP + c]);
       }
-      tmem_st32(tm + lane + TA1 + j0, v1);
-      tmem_st32(tm + lane + TA2 + j0, v2);
+      tmem_st16(tm + lane + TA1 + j0, v1);
+      tmem_st16(tm + lane + TA2 + j0, v2);
     }
     __syncthreads();  // V read out of the scratch tile
-    stage_rows<D, float>(sBuf, LDP, p.d_o, tok0, n, H, h);
+    stage_rows<D, float, PN>(sBuf, LDP, p.d_o, tok0, n, H, h);
     __syncthreads();
     {
-      float v3[32];
+      float v3[16];
 #pragma unroll
-      for (int jj = 0; jj < 32; ++jj) v3[jj] = tf32_round(sBuf[(j0 + jj) * LDP + c]);
-      tmem_st32(tm + lane + TA3 + j0, v3);
+      for (int jj = 0; jj < 16; ++jj) v3[jj] = tf32_round(sBuf[(j0 + jj) * LDP + c]);
+      tmem_st16(tm + lane + TA3 + j0, v3);
     }
     tmem_wait_st();
     __syncthreads();  // dO read out of the scratch tile: it takes the B tiles now
@@ -539,12 +546,12 @@ __global__ void __launch_bounds__(NTH, 1) bwd_prep_kernel(const BwdParams p) {
     unsigned char *bQ = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(sKL) + 1023) & ~uintptr_t(1023));
     // consecutive threads walk each source's contiguous axis (conflict-free reads)
-    for (int e = tid; e < C * C; e += NTH) {
+    for (int e = tid; e < C * C; e += PN) {
       const int a = e >> 6, b = e & 63;
       *reinterpret_cast<float *>(bT + sw128_offset(C, a, b)) = tf32_round(sT[a * C + b]);
       *reinterpret_cast<float *>(bP + sw128_offset(C, b, a)) = tf32_round(sP[a * C + b]);
     }
-    for (int e = tid; e < D * C; e += NTH) {
+    for (int e = tid; e < D * C; e += PN) {
       const int j = e / D, nn = e % D;
       *reinterpret_cast<float *>(bQ + sw128_offset(D, nn, j)) =
           tf32_round(exp2f(sG[j * D + nn]) * sQ[j * D + nn]);
@@ -570,26 +577,23 @@ __global__ void __launch_bounds__(NTH, 1) bwd_prep_kernel(const BwdParams p) {
     tc_fence_after();
     if (done) {
       float v[32];
-      tmem_ld32(tm + lane + TD1 + j0, v);  // W[token][channel]
+      tmem_ld16(tm + lane + TD1 + j0, v);  // W[token][channel]
       tmem_wait_ld();
 #pragma unroll
-      for (int jj = 0; jj < 32; ++jj) p.wW[ch * C * D + (size_t)(j0 + jj) * D + c] = v[jj];
-      tmem_ld32(tm + lane + TD2 + j0, v);  // U~
+      for (int jj = 0; jj < 16; ++jj) p.wW[ch * C * D + (size_t)(j0 + jj) * D + c] = v[jj];
+      tmem_ld16(tm + lane + TD2 + j0, v);  // U~
       tmem_wait_ld();
 #pragma unroll
-      for (int jj = 0; jj < 32; ++jj) p.wU[ch * C * D + (size_t)(j0 + jj) * D + c] = v[jj];
-      tmem_ld32(tm + lane + TD3 + j0, v);  // X
+      for (int jj = 0; jj < 16; ++jj) p.wU[ch * C * D + (size_t)(j0 + jj) * D + c] = v[jj];
+      tmem_ld16(tm + lane + TD3 + j0, v);  // X
       tmem_wait_ld();
 #pragma unroll
-      for (int jj = 0; jj < 32; ++jj) p.wX[ch * C * D + (size_t)(j0 + jj) * D + c] = v[jj];
+      for (int jj = 0; jj < 16; ++jj) p.wX[ch * C * D + (size_t)(j0 + jj) * D + c] = v[jj];
+      const int c0 = 32 * (w >> 2);  // Y[dk][dv] from Y^T (lane = dv), rows c0 .. + 31
+      tmem_ld32(tm + lane + TD4 + c0, v);
+      tmem_wait_ld();
 #pragma unroll
-      for (int half = 0; half < 2; ++half) {  // Y[dk][dv] from Y^T (lane = dv)
-        const int c0 = 64 * (w >> 2) + 32 * half;
-        tmem_ld32(tm + lane + TD4 + c0, v);
-        tmem_wait_ld();
-#pragma unroll
-        for (int jj = 0; jj < 32; ++jj) p.wY[ch * D * D + (size_t)(c0 + jj) * D + c] = v[jj];
-      }
+      for (int jj = 0; jj < 32; ++jj) p.wY[ch * D * D + (size_t)(c0 + jj) * D + c] = v[jj];
     }
     tc_fence_before();
     __syncthreads();
@@ -603,7 +607,7 @@ __global__ void __launch_bounds__(NTH, 1) bwd_prep_kernel(const BwdParams p) {
   } else {
   float acc[4][NJ];
     // W = T Diag(beta) (gamma K)
-    for (int e = tid; e < C * D; e += NTH) {
+    for (int e = tid; e < C * D; e += PN) {
       const int t = e / D, c = e % D;
       sBuf[t * LDP + c] = sB[t] * exp2f(sG[t * D + c]) * sK[t * D + c];
     }
@@ -616,7 +620,7 @@ __global__ void __launch_bounds__(NTH, 1) bwd_prep_kernel(const BwdParams p) {
     // U~ = T Diag(beta) V
     stage_rows<D, TIn>(sBuf, LDP, static_cast<const TIn *>(p.v), tok0, n, H, h);
     __syncthreads();
-    for (int e = tid; e < C * D; e += NTH) sBuf[(e / D) * LDP + e % D] *= sB[e / D];
+    for (int e = tid; e < C * D; e += PN) sBuf[(e / D) * LDP + e % D] *= sB[e / D];
     zero(acc);
     mm_acc<4, NJ>(acc, sT, C, 1, sBuf, LDP, 1, C, sStage);
   #pragma unroll
@@ -632,7 +636,7 @@ __global__ void __launch_bounds__(NTH, 1) bwd_prep_kernel(const BwdParams p) {
   #pragma unroll
       for (int j = 0; j < NJ; ++j) p.wX[ch * C * D + (ty + 16 * i) * D + tx + 16 * j] = acc[i][j];
     // Y = (gamma Q)^T dO
-    for (int e = tid; e < C * D; e += NTH) sQ[e] *= exp2f(sG[e]);
+    for (int e = tid; e < C * D; e += PN) sQ[e] *= exp2f(sG[e]);
     {
       float y[NJ][NJ];
       zero(y);
@@ -645,14 +649,14 @@ __global__ void __launch_bounds__(NTH, 1) bwd_prep_kernel(const BwdParams p) {
   }
 
   // Khat = exp(G_last - G) K, Gam = exp(G_last); A and T for the gradient pass
-  for (int e = tid; e < C * D; e += NTH) {
+  for (int e = tid; e < C * D; e += PN) {
     const int t = e / D, c = e % D;
     const float kh = sK[e] * exp2f(sG[(C - 1) * D + c] - sG[t * D + c]);
     // the tensor-core state pass reads Khat as a tf32 operand, copied as it is
     p.wKh[ch * C * D + e] = kPrepTensorCores<D, TIn> ? tf32_round(kh) : kh;
   }
   if (tid < D) p.wGam[ch * D + tid] = exp2f(sG[(C - 1) * D + tid]);
-  for (int e = tid; e < C * C; e += NTH) {
+  for (int e = tid; e < C * C; e += PN) {
     p.wA[ch * C * C + e] = sA[e];
     p.wT[ch * C * C + e] = sT[e];
   }
@@ -1701,7 +1705,7 @@ cudaError_t launch_bwd_d(const BwdParams &p, cudaStream_t stream) {
   const unsigned chunk_grid = (unsigned)((size_t)p.n_chunks * p.H);
   if (chunk_grid > 0) {
     if ((e = set_smem(bwd_prep_kernel<D, TIn>, PrepLayout<D>::bytes)) != cudaSuccess) return e;
-    bwd_prep_kernel<D, TIn><<<chunk_grid, NTH, PrepLayout<D>::bytes, stream>>>(p);
+    bwd_prep_kernel<D, TIn><<<chunk_grid, prep_threads<D, TIn>(), PrepLayout<D>::bytes, stream>>>(p);
     if ((e = cudaGetLastError()) != cudaSuccess) return e;
   }
   if constexpr (kPrepTensorCores<D, TIn>) {
