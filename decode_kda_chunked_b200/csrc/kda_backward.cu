@@ -1099,19 +1099,29 @@ __global__ void __launch_bounds__(SP_NTH, 1) bwd_sprod_kernel(const BwdParams p)
     asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
   }
 
-  // B operands: U~, W, dO (rows past the chunk's end are zero) and dU, rows = tokens
-  for (int e = tid; e < C * D / 4; e += SP_NTH) {
-    const int t = e >> 5, k = (e & 31) * 4;
-    const float4 utv = *reinterpret_cast<const float4 *>(Ut + t * D + k);
-    const float4 wv = *reinterpret_cast<const float4 *>(p.wW + ch * C * D + t * D + k);
-    const float4 uv = *reinterpret_cast<const float4 *>(p.wX + ch * C * D + t * D + k);
-    const float4 ov = (p.d_o && t < n) ? *reinterpret_cast<const float4 *>(
-                                             p.d_o + ((size_t)(tok0 + t) * H + h) * D + k)
-                                       : make_float4(0.f, 0.f, 0.f, 0.f);
-    *reinterpret_cast<float4 *>(bUt + sw128_chunk(C, t, k)) = tf32_round4(utv);
-    *reinterpret_cast<float4 *>(bW + sw128_chunk(C, t, k)) = tf32_round4(wv);
-    *reinterpret_cast<float4 *>(bDU + sw128_chunk(C, t, k)) = tf32_round4(uv);
-    *reinterpret_cast<float4 *>(bO + sw128_chunk(C, t, k)) = tf32_round4(ov);
+  // B operands: U~, W, dO (rows past the chunk's end are zero) and dU, rows = tokens;
+  // all of a thread's loads are issued before any of its stores
+  {
+    constexpr int NQ = C * D / 4 / SP_NTH;
+    float4 utv[NQ], wv[NQ], uv[NQ], ov[NQ];
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) {
+      const int e = tid + q * SP_NTH, t = e >> 5, k = (e & 31) * 4;
+      utv[q] = *reinterpret_cast<const float4 *>(Ut + t * D + k);
+      wv[q] = *reinterpret_cast<const float4 *>(p.wW + ch * C * D + t * D + k);
+      uv[q] = *reinterpret_cast<const float4 *>(p.wX + ch * C * D + t * D + k);
+      ov[q] = (p.d_o && t < n) ? *reinterpret_cast<const float4 *>(
+                                     p.d_o + ((size_t)(tok0 + t) * H + h) * D + k)
+                               : make_float4(0.f, 0.f, 0.f, 0.f);
+    }
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) {
+      const int e = tid + q * SP_NTH, t = e >> 5, k = (e & 31) * 4;
+      *reinterpret_cast<float4 *>(bUt + sw128_chunk(C, t, k)) = tf32_round4(utv[q]);
+      *reinterpret_cast<float4 *>(bW + sw128_chunk(C, t, k)) = tf32_round4(wv[q]);
+      *reinterpret_cast<float4 *>(bDU + sw128_chunk(C, t, k)) = tf32_round4(uv[q]);
+      *reinterpret_cast<float4 *>(bO + sw128_chunk(C, t, k)) = tf32_round4(ov[q]);
+    }
   }
   tc_fence_before();
   __syncthreads();
