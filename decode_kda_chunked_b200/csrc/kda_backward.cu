@@ -1288,28 +1288,52 @@ __global__ void __launch_bounds__(SP_NTH, 1) bwd_sprod_kernel(const BwdParams p)
   done = __syncthreads_and(done) && mbar_wait(bar + 3, 0);
   if (!done && tid == 0) set_status(p.status, STATUS_TIMEOUT);
   tc_fence_after();
+  // Results through shared memory (the B tiles are free once every product is done):
+  // lane t writes its row segments, then the CTA stores whole rows to the workspace.
+  // Row strides 1,040 and 272 bytes put a warp's 16-byte writes on distinct banks.
+  constexpr int RB = 1040, RS = 272, oSP = 64 * RB, oSZ = oSP + 64 * RS;
   if (done && qd < 2) {
     float v[32];
-    tmem_ld16(tm + lane + TP + 16 * part, v);  // dP row t over T, columns 16 part .. + 15
+    float4 *rb = reinterpret_cast<float4 *>(sb + t * RB);  // [T^T dU | T^T dW] row t
+    float4 *rp = reinterpret_cast<float4 *>(sb + oSP + t * RS) + 4 * part;  // dP
+    float4 *rz = reinterpret_cast<float4 *>(sb + oSZ + t * RS) + 4 * part;  // dZ
+    tmem_ld16(tm + lane + TP + 16 * part, v);
     tmem_wait_ld();
-    float4 *dst = reinterpret_cast<float4 *>(p.wT + ch * C * C + (size_t)t * C + 16 * part);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-    tmem_ld16(tm + lane + TZ + 16 * part, v);  // dZ row t over U, columns 16 part .. + 15
+    for (int q = 0; q < 4; ++q) rp[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+    tmem_ld16(tm + lane + TZ + 16 * part, v);
     tmem_wait_ld();
-    dst = reinterpret_cast<float4 *>(p.wU2 + ch * C * D + (size_t)t * C + 16 * part);
 #pragma unroll
-    for (int q = 0; q < 4; ++q) dst[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
-    // [T^T dU | T^T dW] row t: part p takes columns 64 p .. + 63 (parts 0, 1: T^T dU over
-    // dU; parts 2, 3: T^T dW over Khat)
-    float *row = (part < 2 ? p.wX : p.wKh) + ch * C * D + (size_t)t * D + 64 * (part & 1);
+    for (int q = 0; q < 4; ++q) rz[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
 #pragma unroll
-    for (int hh = 0; hh < 2; ++hh) {
+    for (int hh = 0; hh < 2; ++hh) {  // columns 64 part + 32 hh .. + 31
       tmem_ld32(tm + lane + TB + 64 * part + 32 * hh, v);
       tmem_wait_ld();
-      float4 *d4 = reinterpret_cast<float4 *>(row + 32 * hh);
 #pragma unroll
-      for (int q = 0; q < 8; ++q) d4[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+      for (int q = 0; q < 8; ++q)
+        rb[16 * part + 8 * hh + q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+    }
+  }
+  tc_fence_before();
+  if (__syncthreads_and(done)) {
+    // 6,144 float4: T^T dU over dU, T^T dW over Khat (64 rows x 64 float4), then dP over T
+    // and dZ over U (64 rows x 16 float4 each); a warp stores 512 contiguous bytes
+#pragma unroll 4
+    for (int q = 0; q < 6144 / SP_NTH; ++q) {
+      const int e = tid + q * SP_NTH;
+      float4 x;
+      float *dst;
+      if (e < 4096) {
+        const int row = e >> 6, c4 = e & 63;
+        x = *reinterpret_cast<const float4 *>(sb + row * RB + 16 * c4);
+        dst = (c4 < 32 ? p.wX : p.wKh) + ch * C * D + (size_t)row * D + 4 * (c4 & 31);
+      } else {
+        const int e2 = (e - 4096) & 1023, row = e2 >> 4, c4 = e2 & 15;
+        const bool z = e >= 5120;
+        x = *reinterpret_cast<const float4 *>(sb + (z ? oSZ : oSP) + row * RS + 16 * c4);
+        dst = (z ? p.wU2 + ch * C * D : p.wT + ch * C * C) + (size_t)row * C + 4 * c4;
+      }
+      *reinterpret_cast<float4 *>(dst) = x;
     }
   }
   tc_fence_before();
