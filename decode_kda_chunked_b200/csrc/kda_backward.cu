@@ -217,11 +217,12 @@ __device__ void stage_rows(float *dst, int ld, const TIn *src, int tok0, int n, 
 // g rows into sG, then the in-place chunk-local cumsum scaled by log2(e)
 // (thread = channel); beta into sB.  Padded rows have g = 0 and beta = 0.
 template <int D, int NT = NTH>
-__device__ void stage_gate(float *sG, float *sB, const BwdParams &p, int tok0, int n, int h) {
+__device__ void stage_gate(float *sG, float *sB, const BwdParams &p, int tok0, int n, int h,
+                           int ld = D) {
   if (p.g_logits)
-    stage_rows<D, __nv_bfloat16, NT>(sG, D, p.g_logits, tok0, n, p.H, h);
+    stage_rows<D, __nv_bfloat16, NT>(sG, ld, p.g_logits, tok0, n, p.H, h);
   else
-    stage_rows<D, float, NT>(sG, D, p.g, tok0, n, p.H, h);
+    stage_rows<D, float, NT>(sG, ld, p.g, tok0, n, p.H, h);
   if (threadIdx.x < C)
     sB[threadIdx.x] = threadIdx.x < n ? p.beta[(size_t)(tok0 + threadIdx.x) * p.H + h] : 0.f;
   __syncthreads();
@@ -230,13 +231,13 @@ __device__ void stage_gate(float *sG, float *sB, const BwdParams &p, int tok0, i
     float run = 0.f;
     if (p.g_logits) {
       for (int t = 0; t < C; ++t) {
-        run += t < n ? gate_from_logit(sG[t * D + c]) : 0.f;
-        sG[t * D + c] = run * LOG2E;
+        run += t < n ? gate_from_logit(sG[t * ld + c]) : 0.f;
+        sG[t * ld + c] = run * LOG2E;
       }
     } else {
       for (int t = 0; t < C; ++t) {
-        run += sG[t * D + c];
-        sG[t * D + c] = run * LOG2E;
+        run += sG[t * ld + c];
+        sG[t * ld + c] = run * LOG2E;
       }
     }
   }
@@ -271,9 +272,12 @@ __device__ __forceinline__ float row_sum(float x) {
 // ---------------------------------------------------------------------------
 template <int D>
 struct PrepLayout {
-  static constexpr int LDP = D + 1;
-  static constexpr int oK = 0, oQ = oK + C * D, oG = oQ + C * D, oA = oG + C * D;
-  static constexpr int oP = oA + C * C, oT = oP + C * C, oBuf = oT + C * C;
+  // Row strides: LDP for the scratch tiles; the k, q and g tiles take D + 1 and the A and
+  // P tiles C + 1 (kernels that read them with one lane per row then hit distinct banks)
+  static constexpr int LDP = D + 1, LK = D + 1, LA = C + 1;
+  static constexpr int oK = 0, oQ = oK + C * LK, oG = oQ + C * LK;
+  static constexpr int oA = (oG + C * LK + 255) / 256 * 256;  // keeps oBuf 1024-byte aligned
+  static constexpr int oP = oA + C * LA, oT = oP + C * LA, oBuf = oT + C * C + 128;
   static constexpr int oKL = oBuf + C * LDP, oQL = oKL + 16 * LDP, oStage = oQL + 16 * LDP;
   static constexpr int oB = oStage + stage_floats(D, D);
   static constexpr int oMisc = oB + C;  // two mbarriers (8 bytes each) and the TMEM base address
@@ -310,7 +314,7 @@ __device__ __forceinline__ float tf32_round(float x) {
 template <int D, typename TIn>
 __global__ void __launch_bounds__(prep_threads<D, TIn>(), 1) bwd_prep_kernel(const BwdParams p) {
   using L = PrepLayout<D>;
-  constexpr int NJ = D / 16, LDP = L::LDP, PN = prep_threads<D, TIn>();
+  constexpr int NJ = D / 16, LDP = L::LDP, LK = L::LK, LA = L::LA, PN = prep_threads<D, TIn>();
   extern __shared__ float4 smem_f4[];
   float *sm = reinterpret_cast<float *>(align1024_shared(smem_f4));
   float *sK = sm + L::oK, *sQ = sm + L::oQ, *sG = sm + L::oG, *sA = sm + L::oA;
@@ -337,9 +341,9 @@ __global__ void __launch_bounds__(prep_threads<D, TIn>(), 1) bwd_prep_kernel(con
   }
   bool ap_done = true;
 
-  stage_rows<D, TIn, PN>(sK, D, static_cast<const TIn *>(p.k), tok0, n, H, h);
-  stage_rows<D, TIn, PN>(sQ, D, static_cast<const TIn *>(p.q), tok0, n, H, h);
-  stage_gate<D, PN>(sG, sB, p, tok0, n, h);
+  stage_rows<D, TIn, PN>(sK, LK, static_cast<const TIn *>(p.k), tok0, n, H, h);
+  stage_rows<D, TIn, PN>(sQ, LK, static_cast<const TIn *>(p.q), tok0, n, H, h);
+  stage_gate<D, PN>(sG, sB, p, tok0, n, h, LK);
 
   if constexpr (kPrepTensorCores<D, TIn>) {
     // A and P on the tensor cores, as in the forward: two 32-row blocks b with reference
@@ -365,7 +369,7 @@ __global__ void __launch_bounds__(prep_threads<D, TIn>(), 1) bwd_prep_kernel(con
 #pragma unroll
       for (int jj = 0; jj < 32; ++jj) {
         const int c = c0 + jj;
-        v[jj] = tf32_round(x[i * D + c] * exp2f(sG[i * D + c] - sG[m * D + c]));
+        v[jj] = tf32_round(x[i * LK + c] * exp2f(sG[i * LK + c] - sG[m * LK + c]));
       }
       tmem_st32(tm + lane + TL + c0, v);
     }
@@ -375,10 +379,10 @@ __global__ void __launch_bounds__(prep_threads<D, TIn>(), 1) bwd_prep_kernel(con
       for (int e = tid; e < rows * (D / 4); e += PN) {
         const int j = e / (D / 4), c = (e % (D / 4)) * 4;
         float4 r;
-        r.x = tf32_round(sK[j * D + c] * exp2f(sG[mb * D + c] - sG[j * D + c]));
-        r.y = tf32_round(sK[j * D + c + 1] * exp2f(sG[mb * D + c + 1] - sG[j * D + c + 1]));
-        r.z = tf32_round(sK[j * D + c + 2] * exp2f(sG[mb * D + c + 2] - sG[j * D + c + 2]));
-        r.w = tf32_round(sK[j * D + c + 3] * exp2f(sG[mb * D + c + 3] - sG[j * D + c + 3]));
+        r.x = tf32_round(sK[j * LK + c] * exp2f(sG[mb * LK + c] - sG[j * LK + c]));
+        r.y = tf32_round(sK[j * LK + c + 1] * exp2f(sG[mb * LK + c + 1] - sG[j * LK + c + 1]));
+        r.z = tf32_round(sK[j * LK + c + 2] * exp2f(sG[mb * LK + c + 2] - sG[j * LK + c + 2]));
+        r.w = tf32_round(sK[j * LK + c + 3] * exp2f(sG[mb * LK + c + 3] - sG[j * LK + c + 3]));
         *reinterpret_cast<float4 *>(rp + 16384 * b + sw128_chunk(rows, j, c)) = r;
       }
     }
@@ -413,10 +417,10 @@ __global__ void __launch_bounds__(prep_threads<D, TIn>(), 1) bwd_prep_kernel(con
       tmem_wait_ld();
       if (lr < C) {
 #pragma unroll
-        for (int jj = 0; jj < 16; ++jj) sA[i * C + cb + jj] = (cb + jj < i) ? a0[jj] + a1[jj] : 0.f;
+        for (int jj = 0; jj < 16; ++jj) sA[i * LA + cb + jj] = (cb + jj < i) ? a0[jj] + a1[jj] : 0.f;
       } else {
 #pragma unroll
-        for (int jj = 0; jj < 16; ++jj) sP[i * C + cb + jj] = (cb + jj <= i) ? a0[jj] + a1[jj] : 0.f;
+        for (int jj = 0; jj < 16; ++jj) sP[i * LA + cb + jj] = (cb + jj <= i) ? a0[jj] + a1[jj] : 0.f;
       }
     }
     tc_fence_before();
@@ -432,13 +436,13 @@ __global__ void __launch_bounds__(prep_threads<D, TIn>(), 1) bwd_prep_kernel(con
       __syncthreads();
       for (int e = tid; e < rows * D; e += PN) {
         const int s = e / D, c = e % D;
-        sBuf[s * LDP + c] = sK[s * D + c] * exp2f(sG[r0 * D + c] - sG[s * D + c]);
+        sBuf[s * LDP + c] = sK[s * LK + c] * exp2f(sG[r0 * LK + c] - sG[s * LK + c]);
       }
       for (int e = tid; e < 16 * D; e += PN) {
         const int t = e / D, c = e % D;
-        const float f = exp2f(sG[(r0 + t) * D + c] - sG[r0 * D + c]);
-        sKL[t * LDP + c] = sK[(r0 + t) * D + c] * f;
-        sQL[t * LDP + c] = sQ[(r0 + t) * D + c] * f;
+        const float f = exp2f(sG[(r0 + t) * LK + c] - sG[r0 * LK + c]);
+        sKL[t * LDP + c] = sK[(r0 + t) * LK + c] * f;
+        sQL[t * LDP + c] = sQ[(r0 + t) * LK + c] * f;
       }
       __syncthreads();
       float a[4] = {0.f, 0.f, 0.f, 0.f}, pp[4] = {0.f, 0.f, 0.f, 0.f};
@@ -456,8 +460,8 @@ __global__ void __launch_bounds__(prep_threads<D, TIn>(), 1) bwd_prep_kernel(con
 #pragma unroll
       for (int jj = 0; jj < 4; ++jj) {
         const int s = tx + 16 * jj;
-        sA[t * C + s] = s < t ? a[jj] : 0.f;
-        sP[t * C + s] = s <= t ? pp[jj] : 0.f;
+        sA[t * LA + s] = s < t ? a[jj] : 0.f;
+        sP[t * LA + s] = s <= t ? pp[jj] : 0.f;
       }
     }
     __syncthreads();
@@ -475,7 +479,7 @@ __global__ void __launch_bounds__(prep_threads<D, TIn>(), 1) bwd_prep_kernel(con
     if (tid < NTH)
       for (int i = o; i < o + 16; ++i) {
         float acc = 0.f;
-        for (int s = j + part; s < i; s += 4) acc = fmaf(sA[i * C + s], sT[s * C + j], acc);
+        for (int s = j + part; s < i; s += 4) acc = fmaf(sA[i * LA + s], sT[s * C + j], acc);
         acc += __shfl_xor_sync(0xffffffffu, acc, 1);
         acc += __shfl_xor_sync(0xffffffffu, acc, 2);
         if (part == 0) sT[i * C + j] = i < j ? 0.f : (i == j ? 1.f : -sB[i] * acc);
@@ -489,7 +493,7 @@ __global__ void __launch_bounds__(prep_threads<D, TIn>(), 1) bwd_prep_kernel(con
       for (int a = d; a < 4 && tid < NTH; ++a) {
         const int bb = a - d, i = 16 * a + ty, jc = 16 * bb + tx;
         float y = 0.f;
-        for (int s2 = 16 * bb; s2 < 16 * a; ++s2) y = fmaf(sA[i * C + s2], sT[s2 * C + jc], y);
+        for (int s2 = 16 * bb; s2 < 16 * a; ++s2) y = fmaf(sA[i * LA + s2], sT[s2 * C + jc], y);
         Ys[(bb * 16 + ty) * 17 + tx] = sB[i] * y;
       }
       __syncthreads();
@@ -524,7 +528,7 @@ __global__ void __launch_bounds__(prep_threads<D, TIn>(), 1) bwd_prep_kernel(con
 #pragma unroll
       for (int jj = 0; jj < 16; ++jj) {
         const int j = j0 + jj;
-        v1[jj] = tf32_round(sB[j] * exp2f(sG[j * D + c]) * sK[j * D + c]);
+        v1[jj] = tf32_round(sB[j] * exp2f(sG[j * LK + c]) * sK[j * LK + c]);
         v2[jj] = tf32_round(sB[j] * sBuf[j * LDP + c]);
       }
       tmem_st16(tm + lane + TA1 + j0, v1);
@@ -549,12 +553,12 @@ __global__ void __launch_bounds__(prep_threads<D, TIn>(), 1) bwd_prep_kernel(con
     for (int e = tid; e < C * C; e += PN) {
       const int a = e >> 6, b = e & 63;
       *reinterpret_cast<float *>(bT + sw128_offset(C, a, b)) = tf32_round(sT[a * C + b]);
-      *reinterpret_cast<float *>(bP + sw128_offset(C, b, a)) = tf32_round(sP[a * C + b]);
+      *reinterpret_cast<float *>(bP + sw128_offset(C, b, a)) = tf32_round(sP[a * LA + b]);
     }
     for (int e = tid; e < D * C; e += PN) {
       const int j = e / D, nn = e % D;
       *reinterpret_cast<float *>(bQ + sw128_offset(D, nn, j)) =
-          tf32_round(exp2f(sG[j * D + nn]) * sQ[j * D + nn]);
+          tf32_round(exp2f(sG[j * LK + nn]) * sQ[j * LK + nn]);
     }
     fence_async_smem();
     tc_fence_before();
@@ -609,7 +613,7 @@ __global__ void __launch_bounds__(prep_threads<D, TIn>(), 1) bwd_prep_kernel(con
     // W = T Diag(beta) (gamma K)
     for (int e = tid; e < C * D; e += PN) {
       const int t = e / D, c = e % D;
-      sBuf[t * LDP + c] = sB[t] * exp2f(sG[t * D + c]) * sK[t * D + c];
+      sBuf[t * LDP + c] = sB[t] * exp2f(sG[t * LK + c]) * sK[t * LK + c];
     }
     zero(acc);
     mm_acc<4, NJ>(acc, sT, C, 1, sBuf, LDP, 1, C, sStage);
@@ -630,17 +634,20 @@ __global__ void __launch_bounds__(prep_threads<D, TIn>(), 1) bwd_prep_kernel(con
     // X = P^T dO
     stage_rows<D, float>(sBuf, LDP, p.d_o, tok0, n, H, h);
     zero(acc);
-    mm_acc<4, NJ>(acc, sP, 1, C, sBuf, LDP, 1, C, sStage);
+    mm_acc<4, NJ>(acc, sP, 1, LA, sBuf, LDP, 1, C, sStage);
   #pragma unroll
     for (int i = 0; i < 4; ++i)
   #pragma unroll
       for (int j = 0; j < NJ; ++j) p.wX[ch * C * D + (ty + 16 * i) * D + tx + 16 * j] = acc[i][j];
     // Y = (gamma Q)^T dO
-    for (int e = tid; e < C * D; e += PN) sQ[e] *= exp2f(sG[e]);
+    for (int e = tid; e < C * D; e += PN) {
+      const int at = (e / D) * LK + e % D;
+      sQ[at] *= exp2f(sG[at]);
+    }
     {
       float y[NJ][NJ];
       zero(y);
-      mm_acc<NJ, NJ>(y, sQ, 1, D, sBuf, LDP, 1, C, sStage);
+      mm_acc<NJ, NJ>(y, sQ, 1, LK, sBuf, LDP, 1, C, sStage);
   #pragma unroll
       for (int i = 0; i < NJ; ++i)
   #pragma unroll
@@ -651,13 +658,13 @@ __global__ void __launch_bounds__(prep_threads<D, TIn>(), 1) bwd_prep_kernel(con
   // Khat = exp(G_last - G) K, Gam = exp(G_last); A and T for the gradient pass
   for (int e = tid; e < C * D; e += PN) {
     const int t = e / D, c = e % D;
-    const float kh = sK[e] * exp2f(sG[(C - 1) * D + c] - sG[t * D + c]);
+    const float kh = sK[t * LK + c] * exp2f(sG[(C - 1) * LK + c] - sG[t * LK + c]);
     // the tensor-core state pass reads Khat as a tf32 operand, copied as it is
     p.wKh[ch * C * D + e] = kPrepTensorCores<D, TIn> ? tf32_round(kh) : kh;
   }
-  if (tid < D) p.wGam[ch * D + tid] = exp2f(sG[(C - 1) * D + tid]);
+  if (tid < D) p.wGam[ch * D + tid] = exp2f(sG[(C - 1) * LK + tid]);
   for (int e = tid; e < C * C; e += PN) {
-    p.wA[ch * C * C + e] = sA[e];
+    p.wA[ch * C * C + e] = sA[(e / C) * LA + e % C];
     p.wT[ch * C * C + e] = sT[e];
   }
 }
