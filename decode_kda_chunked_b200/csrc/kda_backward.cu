@@ -209,8 +209,15 @@ __device__ void stage_rows(float *dst, int ld, const TIn *src, int tok0, int n, 
     const int e = threadIdx.x + it * NT, t = e / PER_ROW, cv = e % PER_ROW;
     float x[VEC];
     unpack16(buf[it], src, x);
+    if ((ld & 3) == 0) {  // 16-byte aligned rows: vector stores
 #pragma unroll
-    for (int q = 0; q < VEC; ++q) dst[t * ld + cv * VEC + q] = x[q];
+      for (int q = 0; q < VEC / 4; ++q)
+        *reinterpret_cast<float4 *>(dst + t * ld + cv * VEC + 4 * q) =
+            make_float4(x[4 * q], x[4 * q + 1], x[4 * q + 2], x[4 * q + 3]);
+    } else {
+#pragma unroll
+      for (int q = 0; q < VEC; ++q) dst[t * ld + cv * VEC + q] = x[q];
+    }
   }
 }
 
@@ -1633,9 +1640,22 @@ __global__ void __launch_bounds__(grad_threads<D, TIn>(), 1) bwd_grad_kernel(con
   for (int b = 0; b < 4; ++b) {
     const int r0 = 16 * b, r1 = r0 + 15;
     __syncthreads();
-    for (int e = tid; e < (r0 + 16) * D; e += GN) {
-      const int c = e % D;
-      sO[e - c + gate_pos<TX, NJ>(c)] = sK[e] * exp2f(sG[r0 * D + c] - sG[e]);
+    if constexpr (NJ == 4) {  // one float4 chunk x (columns x + TX q) per step
+      for (int e = tid; e < (r0 + 16) * TX; e += GN) {
+        const int t = e / TX, x = e % TX;
+        float v[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int c = x + TX * q;
+          v[q] = sK[t * D + c] * exp2f(sG[r0 * D + c] - sG[t * D + c]);
+        }
+        *reinterpret_cast<float4 *>(sO + t * D + 4 * x) = make_float4(v[0], v[1], v[2], v[3]);
+      }
+    } else {
+      for (int e = tid; e < (r0 + 16) * D; e += GN) {
+        const int c = e % D;
+        sO[e - c + gate_pos<TX, NJ>(c)] = sK[e] * exp2f(sG[r0 * D + c] - sG[e]);
+      }
     }
     __syncthreads();
     {
@@ -1668,11 +1688,27 @@ __global__ void __launch_bounds__(grad_threads<D, TIn>(), 1) bwd_grad_kernel(con
       }
     }
     __syncthreads();
-    for (int e = r0 * D + tid; e < C * D; e += GN) {
-      const int c = e % D, at = e - c + gate_pos<TX, NJ>(c);
-      const float f = exp2f(sG[e] - sG[r1 * D + c]);
-      sO[at] = sQ[e] * f;
-      sV[at] = sK[e] * f;
+    if constexpr (NJ == 4) {
+      for (int e = r0 * TX + tid; e < C * TX; e += GN) {
+        const int t = e / TX, x = e % TX;
+        float qv[4], kv[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int c = x + TX * q;
+          const float f = exp2f(sG[t * D + c] - sG[r1 * D + c]);
+          qv[q] = sQ[t * D + c] * f;
+          kv[q] = sK[t * D + c] * f;
+        }
+        *reinterpret_cast<float4 *>(sO + t * D + 4 * x) = make_float4(qv[0], qv[1], qv[2], qv[3]);
+        *reinterpret_cast<float4 *>(sV + t * D + 4 * x) = make_float4(kv[0], kv[1], kv[2], kv[3]);
+      }
+    } else {
+      for (int e = r0 * D + tid; e < C * D; e += GN) {
+        const int c = e % D, at = e - c + gate_pos<TX, NJ>(c);
+        const float f = exp2f(sG[e] - sG[r1 * D + c]);
+        sO[at] = sQ[e] * f;
+        sV[at] = sK[e] * f;
+      }
     }
     __syncthreads();
     {
