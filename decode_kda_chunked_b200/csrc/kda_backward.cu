@@ -1560,7 +1560,7 @@ __global__ void __launch_bounds__(grad_threads<D, TIn>(), 1) bwd_grad_kernel(con
     for (int j = 0; j < NJ; ++j) {
       const int c = tx + TX * j;
       rs = fmaf(acc[i][j], sV[t * D + c], rs);
-      sV[t * D + c] = acc[i][j];  // the V tile now holds T^T dU (own elements only)
+      if constexpr (!PRE) sV[t * D + c] = acc[i][j];  // T^T dU for dZ (own elements only)
       if (t < n) p.dv[((size_t)(tok0 + t) * H + h) * D + c] = sB[t] * acc[i][j];
     }
     rs = row_sum<TX>(rs);
@@ -1581,12 +1581,12 @@ __global__ void __launch_bounds__(grad_threads<D, TIn>(), 1) bwd_grad_kernel(con
 #pragma unroll
     for (int j = 0; j < NJ; ++j) {
       const int e = t * D + tx + TX * j;
-      const float kg = exp2f(sG[e]) * sK[e];
+      const float gm = exp2f(sG[e]), kg = gm * sK[e];
       const float dkg = sB[t] * acc[i][j];
-      accK[i][j] = fmaf(dkg, exp2f(sG[e]), accK[i][j]);
+      accK[i][j] = fmaf(dkg, gm, accK[i][j]);
       accG[i][j] = fmaf(dkg, kg, accG[i][j]);
       rs = fmaf(acc[i][j], kg, rs);
-      sO[e] = acc[i][j];  // the dO tile (dW) now holds T^T dW (own elements only)
+      if constexpr (!PRE) sO[e] = acc[i][j];  // T^T dW for dZ (own elements only)
     }
     rs = row_sum<TX>(rs);
     if (tx == 0) sDb[t] += rs;
