@@ -317,6 +317,9 @@ __device__ __forceinline__ float tf32_round(float x) {
   asm("cvt.rn.tf32.f32 %0, %1;" : "=r"(r) : "f"(x));
   return __uint_as_float(r);
 }
+__device__ __forceinline__ float4 tf32_round4(float4 x) {
+  return make_float4(tf32_round(x.x), tf32_round(x.y), tf32_round(x.z), tf32_round(x.w));
+}
 
 template <int D, typename TIn>
 __global__ void __launch_bounds__(prep_threads<D, TIn>(), 1) bwd_prep_kernel(const BwdParams p) {
@@ -383,8 +386,9 @@ __global__ void __launch_bounds__(prep_threads<D, TIn>(), 1) bwd_prep_kernel(con
 #pragma unroll
     for (int b = 0; b < 2; ++b) {
       const int rows = 32 * (b + 1), mb = 32 * b + 15;
+      // consecutive threads take consecutive rows j (distinct banks on both sides)
       for (int e = tid; e < rows * (D / 4); e += PN) {
-        const int j = e / (D / 4), c = (e % (D / 4)) * 4;
+        const int j = e % rows, c = (e / rows) * 4;
         float4 r;
         r.x = tf32_round(sK[j * LK + c] * exp2f(sG[mb * LK + c] - sG[j * LK + c]));
         r.y = tf32_round(sK[j * LK + c + 1] * exp2f(sG[mb * LK + c + 1] - sG[j * LK + c + 1]));
@@ -556,16 +560,28 @@ __global__ void __launch_bounds__(prep_threads<D, TIn>(), 1) bwd_prep_kernel(con
     unsigned char *bP = bT + 64 * 64 * 4;
     unsigned char *bQ = reinterpret_cast<unsigned char *>(
         (reinterpret_cast<uintptr_t>(sKL) + 1023) & ~uintptr_t(1023));
-    // consecutive threads walk each source's contiguous axis (conflict-free reads)
-    for (int e = tid; e < C * C; e += PN) {
-      const int a = e >> 6, b = e & 63;
-      *reinterpret_cast<float *>(bT + sw128_offset(C, a, b)) = tf32_round(sT[a * C + b]);
-      *reinterpret_cast<float *>(bP + sw128_offset(C, b, a)) = tf32_round(sP[a * LA + b]);
+    // each thread writes one 16-byte chunk (four K values of one operand row); consecutive
+    // threads take consecutive rows, so both the source reads and the swizzled stores
+    // fall on distinct banks
+    for (int e = tid; e < C * C / 4; e += PN) {
+      // T (row a, K = b) straight from its rows: a warp's quarter reads and writes one
+      // row's 128 bytes
+      const int a = e >> 4, b0 = (e & 15) * 4;
+      *reinterpret_cast<float4 *>(bT + sw128_chunk(C, a, b0)) =
+          tf32_round4(*reinterpret_cast<const float4 *>(sT + a * C + b0));
+      // P^T (row b = r, K = a)
+      const int r = e & 63, k0 = (e >> 6) * 4;
+      *reinterpret_cast<float4 *>(bP + sw128_chunk(C, r, k0)) = tf32_round4(
+          make_float4(sP[k0 * LA + r], sP[(k0 + 1) * LA + r], sP[(k0 + 2) * LA + r],
+                      sP[(k0 + 3) * LA + r]));
     }
-    for (int e = tid; e < D * C; e += PN) {
-      const int j = e / D, nn = e % D;
-      *reinterpret_cast<float *>(bQ + sw128_offset(D, nn, j)) =
-          tf32_round(exp2f(sG[j * LK + nn]) * sQ[j * LK + nn]);
+    for (int e = tid; e < D * C / 4; e += PN) {  // (gamma Q)^T: row nn = channel, K = token
+      const int nn = e % D, j0 = (e / D) * 4;
+      float x[4];
+#pragma unroll
+      for (int u = 0; u < 4; ++u) x[u] = exp2f(sG[(j0 + u) * LK + nn]) * sQ[(j0 + u) * LK + nn];
+      *reinterpret_cast<float4 *>(bQ + sw128_chunk(D, nn, j0)) =
+          tf32_round4(make_float4(x[0], x[1], x[2], x[3]));
     }
     fence_async_smem();
     tc_fence_before();
@@ -1072,9 +1088,6 @@ struct SprodLayout {
   static constexpr size_t bytes = oMisc + 48 + 1024;
 };
 
-__device__ __forceinline__ float4 tf32_round4(float4 x) {
-  return make_float4(tf32_round(x.x), tf32_round(x.y), tf32_round(x.z), tf32_round(x.w));
-}
 
 __global__ void __launch_bounds__(SP_NTH, 1) bwd_sprod_kernel(const BwdParams p) {
   using L = SprodLayout;
