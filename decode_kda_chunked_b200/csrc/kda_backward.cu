@@ -1262,9 +1262,9 @@ __global__ void __launch_bounds__(SP_NTH, 1) bwd_sprod_kernel(const BwdParams p)
     tmem_ld16(tm + lane + TDW + 16 * part, v);  // dW^T: rows 128 + key of [dU^T ; dW^T]
     tmem_wait_ld();
 #pragma unroll
-    for (int tt = 0; tt < 16; ++tt)
-      *reinterpret_cast<float *>(bDUW + sw128_offset(2 * D, D + lrow, 16 * part + tt)) =
-          tf32_round(v[tt]);
+    for (int q = 0; q < 4; ++q)  // 16-byte chunks; consecutive lanes on consecutive rows
+      *reinterpret_cast<float4 *>(bDUW + sw128_chunk(2 * D, D + lrow, 16 * part + 4 * q)) =
+          tf32_round4(make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]));
   }
   // stage 2: A operands on lanes t = 32 (w % 4) + lane for lane quarters 0 and 1; part
   // w / 4 takes a quarter of the columns
