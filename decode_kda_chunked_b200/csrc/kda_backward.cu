@@ -29,19 +29,20 @@
 //
 // Launches: the forward kernel with a snapshot every 64 tokens (the chunk
 // start states), then
-//   bwd_prep  (CTA per chunk and head): A, T, W, U~, Khat, Gam, X = P^T dO, Y = (gamma Q)^T dO
-//   bwd_state (CTA per request, head and 16 state columns): the serial pass;
-//             dU overwrites X, dSn overwrites Y
-//   bwd_sprod (CTA per chunk and head; bf16 inputs at d = 128): U, d(gamma Q),
-//             dKhat, dW and dGam, the products with the state, on the tensor cores
-//   bwd_grad  (CTA per chunk and head): every token gradient of the chunk
-// The state and gradient passes are fp32 on the CUDA cores: a CTA's 256 threads
-// form a 16 x 16 grid, and thread (ty, tx) owns rows ty + 16 i and columns
-// tx + 16 j of every tile it produces, so per-element folds stay in registers.
-// For bf16 inputs at d = 128 the prep pass forms A and P and runs its four
-// products as tcgen05 tf32 MMAs (transposed to M = 128 TMEM lanes, as in the
-// forward), and so does bwd_sprod with the four products of the state; fp32
-// inputs keep fp32 products throughout.
+//   bwd_prep   (CTA per chunk and head): A, T, W, U~, Khat, Gam, X = P^T dO, Y = (gamma Q)^T dO
+//   bwd_state  the serial pass; dU overwrites X, dSn overwrites Y.  bwd_state_tc (CTA
+//              per request and head; bf16 inputs at d = 128) on the tensor cores with
+//              dS^T in TMEM, else bwd_state (CTA per request, head and 32 state columns)
+//   bwd_sprod  (CTA per chunk and head; bf16 inputs at d = 128): on the tensor cores,
+//              U, d(gamma Q), dKhat, dW and dGam (the products with the state), then
+//              dP, T^T dU, T^T dW and dZ (the products of chunk-sized tiles)
+//   bwd_grad   (CTA per chunk and head): every token gradient of the chunk
+// For bf16 inputs at d = 128 every dense product runs as tcgen05 tf32 MMAs (transposed
+// to M = 128 TMEM lanes, as in the forward) and bwd_grad keeps the gated Gram
+// cotangents and the per-element folds; fp32 inputs keep fp32 products on the CUDA
+// cores throughout.  The CUDA-core passes give thread (ty, tx) of a 16 x TX grid rows
+// ty + 16 i and columns tx + TX j of every tile it produces, so per-element folds stay
+// in registers.
 #include "kda_internal.cuh"
 #include "kda_sm100.cuh"
 
