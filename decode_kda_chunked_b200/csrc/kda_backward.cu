@@ -74,7 +74,8 @@ struct BwdParams {
   const float *snaps;          // [n_snap, H, D, D]
   const float *zero_state;     // D x D zeros
   float *wA, *wT, *wW, *wU, *wKh, *wX, *wY, *wGam;
-  float *wU2;                  // U = U~ - W S per (chunk, head), written by the gradient pass
+  float *wU2;                  // per (chunk, head): U = U~ - W S from the gradient pass (fp32
+                               // inputs), or dZ from bwd_sprod (bf16 inputs at d = 128)
   int n_req, n_chunks, H;
   unsigned int *status;        // device status word (a bounded wait that gave up)
 };
