@@ -139,10 +139,13 @@ struct SplitPlan {
   int n_seg = 0;                    // segments over all requests; 0: no split
   std::vector<int32_t> seg_cu;      // [n_seg + 1] token bounds of the segments
   std::vector<int32_t> first_seg;   // [n_req + 1] first segment of each request
-  std::vector<int32_t> pass1;       // the non-final segments of split requests
+  std::vector<int32_t> pass1;       // local states: middle segments of split requests
+  std::vector<int32_t> first;       // first segments of split requests (prefilled in pass 1)
+  std::vector<int32_t> pass2;       // the other segments (and unsplit requests)
   std::vector<int32_t> seg_snap;    // [n_seg + 1] snapshot rows before each segment
   // workspace layout (byte offsets, 256-aligned)
-  size_t off_cu = 0, off_p1 = 0, off_snap = 0, off_sloc = 0, off_m = 0, off_sin = 0, bytes = 0;
+  size_t off_cu = 0, off_p1 = 0, off_first = 0, off_p2 = 0, off_snap = 0, off_sloc = 0, off_m = 0,
+         off_sin = 0, bytes = 0;
 };
 
 // SMs of the current device.  KDA_TEST_SM_COUNT overrides it, so that host tests
@@ -164,14 +167,14 @@ int device_sm_count() {
 //   - the chains fill at most half of the SMs;
 //   - every segment holds at least 1,024 tokens and starts on a multiple of 32 (of
 //     the snapshot stride when snapshots are taken), so that snapshots tile it;
-//   - the local-state pass (one CTA per non-final segment and head) and the segment
-//     prefill (one CTA per segment and head) each fit in one wave;
+//   - each pass fits in one wave: pass 1 runs, per head, the first segment of every
+//     split request (a prefill from the request's initial state) beside the local
+//     states of its middle segments; pass 2 runs every other segment;
 //   - the estimated time, in tokens of one chain, drops by 15 % or more: the longest
-//     non-final segment at 0.9 (the local-state pass skips q, P and O but keeps the
-//     gate, the row operands and the solve, and adds the transition's columns:
-//     measured 4.25 against 4.7 us per chunk),
-//     plus the longest segment, plus 256 for the extra launches and the combine,
-//     against the longest request unsplit.  (So a two-way split never pays.)
+//     first segment (it bounds pass 1: a middle segment's local state costs 0.9 of
+//     a prefill chunk, measured 4.25 against 4.7 us per chunk), plus the longest
+//     pass-2 segment, plus 256 for the extra launches and the combine, against the
+//     longest request unsplit.  (So a two-way split never pays.)
 // Extra segments go, one at a time, to the request whose longest segment is longest.
 bool plan_split(const kda_prefill_args *a, SplitPlan *pl) {
   if (!a->cu_seqlens_host || a->n_req <= 0 || a->total_tokens <= 0) return false;
@@ -203,13 +206,18 @@ bool plan_split(const kda_prefill_args *a, SplitPlan *pl) {
     }
     return 0;
   };
-  int total = a->n_req, extra = 0;
+  // segments per head in each pass: pass 1 = sum over split requests of parts - 1
+  // (the first segment and the middle ones), pass 2 = every segment but the first
+  // segments of split requests
+  int total = a->n_req, extra = 0, pass2 = a->n_req;
+  auto in_pass2 = [](int n_parts) { return n_parts > 1 ? n_parts - 1 : 1; };
   for (;;) {
     int best = -1, best_parts = 0;
     long best_len = 0;
     for (int r = 0; r < a->n_req; ++r) {
       const int s = next_parts(r);
-      if (s == 0 || total + (s - parts[r]) > max_total || extra + (s - parts[r]) > max_extra)
+      if (s == 0 || pass2 + in_pass2(s) - in_pass2(parts[r]) > max_total ||
+          extra + (s - parts[r]) > max_extra)
         continue;
       const long len = cu[r + 1] - cu[r];
       const long longest = parts[r] == 1 ? len : piece(r, parts[r]);
@@ -222,24 +230,27 @@ bool plan_split(const kda_prefill_args *a, SplitPlan *pl) {
     if (best < 0) break;
     total += best_parts - parts[best];
     extra += best_parts - parts[best];
+    pass2 += in_pass2(best_parts) - in_pass2(parts[best]);
     parts[best] = best_parts;
   }
   if (extra == 0) return false;
-  long longest = 0, longest_seg = 0, longest_nonfinal = 0;
+  long longest = 0, longest_p1 = 0, longest_p2 = 0;
   for (int r = 0; r < a->n_req; ++r) {
     const long len = cu[r + 1] - cu[r];
     longest = len > longest ? len : longest;
     const long p = parts[r] > 1 ? piece(r, parts[r]) : len;
     const long last = len - (parts[r] - 1) * p;
-    longest_seg = std::max(longest_seg, std::max(parts[r] > 1 ? p : 0L, last));
-    if (parts[r] > 1) longest_nonfinal = std::max(longest_nonfinal, p);
+    if (parts[r] > 1) longest_p1 = std::max(longest_p1, p);
+    longest_p2 = std::max(longest_p2, std::max(parts[r] > 2 ? p : 0L, last));
   }
-  if (0.9 * longest_nonfinal + longest_seg + 256.0 > 0.85 * longest) return false;
+  if ((double)longest_p1 + longest_p2 + 256.0 > 0.85 * longest) return false;
 
   pl->n_seg = total;
   pl->seg_cu.assign(1, 0);
   pl->first_seg.assign(1, 0);
   pl->pass1.clear();
+  pl->first.clear();
+  pl->pass2.clear();
   pl->seg_snap.assign(1, 0);
   int32_t snaps_before = 0;
   for (int r = 0; r < a->n_req; ++r) {
@@ -247,7 +258,12 @@ bool plan_split(const kda_prefill_args *a, SplitPlan *pl) {
     const long p = parts[r] > 1 ? piece(r, parts[r]) : (long)(eos - bos);
     for (int k = 0; k < parts[r]; ++k) {
       const int32_t end = k + 1 < parts[r] ? bos + (int32_t)((k + 1) * p) : eos;
-      if (k + 1 < parts[r]) pl->pass1.push_back((int32_t)pl->seg_cu.size() - 1);
+      const int32_t seg = (int32_t)pl->seg_cu.size() - 1;
+      if (parts[r] > 1 && k == 0)
+        pl->first.push_back(seg);
+      else
+        pl->pass2.push_back(seg);
+      if (k > 0 && k + 1 < parts[r]) pl->pass1.push_back(seg);
       pl->seg_cu.push_back(end);
       if (a->snapshot_stride > 0)
         pl->seg_snap.push_back(snaps_before + (end - bos) / a->snapshot_stride);
@@ -264,6 +280,8 @@ bool plan_split(const kda_prefill_args *a, SplitPlan *pl) {
   };
   pl->off_cu = take((n + 1) * sizeof(int32_t));
   pl->off_p1 = take(pl->pass1.size() * sizeof(int32_t));
+  pl->off_first = take(pl->first.size() * sizeof(int32_t));
+  pl->off_p2 = take(pl->pass2.size() * sizeof(int32_t));
   pl->off_snap = take((n + 1) * sizeof(int32_t));
   pl->off_sloc = take(n * state);
   pl->off_m = take(n * (size_t)a->H * a->dk * a->dk * sizeof(float));
@@ -279,11 +297,38 @@ kda_status from_cuda(cudaError_t e) {
   return KDA_ERR_CUDA;
 }
 
-// The split call (see plan_split): local states, combine, segment prefill, final states.
+CUcontext current_context();
+
+// A second stream of the current context, created once and kept: the split call runs
+// the first segments' prefill on it beside the local-state pass.  Calls that share it
+// stay correct (each joins through its own events); they only queue behind each other.
+cudaStream_t side_stream() {
+  static std::mutex mu;
+  static std::vector<std::pair<CUcontext, cudaStream_t>> streams;
+  const CUcontext ctx = current_context();
+  if (!ctx) return nullptr;
+  std::lock_guard<std::mutex> lock(mu);
+  for (const auto &e : streams)
+    if (e.first == ctx) return e.second;
+  cudaStream_t st = nullptr;
+  if (cudaStreamCreateWithFlags(&st, cudaStreamNonBlocking) != cudaSuccess) return nullptr;
+  streams.emplace_back(ctx, st);
+  return st;
+}
+
+// The split call (see plan_split), in two passes:
+//   1. on a second stream, the first segment of every split request from the request's
+//      initial state (o, snapshots; its final state into that segment's S_loc slot),
+//      and on the call's stream the local states and transitions of the middle
+//      segments;
+//   2. after both, the combine per split request from the first segment's final state,
+//      then every other segment from its start state; the final states are copied out.
 kda_status run_split(const kda_prefill_args *a, const SplitPlan &pl, char *ws,
                      const PrefillParams &base, cudaStream_t s) {
   int32_t *seg_cu = reinterpret_cast<int32_t *>(ws + pl.off_cu);
   int32_t *p1 = reinterpret_cast<int32_t *>(ws + pl.off_p1);
+  int32_t *first = reinterpret_cast<int32_t *>(ws + pl.off_first);
+  int32_t *p2 = reinterpret_cast<int32_t *>(ws + pl.off_p2);
   int32_t *seg_snap = reinterpret_cast<int32_t *>(ws + pl.off_snap);
   float *sloc = reinterpret_cast<float *>(ws + pl.off_sloc);
   float *m = reinterpret_cast<float *>(ws + pl.off_m);
@@ -291,52 +336,86 @@ kda_status run_split(const kda_prefill_args *a, const SplitPlan &pl, char *ws,
   const size_t state = (size_t)a->H * a->dk * a->dv, trans = (size_t)a->H * a->dk * a->dk;
   // the plan's small tables (pageable host memory: each copy has left the host
   // buffer when it returns)
-  cudaError_t e = cudaMemcpyAsync(seg_cu, pl.seg_cu.data(), pl.seg_cu.size() * sizeof(int32_t),
-                                  cudaMemcpyHostToDevice, s);
-  if (e == cudaSuccess)
-    e = cudaMemcpyAsync(p1, pl.pass1.data(), pl.pass1.size() * sizeof(int32_t),
-                        cudaMemcpyHostToDevice, s);
-  if (e == cudaSuccess && a->snapshot_stride > 0)
-    e = cudaMemcpyAsync(seg_snap, pl.seg_snap.data(), pl.seg_snap.size() * sizeof(int32_t),
-                        cudaMemcpyHostToDevice, s);
+  cudaError_t e = cudaSuccess;
+  auto put = [&](int32_t *dst, const std::vector<int32_t> &v) {
+    if (e == cudaSuccess && !v.empty())
+      e = cudaMemcpyAsync(dst, v.data(), v.size() * sizeof(int32_t), cudaMemcpyHostToDevice, s);
+  };
+  put(seg_cu, pl.seg_cu);
+  put(p1, pl.pass1);
+  put(first, pl.first);
+  put(p2, pl.pass2);
+  if (a->snapshot_stride > 0) put(seg_snap, pl.seg_snap);
+  // every request's first segment starts from its initial state
+  for (int r = 0; r < a->n_req && e == cudaSuccess; ++r) {
+    const int row0 = pl.first_seg[r];
+    const float *s_init = a->initial_state ? a->initial_state + (size_t)r * state : nullptr;
+    e = s_init ? cudaMemcpyAsync(s_start + row0 * state, s_init, state * sizeof(float),
+                                 cudaMemcpyDeviceToDevice, s)
+               : cudaMemsetAsync(s_start + row0 * state, 0, state * sizeof(float), s);
+  }
   if (e != cudaSuccess) return from_cuda(e);
 
-  // local states and transitions of the non-final segments
-  PrefillParams lp = base;
-  lp.q = nullptr;
-  lp.o = nullptr;
-  lp.initial_state = nullptr;
-  lp.final_state = nullptr;
-  lp.snapshot_stride = 0;
-  lp.cu_snapshots = nullptr;
-  lp.snapshots = nullptr;
-  lp.cu_seqlens = seg_cu;
-  lp.n_req = (int)pl.pass1.size();
-  lp.order = p1;
-  lp.local_mode = 1;
-  lp.s_loc = sloc;
-  lp.m = m;
-  if ((e = launch_prefill_tc(lp, a->in_dtype, KDA_F32, s)) != cudaSuccess) return from_cuda(e);
+  // pass 1: the first segments on the second stream, forked from and joined to s
+  const cudaStream_t side = side_stream();
+  if (!side) return KDA_ERR_CUDA;
+  cudaEvent_t fork = nullptr, join = nullptr;
+  if ((e = cudaEventCreateWithFlags(&fork, cudaEventDisableTiming)) != cudaSuccess)
+    return from_cuda(e);
+  if ((e = cudaEventCreateWithFlags(&join, cudaEventDisableTiming)) != cudaSuccess) {
+    cudaEventDestroy(fork);
+    return from_cuda(e);
+  }
+  PrefillParams fp = base;
+  fp.cu_seqlens = seg_cu;
+  fp.n_req = (int)pl.first.size();
+  fp.order = first;
+  fp.initial_state = s_start;
+  fp.final_state = sloc;  // the first segment has no local state of its own
+  fp.cu_snapshots = a->snapshot_stride > 0 ? seg_snap : nullptr;
+  e = cudaEventRecord(fork, s);
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(side, fork, 0);
+  if (e == cudaSuccess) e = launch_prefill_tc(fp, a->in_dtype, a->out_dtype, side);
+  if (e == cudaSuccess) e = cudaEventRecord(join, side);
+  if (e == cudaSuccess) {
+    // local states and transitions of the middle segments
+    PrefillParams lp = base;
+    lp.q = nullptr;
+    lp.o = nullptr;
+    lp.initial_state = nullptr;
+    lp.final_state = nullptr;
+    lp.snapshot_stride = 0;
+    lp.cu_snapshots = nullptr;
+    lp.snapshots = nullptr;
+    lp.cu_seqlens = seg_cu;
+    lp.n_req = (int)pl.pass1.size();
+    lp.order = p1;
+    lp.local_mode = 1;
+    lp.s_loc = sloc;
+    lp.m = m;
+    e = launch_prefill_tc(lp, a->in_dtype, KDA_F32, s);
+  }
+  if (e == cudaSuccess) e = cudaStreamWaitEvent(s, join, 0);
+  cudaEventDestroy(fork);  // released once recorded work completes
+  cudaEventDestroy(join);
+  if (e != cudaSuccess) return from_cuda(e);
 
-  // start states of every segment: the request's initial state, then the combine
+  // start states of the other segments of split requests: S_in[1] is the first
+  // segment's final state, then S_in[k + 1] = M_k S_in[k] + S_loc_k
   for (int r = 0; r < a->n_req; ++r) {
     const int row0 = pl.first_seg[r], n = pl.first_seg[r + 1] - row0;
-    const float *s_init = a->initial_state ? a->initial_state + (size_t)r * state : nullptr;
-    if (n == 1)
-      e = s_init ? cudaMemcpyAsync(s_start + row0 * state, s_init, state * sizeof(float),
-                                   cudaMemcpyDeviceToDevice, s)
-                 : cudaMemsetAsync(s_start + row0 * state, 0, state * sizeof(float), s);
-    else
-      e = launch_combine(sloc + row0 * state, m + row0 * trans, s_init, n - 1, a->H, a->dk,
-                         a->dv, s_start + row0 * state, s_start + (row0 + n - 1) * state, s);
+    if (n == 1) continue;
+    e = launch_combine(sloc + (row0 + 1) * state, m + (row0 + 1) * trans, sloc + row0 * state,
+                       n - 2, a->H, a->dk, a->dv, s_start + (row0 + 1) * state,
+                       s_start + (row0 + n - 1) * state, s);
     if (e != cudaSuccess) return from_cuda(e);
   }
 
-  // every segment from its start state; the final states land in place
+  // pass 2: every other segment from its start state; the final states land in place
   PrefillParams sp = base;
   sp.cu_seqlens = seg_cu;
-  sp.n_req = pl.n_seg;
-  sp.order = nullptr;
+  sp.n_req = (int)pl.pass2.size();
+  sp.order = p2;
   sp.initial_state = s_start;
   sp.final_state = s_start;
   sp.cu_snapshots = a->snapshot_stride > 0 ? seg_snap : nullptr;

@@ -39,12 +39,13 @@ def _segments(monkeypatch, lengths, H, stride=0, sms=148, dk=128):
 
 
 def test_single_sequence_fills_one_wave_per_pass(monkeypatch):
-    # 32 chains on 148 SMs: at most 148 // 32 = 4 segments per head, in the local-state
-    # pass (one CTA per non-final segment and head) and in the segment prefill
+    # 32 chains on 148 SMs: at most 148 // 32 = 4 segments per head in each pass.  Pass 1
+    # runs the first segment's prefill beside the local states of the three middle ones;
+    # pass 2 runs the other four segments: 5 segments of 1,664 tokens (the last 1,536)
     n, ws = _segments(monkeypatch, [8192], H=32)
-    assert n == 4
+    assert n == 5
     state = 32 * 128 * 128 * 4
-    assert ws >= 3 * 4 * state  # S_loc, M and start states of every segment
+    assert ws >= 3 * 5 * state  # S_loc, M and start states of every segment
 
 
 def test_split_switch_and_unsupported_calls(monkeypatch):
@@ -78,13 +79,16 @@ def test_few_heads_split_down_to_the_minimum_segment(monkeypatch):
 
 
 def test_longest_request_is_split_first(monkeypatch):
-    # 16 heads: up to 148 // 16 = 9 segments.  The 9,000-token request takes the first
-    # three extra ones (pieces 4,512, 3,008, 2,272), the 3,000-token one the next (1,504),
-    # then 9,000 again (1,824, 1,504), and at a tie the first request (3 x 1,024)
-    assert _segments(monkeypatch, [3000, 9000], H=16)[0] == 9
-    # 32 heads: 4 segments in all; two requests cut in two each would not pay
-    assert _segments(monkeypatch, [9000, 9000], H=32)[0] == 0
-    assert _segments(monkeypatch, [9000], H=32)[0] == 4
+    # 16 heads: up to 148 // 16 = 9 segments per head in each pass.  The 9,000-token
+    # request takes the first three extra segments (pieces 4,512, 3,008, 2,272), the
+    # 3,000-token one the next (1,504), then 9,000 again (1,824, 1,504), at a tie the
+    # first request (3 x 1,024), then 9,000 (1,312, 1,152): pass 1 holds 2 + 7 = 9
+    # segments per head, pass 2 the 2 + 7 others
+    assert _segments(monkeypatch, [3000, 9000], H=16)[0] == 11
+    # 32 heads: 4 segments per head in each pass; two requests in three segments each
+    # (first segments of 3,008 tokens in pass 1, the other four in pass 2)
+    assert _segments(monkeypatch, [9000, 9000], H=32)[0] == 6
+    assert _segments(monkeypatch, [9000], H=32)[0] == 5
     # too many chains for any split
     assert _segments(monkeypatch, [3000, 9000], H=64)[0] == 0
 
