@@ -162,9 +162,12 @@ size_t kda_prefill_workspace_size(const kda_prefill_args *args);
  * some request is long enough (segments of at least 1,024 tokens, starting on
  * multiples of 32 or of snapshot_stride), the call is split the way KDA
  * context parallelism splits a sequence ("Kimi K3 开源日来了", Infra section,
- * first layer): the local states and transitions of every non-final segment
- * (kda_chunk_local_state), an exact combine per request (kda_state_combine),
- * then every segment from its start state.  o, the snapshots and the final
+ * first layer): every split request's first segment from its initial state
+ * (on a second stream of the library's, forked from and joined to `stream`)
+ * beside the local states and transitions of the middle segments
+ * (kda_chunk_local_state), an exact combine per request (kda_state_combine)
+ * from the first segment's final state, then every other segment from its
+ * start state.  o, the snapshots and the final
  * states equal the unsplit call's up to rounding (not bit for bit); the call
  * then also makes small host-to-device copies of its segment tables from
  * pageable memory, which a CUDA graph capture does not accept.  The split is
