@@ -356,15 +356,19 @@ kda_status run_split(const kda_prefill_args *a, const SplitPlan &pl, char *ws,
   }
   if (e != cudaSuccess) return from_cuda(e);
 
-  // pass 1: the first segments on the second stream, forked from and joined to s
-  const cudaStream_t side = side_stream();
-  if (!side) return KDA_ERR_CUDA;
+  // pass 1: the first segments on the second stream, forked from and joined to s (on
+  // s itself, one kernel after the other, if no second stream can be had)
+  cudaStream_t side = side_stream();
   cudaEvent_t fork = nullptr, join = nullptr;
-  if ((e = cudaEventCreateWithFlags(&fork, cudaEventDisableTiming)) != cudaSuccess)
-    return from_cuda(e);
-  if ((e = cudaEventCreateWithFlags(&join, cudaEventDisableTiming)) != cudaSuccess) {
+  if (side && cudaEventCreateWithFlags(&fork, cudaEventDisableTiming) != cudaSuccess)
+    side = nullptr;
+  if (side && cudaEventCreateWithFlags(&join, cudaEventDisableTiming) != cudaSuccess) {
     cudaEventDestroy(fork);
-    return from_cuda(e);
+    side = nullptr;
+  }
+  if (!side) {
+    (void)cudaGetLastError();  // a failed event or stream creation is not the call's error
+    fork = join = nullptr;
   }
   PrefillParams fp = base;
   fp.cu_seqlens = seg_cu;
@@ -373,10 +377,14 @@ kda_status run_split(const kda_prefill_args *a, const SplitPlan &pl, char *ws,
   fp.initial_state = s_start;
   fp.final_state = sloc;  // the first segment has no local state of its own
   fp.cu_snapshots = a->snapshot_stride > 0 ? seg_snap : nullptr;
-  e = cudaEventRecord(fork, s);
-  if (e == cudaSuccess) e = cudaStreamWaitEvent(side, fork, 0);
-  if (e == cudaSuccess) e = launch_prefill_tc(fp, a->in_dtype, a->out_dtype, side);
-  if (e == cudaSuccess) e = cudaEventRecord(join, side);
+  if (side) {
+    e = cudaEventRecord(fork, s);
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(side, fork, 0);
+    if (e == cudaSuccess) e = launch_prefill_tc(fp, a->in_dtype, a->out_dtype, side);
+    if (e == cudaSuccess) e = cudaEventRecord(join, side);
+  } else {
+    e = launch_prefill_tc(fp, a->in_dtype, a->out_dtype, s);
+  }
   if (e == cudaSuccess) {
     // local states and transitions of the middle segments
     PrefillParams lp = base;
@@ -395,9 +403,11 @@ kda_status run_split(const kda_prefill_args *a, const SplitPlan &pl, char *ws,
     lp.m = m;
     e = launch_prefill_tc(lp, a->in_dtype, KDA_F32, s);
   }
-  if (e == cudaSuccess) e = cudaStreamWaitEvent(s, join, 0);
-  cudaEventDestroy(fork);  // released once recorded work completes
-  cudaEventDestroy(join);
+  if (side) {
+    if (e == cudaSuccess) e = cudaStreamWaitEvent(s, join, 0);
+    cudaEventDestroy(fork);  // released once recorded work completes
+    cudaEventDestroy(join);
+  }
   if (e != cudaSuccess) return from_cuda(e);
 
   // start states of the other segments of split requests: S_in[1] is the first
