@@ -1082,10 +1082,13 @@ struct SprodLayout {
   static constexpr int D = 128;
   // B operand tiles (byte offsets, 1024-byte aligned): U~ and W back to back (together
   // the K = 256 operand [U~ | W] of dZ), dO, dU and U (64 rows x 128 tf32 each), then
-  // [dU^T ; dW^T] (256 rows x 64 tf32), whose space first holds the dGam partials
-  static constexpr int TILE = C * D * 4;
+  // [dU^T ; dW^T] (256 rows x 64 tf32).  Before U and [dU^T ; dW^T] are written, their
+  // space holds S (row stride LS floats, for both TMEM layouts of it) and, at its end,
+  // the dGam partials.
+  static constexpr int TILE = C * D * 4, LS = D + 4;
   static constexpr int oUt = 0, oW = TILE, oO = 2 * TILE, oDU = 3 * TILE, oU = 4 * TILE;
-  static constexpr int oDUW = 5 * TILE, oPart = oDUW;
+  static constexpr int oDUW = 5 * TILE, oS = oU, oPart = oDUW + 2 * TILE - 4 * D * 4;
+  static_assert(oS + D * LS * 4 <= oPart, "S and the dGam partials overlap");
   static constexpr int oMisc = oDUW + 2 * TILE;  // four mbarriers, then the TMEM address
   static constexpr size_t bytes = oMisc + 48 + 1024;
 };
@@ -1152,6 +1155,23 @@ __global__ void __launch_bounds__(SP_NTH, 1) bwd_sprod_kernel(const BwdParams p)
       *reinterpret_cast<float4 *>(bO + sw128_chunk(C, t, k)) = tf32_round4(ov[q]);
     }
   }
+  // S into shared memory with whole-row loads: the TMEM layouts below read it by rows
+  // (lane = key row) and by columns (lane = value column)
+  float *sS = reinterpret_cast<float *>(sb + L::oS);
+  {
+    constexpr int NQ = D * D / 4 / SP_NTH;
+    float4 sv4[NQ];
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) {
+      const int e = tid + q * SP_NTH;
+      sv4[q] = reinterpret_cast<const float4 *>(S + (size_t)(e >> 5) * D)[e & 31];
+    }
+#pragma unroll
+    for (int q = 0; q < NQ; ++q) {
+      const int e = tid + q * SP_NTH;
+      *reinterpret_cast<float4 *>(sS + (e >> 5) * L::LS + 4 * (e & 31)) = sv4[q];
+    }
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
@@ -1162,12 +1182,12 @@ __global__ void __launch_bounds__(SP_NTH, 1) bwd_sprod_kernel(const BwdParams p)
   {  // S^T: lane = value column, columns = key rows (consecutive lanes read one row)
     float v[32];
 #pragma unroll
-    for (int jj = 0; jj < 32; ++jj) v[jj] = tf32_round(S[(size_t)(32 * part + jj) * D + lrow]);
+    for (int jj = 0; jj < 32; ++jj) v[jj] = tf32_round(sS[(32 * part + jj) * L::LS + lrow]);
     tmem_st32(tm + lane + TST + 32 * part, v);
   }
   {  // S and dSn: lane = key row, columns = value columns; the dGam partial sums
     float a[32], b[32];
-    const float4 *sr = reinterpret_cast<const float4 *>(S + (size_t)lrow * D + 32 * part);
+    const float4 *sr = reinterpret_cast<const float4 *>(sS + lrow * L::LS + 32 * part);
     const float4 *dr = reinterpret_cast<const float4 *>(dSn + (size_t)lrow * D + 32 * part);
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
