@@ -1172,12 +1172,18 @@ __global__ void __launch_bounds__(SP_NTH, 1) bwd_sprod_kernel(const BwdParams p)
       *reinterpret_cast<float4 *>(sS + (e >> 5) * L::LS + 4 * (e & 31)) = sv4[q];
     }
   }
+  // warp w reaches TMEM lanes 32 (w % 4) .. + 31 and takes the 32-column part w / 4
+  const int qd = w & 3, part = w >> 2, lrow = 32 * qd + ln;
+  float4 dn[8];  // dSn row lrow, columns 32 part .. + 31, in flight across the barrier
+  {
+    const float4 *dr = reinterpret_cast<const float4 *>(dSn + (size_t)lrow * D + 32 * part);
+#pragma unroll
+    for (int q = 0; q < 8; ++q) dn[q] = dr[q];
+  }
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tm = *s_tmem;
-  // warp w reaches TMEM lanes 32 (w % 4) .. + 31 and takes the 32-column part w / 4
-  const int qd = w & 3, part = w >> 2, lrow = 32 * qd + ln;
   const uint32_t lane = (uint32_t)(32 * qd) << 16;
   {  // S^T: lane = value column, columns = key rows (consecutive lanes read one row)
     float v[32];
@@ -1188,11 +1194,10 @@ __global__ void __launch_bounds__(SP_NTH, 1) bwd_sprod_kernel(const BwdParams p)
   {  // S and dSn: lane = key row, columns = value columns; the dGam partial sums
     float a[32], b[32];
     const float4 *sr = reinterpret_cast<const float4 *>(sS + lrow * L::LS + 32 * part);
-    const float4 *dr = reinterpret_cast<const float4 *>(dSn + (size_t)lrow * D + 32 * part);
 #pragma unroll
     for (int q = 0; q < 8; ++q) {
       *reinterpret_cast<float4 *>(&a[4 * q]) = sr[q];
-      *reinterpret_cast<float4 *>(&b[4 * q]) = dr[q];
+      *reinterpret_cast<float4 *>(&b[4 * q]) = dn[q];
     }
     float gs = 0.f;
 #pragma unroll
