@@ -1668,114 +1668,249 @@ __global__ void __launch_bounds__(grad_threads<D, TIn>(), 1) bwd_grad_kernel(con
     }
   }
 
-  // Gated Gram cotangents of P (dP in the P tile) and A (dA in the T tile), one row
-  // block at a time, with the block factorisation of exp(G_t - G_s), t >= s:
-  //   lower (row t of block b, reference r0 = 16 b):
-  //     P1_t = sum_{s<=t} dP_ts k_s e^{G_t-G_s}  -> dq, dG += q P1
-  //     A1_t = sum_{s<t}  dA_ts k_s e^{G_t-G_s}  -> dk, dG += k A1     (one k table)
-  //   upper (row s of block b, reference r1 = 16 b + 15):
-  //     P2_s + A2_s = sum_{t>=s} (dP_ts q_t + dA_ts k_t) e^{G_t-G_s}  -> dk, dG -= k (P2 + A2)
-  // The dO and V tiles are dead here and hold the gate tables.
-#pragma unroll
-  for (int b = 0; b < 4; ++b) {
-    const int r0 = 16 * b, r1 = r0 + 15;
-    __syncthreads();
-    if constexpr (NJ == 4) {  // one float4 chunk x (columns x + TX q) per step
-      for (int e = tid; e < (r0 + 16) * TX; e += GN) {
-        const int t = e / TX, x = e % TX;
-        float v[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int c = x + TX * q;
-          v[q] = sK[t * D + c] * exp2f(sG[r0 * D + c] - sG[t * D + c]);
-        }
-        *reinterpret_cast<float4 *>(sO + t * D + 4 * x) = make_float4(v[0], v[1], v[2], v[3]);
-      }
-    } else {
-      for (int e = tid; e < (r0 + 16) * D; e += GN) {
-        const int c = e % D;
-        sO[e - c + gate_pos<TX, NJ>(c)] = sK[e] * exp2f(sG[r0 * D + c] - sG[e]);
-      }
+  if constexpr (PRE) {
+    // Gated Gram cotangents on the tensor cores, one row block b at a time (reference
+    // rows r0 = 16 b and r1 = r0 + 15, as below), transposed to M = 128 TMEM lanes, one
+    // per channel c; tf32 operands rounded to nearest, fp32 accumulation:
+    //   lower: [P1 | A1]^T[c][t] = sum_{s < r0 + 16} Kb^T[c][s] [dP ; dA][t][s],  t in block b
+    //          Kb[s][c] = k_s e^{G_r0 - G_s}  (A, in TMEM);  B rows: 16 dP rows, 16 dA rows
+    //   upper: O2^T[c][s] = sum_{t >= r0} (Q'^T[c][t] dP[t][s] + K'^T[c][t] dA[t][s]),
+    //          s in block b;  Q'_t = q_t e^{G_t - G_r1}, K'_t = k_t e^{G_t - G_r1}
+    // Terms past the triangles vanish (dP and dA are zero there; every factor is finite).
+    // The CUDA cores scale the results by e^{G_t - G_r0} and e^{G_r1 - G_s} and hand them
+    // to each element's owner through shared memory.
+    constexpr uint32_t TLA = 0, TUA = 64, TLD = 192, TUD = 224;  // TMEM columns (of 256)
+    unsigned char *bL = align1024_shared(sO);  // lower B: 32 rows x 64 K (8 KiB)
+    unsigned char *bUp = bL + 8192;            // upper B: 16 rows x 128 K (8 KiB)
+    float *x1 = sV, *x2 = sV + 16 * D, *x3 = sV + 32 * D;  // P1, A1, O2 scaled: [16][D]
+    uint64_t *gbar = reinterpret_cast<uint64_t *>(sStage);  // sStage is unused here
+    uint32_t *g_tmem = reinterpret_cast<uint32_t *>(sStage + 4);
+    const int w = tid >> 5, ln = tid & 31, qd = w & 3, cg = w >> 2, c = 32 * qd + ln;
+    const uint32_t lane = (uint32_t)(32 * qd) << 16;
+    if (w == 0) {
+      tmem_alloc(g_tmem, 256);
+      tmem_relinquish();
     }
+    if (tid == 0) {
+      mbar_init(gbar, 1);
+      asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+    }
+    tc_fence_before();
     __syncthreads();
-    {
-      const int t = r0 + ty;
-      float op[NJ], oa[NJ];
+    tc_fence_after();
+    const uint32_t tm = *g_tmem;
+    bool ok = true;
+#pragma unroll  // the owners' accumulators are indexed by b
+    for (int b = 0; b < 4; ++b) {
+      const int r0 = 16 * b, r1 = r0 + 15, KL = r0 + 16, KU = C - r0;
+      // A operands: lane c, 8 columns per store; warp column group cg takes every 4th 8
+      for (int s0 = 8 * cg; s0 < KL; s0 += 32) {
+        float v[8];
 #pragma unroll
-      for (int j = 0; j < NJ; ++j) op[j] = oa[j] = 0.f;
-#pragma unroll 4
-      for (int s2 = 0; s2 <= t; ++s2) {
-        const float dp = sP[t * C + s2], da = sT[t * C + s2];
-        float tb[NJ];
+        for (int u = 0; u < 8; ++u) {
+          const int s2 = s0 + u;
+          v[u] = tf32_round(sK[s2 * D + c] * exp2f(sG[r0 * D + c] - sG[s2 * D + c]));
+        }
+        tmem_st8(tm + lane + TLA + s0, v);
+      }
+      for (int u0 = 8 * cg; u0 < 2 * KU; u0 += 32) {
+        const bool kq = u0 >= KU;  // K' half (8-column groups never straddle KU)
+        const float *src = kq ? sK : sQ;
+        float v[8];
 #pragma unroll
-        for (int q = 0; q < NJ / 4; ++q)
-          *reinterpret_cast<float4 *>(&tb[4 * q]) =
-              *reinterpret_cast<const float4 *>(sO + s2 * D + 4 * gate_chunk<TX, NJ>(tx, q));
+        for (int u = 0; u < 8; ++u) {
+          const int t = r0 + u0 + u - (kq ? KU : 0);
+          v[u] = tf32_round(src[t * D + c] * exp2f(sG[t * D + c] - sG[r1 * D + c]));
+        }
+        tmem_st8(tm + lane + TUA + u0, v);
+      }
+      // B operands, one 16-byte chunk per step
+      for (int e = tid; e < 32 * (KL / 4); e += GN) {  // rows n (dP, then dA), K = s
+        const int nrow = e / (KL / 4), k0 = 4 * (e % (KL / 4));
+        const float *row = (nrow < 16 ? sP : sT) + (r0 + (nrow & 15)) * C + k0;
+        *reinterpret_cast<float4 *>(bL + sw128_chunk(32, nrow, k0)) =
+            tf32_round4(*reinterpret_cast<const float4 *>(row));
+      }
+      for (int e = tid; e < 16 * (2 * KU / 4); e += GN) {  // rows n = s - r0, K = t' (dP, dA)
+        const int nrow = e & 15, k0 = 4 * (e >> 4);
+        const bool ka = k0 >= KU;
+        const float *col = (ka ? sT : sP) + (r0 + k0 - (ka ? KU : 0)) * C + r0 + nrow;
+        *reinterpret_cast<float4 *>(bUp + sw128_chunk(16, nrow, k0)) =
+            tf32_round4(make_float4(col[0], col[C], col[2 * C], col[3 * C]));
+      }
+      tmem_wait_st();
+      fence_async_smem();
+      tc_fence_before();
+      __syncthreads();
+      tc_fence_after();
+      if (tid == 0 && ok) {
+        const uint32_t lb = smem_u32(bL), ub = smem_u32(bUp);
+        for (int ks = 0; ks < KL / 8; ++ks)
+          mma_tf32_ts(tm + TLD, tm + TLA + 8 * ks, sw128_desc(lb, 32, ks), idesc_tf32(32), ks > 0);
+        for (int ks = 0; ks < 2 * KU / 8; ++ks)
+          mma_tf32_ts(tm + TUD, tm + TUA + 8 * ks, sw128_desc(ub, 16, ks), idesc_tf32(16), ks > 0);
+        mma_commit(gbar);
+      }
+      ok = ok && mbar_wait(gbar, (uint32_t)(b & 1));
+      tc_fence_after();
+      if (ok) {  // lane c: column group cg reads 8 of the 32 + 16 result columns
+        float v[8];
+        const int tb = 8 * (cg & 1);  // rows t (or s) tb .. tb + 7 of the block
+        tmem_ld8(tm + lane + TLD + 8 * cg, v);  // P1 (cg 0, 1) or A1 (cg 2, 3)
+        tmem_wait_ld();
+        float *dst = cg < 2 ? x1 : x2;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          const int t = r0 + tb + u;
+          dst[(tb + u) * D + c] = v[u] * exp2f(sG[t * D + c] - sG[r0 * D + c]);
+        }
+        if (cg < 2) {
+          tmem_ld8(tm + lane + TUD + tb, v);  // O2
+          tmem_wait_ld();
+#pragma unroll
+          for (int u = 0; u < 8; ++u) {
+            const int s2 = r0 + tb + u;
+            x3[(tb + u) * D + c] = v[u] * exp2f(sG[r1 * D + c] - sG[s2 * D + c]);
+          }
+        }
+      }
+      tc_fence_before();
+      ok = __syncthreads_and(ok);
+      tc_fence_after();
+      if (ok) {  // the element owners: row t = r0 + ty, columns tx + TX j
 #pragma unroll
         for (int j = 0; j < NJ; ++j) {
-          op[j] = fmaf(dp, tb[j], op[j]);
-          oa[j] = fmaf(da, tb[j], oa[j]);
+          const int cc = tx + TX * j, e = ty * D + cc, et = (r0 + ty) * D + cc;
+          const float p1 = x1[e], a1 = x2[e], o2 = x3[e];
+          accQ[b][j] += p1;
+          accK[b][j] += a1 + o2;
+          accG[b][j] = fmaf(sQ[et], p1, fmaf(sK[et], a1 - o2, accG[b][j]));
         }
       }
-#pragma unroll
-      for (int j = 0; j < NJ; ++j) {
-        const int c = tx + TX * j, e = t * D + c;
-        const float f = exp2f(sG[e] - sG[r0 * D + c]);
-        const float p1 = op[j] * f, a1 = oa[j] * f;
-        accQ[b][j] += p1;
-        accK[b][j] += a1;
-        accG[b][j] = fmaf(sQ[e], p1, fmaf(sK[e], a1, accG[b][j]));
-      }
+      __syncthreads();  // x tiles, B tiles and TMEM are free for the next block
     }
-    __syncthreads();
-    if constexpr (NJ == 4) {
-      for (int e = r0 * TX + tid; e < C * TX; e += GN) {
-        const int t = e / TX, x = e % TX;
-        float qv[4], kv[4];
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int c = x + TX * q;
-          const float f = exp2f(sG[t * D + c] - sG[r1 * D + c]);
-          qv[q] = sQ[t * D + c] * f;
-          kv[q] = sK[t * D + c] * f;
-        }
-        *reinterpret_cast<float4 *>(sO + t * D + 4 * x) = make_float4(qv[0], qv[1], qv[2], qv[3]);
-        *reinterpret_cast<float4 *>(sV + t * D + 4 * x) = make_float4(kv[0], kv[1], kv[2], kv[3]);
-      }
-    } else {
-      for (int e = r0 * D + tid; e < C * D; e += GN) {
-        const int c = e % D, at = e - c + gate_pos<TX, NJ>(c);
-        const float f = exp2f(sG[e] - sG[r1 * D + c]);
-        sO[at] = sQ[e] * f;
-        sV[at] = sK[e] * f;
-      }
+    if (!ok && tid == 0) {
+      set_status(p.status, STATUS_TIMEOUT);
+      mma_commit(gbar);  // covers every product issued
+      mbar_wait(gbar, 0, 100000000ull);
+      mbar_wait(gbar, 1, 100000000ull);
     }
+    tc_fence_before();
     __syncthreads();
-    {
-      const int s2 = r0 + ty;
-      float o2[NJ];
-#pragma unroll
-      for (int j = 0; j < NJ; ++j) o2[j] = 0.f;
-#pragma unroll 4
-      for (int t = s2; t < C; ++t) {
-        const float dp = sP[t * C + s2], da = sT[t * C + s2];
-        float qb[NJ], kb[NJ];
-#pragma unroll
-        for (int q = 0; q < NJ / 4; ++q) {
-          *reinterpret_cast<float4 *>(&qb[4 * q]) =
-              *reinterpret_cast<const float4 *>(sO + t * D + 4 * gate_chunk<TX, NJ>(tx, q));
-          *reinterpret_cast<float4 *>(&kb[4 * q]) =
-              *reinterpret_cast<const float4 *>(sV + t * D + 4 * gate_chunk<TX, NJ>(tx, q));
+    if (w == 0) {
+      tc_fence_after();
+      tmem_dealloc(tm, 256);
+    }
+  } else {
+    // Gated Gram cotangents of P (dP in the P tile) and A (dA in the T tile), one row
+    // block at a time, with the block factorisation of exp(G_t - G_s), t >= s:
+    //   lower (row t of block b, reference r0 = 16 b):
+    //     P1_t = sum_{s<=t} dP_ts k_s e^{G_t-G_s}  -> dq, dG += q P1
+    //     A1_t = sum_{s<t}  dA_ts k_s e^{G_t-G_s}  -> dk, dG += k A1     (one k table)
+    //   upper (row s of block b, reference r1 = 16 b + 15):
+    //     P2_s + A2_s = sum_{t>=s} (dP_ts q_t + dA_ts k_t) e^{G_t-G_s}  -> dk, dG -= k (P2 + A2)
+    // The dO and V tiles are dead here and hold the gate tables.
+  #pragma unroll
+    for (int b = 0; b < 4; ++b) {
+      const int r0 = 16 * b, r1 = r0 + 15;
+      __syncthreads();
+      if constexpr (NJ == 4) {  // one float4 chunk x (columns x + TX q) per step
+        for (int e = tid; e < (r0 + 16) * TX; e += GN) {
+          const int t = e / TX, x = e % TX;
+          float v[4];
+  #pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int c = x + TX * q;
+            v[q] = sK[t * D + c] * exp2f(sG[r0 * D + c] - sG[t * D + c]);
+          }
+          *reinterpret_cast<float4 *>(sO + t * D + 4 * x) = make_float4(v[0], v[1], v[2], v[3]);
         }
-#pragma unroll
-        for (int j = 0; j < NJ; ++j) o2[j] = fmaf(dp, qb[j], fmaf(da, kb[j], o2[j]));
+      } else {
+        for (int e = tid; e < (r0 + 16) * D; e += GN) {
+          const int c = e % D;
+          sO[e - c + gate_pos<TX, NJ>(c)] = sK[e] * exp2f(sG[r0 * D + c] - sG[e]);
+        }
       }
-#pragma unroll
-      for (int j = 0; j < NJ; ++j) {
-        const int c = tx + TX * j, e = s2 * D + c;
-        const float v2 = o2[j] * exp2f(sG[r1 * D + c] - sG[e]);
-        accK[b][j] += v2;
-        accG[b][j] = fmaf(-sK[e], v2, accG[b][j]);
+      __syncthreads();
+      {
+        const int t = r0 + ty;
+        float op[NJ], oa[NJ];
+  #pragma unroll
+        for (int j = 0; j < NJ; ++j) op[j] = oa[j] = 0.f;
+  #pragma unroll 4
+        for (int s2 = 0; s2 <= t; ++s2) {
+          const float dp = sP[t * C + s2], da = sT[t * C + s2];
+          float tb[NJ];
+  #pragma unroll
+          for (int q = 0; q < NJ / 4; ++q)
+            *reinterpret_cast<float4 *>(&tb[4 * q]) =
+                *reinterpret_cast<const float4 *>(sO + s2 * D + 4 * gate_chunk<TX, NJ>(tx, q));
+  #pragma unroll
+          for (int j = 0; j < NJ; ++j) {
+            op[j] = fmaf(dp, tb[j], op[j]);
+            oa[j] = fmaf(da, tb[j], oa[j]);
+          }
+        }
+  #pragma unroll
+        for (int j = 0; j < NJ; ++j) {
+          const int c = tx + TX * j, e = t * D + c;
+          const float f = exp2f(sG[e] - sG[r0 * D + c]);
+          const float p1 = op[j] * f, a1 = oa[j] * f;
+          accQ[b][j] += p1;
+          accK[b][j] += a1;
+          accG[b][j] = fmaf(sQ[e], p1, fmaf(sK[e], a1, accG[b][j]));
+        }
+      }
+      __syncthreads();
+      if constexpr (NJ == 4) {
+        for (int e = r0 * TX + tid; e < C * TX; e += GN) {
+          const int t = e / TX, x = e % TX;
+          float qv[4], kv[4];
+  #pragma unroll
+          for (int q = 0; q < 4; ++q) {
+            const int c = x + TX * q;
+            const float f = exp2f(sG[t * D + c] - sG[r1 * D + c]);
+            qv[q] = sQ[t * D + c] * f;
+            kv[q] = sK[t * D + c] * f;
+          }
+          *reinterpret_cast<float4 *>(sO + t * D + 4 * x) = make_float4(qv[0], qv[1], qv[2], qv[3]);
+          *reinterpret_cast<float4 *>(sV + t * D + 4 * x) = make_float4(kv[0], kv[1], kv[2], kv[3]);
+        }
+      } else {
+        for (int e = r0 * D + tid; e < C * D; e += GN) {
+          const int c = e % D, at = e - c + gate_pos<TX, NJ>(c);
+          const float f = exp2f(sG[e] - sG[r1 * D + c]);
+          sO[at] = sQ[e] * f;
+          sV[at] = sK[e] * f;
+        }
+      }
+      __syncthreads();
+      {
+        const int s2 = r0 + ty;
+        float o2[NJ];
+  #pragma unroll
+        for (int j = 0; j < NJ; ++j) o2[j] = 0.f;
+  #pragma unroll 4
+        for (int t = s2; t < C; ++t) {
+          const float dp = sP[t * C + s2], da = sT[t * C + s2];
+          float qb[NJ], kb[NJ];
+  #pragma unroll
+          for (int q = 0; q < NJ / 4; ++q) {
+            *reinterpret_cast<float4 *>(&qb[4 * q]) =
+                *reinterpret_cast<const float4 *>(sO + t * D + 4 * gate_chunk<TX, NJ>(tx, q));
+            *reinterpret_cast<float4 *>(&kb[4 * q]) =
+                *reinterpret_cast<const float4 *>(sV + t * D + 4 * gate_chunk<TX, NJ>(tx, q));
+          }
+  #pragma unroll
+          for (int j = 0; j < NJ; ++j) o2[j] = fmaf(dp, qb[j], fmaf(da, kb[j], o2[j]));
+        }
+  #pragma unroll
+        for (int j = 0; j < NJ; ++j) {
+          const int c = tx + TX * j, e = s2 * D + c;
+          const float v2 = o2[j] * exp2f(sG[r1 * D + c] - sG[e]);
+          accK[b][j] += v2;
+          accG[b][j] = fmaf(-sK[e], v2, accG[b][j]);
+        }
       }
     }
   }
