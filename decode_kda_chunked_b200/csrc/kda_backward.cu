@@ -38,9 +38,9 @@
 //              dP, T^T dU, T^T dW and dZ (the products of chunk-sized tiles)
 //   bwd_grad   (CTA per chunk and head): every token gradient of the chunk
 // For bf16 inputs at d = 128 every dense product runs as tcgen05 tf32 MMAs (transposed
-// to M = 128 TMEM lanes, as in the forward) and bwd_grad keeps the gated Gram
-// cotangents and the per-element folds; fp32 inputs keep fp32 products on the CUDA
-// cores throughout.  The CUDA-core passes give thread (ty, tx) of a 16 x TX grid rows
+// to M = 128 TMEM lanes, as in the forward), the gated Gram cotangents of bwd_grad
+// included, and the CUDA cores keep the per-element folds; fp32 inputs keep fp32
+// products on the CUDA cores throughout.  The CUDA-core passes give thread (ty, tx) of a 16 x TX grid rows
 // ty + 16 i and columns tx + TX j of every tile it produces, so per-element folds stay
 // in registers.
 #include "kda_internal.cuh"
