@@ -1443,11 +1443,25 @@ __global__ void __launch_bounds__(grad_threads<D, TIn>(), 1) bwd_grad_kernel(con
   const float *Ut = p.wU + ch * C * D;
   float *U = p.wU2 + ch * C * D;
 
+  if constexpr (PRE) {
+    // bwd_sprod's d(gamma Q), dP and dZ tiles copied in while the rows stage: into the
+    // O tile (dO is not staged here) and the P and T tiles they are folded into
+    const float4 *gq = reinterpret_cast<const float4 *>(dSn);
+    const float4 *gp = reinterpret_cast<const float4 *>(p.wT + ch * C * C);
+    const float4 *gz = reinterpret_cast<const float4 *>(U);  // dZ over U, [C][C]
+    for (int e = tid; e < C * D / 4; e += GN) cp_async16(sO + 4 * e, gq + e);
+    for (int e = tid; e < C * C / 4; e += GN) {
+      cp_async16(sP + 4 * e, gp + e);
+      cp_async16(sT + 4 * e, gz + e);
+    }
+    cp_async_commit();
+  }
   stage_rows<D, TIn, GN>(sK, D, static_cast<const TIn *>(p.k), tok0, n, H, h);
   stage_rows<D, TIn, GN>(sQ, D, static_cast<const TIn *>(p.q), tok0, n, H, h);
   stage_rows<D, TIn, GN>(sV, D, static_cast<const TIn *>(p.v), tok0, n, H, h);
   if constexpr (!PRE) stage_rows<D, float, GN>(sO, D, p.d_o, tok0, n, H, h);  // PRE: not read
   if (tid < C) sDb[tid] = 0.f;
+  if constexpr (PRE) cp_async_wait<0>();  // made visible by stage_gate's barriers
   stage_gate<D, GN>(sG, sB, p, tok0, n, h);
 
   // the thread's elements: rows ty + 16 i, columns tx + TX j
@@ -1480,7 +1494,7 @@ __global__ void __launch_bounds__(grad_threads<D, TIn>(), 1) bwd_grad_kernel(con
   }
   // d(gamma Q) = dO S^T  ->  dQ = d(gamma Q) gamma,  dG = d(gamma Q) gamma q
   if constexpr (PRE) {
-    load_own(dSn);  // bwd_sprod put d(gamma Q) over the first half of the dSn tile
+    load_own(sO);  // bwd_sprod's d(gamma Q), copied into the O tile above
   } else {
     zero(acc);
     mm_acc<4, NJ>(acc, sO, D, 1, S, 1, D, D, sStage);
@@ -1502,7 +1516,7 @@ __global__ void __launch_bounds__(grad_threads<D, TIn>(), 1) bwd_grad_kernel(con
 #pragma unroll
       for (int i = 0; i < 4; ++i)
 #pragma unroll
-        for (int j = 0; j < NC; ++j) pp[i][j] = p.wT[ch * C * C + (ty + 16 * i) * C + tx + TX * j];
+        for (int j = 0; j < NC; ++j) pp[i][j] = sP[(ty + 16 * i) * C + tx + TX * j];  // dP
     } else {
       zero(pp);
       mm_acc<4, NC>(pp, sO, D, 1, U, 1, D, D, sStage);
@@ -1645,7 +1659,7 @@ __global__ void __launch_bounds__(grad_threads<D, TIn>(), 1) bwd_grad_kernel(con
       for (int i = 0; i < 4; ++i)
 #pragma unroll
         for (int j = 0; j < NC; ++j)
-          tt[i][j] = -p.wU2[ch * C * D + (ty + 16 * i) * C + tx + TX * j];
+          tt[i][j] = -sT[(ty + 16 * i) * C + tx + TX * j];  // dZ, copied in above
     } else {
       zero(tt);
       mm_acc<4, NC>(tt, sV, D, 1, Ut, 1, D, D, sStage);
