@@ -271,7 +271,10 @@ __global__ void __launch_bounds__(NT + 64, 1)
   const int rem = (int)(blockIdx.x % pairs);
   const int r = p.order ? p.order[rem / H] : rem / H;
   const int h = rem % H;
-  const bool has_q = !p.local_mode;  // (a runtime flag keeps the register allocation tight)
+  // q, P and O only where o is written: not in the local-state pass, nor in a run that
+  // only wants states (the backward's recompute).  A runtime flag keeps the register
+  // allocation tight.
+  const bool has_q = !p.local_mode && p.o != nullptr;
   const uint64_t wait_ns = p.wait_ns ? p.wait_ns : 2000000000ull;
   const int bos = p.cu_seqlens[r], eos = p.cu_seqlens[r + 1];
   const int len = eos - bos;
