@@ -128,12 +128,14 @@ size_t prefill_ws(int n_req) {
 // A (request, head) chain is one CTA of the tensor-core kernel, and its chunks run
 // in order, so a call with fewer chains than SMs leaves most of the GPU idle.  Such a
 // call is run as KDA context parallelism inside one device ("Kimi K3 开源日来了",
-// Infra section, first layer): long requests are cut into segments; a local-state
-// pass gives each non-final segment its zero-start state S_loc and transition M (one
-// CTA per segment and head, all in one wave); an exact combine per request recovers
-// every segment's start state; and one prefill over all segments, each from its
-// start state, writes o, the snapshots and (through the last segment) the final
-// state.  The results equal the unsplit call's up to rounding.
+// Infra section, first layer): long requests are cut into segments.  Pass 1 runs
+// each split request's first segment from its initial state on a second stream,
+// beside a local-state pass that gives every middle segment its zero-start state S_loc
+// and transition M (one CTA per segment and head, all in one wave); an exact combine
+// per request then recovers the other segments' start states from the first
+// segment's final state; and pass 2 runs every other segment from its start state,
+// writing o, the snapshots and (through the last segment) the final state.  The
+// results equal the unsplit call's up to rounding.
 // ---------------------------------------------------------------------------
 struct SplitPlan {
   int n_seg = 0;                    // segments over all requests; 0: no split
