@@ -480,40 +480,40 @@ __global__ void __launch_bounds__(prep_threads<D, TIn>(), 1) bwd_prep_kernel(con
     __syncthreads();
   }
   // T = (I + Diag(beta) A)^-1, blocked.  (1) The four 16x16 diagonal blocks by forward
-  // substitution: column task j = tid / 4 (block j / 16), its four threads split each
-  // row's sum and combine it with two shuffles inside their aligned group of four.
+  // substitution: column task j = tid / SP (block j / 16), its SP = PN / 64 threads (4
+  // or 8) split each row's sum and combine it with shuffles inside their aligned group.
   // (2) The blocks below the diagonal, one block diagonal d at a time:
-  //     T_ab = -T_aa sum_{c=b}^{a-1} N_ac T_cb,  N = Diag(beta) A,  b = a - d.
-  // Both steps run on threads 0..255 (16 x 16 for the second); the others wait at the
-  // CTA barriers.
+  //     T_ab = -T_aa sum_{c=b}^{a-1} N_ac T_cb,  N = Diag(beta) A,  b = a - d,
+  // on a 16 x 16 grid per 256 threads (with 512, the two halves take alternate blocks a).
   {
-    const int task = tid >> 2, part = tid & 3;
+    constexpr int SP = PN / 64;
+    const int task = tid / SP, part = tid % SP;
     const int o = 16 * (task >> 4), j = o + (task & 15);
-    if (tid < NTH)
-      for (int i = o; i < o + 16; ++i) {
-        float acc = 0.f;
-        for (int s = j + part; s < i; s += 4) acc = fmaf(sA[i * LA + s], sT[s * C + j], acc);
-        acc += __shfl_xor_sync(0xffffffffu, acc, 1);
-        acc += __shfl_xor_sync(0xffffffffu, acc, 2);
-        if (part == 0) sT[i * C + j] = i < j ? 0.f : (i == j ? 1.f : -sB[i] * acc);
-        __syncwarp();
-      }
+    for (int i = o; i < o + 16; ++i) {
+      float acc = 0.f;
+      for (int s = j + part; s < i; s += SP) acc = fmaf(sA[i * LA + s], sT[s * C + j], acc);
+#pragma unroll
+      for (int off = 1; off < SP; off <<= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      if (part == 0) sT[i * C + j] = i < j ? 0.f : (i == j ? 1.f : -sB[i] * acc);
+      __syncwarp();
+    }
     for (int e = tid; e < C * C; e += PN)  // blocks above the diagonal
       if ((e / C) >> 4 < (e % C) >> 4) sT[e] = 0.f;
     float *Ys = sBuf;  // [3][16][17] scratch: N_a. T_.b of one block diagonal
+    const int half = tid / NTH, sy = (tid % NTH) >> 4, sx = tid & 15;
     for (int d = 1; d < 4; ++d) {
       __syncthreads();
-      for (int a = d; a < 4 && tid < NTH; ++a) {
-        const int bb = a - d, i = 16 * a + ty, jc = 16 * bb + tx;
+      for (int a = d + half; a < 4; a += PN / NTH) {
+        const int bb = a - d, i = 16 * a + sy, jc = 16 * bb + sx;
         float y = 0.f;
         for (int s2 = 16 * bb; s2 < 16 * a; ++s2) y = fmaf(sA[i * LA + s2], sT[s2 * C + jc], y);
-        Ys[(bb * 16 + ty) * 17 + tx] = sB[i] * y;
+        Ys[(bb * 16 + sy) * 17 + sx] = sB[i] * y;
       }
       __syncthreads();
-      for (int a = d; a < 4 && tid < NTH; ++a) {
-        const int bb = a - d, i = 16 * a + ty, jc = 16 * bb + tx;
+      for (int a = d + half; a < 4; a += PN / NTH) {
+        const int bb = a - d, i = 16 * a + sy, jc = 16 * bb + sx;
         float t = 0.f;
-        for (int r = 16 * a; r <= i; ++r) t = fmaf(sT[i * C + r], Ys[(bb * 16 + r - 16 * a) * 17 + tx], t);
+        for (int r = 16 * a; r <= i; ++r) t = fmaf(sT[i * C + r], Ys[(bb * 16 + r - 16 * a) * 17 + sx], t);
         sT[i * C + jc] = -t;
       }
     }
