@@ -308,8 +308,8 @@ template <int D, typename TIn>
 __host__ __device__ constexpr int grad_threads() { return kPrepTensorCores<D, TIn> ? 512 : 256; }
 
 // Threads of the prep pass: 512 when its products run on the tensor cores (16 warps
-// share the operand staging and read-out; the triangular solve runs on the first 256),
-// else 256 (its fp32 tile products assume a 16 x 16 thread grid).
+// share the operand staging, the read-out and the triangular solve), else 256 (its
+// fp32 tile products assume a 16 x 16 thread grid).
 template <int D, typename TIn>
 __host__ __device__ constexpr int prep_threads() { return kPrepTensorCores<D, TIn> ? 512 : 256; }
 
